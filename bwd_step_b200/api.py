@@ -1,0 +1,129 @@
+"""Thin Python binding of the step's C ABI (argument marshalling only).
+
+Every computation runs in the CUDA library; this module only turns torch
+tensors (device memory allocated by PyTorch) into pointers and checks their
+dtype, device and contiguity.
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import NcConfig, lib
+
+PRECISIONS = {"bf16": _lib.NC_PREC_BF16, "fp32": _lib.NC_PREC_FP32_DEBUG}
+
+
+class NcError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {lib().nc_status_string(code).decode()} ({code})")
+
+
+def _ok(code: int, what: str):
+    if code != _lib.NC_OK:
+        raise NcError(code, what)
+
+
+def _stream_handle(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Model:
+    """A model handle: shape, precision and the flat parameter layout."""
+
+    def __init__(self, cfg, precision: str = "bf16"):
+        get = (lambda k: cfg[k]) if isinstance(cfg, dict) else (lambda k: getattr(cfg, k))
+        self.cfg = NcConfig(get("vocab"), get("d_model"), get("n_layer"), get("n_head"), get("n_kv_head"),
+                            get("head_dim"), get("mlp_mult"), float(get("softcap")), float(get("rope_base")))
+        self.precision = precision
+        h = ctypes.c_void_p()
+        _ok(lib().nc_model_create(ctypes.byref(self.cfg), PRECISIONS[precision], ctypes.byref(h)),
+            "nc_model_create")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().nc_model_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def weight_dtype(self):
+        import torch
+        return torch.bfloat16 if self.precision == "bf16" else torch.float32
+
+    def num_params(self) -> int:
+        return int(lib().nc_num_params(self._h))
+
+    def layout(self):
+        out = []
+        i = 0
+        name, off = ctypes.c_char_p(), ctypes.c_int64()
+        r, c = ctypes.c_int(), ctypes.c_int()
+        while lib().nc_param_layout(self._h, i, ctypes.byref(name), ctypes.byref(off), ctypes.byref(r),
+                                    ctypes.byref(c)) == _lib.NC_OK:
+            out.append((name.value.decode(), r.value, c.value, off.value))
+            i += 1
+        return out
+
+    def workspace_bytes(self, B: int, T: int) -> int:
+        return int(lib().nc_workspace_bytes(self._h, B, T))
+
+    def forward_backward(self, tokens, targets, weights, grads, loss, workspace, stream=None):
+        """One step on device tensors; grads (fp32) and loss (fp32 [1]) are overwritten."""
+        import torch
+        B, T = tokens.shape
+        _ok(lib().nc_forward_backward(self._h, _ptr(tokens, torch.int32, "tokens"),
+                                      _ptr(targets, torch.int32, "targets"), B, T,
+                                      _ptr(weights, self.weight_dtype, "weights"),
+                                      _ptr(grads, torch.float32, "grads"), _ptr(loss, torch.float32, "loss"),
+                                      _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+                                      ctypes.c_void_p(_stream_handle(stream))), "nc_forward_backward")
+
+    def forward_backward_host(self, h_tokens, h_targets, weights, grads, workspace, stream=None) -> float:
+        """One step with host (ideally pinned) int32 token/target tensors; returns the loss."""
+        import torch
+        B, T = h_tokens.shape
+        out = ctypes.c_float()
+        _ok(lib().nc_forward_backward_host(self._h, _ptr(h_tokens, torch.int32, "tokens"),
+                                           _ptr(h_targets, torch.int32, "targets"), B, T,
+                                           _ptr(weights, self.weight_dtype, "weights"),
+                                           _ptr(grads, torch.float32, "grads"), ctypes.byref(out),
+                                           _ptr(workspace, None, "workspace"),
+                                           workspace.numel() * workspace.element_size(),
+                                           ctypes.c_void_p(_stream_handle(stream))), "nc_forward_backward_host")
+        return out.value
+
+    def forward_logits(self, tokens, weights, logits, workspace, stream=None):
+        import torch
+        B, T = tokens.shape
+        _ok(lib().nc_forward_logits(self._h, _ptr(tokens, torch.int32, "tokens"), B, T,
+                                    _ptr(weights, self.weight_dtype, "weights"),
+                                    _ptr(logits, self.weight_dtype, "logits"), _ptr(workspace, None, "workspace"),
+                                    workspace.numel() * workspace.element_size(),
+                                    ctypes.c_void_p(_stream_handle(stream))), "nc_forward_logits")
+
+    def check(self, stream=None) -> int:
+        """Synchronise the stream and return (and clear) the device status code."""
+        return int(lib().nc_check(self._h, ctypes.c_void_p(_stream_handle(stream))))
+
+    def debug_expired_wait(self, max_iters: int, stream=None):
+        _ok(lib().nc_debug_expired_wait(self._h, max_iters, ctypes.c_void_p(_stream_handle(stream))),
+            "nc_debug_expired_wait")

@@ -1,0 +1,100 @@
+// Host-side launchers of the step's kernels (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace nc {
+
+enum DType : int { DT_F32 = 0, DT_BF16 = 1 };
+inline size_t dt_size(DType t) { return t == DT_BF16 ? 2 : 4; }
+
+// ---------------------------------------------------------------- memory-bound
+// cos/sin [T, hd/2] of pos * base^(-2j/hd), evaluated in double.
+cudaError_t launch_rope_table(float* cos_t, float* sin_t, int T, int hd, float base, cudaStream_t s);
+
+// x[m] = rmsnorm(wte[idx[m]]) (fp32 residual stream), r0[m] = its inverse RMS.
+cudaError_t launch_embed_norm_fwd(DType wt, const int32_t* idx, const void* wte, int M, int V, int d,
+                                  float* x, float* r0, int* status, cudaStream_t s);
+// y = x * r, r = (mean(x^2)+eps)^-1/2 per row; y in activation type.
+cudaError_t launch_rmsnorm_fwd(DType at, const float* x, void* y, float* r, int M, int d, cudaStream_t s);
+// dx = (accumulate ? dx : 0) + r*(dy - y*mean(dy*y)); optional dxb = dx in activation type.
+cudaError_t launch_rmsnorm_bwd(DType at, const float* dy, const void* y, const float* r, float* dx,
+                               bool accumulate, void* dxb, int M, int d, cudaStream_t s);
+// de = gradient through the token-embedding norm, recomputing y = wte[idx]*r0.
+cudaError_t launch_embed_norm_bwd(DType wt, const float* dx, const int32_t* idx, const void* wte,
+                                  const float* r0, float* de, int M, int V, int d, cudaStream_t s);
+// In place on the fused qkv rows [M, (H+2nkv)*hd]: q,k <- rope(rmsnorm_hd(q,k)); rqk [M, H+nkv].
+cudaError_t launch_qknorm_rope_fwd(DType at, void* qkv, float* rqk, const float* cos_t, const float* sin_t,
+                                   int M, int T, int H, int nkv, int hd, cudaStream_t s);
+// In place on the q,k parts of dqkv: inverse rotation then RMSNorm backward.
+cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const float* rqk,
+                                   const float* cos_t, const float* sin_t, int M, int T, int H, int nkv,
+                                   int hd, cudaStream_t s);
+// Cross-entropy over R rows of softcapped logits z [R, V] (fp32):
+// loss_rows[r] = lse - z[tgt]; dl = inv_M*(softmax - onehot)*(1-(z/cap)^2).
+cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R, int V, float cap,
+                            float inv_M, float* loss_rows, void* dl, int* status, cudaStream_t s);
+// loss = mean(loss_rows[0..M)), fixed summation order.
+cudaError_t launch_loss_reduce(const float* loss_rows, int M, float* loss, cudaStream_t s);
+
+struct EmbedScratch {
+    int* count;    // [V]
+    int* offset;   // [V+1]
+    int* cursor;   // [V]
+    int* perm;     // [M]
+    int* perm2;    // [M]
+    int* active;   // [V]
+    int* n_active; // [1]
+};
+size_t embed_scratch_bytes(int M, int V);
+EmbedScratch embed_scratch_carve(void* base, int M, int V);
+// dwte[v] = sum over positions m with idx[m] == v of de[m], in increasing m;
+// rows of unused ids are zero.  Deterministic.
+cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int V, int d, float* dwte,
+                                 EmbedScratch sc, cudaStream_t s);
+// out[i] = sum_{s < splits} part[s*n + i] in increasing s.
+cudaError_t launch_splitk_reduce(const float* part, int splits, size_t n, float* out, bool accumulate,
+                                 cudaStream_t s);
+
+// ---------------------------------------------------------------- GEMM
+// C[m,n] = sum_k A(m,k) * B(n,k).
+//   A(m,k) = a_kmajor ? A[m*lda + k] : A[k*lda + m]
+//   B(n,k) = b_kmajor ? B[n*ldb + k] : B[k*ldb + n]
+enum Epi : int {
+    EPI_STORE = 0,      // C = acc                         (C fp32 or activation type)
+    EPI_ACCUM = 1,      // C += acc                        (C fp32)
+    EPI_RELU2 = 2,      // C = relu(acc)^2, C2 = relu(acc) (activation type)
+    EPI_RELU2_BWD = 3,  // C = acc * 2 * aux               (aux = relu(u), activation type)
+    EPI_SOFTCAP = 4,    // C = cap * tanh(acc / cap)       (C fp32 or activation type)
+};
+
+struct GemmDesc {
+    int M = 0, N = 0, K = 0;
+    DType in_t = DT_F32;  // type of A and B
+    const void* A = nullptr; int64_t lda = 0; bool a_kmajor = true;
+    const void* B = nullptr; int64_t ldb = 0; bool b_kmajor = true;
+    Epi epi = EPI_STORE;
+    void* C = nullptr; int64_t ldc = 0; DType c_t = DT_F32;
+    void* C2 = nullptr; int64_t ldc2 = 0;
+    const void* aux = nullptr; int64_t ldaux = 0;
+    float cap = 0.f;
+};
+
+// Plain fp32-FMA tiled GEMM (any strides, any sizes).
+cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+// qkv rows [B*T, (H+2nkv)*hd] hold q (post norm+rope), k (same), v.
+// o [B*T, H*hd]; lse [B*T, H] (natural log).
+cudaError_t launch_attention_fwd_simt(DType at, const void* qkv, void* o, float* lse, int B, int T, int H,
+                                      int nkv, int hd, cudaStream_t s);
+// Writes dq (into the q columns), dk, dv of dqkv.  Dbuf [B*T, H] scratch.
+cudaError_t launch_attention_bwd_simt(DType at, const void* qkv, const void* o, const void* dO,
+                                      const float* lse, float* Dbuf, void* dqkv, int B, int T, int H,
+                                      int nkv, int hd, cudaStream_t s);
+
+// ---------------------------------------------------------------- bounded wait
+cudaError_t launch_expired_wait(int* status, int max_iters, cudaStream_t s);
+
+}  // namespace nc

@@ -1,0 +1,573 @@
+// Memory-bound kernels of the step: token-embedding gather + norm, the
+// parameter-free RMSNorm forward/backward, QK-norm fused with RoPE (forward
+// and backward), the LM-head cross-entropy over a chunk of rows, the loss
+// mean, the deterministic embedding-gradient scatter and the split-K reduce.
+//
+// Model items (nanochat announcement, vpshk.cn, architecture list): RMSNorm
+// without learnable parameters, normalised token embedding, rotary embedding,
+// QK-norm, logit softcap.  One warp owns one row (d % 64 == 0), every lane
+// moves 8 elements per step with 16-byte accesses, and row statistics are
+// reduced with warp shuffles.
+#include "common.cuh"
+#include "kernels.h"
+#include <math.h>
+
+namespace nc {
+
+namespace {
+
+__device__ __forceinline__ void load8(const float* p, float* o) { load_vec(p, o); load_vec(p + 4, o + 4); }
+__device__ __forceinline__ void load8(const bf16* p, float* o) { load_vec(p, o); }
+__device__ __forceinline__ void store8(float* p, const float* v) { store_vec(p, v); store_vec(p + 4, v + 4); }
+__device__ __forceinline__ void store8(bf16* p, const float* v) { store_vec(p, v); }
+
+constexpr int kRowWarps = 8;  // rows per 256-thread block
+
+inline int row_blocks(int M) { return (M + kRowWarps - 1) / kRowWarps; }
+
+// ---------------------------------------------------------------- RoPE table
+__global__ void rope_table_kernel(float* c, float* s, int T, int hd, double base) {
+    int half = hd / 2;
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= T * half) return;
+    int pos = i / half, j = i % half;
+    double theta = pow(base, -2.0 * (double)j / (double)hd);
+    double ang = (double)pos * theta;
+    c[i] = (float)cos(ang);
+    s[i] = (float)sin(ang);
+}
+
+// ---------------------------------------------------------------- embedding
+template <typename W>
+__global__ void embed_norm_fwd_kernel(const int32_t* __restrict__ idx, const W* __restrict__ wte, int M,
+                                      int V, int d, float* __restrict__ x, float* __restrict__ r0,
+                                      int* status) {
+    int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+    int lane = threadIdx.x & 31;
+    if (row >= M) return;
+    int id = idx[row];
+    bool bad = id < 0 || id >= V;
+    if (bad && lane == 0) set_status(status, ST_BAD_TOKEN);
+    const W* src = wte + (size_t)(bad ? 0 : id) * d;
+    float ss = 0.f;
+    for (int c = lane * 8; c < d; c += 256) {
+        float v[8];
+        load8(src + c, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss += v[k] * v[k];
+    }
+    ss = warp_sum(ss);
+    float r = bad ? 0.f : rsqrtf(ss / (float)d + kRmsEps);
+    float* dst = x + (size_t)row * d;
+    for (int c = lane * 8; c < d; c += 256) {
+        float v[8];
+        load8(src + c, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] *= r;
+        store8(dst + c, v);
+    }
+    if (lane == 0) r0[row] = r;
+}
+
+template <typename W>
+__global__ void embed_norm_bwd_kernel(const float* __restrict__ dx, const int32_t* __restrict__ idx,
+                                      const W* __restrict__ wte, const float* __restrict__ r0,
+                                      float* __restrict__ de, int M, int V, int d) {
+    int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+    int lane = threadIdx.x & 31;
+    if (row >= M) return;
+    int id = idx[row];
+    bool bad = id < 0 || id >= V;
+    const W* src = wte + (size_t)(bad ? 0 : id) * d;
+    const float* g = dx + (size_t)row * d;
+    float r = r0[row];
+    float dot = 0.f;
+    for (int c = lane * 8; c < d; c += 256) {
+        float e[8], gg[8];
+        load8(src + c, e);
+        load8(g + c, gg);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) dot += gg[k] * e[k] * r;
+    }
+    dot = warp_sum(dot) / (float)d;
+    float* dst = de + (size_t)row * d;
+    for (int c = lane * 8; c < d; c += 256) {
+        float e[8], gg[8], o[8];
+        load8(src + c, e);
+        load8(g + c, gg);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[k] = r * (gg[k] - e[k] * r * dot);
+        store8(dst + c, o);
+    }
+}
+
+// ---------------------------------------------------------------- RMSNorm
+template <typename A>
+__global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, A* __restrict__ y, float* __restrict__ r,
+                                   int M, int d) {
+    int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+    int lane = threadIdx.x & 31;
+    if (row >= M) return;
+    const float* src = x + (size_t)row * d;
+    float ss = 0.f;
+    for (int c = lane * 8; c < d; c += 256) {
+        float v[8];
+        load8(src + c, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss += v[k] * v[k];
+    }
+    ss = warp_sum(ss);
+    float rr = rsqrtf(ss / (float)d + kRmsEps);
+    A* dst = y + (size_t)row * d;
+    for (int c = lane * 8; c < d; c += 256) {
+        float v[8];
+        load8(src + c, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] *= rr;
+        store8(dst + c, v);
+    }
+    if (lane == 0) r[row] = rr;
+}
+
+template <typename A>
+__global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const A* __restrict__ y,
+                                   const float* __restrict__ r, float* dx, bool accumulate, A* dxb,
+                                   int M, int d) {
+    int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+    int lane = threadIdx.x & 31;
+    if (row >= M) return;
+    const float* g = dy + (size_t)row * d;
+    const A* yy = y + (size_t)row * d;
+    float dot = 0.f;
+    for (int c = lane * 8; c < d; c += 256) {
+        float a[8], b[8];
+        load8(g + c, a);
+        load8(yy + c, b);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) dot += a[k] * b[k];
+    }
+    dot = warp_sum(dot) / (float)d;
+    float rr = r[row];
+    float* out = dx + (size_t)row * d;
+    for (int c = lane * 8; c < d; c += 256) {
+        float a[8], b[8], o[8];
+        load8(g + c, a);
+        load8(yy + c, b);
+        if (accumulate) load8(out + c, o);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            float v = rr * (a[k] - b[k] * dot);
+            o[k] = accumulate ? o[k] + v : v;
+        }
+        store8(out + c, o);
+        if (dxb) store8(dxb + (size_t)row * d + c, o);
+    }
+}
+
+// ---------------------------------------------------------------- QK-norm + RoPE
+// A group of G lanes (G = min(32, hd/2)) owns one head vector; lane li holds
+// the pairs (j, j + hd/2) for j = li + p*G.
+template <typename A>
+__global__ void qknorm_rope_fwd_kernel(A* qkv, float* __restrict__ rqk, const float* __restrict__ cos_t,
+                                       const float* __restrict__ sin_t, int M, int T, int H, int nkv,
+                                       int hd, int G) {
+    int t = blockIdx.x * blockDim.x + threadIdx.x;
+    int nh = H + nkv;
+    int vi = t / G, li = t % G;
+    bool active = vi < M * nh;
+    int m = active ? vi / nh : 0, head = active ? vi % nh : 0;
+    int pos = m % T, half = hd >> 1, P = half / G;
+    A* v = qkv + (size_t)m * (size_t)(H + 2 * nkv) * hd + (size_t)head * hd;
+    float x1[2] = {0.f, 0.f}, x2[2] = {0.f, 0.f};
+    float ss = 0.f;
+    if (active) {
+        for (int p = 0; p < P; ++p) {
+            int j = li + p * G;
+            x1[p] = tof(v[j]);
+            x2[p] = tof(v[j + half]);
+            ss += x1[p] * x1[p] + x2[p] * x2[p];
+        }
+    }
+    for (int o = G >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (!active) return;
+    float r = rsqrtf(ss / (float)hd + kRmsEps);
+    for (int p = 0; p < P; ++p) {
+        int j = li + p * G;
+        float c = cos_t[pos * half + j], s = sin_t[pos * half + j];
+        float a = x1[p] * r, b = x2[p] * r;
+        v[j] = fromf<A>(a * c - b * s);
+        v[j + half] = fromf<A>(a * s + b * c);
+    }
+    if (li == 0) rqk[(size_t)m * nh + head] = r;
+}
+
+template <typename A>
+__global__ void qknorm_rope_bwd_kernel(A* dqkv, const A* __restrict__ qkv, const float* __restrict__ rqk,
+                                       const float* __restrict__ cos_t, const float* __restrict__ sin_t,
+                                       int M, int T, int H, int nkv, int hd, int G) {
+    int t = blockIdx.x * blockDim.x + threadIdx.x;
+    int nh = H + nkv;
+    int vi = t / G, li = t % G;
+    bool active = vi < M * nh;
+    int m = active ? vi / nh : 0, head = active ? vi % nh : 0;
+    int pos = m % T, half = hd >> 1, P = half / G;
+    size_t off = (size_t)m * (size_t)(H + 2 * nkv) * hd + (size_t)head * hd;
+    A* g = dqkv + off;
+    const A* y = qkv + off;
+    float g1[2] = {0.f, 0.f}, g2[2] = {0.f, 0.f}, y1[2] = {0.f, 0.f}, y2[2] = {0.f, 0.f};
+    float dot = 0.f;
+    if (active) {
+        for (int p = 0; p < P; ++p) {
+            int j = li + p * G;
+            float c = cos_t[pos * half + j], s = sin_t[pos * half + j];
+            float a = tof(g[j]), b = tof(g[j + half]);
+            g1[p] = a * c + b * s;       // inverse rotation of the gradient
+            g2[p] = -a * s + b * c;
+            float u = tof(y[j]), w = tof(y[j + half]);
+            y1[p] = u * c + w * s;       // normalised vector before rotation
+            y2[p] = -u * s + w * c;
+            dot += g1[p] * y1[p] + g2[p] * y2[p];
+        }
+    }
+    for (int o = G >> 1; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (!active) return;
+    dot /= (float)hd;
+    float r = rqk[(size_t)m * nh + head];
+    for (int p = 0; p < P; ++p) {
+        int j = li + p * G;
+        g[j] = fromf<A>(r * (g1[p] - y1[p] * dot));
+        g[j + half] = fromf<A>(r * (g2[p] - y2[p] * dot));
+    }
+}
+
+// ---------------------------------------------------------------- cross-entropy
+struct MaxSum { float m, s; };
+
+__device__ __forceinline__ MaxSum ms_combine(MaxSum a, MaxSum b) {
+    if (b.s == 0.f) return a;
+    if (a.s == 0.f) return b;
+    float m = fmaxf(a.m, b.m);
+    return {m, a.s * __expf(a.m - m) + b.s * __expf(b.m - m)};
+}
+
+template <typename D>
+__global__ void ce_chunk_kernel(const float* __restrict__ z, const int32_t* __restrict__ tgt, int R, int V,
+                                float cap, float inv_M, float* __restrict__ loss_rows, D* __restrict__ dl,
+                                int* status) {
+    __shared__ MaxSum red[32];
+    __shared__ float s_lse;
+    int row = blockIdx.x;
+    const float* zr = z + (size_t)row * V;
+    MaxSum acc = {-INFINITY, 0.f};
+    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
+        float4 v = *reinterpret_cast<const float4*>(zr + c);
+        float m4 = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+        float m = fmaxf(acc.m, m4);
+        float s = (acc.s == 0.f ? 0.f : acc.s * expf(acc.m - m));
+        s += expf(v.x - m) + expf(v.y - m) + expf(v.z - m) + expf(v.w - m);
+        acc = {m, s};
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        MaxSum other = {__shfl_xor_sync(0xffffffffu, acc.m, o), __shfl_xor_sync(0xffffffffu, acc.s, o)};
+        acc = ms_combine(acc, other);
+    }
+    int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[w] = acc;
+    __syncthreads();
+    if (w == 0) {
+        int nw = blockDim.x >> 5;
+        acc = lane < nw ? red[lane] : MaxSum{-INFINITY, 0.f};
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            MaxSum other = {__shfl_xor_sync(0xffffffffu, acc.m, o), __shfl_xor_sync(0xffffffffu, acc.s, o)};
+            acc = ms_combine(acc, other);
+        }
+        if (lane == 0) s_lse = acc.m + logf(acc.s);
+    }
+    __syncthreads();
+    float lse = s_lse;
+    int t = tgt[row];
+    bool bad = t < 0 || t >= V;
+    if (threadIdx.x == 0) {
+        if (bad) set_status(status, ST_BAD_TOKEN);
+        loss_rows[row] = bad ? 0.f : lse - zr[t];
+    }
+    D* out = dl + (size_t)row * V;
+    float inv_cap = 1.f / cap;
+    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
+        float4 v = *reinterpret_cast<const float4*>(zr + c);
+        float zz[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float p = expf(zz[k] - lse) - ((c + k) == t ? 1.f : 0.f);
+            float q = zz[k] * inv_cap;
+            out[c + k] = fromf<D>(bad ? 0.f : p * inv_M * (1.f - q * q));
+        }
+    }
+}
+
+__global__ void loss_reduce_kernel(const float* __restrict__ rows, int M, float* loss) {
+    __shared__ float sh[1024];
+    float s = 0.f;
+    for (int i = threadIdx.x; i < M; i += blockDim.x) s += rows[i];
+    sh[threadIdx.x] = s;
+    __syncthreads();
+    for (int o = blockDim.x >> 1; o > 0; o >>= 1) {
+        if ((int)threadIdx.x < o) sh[threadIdx.x] += sh[threadIdx.x + o];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *loss = sh[0] / (float)M;
+}
+
+// ---------------------------------------------------------------- embedding scatter
+__global__ void emb_hist_kernel(const int32_t* __restrict__ idx, int M, int V, int* count) {
+    int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= M) return;
+    int id = idx[m];
+    if (id >= 0 && id < V) atomicAdd(&count[id], 1);
+}
+
+// Single block of 1024 threads: exclusive scan of count[V] into offset[V+1]
+// and compaction of the ids with count > 0 into active[].
+__global__ void emb_scan_kernel(const int* __restrict__ count, int V, int* offset, int* active,
+                                int* n_active) {
+    __shared__ int sc[1024], sf[1024];
+    int t = threadIdx.x;
+    int per = (V + 1023) / 1024;
+    int lo = min(V, t * per), hi = min(V, lo + per);
+    int c = 0, f = 0;
+    for (int i = lo; i < hi; ++i) { int k = count[i]; c += k; f += k > 0; }
+    sc[t] = c; sf[t] = f;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        int a = t >= o ? sc[t - o] : 0, b = t >= o ? sf[t - o] : 0;
+        __syncthreads();
+        sc[t] += a; sf[t] += b;
+        __syncthreads();
+    }
+    int base_c = sc[t] - c, base_f = sf[t] - f;
+    for (int i = lo; i < hi; ++i) {
+        int k = count[i];
+        offset[i] = base_c;
+        if (k > 0) active[base_f++] = i;
+        base_c += k;
+    }
+    if (t == 1023) { offset[V] = sc[1023]; *n_active = sf[1023]; }
+}
+
+__global__ void emb_fill_kernel(const int32_t* __restrict__ idx, int M, int V, const int* __restrict__ offset,
+                                int* cursor, int* perm) {
+    int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= M) return;
+    int id = idx[m];
+    if (id < 0 || id >= V) return;
+    perm[offset[id] + atomicAdd(&cursor[id], 1)] = m;
+}
+
+// Puts the positions of every id in increasing order (the fill order above
+// depends on atomic timing; this makes the final order unique).
+__global__ void emb_canon_kernel(const int32_t* __restrict__ idx, int V, const int* __restrict__ offset,
+                                 const int* __restrict__ perm, int* perm2) {
+    int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= offset[V]) return;
+    int p = perm[s];
+    int v = idx[p];
+    int lo = offset[v], hi = offset[v + 1], rank = 0;
+    for (int u = lo; u < hi; ++u) rank += perm[u] < p;
+    perm2[lo + rank] = p;
+}
+
+__global__ void emb_segsum_kernel(const float* __restrict__ de, int d, const int* __restrict__ offset,
+                                  const int* __restrict__ perm2, const int* __restrict__ active,
+                                  const int* __restrict__ n_active, float* __restrict__ dwte) {
+    int k = blockIdx.x;
+    if (k >= *n_active) return;
+    int v = active[k];
+    int lo = offset[v], hi = offset[v + 1];
+    for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = lo; s < hi; ++s) {
+            float4 g = *reinterpret_cast<const float4*>(de + (size_t)perm2[s] * d + c);
+            acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
+        }
+        *reinterpret_cast<float4*>(dwte + (size_t)v * d + c) = acc;
+    }
+}
+
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, size_t n4,
+                                     float* __restrict__ out, bool accumulate) {
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const float4* p = reinterpret_cast<const float4*>(part);
+    float4 acc = accumulate ? reinterpret_cast<float4*>(out)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < splits; ++s) {
+        float4 g = p[(size_t)s * n4 + i];
+        acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
+    }
+    reinterpret_cast<float4*>(out)[i] = acc;
+}
+
+// ---------------------------------------------------------------- bounded wait
+// Waits on an mbarrier that nobody arrives at; each try_wait is bounded by
+// the hardware's time limit and the loop by max_iters.  On expiry it records
+// ST_TIMEOUT and returns.
+__global__ void expired_wait_kernel(int* status, int max_iters) {
+    __shared__ __align__(8) uint64_t bar;
+    uint32_t addr = (uint32_t)__cvta_generic_to_shared(&bar);
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(addr));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x != 0) return;
+    uint32_t done = 0;
+    for (int it = 0; it < max_iters && !done; ++it) {
+        asm volatile(
+            "{\n .reg .pred p;\n"
+            " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done)
+            : "r"(addr)
+            : "memory");
+    }
+    if (!done) set_status(status, ST_TIMEOUT);
+}
+
+}  // namespace
+
+// ============================================================================ launchers
+cudaError_t launch_rope_table(float* c, float* s, int T, int hd, float base, cudaStream_t st) {
+    int n = T * (hd / 2);
+    rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(c, s, T, hd, (double)base);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_embed_norm_fwd(DType wt, const int32_t* idx, const void* wte, int M, int V, int d,
+                                  float* x, float* r0, int* status, cudaStream_t s) {
+    if (wt == DT_BF16)
+        embed_norm_fwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(idx, (const bf16*)wte, M, V, d, x, r0, status);
+    else
+        embed_norm_fwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(idx, (const float*)wte, M, V, d, x, r0, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm_fwd(DType at, const float* x, void* y, float* r, int M, int d, cudaStream_t s) {
+    if (at == DT_BF16)
+        rmsnorm_fwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(x, (bf16*)y, r, M, d);
+    else
+        rmsnorm_fwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(x, (float*)y, r, M, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rmsnorm_bwd(DType at, const float* dy, const void* y, const float* r, float* dx,
+                               bool accumulate, void* dxb, int M, int d, cudaStream_t s) {
+    if (at == DT_BF16)
+        rmsnorm_bwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(dy, (const bf16*)y, r, dx, accumulate,
+                                                               (bf16*)dxb, M, d);
+    else
+        rmsnorm_bwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(dy, (const float*)y, r, dx, accumulate,
+                                                                (float*)dxb, M, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_embed_norm_bwd(DType wt, const float* dx, const int32_t* idx, const void* wte,
+                                  const float* r0, float* de, int M, int V, int d, cudaStream_t s) {
+    if (wt == DT_BF16)
+        embed_norm_bwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(dx, idx, (const bf16*)wte, r0, de, M, V, d);
+    else
+        embed_norm_bwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(dx, idx, (const float*)wte, r0, de, M, V, d);
+    return cudaGetLastError();
+}
+
+static inline int qk_group(int hd) { return hd / 2 < 32 ? hd / 2 : 32; }
+
+cudaError_t launch_qknorm_rope_fwd(DType at, void* qkv, float* rqk, const float* c, const float* sn, int M,
+                                   int T, int H, int nkv, int hd, cudaStream_t s) {
+    int G = qk_group(hd);
+    long long threads = (long long)M * (H + nkv) * G;
+    int blocks = (int)((threads + 255) / 256);
+    if (at == DT_BF16)
+        qknorm_rope_fwd_kernel<bf16><<<blocks, 256, 0, s>>>((bf16*)qkv, rqk, c, sn, M, T, H, nkv, hd, G);
+    else
+        qknorm_rope_fwd_kernel<float><<<blocks, 256, 0, s>>>((float*)qkv, rqk, c, sn, M, T, H, nkv, hd, G);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const float* rqk, const float* c,
+                                   const float* sn, int M, int T, int H, int nkv, int hd, cudaStream_t s) {
+    int G = qk_group(hd);
+    long long threads = (long long)M * (H + nkv) * G;
+    int blocks = (int)((threads + 255) / 256);
+    if (at == DT_BF16)
+        qknorm_rope_bwd_kernel<bf16><<<blocks, 256, 0, s>>>((bf16*)dqkv, (const bf16*)qkv, rqk, c, sn, M, T, H,
+                                                            nkv, hd, G);
+    else
+        qknorm_rope_bwd_kernel<float><<<blocks, 256, 0, s>>>((float*)dqkv, (const float*)qkv, rqk, c, sn, M, T,
+                                                             H, nkv, hd, G);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R, int V, float cap, float inv_M,
+                            float* loss_rows, void* dl, int* status, cudaStream_t s) {
+    if (R <= 0) return cudaSuccess;
+    if (dlt == DT_BF16)
+        ce_chunk_kernel<bf16><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (bf16*)dl, status);
+    else
+        ce_chunk_kernel<float><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (float*)dl, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_loss_reduce(const float* rows, int M, float* loss, cudaStream_t s) {
+    loss_reduce_kernel<<<1, 1024, 0, s>>>(rows, M, loss);
+    return cudaGetLastError();
+}
+
+static inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t embed_scratch_bytes(int M, int V) {
+    return al256(4ull * V) * 2 + al256(4ull * (V + 1)) + al256(4ull * M) * 2 + al256(4ull * V) + 256;
+}
+
+EmbedScratch embed_scratch_carve(void* base, int M, int V) {
+    char* p = (char*)base;
+    EmbedScratch s;
+    s.count = (int*)p;   p += al256(4ull * V);
+    s.cursor = (int*)p;  p += al256(4ull * V);   // count and cursor adjacent: one memset
+    s.offset = (int*)p;  p += al256(4ull * (V + 1));
+    s.perm = (int*)p;    p += al256(4ull * M);
+    s.perm2 = (int*)p;   p += al256(4ull * M);
+    s.active = (int*)p;  p += al256(4ull * V);
+    s.n_active = (int*)p;
+    return s;
+}
+
+cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int V, int d, float* dwte,
+                                 EmbedScratch sc, cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(sc.count, 0, 2 * al256(4ull * V), s);  // count + cursor
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(dwte, 0, sizeof(float) * (size_t)V * d, s);
+    if (e != cudaSuccess) return e;
+    int mb = (M + 255) / 256;
+    emb_hist_kernel<<<mb, 256, 0, s>>>(idx, M, V, sc.count);
+    emb_scan_kernel<<<1, 1024, 0, s>>>(sc.count, V, sc.offset, sc.active, sc.n_active);
+    emb_fill_kernel<<<mb, 256, 0, s>>>(idx, M, V, sc.offset, sc.cursor, sc.perm);
+    emb_canon_kernel<<<mb, 256, 0, s>>>(idx, V, sc.offset, sc.perm, sc.perm2);
+    int nb = M < V ? M : V;
+    emb_segsum_kernel<<<nb, 128, 0, s>>>(de, d, sc.offset, sc.perm2, sc.active, sc.n_active, dwte);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_splitk_reduce(const float* part, int splits, size_t n, float* out, bool accumulate,
+                                 cudaStream_t s) {
+    size_t n4 = n / 4;
+    splitk_reduce_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(part, splits, n4, out, accumulate);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_expired_wait(int* status, int max_iters, cudaStream_t s) {
+    expired_wait_kernel<<<1, 32, 0, s>>>(status, max_iters);
+    return cudaGetLastError();
+}
+
+}  // namespace nc

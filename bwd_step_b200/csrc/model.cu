@@ -1,0 +1,450 @@
+// C ABI of the step (nanochat_b200.h) and the host-side orchestration: config
+// validation, the flat parameter layout, the workspace plan, and the launch
+// sequence of the forward+backward pass on one stream.
+//
+// Model (nanochat announcement, vpshk.cn, architecture list): normalised
+// token embedding -> n_layer pre-norm blocks [x += Wo attn(rope(norm(q)),
+// rope(norm(k)), v); x += Wproj relu(Wfc norm(x))^2] -> final norm -> untied
+// LM head -> tanh softcap -> mean next-token cross-entropy.
+#include "nanochat_b200.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "gemm_tc.h"
+#include "attention_tc.h"
+
+#include <string>
+#include <vector>
+#include <algorithm>
+
+using namespace nc;
+
+struct ParamEntry { std::string name; int64_t offset; int rows, cols; };
+
+struct nc_model {
+    nc_config cfg;
+    nc_precision prec;
+    int device = 0;
+    int* status = nullptr;  // device int[64]: [0] = status flags, [1] = loss scratch for the host variant
+    std::vector<ParamEntry> layout;
+    int64_t nparams = 0;
+    int V, d, L, H, nkv, hd, F, Nqkv;
+    DType at;  // weight / activation type
+    bool tc = false;  // tcgen05 path available (bf16 on sm_100)
+};
+
+namespace {
+
+#define CK(x) do { cudaError_t e_ = (x); if (e_ != cudaSuccess) return NC_ERR_CUDA; } while (0)
+
+inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Plan {
+    int B = 0, T = 0, M = 0, R = 0;
+    size_t total = 0;
+    size_t tok, tgt, cosb, sinb, x, dx, g, dxb, xf, r0, rf;
+    size_t layers, lay_stride;
+    size_t l_a, l_r1, l_qkv, l_rqk, l_o, l_lse, l_m, l_r2, l_ru, l_h;
+    size_t du, dO, dqkv, Dbuf, zc, dlc, loss_rows, emb, splitk, splitk_bytes, attn_ws, attn_ws_bytes;
+};
+
+// Rows of the LM head processed at once: the [R, V] fp32 logit chunk plus its
+// gradient stay near 1.5 GiB, so the full [B*T, V] logit tensor is never
+// materialised.
+int lm_chunk_rows(const nc_model* m, int M) {
+    size_t per_row = (size_t)m->V * (4 + dt_size(m->at));
+    size_t budget = (size_t)1536 << 20;
+    size_t R = budget / per_row;
+    R = std::max<size_t>(128, R / 128 * 128);
+    return (int)std::min<size_t>(R, (size_t)M);
+}
+
+Plan make_plan(const nc_model* m, int B, int T) {
+    Plan p;
+    p.B = B; p.T = T; p.M = B * T;
+    const size_t M = p.M, d = m->d, A = dt_size(m->at);
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off += al256(bytes); return o; };
+    p.tok = take(4 * M);
+    p.tgt = take(4 * M);
+    p.cosb = take(4ull * T * (m->hd / 2));
+    p.sinb = take(4ull * T * (m->hd / 2));
+    p.x = take(4 * M * d);
+    p.dx = take(4 * M * d);
+    p.g = take(4 * M * d);
+    p.dxb = take(A * M * d);
+    p.xf = take(A * M * d);
+    p.r0 = take(4 * M);
+    p.rf = take(4 * M);
+    // per-layer saved activations
+    size_t lo = 0;
+    auto ltake = [&](size_t bytes) { size_t o = lo; lo += al256(bytes); return o; };
+    p.l_a = ltake(A * M * d);
+    p.l_r1 = ltake(4 * M);
+    p.l_qkv = ltake(A * M * m->Nqkv);
+    p.l_rqk = ltake(4 * M * (m->H + m->nkv));
+    p.l_o = ltake(A * M * m->H * m->hd);
+    p.l_lse = ltake(4 * M * m->H);
+    p.l_m = ltake(A * M * d);
+    p.l_r2 = ltake(4 * M);
+    p.l_ru = ltake(A * M * m->F);
+    p.l_h = ltake(A * M * m->F);
+    p.lay_stride = lo;
+    p.layers = take(lo * m->L);
+    p.du = take(A * M * m->F);
+    p.dO = take(A * M * m->H * m->hd);
+    p.dqkv = take(A * M * m->Nqkv);
+    p.Dbuf = take(4 * M * m->H);
+    p.R = lm_chunk_rows(m, p.M);
+    p.zc = take(4ull * p.R * m->V);
+    p.dlc = take(A * (size_t)p.R * m->V);
+    p.loss_rows = take(4 * M);
+    p.emb = take(embed_scratch_bytes(p.M, m->V));
+    p.splitk_bytes = m->tc ? gemm_tc_splitk_bytes(m->V, m->d, m->F, m->Nqkv, m->H * m->hd) : 0;
+    p.splitk = take(p.splitk_bytes);
+    p.attn_ws_bytes = m->tc ? attention_tc_workspace_bytes(B, T, m->H, m->nkv, m->hd) : 0;
+    p.attn_ws = take(p.attn_ws_bytes);
+    p.total = off;
+    return p;
+}
+
+struct Ctx {
+    nc_model* m;
+    Plan p;
+    char* ws;
+    cudaStream_t s;
+    template <typename T = void> T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
+    char* layer(int l) const { return ws + p.layers + (size_t)l * p.lay_stride; }
+};
+
+// C = A B^T with the tensor-core kernel where it applies, else the FMA kernel.
+int run_gemm(const Ctx& c, const GemmDesc& g) {
+    if (c.m->tc && g.in_t == DT_BF16) {
+        int r = gemm_tc(g, c.ws + c.p.splitk, c.p.splitk_bytes, c.s);
+        if (r == 0) return NC_OK;
+        if (r < 0) return NC_ERR_CUDA;
+        // r > 0: shape not taken by the tensor-core kernel, fall through
+    }
+    CK(gemm_simt(g, c.s));
+    return NC_OK;
+}
+
+GemmDesc mk(const nc_model* m, int M, int N, int K, const void* A, int64_t lda, bool ak, const void* B,
+            int64_t ldb, bool bk, Epi epi, void* C, int64_t ldc, DType ct) {
+    GemmDesc g;
+    g.M = M; g.N = N; g.K = K; g.in_t = m->at;
+    g.A = A; g.lda = lda; g.a_kmajor = ak;
+    g.B = B; g.ldb = ldb; g.b_kmajor = bk;
+    g.epi = epi; g.C = C; g.ldc = ldc; g.c_t = ct;
+    g.cap = m->cfg.softcap;
+    return g;
+}
+
+#define RG(x) do { int r_ = (x); if (r_ != NC_OK) return r_; } while (0)
+
+int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
+    const nc_model* m = c.m;
+    if (m->tc) {
+        int r = attention_tc_fwd(qkv, o, lse, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.ws + c.p.attn_ws,
+                                 c.p.attn_ws_bytes, c.s);
+        if (r == 0) return NC_OK;
+        if (r < 0) return NC_ERR_CUDA;
+    }
+    CK(launch_attention_fwd_simt(m->at, qkv, o, lse, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.s));
+    return NC_OK;
+}
+
+int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv) {
+    const nc_model* m = c.m;
+    float* Dbuf = c.at<float>(c.p.Dbuf);
+    if (m->tc) {
+        int r = attention_tc_bwd(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd,
+                                 c.ws + c.p.attn_ws, c.p.attn_ws_bytes, c.s);
+        if (r == 0) return NC_OK;
+        if (r < 0) return NC_ERR_CUDA;
+    }
+    CK(launch_attention_bwd_simt(m->at, qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.s));
+    return NC_OK;
+}
+
+struct W {  // weight pointers of one call
+    const char* base; size_t es; const nc_model* m;
+    const void* p(int idx) const { return base + (size_t)m->layout[idx].offset * es; }
+    const void* wte() const { return p(0); }
+    const void* wqkv(int l) const { return p(1 + 6 * l); }
+    const void* wo(int l) const { return p(1 + 6 * l + 3); }
+    const void* wfc(int l) const { return p(1 + 6 * l + 4); }
+    const void* wproj(int l) const { return p(1 + 6 * l + 5); }
+    const void* wlm() const { return p(1 + 6 * m->L); }
+};
+
+// Forward through the blocks; with `save` every layer keeps its own
+// activations for the backward, otherwise layer slot 0 is reused.
+int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save) {
+    nc_model* m = c.m;
+    const int M = c.p.M, d = m->d;
+    float* x = c.at<float>(c.p.x);
+    const float* cs = c.at<float>(c.p.cosb);
+    const float* sn = c.at<float>(c.p.sinb);
+    CK(launch_rope_table(c.at<float>(c.p.cosb), c.at<float>(c.p.sinb), c.p.T, m->hd, m->cfg.rope_base, c.s));
+    CK(launch_embed_norm_fwd(m->at, tok, w.wte(), M, m->V, d, x, c.at<float>(c.p.r0), m->status, c.s));
+    const size_t Hhd = (size_t)m->H * m->hd;
+    for (int l = 0; l < m->L; ++l) {
+        char* lb = c.layer(save ? l : 0);
+        void* a = lb + c.p.l_a;
+        void* qkv = lb + c.p.l_qkv;
+        void* o = lb + c.p.l_o;
+        void* mm = lb + c.p.l_m;
+        void* ru = lb + c.p.l_ru;
+        void* h = lb + c.p.l_h;
+        CK(launch_rmsnorm_fwd(m->at, x, a, (float*)(lb + c.p.l_r1), M, d, c.s));
+        RG(run_gemm(c, mk(m, M, m->Nqkv, d, a, d, true, w.wqkv(l), d, true, EPI_STORE, qkv, m->Nqkv, m->at)));
+        CK(launch_qknorm_rope_fwd(m->at, qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, c.p.T, m->H, m->nkv, m->hd,
+                                  c.s));
+        RG(attention_fwd(c, qkv, o, (float*)(lb + c.p.l_lse)));
+        RG(run_gemm(c, mk(m, M, d, (int)Hhd, o, Hhd, true, w.wo(l), Hhd, true, EPI_ACCUM, x, d, DT_F32)));
+        CK(launch_rmsnorm_fwd(m->at, x, mm, (float*)(lb + c.p.l_r2), M, d, c.s));
+        GemmDesc fc = mk(m, M, m->F, d, mm, d, true, w.wfc(l), d, true, EPI_RELU2, h, m->F, m->at);
+        fc.C2 = ru; fc.ldc2 = m->F;
+        RG(run_gemm(c, fc));
+        RG(run_gemm(c, mk(m, M, d, m->F, h, m->F, true, w.wproj(l), m->F, true, EPI_ACCUM, x, d, DT_F32)));
+    }
+    CK(launch_rmsnorm_fwd(m->at, x, c.at(c.p.xf), c.at<float>(c.p.rf), M, d, c.s));
+    return NC_OK;
+}
+
+int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, const void* weights, float* grads,
+         float* loss, void* workspace, cudaStream_t s) {
+    Ctx c{m, make_plan(m, B, T), (char*)workspace, s};
+    W w{(const char*)weights, dt_size(m->at), m};
+    const int M = c.p.M, d = m->d, V = m->V, F = m->F, Nqkv = m->Nqkv;
+    const int Hhd = m->H * m->hd;
+    auto G = [&](int idx) { return grads + m->layout[idx].offset; };
+    RG(forward_blocks(c, w, tok, true));
+
+    // ---- LM head + softcap + cross-entropy, then its backward, R rows at a time
+    void* xf = c.at(c.p.xf);
+    float* gbuf = c.at<float>(c.p.g);
+    float* zc = c.at<float>(c.p.zc);
+    void* dlc = c.at(c.p.dlc);
+    float* loss_rows = c.at<float>(c.p.loss_rows);
+    const size_t A = dt_size(m->at);
+    float* dwlm = G(1 + 6 * m->L);
+    for (int r0 = 0; r0 < M; r0 += c.p.R) {
+        int rc = std::min(c.p.R, M - r0);
+        const char* xfc = (const char*)xf + (size_t)r0 * d * A;
+        RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, DT_F32)));
+        CK(launch_ce_chunk(m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M, loss_rows + r0, dlc,
+                           m->status, s));
+        RG(run_gemm(c, mk(m, rc, d, V, dlc, V, true, w.wlm(), d, false, EPI_STORE, gbuf + (size_t)r0 * d, d,
+                          DT_F32)));
+        RG(run_gemm(c, mk(m, V, d, rc, dlc, V, false, xfc, d, false, r0 == 0 ? EPI_STORE : EPI_ACCUM, dwlm, d,
+                          DT_F32)));
+    }
+    CK(launch_loss_reduce(loss_rows, M, loss, s));
+
+    // ---- backward through the blocks
+    float* dx = c.at<float>(c.p.dx);
+    void* dxb = c.at(c.p.dxb);
+    CK(launch_rmsnorm_bwd(m->at, gbuf, xf, c.at<float>(c.p.rf), dx, false, dxb, M, d, s));
+    void* du = c.at(c.p.du);
+    void* dO = c.at(c.p.dO);
+    void* dqkv = c.at(c.p.dqkv);
+    const float* cs = c.at<float>(c.p.cosb);
+    const float* sn = c.at<float>(c.p.sinb);
+    for (int l = m->L - 1; l >= 0; --l) {
+        char* lb = c.layer(l);
+        int base = 1 + 6 * l;
+        // MLP: x_out = x_mid + h Wproj^T, h = relu(u)^2, u = m Wfc^T
+        GemmDesc g1 = mk(m, M, F, d, dxb, d, true, w.wproj(l), F, false, EPI_RELU2_BWD, du, F, m->at);
+        g1.aux = lb + c.p.l_ru; g1.ldaux = F;
+        RG(run_gemm(c, g1));
+        RG(run_gemm(c, mk(m, d, F, M, dxb, d, false, lb + c.p.l_h, F, false, EPI_STORE, G(base + 5), F, DT_F32)));
+        RG(run_gemm(c, mk(m, M, d, F, du, F, true, w.wfc(l), d, false, EPI_STORE, gbuf, d, DT_F32)));
+        RG(run_gemm(c, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32)));
+        CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_m, (float*)(lb + c.p.l_r2), dx, true, dxb, M, d, s));
+        // attention: x_mid = x_in + o Wo^T
+        RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at)));
+        RG(run_gemm(c, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
+                          DT_F32)));
+        RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), dqkv));
+        CK(launch_qknorm_rope_bwd(m->at, dqkv, lb + c.p.l_qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, T, m->H,
+                                  m->nkv, m->hd, s));
+        RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, DT_F32)));
+        RG(run_gemm(c, mk(m, Nqkv, d, M, dqkv, Nqkv, false, lb + c.p.l_a, d, false, EPI_STORE, G(base), d,
+                          DT_F32)));
+        CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_a, (float*)(lb + c.p.l_r1), dx, true, l > 0 ? dxb : nullptr,
+                              M, d, s));
+    }
+    // ---- token embedding: norm backward, then the deterministic scatter-add
+    CK(launch_embed_norm_bwd(m->at, dx, tok, w.wte(), c.at<float>(c.p.r0), gbuf, M, V, d, s));
+    CK(launch_embed_scatter(tok, gbuf, M, V, d, G(0), embed_scratch_carve(c.ws + c.p.emb, M, V), s));
+    return NC_OK;
+}
+
+int validate_call(nc_model* m, int B, int T, size_t ws_bytes, const void* const* ptrs, int nptr) {
+    if (!m || B <= 0 || T <= 0) return NC_ERR_INVALID_ARG;
+    if ((long long)B * T > (1 << 24)) return NC_ERR_UNSUPPORTED_SHAPE;
+    for (int i = 0; i < nptr; ++i)
+        if (!ptrs[i]) return NC_ERR_INVALID_ARG;
+    if (ws_bytes < make_plan(m, B, T).total) return NC_ERR_WORKSPACE_TOO_SMALL;
+    return NC_OK;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+extern "C" {
+
+int nc_model_create(const nc_config* cfg, nc_precision prec, nc_model** out) {
+    if (!out) return NC_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!cfg) return NC_ERR_INVALID_ARG;
+    if (prec != NC_PREC_BF16 && prec != NC_PREC_FP32_DEBUG) return NC_ERR_INVALID_ARG;
+    const nc_config& c = *cfg;
+    if (c.vocab <= 0 || c.d_model <= 0 || c.n_layer <= 0 || c.n_head <= 0 || c.n_kv_head <= 0 ||
+        c.head_dim <= 0 || c.mlp_mult <= 0 || !(c.softcap > 0.f) || !(c.rope_base > 1.f))
+        return NC_ERR_INVALID_ARG;
+    if (c.vocab % 64 || c.d_model % 64 || c.n_head % c.n_kv_head) return NC_ERR_UNSUPPORTED_SHAPE;
+    if (c.head_dim != 16 && c.head_dim != 32 && c.head_dim != 64 && c.head_dim != 128)
+        return NC_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)c.vocab * c.d_model > (1ll << 31) || (long long)c.mlp_mult * c.d_model > (1 << 20))
+        return NC_ERR_UNSUPPORTED_SHAPE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NC_ERR_NO_DEVICE;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10)
+        return NC_ERR_NO_DEVICE;
+    nc_model* m = new nc_model();
+    m->cfg = c;
+    m->prec = prec;
+    m->device = dev;
+    m->V = c.vocab; m->d = c.d_model; m->L = c.n_layer; m->H = c.n_head; m->nkv = c.n_kv_head;
+    m->hd = c.head_dim; m->F = c.mlp_mult * c.d_model; m->Nqkv = (c.n_head + 2 * c.n_kv_head) * c.head_dim;
+    m->at = prec == NC_PREC_BF16 ? DT_BF16 : DT_F32;
+    m->tc = prec == NC_PREC_BF16;
+    int64_t off = 0;
+    auto add = [&](const std::string& n, int r, int cc) { m->layout.push_back({n, off, r, cc}); off += (int64_t)r * cc; };
+    add("wte", m->V, m->d);
+    for (int l = 0; l < m->L; ++l) {
+        std::string p = "h." + std::to_string(l) + ".";
+        add(p + "wq", m->H * m->hd, m->d);
+        add(p + "wk", m->nkv * m->hd, m->d);
+        add(p + "wv", m->nkv * m->hd, m->d);
+        add(p + "wo", m->d, m->H * m->hd);
+        add(p + "wfc", m->F, m->d);
+        add(p + "wproj", m->d, m->F);
+    }
+    add("wlm", m->V, m->d);
+    m->nparams = off;
+    if (cudaMalloc(&m->status, 64 * sizeof(int)) != cudaSuccess ||
+        cudaMemset(m->status, 0, 64 * sizeof(int)) != cudaSuccess) {
+        cudaFree(m->status);
+        delete m;
+        return NC_ERR_CUDA;
+    }
+    *out = m;
+    return NC_OK;
+}
+
+void nc_model_destroy(nc_model* m) {
+    if (!m) return;
+    cudaFree(m->status);
+    delete m;
+}
+
+int64_t nc_num_params(const nc_model* m) { return m ? m->nparams : 0; }
+
+int nc_param_layout(const nc_model* m, int i, const char** name, int64_t* offset, int* rows, int* cols) {
+    if (!m || i < 0 || i >= (int)m->layout.size()) return NC_ERR_INVALID_ARG;
+    const ParamEntry& e = m->layout[i];
+    if (name) *name = e.name.c_str();
+    if (offset) *offset = e.offset;
+    if (rows) *rows = e.rows;
+    if (cols) *cols = e.cols;
+    return NC_OK;
+}
+
+size_t nc_workspace_bytes(const nc_model* m, int B, int T) {
+    if (!m || B <= 0 || T <= 0 || (long long)B * T > (1 << 24)) return 0;
+    return make_plan(m, B, T).total;
+}
+
+int nc_forward_backward(nc_model* m, const int32_t* tokens, const int32_t* targets, int B, int T,
+                        const void* weights, float* grads, float* loss, void* workspace, size_t ws_bytes,
+                        void* stream) {
+    const void* ptrs[] = {tokens, targets, weights, grads, loss, workspace};
+    int v = validate_call(m, B, T, ws_bytes, ptrs, 6);
+    if (v != NC_OK) return v;
+    int r = step(m, tokens, targets, B, T, weights, grads, loss, workspace, (cudaStream_t)stream);
+    if (r != NC_OK) return r;
+    return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+int nc_forward_backward_host(nc_model* m, const int32_t* h_tokens, const int32_t* h_targets, int B, int T,
+                             const void* weights, float* grads, float* h_loss, void* workspace, size_t ws_bytes,
+                             void* stream) {
+    const void* ptrs[] = {h_tokens, h_targets, weights, grads, h_loss, workspace};
+    int v = validate_call(m, B, T, ws_bytes, ptrs, 6);
+    if (v != NC_OK) return v;
+    cudaStream_t s = (cudaStream_t)stream;
+    Plan p = make_plan(m, B, T);
+    char* ws = (char*)workspace;
+    int32_t* dtok = (int32_t*)(ws + p.tok);
+    int32_t* dtgt = (int32_t*)(ws + p.tgt);
+    size_t bytes = sizeof(int32_t) * (size_t)B * T;
+    CK(cudaMemcpyAsync(dtok, h_tokens, bytes, cudaMemcpyHostToDevice, s));
+    CK(cudaMemcpyAsync(dtgt, h_targets, bytes, cudaMemcpyHostToDevice, s));
+    float* dloss = (float*)(m->status + 1);
+    int r = step(m, dtok, dtgt, B, T, weights, grads, dloss, workspace, s);
+    if (r != NC_OK) return r;
+    CK(cudaMemcpyAsync(h_loss, dloss, sizeof(float), cudaMemcpyDeviceToHost, s));
+    CK(cudaStreamSynchronize(s));
+    return NC_OK;
+}
+
+int nc_forward_logits(nc_model* m, const int32_t* tokens, int B, int T, const void* weights, void* logits,
+                      void* workspace, size_t ws_bytes, void* stream) {
+    const void* ptrs[] = {tokens, weights, logits, workspace};
+    int v = validate_call(m, B, T, ws_bytes, ptrs, 4);
+    if (v != NC_OK) return v;
+    Ctx c{m, make_plan(m, B, T), (char*)workspace, (cudaStream_t)stream};
+    W w{(const char*)weights, dt_size(m->at), m};
+    RG(forward_blocks(c, w, tokens, false));
+    RG(run_gemm(c, mk(m, c.p.M, m->V, m->d, c.at(c.p.xf), m->d, true, w.wlm(), m->d, true, EPI_SOFTCAP, logits,
+                      m->V, m->at)));
+    return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+int nc_check(nc_model* m, void* stream) {
+    if (!m) return NC_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NC_ERR_CUDA;
+    int st = 0;
+    if (cudaMemcpy(&st, m->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NC_ERR_CUDA;
+    if (cudaMemset(m->status, 0, sizeof(int)) != cudaSuccess) return NC_ERR_CUDA;
+    if (st & ST_TIMEOUT) return NC_ERR_DEVICE_TIMEOUT;
+    if (st & ST_BAD_TOKEN) return NC_ERR_BAD_TOKEN;
+    return NC_OK;
+}
+
+const char* nc_status_string(int code) {
+    switch (code) {
+        case NC_OK: return "ok";
+        case NC_ERR_INVALID_ARG: return "invalid argument";
+        case NC_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case NC_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case NC_ERR_CUDA: return "CUDA error";
+        case NC_ERR_BAD_TOKEN: return "token or target id out of range";
+        case NC_ERR_DEVICE_TIMEOUT: return "bounded device wait expired";
+        case NC_ERR_NO_DEVICE: return "no sm_100 CUDA device";
+    }
+    return "unknown status";
+}
+
+int nc_debug_expired_wait(nc_model* m, int max_iters, void* stream) {
+    if (!m || max_iters <= 0) return NC_ERR_INVALID_ARG;
+    CK(launch_expired_wait(m->status, max_iters, (cudaStream_t)stream));
+    return NC_OK;
+}
+
+}  // extern "C"

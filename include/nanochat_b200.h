@@ -1,0 +1,148 @@
+/*
+ * nanochat_b200.h -- C ABI of the B200 (sm_100a) forward+backward pretraining
+ * step of the nanochat-style dense decoder.
+ *
+ * The model is the one listed in the architecture section of the nanochat
+ * announcement (vpshk.cn, "Andrej Karpathy open-sources nanochat"): a dense,
+ * Llama-like decoder with rotary position embeddings only, QK-norm, untied
+ * embedding and unembedding, a normalised token embedding, a relu^2 MLP,
+ * parameter-free RMSNorm, bias-free linears, multi-query attention and a
+ * tanh logit softcap.  The loss is the mean next-token cross-entropy over all
+ * B*T positions, and the step returns the gradient of that mean with respect
+ * to every weight.  Readings of points the pages leave open (RMSNorm eps,
+ * final norm, RoPE pairing and frequencies, attention scale, causal mask) are
+ * fixed here and stated next to the declarations they affect.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named d_* or documented as "device" are device memory owned by
+ *     the caller.  The library never frees them and never keeps them after the
+ *     call returns (it only enqueues work that reads or writes them).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls only enqueue work; they do not synchronise, except
+ *     nc_check and nc_forward_backward_host (see there).
+ *   - Return values are NC_OK (0) or a negative NC_ERR_* code describing
+ *     argument validation or launch failure.  Errors found on the device
+ *     (token id out of range, a bounded wait that expired) are recorded in a
+ *     device status word owned by the model and reported by nc_check.
+ *   - All matrices are row-major.  A linear layer is y = x W^T with W stored
+ *     [out, in].
+ */
+#ifndef NANOCHAT_B200_H
+#define NANOCHAT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define NC_OK                       0
+#define NC_ERR_INVALID_ARG         -1  /* null pointer, non-positive size, bad index      */
+#define NC_ERR_UNSUPPORTED_SHAPE   -2  /* config outside what the kernels implement      */
+#define NC_ERR_WORKSPACE_TOO_SMALL -3  /* ws_bytes < nc_workspace_bytes(model, B, T)      */
+#define NC_ERR_CUDA                -4  /* a CUDA runtime call or kernel launch failed    */
+#define NC_ERR_BAD_TOKEN           -5  /* device: a token or target id outside [0, V)    */
+#define NC_ERR_DEVICE_TIMEOUT      -6  /* device: a bounded wait in a kernel gave up     */
+#define NC_ERR_NO_DEVICE           -7  /* no sm_100 device current when the model was made */
+
+/* Parameter-free RMSNorm epsilon: y = x / sqrt(mean(x^2) + NC_RMS_EPS).  The
+ * pages give no value; 1e-6 is used everywhere (token-embedding norm, the two
+ * pre-norms of every block, QK-norm, final norm). */
+#define NC_RMS_EPS 1e-6f
+
+/* Model shape.  d_model = n_head*head_dim is not required.  MLP hidden width
+ * is mlp_mult*d_model.  Supported: d_model % 64 == 0, head_dim in
+ * {16, 32, 64, 128}, n_head % n_kv_head == 0, vocab % 64 == 0, softcap > 0,
+ * rope_base > 1.  RoPE rotates the pairs (j, j + head_dim/2) of every q and
+ * k head by pos * rope_base^(-2j/head_dim), positions 0..T-1 in each row. */
+typedef struct {
+    int vocab, d_model, n_layer, n_head, n_kv_head, head_dim, mlp_mult;
+    float softcap, rope_base;
+} nc_config;
+
+/* Arithmetic of the step.
+ * NC_PREC_BF16: bf16 weights, bf16 GEMM/attention operands on the tcgen05
+ *   tensor cores with fp32 accumulation; fp32 residual stream, norm
+ *   statistics, softmax and loss.
+ * NC_PREC_FP32_DEBUG: fp32 weights and activations everywhere, plain fp32
+ *   FMA kernels (no tensor cores, no TF32). */
+typedef enum { NC_PREC_BF16 = 0, NC_PREC_FP32_DEBUG = 1 } nc_precision;
+
+typedef struct nc_model nc_model; /* opaque */
+
+/* Validates cfg and creates a model bound to the current CUDA device.  Host
+ * state plus one small device status word (allocated here, freed by
+ * nc_model_destroy).  *out is set to NULL on error. */
+int nc_model_create(const nc_config* cfg, nc_precision prec, nc_model** out);
+void nc_model_destroy(nc_model* m);
+
+/* Number of parameter elements (= elements of the flat weight and gradient
+ * buffers). */
+int64_t nc_num_params(const nc_model* m);
+
+/* Flat parameter layout, entry i in [0, 2 + 6*n_layer): name, element offset,
+ * rows, cols.  Order: "wte" [V,d]; per layer i "h.i.wq" [H*hd,d],
+ * "h.i.wk" [nkv*hd,d], "h.i.wv" [nkv*hd,d], "h.i.wo" [d,H*hd],
+ * "h.i.wfc" [F,d], "h.i.wproj" [d,F]; then "wlm" [V,d].  *name points to
+ * library-owned storage valid for the model's lifetime. */
+int nc_param_layout(const nc_model* m, int i, const char** name, int64_t* offset,
+                    int* rows, int* cols);
+
+/* Bytes of device workspace nc_forward_backward / nc_forward_logits need for
+ * batch B and sequence length T.  Returns 0 for invalid B, T. */
+size_t nc_workspace_bytes(const nc_model* m, int B, int T);
+
+/* One forward+backward step (the hot path).
+ *   tokens, targets: device int32 [B, T], row-major contiguous.  targets are
+ *     the next-token ids (tokens shifted by one in the caller's stream).
+ *   weights: device, nc_num_params elements, bf16 (NC_PREC_BF16) or fp32
+ *     (NC_PREC_FP32_DEBUG), in the nc_param_layout order.
+ *   grads: device fp32, nc_num_params elements; OVERWRITTEN with the gradient
+ *     of the mean loss (not accumulated).
+ *   loss: device fp32 scalar; receives mean_{b,t} [logsumexp(z) - z[target]]
+ *     with z = softcap * tanh(logits / softcap).
+ *   workspace: device, at least nc_workspace_bytes(m, B, T) bytes, 256-byte
+ *     aligned; its contents on entry are ignored.
+ * The full [B*T, V] logit tensor is never written to memory.  Results are
+ * bitwise reproducible for a given model, inputs and workspace size. */
+int nc_forward_backward(nc_model* m, const int32_t* tokens, const int32_t* targets,
+                        int B, int T, const void* weights, float* grads, float* loss,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Same step with the per-step inputs and the result in HOST memory:
+ * h_tokens / h_targets are host int32 [B, T] (pinned memory gives an
+ * asynchronous copy), h_loss a host float.  The ids are copied into the
+ * workspace, the step is enqueued on `stream`, the loss is copied back, and
+ * the call synchronises `stream` before returning.  Weights, grads and the
+ * workspace are device memory as for nc_forward_backward. */
+int nc_forward_backward_host(nc_model* m, const int32_t* h_tokens, const int32_t* h_targets,
+                             int B, int T, const void* weights, float* grads, float* h_loss,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Forward pass only; writes the softcapped logits z [B, T, V] (bf16 for
+ * NC_PREC_BF16, fp32 for NC_PREC_FP32_DEBUG) to the device buffer `logits`.
+ * This is the only call that materialises logits. */
+int nc_forward_logits(nc_model* m, const int32_t* tokens, int B, int T, const void* weights,
+                      void* logits, void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word:
+ * NC_OK, NC_ERR_BAD_TOKEN or NC_ERR_DEVICE_TIMEOUT (or NC_ERR_CUDA if the
+ * stream reported an error). */
+int nc_check(nc_model* m, void* stream);
+
+/* Static description of a return code. */
+const char* nc_status_string(int code);
+
+/* Test hook for the bounded device wait: launches one kernel that waits on an
+ * mbarrier nobody arrives at, with an iteration cap of `max_iters`; when the
+ * cap is hit the kernel records NC_ERR_DEVICE_TIMEOUT in the status word and
+ * returns (no trap, the context stays usable).  Read the result with
+ * nc_check. */
+int nc_debug_expired_wait(nc_model* m, int max_iters, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NANOCHAT_B200_H */

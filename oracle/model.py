@@ -229,11 +229,11 @@ def _row_forward(cfg, P, idx, cos, sin, keep):
     return saved
 
 
-def _row_backward(cfg, P, G, idx, saved, dxf, cos, sin):
+def _row_backward(cfg, P, G, idx, saved, dxf, cos, sin, min_layer=0):
     T = idx.shape[0]
     H, nkv, hd = cfg.n_head, cfg.n_kv_head, cfg.head_dim
     dx = rmsnorm_backward(dxf, saved["xf"], saved["rf"])
-    for i in reversed(range(cfg.n_layer)):
+    for i in reversed(range(min_layer, cfg.n_layer)):
         s = saved["layers"][i]
         # x_out = x_mid + relu(m Wfc^T)^2 Wproj^T
         dh = dx @ P[f"h.{i}.wproj"]
@@ -254,15 +254,19 @@ def _row_backward(cfg, P, G, idx, saved, dxf, cos, sin):
         G[f"h.{i}.wv"] += dv.T @ a
         da = dq @ P[f"h.{i}.wq"] + dk @ P[f"h.{i}.wk"] + dv @ P[f"h.{i}.wv"]
         dx = dx + rmsnorm_backward(da, a, s["r1"])
+    if min_layer > 0:
+        return
     de = rmsnorm_backward(dx, saved["x0"], saved["r0"])
     np.add.at(G["wte"], idx, de)
 
 
-def step(cfg, weights, tokens, targets):
+def step(cfg, weights, tokens, targets, min_layer=0):
     """Mean cross-entropy loss and the gradient of every weight.
 
     weights: flat vector in `layout` order (any float dtype; used as float64).
     tokens, targets: int [B, T].  Returns (loss: float, grads: flat float64).
+    min_layer > 0 stops the backward after layer min_layer (used to bound the
+    cost on large shapes): gradients of layers below it and of wte stay zero.
     """
     tokens = np.asarray(tokens)
     targets = np.asarray(targets)
@@ -281,7 +285,7 @@ def step(cfg, weights, tokens, targets):
         losses, dxf, dwlm = lm_head_loss(saved["xf"], P["wlm"], targets[b], cfg.softcap, scale)
         G["wlm"] += dwlm
         total += losses.sum()
-        _row_backward(cfg, P, G, tokens[b], saved, dxf, cos, sin)
+        _row_backward(cfg, P, G, tokens[b], saved, dxf, cos, sin, min_layer)
     return total * scale, grads
 
 

@@ -1,0 +1,77 @@
+"""CPU-side checks of the C ABI: the in-tree library loads, exports every
+entry point the public header declares, and refuses to run without a GPU."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import bwd_step_b200
+from bwd_step_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(nc_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("nc_model_create", "nc_forward_backward", "nc_forward_logits", "nc_workspace_bytes",
+              "nc_param_layout", "nc_check"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = bwd_step_b200.lib()
+    for n in sorted(_declared()):
+        assert hasattr(L, n), n
+        assert n in _lib.SIGNATURES, f"binding lacks {n}"
+
+
+def test_status_strings():
+    L = bwd_step_b200.lib()
+    for code in range(-7, 1):
+        assert L.nc_status_string(code)
+    assert L.nc_status_string(0) == b"ok"
+
+
+def test_create_rejects_bad_config_without_touching_a_device():
+    cfg = _lib.NcConfig(512, 64, 2, 4, 1, 16, 4, 15.0, 10000.0)
+    out = ctypes.c_void_p()
+    L = bwd_step_b200.lib()
+    assert L.nc_model_create(None, 0, ctypes.byref(out)) == _lib.NC_ERR_INVALID_ARG
+    assert L.nc_model_create(ctypes.byref(cfg), 7, ctypes.byref(out)) == _lib.NC_ERR_INVALID_ARG
+    bad = _lib.NcConfig(512, 64, 2, 4, 1, 24, 4, 15.0, 10000.0)  # head_dim 24
+    assert L.nc_model_create(ctypes.byref(bad), 0, ctypes.byref(out)) == _lib.NC_ERR_UNSUPPORTED_SHAPE
+    bad = _lib.NcConfig(512, 64, 2, 3, 2, 16, 4, 15.0, 10000.0)  # n_head % n_kv_head
+    assert L.nc_model_create(ctypes.byref(bad), 0, ctypes.byref(out)) == _lib.NC_ERR_UNSUPPORTED_SHAPE
+    bad = _lib.NcConfig(512, 64, 2, 4, 1, 16, 4, -1.0, 10000.0)  # softcap <= 0
+    assert L.nc_model_create(ctypes.byref(bad), 0, ctypes.byref(out)) == _lib.NC_ERR_INVALID_ARG
+    assert out.value is None
+
+
+def test_no_cpu_fallback():
+    """Without a CUDA device the product path refuses to run."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(bwd_step_b200.NcError) as e:
+        bwd_step_b200.Model({"vocab": 512, "d_model": 64, "n_layer": 2, "n_head": 4, "n_kv_head": 1,
+                             "head_dim": 16, "mlp_mult": 4, "softcap": 15.0, "rope_base": 10000.0})
+    assert e.value.code == _lib.NC_ERR_NO_DEVICE
+
+
+def test_product_path_does_not_reference_the_oracle():
+    pkg = os.path.join(ROOT, "bwd_step_b200")
+    for path in glob.glob(os.path.join(pkg, "**", "*.*"), recursive=True):
+        if path.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+            src = open(path).read()
+            assert not re.search(r"\boracle\b", src), path

@@ -368,3 +368,16 @@ def test_tiny_golden_regression():
     G = oracle.views(TINY.model, g)
     for name in G:
         assert abs(np.linalg.norm(G[name]) - vals["norm." + name]) <= 1e-12 * vals["norm." + name] + 1e-300
+
+
+def test_truncated_backward_matches_full_on_the_layers_it_keeps():
+    cfg, w, tok, tgt = _tiny_inputs(seed_w=61)
+    loss, g = oracle.step(cfg, w, tok, tgt)
+    loss1, g1 = oracle.step(cfg, w, tok, tgt, min_layer=1)
+    assert loss1 == loss
+    G, G1 = oracle.views(cfg, g), oracle.views(cfg, g1)
+    for name in G:
+        if name.startswith("h.1.") or name == "wlm":
+            np.testing.assert_array_equal(G1[name], G[name])
+        else:
+            assert np.all(G1[name] == 0)
