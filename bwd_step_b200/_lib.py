@@ -24,6 +24,11 @@ NC_PREC_BF16 = 0
 NC_PREC_FP32_DEBUG = 1
 
 
+class NcProfileRow(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_char_p), ("launches", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
 class NcConfig(ctypes.Structure):
     _fields_ = [("vocab", ctypes.c_int), ("d_model", ctypes.c_int), ("n_layer", ctypes.c_int),
                 ("n_head", ctypes.c_int), ("n_kv_head", ctypes.c_int), ("head_dim", ctypes.c_int),
@@ -47,7 +52,14 @@ SIGNATURES = {
     "nc_forward_logits": (_I, [_P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "nc_check": (_I, [_P, _P]),
     "nc_status_string": (ctypes.c_char_p, [_I]),
+    "nc_profile_enable": (_I, [_P, _I]),
+    "nc_profile_read": (_I, [_P, _P, ctypes.POINTER(NcProfileRow), _I]),
+    "nc_launch_count": (ctypes.c_int64, []),
     "nc_debug_expired_wait": (_I, [_P, _I, _P]),
+    # include/nanochat_b200_testing.h
+    "nc_test_gemm": (_I, [_I, _I, _I, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _P,
+                          ctypes.c_int64, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_float, _I, _P,
+                          _SZ, _P, _P]),
 }
 
 _lib = None

@@ -40,6 +40,11 @@ def _ptr(t, dtype=None, name="tensor"):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def launch_count() -> int:
+    """Kernels launched by the CUDA library in this process so far."""
+    return int(lib().nc_launch_count())
+
+
 class Model:
     """A model handle: shape, precision and the flat parameter layout."""
 
@@ -123,6 +128,19 @@ class Model:
     def check(self, stream=None) -> int:
         """Synchronise the stream and return (and clear) the device status code."""
         return int(lib().nc_check(self._h, ctypes.c_void_p(_stream_handle(stream))))
+
+    def profile(self, enable: bool):
+        """Start (clearing) or stop per-kernel-class event timing."""
+        _ok(lib().nc_profile_enable(self._h, 1 if enable else 0), "nc_profile_enable")
+
+    def profile_read(self, stream=None):
+        """Aggregated rows {kernel, launches, ms, flops, bytes} (synchronises the stream)."""
+        rows = (_lib.NcProfileRow * 32)()
+        n = lib().nc_profile_read(self._h, ctypes.c_void_p(_stream_handle(stream)), rows, 32)
+        if n < 0:
+            raise NcError(n, "nc_profile_read")
+        return [dict(kernel=r.kernel.decode(), launches=r.launches, ms=r.ms, flops=r.flops, bytes=r.bytes)
+                for r in rows[:n]]
 
     def debug_expired_wait(self, max_iters: int, stream=None):
         _ok(lib().nc_debug_expired_wait(self._h, max_iters, ctypes.c_void_p(_stream_handle(stream))),

@@ -257,6 +257,7 @@ template <typename A, int HD>
 cudaError_t fwd_t(const void* qkv, void* o, float* lse, int B, int T, int H, int nkv, cudaStream_t s) {
     dim3 grid((T + WPB - 1) / WPB, H, B);
     attn_fwd_kernel<A, HD><<<grid, 256, 0, s>>>((const A*)qkv, (A*)o, lse, T, H, nkv);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -269,6 +270,7 @@ cudaError_t bwd_t(const void* qkv, const void* o, const void* dO, const float* l
     attn_bwd_dq_kernel<A, HD><<<gq, 256, 0, s>>>((const A*)qkv, (const A*)dO, lse, Dbuf, (A*)dqkv, T, H, nkv);
     dim3 gk((T + WPB - 1) / WPB, nkv, B);
     attn_bwd_dkv_kernel<A, HD><<<gk, 256, 0, s>>>((const A*)qkv, (const A*)dO, lse, Dbuf, (A*)dqkv, T, H, nkv);
+    count_launch(3);
     return cudaGetLastError();
 }
 

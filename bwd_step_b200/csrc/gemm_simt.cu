@@ -93,6 +93,7 @@ cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t s) {
     if (grid.y > 65535) return cudaErrorInvalidConfiguration;
     if (g.in_t == DT_BF16) gemm_simt_kernel<bf16><<<grid, 256, 0, s>>>(g);
     else gemm_simt_kernel<float><<<grid, 256, 0, s>>>(g);
+    count_launch();
     return cudaGetLastError();
 }
 

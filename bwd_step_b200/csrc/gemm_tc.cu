@@ -1,5 +1,376 @@
+// tcgen05 GEMM for the step's linears: C = A B^T with bf16 operands and fp32
+// accumulation in tensor memory (TMEM).  It serves every dense contraction of
+// the bias-free linears (nanochat announcement, vpshk.cn, architecture list:
+// "no biases in linear layers") in the forward and in both backward products
+// (dX = dY W, dW = dY^T X), and the untied LM head.
+//
+// Design (one CTA per SM, persistent over output tiles):
+//   warp 0     TMA producer: 128x64 A and 256x64 B bf16 tiles, 128-byte
+//              swizzle, into a 4-stage shared-memory ring;
+//   warp 1     allocates 512 TMEM columns and issues tcgen05.mma
+//              (M=128, N=256, K=16) from one thread; commits release ring
+//              slots and hand finished accumulators to the epilogue;
+//   warps 2-5  epilogue: tcgen05.ld of their 32 TMEM lanes (one output row per
+//              thread), fused elementwise work, 16-byte global stores.
+// Two 256-column accumulators let the epilogue of one tile overlap the main
+// loop of the next.  Operands may be K-major or M/N-major (the backward
+// products read activations and weights transposed without a copy).
+// Split-K (fixed order, deterministic reduction) is used when there are too
+// few output tiles to fill the SMs.  Every mbarrier wait is bounded.
 #include "gemm_tc.h"
+#include "tc_common.cuh"
+#include <cudaTypedefs.h>
+#include <algorithm>
+
 namespace nc {
-int gemm_tc(const GemmDesc&, void*, size_t, cudaStream_t) { return 1; }
-size_t gemm_tc_splitk_bytes(int, int, int, int, int) { return 0; }
+namespace {
+using namespace tc;
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 2 * BN;
+constexpr int NTHREADS = 192;
+constexpr int MAX_SPLITS = 8;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+
+struct TcParams {
+    int M, N, K;
+    int tiles_m, tiles_n, splits, kb_per_split, num_kb, num_units, tn_fast;
+    int a_mn, b_mn;
+    int epi, c_bf16, vec_ok;
+    void* C; int64_t ldc;
+    void* C2; int64_t ldc2;
+    const bf16* aux; int64_t ldaux;
+    float cap;
+    float* part;  // split-K partial sums [splits][M][N], or null
+    int* status;
+};
+
+__device__ __forceinline__ void decode(const TcParams& p, int u, int& tm, int& tn, int& ks) {
+    int tile = u % (p.tiles_m * p.tiles_n);
+    ks = u / (p.tiles_m * p.tiles_n);
+    if (p.tn_fast) { tm = tile / p.tiles_n; tn = tile % p.tiles_n; }
+    else { tn = tile / p.tiles_m; tm = tile % p.tiles_m; }
+}
+
+__device__ __forceinline__ void store_row_f32(float* dst, const float* v, int nv, bool vec) {
+    if (vec && nv == 32) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+        for (int i = 0; i < nv; ++i) dst[i] = v[i];
+    }
+}
+__device__ __forceinline__ void store_row_bf16(bf16* dst, const float* v, int nv, bool vec) {
+    if (vec && nv == 32) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) store_vec(dst + 8 * i, v + 8 * i);
+    } else {
+        for (int i = 0; i < nv; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+    }
+}
+__device__ __forceinline__ void store_row(void* C, bool bf, int64_t off, const float* v, int nv, bool vec) {
+    if (bf) store_row_bf16(reinterpret_cast<bf16*>(C) + off, v, nv, vec);
+    else store_row_f32(reinterpret_cast<float*>(C) + off, v, nv, vec);
+}
+
+// Epilogue of 32 consecutive columns n0.. of one output row.
+__device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int n0, float* v) {
+    const int nv = min(32, p.N - n0);
+    const bool vec = p.vec_ok != 0;
+    if (p.part) {
+        store_row_f32(p.part + ((size_t)ks * p.M + row) * p.N + n0, v, nv, vec);
+        return;
+    }
+    const int64_t off = (int64_t)row * p.ldc + n0;
+    switch (p.epi) {
+        case EPI_STORE: store_row(p.C, p.c_bf16, off, v, nv, vec); break;
+        case EPI_ACCUM: {
+            float* c = reinterpret_cast<float*>(p.C) + off;
+            if (vec && nv == 32) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float4 o = reinterpret_cast<float4*>(c)[i];
+                    v[4 * i] += o.x; v[4 * i + 1] += o.y; v[4 * i + 2] += o.z; v[4 * i + 3] += o.w;
+                }
+            } else {
+                for (int i = 0; i < nv; ++i) v[i] += c[i];
+            }
+            store_row_f32(c, v, nv, vec);
+        } break;
+        case EPI_RELU2: {
+            float r[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) { r[i] = fmaxf(v[i], 0.f); v[i] = r[i] * r[i]; }
+            store_row_bf16(reinterpret_cast<bf16*>(p.C) + off, v, nv, vec);
+            store_row_bf16(reinterpret_cast<bf16*>(p.C2) + (int64_t)row * p.ldc2 + n0, r, nv, vec);
+        } break;
+        case EPI_RELU2_BWD: {
+            const bf16* a = p.aux + (int64_t)row * p.ldaux + n0;
+            if (vec && nv == 32) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float u[8];
+                    load_vec(a + 8 * i, u);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[8 * i + j] *= 2.f * u[j];
+                }
+            } else {
+                for (int i = 0; i < nv; ++i) v[i] *= 2.f * __bfloat162float(a[i]);
+            }
+            store_row_bf16(reinterpret_cast<bf16*>(p.C) + off, v, nv, vec);
+        } break;
+        case EPI_SOFTCAP: {
+            const float ic = 1.f / p.cap;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = p.cap * tanhf(v[i] * ic);
+            store_row(p.C, p.c_bf16, off, v, nv, vec);
+        } break;
+    }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * STAGE_BYTES);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t tiles_base = smem_u32(smem);
+    const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * STAGES;
+    const uint32_t bar_tfull = bar_empty + 8 * STAGES, bar_tempty = bar_tfull + 16;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(bar_full + 8 * s, 1); mbar_init(bar_empty + 8 * s, 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(bar_tfull + 8 * b, 1); mbar_init(bar_tempty + 8 * b, 4); }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    if (warp == 0 && lane == 0) { tma_prefetch(&tmA); tma_prefetch(&tmB); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, issued_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+                int tm, tn, ks;
+                decode(p, u, tm, tn, ks);
+                const int kb0 = ks * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+                    const uint32_t fb = bar_full + 8 * stage;
+                    const uint32_t sa = tiles_base + stage * STAGE_BYTES, sb = sa + A_BYTES;
+                    mbar_expect_tx(fb, STAGE_BYTES);
+                    if (!p.a_mn) {
+                        tma_load_2d(sa, &tmA, kb * BK, tm * BM, fb);
+                    } else {
+                        tma_load_2d(sa, &tmA, tm * BM, kb * BK, fb);
+                        tma_load_2d(sa + 8192, &tmA, tm * BM + 64, kb * BK, fb);
+                    }
+                    if (!p.b_mn) {
+                        tma_load_2d(sb, &tmB, kb * BK, tn * BN, fb);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) tma_load_2d(sb + j * 8192, &tmB, tn * BN + 64 * j, kb * BK, fb);
+                    }
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                // Let the copies already in flight land before the block exits.
+                for (int s = 0; s < STAGES; ++s) {
+                    if (!(issued >> s & 1)) continue;
+                    uint64_t t0 = globaltimer();
+                    while (!mbar_try(bar_full + 8 * s, (issued_phase >> s) & 1) && globaltimer() - t0 < 1000000ull) {}
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer
+            const uint32_t idesc = idesc_bf16(BM, BN, p.a_mn != 0, p.b_mn != 0);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+                int tm, tn, ks;
+                decode(p, u, tm, tn, ks);
+                const int kb0 = ks * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * BN;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = tiles_base + stage * STAGE_BYTES, sb = sa + A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const uint64_t ad = p.a_mn ? smem_desc(sa + k * 2048, 8192, 1024) : smem_desc(sa + k * 32, 16, 1024);
+                        const uint64_t bd = p.b_mn ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
+                        mma_bf16(d, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar_empty + 8 * stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(bar_tfull + 8 * acc);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+        }
+    } else {
+        // ---------------- epilogue warps 2..5; warp w reads TMEM lanes 32*(w%4)..
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+            int tm, tn, ks;
+            decode(p, u, tm, tn, ks);
+            if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, p.status)) break;
+            tc_fence_after();
+            const int row = tm * BM + q * 32 + lane;
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n0 = tn * BN + c * 32;
+                if (n0 >= p.N) break;
+                float v[32];
+                tmem_ld32(tb + c * 32, v);
+                if (row < p.M) epilogue(p, ks, row, n0, v);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [outer, inner] array with row stride ld
+// elements; box [box_outer, box_inner], 128-byte swizzle, zero fill out of range.
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner,
+              uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+}  // namespace
+
+size_t gemm_tc_splitk_bytes(size_t max_out_elems) { return (size_t)MAX_SPLITS * max_out_elems * sizeof(float); }
+
+int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s) {
+    if (g.in_t != DT_BF16) return 1;
+    if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 1;
+    auto al16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
+    if (!al16(g.A) || !al16(g.B) || (g.lda * 2) % 16 || (g.ldb * 2) % 16) return 1;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
+            cudaSuccess)
+            return -1;
+        attr_set = true;
+    }
+    CUtensorMap ta, tb;
+    bool ok = g.a_kmajor ? make_map(&ta, g.A, g.K, g.M, g.lda, 64, BM) : make_map(&ta, g.A, g.M, g.K, g.lda, 64, 64);
+    ok = ok && (g.b_kmajor ? make_map(&tb, g.B, g.K, g.N, g.ldb, 64, BN) : make_map(&tb, g.B, g.N, g.K, g.ldb, 64, 64));
+    if (!ok) return 1;
+
+    TcParams p{};
+    p.M = g.M; p.N = g.N; p.K = g.K;
+    p.tiles_m = (g.M + BM - 1) / BM;
+    p.tiles_n = (g.N + BN - 1) / BN;
+    p.num_kb = (g.K + BK - 1) / BK;
+    p.tn_fast = p.tiles_n <= p.tiles_m ? 1 : 0;
+    p.a_mn = g.a_kmajor ? 0 : 1;
+    p.b_mn = g.b_kmajor ? 0 : 1;
+    p.epi = g.epi;
+    p.c_bf16 = g.c_t == DT_BF16 ? 1 : 0;
+    p.C = g.C; p.ldc = g.ldc; p.C2 = g.C2; p.ldc2 = g.ldc2;
+    p.aux = reinterpret_cast<const bf16*>(g.aux); p.ldaux = g.ldaux;
+    p.cap = g.cap;
+    p.status = g.status;
+    const int esz = p.c_bf16 ? 2 : 4;
+    bool vec = al16(g.C) && (g.ldc * esz) % 16 == 0;
+    if (g.epi == EPI_RELU2) vec = vec && al16(g.C2) && (g.ldc2 * 2) % 16 == 0;
+    if (g.epi == EPI_RELU2_BWD) vec = vec && al16(g.aux) && (g.ldaux * 2) % 16 == 0;
+
+    // split-K when the output tiles cannot fill the SMs
+    const int sms = num_sms();
+    const int tiles = p.tiles_m * p.tiles_n;
+    int splits = 1;
+    const bool can_split = (g.epi == EPI_STORE || g.epi == EPI_ACCUM) && !p.c_bf16 && g.ldc == g.N && splitk &&
+                           g.N % 4 == 0;
+    if (can_split && tiles < 2 * sms) {
+        double best = (double)((tiles + sms - 1) / sms);
+        for (int sp = 2; sp <= MAX_SPLITS; ++sp) {
+            if (p.num_kb / sp < 8) break;
+            if ((size_t)sp * g.M * g.N * sizeof(float) > splitk_bytes) break;
+            double cost = (double)((tiles * sp + sms - 1) / sms) / sp;
+            if (cost < best - 1e-9) { best = cost; splits = sp; }
+        }
+    }
+    p.kb_per_split = (p.num_kb + splits - 1) / splits;
+    p.splits = (p.num_kb + p.kb_per_split - 1) / p.kb_per_split;
+    p.part = p.splits > 1 ? reinterpret_cast<float*>(splitk) : nullptr;
+    p.vec_ok = (p.part ? (g.N % 4 == 0) : vec) ? 1 : 0;
+    p.num_units = tiles * p.splits;
+    const int grid = std::min(p.num_units, sms);
+    gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return -1;
+    if (p.part) {
+        if (launch_splitk_reduce(p.part, p.splits, (size_t)g.M * g.N, reinterpret_cast<float*>(g.C),
+                                 g.epi == EPI_ACCUM, s) != cudaSuccess)
+            return -1;
+    }
+    return 0;
+}
+
 }  // namespace nc

@@ -8,5 +8,6 @@ namespace nc {
 // layout is not taken (the caller falls back), < 0 on a CUDA error.
 // `splitk` is scratch for split-K partial sums (gemm_tc_splitk_bytes bytes).
 int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s);
-size_t gemm_tc_splitk_bytes(int V, int d, int F, int Nqkv, int Hhd);
+// Split-K scratch for outputs of at most max_out_elems fp32 elements.
+size_t gemm_tc_splitk_bytes(size_t max_out_elems);
 }  // namespace nc

@@ -4,7 +4,13 @@
 #include <stdint.h>
 #include <stddef.h>
 
+#include <atomic>
+
 namespace nc {
+
+// Kernels launched by this library so far (process-wide), for launch accounting.
+extern std::atomic<long long> g_launches;
+inline void count_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 enum DType : int { DT_F32 = 0, DT_BF16 = 1 };
 inline size_t dt_size(DType t) { return t == DT_BF16 ? 2 : 4; }
@@ -79,6 +85,7 @@ struct GemmDesc {
     void* C2 = nullptr; int64_t ldc2 = 0;
     const void* aux = nullptr; int64_t ldaux = 0;
     float cap = 0.f;
+    int* status = nullptr;  // device status word for bounded-wait timeouts
 };
 
 // Plain fp32-FMA tiled GEMM (any strides, any sizes).

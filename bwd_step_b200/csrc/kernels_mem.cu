@@ -436,10 +436,13 @@ __global__ void expired_wait_kernel(int* status, int max_iters) {
 
 }  // namespace
 
+std::atomic<long long> g_launches{0};
+
 // ============================================================================ launchers
 cudaError_t launch_rope_table(float* c, float* s, int T, int hd, float base, cudaStream_t st) {
     int n = T * (hd / 2);
     rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(c, s, T, hd, (double)base);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -449,6 +452,7 @@ cudaError_t launch_embed_norm_fwd(DType wt, const int32_t* idx, const void* wte,
         embed_norm_fwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(idx, (const bf16*)wte, M, V, d, x, r0, status);
     else
         embed_norm_fwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(idx, (const float*)wte, M, V, d, x, r0, status);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -457,6 +461,7 @@ cudaError_t launch_rmsnorm_fwd(DType at, const float* x, void* y, float* r, int 
         rmsnorm_fwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(x, (bf16*)y, r, M, d);
     else
         rmsnorm_fwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(x, (float*)y, r, M, d);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -468,6 +473,7 @@ cudaError_t launch_rmsnorm_bwd(DType at, const float* dy, const void* y, const f
     else
         rmsnorm_bwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(dy, (const float*)y, r, dx, accumulate,
                                                                 (float*)dxb, M, d);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -477,6 +483,7 @@ cudaError_t launch_embed_norm_bwd(DType wt, const float* dx, const int32_t* idx,
         embed_norm_bwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(dx, idx, (const bf16*)wte, r0, de, M, V, d);
     else
         embed_norm_bwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(dx, idx, (const float*)wte, r0, de, M, V, d);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -491,6 +498,7 @@ cudaError_t launch_qknorm_rope_fwd(DType at, void* qkv, float* rqk, const float*
         qknorm_rope_fwd_kernel<bf16><<<blocks, 256, 0, s>>>((bf16*)qkv, rqk, c, sn, M, T, H, nkv, hd, G);
     else
         qknorm_rope_fwd_kernel<float><<<blocks, 256, 0, s>>>((float*)qkv, rqk, c, sn, M, T, H, nkv, hd, G);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -505,6 +513,7 @@ cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const 
     else
         qknorm_rope_bwd_kernel<float><<<blocks, 256, 0, s>>>((float*)dqkv, (const float*)qkv, rqk, c, sn, M, T,
                                                              H, nkv, hd, G);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -515,11 +524,13 @@ cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R
         ce_chunk_kernel<bf16><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (bf16*)dl, status);
     else
         ce_chunk_kernel<float><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (float*)dl, status);
+    count_launch();
     return cudaGetLastError();
 }
 
 cudaError_t launch_loss_reduce(const float* rows, int M, float* loss, cudaStream_t s) {
     loss_reduce_kernel<<<1, 1024, 0, s>>>(rows, M, loss);
+    count_launch();
     return cudaGetLastError();
 }
 
@@ -555,6 +566,7 @@ cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int
     emb_canon_kernel<<<mb, 256, 0, s>>>(idx, V, sc.offset, sc.perm, sc.perm2);
     int nb = M < V ? M : V;
     emb_segsum_kernel<<<nb, 128, 0, s>>>(de, d, sc.offset, sc.perm2, sc.active, sc.n_active, dwte);
+    count_launch(5);
     return cudaGetLastError();
 }
 
@@ -562,11 +574,13 @@ cudaError_t launch_splitk_reduce(const float* part, int splits, size_t n, float*
                                  cudaStream_t s) {
     size_t n4 = n / 4;
     splitk_reduce_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(part, splits, n4, out, accumulate);
+    count_launch();
     return cudaGetLastError();
 }
 
 cudaError_t launch_expired_wait(int* status, int max_iters, cudaStream_t s) {
     expired_wait_kernel<<<1, 32, 0, s>>>(status, max_iters);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -30,6 +30,20 @@ struct nc_model {
     int V, d, L, H, nkv, hd, F, Nqkv;
     DType at;  // weight / activation type
     bool tc = false;  // tcgen05 path available (bf16 on sm_100)
+    // profiler: CUDA events around every launch while enabled
+    struct Rec { int cls; cudaEvent_t a, b; double flops, bytes; long long launches; };
+    bool prof_on = false;
+    std::vector<cudaEvent_t> ev_pool;
+    size_t ev_next = 0;
+    std::vector<Rec> recs;
+    cudaEvent_t event() {
+        if (ev_next == ev_pool.size()) {
+            cudaEvent_t e = nullptr;
+            if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+            ev_pool.push_back(e);
+        }
+        return ev_pool[ev_next++];
+    }
 };
 
 namespace {
@@ -99,7 +113,8 @@ Plan make_plan(const nc_model* m, int B, int T) {
     p.dlc = take(A * (size_t)p.R * m->V);
     p.loss_rows = take(4 * M);
     p.emb = take(embed_scratch_bytes(p.M, m->V));
-    p.splitk_bytes = m->tc ? gemm_tc_splitk_bytes(m->V, m->d, m->F, m->Nqkv, m->H * m->hd) : 0;
+    size_t max_out = std::max({(size_t)p.R * d, (size_t)m->F * d, (size_t)m->H * m->hd * d, (size_t)m->Nqkv * d});
+    p.splitk_bytes = m->tc ? gemm_tc_splitk_bytes(max_out) : 0;
     p.splitk = take(p.splitk_bytes);
     p.attn_ws_bytes = m->tc ? attention_tc_workspace_bytes(B, T, m->H, m->nkv, m->hd) : 0;
     p.attn_ws = take(p.attn_ws_bytes);
@@ -116,13 +131,42 @@ struct Ctx {
     char* layer(int l) const { return ws + p.layers + (size_t)l * p.lay_stride; }
 };
 
+enum ProfCls {
+    P_GEMM_TC = 0, P_GEMM_FMA, P_ATTN_FWD, P_ATTN_BWD, P_NORM_FWD, P_NORM_BWD, P_QKROPE_FWD, P_QKROPE_BWD,
+    P_EMBED_FWD, P_EMBED_BWD, P_CE, P_OTHER, P_COUNT
+};
+const char* const kProfNames[P_COUNT] = {
+    "gemm_tcgen05", "gemm_fma", "attention_fwd", "attention_bwd", "rmsnorm_fwd", "rmsnorm_bwd",
+    "qknorm_rope_fwd", "qknorm_rope_bwd", "embed_fwd", "embed_bwd", "cross_entropy", "other"};
+
+// Records a CUDA event pair around the launches made in its lifetime (only
+// while profiling is enabled), with the algorithmic FLOPs / HBM bytes of the work.
+struct Prof {
+    nc_model* m; cudaStream_t s; int cls; double flops, bytes; cudaEvent_t a = nullptr; long long l0 = 0;
+    Prof(const Ctx& c, int cls_, double f, double b) : m(c.m), s(c.s), cls(cls_), flops(f), bytes(b) {
+        if (m->prof_on && (a = m->event())) { cudaEventRecord(a, s); l0 = g_launches.load(); }
+    }
+    ~Prof() {
+        if (!a) return;
+        cudaEvent_t b = m->event();
+        if (!b) return;
+        cudaEventRecord(b, s);
+        m->recs.push_back({cls, a, b, flops, bytes, g_launches.load() - l0});
+    }
+};
+
 // C = A B^T with the tensor-core kernel where it applies, else the FMA kernel.
 int run_gemm(const Ctx& c, const GemmDesc& g) {
+    const double es = g.in_t == DT_BF16 ? 2.0 : 4.0;
+    Prof pr(c, P_GEMM_TC, 2.0 * g.M * g.N * (double)g.K,
+            es * ((double)g.M * g.K + (double)g.N * g.K) + (g.c_t == DT_BF16 ? 2.0 : 4.0) * g.M * (double)g.N);
+    pr.cls = (c.m->tc && g.in_t == DT_BF16) ? P_GEMM_TC : P_GEMM_FMA;
     if (c.m->tc && g.in_t == DT_BF16) {
         int r = gemm_tc(g, c.ws + c.p.splitk, c.p.splitk_bytes, c.s);
         if (r == 0) return NC_OK;
         if (r < 0) return NC_ERR_CUDA;
         // r > 0: shape not taken by the tensor-core kernel, fall through
+        pr.cls = P_GEMM_FMA;
     }
     CK(gemm_simt(g, c.s));
     return NC_OK;
@@ -136,13 +180,21 @@ GemmDesc mk(const nc_model* m, int M, int N, int K, const void* A, int64_t lda, 
     g.B = B; g.ldb = ldb; g.b_kmajor = bk;
     g.epi = epi; g.C = C; g.ldc = ldc; g.c_t = ct;
     g.cap = m->cfg.softcap;
+    g.status = m->status;
     return g;
 }
 
 #define RG(x) do { int r_ = (x); if (r_ != NC_OK) return r_; } while (0)
 
+// Causal attention FLOPs of one pass over the batch: QK^T and PV over the
+// T(T+1)/2 visible (query, key) pairs of every head.
+double attn_flops(const Ctx& c) {
+    return 4.0 * c.p.B * c.m->H * (double)c.m->hd * (double)c.p.T * (c.p.T + 1) / 2.0;
+}
+
 int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
     const nc_model* m = c.m;
+    Prof pr(c, P_ATTN_FWD, attn_flops(c), 0.0);
     if (m->tc) {
         int r = attention_tc_fwd(qkv, o, lse, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.ws + c.p.attn_ws,
                                  c.p.attn_ws_bytes, c.s);
@@ -155,6 +207,7 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
 
 int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv) {
     const nc_model* m = c.m;
+    Prof pr(c, P_ATTN_BWD, 2.0 * attn_flops(c), 0.0);
     float* Dbuf = c.at<float>(c.p.Dbuf);
     if (m->tc) {
         int r = attention_tc_bwd(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd,
@@ -185,8 +238,12 @@ int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save) {
     float* x = c.at<float>(c.p.x);
     const float* cs = c.at<float>(c.p.cosb);
     const float* sn = c.at<float>(c.p.sinb);
-    CK(launch_rope_table(c.at<float>(c.p.cosb), c.at<float>(c.p.sinb), c.p.T, m->hd, m->cfg.rope_base, c.s));
-    CK(launch_embed_norm_fwd(m->at, tok, w.wte(), M, m->V, d, x, c.at<float>(c.p.r0), m->status, c.s));
+    {
+        Prof pr(c, P_OTHER, 0.0, 8.0 * c.p.T * (m->hd / 2));
+        CK(launch_rope_table(c.at<float>(c.p.cosb), c.at<float>(c.p.sinb), c.p.T, m->hd, m->cfg.rope_base, c.s));
+    }
+    const double A = (double)dt_size(m->at);
+    { Prof pr(c, P_EMBED_FWD, 0.0, (double)M * (A * d + 4.0 * d + 8.0)); CK(launch_embed_norm_fwd(m->at, tok, w.wte(), M, m->V, d, x, c.at<float>(c.p.r0), m->status, c.s)); }
     const size_t Hhd = (size_t)m->H * m->hd;
     for (int l = 0; l < m->L; ++l) {
         char* lb = c.layer(save ? l : 0);
@@ -196,19 +253,22 @@ int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save) {
         void* mm = lb + c.p.l_m;
         void* ru = lb + c.p.l_ru;
         void* h = lb + c.p.l_h;
-        CK(launch_rmsnorm_fwd(m->at, x, a, (float*)(lb + c.p.l_r1), M, d, c.s));
+        { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, a, (float*)(lb + c.p.l_r1), M, d, c.s)); }
         RG(run_gemm(c, mk(m, M, m->Nqkv, d, a, d, true, w.wqkv(l), d, true, EPI_STORE, qkv, m->Nqkv, m->at)));
-        CK(launch_qknorm_rope_fwd(m->at, qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, c.p.T, m->H, m->nkv, m->hd,
-                                  c.s));
+        {
+            Prof pr(c, P_QKROPE_FWD, 0.0, (double)M * (m->H + m->nkv) * (2.0 * A * m->hd + 4.0));
+            CK(launch_qknorm_rope_fwd(m->at, qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, c.p.T, m->H, m->nkv, m->hd,
+                                      c.s));
+        }
         RG(attention_fwd(c, qkv, o, (float*)(lb + c.p.l_lse)));
         RG(run_gemm(c, mk(m, M, d, (int)Hhd, o, Hhd, true, w.wo(l), Hhd, true, EPI_ACCUM, x, d, DT_F32)));
-        CK(launch_rmsnorm_fwd(m->at, x, mm, (float*)(lb + c.p.l_r2), M, d, c.s));
+        { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, mm, (float*)(lb + c.p.l_r2), M, d, c.s)); }
         GemmDesc fc = mk(m, M, m->F, d, mm, d, true, w.wfc(l), d, true, EPI_RELU2, h, m->F, m->at);
         fc.C2 = ru; fc.ldc2 = m->F;
         RG(run_gemm(c, fc));
         RG(run_gemm(c, mk(m, M, d, m->F, h, m->F, true, w.wproj(l), m->F, true, EPI_ACCUM, x, d, DT_F32)));
     }
-    CK(launch_rmsnorm_fwd(m->at, x, c.at(c.p.xf), c.at<float>(c.p.rf), M, d, c.s));
+    { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, c.at(c.p.xf), c.at<float>(c.p.rf), M, d, c.s)); }
     return NC_OK;
 }
 
@@ -233,19 +293,22 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         int rc = std::min(c.p.R, M - r0);
         const char* xfc = (const char*)xf + (size_t)r0 * d * A;
         RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, DT_F32)));
-        CK(launch_ce_chunk(m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M, loss_rows + r0, dlc,
-                           m->status, s));
+        {
+            Prof pr(c, P_CE, 0.0, (double)rc * V * (4.0 + A));
+            CK(launch_ce_chunk(m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M, loss_rows + r0, dlc,
+                               m->status, s));
+        }
         RG(run_gemm(c, mk(m, rc, d, V, dlc, V, true, w.wlm(), d, false, EPI_STORE, gbuf + (size_t)r0 * d, d,
                           DT_F32)));
         RG(run_gemm(c, mk(m, V, d, rc, dlc, V, false, xfc, d, false, r0 == 0 ? EPI_STORE : EPI_ACCUM, dwlm, d,
                           DT_F32)));
     }
-    CK(launch_loss_reduce(loss_rows, M, loss, s));
+    { Prof pr(c, P_OTHER, 0.0, 4.0 * M); CK(launch_loss_reduce(loss_rows, M, loss, s)); }
 
     // ---- backward through the blocks
     float* dx = c.at<float>(c.p.dx);
     void* dxb = c.at(c.p.dxb);
-    CK(launch_rmsnorm_bwd(m->at, gbuf, xf, c.at<float>(c.p.rf), dx, false, dxb, M, d, s));
+    { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (8.0 * d + 2.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, xf, c.at<float>(c.p.rf), dx, false, dxb, M, d, s)); }
     void* du = c.at(c.p.du);
     void* dO = c.at(c.p.dO);
     void* dqkv = c.at(c.p.dqkv);
@@ -261,23 +324,33 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         RG(run_gemm(c, mk(m, d, F, M, dxb, d, false, lb + c.p.l_h, F, false, EPI_STORE, G(base + 5), F, DT_F32)));
         RG(run_gemm(c, mk(m, M, d, F, du, F, true, w.wfc(l), d, false, EPI_STORE, gbuf, d, DT_F32)));
         RG(run_gemm(c, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32)));
-        CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_m, (float*)(lb + c.p.l_r2), dx, true, dxb, M, d, s));
+        { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (12.0 * d + 2.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_m, (float*)(lb + c.p.l_r2), dx, true, dxb, M, d, s)); }
         // attention: x_mid = x_in + o Wo^T
         RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at)));
         RG(run_gemm(c, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
                           DT_F32)));
         RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), dqkv));
-        CK(launch_qknorm_rope_bwd(m->at, dqkv, lb + c.p.l_qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, T, m->H,
-                                  m->nkv, m->hd, s));
+        {
+            Prof pr(c, P_QKROPE_BWD, 0.0, (double)M * (m->H + m->nkv) * (3.0 * A * m->hd + 4.0));
+            CK(launch_qknorm_rope_bwd(m->at, dqkv, lb + c.p.l_qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, T, m->H,
+                                      m->nkv, m->hd, s));
+        }
         RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, DT_F32)));
         RG(run_gemm(c, mk(m, Nqkv, d, M, dqkv, Nqkv, false, lb + c.p.l_a, d, false, EPI_STORE, G(base), d,
                           DT_F32)));
-        CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_a, (float*)(lb + c.p.l_r1), dx, true, l > 0 ? dxb : nullptr,
-                              M, d, s));
+        {
+            Prof pr(c, P_NORM_BWD, 0.0, (double)M * (12.0 * d + (l > 0 ? 2.0 : 1.0) * A * d + 4.0));
+            CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_a, (float*)(lb + c.p.l_r1), dx, true,
+                                  l > 0 ? dxb : nullptr, M, d, s));
+        }
     }
     // ---- token embedding: norm backward, then the deterministic scatter-add
-    CK(launch_embed_norm_bwd(m->at, dx, tok, w.wte(), c.at<float>(c.p.r0), gbuf, M, V, d, s));
-    CK(launch_embed_scatter(tok, gbuf, M, V, d, G(0), embed_scratch_carve(c.ws + c.p.emb, M, V), s));
+    {
+        // norm backward (dx, Wte row, r0 -> de), then de read once and dWte written once
+        Prof pr(c, P_EMBED_BWD, 0.0, (double)M * (8.0 * d + A * d + 8.0) + 4.0 * M * d + 4.0 * (double)V * d);
+        CK(launch_embed_norm_bwd(m->at, dx, tok, w.wte(), c.at<float>(c.p.r0), gbuf, M, V, d, s));
+        CK(launch_embed_scatter(tok, gbuf, M, V, d, G(0), embed_scratch_carve(c.ws + c.p.emb, M, V), s));
+    }
     return NC_OK;
 }
 
@@ -348,6 +421,7 @@ int nc_model_create(const nc_config* cfg, nc_precision prec, nc_model** out) {
 
 void nc_model_destroy(nc_model* m) {
     if (!m) return;
+    for (cudaEvent_t e : m->ev_pool) cudaEventDestroy(e);
     cudaFree(m->status);
     delete m;
 }
@@ -441,6 +515,37 @@ const char* nc_status_string(int code) {
     return "unknown status";
 }
 
+int nc_profile_enable(nc_model* m, int enable) {
+    if (!m) return NC_ERR_INVALID_ARG;
+    if (enable) { m->recs.clear(); m->ev_next = 0; }
+    m->prof_on = enable != 0;
+    return NC_OK;
+}
+
+int nc_profile_read(nc_model* m, void* stream, nc_profile_row* rows, int max_rows) {
+    if (!m || (!rows && max_rows > 0)) return NC_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return NC_ERR_CUDA;
+    nc_profile_row agg[P_COUNT] = {};
+    bool seen[P_COUNT] = {};
+    for (const auto& r : m->recs) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return NC_ERR_CUDA;
+        nc_profile_row& a = agg[r.cls];
+        a.kernel = kProfNames[r.cls];
+        a.launches += r.launches;
+        a.ms += ms;
+        a.flops += r.flops;
+        a.bytes += r.bytes;
+        seen[r.cls] = true;
+    }
+    int n = 0;
+    for (int k = 0; k < P_COUNT; ++k)
+        if (seen[k] && n < max_rows) rows[n++] = agg[k];
+    return n;
+}
+
+int64_t nc_launch_count(void) { return g_launches.load(); }
+
 int nc_debug_expired_wait(nc_model* m, int max_iters, void* stream) {
     if (!m || max_iters <= 0) return NC_ERR_INVALID_ARG;
     CK(launch_expired_wait(m->status, max_iters, (cudaStream_t)stream));
@@ -448,3 +553,27 @@ int nc_debug_expired_wait(nc_model* m, int max_iters, void* stream) {
 }
 
 }  // extern "C"
+
+// ============================================================================ testing ABI
+#include "nanochat_b200_testing.h"
+
+extern "C" int nc_test_gemm(int M, int N, int K, int in_bf16, const void* A, int64_t lda, int a_kmajor,
+                            const void* B, int64_t ldb, int b_kmajor, int epi, void* C, int64_t ldc, int c_bf16,
+                            void* C2, int64_t ldc2, const void* aux, int64_t ldaux, float cap, int use_tc,
+                            void* scratch, size_t scratch_bytes, int* status, void* stream) {
+    if (M <= 0 || N <= 0 || K <= 0 || !A || !B || !C || epi < 0 || epi > 4) return NC_ERR_INVALID_ARG;
+    if ((epi == EPI_RELU2 && !C2) || (epi == EPI_RELU2_BWD && !aux)) return NC_ERR_INVALID_ARG;
+    GemmDesc g;
+    g.M = M; g.N = N; g.K = K; g.in_t = in_bf16 ? DT_BF16 : DT_F32;
+    g.A = A; g.lda = lda; g.a_kmajor = a_kmajor != 0;
+    g.B = B; g.ldb = ldb; g.b_kmajor = b_kmajor != 0;
+    g.epi = (Epi)epi; g.C = C; g.ldc = ldc; g.c_t = c_bf16 ? DT_BF16 : DT_F32;
+    g.C2 = C2; g.ldc2 = ldc2; g.aux = aux; g.ldaux = ldaux; g.cap = cap; g.status = status;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (use_tc) {
+        int r = gemm_tc(g, scratch, scratch_bytes, s);
+        if (r > 0) return NC_ERR_UNSUPPORTED_SHAPE;
+        return r == 0 ? NC_OK : NC_ERR_CUDA;
+    }
+    return gemm_simt(g, s) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}

@@ -135,6 +135,26 @@ int nc_check(nc_model* m, void* stream);
 /* Static description of a return code. */
 const char* nc_status_string(int code);
 
+/* Per-kernel-class timing.  While enabled, every launch made by this model
+ * is bracketed by CUDA events on its stream, tagged with the kernel class and
+ * the algorithmic work of the call (FLOPs for contractions, HBM bytes for the
+ * memory-bound kernels).  nc_profile_enable(m, 1) clears the record and
+ * starts; (m, 0) stops.  nc_profile_read synchronises `stream` and writes up
+ * to max_rows aggregated rows (one per kernel class seen); returns the number
+ * of rows or a negative code.  `kernel` points to static storage. */
+typedef struct {
+    const char* kernel;
+    int64_t launches;  /* kernel launches of this class */
+    double ms;         /* summed event time */
+    double flops;      /* algorithmic FLOPs */
+    double bytes;      /* algorithmic HBM bytes */
+} nc_profile_row;
+int nc_profile_enable(nc_model* m, int enable);
+int nc_profile_read(nc_model* m, void* stream, nc_profile_row* rows, int max_rows);
+
+/* Kernels launched by the library in this process so far. */
+int64_t nc_launch_count(void);
+
 /* Test hook for the bounded device wait: launches one kernel that waits on an
  * mbarrier nobody arrives at, with an iteration cap of `max_iters`; when the
  * cap is hit the kernel records NC_ERR_DEVICE_TIMEOUT in the status word and
