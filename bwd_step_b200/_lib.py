@@ -60,6 +60,7 @@ SIGNATURES = {
     "nc_test_gemm": (_I, [_I, _I, _I, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _P,
                           ctypes.c_int64, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_float, _I, _P,
                           _SZ, _P, _P]),
+    "nc_test_attention": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P]),
 }
 
 _lib = None

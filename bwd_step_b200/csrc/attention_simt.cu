@@ -305,6 +305,16 @@ cudaError_t launch_attention_fwd_simt(DType at, const void* qkv, void* o, float*
                          : fwd_d<float>(qkv, o, lse, B, T, H, nkv, hd, s);
 }
 
+cudaError_t launch_attention_bwd_dot(DType at, const void* o, const void* dO, float* D, int MH, int hd,
+                                     cudaStream_t s) {
+    if (at == DT_BF16)
+        attn_bwd_dot_kernel<bf16><<<(MH + WPB - 1) / WPB, 256, 0, s>>>((const bf16*)o, (const bf16*)dO, D, MH, hd);
+    else
+        attn_bwd_dot_kernel<float><<<(MH + WPB - 1) / WPB, 256, 0, s>>>((const float*)o, (const float*)dO, D, MH, hd);
+    count_launch();
+    return cudaGetLastError();
+}
+
 cudaError_t launch_attention_bwd_simt(DType at, const void* qkv, const void* o, const void* dO,
                                       const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int nkv,
                                       int hd, cudaStream_t s) {

@@ -1,7 +1,825 @@
+// Causal multi-query attention on the tcgen05 tensor cores (bf16 operands,
+// fp32 accumulation in TMEM, fp32 softmax).  Model item: multi-query
+// attention, every query head reading the one shared K/V head (nanochat
+// announcement, vpshk.cn, architecture list), causal within a row, scores
+// scaled by 1/sqrt(hd).
+//
+// Forward, one CTA per (query block of 128 positions, head, batch row):
+//   warp 0     TMA: the Q tile once, then K_j / V_j tiles (2-stage rings)
+//              for key blocks j = 0..qb (causal: blocks past the diagonal
+//              are never loaded);
+//   warp 1     tcgen05.mma: S_j = Q K_j^T into one of two TMEM score
+//              buffers, then O += P_{j-1} V_{j-1} (issued one block behind,
+//              so the next score tile is computed while softmax runs);
+//   warps 2-5  softmax, one query row per thread: scores from TMEM, causal
+//              mask on the diagonal block, running max in the log2 domain
+//              with lazy rescaling of O (only when the max grows by more
+//              than 2^8), P as bf16 into shared memory in the 128-byte
+//              swizzled K-major layout the next MMA reads.
+// The K/V head is shared by all query heads; its tiles are re-read by the
+// H CTAs of a query block from L2.
 #include "attention_tc.h"
+#include "tc_common.cuh"
+#include <cudaTypedefs.h>
+
 namespace nc {
-int attention_tc_fwd(const void*, void*, float*, int, int, int, int, int, void*, size_t, cudaStream_t) { return 1; }
-int attention_tc_bwd(const void*, const void*, const void*, const float*, float*, void*, int, int, int, int, int,
-                     void*, size_t, cudaStream_t) { return 1; }
+namespace {
+using namespace tc;
+
+constexpr int NT = 192;
+constexpr int STG = 2;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
+
+struct AttnParams {
+    int B, T, H, nkv, nqb;
+    float scale_log2;  // log2(e) / sqrt(hd)
+    bf16* o;
+    float* lse;
+    int* status;
+};
+
+template <int HD>
+struct FwdLayout {
+    static constexpr int KB = HD / 64;          // 64-column blocks of the head dim
+    static constexpr int TILE = KB * 16384;     // [128 x HD] bf16, 128B-swizzled
+    static constexpr int Q = 0;
+    static constexpr int K = Q + TILE;
+    static constexpr int V = K + STG * TILE;
+    static constexpr int P = V + STG * TILE;    // [128 x 128] bf16
+    static constexpr int BAR = P + 32768;
+    static constexpr int BYTES = BAR + 256 + 1024;  // + barriers, + alignment slack
+};
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int HD>
+__global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnParams p) {
+    using Lay = FwdLayout<HD>;
+    constexpr int KB = Lay::KB;
+    constexpr int TILE = Lay::TILE;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t base = smem_u32(smem);
+    const uint32_t sQ = base + Lay::Q, sK = base + Lay::K, sV = base + Lay::V, sP = base + Lay::P;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
+    const uint32_t b0 = smem_u32(bars);
+    const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 24, v_full = b0 + 40, v_empty = b0 + 56;
+    const uint32_t s_full = b0 + 72, s_empty = b0 + 88, p_full = b0 + 104, o_done = b0 + 112;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qb = p.nqb - 1 - (int)blockIdx.x;  // largest blocks first
+    const int h = blockIdx.y, b = blockIdx.z, g = h / (p.H / p.nkv);
+    const int nblk = qb + 1;
+    const int row0 = b * p.T;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < STG; ++s) {
+            mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1);
+            mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1);
+        }
+        for (int s = 0; s < 2; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(s_empty + 8 * s, 4); }
+        mbar_init(p_full, 4);
+        mbar_init(o_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+    if (warp == 0 && lane == 0) tma_prefetch(&tm);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tO = tmem + 256;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const int xq = h * HD, xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
+            mbar_expect_tx(q_full, TILE);
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) tma_load_2d(sQ + kb * 16384, &tm, xq + kb * 64, row0 + qb * 128, q_full);
+            int issued = 0;
+            for (int j = 0; j < nblk; ++j) {
+                const int st = j % STG;
+                const uint32_t ph = (j / STG) & 1;
+                if (!mbar_wait(k_empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(k_full + 8 * st, TILE);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_2d(sK + st * TILE + kb * 16384, &tm, xk + kb * 64, row0 + j * 128, k_full + 8 * st);
+                if (!mbar_wait(v_empty + 8 * st, ph ^ 1, abort_flag, p.status)) { issued = j + 1; break; }
+                mbar_expect_tx(v_full + 8 * st, TILE);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_2d(sV + st * TILE + kb * 16384, &tm, xv + kb * 64, row0 + j * 128, v_full + 8 * st);
+                issued = j + 1;
+            }
+            if (*abort_flag) {
+                // let copies in flight land before the block exits
+                uint64_t t0 = globaltimer();
+                while (!mbar_try(q_full, 0) && globaltimer() - t0 < 1000000ull) {}
+                for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j) {
+                    const int st = j % STG;
+                    const uint32_t ph = (j / STG) & 1;
+                    t0 = globaltimer();
+                    while (!mbar_try(k_full + 8 * st, ph) && globaltimer() - t0 < 1000000ull) {}
+                    t0 = globaltimer();
+                    while (!mbar_try(v_full + 8 * st, ph) && globaltimer() - t0 < 1000000ull) {}
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(128, 128, false, false);
+            const uint32_t id_o = idesc_bf16(128, HD, false, true);
+            bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+            for (int j = 0; ok && j <= nblk; ++j) {
+                if (j < nblk) {
+                    const int st = j % STG, sb = j & 1;
+                    if (!mbar_wait(k_full + 8 * st, (j / STG) & 1, abort_flag, p.status)) break;
+                    if (!mbar_wait(s_empty + 8 * sb, ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < HD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16(tS + sb * 128, smem_desc(sQ + off, 16, 1024), smem_desc(sK + st * TILE + off, 16, 1024),
+                                 id_s, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(s_full + 8 * sb);
+                    mma_commit(k_empty + 8 * st);
+                }
+                if (j > 0) {
+                    const int jj = j - 1, st = jj % STG;
+                    if (!mbar_wait(p_full, jj & 1, abort_flag, p.status)) break;
+                    if (!mbar_wait(v_full + 8 * st, (jj / STG) & 1, abort_flag, p.status)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t offp = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16(tO, smem_desc(sP + offp, 16, 1024), smem_desc(sV + st * TILE + ks * 2048, 16384, 1024),
+                                 id_o, (jj > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(o_done);
+                    mma_commit(v_empty + 8 * st);
+                }
+            }
+        }
+    } else {
+        // ---------------- softmax warps: warp w reads TMEM lanes 32*(w%4)..
+        const int q = warp & 3;
+        const int r = q * 32 + lane;  // row of the tile
+        const int qpos = qb * 128 + r;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nblk; ++j) {
+            const int sb = j & 1;
+            if (!warp_wait(s_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+            float s[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + sb * 128 + c * 32, s + 32 * c);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_empty + 8 * sb);
+            float mx = -INFINITY;
+            if (j == qb) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    s[c] = (c <= r) ? s[c] * p.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, s[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    s[c] *= p.scale_log2;
+                    mx = fmaxf(mx, s[c]);
+                }
+            }
+            const bool rescale = mx > m + 8.f;
+            const float mu = rescale ? mx : m;
+            const float alpha = rescale ? ex2(m - mx) : 1.f;
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+                s[c] = ex2(s[c] - mu);
+                sum += s[c];
+            }
+            if (j > 0) {
+                if (!warp_wait(o_done, (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                    for (int c = 0; c < HD / 32; ++c) {
+                        float o[32];
+                        tmem_ld32(tO + lane_off + c * 32, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                        tmem_st32(tO + lane_off + c * 32, o);
+                    }
+                }
+            }
+            l = l * alpha + sum;
+            m = mu;
+            uint8_t* prow = smem + Lay::P + r * 128;
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) {
+                    const float* v = s + kb * 64 + c8 * 8;
+                    uint4 u = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                         pack_bf16(v[6], v[7]));
+                    *reinterpret_cast<uint4*>(prow + kb * 16384 + ((c8 ^ (r & 7)) << 4)) = u;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        if (ok && warp_wait(o_done, (nblk - 1) & 1, abort_flag, p.status)) {
+            tc_fence_after();
+            const float inv = 1.f / l;
+            const bool live = qpos < p.T;
+            bf16* orow = p.o + ((size_t)row0 + qpos) * (size_t)(p.H * HD) + h * HD;
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                float o[32];
+                tmem_ld32(tO + lane_off + c * 32, o);
+                if (live) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint4 u = make_uint4(pack_bf16(o[8 * i] * inv, o[8 * i + 1] * inv),
+                                             pack_bf16(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                             pack_bf16(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                             pack_bf16(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+                        *reinterpret_cast<uint4*>(orow + c * 32 + 8 * i) = u;
+                    }
+                }
+            }
+            if (live) p.lse[((size_t)row0 + qpos) * p.H + h] = (m + __log2f(l)) * kLn2;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+
+// ============================================================================ backward
+// dQ, one CTA per (query block of 128, head, batch row): for key blocks
+// j = 0..qb, S = Q K_j^T and dP = dO V_j^T into TMEM; per query row (one per
+// thread) P = 2^(S*scale*log2e - lse*log2e) with the causal mask, dS = P (dP - D)
+// as bf16 into shared memory; dQ += dS K_j with the K_j tile read again as an
+// MN-major operand.  dq = dQ / sqrt(hd).
+template <int HD>
+struct DqLayout {
+    static constexpr int KB = HD / 64;
+    static constexpr int TILE = KB * 16384;
+    static constexpr int Q = 0;
+    static constexpr int DO = Q + TILE;
+    static constexpr int K = DO + TILE;
+    static constexpr int V = K + STG * TILE;
+    static constexpr int DS = V + STG * TILE;
+    static constexpr int BAR = DS + 32768;
+    static constexpr int BYTES = BAR + 256 + 1024;
+};
+
+struct BwdParams {
+    int B, T, H, nkv, nqb;
+    float scale_log2, scale;
+    const float* lse;
+    const float* D;
+    bf16* dqkv;
+    int* status;
+};
+
+__device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
+    uint64_t t0 = globaltimer();
+    while (!mbar_try(bar, parity) && globaltimer() - t0 < 1000000ull) {}
+}
+
+template <int HD>
+__global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
+                                                           const __grid_constant__ CUtensorMap tmDO,
+                                                           const BwdParams p) {
+    using Lay = DqLayout<HD>;
+    constexpr int KB = Lay::KB, TILE = Lay::TILE;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t base = smem_u32(smem);
+    const uint32_t sQ = base + Lay::Q, sDO = base + Lay::DO, sK = base + Lay::K, sV = base + Lay::V;
+    const uint32_t sDS = base + Lay::DS;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
+    const uint32_t b0 = smem_u32(bars);
+    const uint32_t qd_full = b0, k_full = b0 + 8, k_empty = b0 + 24, v_full = b0 + 40, v_empty = b0 + 56;
+    const uint32_t s_full = b0 + 72, s_empty = b0 + 80, ds_full = b0 + 88, ds_done = b0 + 96;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qb = p.nqb - 1 - (int)blockIdx.x;
+    const int h = blockIdx.y, b = blockIdx.z, g = h / (p.H / p.nkv);
+    const int nblk = qb + 1;
+    const int row0 = b * p.T;
+    const int Nqkv = (p.H + 2 * p.nkv) * HD;
+
+    if (threadIdx.x == 0) {
+        mbar_init(qd_full, 1);
+        for (int s = 0; s < STG; ++s) {
+            mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1);
+            mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1);
+        }
+        mbar_init(s_full, 1); mbar_init(s_empty, 4); mbar_init(ds_full, 4); mbar_init(ds_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+    if (warp == 0 && lane == 0) { tma_prefetch(&tmQKV); tma_prefetch(&tmDO); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const int xq = h * HD, xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
+            mbar_expect_tx(qd_full, 2 * TILE);
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_2d(sQ + kb * 16384, &tmQKV, xq + kb * 64, row0 + qb * 128, qd_full);
+                tma_load_2d(sDO + kb * 16384, &tmDO, h * HD + kb * 64, row0 + qb * 128, qd_full);
+            }
+            int issued = 0;
+            for (int j = 0; j < nblk; ++j) {
+                const int st = j % STG;
+                const uint32_t ph = (j / STG) & 1;
+                if (!mbar_wait(k_empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
+                if (!mbar_wait(v_empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(k_full + 8 * st, TILE);
+                mbar_expect_tx(v_full + 8 * st, TILE);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_2d(sK + st * TILE + kb * 16384, &tmQKV, xk + kb * 64, row0 + j * 128, k_full + 8 * st);
+                    tma_load_2d(sV + st * TILE + kb * 16384, &tmQKV, xv + kb * 64, row0 + j * 128, v_full + 8 * st);
+                }
+                issued = j + 1;
+            }
+            if (*abort_flag) {
+                drain(qd_full, 0);
+                for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j) {
+                    drain(k_full + 8 * (j % STG), (j / STG) & 1);
+                    drain(v_full + 8 * (j % STG), (j / STG) & 1);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(128, 128, false, false);
+            const uint32_t id_q = idesc_bf16(128, HD, false, true);
+            if (mbar_wait(qd_full, 0, abort_flag, p.status)) {
+                for (int j = 0; j < nblk; ++j) {
+                    const int st = j % STG;
+                    const uint32_t ph = (j / STG) & 1;
+                    if (!mbar_wait(k_full + 8 * st, ph, abort_flag, p.status)) break;
+                    if (!mbar_wait(v_full + 8 * st, ph, abort_flag, p.status)) break;
+                    if (!mbar_wait(s_empty, (j & 1) ^ 1, abort_flag, p.status)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < HD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16(tS, smem_desc(sQ + off, 16, 1024), smem_desc(sK + st * TILE + off, 16, 1024), id_s,
+                                 ks > 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int ks = 0; ks < HD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16(tdP, smem_desc(sDO + off, 16, 1024), smem_desc(sV + st * TILE + off, 16, 1024), id_s,
+                                 ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(s_full);
+                    mma_commit(v_empty + 8 * st);
+                    if (!mbar_wait(ds_full, j & 1, abort_flag, p.status)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t offd = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16(tdQ, smem_desc(sDS + offd, 16, 1024), smem_desc(sK + st * TILE + ks * 2048, 16384, 1024),
+                                 id_q, (j > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(ds_done);
+                    mma_commit(k_empty + 8 * st);
+                }
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const int qpos = qb * 128 + r;
+        const bool live = qpos < p.T;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const float lse2 = live ? p.lse[((size_t)row0 + qpos) * p.H + h] * kLog2e : 0.f;
+        const float Dr = live ? p.D[((size_t)row0 + qpos) * p.H + h] : 0.f;
+        bool ok = true;
+        for (int j = 0; j < nblk && ok; ++j) {
+            if (!warp_wait(s_full, j & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+            if (j > 0 && !warp_wait(ds_done, (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            uint8_t* drow = smem + Lay::DS + r * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float sv[32], dp[32];
+                tmem_ld32(tS + lane_off + c * 32, sv);
+                tmem_ld32(tdP + lane_off + c * 32, dp);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool valid = live && (j < qb || c * 32 + i <= r);
+                    const float P = valid ? ex2(sv[i] * p.scale_log2 - lse2) : 0.f;
+                    sv[i] = P * (dp[i] - Dr);
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const int idx = (c & 1) * 4 + t;
+                    const float* v = sv + 8 * t;
+                    *reinterpret_cast<uint4*>(drow + (c >> 1) * 16384 + ((idx ^ (r & 7)) << 4)) =
+                        make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                   pack_bf16(v[6], v[7]));
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) { mbar_arrive(s_empty); mbar_arrive(ds_full); }
+        }
+        if (ok && warp_wait(ds_done, (nblk - 1) & 1, abort_flag, p.status)) {
+            tc_fence_after();
+            bf16* out = p.dqkv + ((size_t)row0 + qpos) * Nqkv + h * HD;
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                float o[32];
+                tmem_ld32(tdQ + lane_off + c * 32, o);
+                if (live) {
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        *reinterpret_cast<uint4*>(out + c * 32 + 8 * t) = make_uint4(
+                            pack_bf16(o[8 * t] * p.scale, o[8 * t + 1] * p.scale),
+                            pack_bf16(o[8 * t + 2] * p.scale, o[8 * t + 3] * p.scale),
+                            pack_bf16(o[8 * t + 4] * p.scale, o[8 * t + 5] * p.scale),
+                            pack_bf16(o[8 * t + 6] * p.scale, o[8 * t + 7] * p.scale));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// dK / dV, one CTA per (key block of 128, kv head, batch row): loops over the
+// units (query block of 64, query head of this kv group) that can see the
+// key block, in a fixed order (deterministic, no atomics).  Per unit, with
+// the key row as the MMA M dimension: S^T = K Q^T and dP^T = V dO^T into
+// double-buffered TMEM; per key row (one per thread) P^T with the causal
+// mask and dS^T = P^T (dP^T - D) as bf16 into shared memory; dV += P^T dO and
+// dK += dS^T Q accumulate in TMEM over all units.  dk = dK / sqrt(hd).
+template <int HD>
+struct DkvLayout {
+    static constexpr int KB = HD / 64;
+    static constexpr int TILE = KB * 16384;   // [128 x HD]
+    static constexpr int HTILE = KB * 8192;   // [64 x HD]
+    static constexpr int K = 0;
+    static constexpr int V = K + TILE;
+    static constexpr int Q = V + TILE;
+    static constexpr int DO = Q + STG * HTILE;
+    static constexpr int PT = DO + STG * HTILE;
+    static constexpr int DST = PT + 16384;
+    static constexpr int LSE = DST + 16384;   // [2][64] floats, log2 units
+    static constexpr int DD = LSE + 512;      // [2][64] floats
+    static constexpr int BAR = DD + 512;
+    static constexpr int BYTES = BAR + 256 + 1024;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmKV,
+                                                            const __grid_constant__ CUtensorMap tmQ64,
+                                                            const __grid_constant__ CUtensorMap tmDO64,
+                                                            const BwdParams p) {
+    using Lay = DkvLayout<HD>;
+    constexpr int KB = Lay::KB, TILE = Lay::TILE, HTILE = Lay::HTILE;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t base = smem_u32(smem);
+    const uint32_t sK = base + Lay::K, sV = base + Lay::V, sQ = base + Lay::Q, sDO = base + Lay::DO;
+    const uint32_t sPT = base + Lay::PT, sDST = base + Lay::DST;
+    float* lse_s = reinterpret_cast<float*>(smem + Lay::LSE);
+    float* d_s = reinterpret_cast<float*>(smem + Lay::DD);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
+    const uint32_t b0 = smem_u32(bars);
+    const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24, st_full = b0 + 40, st_empty = b0 + 56;
+    const uint32_t pd_full = b0 + 72, pd_done = b0 + 80, stage_ready = b0 + 88;  // stage_ready[2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int kvb = blockIdx.x;  // largest amount of work first
+    const int g = blockIdx.y, b = blockIdx.z;
+    const int Hg = p.H / p.nkv;
+    const int row0 = b * p.T;
+    const int Nqkv = (p.H + 2 * p.nkv) * HD;
+    const int nq64 = (p.T + 63) / 64;
+    const int i0 = 2 * kvb;
+    const int nunits = (nq64 - i0) * Hg;
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < STG; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
+        for (int s = 0; s < 2; ++s) { mbar_init(st_full + 8 * s, 1); mbar_init(st_empty + 8 * s, 4); }
+        mbar_init(pd_full, 4);
+        mbar_init(pd_done, 1);
+        mbar_init(stage_ready, 128);
+        mbar_init(stage_ready + 8, 128);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
+    if (warp == 0 && lane == 0) { tma_prefetch(&tmKV); tma_prefetch(&tmQ64); tma_prefetch(&tmDO64); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tSt = tmem, tdPt = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + HD;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const int xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
+            mbar_expect_tx(kv_full, 2 * TILE);
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_2d(sK + kb * 16384, &tmKV, xk + kb * 64, row0 + kvb * 128, kv_full);
+                tma_load_2d(sV + kb * 16384, &tmKV, xv + kb * 64, row0 + kvb * 128, kv_full);
+            }
+            int issued = 0;
+            for (int u = 0; u < nunits; ++u) {
+                const int st = u % STG;
+                const int i = i0 + u / Hg, h = g * Hg + u % Hg;
+                if (!mbar_wait(qo_empty + 8 * st, ((u / STG) & 1) ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(qo_full + 8 * st, 2 * HTILE);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_2d(sQ + st * HTILE + kb * 8192, &tmQ64, h * HD + kb * 64, row0 + i * 64, qo_full + 8 * st);
+                    tma_load_2d(sDO + st * HTILE + kb * 8192, &tmDO64, h * HD + kb * 64, row0 + i * 64,
+                                qo_full + 8 * st);
+                }
+                issued = u + 1;
+            }
+            if (*abort_flag) {
+                drain(kv_full, 0);
+                for (int u = (issued > STG ? issued - STG : 0); u < issued; ++u)
+                    drain(qo_full + 8 * (u % STG), (u / STG) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id_st = idesc_bf16(128, 64, false, false);
+            const uint32_t id_kv = idesc_bf16(128, HD, false, true);
+            if (mbar_wait(kv_full, 0, abort_flag, p.status)) {
+                for (int u = 0; u <= nunits; ++u) {
+                    if (u < nunits) {
+                        const int st = u % STG, sb = u & 1;
+                        if (!mbar_wait(qo_full + 8 * st, (u / STG) & 1, abort_flag, p.status)) break;
+                        if (!mbar_wait(st_empty + 8 * sb, ((u >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < HD / 16; ++ks) {
+                            const uint32_t ok_ = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            const uint32_t oq = (ks >> 2) * 8192 + (ks & 3) * 32;
+                            mma_bf16(tSt + sb * 64, smem_desc(sK + ok_, 16, 1024),
+                                     smem_desc(sQ + st * HTILE + oq, 16, 1024), id_st, ks > 0 ? 1u : 0u);
+                            mma_bf16(tdPt + sb * 64, smem_desc(sV + ok_, 16, 1024),
+                                     smem_desc(sDO + st * HTILE + oq, 16, 1024), id_st, ks > 0 ? 1u : 0u);
+                        }
+                        mma_commit(st_full + 8 * sb);
+                    }
+                    if (u > 0) {
+                        const int uu = u - 1, st = uu % STG;
+                        if (!mbar_wait(pd_full, uu & 1, abort_flag, p.status)) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            mma_bf16(tdV, smem_desc(sPT + ks * 32, 16, 1024),
+                                     smem_desc(sDO + st * HTILE + ks * 2048, 8192, 1024), id_kv,
+                                     (uu > 0 || ks > 0) ? 1u : 0u);
+                            mma_bf16(tdK, smem_desc(sDST + ks * 32, 16, 1024),
+                                     smem_desc(sQ + st * HTILE + ks * 2048, 8192, 1024), id_kv,
+                                     (uu > 0 || ks > 0) ? 1u : 0u);
+                        }
+                        mma_commit(pd_done);
+                        mma_commit(qo_empty + 8 * st);
+                    }
+                }
+            }
+        }
+    } else {
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const int t = threadIdx.x - 64;  // 0..127
+        const int kpos = kvb * 128 + r;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        bool ok = true;
+        for (int u = 0; u < nunits; ++u) {
+            const int sb = u & 1, buf = u & 1;
+            const int i = i0 + u / Hg, h = g * Hg + u % Hg;
+            {
+                const int qq = i * 64 + (t & 63);
+                const bool inr = qq < p.T;
+                const size_t idx = ((size_t)row0 + qq) * p.H + h;
+                if (t < 64) lse_s[buf * 64 + t] = inr ? p.lse[idx] * kLog2e : INFINITY;
+                else d_s[buf * 64 + (t - 64)] = inr ? p.D[idx] : 0.f;
+            }
+            mbar_arrive(stage_ready + 8 * buf);
+            if (!warp_wait(stage_ready + 8 * buf, (u >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            if (!warp_wait(st_full + 8 * sb, (u >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+            if (u > 0 && !warp_wait(pd_done, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            uint8_t* prow = smem + Lay::PT + r * 128;
+            uint8_t* drow = smem + Lay::DST + r * 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                float sv[32], dp[32];
+                tmem_ld32(tSt + lane_off + sb * 64 + c * 32, sv);
+                tmem_ld32(tdPt + lane_off + sb * 64 + c * 32, dp);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int qc = c * 32 + e;
+                    const bool valid = i * 64 + qc >= kpos;
+                    const float P = valid ? ex2(sv[e] * p.scale_log2 - lse_s[buf * 64 + qc]) : 0.f;
+                    dp[e] = P * (dp[e] - d_s[buf * 64 + qc]);
+                    sv[e] = P;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int idx = c * 4 + k;
+                    const uint32_t sw = (uint32_t)((idx ^ (r & 7)) << 4);
+                    const float* a = sv + 8 * k;
+                    const float* d = dp + 8 * k;
+                    *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]),
+                                                                      pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
+                    *reinterpret_cast<uint4*>(drow + sw) = make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]),
+                                                                      pack_bf16(d[4], d[5]), pack_bf16(d[6], d[7]));
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) { mbar_arrive(st_empty + 8 * sb); mbar_arrive(pd_full); }
+        }
+        if (ok && warp_wait(pd_done, (nunits - 1) & 1, abort_flag, p.status)) {
+            tc_fence_after();
+            const bool live = kpos < p.T;
+            bf16* out_k = p.dqkv + ((size_t)row0 + kpos) * Nqkv + (p.H + g) * HD;
+            bf16* out_v = p.dqkv + ((size_t)row0 + kpos) * Nqkv + (p.H + p.nkv + g) * HD;
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                float v[32], k[32];
+                tmem_ld32(tdV + lane_off + c * 32, v);
+                tmem_ld32(tdK + lane_off + c * 32, k);
+                if (live) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        *reinterpret_cast<uint4*>(out_v + c * 32 + 8 * e) =
+                            make_uint4(pack_bf16(v[8 * e], v[8 * e + 1]), pack_bf16(v[8 * e + 2], v[8 * e + 3]),
+                                       pack_bf16(v[8 * e + 4], v[8 * e + 5]), pack_bf16(v[8 * e + 6], v[8 * e + 7]));
+                        *reinterpret_cast<uint4*>(out_k + c * 32 + 8 * e) = make_uint4(
+                            pack_bf16(k[8 * e] * p.scale, k[8 * e + 1] * p.scale),
+                            pack_bf16(k[8 * e + 2] * p.scale, k[8 * e + 3] * p.scale),
+                            pack_bf16(k[8 * e + 4] * p.scale, k[8 * e + 5] * p.scale),
+                            pack_bf16(k[8 * e + 6] * p.scale, k[8 * e + 7] * p.scale));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// Tensor map over a row-major bf16 [rows, cols] array, box [box_rows, 64],
+// 128-byte swizzle, zero fill past the last row.
+bool map_rows(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+template <int HD>
+int fwd_launch(const CUtensorMap& map, const AttnParams& p, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(attn_fwd_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 FwdLayout<HD>::BYTES) != cudaSuccess)
+            return -1;
+        attr = true;
+    }
+    dim3 grid(p.nqb, p.H, p.B);
+    attn_fwd_tc_kernel<HD><<<grid, NT, FwdLayout<HD>::BYTES, s>>>(map, p);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+template <int HD>
+int bwd_launch(const CUtensorMap& kv, const CUtensorMap& q64, const CUtensorMap& do128, const CUtensorMap& do64,
+               const BwdParams& p, cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(attn_dq_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DqLayout<HD>::BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(attn_dkv_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DkvLayout<HD>::BYTES) != cudaSuccess)
+            return -1;
+        attr = true;
+    }
+    attn_dq_tc_kernel<HD><<<dim3(p.nqb, p.H, p.B), NT, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
+    attn_dkv_tc_kernel<HD><<<dim3(p.nqb, p.nkv, p.B), NT, DkvLayout<HD>::BYTES, s>>>(kv, q64, do64, p);
+    count_launch(2);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace
+
+int attention_tc_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, int nkv, int hd, void*, size_t,
+                     int* status, cudaStream_t s) {
+    if (hd != 64 && hd != 128) return 1;
+    if (!aligned16(qkv) || !aligned16(o) || B > 65535 || H > 65535) return 1;
+    const int Nqkv = (H + 2 * nkv) * hd;
+    CUtensorMap map;
+    if (!map_rows(&map, qkv, Nqkv, (uint64_t)B * T, 128)) return 1;
+    AttnParams p;
+    p.B = B; p.T = T; p.H = H; p.nkv = nkv; p.nqb = (T + 127) / 128;
+    p.scale_log2 = kLog2e / sqrtf((float)hd);
+    p.o = reinterpret_cast<bf16*>(o);
+    p.lse = lse;
+    p.status = status;
+    return hd == 128 ? fwd_launch<128>(map, p, s) : fwd_launch<64>(map, p, s);
+}
+
+int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
+                     int B, int T, int H, int nkv, int hd, void*, size_t, int* status, cudaStream_t s) {
+    if (hd != 64 && hd != 128) return 1;
+    if (!aligned16(qkv) || !aligned16(o) || !aligned16(dO) || !aligned16(dqkv) || B > 65535 || H > 65535) return 1;
+    const int Nqkv = (H + 2 * nkv) * hd;
+    CUtensorMap kv, q64, do128, do64;
+    if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&q64, qkv, Nqkv, (uint64_t)B * T, 64) ||
+        !map_rows(&do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128) ||
+        !map_rows(&do64, dO, (uint64_t)H * hd, (uint64_t)B * T, 64))
+        return 1;
+    if (launch_attention_bwd_dot(DT_BF16, o, dO, Dbuf, B * T * H, hd, s) != cudaSuccess) return -1;
+    BwdParams p;
+    p.B = B; p.T = T; p.H = H; p.nkv = nkv; p.nqb = (T + 127) / 128;
+    p.scale = 1.f / sqrtf((float)hd);
+    p.scale_log2 = kLog2e * p.scale;
+    p.lse = lse; p.D = Dbuf;
+    p.dqkv = reinterpret_cast<bf16*>(dqkv);
+    p.status = status;
+    return hd == 128 ? bwd_launch<128>(kv, q64, do128, do64, p, s) : bwd_launch<64>(kv, q64, do128, do64, p, s);
+}
+
 size_t attention_tc_workspace_bytes(int, int, int, int, int) { return 0; }
+
 }  // namespace nc

@@ -6,8 +6,8 @@ namespace nc {
 // Return 0 when done, > 0 when the shape is not taken (caller falls back),
 // < 0 on a CUDA error.
 int attention_tc_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, int nkv, int hd, void* ws,
-                     size_t ws_bytes, cudaStream_t s);
+                     size_t ws_bytes, int* status, cudaStream_t s);
 int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
-                     int B, int T, int H, int nkv, int hd, void* ws, size_t ws_bytes, cudaStream_t s);
+                     int B, int T, int H, int nkv, int hd, void* ws, size_t ws_bytes, int* status, cudaStream_t s);
 size_t attention_tc_workspace_bytes(int B, int T, int H, int nkv, int hd);
 }  // namespace nc

@@ -236,7 +236,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
             int tm, tn, ks;
             decode(p, u, tm, tn, ks);
-            if (!mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, p.status)) break;
+            if (!warp_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, p.status)) break;
             tc_fence_after();
             const int row = tm * BM + q * 32 + lane;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;

@@ -101,6 +101,10 @@ cudaError_t launch_attention_bwd_simt(DType at, const void* qkv, const void* o, 
                                       const float* lse, float* Dbuf, void* dqkv, int B, int T, int H,
                                       int nkv, int hd, cudaStream_t s);
 
+// D[row, h] = sum_c dO[row, h, c] * o[row, h, c] (softmax backward row term).
+cudaError_t launch_attention_bwd_dot(DType at, const void* o, const void* dO, float* D, int MH, int hd,
+                                     cudaStream_t s);
+
 // ---------------------------------------------------------------- bounded wait
 cudaError_t launch_expired_wait(int* status, int max_iters, cudaStream_t s);
 

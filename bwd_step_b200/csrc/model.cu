@@ -197,7 +197,7 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
     Prof pr(c, P_ATTN_FWD, attn_flops(c), 0.0);
     if (m->tc) {
         int r = attention_tc_fwd(qkv, o, lse, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.ws + c.p.attn_ws,
-                                 c.p.attn_ws_bytes, c.s);
+                                 c.p.attn_ws_bytes, m->status, c.s);
         if (r == 0) return NC_OK;
         if (r < 0) return NC_ERR_CUDA;
     }
@@ -211,7 +211,7 @@ int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, 
     float* Dbuf = c.at<float>(c.p.Dbuf);
     if (m->tc) {
         int r = attention_tc_bwd(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd,
-                                 c.ws + c.p.attn_ws, c.p.attn_ws_bytes, c.s);
+                                 c.ws + c.p.attn_ws, c.p.attn_ws_bytes, m->status, c.s);
         if (r == 0) return NC_OK;
         if (r < 0) return NC_ERR_CUDA;
     }
@@ -576,4 +576,28 @@ extern "C" int nc_test_gemm(int M, int N, int K, int in_bf16, const void* A, int
         return r == 0 ? NC_OK : NC_ERR_CUDA;
     }
     return gemm_simt(g, s) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+extern "C" int nc_test_attention(int B, int T, int H, int nkv, int hd, const void* qkv, void* o, float* lse,
+                                 const void* dO, void* dqkv, float* Dbuf, int use_tc, int* status, void* stream) {
+    if (B <= 0 || T <= 0 || H <= 0 || nkv <= 0 || H % nkv || !qkv || !o || !lse) return NC_ERR_INVALID_ARG;
+    if (hd != 16 && hd != 32 && hd != 64 && hd != 128) return NC_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (use_tc) {
+        int r = attention_tc_fwd(qkv, o, lse, B, T, H, nkv, hd, nullptr, 0, status, s);
+        if (r != 0) return r > 0 ? NC_ERR_UNSUPPORTED_SHAPE : NC_ERR_CUDA;
+        if (dO) {
+            if (!dqkv || !Dbuf) return NC_ERR_INVALID_ARG;
+            r = attention_tc_bwd(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, nullptr, 0, status, s);
+            if (r != 0) return r > 0 ? NC_ERR_UNSUPPORTED_SHAPE : NC_ERR_CUDA;
+        }
+        return NC_OK;
+    }
+    if (launch_attention_fwd_simt(DT_BF16, qkv, o, lse, B, T, H, nkv, hd, s) != cudaSuccess) return NC_ERR_CUDA;
+    if (dO) {
+        if (!dqkv || !Dbuf) return NC_ERR_INVALID_ARG;
+        if (launch_attention_bwd_simt(DT_BF16, qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, s) != cudaSuccess)
+            return NC_ERR_CUDA;
+    }
+    return NC_OK;
 }

@@ -1,0 +1,68 @@
+"""Unit tests of the causal multi-query attention kernels (tcgen05 and
+plain-FMA) through the testing ABI, against the oracle's attention forward and
+backward in float64 on the same bf16 inputs."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from bwd_step_b200 import lib  # noqa: E402
+
+P = ctypes.c_void_p
+
+
+def _bf16(x):
+    return torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+
+
+def _run(B, T, H, nkv, hd, use_tc, seed=0, scale=1.0):
+    rng = np.random.default_rng(seed)
+    Nqkv = (H + 2 * nkv) * hd
+    qkv = _bf16(rng.standard_normal((B * T, Nqkv)) * scale)
+    dO = _bf16(rng.standard_normal((B * T, H * hd)))
+    qkv_d, dO_d = qkv.cuda(), dO.cuda()
+    o = torch.full((B * T, H * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B * T, H), float("nan"), dtype=torch.float32, device="cuda")
+    dqkv = torch.full((B * T, Nqkv), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Dbuf = torch.empty((B * T, H), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    r = lib().nc_test_attention(B, T, H, nkv, hd, P(qkv_d.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
+                                P(dO_d.data_ptr()), P(dqkv.data_ptr()), P(Dbuf.data_ptr()), use_tc,
+                                P(status.data_ptr()), P(torch.cuda.current_stream().cuda_stream))
+    assert r == 0, r
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    q64 = qkv.double().numpy().reshape(B, T, H + 2 * nkv, hd)
+    do64 = dO.double().numpy().reshape(B, T, H, hd)
+    got_o = o.double().cpu().numpy().reshape(B, T, H, hd)
+    got_d = dqkv.double().cpu().numpy().reshape(B, T, H + 2 * nkv, hd)
+    for b in range(B):
+        q, k, v = q64[b, :, :H], q64[b, :, H:H + nkv], q64[b, :, H + nkv:]
+        ref_o = oracle.attention(q, k, v)
+        dq, dk, dv = oracle.attention_backward(q, k, v, do64[b])
+        for name, got, ref in (("o", got_o[b], ref_o), ("dq", got_d[b, :, :H], dq),
+                               ("dk", got_d[b, :, H:H + nkv], dk), ("dv", got_d[b, :, H + nkv:], dv)):
+            err = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+            assert err <= 1.5e-2, (name, b, err)
+
+
+@pytest.mark.parametrize("hd", [64, 128])
+@pytest.mark.parametrize("B,T,H,nkv", [(1, 128, 1, 1), (2, 300, 4, 1), (1, 513, 3, 1), (2, 256, 4, 2),
+                                       (1, 1024, 2, 1), (3, 64, 2, 1)])
+def test_tcgen05_attention(B, T, H, nkv, hd):
+    _run(B, T, H, nkv, hd, 1, seed=T + H)
+
+
+def test_tcgen05_attention_sharp_softmax():
+    # large scores: exercises the running-max rescale of the output
+    _run(1, 640, 2, 1, 128, 1, seed=3, scale=4.0)
+
+
+@pytest.mark.parametrize("hd", [16, 64])
+def test_fma_attention(hd):
+    _run(2, 150, 4, 1, hd, 0, seed=5)
