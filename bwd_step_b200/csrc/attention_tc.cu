@@ -764,21 +764,44 @@ int fwd_launch(const CUtensorMap& map, const AttnParams& p, cudaStream_t s) {
 }
 
 template <int HD>
-int bwd_launch(const CUtensorMap& kv, const CUtensorMap& q64, const CUtensorMap& do128, const CUtensorMap& do64,
-               const BwdParams& p, cudaStream_t s) {
+int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(attn_dq_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 DqLayout<HD>::BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(attn_dkv_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 DkvLayout<HD>::BYTES) != cudaSuccess)
+                                 DqLayout<HD>::BYTES) != cudaSuccess)
             return -1;
         attr = true;
     }
     attn_dq_tc_kernel<HD><<<dim3(p.nqb, p.H, p.B), NT, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
-    attn_dkv_tc_kernel<HD><<<dim3(p.nqb, p.nkv, p.B), NT, DkvLayout<HD>::BYTES, s>>>(kv, q64, do64, p);
-    count_launch(2);
+    count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+template <int HD>
+int dkv_launch(const CUtensorMap& kv, const CUtensorMap& q64, const CUtensorMap& do64, const BwdParams& p,
+               cudaStream_t s) {
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(attn_dkv_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DkvLayout<HD>::BYTES) != cudaSuccess)
+            return -1;
+        attr = true;
+    }
+    attn_dkv_tc_kernel<HD><<<dim3(p.nqb, p.nkv, p.B), NT, DkvLayout<HD>::BYTES, s>>>(kv, q64, do64, p);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+BwdParams bwd_params(const float* lse, const float* Dbuf, void* dqkv, int B, int T, int H, int nkv, int hd,
+                     int* status) {
+    BwdParams p;
+    p.B = B; p.T = T; p.H = H; p.nkv = nkv; p.nqb = (T + 127) / 128;
+    p.scale = 1.f / sqrtf((float)hd);
+    p.scale_log2 = kLog2e * p.scale;
+    p.lse = lse; p.D = Dbuf;
+    p.dqkv = reinterpret_cast<bf16*>(dqkv);
+    p.status = status;
+    return p;
 }
 
 }  // namespace
@@ -799,25 +822,39 @@ int attention_tc_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, 
     return hd == 128 ? fwd_launch<128>(map, p, s) : fwd_launch<64>(map, p, s);
 }
 
-int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
-                     int B, int T, int H, int nkv, int hd, void*, size_t, int* status, cudaStream_t s) {
-    if (hd != 64 && hd != 128) return 1;
+bool attention_tc_bwd_supported(int hd) { return hd == 64 || hd == 128; }
+
+int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
+                        int B, int T, int H, int nkv, int hd, int* status, cudaStream_t s) {
+    if (!attention_tc_bwd_supported(hd)) return 1;
     if (!aligned16(qkv) || !aligned16(o) || !aligned16(dO) || !aligned16(dqkv) || B > 65535 || H > 65535) return 1;
     const int Nqkv = (H + 2 * nkv) * hd;
-    CUtensorMap kv, q64, do128, do64;
-    if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&q64, qkv, Nqkv, (uint64_t)B * T, 64) ||
-        !map_rows(&do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128) ||
-        !map_rows(&do64, dO, (uint64_t)H * hd, (uint64_t)B * T, 64))
+    CUtensorMap kv, do128;
+    if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128))
         return 1;
     if (launch_attention_bwd_dot(DT_BF16, o, dO, Dbuf, B * T * H, hd, s) != cudaSuccess) return -1;
-    BwdParams p;
-    p.B = B; p.T = T; p.H = H; p.nkv = nkv; p.nqb = (T + 127) / 128;
-    p.scale = 1.f / sqrtf((float)hd);
-    p.scale_log2 = kLog2e * p.scale;
-    p.lse = lse; p.D = Dbuf;
-    p.dqkv = reinterpret_cast<bf16*>(dqkv);
-    p.status = status;
-    return hd == 128 ? bwd_launch<128>(kv, q64, do128, do64, p, s) : bwd_launch<64>(kv, q64, do128, do64, p, s);
+    BwdParams p = bwd_params(lse, Dbuf, dqkv, B, T, H, nkv, hd, status);
+    return hd == 128 ? dq_launch<128>(kv, do128, p, s) : dq_launch<64>(kv, do128, p, s);
+}
+
+int attention_tc_bwd_dkv(const void* qkv, const void* dO, const float* lse, const float* Dbuf, void* dqkv, int B,
+                         int T, int H, int nkv, int hd, int* status, cudaStream_t s) {
+    if (!attention_tc_bwd_supported(hd)) return 1;
+    if (!aligned16(qkv) || !aligned16(dO) || !aligned16(dqkv) || B > 65535 || nkv > 65535) return 1;
+    const int Nqkv = (H + 2 * nkv) * hd;
+    CUtensorMap kv, q64, do64;
+    if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&q64, qkv, Nqkv, (uint64_t)B * T, 64) ||
+        !map_rows(&do64, dO, (uint64_t)H * hd, (uint64_t)B * T, 64))
+        return 1;
+    BwdParams p = bwd_params(lse, Dbuf, dqkv, B, T, H, nkv, hd, status);
+    return hd == 128 ? dkv_launch<128>(kv, q64, do64, p, s) : dkv_launch<64>(kv, q64, do64, p, s);
+}
+
+int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
+                     int B, int T, int H, int nkv, int hd, void*, size_t, int* status, cudaStream_t s) {
+    int r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s);
+    if (r != 0) return r;
+    return attention_tc_bwd_dkv(qkv, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s);
 }
 
 size_t attention_tc_workspace_bytes(int, int, int, int, int) { return 0; }

@@ -45,16 +45,21 @@ cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R
 cudaError_t launch_loss_reduce(const float* loss_rows, int M, float* loss, cudaStream_t s);
 
 struct EmbedScratch {
-    int* count;    // [V]
-    int* offset;   // [V+1]
-    int* cursor;   // [V]
-    int* perm;     // [M]
-    int* perm2;    // [M]
-    int* active;   // [V]
-    int* n_active; // [1]
+    int* count;        // [V] positions per id
+    int* offset;       // [V+1] first slot of each id
+    int* cursor;       // [V]
+    int* perm;         // [M] positions bucketed by id
+    int* perm2;        // [M] same, increasing position within a bucket
+    int* active;       // [V] ids that occur
+    int* n_active;     // [1]
+    int* piece_base;   // [V] first piece of each id
+    int* part_base;    // [V] first partial-sum slot of each multi-piece id
+    int* piece_bucket; // [pieces] id of each piece
+    int* totals;       // [2] pieces, partial slots
+    float* partial;    // [partial slots, d] piece sums of multi-piece ids
 };
-size_t embed_scratch_bytes(int M, int V);
-EmbedScratch embed_scratch_carve(void* base, int M, int V);
+size_t embed_scratch_bytes(int M, int V, int d);
+EmbedScratch embed_scratch_carve(void* base, int M, int V, int d);
 // dwte[v] = sum over positions m with idx[m] == v of de[m], in increasing m;
 // rows of unused ids are zero.  Deterministic.
 cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int V, int d, float* dwte,

@@ -321,6 +321,14 @@ __global__ void loss_reduce_kernel(const float* __restrict__ rows, int M, float*
 }
 
 // ---------------------------------------------------------------- embedding scatter
+// dWte[v] = sum of de[m] over the positions m with idx[m] == v, in increasing m.
+// Positions are bucketed by id (counting sort, then a canonical in-bucket
+// order), each bucket's slot range is cut into pieces of kPiece slots, every
+// piece is summed by its own CTA (hot ids under a Zipf law span many pieces),
+// and buckets with several pieces add their piece sums in piece order.  All
+// orders are fixed, so the result is bitwise reproducible.
+constexpr int kPiece = 64;
+
 __global__ void emb_hist_kernel(const int32_t* __restrict__ idx, int M, int V, int* count) {
     int m = blockIdx.x * blockDim.x + threadIdx.x;
     if (m >= M) return;
@@ -328,32 +336,45 @@ __global__ void emb_hist_kernel(const int32_t* __restrict__ idx, int M, int V, i
     if (id >= 0 && id < V) atomicAdd(&count[id], 1);
 }
 
-// Single block of 1024 threads: exclusive scan of count[V] into offset[V+1]
-// and compaction of the ids with count > 0 into active[].
-__global__ void emb_scan_kernel(const int* __restrict__ count, int V, int* offset, int* active,
-                                int* n_active) {
-    __shared__ int sc[1024], sf[1024];
+// Single block of 1024 threads: exclusive scans over the V buckets of
+// (count, used?, pieces, partial pieces) and the list of used ids.
+__global__ void emb_scan_kernel(const int* __restrict__ count, int V, int* offset, int* active, int* n_active,
+                                int* piece_base, int* part_base, int* totals) {
+    __shared__ int sc[1024], sf[1024], sp[1024], sq[1024];
     int t = threadIdx.x;
     int per = (V + 1023) / 1024;
     int lo = min(V, t * per), hi = min(V, lo + per);
-    int c = 0, f = 0;
-    for (int i = lo; i < hi; ++i) { int k = count[i]; c += k; f += k > 0; }
-    sc[t] = c; sf[t] = f;
+    int c = 0, f = 0, pc = 0, pq = 0;
+    for (int i = lo; i < hi; ++i) {
+        int k = count[i];
+        int np = (k + kPiece - 1) / kPiece;
+        c += k; f += k > 0; pc += np; pq += np > 1 ? np : 0;
+    }
+    sc[t] = c; sf[t] = f; sp[t] = pc; sq[t] = pq;
     __syncthreads();
     for (int o = 1; o < 1024; o <<= 1) {
         int a = t >= o ? sc[t - o] : 0, b = t >= o ? sf[t - o] : 0;
+        int e = t >= o ? sp[t - o] : 0, g = t >= o ? sq[t - o] : 0;
         __syncthreads();
-        sc[t] += a; sf[t] += b;
+        sc[t] += a; sf[t] += b; sp[t] += e; sq[t] += g;
         __syncthreads();
     }
-    int base_c = sc[t] - c, base_f = sf[t] - f;
+    int bc = sc[t] - c, bf = sf[t] - f, bp = sp[t] - pc, bq = sq[t] - pq;
     for (int i = lo; i < hi; ++i) {
         int k = count[i];
-        offset[i] = base_c;
-        if (k > 0) active[base_f++] = i;
-        base_c += k;
+        int np = (k + kPiece - 1) / kPiece;
+        offset[i] = bc;
+        piece_base[i] = bp;
+        part_base[i] = bq;
+        if (k > 0) active[bf++] = i;
+        bc += k; bp += np; bq += np > 1 ? np : 0;
     }
-    if (t == 1023) { offset[V] = sc[1023]; *n_active = sf[1023]; }
+    if (t == 1023) {
+        offset[V] = sc[1023];
+        *n_active = sf[1023];
+        totals[0] = sp[1023];  // pieces
+        totals[1] = sq[1023];  // partial slots
+    }
 }
 
 __global__ void emb_fill_kernel(const int32_t* __restrict__ idx, int M, int V, const int* __restrict__ offset,
@@ -378,21 +399,77 @@ __global__ void emb_canon_kernel(const int32_t* __restrict__ idx, int V, const i
     perm2[lo + rank] = p;
 }
 
-__global__ void emb_segsum_kernel(const float* __restrict__ de, int d, const int* __restrict__ offset,
-                                  const int* __restrict__ perm2, const int* __restrict__ active,
-                                  const int* __restrict__ n_active, float* __restrict__ dwte) {
+// piece -> bucket map, one thread per used bucket.
+__global__ void emb_pieces_kernel(const int* __restrict__ count, const int* __restrict__ active,
+                                  const int* __restrict__ n_active, const int* __restrict__ piece_base,
+                                  int* piece_bucket) {
+    int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= *n_active) return;
+    int v = active[k];
+    int np = (count[v] + kPiece - 1) / kPiece;
+    for (int j = 0; j < np; ++j) piece_bucket[piece_base[v] + j] = v;
+}
+
+// One CTA per piece: sums its <= kPiece rows of de in slot order.
+__global__ void emb_piece_sum_kernel(const float* __restrict__ de, int d, const int* __restrict__ count,
+                                     const int* __restrict__ offset, const int* __restrict__ perm2,
+                                     const int* __restrict__ piece_base, const int* __restrict__ part_base,
+                                     const int* __restrict__ piece_bucket, const int* __restrict__ totals,
+                                     float* __restrict__ dwte, float* __restrict__ partial) {
+    __shared__ int rows[kPiece];
+    int pc = blockIdx.x;
+    if (pc >= totals[0]) return;
+    int v = piece_bucket[pc];
+    int k = pc - piece_base[v];
+    int lo = offset[v] + k * kPiece, hi = min(offset[v + 1], lo + kPiece);
+    int n = hi - lo;
+    if ((int)threadIdx.x < n) rows[threadIdx.x] = perm2[lo + threadIdx.x];
+    __syncthreads();
+    int np = (count[v] + kPiece - 1) / kPiece;
+    float* dst = np == 1 ? dwte + (size_t)v * d : partial + (size_t)(part_base[v] + k) * d;
+    for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+        int s = 0;
+        for (; s + 1 < n; s += 2) {
+            float4 g0 = *reinterpret_cast<const float4*>(de + (size_t)rows[s] * d + c);
+            float4 g1 = *reinterpret_cast<const float4*>(de + (size_t)rows[s + 1] * d + c);
+            a0.x += g0.x; a0.y += g0.y; a0.z += g0.z; a0.w += g0.w;
+            a1.x += g1.x; a1.y += g1.y; a1.z += g1.z; a1.w += g1.w;
+        }
+        a0.x += a1.x; a0.y += a1.y; a0.z += a1.z; a0.w += a1.w;
+        if (s < n) {
+            float4 g = *reinterpret_cast<const float4*>(de + (size_t)rows[s] * d + c);
+            a0.x += g.x; a0.y += g.y; a0.z += g.z; a0.w += g.w;
+        }
+        *reinterpret_cast<float4*>(dst + c) = a0;
+    }
+}
+
+// Buckets with several pieces: add the piece sums in piece order.
+__global__ void emb_combine_kernel(int d, const int* __restrict__ count, const int* __restrict__ active,
+                                   const int* __restrict__ n_active, const int* __restrict__ part_base,
+                                   const float* __restrict__ partial, float* __restrict__ dwte) {
     int k = blockIdx.x;
     if (k >= *n_active) return;
     int v = active[k];
-    int lo = offset[v], hi = offset[v + 1];
+    int np = (count[v] + kPiece - 1) / kPiece;
+    if (np < 2) return;
+    const float* src = partial + (size_t)part_base[v] * d;
     for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = lo; s < hi; ++s) {
-            float4 g = *reinterpret_cast<const float4*>(de + (size_t)perm2[s] * d + c);
+        float4 acc = *reinterpret_cast<const float4*>(src + c);
+        for (int j = 1; j < np; ++j) {
+            float4 g = *reinterpret_cast<const float4*>(src + (size_t)j * d + c);
             acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
         }
         *reinterpret_cast<float4*>(dwte + (size_t)v * d + c) = acc;
     }
+}
+
+// Rows of ids that never occur get exact zeros (every dWte row is written once).
+__global__ void emb_zero_unused_kernel(const int* __restrict__ count, int V, int d4, float* __restrict__ dwte) {
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (size_t)V * d4) return;
+    if (count[i / d4] == 0) reinterpret_cast<float4*>(dwte)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, size_t n4,
@@ -536,20 +613,31 @@ cudaError_t launch_loss_reduce(const float* rows, int M, float* loss, cudaStream
 
 static inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t embed_scratch_bytes(int M, int V) {
-    return al256(4ull * V) * 2 + al256(4ull * (V + 1)) + al256(4ull * M) * 2 + al256(4ull * V) + 256;
+static inline int emb_max_pieces(int M, int V) { return M / kPiece + (M < V ? M : V) + 1; }
+static inline int emb_max_partials(int M) { return 2 * (M / kPiece) + 2; }
+
+size_t embed_scratch_bytes(int M, int V, int d) {
+    return al256(4ull * V) * 2 + al256(4ull * (V + 1)) + al256(4ull * M) * 2 + al256(4ull * V) + 256 +
+           al256(4ull * V) * 2 + al256(4ull * emb_max_pieces(M, V)) + 256 +
+           al256(4ull * emb_max_partials(M) * d);
 }
 
-EmbedScratch embed_scratch_carve(void* base, int M, int V) {
+EmbedScratch embed_scratch_carve(void* base, int M, int V, int d) {
     char* p = (char*)base;
     EmbedScratch s;
-    s.count = (int*)p;   p += al256(4ull * V);
-    s.cursor = (int*)p;  p += al256(4ull * V);   // count and cursor adjacent: one memset
-    s.offset = (int*)p;  p += al256(4ull * (V + 1));
-    s.perm = (int*)p;    p += al256(4ull * M);
-    s.perm2 = (int*)p;   p += al256(4ull * M);
-    s.active = (int*)p;  p += al256(4ull * V);
-    s.n_active = (int*)p;
+    s.count = (int*)p;        p += al256(4ull * V);
+    s.cursor = (int*)p;       p += al256(4ull * V);   // count and cursor adjacent: one memset
+    s.offset = (int*)p;       p += al256(4ull * (V + 1));
+    s.perm = (int*)p;         p += al256(4ull * M);
+    s.perm2 = (int*)p;        p += al256(4ull * M);
+    s.active = (int*)p;       p += al256(4ull * V);
+    s.n_active = (int*)p;     p += 256;
+    s.piece_base = (int*)p;   p += al256(4ull * V);
+    s.part_base = (int*)p;    p += al256(4ull * V);
+    s.piece_bucket = (int*)p; p += al256(4ull * emb_max_pieces(M, V));
+    s.totals = (int*)p;       p += 256;
+    s.partial = (float*)p;
+    (void)d;
     return s;
 }
 
@@ -557,16 +645,22 @@ cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int
                                  EmbedScratch sc, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(sc.count, 0, 2 * al256(4ull * V), s);  // count + cursor
     if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(dwte, 0, sizeof(float) * (size_t)V * d, s);
-    if (e != cudaSuccess) return e;
     int mb = (M + 255) / 256;
     emb_hist_kernel<<<mb, 256, 0, s>>>(idx, M, V, sc.count);
-    emb_scan_kernel<<<1, 1024, 0, s>>>(sc.count, V, sc.offset, sc.active, sc.n_active);
+    emb_scan_kernel<<<1, 1024, 0, s>>>(sc.count, V, sc.offset, sc.active, sc.n_active, sc.piece_base, sc.part_base,
+                                       sc.totals);
     emb_fill_kernel<<<mb, 256, 0, s>>>(idx, M, V, sc.offset, sc.cursor, sc.perm);
     emb_canon_kernel<<<mb, 256, 0, s>>>(idx, V, sc.offset, sc.perm, sc.perm2);
-    int nb = M < V ? M : V;
-    emb_segsum_kernel<<<nb, 128, 0, s>>>(de, d, sc.offset, sc.perm2, sc.active, sc.n_active, dwte);
-    count_launch(5);
+    int na = M < V ? M : V;
+    emb_pieces_kernel<<<(na + 255) / 256, 256, 0, s>>>(sc.count, sc.active, sc.n_active, sc.piece_base,
+                                                      sc.piece_bucket);
+    emb_piece_sum_kernel<<<emb_max_pieces(M, V), 128, 0, s>>>(de, d, sc.count, sc.offset, sc.perm2, sc.piece_base,
+                                                             sc.part_base, sc.piece_bucket, sc.totals, dwte,
+                                                             sc.partial);
+    emb_combine_kernel<<<na, 128, 0, s>>>(d, sc.count, sc.active, sc.n_active, sc.part_base, sc.partial, dwte);
+    size_t n4 = (size_t)V * (d / 4);
+    emb_zero_unused_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(sc.count, V, d / 4, dwte);
+    count_launch(9);
     return cudaGetLastError();
 }
 

@@ -112,7 +112,7 @@ Plan make_plan(const nc_model* m, int B, int T) {
     p.zc = take(4ull * p.R * m->V);
     p.dlc = take(A * (size_t)p.R * m->V);
     p.loss_rows = take(4 * M);
-    p.emb = take(embed_scratch_bytes(p.M, m->V));
+    p.emb = take(embed_scratch_bytes(p.M, m->V, m->d));
     size_t max_out = std::max({(size_t)p.R * d, (size_t)m->F * d, (size_t)m->H * m->hd * d, (size_t)m->Nqkv * d});
     p.splitk_bytes = m->tc ? gemm_tc_splitk_bytes(max_out) : 0;
     p.splitk = take(p.splitk_bytes);
@@ -132,11 +132,15 @@ struct Ctx {
 };
 
 enum ProfCls {
-    P_GEMM_TC = 0, P_GEMM_FMA, P_ATTN_FWD, P_ATTN_BWD, P_NORM_FWD, P_NORM_BWD, P_QKROPE_FWD, P_QKROPE_BWD,
+    P_GEMM_FWD = 0, P_GEMM_DGRAD, P_GEMM_WGRAD, P_GEMM_LM_Z, P_GEMM_LM_DX, P_GEMM_LM_DW, P_GEMM_FMA,
+    P_ATTN_FWD, P_ATTN_BWD, P_ATTN_BWD_DQ, P_ATTN_BWD_DKV, P_NORM_FWD, P_NORM_BWD, P_QKROPE_FWD, P_QKROPE_BWD,
     P_EMBED_FWD, P_EMBED_BWD, P_CE, P_OTHER, P_COUNT
 };
+// tcgen05 GEMM launches are tagged by role: forward y = x W^T, input
+// gradient dX = dY W, weight gradient dW = dY^T X, and the three LM-head products.
 const char* const kProfNames[P_COUNT] = {
-    "gemm_tcgen05", "gemm_fma", "attention_fwd", "attention_bwd", "rmsnorm_fwd", "rmsnorm_bwd",
+    "gemm_fwd", "gemm_dgrad", "gemm_wgrad", "gemm_lmhead_z", "gemm_lmhead_dx", "gemm_lmhead_dw", "gemm_fma",
+    "attention_fwd", "attention_bwd", "attention_bwd_dq", "attention_bwd_dkv", "rmsnorm_fwd", "rmsnorm_bwd",
     "qknorm_rope_fwd", "qknorm_rope_bwd", "embed_fwd", "embed_bwd", "cross_entropy", "other"};
 
 // Records a CUDA event pair around the launches made in its lifetime (only
@@ -156,11 +160,11 @@ struct Prof {
 };
 
 // C = A B^T with the tensor-core kernel where it applies, else the FMA kernel.
-int run_gemm(const Ctx& c, const GemmDesc& g) {
+int run_gemm(const Ctx& c, const GemmDesc& g, int role) {
     const double es = g.in_t == DT_BF16 ? 2.0 : 4.0;
-    Prof pr(c, P_GEMM_TC, 2.0 * g.M * g.N * (double)g.K,
+    Prof pr(c, role, 2.0 * g.M * g.N * (double)g.K,
             es * ((double)g.M * g.K + (double)g.N * g.K) + (g.c_t == DT_BF16 ? 2.0 : 4.0) * g.M * (double)g.N);
-    pr.cls = (c.m->tc && g.in_t == DT_BF16) ? P_GEMM_TC : P_GEMM_FMA;
+    pr.cls = (c.m->tc && g.in_t == DT_BF16) ? role : P_GEMM_FMA;
     if (c.m->tc && g.in_t == DT_BF16) {
         int r = gemm_tc(g, c.ws + c.p.splitk, c.p.splitk_bytes, c.s);
         if (r == 0) return NC_OK;
@@ -207,14 +211,21 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
 
 int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv) {
     const nc_model* m = c.m;
-    Prof pr(c, P_ATTN_BWD, 2.0 * attn_flops(c), 0.0);
     float* Dbuf = c.at<float>(c.p.Dbuf);
-    if (m->tc) {
-        int r = attention_tc_bwd(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd,
-                                 c.ws + c.p.attn_ws, c.p.attn_ws_bytes, m->status, c.s);
+    if (m->tc && attention_tc_bwd_supported(m->hd)) {
+        int r;
+        {
+            Prof pr(c, P_ATTN_BWD_DQ, attn_flops(c), 0.0);
+            r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s);
+        }
+        if (r == 0) {
+            Prof pr(c, P_ATTN_BWD_DKV, attn_flops(c), 0.0);
+            r = attention_tc_bwd_dkv(qkv, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s);
+        }
         if (r == 0) return NC_OK;
         if (r < 0) return NC_ERR_CUDA;
     }
+    Prof pr(c, P_ATTN_BWD, 2.0 * attn_flops(c), 0.0);
     CK(launch_attention_bwd_simt(m->at, qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.s));
     return NC_OK;
 }
@@ -254,19 +265,19 @@ int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save) {
         void* ru = lb + c.p.l_ru;
         void* h = lb + c.p.l_h;
         { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, a, (float*)(lb + c.p.l_r1), M, d, c.s)); }
-        RG(run_gemm(c, mk(m, M, m->Nqkv, d, a, d, true, w.wqkv(l), d, true, EPI_STORE, qkv, m->Nqkv, m->at)));
+        RG(run_gemm(c, mk(m, M, m->Nqkv, d, a, d, true, w.wqkv(l), d, true, EPI_STORE, qkv, m->Nqkv, m->at), P_GEMM_FWD));
         {
             Prof pr(c, P_QKROPE_FWD, 0.0, (double)M * (m->H + m->nkv) * (2.0 * A * m->hd + 4.0));
             CK(launch_qknorm_rope_fwd(m->at, qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, c.p.T, m->H, m->nkv, m->hd,
                                       c.s));
         }
         RG(attention_fwd(c, qkv, o, (float*)(lb + c.p.l_lse)));
-        RG(run_gemm(c, mk(m, M, d, (int)Hhd, o, Hhd, true, w.wo(l), Hhd, true, EPI_ACCUM, x, d, DT_F32)));
+        RG(run_gemm(c, mk(m, M, d, (int)Hhd, o, Hhd, true, w.wo(l), Hhd, true, EPI_ACCUM, x, d, DT_F32), P_GEMM_FWD));
         { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, mm, (float*)(lb + c.p.l_r2), M, d, c.s)); }
         GemmDesc fc = mk(m, M, m->F, d, mm, d, true, w.wfc(l), d, true, EPI_RELU2, h, m->F, m->at);
         fc.C2 = ru; fc.ldc2 = m->F;
-        RG(run_gemm(c, fc));
-        RG(run_gemm(c, mk(m, M, d, m->F, h, m->F, true, w.wproj(l), m->F, true, EPI_ACCUM, x, d, DT_F32)));
+        RG(run_gemm(c, fc, P_GEMM_FWD));
+        RG(run_gemm(c, mk(m, M, d, m->F, h, m->F, true, w.wproj(l), m->F, true, EPI_ACCUM, x, d, DT_F32), P_GEMM_FWD));
     }
     { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, c.at(c.p.xf), c.at<float>(c.p.rf), M, d, c.s)); }
     return NC_OK;
@@ -292,16 +303,16 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     for (int r0 = 0; r0 < M; r0 += c.p.R) {
         int rc = std::min(c.p.R, M - r0);
         const char* xfc = (const char*)xf + (size_t)r0 * d * A;
-        RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, DT_F32)));
+        RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, DT_F32), P_GEMM_LM_Z));
         {
             Prof pr(c, P_CE, 0.0, (double)rc * V * (4.0 + A));
             CK(launch_ce_chunk(m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M, loss_rows + r0, dlc,
                                m->status, s));
         }
         RG(run_gemm(c, mk(m, rc, d, V, dlc, V, true, w.wlm(), d, false, EPI_STORE, gbuf + (size_t)r0 * d, d,
-                          DT_F32)));
+                          DT_F32), P_GEMM_LM_DX));
         RG(run_gemm(c, mk(m, V, d, rc, dlc, V, false, xfc, d, false, r0 == 0 ? EPI_STORE : EPI_ACCUM, dwlm, d,
-                          DT_F32)));
+                          DT_F32), P_GEMM_LM_DW));
     }
     { Prof pr(c, P_OTHER, 0.0, 4.0 * M); CK(launch_loss_reduce(loss_rows, M, loss, s)); }
 
@@ -320,24 +331,27 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         // MLP: x_out = x_mid + h Wproj^T, h = relu(u)^2, u = m Wfc^T
         GemmDesc g1 = mk(m, M, F, d, dxb, d, true, w.wproj(l), F, false, EPI_RELU2_BWD, du, F, m->at);
         g1.aux = lb + c.p.l_ru; g1.ldaux = F;
-        RG(run_gemm(c, g1));
-        RG(run_gemm(c, mk(m, d, F, M, dxb, d, false, lb + c.p.l_h, F, false, EPI_STORE, G(base + 5), F, DT_F32)));
-        RG(run_gemm(c, mk(m, M, d, F, du, F, true, w.wfc(l), d, false, EPI_STORE, gbuf, d, DT_F32)));
-        RG(run_gemm(c, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32)));
+        RG(run_gemm(c, g1, P_GEMM_DGRAD));
+        RG(run_gemm(c, mk(m, d, F, M, dxb, d, false, lb + c.p.l_h, F, false, EPI_STORE, G(base + 5), F, DT_F32),
+                    P_GEMM_WGRAD));
+        RG(run_gemm(c, mk(m, M, d, F, du, F, true, w.wfc(l), d, false, EPI_STORE, gbuf, d, DT_F32), P_GEMM_DGRAD));
+        RG(run_gemm(c, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32),
+                    P_GEMM_WGRAD));
         { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (12.0 * d + 2.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_m, (float*)(lb + c.p.l_r2), dx, true, dxb, M, d, s)); }
         // attention: x_mid = x_in + o Wo^T
-        RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at)));
+        RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at), P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
-                          DT_F32)));
+                          DT_F32), P_GEMM_WGRAD));
         RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), dqkv));
         {
             Prof pr(c, P_QKROPE_BWD, 0.0, (double)M * (m->H + m->nkv) * (3.0 * A * m->hd + 4.0));
             CK(launch_qknorm_rope_bwd(m->at, dqkv, lb + c.p.l_qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, T, m->H,
                                       m->nkv, m->hd, s));
         }
-        RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, DT_F32)));
+        RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, DT_F32),
+                    P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, Nqkv, d, M, dqkv, Nqkv, false, lb + c.p.l_a, d, false, EPI_STORE, G(base), d,
-                          DT_F32)));
+                          DT_F32), P_GEMM_WGRAD));
         {
             Prof pr(c, P_NORM_BWD, 0.0, (double)M * (12.0 * d + (l > 0 ? 2.0 : 1.0) * A * d + 4.0));
             CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_a, (float*)(lb + c.p.l_r1), dx, true,
@@ -349,7 +363,7 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         // norm backward (dx, Wte row, r0 -> de), then de read once and dWte written once
         Prof pr(c, P_EMBED_BWD, 0.0, (double)M * (8.0 * d + A * d + 8.0) + 4.0 * M * d + 4.0 * (double)V * d);
         CK(launch_embed_norm_bwd(m->at, dx, tok, w.wte(), c.at<float>(c.p.r0), gbuf, M, V, d, s));
-        CK(launch_embed_scatter(tok, gbuf, M, V, d, G(0), embed_scratch_carve(c.ws + c.p.emb, M, V), s));
+        CK(launch_embed_scatter(tok, gbuf, M, V, d, G(0), embed_scratch_carve(c.ws + c.p.emb, M, V, d), s));
     }
     return NC_OK;
 }
@@ -485,7 +499,7 @@ int nc_forward_logits(nc_model* m, const int32_t* tokens, int B, int T, const vo
     W w{(const char*)weights, dt_size(m->at), m};
     RG(forward_blocks(c, w, tokens, false));
     RG(run_gemm(c, mk(m, c.p.M, m->V, m->d, c.at(c.p.xf), m->d, true, w.wlm(), m->d, true, EPI_SOFTCAP, logits,
-                      m->V, m->at)));
+                      m->V, m->at), P_GEMM_LM_Z));
     return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

@@ -1,0 +1,132 @@
+"""Per-kernel timing of the step's building blocks on synthetic inputs.
+
+    python -m bwd_step_b200.kernel_bench gemm [--only NAME] [--iters N]
+    python -m bwd_step_b200.kernel_bench attention [--iters N]
+
+`gemm` runs every GEMM shape of one depth-20 step (32768 tokens, d 1280,
+MLP 5120, 10x128 MQA, vocab 65536 with a 4096-row LM-head chunk) through the
+testing ABI with its real operand layouts and fused epilogue, and prints
+TFLOP/s from CUDA events.  `attention` times the tcgen05 attention forward and
+backward at seq 2048, batch 16.  Each case holds at most a few GB on the device.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+
+import torch
+
+from . import lib
+
+P = ctypes.c_void_p
+
+M, D, F, NQKV, HHD, V, R = 32768, 1280, 5120, 1536, 1280, 65536, 4096
+
+# name: (M, N, K, a_kmajor, b_kmajor, epi, c_bf16)
+GEMMS = {
+    "fwd_qkv": (M, NQKV, D, 1, 1, 0, 1),
+    "fwd_oproj": (M, D, HHD, 1, 1, 1, 0),
+    "fwd_fc_relu2": (M, F, D, 1, 1, 2, 1),
+    "fwd_proj": (M, D, F, 1, 1, 1, 0),
+    "dgrad_fc_relu2bwd": (M, F, D, 1, 0, 3, 1),
+    "dgrad_mlp_in": (M, D, F, 1, 0, 0, 0),
+    "dgrad_oproj": (M, HHD, D, 1, 0, 0, 1),
+    "dgrad_qkv": (M, D, NQKV, 1, 0, 0, 0),
+    "wgrad_proj": (D, F, M, 0, 0, 0, 0),
+    "wgrad_fc": (F, D, M, 0, 0, 0, 0),
+    "wgrad_oproj": (D, HHD, M, 0, 0, 0, 0),
+    "wgrad_qkv": (NQKV, D, M, 0, 0, 0, 0),
+    "lmhead_z": (R, V, D, 1, 1, 4, 0),
+    "lmhead_dx": (R, D, V, 1, 0, 0, 0),
+    "lmhead_dw": (V, D, R, 0, 0, 1, 0),
+}
+
+
+def _timed(fn, iters):
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def bench_gemm(name, iters):
+    m, n, k, ak, bk, epi, cbf = GEMMS[name]
+    g = torch.Generator(device="cuda").manual_seed(0)
+    A = (torch.randn(m * k, device="cuda", generator=g) * 0.1).to(torch.bfloat16)
+    B = (torch.randn(n * k, device="cuda", generator=g) * 0.1).to(torch.bfloat16)
+    C = torch.zeros(m * n, device="cuda", dtype=torch.bfloat16 if cbf else torch.float32)
+    C2 = torch.zeros(m * n, device="cuda", dtype=torch.bfloat16) if epi == 2 else None
+    aux = torch.rand(m * n, device="cuda", generator=g).to(torch.bfloat16) if epi == 3 else None
+    scratch = torch.empty(8 * 4 * max(R * D, F * D), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lda = k if ak else m
+    ldb = k if bk else n
+    stream = P(torch.cuda.current_stream().cuda_stream)
+
+    def run():
+        r = lib().nc_test_gemm(m, n, k, 1, P(A.data_ptr()), lda, ak, P(B.data_ptr()), ldb, bk, epi, P(C.data_ptr()),
+                               n, cbf, P(C2.data_ptr() if C2 is not None else 0), n,
+                               P(aux.data_ptr() if aux is not None else 0), n, ctypes.c_float(15.0), 1,
+                               P(scratch.data_ptr()), scratch.numel(), P(status.data_ptr()), stream)
+        assert r == 0, r
+
+    ms = _timed(run, iters)
+    assert status.item() == 0
+    return {"kernel": f"gemm_{name}", "M": m, "N": n, "K": k, "ms": ms, "tflops": 2.0 * m * n * k / ms / 1e9}
+
+
+def bench_attention(iters, B=16, T=2048, H=10, nkv=1, hd=128):
+    g = torch.Generator(device="cuda").manual_seed(0)
+    nq = (H + 2 * nkv) * hd
+    qkv = torch.randn(B * T * nq, device="cuda", generator=g).to(torch.bfloat16)
+    dO = torch.randn(B * T * H * hd, device="cuda", generator=g).to(torch.bfloat16)
+    o = torch.empty(B * T * H * hd, device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty(B * T * H, device="cuda", dtype=torch.float32)
+    dqkv = torch.empty_like(qkv)
+    Dbuf = torch.empty_like(lse)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = P(torch.cuda.current_stream().cuda_stream)
+
+    def fwd():
+        assert lib().nc_test_attention(B, T, H, nkv, hd, P(qkv.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
+                                       P(0), P(0), P(0), 1, P(status.data_ptr()), stream) == 0
+
+    def both():
+        assert lib().nc_test_attention(B, T, H, nkv, hd, P(qkv.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
+                                       P(dO.data_ptr()), P(dqkv.data_ptr()), P(Dbuf.data_ptr()), 1,
+                                       P(status.data_ptr()), stream) == 0
+
+    flops = 4.0 * B * H * hd * T * (T + 1) / 2
+    t_f = _timed(fwd, iters)
+    t_b = _timed(both, iters) - t_f
+    assert status.item() == 0
+    return [{"kernel": "attention_fwd", "ms": t_f, "tflops": flops / t_f / 1e9},
+            {"kernel": "attention_bwd", "ms": t_b, "tflops": 2 * flops / t_b / 1e9}]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("what", choices=["gemm", "attention"])
+    ap.add_argument("--only", default=None)
+    ap.add_argument("--iters", type=int, default=10)
+    args = ap.parse_args()
+    if args.what == "gemm":
+        for name in GEMMS:
+            if args.only and args.only != name:
+                continue
+            print(json.dumps(bench_gemm(name, args.iters)), flush=True)
+            torch.cuda.empty_cache()
+    else:
+        for r in bench_attention(args.iters):
+            print(json.dumps(r), flush=True)
+
+
+if __name__ == "__main__":
+    main()
