@@ -56,6 +56,7 @@ SIGNATURES = {
     "nc_profile_read": (_I, [_P, _P, ctypes.POINTER(NcProfileRow), _I]),
     "nc_launch_count": (ctypes.c_int64, []),
     "nc_debug_expired_wait": (_I, [_P, _I, _P]),
+    "nc_gemm_wgrad_noalloc": (_I, [_I, _I, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _I, _P, _P]),
     # include/nanochat_b200_testing.h
     "nc_test_gemm": (_I, [_I, _I, _I, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _P,
                           ctypes.c_int64, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_float, _I, _P,

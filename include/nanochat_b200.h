@@ -155,6 +155,39 @@ int nc_profile_read(nc_model* m, void* stream, nc_profile_row* rows, int max_row
 /* Kernels launched by the library in this process so far. */
 int64_t nc_launch_count(void);
 
+/* Weight-gradient GEMM that allocates no memory at all.
+ *
+ * No counterpart in the paper: this is an extra entry point of this library.
+ * Some callers cannot call cudaMalloc: frameworks whose caching allocator
+ * reserves the device memory up front and owns every later allocation,
+ * latency-critical loops where an allocation (which may synchronise the
+ * device) is not acceptable, and hosts with a fixed memory budget fixed at
+ * start-up.  They can still pass their own inputs and outputs.
+ *
+ * Computes dw[o, i] (+)= sum_{t < rows} dy[t, o] * x[t, i] -- the gradient of a
+ * bias-free linear y = x W^T -- on the tcgen05 tensor cores:
+ *   dy: device bf16 [rows, ld_dy] (first n_out columns used)
+ *   x:  device bf16 [rows, ld_x]  (first n_in columns used)
+ *   dw: device fp32 [n_out, n_in], contiguous; overwritten, or added to when
+ *       accumulate != 0
+ *   status: device int status word for the bounded waits (may be NULL)
+ * Rows must be 16-byte aligned (ld_dy, ld_x multiples of 8).
+ *
+ * Split-K partial sums live in one file-scope static device array of
+ * NC_WGRAD_NOALLOC_SCRATCH_BYTES; every GPU that loads the library holds it
+ * until the process exits.  Results of shape n_out * n_in * 4 * 2 bytes
+ * larger than that array (room for two partials) are rejected with
+ * NC_ERR_UNSUPPORTED_SHAPE.  Every call shares the array and it keeps the
+ * last call's contents; each call overwrites every partial it reads, so
+ * nothing has to start at zero.  Calls that overlap on the GPU (other
+ * streams, other host threads) race on the array: serialise them.  The first
+ * call on a device looks up the array's device address with
+ * cudaGetSymbolAddress (with that device current); make that first call
+ * before any stream capture. */
+#define NC_WGRAD_NOALLOC_SCRATCH_BYTES (64u << 20)
+int nc_gemm_wgrad_noalloc(int rows, int n_out, int n_in, const void* dy, int64_t ld_dy, const void* x,
+                          int64_t ld_x, float* dw, int accumulate, int* status, void* stream);
+
 /* Test hook for the bounded device wait: launches one kernel that waits on an
  * mbarrier nobody arrives at, with an iteration cap of `max_iters`; when the
  * cap is hit the kernel records NC_ERR_DEVICE_TIMEOUT in the status word and
