@@ -84,13 +84,13 @@ __global__ void __launch_bounds__(256) attn_fwd_kernel(const A* __restrict__ qkv
         int c = lane + 32 * i;
         if (c < HD) o[row * (size_t)(H * HD) + h * HD + c] = fromf<A>(acc[i] * inv);
     }
-    if (lane == 0) lse[row * H + h] = m + logf(l);
+    if (lane == 0) lse[((size_t)b * H + h) * attn_tpad(T) + p] = m + logf(l);
 }
 
-// D[row, h] = sum_c dO[row, h, c] * o[row, h, c]; one warp per (row, head).
+// D[b, h, t] = sum_c dO[row, h, c] * o[row, h, c]; one warp per (row, head).
 template <typename A>
 __global__ void attn_bwd_dot_kernel(const A* __restrict__ o, const A* __restrict__ dO, float* __restrict__ D,
-                                    int MH, int hd) {
+                                    int MH, int T, int H, int hd) {
     int wid = blockIdx.x * WPB + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (wid >= MH) return;
     const A* a = o + (size_t)wid * hd;
@@ -98,7 +98,8 @@ __global__ void attn_bwd_dot_kernel(const A* __restrict__ o, const A* __restrict
     float s = 0.f;
     for (int c = lane; c < hd; c += 32) s += tof(a[c]) * tof(b[c]);
     s = warp_sum(s);
-    if (lane == 0) D[wid] = s;
+    int row = wid / H, h = wid % H;
+    if (lane == 0) D[((size_t)(row / T) * H + h) * attn_tpad(T) + row % T] = s;
 }
 
 template <typename A, int HD>
@@ -122,8 +123,9 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const A* __restrict__ 
         Qs[w][c] = live ? tof(base[(size_t)p * ld + h * HD + c]) : 0.f;
         Gs[w][c] = live ? tof(dO[row * (size_t)(H * HD) + h * HD + c]) : 0.f;
     }
-    float L = live ? lse[row * H + h] : 0.f;
-    float Dr = live ? D[row * H + h] : 0.f;
+    const size_t si = ((size_t)b * H + h) * attn_tpad(T) + (live ? p : 0);
+    float L = live ? lse[si] : 0.f;
+    float Dr = live ? D[si] : 0.f;
     float acc[NI];
 #pragma unroll
     for (int i = 0; i < NI; ++i) acc[i] = 0.f;
@@ -209,9 +211,9 @@ __global__ void __launch_bounds__(256) attn_bwd_dkv_kernel(const A* __restrict__
             int rr = r0 + threadIdx.x;
             bool ok = rr < NR;
             int qi = i0 + rr / Hg, hh = g * Hg + rr % Hg;
-            size_t qrow = (size_t)b * T + qi;
-            Ls[threadIdx.x] = ok ? lse[qrow * H + hh] : 0.f;
-            Ds[threadIdx.x] = ok ? D[qrow * H + hh] : 0.f;
+            size_t si = ((size_t)b * H + hh) * attn_tpad(T) + qi;
+            Ls[threadIdx.x] = ok ? lse[si] : 0.f;
+            Ds[threadIdx.x] = ok ? D[si] : 0.f;
         }
         __syncthreads();
         if (!live) continue;
@@ -265,7 +267,7 @@ template <typename A, int HD>
 cudaError_t bwd_t(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
                   int B, int T, int H, int nkv, cudaStream_t s) {
     int MH = B * T * H;
-    attn_bwd_dot_kernel<A><<<(MH + WPB - 1) / WPB, 256, 0, s>>>((const A*)o, (const A*)dO, Dbuf, MH, HD);
+    attn_bwd_dot_kernel<A><<<(MH + WPB - 1) / WPB, 256, 0, s>>>((const A*)o, (const A*)dO, Dbuf, MH, T, H, HD);
     dim3 gq((T + WPB - 1) / WPB, H, B);
     attn_bwd_dq_kernel<A, HD><<<gq, 256, 0, s>>>((const A*)qkv, (const A*)dO, lse, Dbuf, (A*)dqkv, T, H, nkv);
     dim3 gk((T + WPB - 1) / WPB, nkv, B);
@@ -305,12 +307,15 @@ cudaError_t launch_attention_fwd_simt(DType at, const void* qkv, void* o, float*
                          : fwd_d<float>(qkv, o, lse, B, T, H, nkv, hd, s);
 }
 
-cudaError_t launch_attention_bwd_dot(DType at, const void* o, const void* dO, float* D, int MH, int hd,
+cudaError_t launch_attention_bwd_dot(DType at, const void* o, const void* dO, float* D, int B, int T, int H, int hd,
                                      cudaStream_t s) {
+    const int MH = B * T * H;
     if (at == DT_BF16)
-        attn_bwd_dot_kernel<bf16><<<(MH + WPB - 1) / WPB, 256, 0, s>>>((const bf16*)o, (const bf16*)dO, D, MH, hd);
+        attn_bwd_dot_kernel<bf16><<<(MH + WPB - 1) / WPB, 256, 0, s>>>((const bf16*)o, (const bf16*)dO, D, MH, T, H,
+                                                                       hd);
     else
-        attn_bwd_dot_kernel<float><<<(MH + WPB - 1) / WPB, 256, 0, s>>>((const float*)o, (const float*)dO, D, MH, hd);
+        attn_bwd_dot_kernel<float><<<(MH + WPB - 1) / WPB, 256, 0, s>>>((const float*)o, (const float*)dO, D, MH, T,
+                                                                        H, hd);
     count_launch();
     return cudaGetLastError();
 }

@@ -73,8 +73,8 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb = p.nqb - 1 - (int)blockIdx.x;  // largest blocks first
-    const int h = blockIdx.y, b = blockIdx.z, g = h / (p.H / p.nkv);
+    const int qb = p.nqb - 1 - (int)blockIdx.z;  // grid z slowest: the longest blocks launch first
+    const int h = blockIdx.x, b = blockIdx.y, g = h / (p.H / p.nkv);
     const int nblk = qb + 1;
     const int row0 = b * p.T;
 
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                     }
                 }
             }
-            if (live) p.lse[((size_t)row0 + qpos) * p.H + h] = (m + __log2f(l)) * kLn2;
+            if (live) p.lse[((size_t)b * p.H + h) * attn_tpad(p.T) + qpos] = (m + __log2f(l)) * kLn2;
         }
     }
     tc_fence_before();
@@ -327,8 +327,8 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb = p.nqb - 1 - (int)blockIdx.x;
-    const int h = blockIdx.y, b = blockIdx.z, g = h / (p.H / p.nkv);
+    const int qb = p.nqb - 1 - (int)blockIdx.z;  // longest blocks launch first
+    const int h = blockIdx.x, b = blockIdx.y, g = h / (p.H / p.nkv);
     const int nblk = qb + 1;
     const int row0 = b * p.T;
     const int Nqkv = (p.H + 2 * p.nkv) * HD;
@@ -428,8 +428,9 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
         const int qpos = qb * 128 + r;
         const bool live = qpos < p.T;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const float lse2 = live ? p.lse[((size_t)row0 + qpos) * p.H + h] * kLog2e : 0.f;
-        const float Dr = live ? p.D[((size_t)row0 + qpos) * p.H + h] : 0.f;
+        const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + (live ? qpos : 0);
+        const float lse2 = live ? p.lse[si] * kLog2e : 0.f;
+        const float Dr = live ? p.D[si] : 0.f;
         bool ok = true;
         for (int j = 0; j < nblk && ok; ++j) {
             if (!warp_wait(s_full, j & 1, abort_flag, p.status)) { ok = false; break; }
@@ -506,8 +507,8 @@ struct DkvLayout {
     static constexpr int DO = Q + STG * HTILE;
     static constexpr int PT = DO + STG * HTILE;
     static constexpr int DST = PT + 16384;
-    static constexpr int LSE = DST + 16384;   // [2][64] floats, log2 units
-    static constexpr int DD = LSE + 512;      // [2][64] floats
+    static constexpr int LSE = DST + 16384;   // [STG][64] floats: lse of the unit's queries
+    static constexpr int DD = LSE + 512;      // [STG][64] floats: D of the unit's queries
     static constexpr int BAR = DD + 512;
     static constexpr int BYTES = BAR + 256 + 1024;
 };
@@ -529,13 +530,13 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24, st_full = b0 + 40, st_empty = b0 + 56;
-    const uint32_t pd_full = b0 + 72, pd_done = b0 + 80, stage_ready = b0 + 88;  // stage_ready[2]
+    const uint32_t pd_full = b0 + 72, pd_done = b0 + 80;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kvb = blockIdx.x;  // largest amount of work first
-    const int g = blockIdx.y, b = blockIdx.z;
+    const int kvb = blockIdx.z;  // grid z slowest: key block 0 (the most units) launches first
+    const int g = blockIdx.y, b = blockIdx.x;
     const int Hg = p.H / p.nkv;
     const int row0 = b * p.T;
     const int Nqkv = (p.H + 2 * p.nkv) * HD;
@@ -549,8 +550,6 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
         for (int s = 0; s < 2; ++s) { mbar_init(st_full + 8 * s, 1); mbar_init(st_empty + 8 * s, 4); }
         mbar_init(pd_full, 4);
         mbar_init(pd_done, 1);
-        mbar_init(stage_ready, 128);
-        mbar_init(stage_ready + 8, 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -576,7 +575,10 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
                 const int st = u % STG;
                 const int i = i0 + u / Hg, h = g * Hg + u % Hg;
                 if (!mbar_wait(qo_empty + 8 * st, ((u / STG) & 1) ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(qo_full + 8 * st, 2 * HTILE);
+                mbar_expect_tx(qo_full + 8 * st, 2 * HTILE + 512);
+                const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + (size_t)i * 64;
+                bulk_load(base + Lay::LSE + st * 256, p.lse + si, 256, qo_full + 8 * st);
+                bulk_load(base + Lay::DD + st * 256, p.D + si, 256, qo_full + 8 * st);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
                     tma_load_2d(sQ + st * HTILE + kb * 8192, &tmQ64, h * HD + kb * 64, row0 + i * 64, qo_full + 8 * st);
@@ -640,20 +642,16 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         bool ok = true;
         for (int u = 0; u < nunits; ++u) {
-            const int sb = u & 1, buf = u & 1;
-            const int i = i0 + u / Hg, h = g * Hg + u % Hg;
-            {
-                const int qq = i * 64 + (t & 63);
-                const bool inr = qq < p.T;
-                const size_t idx = ((size_t)row0 + qq) * p.H + h;
-                if (t < 64) lse_s[buf * 64 + t] = inr ? p.lse[idx] * kLog2e : INFINITY;
-                else d_s[buf * 64 + (t - 64)] = inr ? p.D[idx] : 0.f;
-            }
-            mbar_arrive(stage_ready + 8 * buf);
-            if (!warp_wait(stage_ready + 8 * buf, (u >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            const int sb = u & 1, st = u % STG;
+            const int i = i0 + u / Hg;
             if (!warp_wait(st_full + 8 * sb, (u >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            // this unit's Q/dO/lse/D stage has landed (the phase cannot move on
+            // before this warp finishes the unit, which frees the stage)
+            if (!warp_wait(qo_full + 8 * st, (u / STG) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
             if (u > 0 && !warp_wait(pd_done, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            const float* lse_u = lse_s + st * 64;
+            const float* d_u = d_s + st * 64;
             uint8_t* prow = smem + Lay::PT + r * 128;
             uint8_t* drow = smem + Lay::DST + r * 128;
 #pragma unroll
@@ -663,10 +661,10 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
                 tmem_ld32(tdPt + lane_off + sb * 64 + c * 32, dp);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const int qc = c * 32 + e;
-                    const bool valid = i * 64 + qc >= kpos;
-                    const float P = valid ? ex2(sv[e] * p.scale_log2 - lse_s[buf * 64 + qc]) : 0.f;
-                    dp[e] = P * (dp[e] - d_s[buf * 64 + qc]);
+                    const int qc = c * 32 + e, qpos = i * 64 + qc;
+                    const bool valid = qpos >= kpos && qpos < p.T;
+                    const float P = valid ? ex2(sv[e] * p.scale_log2 - lse_u[qc] * kLog2e) : 0.f;
+                    dp[e] = valid ? P * (dp[e] - d_u[qc]) : 0.f;
                     sv[e] = P;
                 }
 #pragma unroll
@@ -757,7 +755,7 @@ int fwd_launch(const CUtensorMap& map, const AttnParams& p, cudaStream_t s) {
             return -1;
         attr = true;
     }
-    dim3 grid(p.nqb, p.H, p.B);
+    dim3 grid(p.H, p.B, p.nqb);
     attn_fwd_tc_kernel<HD><<<grid, NT, FwdLayout<HD>::BYTES, s>>>(map, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
@@ -772,7 +770,7 @@ int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& 
             return -1;
         attr = true;
     }
-    attn_dq_tc_kernel<HD><<<dim3(p.nqb, p.H, p.B), NT, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
+    attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NT, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -787,7 +785,7 @@ int dkv_launch(const CUtensorMap& kv, const CUtensorMap& q64, const CUtensorMap&
             return -1;
         attr = true;
     }
-    attn_dkv_tc_kernel<HD><<<dim3(p.nqb, p.nkv, p.B), NT, DkvLayout<HD>::BYTES, s>>>(kv, q64, do64, p);
+    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NT, DkvLayout<HD>::BYTES, s>>>(kv, q64, do64, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -832,7 +830,7 @@ int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const fl
     CUtensorMap kv, do128;
     if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128))
         return 1;
-    if (launch_attention_bwd_dot(DT_BF16, o, dO, Dbuf, B * T * H, hd, s) != cudaSuccess) return -1;
+    if (launch_attention_bwd_dot(DT_BF16, o, dO, Dbuf, B, T, H, hd, s) != cudaSuccess) return -1;
     BwdParams p = bwd_params(lse, Dbuf, dqkv, B, T, H, nkv, hd, status);
     return hd == 128 ? dq_launch<128>(kv, do128, p, s) : dq_launch<64>(kv, do128, p, s);
 }

@@ -59,7 +59,9 @@ __device__ __forceinline__ void store_row_f32(float* dst, const float* v, int nv
         for (int i = 0; i < 8; ++i)
             reinterpret_cast<float4*>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     } else {
-        for (int i = 0; i < nv; ++i) dst[i] = v[i];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < nv) dst[i] = v[i];
     }
 }
 __device__ __forceinline__ void store_row_bf16(bf16* dst, const float* v, int nv, bool vec) {
@@ -67,7 +69,9 @@ __device__ __forceinline__ void store_row_bf16(bf16* dst, const float* v, int nv
 #pragma unroll
         for (int i = 0; i < 4; ++i) store_vec(dst + 8 * i, v + 8 * i);
     } else {
-        for (int i = 0; i < nv; ++i) dst[i] = __float2bfloat16_rn(v[i]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < nv) dst[i] = __float2bfloat16_rn(v[i]);
     }
 }
 __device__ __forceinline__ void store_row(void* C, bool bf, int64_t off, const float* v, int nv, bool vec) {
@@ -95,7 +99,9 @@ __device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int
                     v[4 * i] += o.x; v[4 * i + 1] += o.y; v[4 * i + 2] += o.z; v[4 * i + 3] += o.w;
                 }
             } else {
-                for (int i = 0; i < nv; ++i) v[i] += c[i];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < nv) v[i] += c[i];
             }
             store_row_f32(c, v, nv, vec);
         } break;
@@ -117,7 +123,9 @@ __device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int
                     for (int j = 0; j < 8; ++j) v[8 * i + j] *= 2.f * u[j];
                 }
             } else {
-                for (int i = 0; i < nv; ++i) v[i] *= 2.f * __bfloat162float(a[i]);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < nv) v[i] *= 2.f * __bfloat162float(a[i]);
             }
             store_row_bf16(reinterpret_cast<bf16*>(p.C) + off, v, nv, vec);
         } break;

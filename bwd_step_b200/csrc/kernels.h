@@ -98,7 +98,11 @@ cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
 // qkv rows [B*T, (H+2nkv)*hd] hold q (post norm+rope), k (same), v.
-// o [B*T, H*hd]; lse [B*T, H] (natural log).
+// o [B*T, H*hd].  Per-(row, head) softmax statistics (lse, natural log, and
+// the backward's D) are stored head-major with the sequence padded to a
+// multiple of 64: index (b*H + h)*attn_tpad(T) + t.
+__host__ __device__ inline int attn_tpad(int T) { return (T + 63) / 64 * 64; }
+inline size_t attn_stat_elems(int B, int T, int H) { return (size_t)B * H * attn_tpad(T); }
 cudaError_t launch_attention_fwd_simt(DType at, const void* qkv, void* o, float* lse, int B, int T, int H,
                                       int nkv, int hd, cudaStream_t s);
 // Writes dq (into the q columns), dk, dv of dqkv.  Dbuf [B*T, H] scratch.
@@ -106,8 +110,8 @@ cudaError_t launch_attention_bwd_simt(DType at, const void* qkv, const void* o, 
                                       const float* lse, float* Dbuf, void* dqkv, int B, int T, int H,
                                       int nkv, int hd, cudaStream_t s);
 
-// D[row, h] = sum_c dO[row, h, c] * o[row, h, c] (softmax backward row term).
-cudaError_t launch_attention_bwd_dot(DType at, const void* o, const void* dO, float* D, int MH, int hd,
+// D[b, h, t] = sum_c dO[b*T+t, h, c] * o[b*T+t, h, c] (softmax backward row term).
+cudaError_t launch_attention_bwd_dot(DType at, const void* o, const void* dO, float* D, int B, int T, int H, int hd,
                                      cudaStream_t s);
 
 // ---------------------------------------------------------------- bounded wait

@@ -97,7 +97,7 @@ Plan make_plan(const nc_model* m, int B, int T) {
     p.l_qkv = ltake(A * M * m->Nqkv);
     p.l_rqk = ltake(4 * M * (m->H + m->nkv));
     p.l_o = ltake(A * M * m->H * m->hd);
-    p.l_lse = ltake(4 * M * m->H);
+    p.l_lse = ltake(4 * attn_stat_elems(B, T, m->H));
     p.l_m = ltake(A * M * d);
     p.l_r2 = ltake(4 * M);
     p.l_ru = ltake(A * M * m->F);
@@ -107,7 +107,7 @@ Plan make_plan(const nc_model* m, int B, int T) {
     p.du = take(A * M * m->F);
     p.dO = take(A * M * m->H * m->hd);
     p.dqkv = take(A * M * m->Nqkv);
-    p.Dbuf = take(4 * M * m->H);
+    p.Dbuf = take(4 * attn_stat_elems(B, T, m->H));
     p.R = lm_chunk_rows(m, p.M);
     p.zc = take(4ull * p.R * m->V);
     p.dlc = take(A * (size_t)p.R * m->V);

@@ -88,7 +88,7 @@ def bench_attention(iters, B=16, T=2048, H=10, nkv=1, hd=128):
     qkv = torch.randn(B * T * nq, device="cuda", generator=g).to(torch.bfloat16)
     dO = torch.randn(B * T * H * hd, device="cuda", generator=g).to(torch.bfloat16)
     o = torch.empty(B * T * H * hd, device="cuda", dtype=torch.bfloat16)
-    lse = torch.empty(B * T * H, device="cuda", dtype=torch.float32)
+    lse = torch.empty(B * H * ((T + 63) // 64 * 64), device="cuda", dtype=torch.float32)
     dqkv = torch.empty_like(qkv)
     Dbuf = torch.empty_like(lse)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
