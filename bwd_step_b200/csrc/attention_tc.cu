@@ -276,11 +276,13 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 
 
 // ============================================================================ backward
-// dQ, one CTA per (query block of 128, head, batch row): for key blocks
-// j = 0..qb, S = Q K_j^T and dP = dO V_j^T into TMEM; per query row (one per
-// thread) P = 2^(S*scale*log2e - lse*log2e) with the causal mask, dS = P (dP - D)
-// as bf16 into shared memory; dQ += dS K_j with the K_j tile read again as an
-// MN-major operand.  dq = dQ / sqrt(hd).
+// dQ, one CTA per (query block of 128, head, batch row).  Key blocks j = 0..qb
+// are processed as 64-key sub-blocks t: S_t = Q K_t^T and dP_t = dO V_t^T into
+// one of two TMEM buffers; per query row (one per thread)
+// P = 2^(S*scale*log2e - lse*log2e) with the causal mask and dS = P (dP - D),
+// as bf16 into one of two shared-memory tiles; dQ += dS_{t-1} K_{t-1} is issued
+// one sub-block behind, with the K tile read again as an MN-major operand.
+// dq = dQ / sqrt(hd).
 template <int HD>
 struct DqLayout {
     static constexpr int KB = HD / 64;
@@ -289,7 +291,7 @@ struct DqLayout {
     static constexpr int DO = Q + TILE;
     static constexpr int K = DO + TILE;
     static constexpr int V = K + STG * TILE;
-    static constexpr int DS = V + STG * TILE;
+    static constexpr int DS = V + STG * TILE;   // [2][128 x 64] bf16
     static constexpr int BAR = DS + 32768;
     static constexpr int BYTES = BAR + 256 + 1024;
 };
@@ -322,24 +324,25 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t qd_full = b0, k_full = b0 + 8, k_empty = b0 + 24, v_full = b0 + 40, v_empty = b0 + 56;
-    const uint32_t s_full = b0 + 72, s_empty = b0 + 80, ds_full = b0 + 88, ds_done = b0 + 96;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    const uint32_t s_full = b0 + 72, s_empty = b0 + 88, ds_full = b0 + 104, ds_done = b0 + 120;  // each [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qb = p.nqb - 1 - (int)blockIdx.z;  // longest blocks launch first
     const int h = blockIdx.x, b = blockIdx.y, g = h / (p.H / p.nkv);
-    const int nblk = qb + 1;
+    const int nblk = qb + 1, nsub = 2 * nblk;
     const int row0 = b * p.T;
     const int Nqkv = (p.H + 2 * p.nkv) * HD;
 
     if (threadIdx.x == 0) {
         mbar_init(qd_full, 1);
-        for (int s = 0; s < STG; ++s) {
+        for (int s = 0; s < 2; ++s) {
             mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1);
             mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1);
+            mbar_init(s_full + 8 * s, 1); mbar_init(s_empty + 8 * s, 4);
+            mbar_init(ds_full + 8 * s, 4); mbar_init(ds_done + 8 * s, 1);
         }
-        mbar_init(s_full, 1); mbar_init(s_empty, 4); mbar_init(ds_full, 4); mbar_init(ds_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -385,40 +388,42 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id_s = idesc_bf16(128, 128, false, false);
+            const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t id_q = idesc_bf16(128, HD, false, true);
             if (mbar_wait(qd_full, 0, abort_flag, p.status)) {
-                for (int j = 0; j < nblk; ++j) {
-                    const int st = j % STG;
-                    const uint32_t ph = (j / STG) & 1;
-                    if (!mbar_wait(k_full + 8 * st, ph, abort_flag, p.status)) break;
-                    if (!mbar_wait(v_full + 8 * st, ph, abort_flag, p.status)) break;
-                    if (!mbar_wait(s_empty, (j & 1) ^ 1, abort_flag, p.status)) break;
-                    tc_fence_after();
+                for (int t = 0; t <= nsub; ++t) {
+                    if (t < nsub) {
+                        const int j = t >> 1, hf = t & 1, st = j % STG, sb = t & 1;
+                        if (hf == 0) {
+                            if (!mbar_wait(k_full + 8 * st, (j / STG) & 1, abort_flag, p.status)) break;
+                            if (!mbar_wait(v_full + 8 * st, (j / STG) & 1, abort_flag, p.status)) break;
+                        }
+                        if (!mbar_wait(s_empty + 8 * sb, ((t >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+                        tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < HD / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16(tS, smem_desc(sQ + off, 16, 1024), smem_desc(sK + st * TILE + off, 16, 1024), id_s,
-                                 ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < HD / 16; ++ks) {
+                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                            const uint32_t offk = st * TILE + (ks >> 2) * 16384 + hf * 8192 + (ks & 3) * 32;
+                            mma_bf16(tS + sb * 64, smem_desc(sQ + off, 16, 1024), smem_desc(sK + offk, 16, 1024), id_s,
+                                     ks > 0 ? 1u : 0u);
+                            mma_bf16(tdP + sb * 64, smem_desc(sDO + off, 16, 1024), smem_desc(sV + offk, 16, 1024),
+                                     id_s, ks > 0 ? 1u : 0u);
+                        }
+                        mma_commit(s_full + 8 * sb);
+                        if (hf == 1) mma_commit(v_empty + 8 * st);
                     }
+                    if (t > 0) {
+                        const int tt = t - 1, jj = tt >> 1, hh = tt & 1, st = jj % STG, db = tt & 1;
+                        if (!mbar_wait(ds_full + 8 * db, (tt >> 1) & 1, abort_flag, p.status)) break;
+                        tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < HD / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16(tdP, smem_desc(sDO + off, 16, 1024), smem_desc(sV + st * TILE + off, 16, 1024), id_s,
-                                 ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16(tdQ, smem_desc(sDS + db * 16384 + ks * 32, 16, 1024),
+                                     smem_desc(sK + st * TILE + hh * 8192 + ks * 2048, 16384, 1024), id_q,
+                                     (tt > 0 || ks > 0) ? 1u : 0u);
+                        mma_commit(ds_done + 8 * db);
+                        if (hh == 1) mma_commit(k_empty + 8 * st);
                     }
-                    mma_commit(s_full);
-                    mma_commit(v_empty + 8 * st);
-                    if (!mbar_wait(ds_full, j & 1, abort_flag, p.status)) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t offd = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16(tdQ, smem_desc(sDS + offd, 16, 1024), smem_desc(sK + st * TILE + ks * 2048, 16384, 1024),
-                                 id_q, (j > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    mma_commit(ds_done);
-                    mma_commit(k_empty + 8 * st);
                 }
             }
         }
@@ -432,37 +437,46 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
         const float lse2 = live ? p.lse[si] * kLog2e : 0.f;
         const float Dr = live ? p.D[si] : 0.f;
         bool ok = true;
-        for (int j = 0; j < nblk && ok; ++j) {
-            if (!warp_wait(s_full, j & 1, abort_flag, p.status)) { ok = false; break; }
+        for (int t = 0; t < nsub; ++t) {
+            const int j = t >> 1, hf = t & 1, sb = t & 1;
+            if (!warp_wait(s_full + 8 * sb, (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            if (j > 0 && !warp_wait(ds_done, (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            uint8_t* drow = smem + Lay::DS + r * 128;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float sv[32], dp[32];
-                tmem_ld32(tS + lane_off + c * 32, sv);
-                tmem_ld32(tdP + lane_off + c * 32, dp);
+            float d0[32], d1[32];
+            {
+                float sv[32];
+                tmem_ld32(tS + lane_off + sb * 64, sv);
+                tmem_ld32(tdP + lane_off + sb * 64, d0);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const bool valid = live && (j < qb || c * 32 + i <= r);
-                    const float P = valid ? ex2(sv[i] * p.scale_log2 - lse2) : 0.f;
-                    sv[i] = P * (dp[i] - Dr);
+                    const bool valid = live && (j < qb || hf * 64 + i <= r);
+                    d0[i] = valid ? ex2(sv[i] * p.scale_log2 - lse2) * (d0[i] - Dr) : 0.f;
                 }
+                tmem_ld32(tS + lane_off + sb * 64 + 32, sv);
+                tmem_ld32(tdP + lane_off + sb * 64 + 32, d1);
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const int idx = (c & 1) * 4 + t;
-                    const float* v = sv + 8 * t;
-                    *reinterpret_cast<uint4*>(drow + (c >> 1) * 16384 + ((idx ^ (r & 7)) << 4)) =
-                        make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                                   pack_bf16(v[6], v[7]));
+                for (int i = 0; i < 32; ++i) {
+                    const bool valid = live && (j < qb || hf * 64 + 32 + i <= r);
+                    d1[i] = valid ? ex2(sv[i] * p.scale_log2 - lse2) * (d1[i] - Dr) : 0.f;
                 }
             }
             tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_empty + 8 * sb);
+            // dS buffer sb was last read by the dQ MMAs of sub-block t-2
+            if (t > 1 && !warp_wait(ds_done + 8 * sb, ((t >> 1) - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            uint8_t* drow = smem + Lay::DS + sb * 16384 + r * 128;
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {
+                const float* v = c8 < 4 ? d0 + 8 * c8 : d1 + 8 * (c8 - 4);
+                *reinterpret_cast<uint4*>(drow + ((c8 ^ (r & 7)) << 4)) =
+                    make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                               pack_bf16(v[6], v[7]));
+            }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) { mbar_arrive(s_empty); mbar_arrive(ds_full); }
+            if (lane == 0) mbar_arrive(ds_full + 8 * sb);
         }
-        if (ok && warp_wait(ds_done, (nblk - 1) & 1, abort_flag, p.status)) {
+        if (ok && warp_wait(ds_done + 8 * ((nsub - 1) & 1), ((nsub - 1) >> 1) & 1, abort_flag, p.status)) {
             tc_fence_after();
             bf16* out = p.dqkv + ((size_t)row0 + qpos) * Nqkv + h * HD;
 #pragma unroll
@@ -471,12 +485,12 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
                 tmem_ld32(tdQ + lane_off + c * 32, o);
                 if (live) {
 #pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        *reinterpret_cast<uint4*>(out + c * 32 + 8 * t) = make_uint4(
-                            pack_bf16(o[8 * t] * p.scale, o[8 * t + 1] * p.scale),
-                            pack_bf16(o[8 * t + 2] * p.scale, o[8 * t + 3] * p.scale),
-                            pack_bf16(o[8 * t + 4] * p.scale, o[8 * t + 5] * p.scale),
-                            pack_bf16(o[8 * t + 6] * p.scale, o[8 * t + 7] * p.scale));
+                    for (int t4 = 0; t4 < 4; ++t4)
+                        *reinterpret_cast<uint4*>(out + c * 32 + 8 * t4) = make_uint4(
+                            pack_bf16(o[8 * t4] * p.scale, o[8 * t4 + 1] * p.scale),
+                            pack_bf16(o[8 * t4 + 2] * p.scale, o[8 * t4 + 3] * p.scale),
+                            pack_bf16(o[8 * t4 + 4] * p.scale, o[8 * t4 + 5] * p.scale),
+                            pack_bf16(o[8 * t4 + 6] * p.scale, o[8 * t4 + 7] * p.scale));
                 }
             }
         }
@@ -505,9 +519,9 @@ struct DkvLayout {
     static constexpr int V = K + TILE;
     static constexpr int Q = V + TILE;
     static constexpr int DO = Q + STG * HTILE;
-    static constexpr int PT = DO + STG * HTILE;
-    static constexpr int DST = PT + 16384;
-    static constexpr int LSE = DST + 16384;   // [STG][64] floats: lse of the unit's queries
+    static constexpr int PT = DO + STG * HTILE;   // [2][128 x 64] bf16, by unit parity
+    static constexpr int DST = PT + 2 * 16384;    // [2][128 x 64] bf16, by unit parity
+    static constexpr int LSE = DST + 2 * 16384;   // [STG][64] floats: lse of the unit's queries
     static constexpr int DD = LSE + 512;      // [STG][64] floats: D of the unit's queries
     static constexpr int BAR = DD + 512;
     static constexpr int BYTES = BAR + 256 + 1024;
@@ -530,7 +544,9 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24, st_full = b0 + 40, st_empty = b0 + 56;
-    const uint32_t pd_full = b0 + 72, pd_done = b0 + 80;
+    // pd_done[b] completes after the dV/dK MMAs of the units with parity b
+    // (once per two units), so a wait on it can never be lapped.
+    const uint32_t pd_full = b0 + 72, pd_done = b0 + 80;  // pd_done[2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -550,6 +566,7 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
         for (int s = 0; s < 2; ++s) { mbar_init(st_full + 8 * s, 1); mbar_init(st_empty + 8 * s, 4); }
         mbar_init(pd_full, 4);
         mbar_init(pd_done, 1);
+        mbar_init(pd_done + 8, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -621,14 +638,15 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
                         tc_fence_after();
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks) {
-                            mma_bf16(tdV, smem_desc(sPT + ks * 32, 16, 1024),
+                            const uint32_t pb = (uu & 1) * 16384 + ks * 32;
+                            mma_bf16(tdV, smem_desc(sPT + pb, 16, 1024),
                                      smem_desc(sDO + st * HTILE + ks * 2048, 8192, 1024), id_kv,
                                      (uu > 0 || ks > 0) ? 1u : 0u);
-                            mma_bf16(tdK, smem_desc(sDST + ks * 32, 16, 1024),
+                            mma_bf16(tdK, smem_desc(sDST + pb, 16, 1024),
                                      smem_desc(sQ + st * HTILE + ks * 2048, 8192, 1024), id_kv,
                                      (uu > 0 || ks > 0) ? 1u : 0u);
                         }
-                        mma_commit(pd_done);
+                        mma_commit(pd_done + 8 * (uu & 1));
                         mma_commit(qo_empty + 8 * st);
                     }
                 }
@@ -649,11 +667,15 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
             // before this warp finishes the unit, which frees the stage)
             if (!warp_wait(qo_full + 8 * st, (u / STG) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            if (u > 0 && !warp_wait(pd_done, (u - 1) & 1, abort_flag, p.status)) { ok = false; break; }
             const float* lse_u = lse_s + st * 64;
             const float* d_u = d_s + st * 64;
-            uint8_t* prow = smem + Lay::PT + r * 128;
-            uint8_t* drow = smem + Lay::DST + r * 128;
+            // P^T / dS^T buffer (u & 1) was last read by the dV/dK MMAs of unit u-2
+            if (u > 1 && !warp_wait(pd_done + 8 * (u & 1), ((u >> 1) - 1) & 1, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            uint8_t* prow = smem + Lay::PT + (u & 1) * 16384 + r * 128;
+            uint8_t* drow = smem + Lay::DST + (u & 1) * 16384 + r * 128;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 float sv[32], dp[32];
@@ -684,7 +706,7 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
             __syncwarp();
             if (lane == 0) { mbar_arrive(st_empty + 8 * sb); mbar_arrive(pd_full); }
         }
-        if (ok && warp_wait(pd_done, (nunits - 1) & 1, abort_flag, p.status)) {
+        if (ok && warp_wait(pd_done + 8 * ((nunits - 1) & 1), ((nunits - 1) >> 1) & 1, abort_flag, p.status)) {
             tc_fence_after();
             const bool live = kpos < p.T;
             bf16* out_k = p.dqkv + ((size_t)row0 + kpos) * Nqkv + (p.H + g) * HD;
