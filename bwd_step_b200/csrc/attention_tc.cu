@@ -26,7 +26,8 @@ namespace nc {
 namespace {
 using namespace tc;
 
-constexpr int NT = 192;
+constexpr int NT = 192;   // forward: producer, MMA, 4 softmax warps
+constexpr int NTB = 320;  // backward: producer, MMA, 8 softmax warps (two per TMEM lane quarter)
 constexpr int STG = 2;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
@@ -311,7 +312,7 @@ __device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
 }
 
 template <int HD>
-__global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
+__global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
                                                            const __grid_constant__ CUtensorMap tmDO,
                                                            const BwdParams p) {
     using Lay = DqLayout<HD>;
@@ -340,8 +341,8 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
         for (int s = 0; s < 2; ++s) {
             mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1);
             mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1);
-            mbar_init(s_full + 8 * s, 1); mbar_init(s_empty + 8 * s, 4);
-            mbar_init(ds_full + 8 * s, 4); mbar_init(ds_done + 8 * s, 1);
+            mbar_init(s_full + 8 * s, 1); mbar_init(s_empty + 8 * s, 8);
+            mbar_init(ds_full + 8 * s, 8); mbar_init(ds_done + 8 * s, 1);
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -428,7 +429,8 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
             }
         }
     } else {
-        const int q = warp & 3;
+        // warps 2..9: TMEM lane quarter q = warp % 4 (query rows), key half ch of each sub-block
+        const int q = warp & 3, ch = (warp - 2) >> 2;
         const int r = q * 32 + lane;
         const int qpos = qb * 128 + r;
         const bool live = qpos < p.T;
@@ -441,22 +443,15 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
             const int j = t >> 1, hf = t & 1, sb = t & 1;
             if (!warp_wait(s_full + 8 * sb, (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            float d0[32], d1[32];
+            float d0[32];
             {
                 float sv[32];
-                tmem_ld32(tS + lane_off + sb * 64, sv);
-                tmem_ld32(tdP + lane_off + sb * 64, d0);
+                tmem_ld32(tS + lane_off + sb * 64 + ch * 32, sv);
+                tmem_ld32(tdP + lane_off + sb * 64 + ch * 32, d0);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const bool valid = live && (j < qb || hf * 64 + i <= r);
+                    const bool valid = live && (j < qb || hf * 64 + ch * 32 + i <= r);
                     d0[i] = valid ? ex2(sv[i] * p.scale_log2 - lse2) * (d0[i] - Dr) : 0.f;
-                }
-                tmem_ld32(tS + lane_off + sb * 64 + 32, sv);
-                tmem_ld32(tdP + lane_off + sb * 64 + 32, d1);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const bool valid = live && (j < qb || hf * 64 + 32 + i <= r);
-                    d1[i] = valid ? ex2(sv[i] * p.scale_log2 - lse2) * (d1[i] - Dr) : 0.f;
                 }
             }
             tc_fence_before();
@@ -466,8 +461,9 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
             if (t > 1 && !warp_wait(ds_done + 8 * sb, ((t >> 1) - 1) & 1, abort_flag, p.status)) { ok = false; break; }
             uint8_t* drow = smem + Lay::DS + sb * 16384 + r * 128;
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-                const float* v = c8 < 4 ? d0 + 8 * c8 : d1 + 8 * (c8 - 4);
+            for (int k = 0; k < 4; ++k) {
+                const float* v = d0 + 8 * k;
+                const int c8 = ch * 4 + k;
                 *reinterpret_cast<uint4*>(drow + ((c8 ^ (r & 7)) << 4)) =
                     make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
                                pack_bf16(v[6], v[7]));
@@ -480,7 +476,8 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
             tc_fence_after();
             bf16* out = p.dqkv + ((size_t)row0 + qpos) * Nqkv + h * HD;
 #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
+            for (int cc = 0; cc < HD / 64; ++cc) {
+                const int c = ch * (HD / 64) + cc;
                 float o[32];
                 tmem_ld32(tdQ + lane_off + c * 32, o);
                 if (live) {
@@ -510,6 +507,8 @@ __global__ void __launch_bounds__(NT, 1) attn_dq_tc_kernel(const __grid_constant
 // double-buffered TMEM; per key row (one per thread) P^T with the causal
 // mask and dS^T = P^T (dP^T - D) as bf16 into shared memory; dV += P^T dO and
 // dK += dS^T Q accumulate in TMEM over all units.  dk = dK / sqrt(hd).
+constexpr int DKV_STG = 3;  // Q/dO/lse/D stages of the dK/dV kernel
+
 template <int HD>
 struct DkvLayout {
     static constexpr int KB = HD / 64;
@@ -518,17 +517,18 @@ struct DkvLayout {
     static constexpr int K = 0;
     static constexpr int V = K + TILE;
     static constexpr int Q = V + TILE;
-    static constexpr int DO = Q + STG * HTILE;
-    static constexpr int PT = DO + STG * HTILE;   // [2][128 x 64] bf16, by unit parity
-    static constexpr int DST = PT + 2 * 16384;    // [2][128 x 64] bf16, by unit parity
-    static constexpr int LSE = DST + 2 * 16384;   // [STG][64] floats: lse of the unit's queries
-    static constexpr int DD = LSE + 512;      // [STG][64] floats: D of the unit's queries
-    static constexpr int BAR = DD + 512;
+    static constexpr int DO = Q + DKV_STG * HTILE;
+    static constexpr int PT = DO + DKV_STG * HTILE;  // [2][128 x 64] bf16, by unit parity
+    static constexpr int DST = PT + 2 * 16384;       // [2][128 x 64] bf16, by unit parity
+    static constexpr int LSE = DST + 2 * 16384;      // [DKV_STG][64] floats: lse of the unit's queries
+    static constexpr int DD = LSE + DKV_STG * 256;   // [DKV_STG][64] floats: D of the unit's queries
+    static constexpr int BAR = DD + DKV_STG * 256;
     static constexpr int BYTES = BAR + 256 + 1024;
+    static_assert(BYTES <= 232448, "dK/dV shared memory exceeds the per-block limit");
 };
 
 template <int HD>
-__global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmKV,
+__global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmKV,
                                                             const __grid_constant__ CUtensorMap tmQ64,
                                                             const __grid_constant__ CUtensorMap tmDO64,
                                                             const BwdParams p) {
@@ -543,10 +543,11 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
     float* d_s = reinterpret_cast<float*>(smem + Lay::DD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
-    const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24, st_full = b0 + 40, st_empty = b0 + 56;
+    const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 32;  // qo_*[DKV_STG]
+    const uint32_t st_full = b0 + 56, st_empty = b0 + 72;              // [2]
     // pd_done[b] completes after the dV/dK MMAs of the units with parity b
     // (once per two units), so a wait on it can never be lapped.
-    const uint32_t pd_full = b0 + 72, pd_done = b0 + 80;  // pd_done[2]
+    const uint32_t pd_full = b0 + 88, pd_done = b0 + 96;               // pd_done[2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -562,9 +563,9 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
-        for (int s = 0; s < STG; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(st_full + 8 * s, 1); mbar_init(st_empty + 8 * s, 4); }
-        mbar_init(pd_full, 4);
+        for (int s = 0; s < DKV_STG; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
+        for (int s = 0; s < 2; ++s) { mbar_init(st_full + 8 * s, 1); mbar_init(st_empty + 8 * s, 8); }
+        mbar_init(pd_full, 8);
         mbar_init(pd_done, 1);
         mbar_init(pd_done + 8, 1);
         *abort_flag = 0;
@@ -589,9 +590,9 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
             }
             int issued = 0;
             for (int u = 0; u < nunits; ++u) {
-                const int st = u % STG;
+                const int st = u % DKV_STG;
                 const int i = i0 + u / Hg, h = g * Hg + u % Hg;
-                if (!mbar_wait(qo_empty + 8 * st, ((u / STG) & 1) ^ 1, abort_flag, p.status)) break;
+                if (!mbar_wait(qo_empty + 8 * st, ((u / DKV_STG) & 1) ^ 1, abort_flag, p.status)) break;
                 mbar_expect_tx(qo_full + 8 * st, 2 * HTILE + 512);
                 const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + (size_t)i * 64;
                 bulk_load(base + Lay::LSE + st * 256, p.lse + si, 256, qo_full + 8 * st);
@@ -606,8 +607,8 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
             }
             if (*abort_flag) {
                 drain(kv_full, 0);
-                for (int u = (issued > STG ? issued - STG : 0); u < issued; ++u)
-                    drain(qo_full + 8 * (u % STG), (u / STG) & 1);
+                for (int u = (issued > DKV_STG ? issued - DKV_STG : 0); u < issued; ++u)
+                    drain(qo_full + 8 * (u % DKV_STG), (u / DKV_STG) & 1);
             }
         }
     } else if (warp == 1) {
@@ -617,8 +618,8 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
             if (mbar_wait(kv_full, 0, abort_flag, p.status)) {
                 for (int u = 0; u <= nunits; ++u) {
                     if (u < nunits) {
-                        const int st = u % STG, sb = u & 1;
-                        if (!mbar_wait(qo_full + 8 * st, (u / STG) & 1, abort_flag, p.status)) break;
+                        const int st = u % DKV_STG, sb = u & 1;
+                        if (!mbar_wait(qo_full + 8 * st, (u / DKV_STG) & 1, abort_flag, p.status)) break;
                         if (!mbar_wait(st_empty + 8 * sb, ((u >> 1) & 1) ^ 1, abort_flag, p.status)) break;
                         tc_fence_after();
 #pragma unroll
@@ -633,7 +634,7 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
                         mma_commit(st_full + 8 * sb);
                     }
                     if (u > 0) {
-                        const int uu = u - 1, st = uu % STG;
+                        const int uu = u - 1, st = uu % DKV_STG;
                         if (!mbar_wait(pd_full, uu & 1, abort_flag, p.status)) break;
                         tc_fence_after();
 #pragma unroll
@@ -653,22 +654,36 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
             }
         }
     } else {
-        const int q = warp & 3;
+        // warps 2..9: TMEM lane quarter q = warp % 4 (key rows), query half ch of each unit
+        const int q = warp & 3, ch = (warp - 2) >> 2;
         const int r = q * 32 + lane;
-        const int t = threadIdx.x - 64;  // 0..127
         const int kpos = kvb * 128 + r;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         bool ok = true;
         for (int u = 0; u < nunits; ++u) {
-            const int sb = u & 1, st = u % STG;
+            const int sb = u & 1, st = u % DKV_STG;
             const int i = i0 + u / Hg;
             if (!warp_wait(st_full + 8 * sb, (u >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             // this unit's Q/dO/lse/D stage has landed (the phase cannot move on
             // before this warp finishes the unit, which frees the stage)
-            if (!warp_wait(qo_full + 8 * st, (u / STG) & 1, abort_flag, p.status)) { ok = false; break; }
+            if (!warp_wait(qo_full + 8 * st, (u / DKV_STG) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
             const float* lse_u = lse_s + st * 64;
             const float* d_u = d_s + st * 64;
+            float sv[32], dp[32];
+            tmem_ld32(tSt + lane_off + sb * 64 + ch * 32, sv);
+            tmem_ld32(tdPt + lane_off + sb * 64 + ch * 32, dp);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(st_empty + 8 * sb);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int qc = ch * 32 + e, qpos = i * 64 + qc;
+                const bool valid = qpos >= kpos && qpos < p.T;
+                const float P = valid ? ex2(sv[e] * p.scale_log2 - lse_u[qc] * kLog2e) : 0.f;
+                dp[e] = valid ? P * (dp[e] - d_u[qc]) : 0.f;
+                sv[e] = P;
+            }
             // P^T / dS^T buffer (u & 1) was last read by the dV/dK MMAs of unit u-2
             if (u > 1 && !warp_wait(pd_done + 8 * (u & 1), ((u >> 1) - 1) & 1, abort_flag, p.status)) {
                 ok = false;
@@ -677,57 +692,39 @@ __global__ void __launch_bounds__(NT, 1) attn_dkv_tc_kernel(const __grid_constan
             uint8_t* prow = smem + Lay::PT + (u & 1) * 16384 + r * 128;
             uint8_t* drow = smem + Lay::DST + (u & 1) * 16384 + r * 128;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                float sv[32], dp[32];
-                tmem_ld32(tSt + lane_off + sb * 64 + c * 32, sv);
-                tmem_ld32(tdPt + lane_off + sb * 64 + c * 32, dp);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int qc = c * 32 + e, qpos = i * 64 + qc;
-                    const bool valid = qpos >= kpos && qpos < p.T;
-                    const float P = valid ? ex2(sv[e] * p.scale_log2 - lse_u[qc] * kLog2e) : 0.f;
-                    dp[e] = valid ? P * (dp[e] - d_u[qc]) : 0.f;
-                    sv[e] = P;
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int idx = c * 4 + k;
-                    const uint32_t sw = (uint32_t)((idx ^ (r & 7)) << 4);
-                    const float* a = sv + 8 * k;
-                    const float* d = dp + 8 * k;
-                    *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]),
-                                                                      pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
-                    *reinterpret_cast<uint4*>(drow + sw) = make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]),
-                                                                      pack_bf16(d[4], d[5]), pack_bf16(d[6], d[7]));
-                }
+            for (int k = 0; k < 4; ++k) {
+                const int idx = ch * 4 + k;
+                const uint32_t sw = (uint32_t)((idx ^ (r & 7)) << 4);
+                const float* a = sv + 8 * k;
+                const float* d = dp + 8 * k;
+                *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]),
+                                                                  pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
+                *reinterpret_cast<uint4*>(drow + sw) = make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]),
+                                                                  pack_bf16(d[4], d[5]), pack_bf16(d[6], d[7]));
             }
-            tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) { mbar_arrive(st_empty + 8 * sb); mbar_arrive(pd_full); }
+            if (lane == 0) mbar_arrive(pd_full);
         }
         if (ok && warp_wait(pd_done + 8 * ((nunits - 1) & 1), ((nunits - 1) >> 1) & 1, abort_flag, p.status)) {
             tc_fence_after();
             const bool live = kpos < p.T;
-            bf16* out_k = p.dqkv + ((size_t)row0 + kpos) * Nqkv + (p.H + g) * HD;
-            bf16* out_v = p.dqkv + ((size_t)row0 + kpos) * Nqkv + (p.H + p.nkv + g) * HD;
+            // the first four softmax warps write dV, the other four dK
+            bf16* out = p.dqkv + ((size_t)row0 + kpos) * Nqkv + (ch == 0 ? (p.H + p.nkv + g) : (p.H + g)) * HD;
+            const uint32_t tsrc = ch == 0 ? tdV : tdK;
+            const float sc = ch == 0 ? 1.f : p.scale;
 #pragma unroll
             for (int c = 0; c < HD / 32; ++c) {
-                float v[32], k[32];
-                tmem_ld32(tdV + lane_off + c * 32, v);
-                tmem_ld32(tdK + lane_off + c * 32, k);
+                float v[32];
+                tmem_ld32(tsrc + lane_off + c * 32, v);
                 if (live) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        *reinterpret_cast<uint4*>(out_v + c * 32 + 8 * e) =
-                            make_uint4(pack_bf16(v[8 * e], v[8 * e + 1]), pack_bf16(v[8 * e + 2], v[8 * e + 3]),
-                                       pack_bf16(v[8 * e + 4], v[8 * e + 5]), pack_bf16(v[8 * e + 6], v[8 * e + 7]));
-                        *reinterpret_cast<uint4*>(out_k + c * 32 + 8 * e) = make_uint4(
-                            pack_bf16(k[8 * e] * p.scale, k[8 * e + 1] * p.scale),
-                            pack_bf16(k[8 * e + 2] * p.scale, k[8 * e + 3] * p.scale),
-                            pack_bf16(k[8 * e + 4] * p.scale, k[8 * e + 5] * p.scale),
-                            pack_bf16(k[8 * e + 6] * p.scale, k[8 * e + 7] * p.scale));
-                    }
+                    for (int e = 0; e < 4; ++e)
+                        *reinterpret_cast<uint4*>(out + c * 32 + 8 * e) =
+                            make_uint4(pack_bf16(v[8 * e] * sc, v[8 * e + 1] * sc),
+                                       pack_bf16(v[8 * e + 2] * sc, v[8 * e + 3] * sc),
+                                       pack_bf16(v[8 * e + 4] * sc, v[8 * e + 5] * sc),
+                                       pack_bf16(v[8 * e + 6] * sc, v[8 * e + 7] * sc));
                 }
             }
         }
@@ -792,7 +789,7 @@ int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& 
             return -1;
         attr = true;
     }
-    attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NT, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
+    attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NTB, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -807,7 +804,7 @@ int dkv_launch(const CUtensorMap& kv, const CUtensorMap& q64, const CUtensorMap&
             return -1;
         attr = true;
     }
-    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NT, DkvLayout<HD>::BYTES, s>>>(kv, q64, do64, p);
+    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NTB, DkvLayout<HD>::BYTES, s>>>(kv, q64, do64, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

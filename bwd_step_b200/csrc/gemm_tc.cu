@@ -269,6 +269,152 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
 }
 
+
+// ------------------------------------------------------------------ CTA-pair kernel
+// Same roles, but a cluster of two CTAs computes a 256x256 output tile with
+// tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 rows of A and
+// 128 of the 256 B rows per 64-deep K slice (32 KB per stage instead of 48 KB
+// for the same work per SM), the even CTA issues the MMAs, which read both
+// CTAs' shared memory and write 128 rows into each CTA's TMEM.  Commits arrive
+// on the matching barriers of both CTAs; each epilogue reads its own TMEM and
+// signals the even CTA that the accumulator may be reused.
+constexpr int STAGES2 = 6;
+constexpr int STAGE2_BYTES = 2 * 128 * BK * 2;  // A 128x64 + B 128x64, bf16
+constexpr size_t SMEM2_BYTES = 1024 + (size_t)STAGES2 * STAGE2_BYTES + 256;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES2 * STAGE2_BYTES);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES2 + 4);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const uint32_t tiles_base = smem_u32(smem);
+    const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * STAGES2;
+    const uint32_t bar_tfull = bar_empty + 8 * STAGES2, bar_tempty = bar_tfull + 16;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES2; ++s) { mbar_init(bar_full + 8 * s, 1); mbar_init(bar_empty + 8 * s, 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(bar_tfull + 8 * b, 1); mbar_init(bar_tempty + 8 * b, 8); }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    if (warp == 0 && lane == 0) { tma_prefetch(&tmA); tma_prefetch(&tmB); }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised before any remote arrive
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs); bytes counted on the even CTA's barrier
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, issued_phase = 0;
+            bool ok = true;
+            for (int u = cluster; ok && u < p.num_units; u += nclusters) {
+                int tm, tn, ks;
+                decode(p, u, tm, tn, ks);
+                const int kb0 = ks * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                const int arow = tm * 256 + (int)rank * 128, brow = tn * BN + (int)rank * 128;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+                    const uint32_t fb = leader_addr(bar_full + 8 * stage);
+                    const uint32_t sa = tiles_base + stage * STAGE2_BYTES, sb = sa + 16384;
+                    if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * STAGE2_BYTES);
+                    if (!p.a_mn) {
+                        tma_load_2d_pair(sa, &tmA, kb * BK, arow, fb);
+                    } else {
+                        tma_load_2d_pair(sa, &tmA, arow, kb * BK, fb);
+                        tma_load_2d_pair(sa + 8192, &tmA, arow + 64, kb * BK, fb);
+                    }
+                    if (!p.b_mn) {
+                        tma_load_2d_pair(sb, &tmB, kb * BK, brow, fb);
+                    } else {
+                        tma_load_2d_pair(sb, &tmB, brow, kb * BK, fb);
+                        tma_load_2d_pair(sb + 8192, &tmB, brow + 64, kb * BK, fb);
+                    }
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES2) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok && rank == 0) {
+                for (int s = 0; s < STAGES2; ++s) {
+                    if (!(issued >> s & 1)) continue;
+                    uint64_t t0 = globaltimer();
+                    while (!mbar_try(bar_full + 8 * s, (issued_phase >> s) & 1) && globaltimer() - t0 < 1000000ull) {}
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer (even CTA only)
+            const uint32_t idesc = idesc_bf16(256, BN, p.a_mn != 0, p.b_mn != 0);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int u = cluster; ok && u < p.num_units; u += nclusters) {
+                int tm, tn, ks;
+                decode(p, u, tm, tn, ks);
+                const int kb0 = ks * p.kb_per_split, kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * BN;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = tiles_base + stage * STAGE2_BYTES, sb = sa + 16384;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const uint64_t ad = p.a_mn ? smem_desc(sa + k * 2048, 8192, 1024) : smem_desc(sa + k * 32, 16, 1024);
+                        const uint64_t bd = p.b_mn ? smem_desc(sb + k * 2048, 8192, 1024) : smem_desc(sb + k * 32, 16, 1024);
+                        mma_bf16_pair(d, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                    }
+                    mma_commit_pair(bar_empty + 8 * stage);
+                    if (++stage == STAGES2) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit_pair(bar_tfull + 8 * acc);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+            }
+        }
+    } else {
+        // ---------------- epilogue warps 2..5 of both CTAs
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = cluster; u < p.num_units; u += nclusters) {
+            int tm, tn, ks;
+            decode(p, u, tm, tn, ks);
+            if (!warp_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, p.status)) break;
+            tc_fence_after();
+            const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
+            const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+            for (int c = 0; c < BN / 32; ++c) {
+                const int n0 = tn * BN + c * 32;
+                if (n0 >= p.N) break;
+                float v[32];
+                tmem_ld32(tb + c * 32, v);
+                if (row < p.M) epilogue(p, ks, row, n0, v);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_addr(bar_tempty + 8 * acc));
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+    tc_fence_before();
+    cluster_sync();  // no CTA leaves while its pair may still signal or read it
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -325,14 +471,19 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
             return -1;
         attr_set = true;
     }
-    CUtensorMap ta, tb;
-    bool ok = g.a_kmajor ? make_map(&ta, g.A, g.K, g.M, g.lda, 64, BM) : make_map(&ta, g.A, g.M, g.K, g.lda, 64, 64);
-    ok = ok && (g.b_kmajor ? make_map(&tb, g.B, g.K, g.N, g.ldb, 64, BN) : make_map(&tb, g.B, g.N, g.K, g.ldb, 64, 64));
-    if (!ok) return 1;
+    static bool attr2_set = false;
+    if (!attr2_set) {
+        if (cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_BYTES) !=
+            cudaSuccess)
+            return -1;
+        attr2_set = true;
+    }
 
+    // CTA pairs (256x256 tiles) when there are at least 256 rows
+    const bool pair = g.M >= 256;
     TcParams p{};
     p.M = g.M; p.N = g.N; p.K = g.K;
-    p.tiles_m = (g.M + BM - 1) / BM;
+    p.tiles_m = pair ? (g.M + 255) / 256 : (g.M + BM - 1) / BM;
     p.tiles_n = (g.N + BN - 1) / BN;
     p.num_kb = (g.K + BK - 1) / BK;
     p.tn_fast = p.tiles_n <= p.tiles_m ? 1 : 0;
@@ -349,8 +500,15 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     if (g.epi == EPI_RELU2) vec = vec && al16(g.C2) && (g.ldc2 * 2) % 16 == 0;
     if (g.epi == EPI_RELU2_BWD) vec = vec && al16(g.aux) && (g.ldaux * 2) % 16 == 0;
 
-    // split-K when the output tiles cannot fill the SMs
-    const int sms = num_sms();
+    CUtensorMap ta, tb;
+    const uint32_t brows = pair ? 128 : BN;  // B rows per CTA per K slice
+    bool ok = g.a_kmajor ? make_map(&ta, g.A, g.K, g.M, g.lda, 64, BM) : make_map(&ta, g.A, g.M, g.K, g.lda, 64, 64);
+    ok = ok && (g.b_kmajor ? make_map(&tb, g.B, g.K, g.N, g.ldb, 64, brows)
+                           : make_map(&tb, g.B, g.N, g.K, g.ldb, 64, 64));
+    if (!ok) return 1;
+
+    // split-K when the output tiles cannot fill the SMs (a pair counts as one unit of two SMs)
+    const int sms = pair ? num_sms() / 2 : num_sms();
     const int tiles = p.tiles_m * p.tiles_n;
     int splits = 1;
     const bool can_split = (g.epi == EPI_STORE || g.epi == EPI_ACCUM) && !p.c_bf16 && g.ldc == g.N && splitk &&
@@ -370,7 +528,8 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     p.vec_ok = (p.part ? (g.N % 4 == 0) : vec) ? 1 : 0;
     p.num_units = tiles * p.splits;
     const int grid = std::min(p.num_units, sms);
-    gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    if (pair) gemm_tc2_kernel<<<2 * grid, NTHREADS, SMEM2_BYTES, s>>>(ta, tb, p);
+    else gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, p);
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return -1;
     if (p.part) {
