@@ -304,7 +304,63 @@ struct BwdParams {
     const float* D;
     bf16* dqkv;
     int* status;
+    // When rqk is set, dq and dk are written as gradients of the pre-norm
+    // projections (QK-norm and RoPE backward fused): qkv holds the saved
+    // post-RoPE vectors, rqk their inverse RMS [B*T, H+nkv], cos/sin [T, hd/2].
+    const bf16* qkv;
+    const float* rqk;
+    const float* cos_t;
+    const float* sin_t;
 };
+
+// Writes the gradient of the pre-norm projection for one head row: g = scale *
+// (the TMEM row at tsrc) is the gradient of y = rope(rmsnorm(x)); with the
+// saved y, u = R^T g and w = R^T y (inverse rotation of the pairs (j, j+HD/2))
+// give dx = r * (u - w * mean(u * w)).  Two passes over TMEM keep registers low.
+template <int HD>
+__device__ __forceinline__ void store_grad_through_qknorm(uint32_t tsrc, float scale, const bf16* y, float r,
+                                                          const float* cs, const float* sn, bf16* out, bool live) {
+    constexpr int NC = HD / 32, HALF = HD / 2;
+    float dot = 0.f;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const float mdot = dot / (float)HD;
+#pragma unroll 1
+        for (int c = 0; c < NC / 2; ++c) {
+            float g1[32], g2[32];
+            tmem_ld32(tsrc + c * 32, g1);
+            tmem_ld32(tsrc + (c + NC / 2) * 32, g2);
+            if (!live) continue;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+                float y1[8], y2[8];
+                load_vec(y + c * 32 + i, y1);
+                load_vec(y + HALF + c * 32 + i, y2);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int j = c * 32 + i + e;
+                    const float co = cs[j], si = sn[j];
+                    const float a = g1[i + e] * scale, b = g2[i + e] * scale;
+                    const float u1 = a * co + b * si, u2 = b * co - a * si;
+                    const float w1 = y1[e] * co + y2[e] * si, w2 = y2[e] * co - y1[e] * si;
+                    if (pass == 0) {
+                        dot += u1 * w1 + u2 * w2;
+                    } else {
+                        g1[i + e] = r * (u1 - w1 * mdot);
+                        g2[i + e] = r * (u2 - w2 * mdot);
+                    }
+                }
+            }
+            if (pass == 1) {
+#pragma unroll
+                for (int t4 = 0; t4 < 4; ++t4) {
+                    store_vec(out + c * 32 + 8 * t4, g1 + 8 * t4);
+                    store_vec(out + HALF + c * 32 + 8 * t4, g2 + 8 * t4);
+                }
+            }
+        }
+    }
+}
 
 __device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
     uint64_t t0 = globaltimer();
@@ -475,6 +531,17 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
         if (ok && warp_wait(ds_done + 8 * ((nsub - 1) & 1), ((nsub - 1) >> 1) & 1, abort_flag, p.status)) {
             tc_fence_after();
             bf16* out = p.dqkv + ((size_t)row0 + qpos) * Nqkv + h * HD;
+            if (p.rqk) {
+                // the first four softmax warps write whole rows through the QK-norm backward
+                if (ch == 0) {
+                    const size_t rowi = (size_t)row0 + (live ? qpos : 0);
+                    const int pos = live ? qpos : 0;
+                    store_grad_through_qknorm<HD>(tdQ + lane_off, p.scale, p.qkv + rowi * Nqkv + h * HD,
+                                                  live ? p.rqk[rowi * (p.H + p.nkv) + h] : 0.f,
+                                                  p.cos_t + (size_t)pos * (HD / 2), p.sin_t + (size_t)pos * (HD / 2),
+                                                  out, live);
+                }
+            } else
 #pragma unroll
             for (int cc = 0; cc < HD / 64; ++cc) {
                 const int c = ch * (HD / 64) + cc;
@@ -709,6 +776,16 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         if (ok && warp_wait(pd_done + 8 * ((nunits - 1) & 1), ((nunits - 1) >> 1) & 1, abort_flag, p.status)) {
             tc_fence_after();
             const bool live = kpos < p.T;
+            if (p.rqk && ch == 1) {
+                // dK through the QK-norm backward (the other four warps write dV below)
+                const size_t rowi = (size_t)row0 + (live ? kpos : 0);
+                const int pos = live ? kpos : 0;
+                bf16* outk = p.dqkv + rowi * Nqkv + (p.H + g) * HD;
+                store_grad_through_qknorm<HD>(tdK + lane_off, p.scale, p.qkv + rowi * Nqkv + (p.H + g) * HD,
+                                              live ? p.rqk[rowi * (p.H + p.nkv) + p.H + g] : 0.f,
+                                              p.cos_t + (size_t)pos * (HD / 2), p.sin_t + (size_t)pos * (HD / 2),
+                                              outk, live);
+            } else {
             // the first four softmax warps write dV, the other four dK
             bf16* out = p.dqkv + ((size_t)row0 + kpos) * Nqkv + (ch == 0 ? (p.H + p.nkv + g) : (p.H + g)) * HD;
             const uint32_t tsrc = ch == 0 ? tdV : tdK;
@@ -726,6 +803,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                                        pack_bf16(v[8 * e + 4] * sc, v[8 * e + 5] * sc),
                                        pack_bf16(v[8 * e + 6] * sc, v[8 * e + 7] * sc));
                 }
+            }
             }
         }
     }
@@ -811,7 +889,7 @@ int dkv_launch(const CUtensorMap& kv, const CUtensorMap& q64, const CUtensorMap&
 
 BwdParams bwd_params(const float* lse, const float* Dbuf, void* dqkv, int B, int T, int H, int nkv, int hd,
                      int* status) {
-    BwdParams p;
+    BwdParams p{};
     p.B = B; p.T = T; p.H = H; p.nkv = nkv; p.nqb = (T + 127) / 128;
     p.scale = 1.f / sqrtf((float)hd);
     p.scale_log2 = kLog2e * p.scale;
@@ -842,7 +920,7 @@ int attention_tc_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, 
 bool attention_tc_bwd_supported(int hd) { return hd == 64 || hd == 128; }
 
 int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
-                        int B, int T, int H, int nkv, int hd, int* status, cudaStream_t s) {
+                        int B, int T, int H, int nkv, int hd, int* status, cudaStream_t s, const QkNormFuse* fuse) {
     if (!attention_tc_bwd_supported(hd)) return 1;
     if (!aligned16(qkv) || !aligned16(o) || !aligned16(dO) || !aligned16(dqkv) || B > 65535 || H > 65535) return 1;
     const int Nqkv = (H + 2 * nkv) * hd;
@@ -851,11 +929,15 @@ int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const fl
         return 1;
     if (launch_attention_bwd_dot(DT_BF16, o, dO, Dbuf, B, T, H, hd, s) != cudaSuccess) return -1;
     BwdParams p = bwd_params(lse, Dbuf, dqkv, B, T, H, nkv, hd, status);
+    if (fuse) {
+        p.qkv = reinterpret_cast<const bf16*>(qkv);
+        p.rqk = fuse->rqk; p.cos_t = fuse->cos_t; p.sin_t = fuse->sin_t;
+    }
     return hd == 128 ? dq_launch<128>(kv, do128, p, s) : dq_launch<64>(kv, do128, p, s);
 }
 
 int attention_tc_bwd_dkv(const void* qkv, const void* dO, const float* lse, const float* Dbuf, void* dqkv, int B,
-                         int T, int H, int nkv, int hd, int* status, cudaStream_t s) {
+                         int T, int H, int nkv, int hd, int* status, cudaStream_t s, const QkNormFuse* fuse) {
     if (!attention_tc_bwd_supported(hd)) return 1;
     if (!aligned16(qkv) || !aligned16(dO) || !aligned16(dqkv) || B > 65535 || nkv > 65535) return 1;
     const int Nqkv = (H + 2 * nkv) * hd;
@@ -864,14 +946,18 @@ int attention_tc_bwd_dkv(const void* qkv, const void* dO, const float* lse, cons
         !map_rows(&do64, dO, (uint64_t)H * hd, (uint64_t)B * T, 64))
         return 1;
     BwdParams p = bwd_params(lse, Dbuf, dqkv, B, T, H, nkv, hd, status);
+    if (fuse) {
+        p.qkv = reinterpret_cast<const bf16*>(qkv);
+        p.rqk = fuse->rqk; p.cos_t = fuse->cos_t; p.sin_t = fuse->sin_t;
+    }
     return hd == 128 ? dkv_launch<128>(kv, q64, do64, p, s) : dkv_launch<64>(kv, q64, do64, p, s);
 }
 
 int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
                      int B, int T, int H, int nkv, int hd, void*, size_t, int* status, cudaStream_t s) {
-    int r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s);
+    int r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s, nullptr);
     if (r != 0) return r;
-    return attention_tc_bwd_dkv(qkv, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s);
+    return attention_tc_bwd_dkv(qkv, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s, nullptr);
 }
 
 size_t attention_tc_workspace_bytes(int, int, int, int, int) { return 0; }

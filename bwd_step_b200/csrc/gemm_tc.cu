@@ -44,6 +44,10 @@ struct TcParams {
     float cap;
     float* part;  // split-K partial sums [splits][M][N], or null
     int* status;
+    int hd, T, qk_heads;
+    float* rqk;
+    const float* cos_t;
+    const float* sin_t;
 };
 
 __device__ __forceinline__ void decode(const TcParams& p, int u, int& tm, int& tn, int& ks) {
@@ -135,6 +139,68 @@ __device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int
             for (int i = 0; i < 32; ++i) v[i] = p.cap * tanhf(v[i] * ic);
             store_row(p.C, p.c_bf16, off, v, nv, vec);
         } break;
+    }
+}
+
+// Fused QK-norm + RoPE epilogue over one 256-column tile of the qkv
+// projection (nanochat announcement, vpshk.cn, architecture list: rotary
+// embeddings, QK norm): every head of HD columns is loaded whole from TMEM,
+// normalised by its RMS (no parameters), rotated pair-wise (j, j + HD/2) by the
+// row's position, and stored as bf16; value heads are stored unchanged.
+template <int HD>
+__device__ __forceinline__ void epilogue_qkrope(const TcParams& p, int row, int n_tile, uint32_t tb) {
+    constexpr int NC = HD / 32, HALF = HD / 2;
+    const bool live = row < p.M;
+    const int pos = live ? row % p.T : 0;
+    const float* cs = p.cos_t + (size_t)pos * HALF;
+    const float* sn = p.sin_t + (size_t)pos * HALF;
+    bf16* crow = reinterpret_cast<bf16*>(p.C) + (int64_t)row * p.ldc;
+    for (int h0 = 0; h0 < BN; h0 += HD) {
+        const int col = n_tile + h0;
+        if (col >= p.N) break;
+        const int head = col / HD;
+        if (head >= p.qk_heads) {  // value head: plain store
+#pragma unroll 1
+            for (int c = 0; c < NC; ++c) {
+                float v[32];
+                tmem_ld32(tb + h0 + c * 32, v);
+                if (live) store_row_bf16(crow + col + c * 32, v, 32, true);
+            }
+            continue;
+        }
+        // pass 1: sum of squares of the head vector
+        float ss = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+            float v[32];
+            tmem_ld32(tb + h0 + c * 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ss += v[i] * v[i];
+        }
+        const float r = rsqrtf(ss / (float)HD + kRmsEps);
+        if (live) p.rqk[(size_t)row * p.qk_heads + head] = r;
+        // pass 2: rotate the pairs (j, j + HD/2), chunk c with chunk c + NC/2
+#pragma unroll 1
+        for (int c = 0; c < NC / 2; ++c) {
+            float x1[32], x2[32];
+            tmem_ld32(tb + h0 + c * 32, x1);
+            tmem_ld32(tb + h0 + (c + NC / 2) * 32, x2);
+            if (!live) continue;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const float4 c4 = *reinterpret_cast<const float4*>(cs + c * 32 + i);
+                const float4 s4 = *reinterpret_cast<const float4*>(sn + c * 32 + i);
+                const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, ssn[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a = x1[i + e] * r, b = x2[i + e] * r;
+                    x1[i + e] = a * cc[e] - b * ssn[e];
+                    x2[i + e] = a * ssn[e] + b * cc[e];
+                }
+            }
+            store_row_bf16(crow + col + c * 32, x1, 32, true);
+            store_row_bf16(crow + col + (c + NC / 2) * 32, x2, 32, true);
+        }
     }
 }
 
@@ -248,12 +314,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tc_fence_after();
             const int row = tm * BM + q * 32 + lane;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-            for (int c = 0; c < BN / 32; ++c) {
-                const int n0 = tn * BN + c * 32;
-                if (n0 >= p.N) break;
-                float v[32];
-                tmem_ld32(tb + c * 32, v);
-                if (row < p.M) epilogue(p, ks, row, n0, v);
+            if (p.epi == EPI_QKROPE) {
+                if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
+                else epilogue_qkrope<64>(p, row, tn * BN, tb);
+            } else {
+                for (int c = 0; c < BN / 32; ++c) {
+                    const int n0 = tn * BN + c * 32;
+                    if (n0 >= p.N) break;
+                    float v[32];
+                    tmem_ld32(tb + c * 32, v);
+                    if (row < p.M) epilogue(p, ks, row, n0, v);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -394,12 +465,17 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             tc_fence_after();
             const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-            for (int c = 0; c < BN / 32; ++c) {
-                const int n0 = tn * BN + c * 32;
-                if (n0 >= p.N) break;
-                float v[32];
-                tmem_ld32(tb + c * 32, v);
-                if (row < p.M) epilogue(p, ks, row, n0, v);
+            if (p.epi == EPI_QKROPE) {
+                if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
+                else epilogue_qkrope<64>(p, row, tn * BN, tb);
+            } else {
+                for (int c = 0; c < BN / 32; ++c) {
+                    const int n0 = tn * BN + c * 32;
+                    if (n0 >= p.N) break;
+                    float v[32];
+                    tmem_ld32(tb + c * 32, v);
+                    if (row < p.M) epilogue(p, ks, row, n0, v);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -461,6 +537,10 @@ size_t gemm_tc_splitk_bytes(size_t max_out_elems) { return (size_t)MAX_SPLITS * 
 
 int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s) {
     if (g.in_t != DT_BF16) return 1;
+    if (g.epi == EPI_QKROPE &&
+        ((g.hd != 64 && g.hd != 128) || g.c_t != DT_BF16 || g.T <= 0 || !g.rqk || !g.cos_t || !g.sin_t ||
+         (reinterpret_cast<uintptr_t>(g.C) & 15) || (g.ldc % 8) || (g.N % g.hd)))
+        return 1;
     if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 1;
     auto al16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
     if (!al16(g.A) || !al16(g.B) || (g.lda * 2) % 16 || (g.ldb * 2) % 16) return 1;
@@ -495,6 +575,8 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     p.aux = reinterpret_cast<const bf16*>(g.aux); p.ldaux = g.ldaux;
     p.cap = g.cap;
     p.status = g.status;
+    p.hd = g.hd; p.T = g.T; p.qk_heads = g.qk_heads;
+    p.rqk = g.rqk; p.cos_t = g.cos_t; p.sin_t = g.sin_t;
     const int esz = p.c_bf16 ? 2 : 4;
     bool vec = al16(g.C) && (g.ldc * esz) % 16 == 0;
     if (g.epi == EPI_RELU2) vec = vec && al16(g.C2) && (g.ldc2 * 2) % 16 == 0;

@@ -78,6 +78,9 @@ enum Epi : int {
     EPI_RELU2 = 2,      // C = relu(acc)^2, C2 = relu(acc) (activation type)
     EPI_RELU2_BWD = 3,  // C = acc * 2 * aux               (aux = relu(u), activation type)
     EPI_SOFTCAP = 4,    // C = cap * tanh(acc / cap)       (C fp32 or activation type)
+    EPI_QKROPE = 5,     // fused qkv rows: per head of the first qk_heads heads,
+                        // C = rope(rmsnorm_hd(acc)) and rqk = its inverse RMS; other
+                        // columns (v) C = acc.  bf16 C, head_dim 64 or 128 (tcgen05 only)
 };
 
 struct GemmDesc {
@@ -91,6 +94,12 @@ struct GemmDesc {
     const void* aux = nullptr; int64_t ldaux = 0;
     float cap = 0.f;
     int* status = nullptr;  // device status word for bounded-wait timeouts
+    // EPI_QKROPE: head_dim, sequence length (position = row % T), number of
+    // normalised heads (H + n_kv), their inverse RMS [M, qk_heads], RoPE tables [T, hd/2]
+    int hd = 0, T = 0, qk_heads = 0;
+    float* rqk = nullptr;
+    const float* cos_t = nullptr;
+    const float* sin_t = nullptr;
 };
 
 // Plain fp32-FMA tiled GEMM (any strides, any sizes).

@@ -165,79 +165,132 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const A* __rest
 }
 
 // ---------------------------------------------------------------- QK-norm + RoPE
-// A group of G lanes (G = min(32, hd/2)) owns one head vector; lane li holds
-// the pairs (j, j + hd/2) for j = li + p*G.
-template <typename A>
-__global__ void qknorm_rope_fwd_kernel(A* qkv, float* __restrict__ rqk, const float* __restrict__ cos_t,
-                                       const float* __restrict__ sin_t, int M, int T, int H, int nkv,
-                                       int hd, int G) {
-    int t = blockIdx.x * blockDim.x + threadIdx.x;
-    int nh = H + nkv;
-    int vi = t / G, li = t % G;
-    bool active = vi < M * nh;
-    int m = active ? vi / nh : 0, head = active ? vi % nh : 0;
-    int pos = m % T, half = hd >> 1, P = half / G;
-    A* v = qkv + (size_t)m * (size_t)(H + 2 * nkv) * hd + (size_t)head * hd;
-    float x1[2] = {0.f, 0.f}, x2[2] = {0.f, 0.f};
-    float ss = 0.f;
-    if (active) {
-        for (int p = 0; p < P; ++p) {
-            int j = li + p * G;
-            x1[p] = tof(v[j]);
-            x2[p] = tof(v[j + half]);
-            ss += x1[p] * x1[p] + x2[p] * x2[p];
-        }
+// One warp per (token, head) vector of HD elements.  Lane l holds EPL = HD/32
+// consecutive elements (HD = 16: lanes 0..15 one each); the pair partner of
+// element j < HD/2 is element j + HD/2, held by lane l ^ (HD/2/EPL).  Every
+// access is a contiguous EPL-element vector, so a warp reads and writes each
+// head vector in one coalesced request.
+template <int HD> struct QkShape {
+    static constexpr int EPL = HD >= 32 ? HD / 32 : 1;       // elements per lane
+    static constexpr int LANES = HD / EPL;                    // active lanes
+    static constexpr int XOR = (HD / 2) / EPL;                // partner lane offset
+};
+
+// N-element vector access (N*sizeof(A) bytes, naturally aligned here).
+template <typename A, int N>
+__device__ __forceinline__ void ldN(const A* p, float* v) {
+    if constexpr (sizeof(A) == 2 && N == 4) {
+        uint2 u = *reinterpret_cast<const uint2*>(p);
+        float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+        float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+    } else if constexpr (sizeof(A) == 2 && N == 2) {
+        float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+        v[0] = a.x; v[1] = a.y;
+    } else if constexpr (sizeof(A) == 4 && N == 4) {
+        float4 a = *reinterpret_cast<const float4*>(p);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else if constexpr (sizeof(A) == 4 && N == 2) {
+        float2 a = *reinterpret_cast<const float2*>(p);
+        v[0] = a.x; v[1] = a.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i] = tof(p[i]);
     }
-    for (int o = G >> 1; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (!active) return;
-    float r = rsqrtf(ss / (float)hd + kRmsEps);
-    for (int p = 0; p < P; ++p) {
-        int j = li + p * G;
-        float c = cos_t[pos * half + j], s = sin_t[pos * half + j];
-        float a = x1[p] * r, b = x2[p] * r;
-        v[j] = fromf<A>(a * c - b * s);
-        v[j + half] = fromf<A>(a * s + b * c);
+}
+template <typename A, int N>
+__device__ __forceinline__ void stN(A* p, const float* v) {
+    if constexpr (sizeof(A) == 2 && N == 4) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t*>(&a);
+        u.y = *reinterpret_cast<uint32_t*>(&b);
+        *reinterpret_cast<uint2*>(p) = u;
+    } else if constexpr (sizeof(A) == 2 && N == 2) {
+        *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
+    } else if constexpr (sizeof(A) == 4 && N == 4) {
+        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (sizeof(A) == 4 && N == 2) {
+        *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) p[i] = fromf<A>(v[i]);
     }
-    if (li == 0) rqk[(size_t)m * nh + head] = r;
 }
 
-template <typename A>
-__global__ void qknorm_rope_bwd_kernel(A* dqkv, const A* __restrict__ qkv, const float* __restrict__ rqk,
-                                       const float* __restrict__ cos_t, const float* __restrict__ sin_t,
-                                       int M, int T, int H, int nkv, int hd, int G) {
-    int t = blockIdx.x * blockDim.x + threadIdx.x;
-    int nh = H + nkv;
-    int vi = t / G, li = t % G;
-    bool active = vi < M * nh;
-    int m = active ? vi / nh : 0, head = active ? vi % nh : 0;
-    int pos = m % T, half = hd >> 1, P = half / G;
-    size_t off = (size_t)m * (size_t)(H + 2 * nkv) * hd + (size_t)head * hd;
-    A* g = dqkv + off;
-    const A* y = qkv + off;
-    float g1[2] = {0.f, 0.f}, g2[2] = {0.f, 0.f}, y1[2] = {0.f, 0.f}, y2[2] = {0.f, 0.f};
-    float dot = 0.f;
-    if (active) {
-        for (int p = 0; p < P; ++p) {
-            int j = li + p * G;
-            float c = cos_t[pos * half + j], s = sin_t[pos * half + j];
-            float a = tof(g[j]), b = tof(g[j + half]);
-            g1[p] = a * c + b * s;       // inverse rotation of the gradient
-            g2[p] = -a * s + b * c;
-            float u = tof(y[j]), w = tof(y[j + half]);
-            y1[p] = u * c + w * s;       // normalised vector before rotation
-            y2[p] = -u * s + w * c;
-            dot += g1[p] * y1[p] + g2[p] * y2[p];
-        }
+template <typename A, int HD>
+__global__ void __launch_bounds__(256) qknorm_rope_fwd_kernel(A* qkv, float* __restrict__ rqk,
+                                                              const float* __restrict__ cos_t,
+                                                              const float* __restrict__ sin_t, int M, int T, int H,
+                                                              int nkv) {
+    using S = QkShape<HD>;
+    const int nh = H + nkv;
+    const int vi = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (vi >= M * nh) return;
+    const int m = vi / nh, head = vi % nh, pos = m % T;
+    const bool act = lane < S::LANES;
+    const int l = act ? lane : 0;
+    A* v = qkv + (size_t)m * (size_t)(H + 2 * nkv) * HD + (size_t)head * HD + l * S::EPL;
+    float x[S::EPL];
+    ldN<A, S::EPL>(v, x);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < S::EPL; ++i) ss += act ? x[i] * x[i] : 0.f;
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)HD + kRmsEps);
+    const bool first = l * S::EPL < HD / 2;                   // holds x1 of its pairs
+    const int j0 = first ? l * S::EPL : l * S::EPL - HD / 2;   // pair index of element 0
+    float y[S::EPL];
+#pragma unroll
+    for (int i = 0; i < S::EPL; ++i) {
+        const float other = __shfl_xor_sync(0xffffffffu, x[i], S::XOR);
+        const float c = cos_t[pos * (HD / 2) + j0 + i], s = sin_t[pos * (HD / 2) + j0 + i];
+        const float a = (first ? x[i] : other) * r, b = (first ? other : x[i]) * r;
+        y[i] = first ? a * c - b * s : a * s + b * c;
     }
-    for (int o = G >> 1; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (!active) return;
-    dot /= (float)hd;
-    float r = rqk[(size_t)m * nh + head];
-    for (int p = 0; p < P; ++p) {
-        int j = li + p * G;
-        g[j] = fromf<A>(r * (g1[p] - y1[p] * dot));
-        g[j + half] = fromf<A>(r * (g2[p] - y2[p] * dot));
+    if (!act) return;
+    stN<A, S::EPL>(v, y);
+    if (lane == 0) rqk[(size_t)m * nh + head] = r;
+}
+
+template <typename A, int HD>
+__global__ void __launch_bounds__(256) qknorm_rope_bwd_kernel(A* dqkv, const A* __restrict__ qkv,
+                                                              const float* __restrict__ rqk,
+                                                              const float* __restrict__ cos_t,
+                                                              const float* __restrict__ sin_t, int M, int T, int H,
+                                                              int nkv) {
+    using S = QkShape<HD>;
+    const int nh = H + nkv;
+    const int vi = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (vi >= M * nh) return;
+    const int m = vi / nh, head = vi % nh, pos = m % T;
+    const bool act = lane < S::LANES;
+    const int l = act ? lane : 0;
+    const size_t off = (size_t)m * (size_t)(H + 2 * nkv) * HD + (size_t)head * HD + l * S::EPL;
+    float g[S::EPL], y[S::EPL];
+    ldN<A, S::EPL>(dqkv + off, g);
+    ldN<A, S::EPL>(qkv + off, y);
+    const bool first = l * S::EPL < HD / 2;
+    const int j0 = first ? l * S::EPL : l * S::EPL - HD / 2;
+    float gu[S::EPL], yu[S::EPL], dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < S::EPL; ++i) {
+        const float go = __shfl_xor_sync(0xffffffffu, g[i], S::XOR);
+        const float yo = __shfl_xor_sync(0xffffffffu, y[i], S::XOR);
+        const float c = cos_t[pos * (HD / 2) + j0 + i], s = sin_t[pos * (HD / 2) + j0 + i];
+        // inverse rotation of (x1, x2): (x1 c + x2 s, -x1 s + x2 c)
+        const float g1 = first ? g[i] : go, g2 = first ? go : g[i];
+        const float y1 = first ? y[i] : yo, y2 = first ? yo : y[i];
+        gu[i] = first ? g1 * c + g2 * s : -g1 * s + g2 * c;
+        yu[i] = first ? y1 * c + y2 * s : -y1 * s + y2 * c;
+        dot += act ? gu[i] * yu[i] : 0.f;
     }
+    dot = warp_sum(dot) / (float)HD;
+    if (!act) return;
+    const float r = rqk[(size_t)m * nh + head];
+#pragma unroll
+    for (int i = 0; i < S::EPL; ++i) gu[i] = r * (gu[i] - yu[i] * dot);
+    stN<A, S::EPL>(dqkv + off, gu);
 }
 
 // ---------------------------------------------------------------- cross-entropy
@@ -564,34 +617,57 @@ cudaError_t launch_embed_norm_bwd(DType wt, const float* dx, const int32_t* idx,
     return cudaGetLastError();
 }
 
-static inline int qk_group(int hd) { return hd / 2 < 32 ? hd / 2 : 32; }
+template <typename A, int HD>
+static void qk_fwd_t(void* qkv, float* rqk, const float* c, const float* sn, int M, int T, int H, int nkv,
+                     cudaStream_t s) {
+    const long long vecs = (long long)M * (H + nkv);
+    qknorm_rope_fwd_kernel<A, HD><<<(unsigned)((vecs + 7) / 8), 256, 0, s>>>((A*)qkv, rqk, c, sn, M, T, H, nkv);
+}
+template <typename A, int HD>
+static void qk_bwd_t(void* dqkv, const void* qkv, const float* rqk, const float* c, const float* sn, int M, int T,
+                     int H, int nkv, cudaStream_t s) {
+    const long long vecs = (long long)M * (H + nkv);
+    qknorm_rope_bwd_kernel<A, HD><<<(unsigned)((vecs + 7) / 8), 256, 0, s>>>((A*)dqkv, (const A*)qkv, rqk, c, sn, M,
+                                                                              T, H, nkv);
+}
 
-cudaError_t launch_qknorm_rope_fwd(DType at, void* qkv, float* rqk, const float* c, const float* sn, int M,
-                                   int T, int H, int nkv, int hd, cudaStream_t s) {
-    int G = qk_group(hd);
-    long long threads = (long long)M * (H + nkv) * G;
-    int blocks = (int)((threads + 255) / 256);
-    if (at == DT_BF16)
-        qknorm_rope_fwd_kernel<bf16><<<blocks, 256, 0, s>>>((bf16*)qkv, rqk, c, sn, M, T, H, nkv, hd, G);
-    else
-        qknorm_rope_fwd_kernel<float><<<blocks, 256, 0, s>>>((float*)qkv, rqk, c, sn, M, T, H, nkv, hd, G);
+template <typename A>
+static cudaError_t qk_fwd_d(void* qkv, float* rqk, const float* c, const float* sn, int M, int T, int H, int nkv,
+                            int hd, cudaStream_t s) {
+    switch (hd) {
+        case 16: qk_fwd_t<A, 16>(qkv, rqk, c, sn, M, T, H, nkv, s); break;
+        case 32: qk_fwd_t<A, 32>(qkv, rqk, c, sn, M, T, H, nkv, s); break;
+        case 64: qk_fwd_t<A, 64>(qkv, rqk, c, sn, M, T, H, nkv, s); break;
+        case 128: qk_fwd_t<A, 128>(qkv, rqk, c, sn, M, T, H, nkv, s); break;
+        default: return cudaErrorInvalidValue;
+    }
+    count_launch();
+    return cudaGetLastError();
+}
+template <typename A>
+static cudaError_t qk_bwd_d(void* dqkv, const void* qkv, const float* rqk, const float* c, const float* sn, int M,
+                            int T, int H, int nkv, int hd, cudaStream_t s) {
+    switch (hd) {
+        case 16: qk_bwd_t<A, 16>(dqkv, qkv, rqk, c, sn, M, T, H, nkv, s); break;
+        case 32: qk_bwd_t<A, 32>(dqkv, qkv, rqk, c, sn, M, T, H, nkv, s); break;
+        case 64: qk_bwd_t<A, 64>(dqkv, qkv, rqk, c, sn, M, T, H, nkv, s); break;
+        case 128: qk_bwd_t<A, 128>(dqkv, qkv, rqk, c, sn, M, T, H, nkv, s); break;
+        default: return cudaErrorInvalidValue;
+    }
     count_launch();
     return cudaGetLastError();
 }
 
+cudaError_t launch_qknorm_rope_fwd(DType at, void* qkv, float* rqk, const float* c, const float* sn, int M,
+                                   int T, int H, int nkv, int hd, cudaStream_t s) {
+    return at == DT_BF16 ? qk_fwd_d<bf16>(qkv, rqk, c, sn, M, T, H, nkv, hd, s)
+                         : qk_fwd_d<float>(qkv, rqk, c, sn, M, T, H, nkv, hd, s);
+}
+
 cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const float* rqk, const float* c,
                                    const float* sn, int M, int T, int H, int nkv, int hd, cudaStream_t s) {
-    int G = qk_group(hd);
-    long long threads = (long long)M * (H + nkv) * G;
-    int blocks = (int)((threads + 255) / 256);
-    if (at == DT_BF16)
-        qknorm_rope_bwd_kernel<bf16><<<blocks, 256, 0, s>>>((bf16*)dqkv, (const bf16*)qkv, rqk, c, sn, M, T, H,
-                                                            nkv, hd, G);
-    else
-        qknorm_rope_bwd_kernel<float><<<blocks, 256, 0, s>>>((float*)dqkv, (const float*)qkv, rqk, c, sn, M, T,
-                                                             H, nkv, hd, G);
-    count_launch();
-    return cudaGetLastError();
+    return at == DT_BF16 ? qk_bwd_d<bf16>(dqkv, qkv, rqk, c, sn, M, T, H, nkv, hd, s)
+                         : qk_bwd_d<float>(dqkv, qkv, rqk, c, sn, M, T, H, nkv, hd, s);
 }
 
 cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R, int V, float cap, float inv_M,

@@ -209,20 +209,30 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
     return NC_OK;
 }
 
-int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv) {
+// Attention backward.  With rqk set and the tensor-core path, dq and dk come
+// out already through the QK-norm + RoPE backward (*qk_fused = true);
+// otherwise the caller runs that backward as its own kernel (faster on B200:
+// the fused form lengthens the tail of every attention CTA).
+int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv,
+                  const float* rqk, bool* qk_fused) {
     const nc_model* m = c.m;
     float* Dbuf = c.at<float>(c.p.Dbuf);
+    *qk_fused = false;
     if (m->tc && attention_tc_bwd_supported(m->hd)) {
+        QkNormFuse fz{rqk, c.at<float>(c.p.cosb), c.at<float>(c.p.sinb)};
+        const QkNormFuse* fzp = rqk ? &fz : nullptr;
         int r;
         {
             Prof pr(c, P_ATTN_BWD_DQ, attn_flops(c), 0.0);
-            r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s);
+            r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s,
+                                    fzp);
         }
         if (r == 0) {
             Prof pr(c, P_ATTN_BWD_DKV, attn_flops(c), 0.0);
-            r = attention_tc_bwd_dkv(qkv, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s);
+            r = attention_tc_bwd_dkv(qkv, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s,
+                                     fzp);
         }
-        if (r == 0) return NC_OK;
+        if (r == 0) { *qk_fused = fzp != nullptr; return NC_OK; }
         if (r < 0) return NC_ERR_CUDA;
     }
     Prof pr(c, P_ATTN_BWD, 2.0 * attn_flops(c), 0.0);
@@ -265,11 +275,25 @@ int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save) {
         void* ru = lb + c.p.l_ru;
         void* h = lb + c.p.l_h;
         { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, a, (float*)(lb + c.p.l_r1), M, d, c.s)); }
-        RG(run_gemm(c, mk(m, M, m->Nqkv, d, a, d, true, w.wqkv(l), d, true, EPI_STORE, qkv, m->Nqkv, m->at), P_GEMM_FWD));
-        {
+        // q, k, v = a Wq^T, a Wk^T, a Wv^T; then q, k <- rope(rmsnorm(q, k)) per head, fused into
+        // the GEMM epilogue on the tensor-core path
+        bool qk_fused = false;
+        float* rqk = (float*)(lb + c.p.l_rqk);
+        if (m->tc && (m->hd == 64 || m->hd == 128)) {
+            GemmDesc gq = mk(m, M, m->Nqkv, d, a, d, true, w.wqkv(l), d, true, EPI_QKROPE, qkv, m->Nqkv, m->at);
+            gq.hd = m->hd; gq.T = c.p.T; gq.qk_heads = m->H + m->nkv;
+            gq.rqk = rqk; gq.cos_t = cs; gq.sin_t = sn;
+            Prof pr(c, P_GEMM_FWD, 2.0 * M * m->Nqkv * (double)d,
+                    A * ((double)M * d + (double)m->Nqkv * d + (double)M * m->Nqkv));
+            int r = gemm_tc(gq, c.ws + c.p.splitk, c.p.splitk_bytes, c.s);
+            if (r < 0) return NC_ERR_CUDA;
+            qk_fused = r == 0;
+        }
+        if (!qk_fused) {
+            RG(run_gemm(c, mk(m, M, m->Nqkv, d, a, d, true, w.wqkv(l), d, true, EPI_STORE, qkv, m->Nqkv, m->at),
+                        P_GEMM_FWD));
             Prof pr(c, P_QKROPE_FWD, 0.0, (double)M * (m->H + m->nkv) * (2.0 * A * m->hd + 4.0));
-            CK(launch_qknorm_rope_fwd(m->at, qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, c.p.T, m->H, m->nkv, m->hd,
-                                      c.s));
+            CK(launch_qknorm_rope_fwd(m->at, qkv, rqk, cs, sn, M, c.p.T, m->H, m->nkv, m->hd, c.s));
         }
         RG(attention_fwd(c, qkv, o, (float*)(lb + c.p.l_lse)));
         RG(run_gemm(c, mk(m, M, d, (int)Hhd, o, Hhd, true, w.wo(l), Hhd, true, EPI_ACCUM, x, d, DT_F32), P_GEMM_FWD));
@@ -342,8 +366,10 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at), P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
                           DT_F32), P_GEMM_WGRAD));
-        RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), dqkv));
-        {
+        bool qk_fused = false;
+        RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), dqkv, nullptr,
+                         &qk_fused));
+        if (!qk_fused) {
             Prof pr(c, P_QKROPE_BWD, 0.0, (double)M * (m->H + m->nkv) * (3.0 * A * m->hd + 4.0));
             CK(launch_qknorm_rope_bwd(m->at, dqkv, lb + c.p.l_qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, T, m->H,
                                       m->nkv, m->hd, s));
