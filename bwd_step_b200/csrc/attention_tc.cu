@@ -184,8 +184,14 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
             if (!warp_wait(s_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
             float s[128];
+            {
+                uint32_t rr[128];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS + lane_off + sb * 128 + c * 32, s + 32 * c);
+                for (int c = 0; c < 4; ++c) tmem_ld32_issue(tS + lane_off + sb * 128 + c * 32, rr + 32 * c);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(rr[i]);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_empty + 8 * sb);
@@ -502,8 +508,14 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
             float d0[32];
             {
                 float sv[32];
-                tmem_ld32(tS + lane_off + sb * 64 + ch * 32, sv);
-                tmem_ld32(tdP + lane_off + sb * 64 + ch * 32, d0);
+                {
+                    uint32_t rs[32], rd[32];
+                    tmem_ld32_issue(tS + lane_off + sb * 64 + ch * 32, rs);
+                    tmem_ld32_issue(tdP + lane_off + sb * 64 + ch * 32, rd);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(rs[i]); d0[i] = __uint_as_float(rd[i]); }
+                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const bool valid = live && (j < qb || hf * 64 + ch * 32 + i <= r);
@@ -612,9 +624,11 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
     const uint32_t b0 = smem_u32(bars);
     const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 32;  // qo_*[DKV_STG]
     const uint32_t st_full = b0 + 56, st_empty = b0 + 72;              // [2]
-    // pd_done[b] completes after the dV/dK MMAs of the units with parity b
-    // (once per two units), so a wait on it can never be lapped.
-    const uint32_t pd_full = b0 + 88, pd_done = b0 + 96;               // pd_done[2]
+    // pd_full[b] / pd_done[b]: P^T and dS^T of the units with parity b written /
+    // consumed (once per two units each).  Per-parity barriers keep every wait
+    // from being lapped: the softmax warps may run two units ahead of the MMA
+    // thread's wait on pd_full.
+    const uint32_t pd_full = b0 + 88, pd_done = b0 + 104;              // [2] each
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -633,6 +647,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         for (int s = 0; s < DKV_STG; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
         for (int s = 0; s < 2; ++s) { mbar_init(st_full + 8 * s, 1); mbar_init(st_empty + 8 * s, 8); }
         mbar_init(pd_full, 8);
+        mbar_init(pd_full + 8, 8);
         mbar_init(pd_done, 1);
         mbar_init(pd_done + 8, 1);
         *abort_flag = 0;
@@ -702,7 +717,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                     }
                     if (u > 0) {
                         const int uu = u - 1, st = uu % DKV_STG;
-                        if (!mbar_wait(pd_full, uu & 1, abort_flag, p.status)) break;
+                        if (!mbar_wait(pd_full + 8 * (uu & 1), (uu >> 1) & 1, abort_flag, p.status)) break;
                         tc_fence_after();
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks) {
@@ -738,8 +753,14 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             const float* lse_u = lse_s + st * 64;
             const float* d_u = d_s + st * 64;
             float sv[32], dp[32];
-            tmem_ld32(tSt + lane_off + sb * 64 + ch * 32, sv);
-            tmem_ld32(tdPt + lane_off + sb * 64 + ch * 32, dp);
+            {
+                uint32_t rs[32], rd[32];
+                tmem_ld32_issue(tSt + lane_off + sb * 64 + ch * 32, rs);
+                tmem_ld32_issue(tdPt + lane_off + sb * 64 + ch * 32, rd);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(rs[i]); dp[i] = __uint_as_float(rd[i]); }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(st_empty + 8 * sb);
@@ -771,7 +792,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(pd_full);
+            if (lane == 0) mbar_arrive(pd_full + 8 * (u & 1));
         }
         if (ok && warp_wait(pd_done + 8 * ((nunits - 1) & 1), ((nunits - 1) >> 1) & 1, abort_flag, p.status)) {
             tc_fence_after();
