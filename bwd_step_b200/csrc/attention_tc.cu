@@ -100,38 +100,37 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
     const uint32_t tS = tmem, tO = tmem + 256;
 
     if (warp == 0) {
-        if (lane == 0) {
-            const int xq = h * HD, xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
-            mbar_expect_tx(q_full, TILE);
+        // lane 0 loads Q and the K ring, lane 1 the V ring: each waits only on
+        // its own ring, so K tiles run ahead of the V slots that P*V frees late
+        if (lane < 2) {
+            const bool kl = lane == 0;
+            const int xq = h * HD, xkv = kl ? (p.H + g) * HD : (p.H + p.nkv + g) * HD;
+            const uint32_t full = kl ? k_full : v_full, empty = kl ? k_empty : v_empty;
+            const uint32_t dst = kl ? sK : sV;
+            if (kl) {
+                mbar_expect_tx(q_full, TILE);
 #pragma unroll
-            for (int kb = 0; kb < KB; ++kb) tma_load_2d(sQ + kb * 16384, &tm, xq + kb * 64, row0 + qb * 128, q_full);
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_2d(sQ + kb * 16384, &tm, xq + kb * 64, row0 + qb * 128, q_full);
+            }
             int issued = 0;
             for (int j = 0; j < nblk; ++j) {
                 const int st = j % STG;
                 const uint32_t ph = (j / STG) & 1;
-                if (!mbar_wait(k_empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(k_full + 8 * st, TILE);
+                if (!mbar_wait(empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(full + 8 * st, TILE);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb)
-                    tma_load_2d(sK + st * TILE + kb * 16384, &tm, xk + kb * 64, row0 + j * 128, k_full + 8 * st);
-                if (!mbar_wait(v_empty + 8 * st, ph ^ 1, abort_flag, p.status)) { issued = j + 1; break; }
-                mbar_expect_tx(v_full + 8 * st, TILE);
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb)
-                    tma_load_2d(sV + st * TILE + kb * 16384, &tm, xv + kb * 64, row0 + j * 128, v_full + 8 * st);
+                    tma_load_2d(dst + st * TILE + kb * 16384, &tm, xkv + kb * 64, row0 + j * 128, full + 8 * st);
                 issued = j + 1;
             }
             if (*abort_flag) {
                 // let copies in flight land before the block exits
                 uint64_t t0 = globaltimer();
-                while (!mbar_try(q_full, 0) && globaltimer() - t0 < 1000000ull) {}
+                if (kl) while (!mbar_try(q_full, 0) && globaltimer() - t0 < 1000000ull) {}
                 for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j) {
-                    const int st = j % STG;
-                    const uint32_t ph = (j / STG) & 1;
                     t0 = globaltimer();
-                    while (!mbar_try(k_full + 8 * st, ph) && globaltimer() - t0 < 1000000ull) {}
-                    t0 = globaltimer();
-                    while (!mbar_try(v_full + 8 * st, ph) && globaltimer() - t0 < 1000000ull) {}
+                    while (!mbar_try(full + 8 * (j % STG), (j / STG) & 1) && globaltimer() - t0 < 1000000ull) {}
                 }
             }
         }
@@ -418,35 +417,36 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
     const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
 
     if (warp == 0) {
-        if (lane == 0) {
-            const int xq = h * HD, xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
-            mbar_expect_tx(qd_full, 2 * TILE);
+        // lane 0 loads Q, dO and the K ring, lane 1 the V ring (V slots free
+        // early, after dP; K slots late, after dQ)
+        if (lane < 2) {
+            const bool kl = lane == 0;
+            const int xkv = kl ? (p.H + g) * HD : (p.H + p.nkv + g) * HD;
+            const uint32_t full = kl ? k_full : v_full, empty = kl ? k_empty : v_empty;
+            const uint32_t dst = kl ? sK : sV;
+            if (kl) {
+                mbar_expect_tx(qd_full, 2 * TILE);
 #pragma unroll
-            for (int kb = 0; kb < KB; ++kb) {
-                tma_load_2d(sQ + kb * 16384, &tmQKV, xq + kb * 64, row0 + qb * 128, qd_full);
-                tma_load_2d(sDO + kb * 16384, &tmDO, h * HD + kb * 64, row0 + qb * 128, qd_full);
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_2d(sQ + kb * 16384, &tmQKV, h * HD + kb * 64, row0 + qb * 128, qd_full);
+                    tma_load_2d(sDO + kb * 16384, &tmDO, h * HD + kb * 64, row0 + qb * 128, qd_full);
+                }
             }
             int issued = 0;
             for (int j = 0; j < nblk; ++j) {
                 const int st = j % STG;
                 const uint32_t ph = (j / STG) & 1;
-                if (!mbar_wait(k_empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
-                if (!mbar_wait(v_empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(k_full + 8 * st, TILE);
-                mbar_expect_tx(v_full + 8 * st, TILE);
+                if (!mbar_wait(empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(full + 8 * st, TILE);
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_2d(sK + st * TILE + kb * 16384, &tmQKV, xk + kb * 64, row0 + j * 128, k_full + 8 * st);
-                    tma_load_2d(sV + st * TILE + kb * 16384, &tmQKV, xv + kb * 64, row0 + j * 128, v_full + 8 * st);
-                }
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_2d(dst + st * TILE + kb * 16384, &tmQKV, xkv + kb * 64, row0 + j * 128, full + 8 * st);
                 issued = j + 1;
             }
             if (*abort_flag) {
-                drain(qd_full, 0);
-                for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j) {
-                    drain(k_full + 8 * (j % STG), (j / STG) & 1);
-                    drain(v_full + 8 * (j % STG), (j / STG) & 1);
-                }
+                if (kl) drain(qd_full, 0);
+                for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j)
+                    drain(full + 8 * (j % STG), (j / STG) & 1);
             }
         }
     } else if (warp == 1) {

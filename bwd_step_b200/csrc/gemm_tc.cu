@@ -21,6 +21,7 @@
 #include "tc_common.cuh"
 #include <cudaTypedefs.h>
 #include <algorithm>
+#include <cstring>
 
 namespace nc {
 namespace {
@@ -31,7 +32,7 @@ constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTE
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int NTHREADS = 192;
 constexpr int MAX_SPLITS = 8;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 32768 + 256;  // + epilogue staging
 
 struct TcParams {
     int M, N, K;
@@ -48,6 +49,8 @@ struct TcParams {
     float* rqk;
     const float* cos_t;
     const float* sin_t;
+    float2* stats;
+    int tma_out;  // epilogue stages 32x32 sub-tiles in shared memory and writes them by TMA
 };
 
 __device__ __forceinline__ void decode(const TcParams& p, int u, int& tm, int& tn, int& ks) {
@@ -81,6 +84,21 @@ __device__ __forceinline__ void store_row_bf16(bf16* dst, const float* v, int nv
 __device__ __forceinline__ void store_row(void* C, bool bf, int64_t off, const float* v, int nv, bool vec) {
     if (bf) store_row_bf16(reinterpret_cast<bf16*>(C) + off, v, nv, vec);
     else store_row_f32(reinterpret_cast<float*>(C) + off, v, nv, vec);
+}
+
+// Online (max, sum of exp) over the first nv of 32 softcapped logits.
+__device__ __forceinline__ void softcap_stats(const float* z, int nv, float& m, float& s) {
+    float cm = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        if (i < nv) cm = fmaxf(cm, z[i]);
+    const float nm = fmaxf(m, cm);
+    float acc = s * __expf(m - nm);  // m = -inf on the first chunk: s = 0 there
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        if (i < nv) acc += __expf(z[i] - nm);
+    m = nm;
+    s = acc;
 }
 
 // Epilogue of 32 consecutive columns n0.. of one output row.
@@ -139,6 +157,80 @@ __device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int
             for (int i = 0; i < 32; ++i) v[i] = p.cap * tanhf(v[i] * ic);
             store_row(p.C, p.c_bf16, off, v, nv, vec);
         } break;
+    }
+}
+
+// ------------------------------------------------------------------ staged epilogue
+// Each epilogue warp owns two 4 KB staging buffers.  A 32-row x 32-column
+// sub-tile is written into one of them in the layout of the output tensor
+// map's swizzle (fp32: 128-byte rows, 128B swizzle; bf16: 64-byte rows, 64B
+// swizzle; conflict-free for the row-per-thread writes), then one lane issues
+// a TMA store -- or, for the residual-add epilogue, a TMA reduce-add, so C is
+// never read into the SM.  A buffer is reused only after the store issued two
+// chunks earlier has finished reading it.
+constexpr int STAGING_BYTES = 4 * 2 * 4096;
+
+__device__ __forceinline__ void stage_f32(uint8_t* buf, int lane, const float* v) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<float4*>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+            make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+}
+__device__ __forceinline__ void stage_bf16(uint8_t* buf, int lane, const float* v) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) store_vec(reinterpret_cast<bf16*>(buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4)), v + 8 * k);
+}
+
+// One 32-column chunk through the staging buffers; called by all lanes of the warp.
+__device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUtensorMap* tmC, const CUtensorMap* tmC2,
+                                                   uint8_t* stg, int lane, int ks, int row, int row0w, int n0, float* v,
+                                                   int cnt) {
+    uint8_t* buf = stg + (cnt & 1) * 4096;
+    if (cnt >= 2) {
+        if (lane == 0) bulk_wait_read_1();
+        __syncwarp();
+    }
+    const int mode = p.part ? EPI_STORE : p.epi;
+    const bool bf = p.part ? false : p.c_bf16 != 0;
+    if (mode == EPI_RELU2) {
+        float r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) { r[i] = fmaxf(v[i], 0.f); v[i] = r[i] * r[i]; }
+        stage_bf16(buf, lane, v);
+        stage_bf16(buf + 2048, lane, r);
+    } else {
+        if (mode == EPI_RELU2_BWD && row < p.M) {
+            const bf16* a = p.aux + (int64_t)row * p.ldaux + n0;
+            const int nv = min(32, p.N - n0);
+            if (nv == 32) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float u[8];
+                    load_vec(a + 8 * i, u);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) v[8 * i + j] *= 2.f * u[j];
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < nv) v[i] *= 2.f * __bfloat162float(a[i]);
+            }
+        } else if (mode == EPI_SOFTCAP) {
+            const float ic = 1.f / p.cap;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = p.cap * tanhf(v[i] * ic);
+        }
+        if (bf) stage_bf16(buf, lane, v);
+        else stage_f32(buf, lane, v);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        if (p.part) tma_store_3d(tmC, n0, row0w, ks, smem_u32(buf));  // [splits, M, N]: clipped at M per split
+        else if (mode == EPI_ACCUM) tma_reduce_add_2d(tmC, n0, row0w, smem_u32(buf));
+        else tma_store_2d(tmC, n0, row0w, smem_u32(buf));
+        if (mode == EPI_RELU2) tma_store_2d(tmC2, n0, row0w, smem_u32(buf + 2048));
+        bulk_commit();
     }
 }
 
@@ -205,10 +297,12 @@ __device__ __forceinline__ void epilogue_qkrope(const TcParams& p, int row, int 
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2, const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES * STAGE_BYTES);
+    uint8_t* staging = smem + (size_t)STAGES * STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(staging + STAGING_BYTES);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -305,6 +399,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     } else {
         // ---------------- epilogue warps 2..5; warp w reads TMEM lanes 32*(w%4)..
         const int q = warp & 3;
+        uint8_t* stg = staging + (warp - 2) * 8192;
+        int cnt = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
@@ -312,25 +408,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             decode(p, u, tm, tn, ks);
             if (!warp_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, p.status)) break;
             tc_fence_after();
-            const int row = tm * BM + q * 32 + lane;
+            const int row0w = tm * BM + q * 32;
+            const int row = row0w + lane;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             if (p.epi == EPI_QKROPE) {
                 if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
                 else epilogue_qkrope<64>(p, row, tn * BN, tb);
             } else {
+                float smax = -INFINITY, ssum = 0.f;  // softcap row statistics over the tile
                 for (int c = 0; c < BN / 32; ++c) {
                     const int n0 = tn * BN + c * 32;
                     if (n0 >= p.N) break;
                     float v[32];
                     tmem_ld32(tb + c * 32, v);
-                    if (row < p.M) epilogue(p, ks, row, n0, v);
+                    if (p.tma_out) {
+                        epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++);
+                        if (p.stats && row < p.M) softcap_stats(v, min(32, p.N - n0), smax, ssum);
+                    } else if (row < p.M) {
+                        epilogue(p, ks, row, n0, v);
+                        if (p.stats) softcap_stats(v, min(32, p.N - n0), smax, ssum);
+                    }
                 }
+                if (p.stats && row < p.M) p.stats[(size_t)row * p.tiles_n + tn] = make_float2(smax, ssum);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
+        if (lane == 0) bulk_wait_all();  // staged stores finished before the block exits
     }
     tc_fence_before();
     __syncthreads();
@@ -351,13 +457,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 // signals the even CTA that the accumulator may be reused.
 constexpr int STAGES2 = 6;
 constexpr int STAGE2_BYTES = 2 * 128 * BK * 2;  // A 128x64 + B 128x64, bf16
-constexpr size_t SMEM2_BYTES = 1024 + (size_t)STAGES2 * STAGE2_BYTES + 256;
+constexpr size_t SMEM2_BYTES = 1024 + (size_t)STAGES2 * STAGE2_BYTES + STAGING_BYTES + 256;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
-gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2, const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)STAGES2 * STAGE2_BYTES);
+    uint8_t* staging = smem + (size_t)STAGES2 * STAGE2_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(staging + STAGING_BYTES);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES2 + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -456,6 +564,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     } else {
         // ---------------- epilogue warps 2..5 of both CTAs
         const int q = warp & 3;
+        uint8_t* stg = staging + (warp - 2) * 8192;
+        int cnt = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = cluster; u < p.num_units; u += nclusters) {
@@ -463,25 +573,35 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             decode(p, u, tm, tn, ks);
             if (!warp_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, p.status)) break;
             tc_fence_after();
-            const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
+            const int row0w = tm * 256 + (int)rank * 128 + q * 32;
+            const int row = row0w + lane;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             if (p.epi == EPI_QKROPE) {
                 if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
                 else epilogue_qkrope<64>(p, row, tn * BN, tb);
             } else {
+                float smax = -INFINITY, ssum = 0.f;  // softcap row statistics over the tile
                 for (int c = 0; c < BN / 32; ++c) {
                     const int n0 = tn * BN + c * 32;
                     if (n0 >= p.N) break;
                     float v[32];
                     tmem_ld32(tb + c * 32, v);
-                    if (row < p.M) epilogue(p, ks, row, n0, v);
+                    if (p.tma_out) {
+                        epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++);
+                        if (p.stats && row < p.M) softcap_stats(v, min(32, p.N - n0), smax, ssum);
+                    } else if (row < p.M) {
+                        epilogue(p, ks, row, n0, v);
+                        if (p.stats) softcap_stats(v, min(32, p.N - n0), smax, ssum);
+                    }
                 }
+                if (p.stats && row < p.M) p.stats[(size_t)row * p.tiles_n + tn] = make_float2(smax, ssum);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_addr(bar_tempty + 8 * acc));
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
+        if (lane == 0) bulk_wait_all();  // staged stores finished before the block exits
     }
     tc_fence_before();
     cluster_sync();  // no CTA leaves while its pair may still signal or read it
@@ -502,6 +622,34 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
     }
     return fn;
+}
+
+// Tensor map for the staged epilogue's 32x32 output boxes (fp32: 128B
+// swizzle, bf16: 64B swizzle) over a row-major [rows, cols] array.
+bool make_out_map(CUtensorMap* map, void* base, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const uint64_t es = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * es};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Same for the split-K partial sums, fp32 [splits, rows, cols] contiguous.
+bool make_partial_map(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows, uint64_t splits) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cols, rows, splits};
+    cuuint64_t strides[2] = {cols * 4, cols * rows * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2-D bf16 tensor map over a row-major [outer, inner] array with row stride ld
@@ -577,6 +725,7 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     p.status = g.status;
     p.hd = g.hd; p.T = g.T; p.qk_heads = g.qk_heads;
     p.rqk = g.rqk; p.cos_t = g.cos_t; p.sin_t = g.sin_t;
+    p.stats = g.epi == EPI_SOFTCAP ? g.stats : nullptr;
     const int esz = p.c_bf16 ? 2 : 4;
     bool vec = al16(g.C) && (g.ldc * esz) % 16 == 0;
     if (g.epi == EPI_RELU2) vec = vec && al16(g.C2) && (g.ldc2 * 2) % 16 == 0;
@@ -609,9 +758,26 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     p.part = p.splits > 1 ? reinterpret_cast<float*>(splitk) : nullptr;
     p.vec_ok = (p.part ? (g.N % 4 == 0) : vec) ? 1 : 0;
     p.num_units = tiles * p.splits;
+    // staged (TMA) epilogue for the plain, residual-add, relu^2 (both outputs),
+    // relu^2-backward and softcap epilogues, and for split-K partials
+    CUtensorMap tc_out, tc_out2;
+    memset(&tc_out, 0, sizeof(tc_out));
+    memset(&tc_out2, 0, sizeof(tc_out2));
+    p.tma_out = 0;
+    if (p.part) {
+        if (make_partial_map(&tc_out, p.part, g.N, g.M, p.splits)) p.tma_out = 1;
+    } else if (vec && g.epi != EPI_QKROPE) {
+        const bool bf = p.c_bf16 != 0;
+        if (g.epi == EPI_ACCUM && bf) {
+            // reduce-add is fp32 only
+        } else if (make_out_map(&tc_out, g.C, bf, g.N, g.M, g.ldc) &&
+                   (g.epi != EPI_RELU2 || make_out_map(&tc_out2, g.C2, true, g.N, g.M, g.ldc2))) {
+            p.tma_out = 1;
+        }
+    }
     const int grid = std::min(p.num_units, sms);
-    if (pair) gemm_tc2_kernel<<<2 * grid, NTHREADS, SMEM2_BYTES, s>>>(ta, tb, p);
-    else gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, p);
+    if (pair) gemm_tc2_kernel<<<2 * grid, NTHREADS, SMEM2_BYTES, s>>>(ta, tb, tc_out, tc_out2, p);
+    else gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tc_out, tc_out2, p);
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return -1;
     if (p.part) {

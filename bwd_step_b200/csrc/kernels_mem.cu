@@ -303,6 +303,85 @@ __device__ __forceinline__ MaxSum ms_combine(MaxSum a, MaxSum b) {
     return {m, a.s * __expf(a.m - m) + b.s * __expf(b.m - m)};
 }
 
+__device__ __forceinline__ void store4(float* p, const float* v) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store4(bf16* p, const float* v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+}
+
+// Block-wide (max, sum) combine; result valid in every thread.
+__device__ __forceinline__ MaxSum block_ms(MaxSum acc, MaxSum* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        MaxSum other = {__shfl_xor_sync(0xffffffffu, acc.m, o), __shfl_xor_sync(0xffffffffu, acc.s, o)};
+        acc = ms_combine(acc, other);
+    }
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[w] = acc;
+    __syncthreads();
+    if (w == 0) {
+        const int nw = blockDim.x >> 5;
+        acc = lane < nw ? red[lane] : MaxSum{-INFINITY, 0.f};
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            MaxSum other = {__shfl_xor_sync(0xffffffffu, acc.m, o), __shfl_xor_sync(0xffffffffu, acc.s, o)};
+            acc = ms_combine(acc, other);
+        }
+        if (lane == 0) red[0] = acc;
+    }
+    __syncthreads();
+    return red[0];
+}
+
+// dl for one row given its LSE: one pass over z (4 logits per thread step).
+template <typename D>
+__device__ __forceinline__ void ce_write_dl(const float* zr, D* out, int V, int t, bool bad, float lse, float cap,
+                                            float inv_M) {
+    const float inv_cap = 1.f / cap;
+    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
+        const float4 v = *reinterpret_cast<const float4*>(zr + c);
+        const float zz[4] = {v.x, v.y, v.z, v.w};
+        float g[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float pk = __expf(zz[k] - lse) - ((c + k) == t ? 1.f : 0.f);
+            const float q = zz[k] * inv_cap;
+            g[k] = bad ? 0.f : pk * inv_M * (1.f - q * q);
+        }
+        store4(out + c, g);
+    }
+}
+
+// Cross-entropy of one row with its LSE combined from the per-tile (max,
+// sum exp) statistics written by the softcap GEMM epilogue: z is read once.
+template <typename D>
+__global__ void ce_chunk_stats_kernel(const float* __restrict__ z, const int32_t* __restrict__ tgt, int R, int V,
+                                      float cap, float inv_M, float* __restrict__ loss_rows, D* __restrict__ dl,
+                                      int* status, const float2* __restrict__ stats, int ntiles) {
+    __shared__ MaxSum red[32];
+    const int row = blockIdx.x;
+    const float* zr = z + (size_t)row * V;
+    MaxSum acc = {-INFINITY, 0.f};
+    for (int i = threadIdx.x; i < ntiles; i += blockDim.x) {
+        const float2 st = stats[(size_t)row * ntiles + i];
+        acc = ms_combine(acc, MaxSum{st.x, st.y});
+    }
+    acc = block_ms(acc, red);
+    const float lse = acc.m + logf(acc.s);
+    const int t = tgt[row];
+    const bool bad = t < 0 || t >= V;
+    if (threadIdx.x == 0) {
+        if (bad) set_status(status, ST_BAD_TOKEN);
+        loss_rows[row] = bad ? 0.f : lse - zr[t];
+    }
+    ce_write_dl(zr, dl + (size_t)row * V, V, t, bad, lse, cap, inv_M);
+}
+
 template <typename D>
 __global__ void ce_chunk_kernel(const float* __restrict__ z, const int32_t* __restrict__ tgt, int R, int V,
                                 float cap, float inv_M, float* __restrict__ loss_rows, D* __restrict__ dl,
@@ -346,18 +425,7 @@ __global__ void ce_chunk_kernel(const float* __restrict__ z, const int32_t* __re
         if (bad) set_status(status, ST_BAD_TOKEN);
         loss_rows[row] = bad ? 0.f : lse - zr[t];
     }
-    D* out = dl + (size_t)row * V;
-    float inv_cap = 1.f / cap;
-    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
-        float4 v = *reinterpret_cast<const float4*>(zr + c);
-        float zz[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float p = expf(zz[k] - lse) - ((c + k) == t ? 1.f : 0.f);
-            float q = zz[k] * inv_cap;
-            out[c + k] = fromf<D>(bad ? 0.f : p * inv_M * (1.f - q * q));
-        }
-    }
+    ce_write_dl(zr, dl + (size_t)row * V, V, t, bad, lse, cap, inv_M);
 }
 
 __global__ void loss_reduce_kernel(const float* __restrict__ rows, int M, float* loss) {
@@ -671,8 +739,19 @@ cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const 
 }
 
 cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R, int V, float cap, float inv_M,
-                            float* loss_rows, void* dl, int* status, cudaStream_t s) {
+                            float* loss_rows, void* dl, int* status, cudaStream_t s, const float2* stats,
+                            int ntiles) {
     if (R <= 0) return cudaSuccess;
+    if (stats) {
+        if (dlt == DT_BF16)
+            ce_chunk_stats_kernel<bf16><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (bf16*)dl, status,
+                                                          stats, ntiles);
+        else
+            ce_chunk_stats_kernel<float><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (float*)dl, status,
+                                                           stats, ntiles);
+        count_launch();
+        return cudaGetLastError();
+    }
     if (dlt == DT_BF16)
         ce_chunk_kernel<bf16><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (bf16*)dl, status);
     else

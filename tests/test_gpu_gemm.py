@@ -82,6 +82,14 @@ def test_split_k(ak, bk):
     _run(256, 256, 8192, ak, bk, 1, False, scratch_mb=64, seed=4)
 
 
+@pytest.mark.parametrize("M,N", [(896, 768), (200, 520), (1000, 264)])
+def test_split_k_ragged_rows(M, N):
+    # M not a multiple of the tile height: the last tile's extra rows must not
+    # spill into the next split's partial sums
+    _run(M, N, 4096, False, False, 0, False, scratch_mb=128, seed=M)
+    _run(M, N, 4096, False, False, 1, False, scratch_mb=128, seed=M + 1)
+
+
 def test_fma_gemm_matches_too():
     _run(200, 72, 136, False, True, 2, True, use_tc=0)
     _run(200, 72, 136, True, False, 4, False, use_tc=0, scale=3.0)
