@@ -750,8 +750,18 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             // before this warp finishes the unit, which frees the stage)
             if (!warp_wait(qo_full + 8 * st, (u / DKV_STG) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
-            const float* lse_u = lse_s + st * 64;
-            const float* d_u = d_s + st * 64;
+            // this warp's 32 query columns of the unit: lse (to log2 units) and D
+            float l2[32], dd[32];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float4 a = reinterpret_cast<const float4*>(lse_s + st * 64 + ch * 32)[k];
+                const float4 b = reinterpret_cast<const float4*>(d_s + st * 64 + ch * 32)[k];
+                l2[4 * k] = a.x * kLog2e; l2[4 * k + 1] = a.y * kLog2e; l2[4 * k + 2] = a.z * kLog2e;
+                l2[4 * k + 3] = a.w * kLog2e;
+                dd[4 * k] = b.x; dd[4 * k + 1] = b.y; dd[4 * k + 2] = b.z; dd[4 * k + 3] = b.w;
+            }
+            // units whose queries all see every key of the block need no mask
+            const bool full = i * 64 + ch * 32 >= kvb * 128 + 127 && i * 64 + ch * 32 + 31 < p.T;
             float sv[32], dp[32];
             {
                 uint32_t rs[32], rd[32];
@@ -764,13 +774,22 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(st_empty + 8 * sb);
+            if (full) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int qc = ch * 32 + e, qpos = i * 64 + qc;
-                const bool valid = qpos >= kpos && qpos < p.T;
-                const float P = valid ? ex2(sv[e] * p.scale_log2 - lse_u[qc] * kLog2e) : 0.f;
-                dp[e] = valid ? P * (dp[e] - d_u[qc]) : 0.f;
-                sv[e] = P;
+                for (int e = 0; e < 32; ++e) {
+                    const float P = ex2(sv[e] * p.scale_log2 - l2[e]);
+                    dp[e] = P * (dp[e] - dd[e]);
+                    sv[e] = P;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int qpos = i * 64 + ch * 32 + e;
+                    const bool valid = qpos >= kpos && qpos < p.T;
+                    const float P = valid ? ex2(sv[e] * p.scale_log2 - l2[e]) : 0.f;
+                    dp[e] = valid ? P * (dp[e] - dd[e]) : 0.f;
+                    sv[e] = P;
+                }
             }
             // P^T / dS^T buffer (u & 1) was last read by the dV/dK MMAs of unit u-2
             if (u > 1 && !warp_wait(pd_done + 8 * (u & 1), ((u >> 1) - 1) & 1, abort_flag, p.status)) {

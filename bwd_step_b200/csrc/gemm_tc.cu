@@ -49,7 +49,6 @@ struct TcParams {
     float* rqk;
     const float* cos_t;
     const float* sin_t;
-    float2* stats;
     int tma_out;  // epilogue stages 32x32 sub-tiles in shared memory and writes them by TMA
 };
 
@@ -84,21 +83,6 @@ __device__ __forceinline__ void store_row_bf16(bf16* dst, const float* v, int nv
 __device__ __forceinline__ void store_row(void* C, bool bf, int64_t off, const float* v, int nv, bool vec) {
     if (bf) store_row_bf16(reinterpret_cast<bf16*>(C) + off, v, nv, vec);
     else store_row_f32(reinterpret_cast<float*>(C) + off, v, nv, vec);
-}
-
-// Online (max, sum of exp) over the first nv of 32 softcapped logits.
-__device__ __forceinline__ void softcap_stats(const float* z, int nv, float& m, float& s) {
-    float cm = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        if (i < nv) cm = fmaxf(cm, z[i]);
-    const float nm = fmaxf(m, cm);
-    float acc = s * __expf(m - nm);  // m = -inf on the first chunk: s = 0 there
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        if (i < nv) acc += __expf(z[i] - nm);
-    m = nm;
-    s = acc;
 }
 
 // Epilogue of 32 consecutive columns n0.. of one output row.
@@ -415,21 +399,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
                 else epilogue_qkrope<64>(p, row, tn * BN, tb);
             } else {
-                float smax = -INFINITY, ssum = 0.f;  // softcap row statistics over the tile
                 for (int c = 0; c < BN / 32; ++c) {
                     const int n0 = tn * BN + c * 32;
                     if (n0 >= p.N) break;
                     float v[32];
                     tmem_ld32(tb + c * 32, v);
-                    if (p.tma_out) {
-                        epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++);
-                        if (p.stats && row < p.M) softcap_stats(v, min(32, p.N - n0), smax, ssum);
-                    } else if (row < p.M) {
-                        epilogue(p, ks, row, n0, v);
-                        if (p.stats) softcap_stats(v, min(32, p.N - n0), smax, ssum);
-                    }
+                    if (p.tma_out) epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++);
+                    else if (row < p.M) epilogue(p, ks, row, n0, v);
                 }
-                if (p.stats && row < p.M) p.stats[(size_t)row * p.tiles_n + tn] = make_float2(smax, ssum);
             }
             tc_fence_before();
             __syncwarp();
@@ -580,21 +557,14 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
                 else epilogue_qkrope<64>(p, row, tn * BN, tb);
             } else {
-                float smax = -INFINITY, ssum = 0.f;  // softcap row statistics over the tile
                 for (int c = 0; c < BN / 32; ++c) {
                     const int n0 = tn * BN + c * 32;
                     if (n0 >= p.N) break;
                     float v[32];
                     tmem_ld32(tb + c * 32, v);
-                    if (p.tma_out) {
-                        epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++);
-                        if (p.stats && row < p.M) softcap_stats(v, min(32, p.N - n0), smax, ssum);
-                    } else if (row < p.M) {
-                        epilogue(p, ks, row, n0, v);
-                        if (p.stats) softcap_stats(v, min(32, p.N - n0), smax, ssum);
-                    }
+                    if (p.tma_out) epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++);
+                    else if (row < p.M) epilogue(p, ks, row, n0, v);
                 }
-                if (p.stats && row < p.M) p.stats[(size_t)row * p.tiles_n + tn] = make_float2(smax, ssum);
             }
             tc_fence_before();
             __syncwarp();
@@ -725,7 +695,6 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     p.status = g.status;
     p.hd = g.hd; p.T = g.T; p.qk_heads = g.qk_heads;
     p.rqk = g.rqk; p.cos_t = g.cos_t; p.sin_t = g.sin_t;
-    p.stats = g.epi == EPI_SOFTCAP ? g.stats : nullptr;
     const int esz = p.c_bf16 ? 2 : 4;
     bool vec = al16(g.C) && (g.ldc * esz) % 16 == 0;
     if (g.epi == EPI_RELU2) vec = vec && al16(g.C2) && (g.ldc2 * 2) % 16 == 0;

@@ -39,11 +39,8 @@ cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const 
                                    int hd, cudaStream_t s);
 // Cross-entropy over R rows of softcapped logits z [R, V] (fp32):
 // loss_rows[r] = lse - z[tgt]; dl = inv_M*(softmax - onehot)*(1-(z/cap)^2).
-// With stats (from the softcap GEMM epilogue, ntiles per row) the row LSE
-// comes from them and z is read once; otherwise two passes over each row.
 cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R, int V, float cap,
-                            float inv_M, float* loss_rows, void* dl, int* status, cudaStream_t s,
-                            const float2* stats = nullptr, int ntiles = 0);
+                            float inv_M, float* loss_rows, void* dl, int* status, cudaStream_t s);
 // loss = mean(loss_rows[0..M)), fixed summation order.
 cudaError_t launch_loss_reduce(const float* loss_rows, int M, float* loss, cudaStream_t s);
 
@@ -103,9 +100,6 @@ struct GemmDesc {
     float* rqk = nullptr;
     const float* cos_t = nullptr;
     const float* sin_t = nullptr;
-    // EPI_SOFTCAP (tcgen05 only, optional): per row and 256-column tile tn,
-    // stats[row * ceil(N/256) + tn] = (max z, sum exp(z - max)) over the tile.
-    float2* stats = nullptr;
 };
 
 // Plain fp32-FMA tiled GEMM (any strides, any sizes).

@@ -314,30 +314,6 @@ __device__ __forceinline__ void store4(bf16* p, const float* v) {
     *reinterpret_cast<uint2*>(p) = u;
 }
 
-// Block-wide (max, sum) combine; result valid in every thread.
-__device__ __forceinline__ MaxSum block_ms(MaxSum acc, MaxSum* red) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        MaxSum other = {__shfl_xor_sync(0xffffffffu, acc.m, o), __shfl_xor_sync(0xffffffffu, acc.s, o)};
-        acc = ms_combine(acc, other);
-    }
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) red[w] = acc;
-    __syncthreads();
-    if (w == 0) {
-        const int nw = blockDim.x >> 5;
-        acc = lane < nw ? red[lane] : MaxSum{-INFINITY, 0.f};
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            MaxSum other = {__shfl_xor_sync(0xffffffffu, acc.m, o), __shfl_xor_sync(0xffffffffu, acc.s, o)};
-            acc = ms_combine(acc, other);
-        }
-        if (lane == 0) red[0] = acc;
-    }
-    __syncthreads();
-    return red[0];
-}
-
 // dl for one row given its LSE: one pass over z (4 logits per thread step).
 template <typename D>
 __device__ __forceinline__ void ce_write_dl(const float* zr, D* out, int V, int t, bool bad, float lse, float cap,
@@ -355,31 +331,6 @@ __device__ __forceinline__ void ce_write_dl(const float* zr, D* out, int V, int 
         }
         store4(out + c, g);
     }
-}
-
-// Cross-entropy of one row with its LSE combined from the per-tile (max,
-// sum exp) statistics written by the softcap GEMM epilogue: z is read once.
-template <typename D>
-__global__ void ce_chunk_stats_kernel(const float* __restrict__ z, const int32_t* __restrict__ tgt, int R, int V,
-                                      float cap, float inv_M, float* __restrict__ loss_rows, D* __restrict__ dl,
-                                      int* status, const float2* __restrict__ stats, int ntiles) {
-    __shared__ MaxSum red[32];
-    const int row = blockIdx.x;
-    const float* zr = z + (size_t)row * V;
-    MaxSum acc = {-INFINITY, 0.f};
-    for (int i = threadIdx.x; i < ntiles; i += blockDim.x) {
-        const float2 st = stats[(size_t)row * ntiles + i];
-        acc = ms_combine(acc, MaxSum{st.x, st.y});
-    }
-    acc = block_ms(acc, red);
-    const float lse = acc.m + logf(acc.s);
-    const int t = tgt[row];
-    const bool bad = t < 0 || t >= V;
-    if (threadIdx.x == 0) {
-        if (bad) set_status(status, ST_BAD_TOKEN);
-        loss_rows[row] = bad ? 0.f : lse - zr[t];
-    }
-    ce_write_dl(zr, dl + (size_t)row * V, V, t, bad, lse, cap, inv_M);
 }
 
 template <typename D>
@@ -739,23 +690,14 @@ cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const 
 }
 
 cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R, int V, float cap, float inv_M,
-                            float* loss_rows, void* dl, int* status, cudaStream_t s, const float2* stats,
-                            int ntiles) {
+                            float* loss_rows, void* dl, int* status, cudaStream_t s) {
     if (R <= 0) return cudaSuccess;
-    if (stats) {
-        if (dlt == DT_BF16)
-            ce_chunk_stats_kernel<bf16><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (bf16*)dl, status,
-                                                          stats, ntiles);
-        else
-            ce_chunk_stats_kernel<float><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (float*)dl, status,
-                                                           stats, ntiles);
-        count_launch();
-        return cudaGetLastError();
-    }
+    // 1024 threads per row: about 300 rows in flight (76 MB of fp32 logits at V =
+    // 65536), so each row's second pass reads it back from L2, not HBM
     if (dlt == DT_BF16)
-        ce_chunk_kernel<bf16><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (bf16*)dl, status);
+        ce_chunk_kernel<bf16><<<R, 1024, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (bf16*)dl, status);
     else
-        ce_chunk_kernel<float><<<R, 256, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (float*)dl, status);
+        ce_chunk_kernel<float><<<R, 1024, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (float*)dl, status);
     count_launch();
     return cudaGetLastError();
 }

@@ -58,7 +58,7 @@ struct Plan {
     size_t tok, tgt, cosb, sinb, x, dx, g, dxb, xf, r0, rf;
     size_t layers, lay_stride;
     size_t l_a, l_r1, l_qkv, l_rqk, l_o, l_lse, l_m, l_r2, l_ru, l_h;
-    size_t du, dO, dqkv, Dbuf, zc, dlc, loss_rows, ce_stats, emb, splitk, splitk_bytes, attn_ws, attn_ws_bytes;
+    size_t du, dO, dqkv, Dbuf, zc, dlc, loss_rows, emb, splitk, splitk_bytes, attn_ws, attn_ws_bytes;
 };
 
 // Rows of the LM head processed at once: the [R, V] fp32 logit chunk plus its
@@ -112,7 +112,6 @@ Plan make_plan(const nc_model* m, int B, int T) {
     p.zc = take(4ull * p.R * m->V);
     p.dlc = take(A * (size_t)p.R * m->V);
     p.loss_rows = take(4 * M);
-    p.ce_stats = take(8ull * p.R * ((m->V + 255) / 256));
     p.emb = take(embed_scratch_bytes(p.M, m->V, m->d));
     size_t max_out = std::max({(size_t)p.R * d, (size_t)m->F * d, (size_t)m->H * m->hd * d, (size_t)m->Nqkv * d});
     p.splitk_bytes = m->tc ? gemm_tc_splitk_bytes(max_out) : 0;
@@ -328,25 +327,11 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     for (int r0 = 0; r0 < M; r0 += c.p.R) {
         int rc = std::min(c.p.R, M - r0);
         const char* xfc = (const char*)xf + (size_t)r0 * d * A;
-        // softcapped logits of the chunk; on the tensor-core path the epilogue
-        // also leaves each row's (max, sum exp) per 256-column tile, so the
-        // cross-entropy reads the chunk once
-        GemmDesc gz = mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, DT_F32);
-        float2* stats = c.at<float2>(c.p.ce_stats);
-        bool have_stats = false;
-        if (m->tc) {
-            gz.stats = stats;
-            Prof pr(c, P_GEMM_LM_Z, 2.0 * rc * V * (double)d, A * ((double)rc * d + (double)V * d) + 4.0 * rc * V);
-            int r = gemm_tc(gz, c.ws + c.p.splitk, c.p.splitk_bytes, s);
-            if (r < 0) return NC_ERR_CUDA;
-            have_stats = r == 0;
-            gz.stats = nullptr;
-        }
-        if (!have_stats) RG(run_gemm(c, gz, P_GEMM_LM_Z));
+        RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, DT_F32), P_GEMM_LM_Z));
         {
             Prof pr(c, P_CE, 0.0, (double)rc * V * (4.0 + A));
             CK(launch_ce_chunk(m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M, loss_rows + r0, dlc,
-                               m->status, s, have_stats ? stats : nullptr, (V + 255) / 256));
+                               m->status, s));
         }
         RG(run_gemm(c, mk(m, rc, d, V, dlc, V, true, w.wlm(), d, false, EPI_STORE, gbuf + (size_t)r0 * d, d,
                           DT_F32), P_GEMM_LM_DX));
