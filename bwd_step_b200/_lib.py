@@ -9,7 +9,8 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libnanochat_b200.so")
+# NC_LIB_PATH selects another build of the same library (e.g. for A/B timing).
+LIB_PATH = os.environ.get("NC_LIB_PATH") or os.path.join(HERE, "libnanochat_b200.so")
 
 NC_OK = 0
 NC_ERR_INVALID_ARG = -1

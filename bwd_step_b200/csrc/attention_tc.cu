@@ -284,22 +284,26 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 // ============================================================================ backward
 // dQ, one CTA per (query block of 128, head, batch row).  Key blocks j = 0..qb
 // are processed as 64-key sub-blocks t: S_t = Q K_t^T and dP_t = dO V_t^T into
-// one of two TMEM buffers; per query row (one per thread)
+// one of three TMEM buffers; per query row (one per thread)
 // P = 2^(S*scale*log2e - lse*log2e) with the causal mask and dS = P (dP - D),
-// as bf16 into one of two shared-memory tiles; dQ += dS_{t-1} K_{t-1} is issued
-// one sub-block behind, with the K tile read again as an MN-major operand.
+// as bf16 into one of two shared-memory tiles; dQ += dS_{t-2} K_{t-2} is issued
+// two sub-blocks behind (the score MMAs of two sub-blocks cover the softmax
+// round trip), with the K tile read again as an MN-major operand.
 // dq = dQ / sqrt(hd).
 template <int HD>
 struct DqLayout {
     static constexpr int KB = HD / 64;
-    static constexpr int TILE = KB * 16384;
+    static constexpr int TILE = KB * 16384;   // [128 x HD]: Q, dO
+    static constexpr int HTILE = KB * 8192;   // [64 x HD]: a K or V sub-block
+    static constexpr int RING = 4;            // K and V sub-block stages
     static constexpr int Q = 0;
     static constexpr int DO = Q + TILE;
     static constexpr int K = DO + TILE;
-    static constexpr int V = K + STG * TILE;
-    static constexpr int DS = V + STG * TILE;   // [2][128 x 64] bf16
+    static constexpr int V = K + RING * HTILE;
+    static constexpr int DS = V + RING * HTILE;  // [2][128 x 64] bf16
     static constexpr int BAR = DS + 32768;
     static constexpr int BYTES = BAR + 256 + 1024;
+    static_assert(BYTES <= 232448, "dQ shared memory exceeds the per-block limit");
 };
 
 struct BwdParams {
@@ -374,10 +378,11 @@ __device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
 
 template <int HD>
 __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
+                                                           const __grid_constant__ CUtensorMap tmKV64,
                                                            const __grid_constant__ CUtensorMap tmDO,
                                                            const BwdParams p) {
     using Lay = DqLayout<HD>;
-    constexpr int KB = Lay::KB, TILE = Lay::TILE;
+    constexpr int KB = Lay::KB, TILE = Lay::TILE, HTILE = Lay::HTILE, RING = Lay::RING;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t base = smem_u32(smem);
@@ -385,9 +390,11 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
     const uint32_t sDS = base + Lay::DS;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
-    const uint32_t qd_full = b0, k_full = b0 + 8, k_empty = b0 + 24, v_full = b0 + 40, v_empty = b0 + 56;
-    const uint32_t s_full = b0 + 72, s_empty = b0 + 88, ds_full = b0 + 104, ds_done = b0 + 120;  // each [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+    const uint32_t qd_full = b0;
+    const uint32_t k_full = b0 + 8, k_empty = b0 + 40, v_full = b0 + 72, v_empty = b0 + 104;  // [RING]
+    const uint32_t s_full = b0 + 136, s_empty = b0 + 160;  // [3]: S/dP TMEM buffers
+    const uint32_t ds_full = b0 + 184, ds_done = b0 + 200; // [2]: dS smem tiles
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -399,26 +406,26 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
 
     if (threadIdx.x == 0) {
         mbar_init(qd_full, 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < RING; ++s) {
             mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1);
             mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1);
-            mbar_init(s_full + 8 * s, 1); mbar_init(s_empty + 8 * s, 8);
-            mbar_init(ds_full + 8 * s, 8); mbar_init(ds_done + 8 * s, 1);
         }
+        for (int s = 0; s < 2; ++s) { mbar_init(ds_full + 8 * s, 8); mbar_init(ds_done + 8 * s, 1); }
+        for (int s = 0; s < 3; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(s_empty + 8 * s, 8); }
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
-    if (warp == 0 && lane == 0) { tma_prefetch(&tmQKV); tma_prefetch(&tmDO); }
+    if (warp == 0 && lane == 0) { tma_prefetch(&tmQKV); tma_prefetch(&tmKV64); tma_prefetch(&tmDO); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+    const uint32_t tS = tmem, tdP = tmem + 192, tdQ = tmem + 384;  // S[3] and dP[3] of 64 columns
 
     if (warp == 0) {
-        // lane 0 loads Q, dO and the K ring, lane 1 the V ring (V slots free
-        // early, after dP; K slots late, after dQ)
+        // lane 0 loads Q, dO and the K ring, lane 1 the V ring, one 64-key
+        // sub-block per stage (V slots free after dP, K slots after dQ)
         if (lane < 2) {
             const bool kl = lane == 0;
             const int xkv = kl ? (p.H + g) * HD : (p.H + p.nkv + g) * HD;
@@ -433,20 +440,20 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
                 }
             }
             int issued = 0;
-            for (int j = 0; j < nblk; ++j) {
-                const int st = j % STG;
-                const uint32_t ph = (j / STG) & 1;
+            for (int t = 0; t < nsub; ++t) {
+                const int st = t % RING;
+                const uint32_t ph = (t / RING) & 1;
                 if (!mbar_wait(empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(full + 8 * st, TILE);
+                mbar_expect_tx(full + 8 * st, HTILE);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb)
-                    tma_load_2d(dst + st * TILE + kb * 16384, &tmQKV, xkv + kb * 64, row0 + j * 128, full + 8 * st);
-                issued = j + 1;
+                    tma_load_2d(dst + st * HTILE + kb * 8192, &tmKV64, xkv + kb * 64, row0 + t * 64, full + 8 * st);
+                issued = t + 1;
             }
             if (*abort_flag) {
                 if (kl) drain(qd_full, 0);
-                for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j)
-                    drain(full + 8 * (j % STG), (j / STG) & 1);
+                for (int t = (issued > RING ? issued - RING : 0); t < issued; ++t)
+                    drain(full + 8 * (t % RING), (t / RING) & 1);
             }
         }
     } else if (warp == 1) {
@@ -454,38 +461,37 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
             const uint32_t id_s = idesc_bf16(128, 64, false, false);
             const uint32_t id_q = idesc_bf16(128, HD, false, true);
             if (mbar_wait(qd_full, 0, abort_flag, p.status)) {
-                for (int t = 0; t <= nsub; ++t) {
+                for (int t = 0; t <= nsub + 1; ++t) {
                     if (t < nsub) {
-                        const int j = t >> 1, hf = t & 1, st = j % STG, sb = t & 1;
-                        if (hf == 0) {
-                            if (!mbar_wait(k_full + 8 * st, (j / STG) & 1, abort_flag, p.status)) break;
-                            if (!mbar_wait(v_full + 8 * st, (j / STG) & 1, abort_flag, p.status)) break;
-                        }
-                        if (!mbar_wait(s_empty + 8 * sb, ((t >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+                        const int st = t % RING, sb = t % 3;
+                        const uint32_t ph = (t / RING) & 1;
+                        if (!mbar_wait(k_full + 8 * st, ph, abort_flag, p.status)) break;
+                        if (!mbar_wait(v_full + 8 * st, ph, abort_flag, p.status)) break;
+                        if (!mbar_wait(s_empty + 8 * sb, ((t / 3) & 1) ^ 1, abort_flag, p.status)) break;
                         tc_fence_after();
 #pragma unroll
                         for (int ks = 0; ks < HD / 16; ++ks) {
                             const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            const uint32_t offk = st * TILE + (ks >> 2) * 16384 + hf * 8192 + (ks & 3) * 32;
+                            const uint32_t offk = st * HTILE + (ks >> 2) * 8192 + (ks & 3) * 32;
                             mma_bf16(tS + sb * 64, smem_desc(sQ + off, 16, 1024), smem_desc(sK + offk, 16, 1024), id_s,
                                      ks > 0 ? 1u : 0u);
                             mma_bf16(tdP + sb * 64, smem_desc(sDO + off, 16, 1024), smem_desc(sV + offk, 16, 1024),
                                      id_s, ks > 0 ? 1u : 0u);
                         }
                         mma_commit(s_full + 8 * sb);
-                        if (hf == 1) mma_commit(v_empty + 8 * st);
+                        mma_commit(v_empty + 8 * st);
                     }
-                    if (t > 0) {
-                        const int tt = t - 1, jj = tt >> 1, hh = tt & 1, st = jj % STG, db = tt & 1;
+                    if (t > 1) {
+                        const int tt = t - 2, st = tt % RING, db = tt & 1;
                         if (!mbar_wait(ds_full + 8 * db, (tt >> 1) & 1, abort_flag, p.status)) break;
                         tc_fence_after();
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks)
                             mma_bf16(tdQ, smem_desc(sDS + db * 16384 + ks * 32, 16, 1024),
-                                     smem_desc(sK + st * TILE + hh * 8192 + ks * 2048, 16384, 1024), id_q,
+                                     smem_desc(sK + st * HTILE + ks * 2048, 8192, 1024), id_q,
                                      (tt > 0 || ks > 0) ? 1u : 0u);
                         mma_commit(ds_done + 8 * db);
-                        if (hh == 1) mma_commit(k_empty + 8 * st);
+                        mma_commit(k_empty + 8 * st);
                     }
                 }
             }
@@ -502,8 +508,8 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
         const float Dr = live ? p.D[si] : 0.f;
         bool ok = true;
         for (int t = 0; t < nsub; ++t) {
-            const int j = t >> 1, hf = t & 1, sb = t & 1;
-            if (!warp_wait(s_full + 8 * sb, (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            const int j = t >> 1, hf = t & 1, sb = t % 3, db = t & 1;
+            if (!warp_wait(s_full + 8 * sb, (t / 3) & 1, abort_flag, p.status)) { ok = false; break; }
             tc_fence_after();
             float d0[32];
             {
@@ -525,9 +531,9 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_empty + 8 * sb);
-            // dS buffer sb was last read by the dQ MMAs of sub-block t-2
-            if (t > 1 && !warp_wait(ds_done + 8 * sb, ((t >> 1) - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            uint8_t* drow = smem + Lay::DS + sb * 16384 + r * 128;
+            // dS buffer db was last read by the dQ MMAs of sub-block t-2
+            if (t > 1 && !warp_wait(ds_done + 8 * db, ((t >> 1) - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            uint8_t* drow = smem + Lay::DS + db * 16384 + r * 128;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const float* v = d0 + 8 * k;
@@ -538,7 +544,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(ds_full + 8 * sb);
+            if (lane == 0) mbar_arrive(ds_full + 8 * db);
         }
         if (ok && warp_wait(ds_done + 8 * ((nsub - 1) & 1), ((nsub - 1) >> 1) & 1, abort_flag, p.status)) {
             tc_fence_after();
@@ -581,7 +587,9 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
 
 // dK / dV, one CTA per (key block of 128, kv head, batch row): loops over the
 // units (query block of 64, query head of this kv group) that can see the
-// key block, in a fixed order (deterministic, no atomics).  Per unit, with
+// key block, in a fixed order (deterministic, no atomics): query blocks from
+// the last one down, so the CTAs of all key blocks of a batch row read the
+// same Q / dO tiles at about the same time and hit them in L2.  Per unit, with
 // the key row as the MMA M dimension: S^T = K Q^T and dP^T = V dO^T into
 // double-buffered TMEM; per key row (one per thread) P^T with the causal
 // mask and dS^T = P^T (dP^T - D) as bf16 into shared memory; dV += P^T dO and
@@ -673,7 +681,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             int issued = 0;
             for (int u = 0; u < nunits; ++u) {
                 const int st = u % DKV_STG;
-                const int i = i0 + u / Hg, h = g * Hg + u % Hg;
+                const int i = nq64 - 1 - u / Hg, h = g * Hg + u % Hg;  // last query block first
                 if (!mbar_wait(qo_empty + 8 * st, ((u / DKV_STG) & 1) ^ 1, abort_flag, p.status)) break;
                 mbar_expect_tx(qo_full + 8 * st, 2 * HTILE + 512);
                 const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + (size_t)i * 64;
@@ -744,7 +752,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         bool ok = true;
         for (int u = 0; u < nunits; ++u) {
             const int sb = u & 1, st = u % DKV_STG;
-            const int i = i0 + u / Hg;
+            const int i = nq64 - 1 - u / Hg;
             if (!warp_wait(st_full + 8 * sb, (u >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
             // this unit's Q/dO/lse/D stage has landed (the phase cannot move on
             // before this warp finishes the unit, which frees the stage)
@@ -899,7 +907,8 @@ int fwd_launch(const CUtensorMap& map, const AttnParams& p, cudaStream_t s) {
 }
 
 template <int HD>
-int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
+int dq_launch(const CUtensorMap& kv, const CUtensorMap& kv64, const CUtensorMap& do128, const BwdParams& p,
+              cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(attn_dq_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -907,7 +916,7 @@ int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& 
             return -1;
         attr = true;
     }
-    attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NTB, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
+    attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NTB, DqLayout<HD>::BYTES, s>>>(kv, kv64, do128, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -964,8 +973,9 @@ int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const fl
     if (!attention_tc_bwd_supported(hd)) return 1;
     if (!aligned16(qkv) || !aligned16(o) || !aligned16(dO) || !aligned16(dqkv) || B > 65535 || H > 65535) return 1;
     const int Nqkv = (H + 2 * nkv) * hd;
-    CUtensorMap kv, do128;
-    if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128))
+    CUtensorMap kv, kv64, do128;
+    if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&kv64, qkv, Nqkv, (uint64_t)B * T, 64) ||
+        !map_rows(&do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128))
         return 1;
     if (launch_attention_bwd_dot(DT_BF16, o, dO, Dbuf, B, T, H, hd, s) != cudaSuccess) return -1;
     BwdParams p = bwd_params(lse, Dbuf, dqkv, B, T, H, nkv, hd, status);
@@ -973,7 +983,7 @@ int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const fl
         p.qkv = reinterpret_cast<const bf16*>(qkv);
         p.rqk = fuse->rqk; p.cos_t = fuse->cos_t; p.sin_t = fuse->sin_t;
     }
-    return hd == 128 ? dq_launch<128>(kv, do128, p, s) : dq_launch<64>(kv, do128, p, s);
+    return hd == 128 ? dq_launch<128>(kv, kv64, do128, p, s) : dq_launch<64>(kv, kv64, do128, p, s);
 }
 
 int attention_tc_bwd_dkv(const void* qkv, const void* dO, const float* lse, const float* Dbuf, void* dqkv, int B,
