@@ -27,7 +27,6 @@ namespace {
 using namespace tc;
 
 constexpr int NT = 192;   // forward: producer, MMA, 4 softmax warps
-constexpr int NTB = 320;  // backward: producer, MMA, 8 softmax warps (two per TMEM lane quarter)
 constexpr int STG = 2;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
@@ -282,153 +281,157 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 
 
 // ============================================================================ backward
-// dQ, one CTA per (query block of 128, head, batch row).  Key blocks j = 0..qb
-// are processed as 64-key sub-blocks t: S_t = Q K_t^T and dP_t = dO V_t^T into
-// one of three TMEM buffers; per query row (one per thread)
-// P = 2^(S*scale*log2e - lse*log2e) with the causal mask and dS = P (dP - D),
-// as bf16 into one of two shared-memory tiles; dQ += dS_{t-2} K_{t-2} is issued
-// two sub-blocks behind (the score MMAs of two sub-blocks cover the softmax
-// round trip), with the K tile read again as an MN-major operand.
+// Both backward kernels keep every MMA at N = 128 (a 128 x 64 tile runs the
+// tensor core at well under half rate on sm_100a) and feed one operand of the
+// second product from TMEM: the softmax warps write their bf16 result back
+// over the fp32 score columns they have just read, and the MMA reads it there
+// as the A operand.  Sixteen softmax warps (four per TMEM lane quarter, 32
+// columns each) keep the special-function unit busy.
+//
+// dQ, one CTA per (query block of 128, head, batch row), key blocks j = 0..qb:
+//   warp 0      TMA: Q and dO once; K_j into a 3-stage ring (freed by the dQ
+//               MMA), V_j into a 2-stage ring (freed by the dP MMA);
+//   warp 1      tcgen05.mma: S_j = Q K_j^T into one of two TMEM buffers,
+//               dP_j = dO V_j^T into one buffer, then dQ += dS_{j-1} K_{j-1}
+//               with dS read from TMEM and K as an MN-major operand;
+//   warps 2-17  per key block: load the warp's S and dP columns, release dP,
+//               form
+//               P = 2^(S*scale*log2e - lse*log2e) with the causal mask on the
+//               diagonal block and dS = P (dP - D), and store dS as packed
+//               bf16 over the first half of the warp's own S columns.
 // dq = dQ / sqrt(hd).
+constexpr int NTB = 576;  // backward: producer, MMA, 16 softmax warps
+constexpr int NSM = 16;   // softmax warps
+
 template <int HD>
 struct DqLayout {
     static constexpr int KB = HD / 64;
-    static constexpr int TILE = KB * 16384;   // [128 x HD]: Q, dO
-    static constexpr int HTILE = KB * 8192;   // [64 x HD]: a K or V sub-block
-    static constexpr int RING = 4;            // K and V sub-block stages
+    static constexpr int TILE = KB * 16384;  // [128 x HD] bf16, 128B-swizzled: Q, dO, a K or V block
+    static constexpr int KSTG = 3, VSTG = 2;
     static constexpr int Q = 0;
     static constexpr int DO = Q + TILE;
     static constexpr int K = DO + TILE;
-    static constexpr int V = K + RING * HTILE;
-    static constexpr int DS = V + RING * HTILE;  // [2][128 x 64] bf16
-    static constexpr int BAR = DS + 32768;
-    static constexpr int BYTES = BAR + 256 + 1024;
+    static constexpr int V = K + KSTG * TILE;
+    static constexpr int BAR = V + VSTG * TILE;
+    static constexpr int BYTES = BAR + 256;  // the dynamic shared memory base is 1024-aligned (checked)
     static_assert(BYTES <= 232448, "dQ shared memory exceeds the per-block limit");
 };
 
 struct BwdParams {
     int B, T, H, nkv, nqb;
     float scale_log2, scale;
-    const float* lse;
-    const float* D;
+    const float* D;     // [B, H, Tp] rowsum(dO * o)
+    const float* lse2;  // [B, H, Tp] lse * log2(e) (both zero past the sequence end)
     bf16* dqkv;
     int* status;
-    // When rqk is set, dq and dk are written as gradients of the pre-norm
-    // projections (QK-norm and RoPE backward fused): qkv holds the saved
-    // post-RoPE vectors, rqk their inverse RMS [B*T, H+nkv], cos/sin [T, hd/2].
-    const bf16* qkv;
-    const float* rqk;
-    const float* cos_t;
-    const float* sin_t;
 };
-
-// Writes the gradient of the pre-norm projection for one head row: g = scale *
-// (the TMEM row at tsrc) is the gradient of y = rope(rmsnorm(x)); with the
-// saved y, u = R^T g and w = R^T y (inverse rotation of the pairs (j, j+HD/2))
-// give dx = r * (u - w * mean(u * w)).  Two passes over TMEM keep registers low.
-template <int HD>
-__device__ __forceinline__ void store_grad_through_qknorm(uint32_t tsrc, float scale, const bf16* y, float r,
-                                                          const float* cs, const float* sn, bf16* out, bool live) {
-    constexpr int NC = HD / 32, HALF = HD / 2;
-    float dot = 0.f;
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-        const float mdot = dot / (float)HD;
-#pragma unroll 1
-        for (int c = 0; c < NC / 2; ++c) {
-            float g1[32], g2[32];
-            tmem_ld32(tsrc + c * 32, g1);
-            tmem_ld32(tsrc + (c + NC / 2) * 32, g2);
-            if (!live) continue;
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-                float y1[8], y2[8];
-                load_vec(y + c * 32 + i, y1);
-                load_vec(y + HALF + c * 32 + i, y2);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = c * 32 + i + e;
-                    const float co = cs[j], si = sn[j];
-                    const float a = g1[i + e] * scale, b = g2[i + e] * scale;
-                    const float u1 = a * co + b * si, u2 = b * co - a * si;
-                    const float w1 = y1[e] * co + y2[e] * si, w2 = y2[e] * co - y1[e] * si;
-                    if (pass == 0) {
-                        dot += u1 * w1 + u2 * w2;
-                    } else {
-                        g1[i + e] = r * (u1 - w1 * mdot);
-                        g2[i + e] = r * (u2 - w2 * mdot);
-                    }
-                }
-            }
-            if (pass == 1) {
-#pragma unroll
-                for (int t4 = 0; t4 < 4; ++t4) {
-                    store_vec(out + c * 32 + 8 * t4, g1 + 8 * t4);
-                    store_vec(out + HALF + c * 32 + 8 * t4, g2 + 8 * t4);
-                }
-            }
-        }
-    }
-}
 
 __device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
     uint64_t t0 = globaltimer();
     while (!mbar_try(bar, parity) && globaltimer() - t0 < 1000000ull) {}
 }
 
+// sum of the products of two vectors of eight bf16
+__device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
+    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 u = __bfloat1622float2(x[i]), v = __bfloat1622float2(y[i]);
+        s = fmaf(u.x, v.x, s);
+        s = fmaf(u.y, v.y, s);
+    }
+    return s;
+}
+
+// D = rowsum(dO * o) and lse * log2(e) for every (batch row b, head h, position t
+// < Tp), head-major [B, H, Tp], zero past the end of the sequence: HD/8 threads
+// per entry, each with one 16-byte vector of o and dO.
+template <int HD>
+__global__ void __launch_bounds__(256) attn_bwd_stats_kernel(const bf16* __restrict__ o, const bf16* __restrict__ dO,
+                                                             const float* __restrict__ lse, float* __restrict__ D,
+                                                             float* __restrict__ lse2, int B, int T, int H) {
+    constexpr int G = HD / 8;
+    const int Tp = attn_tpad(T);
+    const long long n = (long long)B * H * Tp;
+    const long long w = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / G;
+    const int k = threadIdx.x % G;
+    const int t = (int)(w % Tp);
+    const long long bh = w / Tp;
+    const bool live = w < n && t < T;
+    float s = 0.f;
+    if (live) {
+        const long long row = (bh / H) * T + t;
+        const size_t off = ((size_t)row * H + (size_t)(bh % H)) * HD + 8 * k;
+        s = dot8(*reinterpret_cast<const uint4*>(o + off), *reinterpret_cast<const uint4*>(dO + off));
+    }
+#pragma unroll
+    for (int m = G / 2; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+    if (w < n && k == 0) {
+        D[w] = s;
+        lse2[w] = live ? lse[w] * kLog2e : 0.f;
+    }
+}
+
 template <int HD>
 __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
-                                                           const __grid_constant__ CUtensorMap tmKV64,
                                                            const __grid_constant__ CUtensorMap tmDO,
                                                            const BwdParams p) {
     using Lay = DqLayout<HD>;
-    constexpr int KB = Lay::KB, TILE = Lay::TILE, HTILE = Lay::HTILE, RING = Lay::RING;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    constexpr int KB = Lay::KB, TILE = Lay::TILE, KSTG = Lay::KSTG, VSTG = Lay::VSTG;
+    extern __shared__ __align__(1024) uint8_t smem_dyn[];
+    if ((smem_u32(smem_dyn) & 1023u) != 0) {
+        if (threadIdx.x == 0) set_status(p.status, ST_BAD_LAYOUT);
+        return;
+    }
+    uint8_t* smem = smem_dyn;
     const uint32_t base = smem_u32(smem);
     const uint32_t sQ = base + Lay::Q, sDO = base + Lay::DO, sK = base + Lay::K, sV = base + Lay::V;
-    const uint32_t sDS = base + Lay::DS;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t qd_full = b0;
-    const uint32_t k_full = b0 + 8, k_empty = b0 + 40, v_full = b0 + 72, v_empty = b0 + 104;  // [RING]
-    const uint32_t s_full = b0 + 136, s_empty = b0 + 160;  // [3]: S/dP TMEM buffers
-    const uint32_t ds_full = b0 + 184, ds_done = b0 + 200; // [2]: dS smem tiles
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
+    const uint32_t k_full = b0 + 8, k_empty = b0 + 32;   // [KSTG]
+    const uint32_t v_full = b0 + 56, v_empty = b0 + 72;  // [VSTG]
+    const uint32_t s_full = b0 + 88;                     // [2]: S_j landed in TMEM buffer j & 1
+    const uint32_t dp_full = b0 + 104, dp_free = b0 + 112;
+    const uint32_t ds_full = b0 + 120;                   // [2]: dS_j written over buffer j & 1
+    const uint32_t dq_done = b0 + 136;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qb = p.nqb - 1 - (int)blockIdx.z;  // longest blocks launch first
     const int h = blockIdx.x, b = blockIdx.y, g = h / (p.H / p.nkv);
-    const int nblk = qb + 1, nsub = 2 * nblk;
+    const int nblk = qb + 1;
     const int row0 = b * p.T;
     const int Nqkv = (p.H + 2 * p.nkv) * HD;
 
     if (threadIdx.x == 0) {
         mbar_init(qd_full, 1);
-        for (int s = 0; s < RING; ++s) {
-            mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1);
-            mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1);
-        }
-        for (int s = 0; s < 2; ++s) { mbar_init(ds_full + 8 * s, 8); mbar_init(ds_done + 8 * s, 1); }
-        for (int s = 0; s < 3; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(s_empty + 8 * s, 8); }
+        for (int s = 0; s < KSTG; ++s) { mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1); }
+        for (int s = 0; s < VSTG; ++s) { mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1); }
+        for (int s = 0; s < 2; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(ds_full + 8 * s, NSM); }
+        mbar_init(dp_full, 1);
+        mbar_init(dp_free, NSM);
+        mbar_init(dq_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
-    if (warp == 0 && lane == 0) { tma_prefetch(&tmQKV); tma_prefetch(&tmKV64); tma_prefetch(&tmDO); }
+    if (warp == 0 && lane == 0) { tma_prefetch(&tmQKV); tma_prefetch(&tmDO); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tdP = tmem + 192, tdQ = tmem + 384;  // S[3] and dP[3] of 64 columns
+    const uint32_t tS = tmem, tdP = tmem + 256, tdQ = tmem + 384;  // S[2] of 128 columns, dP, dQ
 
     if (warp == 0) {
-        // lane 0 loads Q, dO and the K ring, lane 1 the V ring, one 64-key
-        // sub-block per stage (V slots free after dP, K slots after dQ)
+        // lane 0 loads Q, dO and the K ring, lane 1 the V ring
         if (lane < 2) {
             const bool kl = lane == 0;
-            const int xkv = kl ? (p.H + g) * HD : (p.H + p.nkv + g) * HD;
+            const int xkv = (kl ? p.H + g : p.H + p.nkv + g) * HD;
+            const int nst = kl ? KSTG : VSTG;
             const uint32_t full = kl ? k_full : v_full, empty = kl ? k_empty : v_empty;
             const uint32_t dst = kl ? sK : sV;
             if (kl) {
@@ -440,139 +443,135 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
                 }
             }
             int issued = 0;
-            for (int t = 0; t < nsub; ++t) {
-                const int st = t % RING;
-                const uint32_t ph = (t / RING) & 1;
-                if (!mbar_wait(empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(full + 8 * st, HTILE);
+            for (int j = 0; j < nblk; ++j) {
+                const int st = j % nst;
+                if (!mbar_wait(empty + 8 * st, ((j / nst) & 1) ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(full + 8 * st, TILE);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb)
-                    tma_load_2d(dst + st * HTILE + kb * 8192, &tmKV64, xkv + kb * 64, row0 + t * 64, full + 8 * st);
-                issued = t + 1;
+                    tma_load_2d(dst + st * TILE + kb * 16384, &tmQKV, xkv + kb * 64, row0 + j * 128, full + 8 * st);
+                issued = j + 1;
             }
             if (*abort_flag) {
                 if (kl) drain(qd_full, 0);
-                for (int t = (issued > RING ? issued - RING : 0); t < issued; ++t)
-                    drain(full + 8 * (t % RING), (t / RING) & 1);
+                for (int j = (issued > nst ? issued - nst : 0); j < issued; ++j) drain(full + 8 * (j % nst), (j / nst) & 1);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id_s = idesc_bf16(128, 64, false, false);
+            const uint32_t id_s = idesc_bf16(128, 128, false, false);
             const uint32_t id_q = idesc_bf16(128, HD, false, true);
-            if (mbar_wait(qd_full, 0, abort_flag, p.status)) {
-                for (int t = 0; t <= nsub + 1; ++t) {
-                    if (t < nsub) {
-                        const int st = t % RING, sb = t % 3;
-                        const uint32_t ph = (t / RING) & 1;
-                        if (!mbar_wait(k_full + 8 * st, ph, abort_flag, p.status)) break;
-                        if (!mbar_wait(v_full + 8 * st, ph, abort_flag, p.status)) break;
-                        if (!mbar_wait(s_empty + 8 * sb, ((t / 3) & 1) ^ 1, abort_flag, p.status)) break;
-                        tc_fence_after();
+            bool ok = mbar_wait(qd_full, 0, abort_flag, p.status);
+            for (int j = 0; ok && j <= nblk; ++j) {
+                if (j < nblk) {
+                    const int kst = j % KSTG, vst = j % VSTG, sb = j & 1;
+                    if (!mbar_wait(k_full + 8 * kst, (j / KSTG) & 1, abort_flag, p.status)) break;
+                    tc_fence_after();
 #pragma unroll
-                        for (int ks = 0; ks < HD / 16; ++ks) {
-                            const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            const uint32_t offk = st * HTILE + (ks >> 2) * 8192 + (ks & 3) * 32;
-                            mma_bf16(tS + sb * 64, smem_desc(sQ + off, 16, 1024), smem_desc(sK + offk, 16, 1024), id_s,
-                                     ks > 0 ? 1u : 0u);
-                            mma_bf16(tdP + sb * 64, smem_desc(sDO + off, 16, 1024), smem_desc(sV + offk, 16, 1024),
-                                     id_s, ks > 0 ? 1u : 0u);
-                        }
-                        mma_commit(s_full + 8 * sb);
-                        mma_commit(v_empty + 8 * st);
+                    for (int ks = 0; ks < HD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16(tS + sb * 128, smem_desc(sQ + off, 16, 1024),
+                                 smem_desc(sK + kst * TILE + off, 16, 1024), id_s, ks > 0 ? 1u : 0u);
                     }
-                    if (t > 1) {
-                        const int tt = t - 2, st = tt % RING, db = tt & 1;
-                        if (!mbar_wait(ds_full + 8 * db, (tt >> 1) & 1, abort_flag, p.status)) break;
-                        tc_fence_after();
+                    mma_commit(s_full + 8 * sb);
+                    if (!mbar_wait(v_full + 8 * vst, (j / VSTG) & 1, abort_flag, p.status)) break;
+                    // the softmax warps have read dP_{j-1} out of TMEM
+                    if (j > 0 && !mbar_wait(dp_free, (j - 1) & 1, abort_flag, p.status)) break;
+                    tc_fence_after();
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            mma_bf16(tdQ, smem_desc(sDS + db * 16384 + ks * 32, 16, 1024),
-                                     smem_desc(sK + st * HTILE + ks * 2048, 8192, 1024), id_q,
-                                     (tt > 0 || ks > 0) ? 1u : 0u);
-                        mma_commit(ds_done + 8 * db);
-                        mma_commit(k_empty + 8 * st);
+                    for (int ks = 0; ks < HD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        mma_bf16(tdP, smem_desc(sDO + off, 16, 1024), smem_desc(sV + vst * TILE + off, 16, 1024),
+                                 id_s, ks > 0 ? 1u : 0u);
                     }
+                    mma_commit(dp_full);
+                    mma_commit(v_empty + 8 * vst);
+                }
+                if (j > 0) {
+                    // dQ += dS_{j-1} K_{j-1}: keys 16kk..16kk+15 sit in the packed columns
+                    // 32*(kk/2) + 8*(kk%2) of the S buffer (written by column group kk/2)
+                    const int jj = j - 1, sb = jj & 1;
+                    if (!mbar_wait(ds_full + 8 * sb, (jj >> 1) & 1, abort_flag, p.status)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tdQ, tS + sb * 128 + 32 * (kk >> 1) + 8 * (kk & 1),
+                                    smem_desc(sK + (jj % KSTG) * TILE + kk * 2048, 16384, 1024), id_q,
+                                    (jj > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(k_empty + 8 * (jj % KSTG));
                 }
             }
+            mma_commit(dq_done);
         }
     } else {
-        // warps 2..9: TMEM lane quarter q = warp % 4 (query rows), key half ch of each sub-block
-        const int q = warp & 3, ch = (warp - 2) >> 2;
+        // warps 2..17: TMEM lane quarter q (query rows), key column group cg (32 keys)
+        const int q = warp & 3, cg = (warp - 2) >> 2;
         const int r = q * 32 + lane;
         const int qpos = qb * 128 + r;
         const bool live = qpos < p.T;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + (live ? qpos : 0);
-        const float lse2 = live ? p.lse[si] * kLog2e : 0.f;
-        const float Dr = live ? p.D[si] : 0.f;
+        const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + qpos;
+        const float Dr = p.D[si], lse2 = p.lse2[si];
         bool ok = true;
-        for (int t = 0; t < nsub; ++t) {
-            const int j = t >> 1, hf = t & 1, sb = t % 3, db = t & 1;
-            if (!warp_wait(s_full + 8 * sb, (t / 3) & 1, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
-            float d0[32];
-            {
-                float sv[32];
-                {
-                    uint32_t rs[32], rd[32];
-                    tmem_ld32_issue(tS + lane_off + sb * 64 + ch * 32, rs);
-                    tmem_ld32_issue(tdP + lane_off + sb * 64 + ch * 32, rd);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(rs[i]); d0[i] = __uint_as_float(rd[i]); }
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const bool valid = live && (j < qb || hf * 64 + ch * 32 + i <= r);
-                    d0[i] = valid ? ex2(sv[i] * p.scale_log2 - lse2) * (d0[i] - Dr) : 0.f;
-                }
+        for (int j = 0; j < nblk; ++j) {
+            const int sb = j & 1;
+            if (!warp_wait(s_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status) ||
+                !warp_wait(dp_full, j & 1, abort_flag, p.status)) {
+                ok = false;
+                break;
             }
+            tc_fence_after();
+            uint32_t rs[32], rd[32];
+            tmem_ld32_issue(tS + lane_off + sb * 128 + cg * 32, rs);
+            tmem_ld32_issue(tdP + lane_off + cg * 32, rd);
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty + 8 * sb);
-            // dS buffer db was last read by the dQ MMAs of sub-block t-2
-            if (t > 1 && !warp_wait(ds_done + 8 * db, ((t >> 1) - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            uint8_t* drow = smem + Lay::DS + db * 16384 + r * 128;
+            if (lane == 0) mbar_arrive(dp_free);
+            // keys j*128 + cg*32 + e, e <= lim, are visible from this row
+            const int lim = !live ? -1 : (j == qb ? r - cg * 32 : 31);
+            uint32_t pk[16];
+            if (__all_sync(0xffffffffu, lim >= 31)) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float* v = d0 + 8 * k;
-                const int c8 = ch * 4 + k;
-                *reinterpret_cast<uint4*>(drow + ((c8 ^ (r & 7)) << 4)) =
-                    make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                               pack_bf16(v[6], v[7]));
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ds_full + 8 * db);
-        }
-        if (ok && warp_wait(ds_done + 8 * ((nsub - 1) & 1), ((nsub - 1) >> 1) & 1, abort_flag, p.status)) {
-            tc_fence_after();
-            bf16* out = p.dqkv + ((size_t)row0 + qpos) * Nqkv + h * HD;
-            if (p.rqk) {
-                // the first four softmax warps write whole rows through the QK-norm backward
-                if (ch == 0) {
-                    const size_t rowi = (size_t)row0 + (live ? qpos : 0);
-                    const int pos = live ? qpos : 0;
-                    store_grad_through_qknorm<HD>(tdQ + lane_off, p.scale, p.qkv + rowi * Nqkv + h * HD,
-                                                  live ? p.rqk[rowi * (p.H + p.nkv) + h] : 0.f,
-                                                  p.cos_t + (size_t)pos * (HD / 2), p.sin_t + (size_t)pos * (HD / 2),
-                                                  out, live);
+                for (int e = 0; e < 32; e += 2) {
+                    const float d0 = ex2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -lse2)) *
+                                     (__uint_as_float(rd[e]) - Dr);
+                    const float d1 = ex2(fmaf(__uint_as_float(rs[e + 1]), p.scale_log2, -lse2)) *
+                                     (__uint_as_float(rd[e + 1]) - Dr);
+                    pk[e >> 1] = pack_bf16(d0, d1);
                 }
-            } else
+            } else {
 #pragma unroll
-            for (int cc = 0; cc < HD / 64; ++cc) {
-                const int c = ch * (HD / 64) + cc;
-                float o[32];
-                tmem_ld32(tdQ + lane_off + c * 32, o);
+                for (int e = 0; e < 32; e += 2) {
+                    const float d0 = e <= lim ? ex2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -lse2)) *
+                                                    (__uint_as_float(rd[e]) - Dr)
+                                              : 0.f;
+                    const float d1 = e + 1 <= lim ? ex2(fmaf(__uint_as_float(rs[e + 1]), p.scale_log2, -lse2)) *
+                                                        (__uint_as_float(rd[e + 1]) - Dr)
+                                                  : 0.f;
+                    pk[e >> 1] = pack_bf16(d0, d1);
+                }
+            }
+            tmem_st16(tS + lane_off + sb * 128 + cg * 32, pk);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ds_full + 8 * sb);
+        }
+        if (ok && warp_wait(dq_done, 0, abort_flag, p.status)) {
+            tc_fence_after();
+            // column group cg writes dq columns 32*cg .. 32*cg+31 (hd 64: groups 0 and 1)
+            if (cg * 32 < HD) {
+                float v[32];
+                tmem_ld32(tdQ + lane_off + cg * 32, v);
                 if (live) {
+                    bf16* out = p.dqkv + ((size_t)row0 + qpos) * Nqkv + h * HD + cg * 32;
 #pragma unroll
-                    for (int t4 = 0; t4 < 4; ++t4)
-                        *reinterpret_cast<uint4*>(out + c * 32 + 8 * t4) = make_uint4(
-                            pack_bf16(o[8 * t4] * p.scale, o[8 * t4 + 1] * p.scale),
-                            pack_bf16(o[8 * t4 + 2] * p.scale, o[8 * t4 + 3] * p.scale),
-                            pack_bf16(o[8 * t4 + 4] * p.scale, o[8 * t4 + 5] * p.scale),
-                            pack_bf16(o[8 * t4 + 6] * p.scale, o[8 * t4 + 7] * p.scale));
+                    for (int e = 0; e < 4; ++e)
+                        *reinterpret_cast<uint4*>(out + 8 * e) =
+                            make_uint4(pack_bf16(v[8 * e] * p.scale, v[8 * e + 1] * p.scale),
+                                       pack_bf16(v[8 * e + 2] * p.scale, v[8 * e + 3] * p.scale),
+                                       pack_bf16(v[8 * e + 4] * p.scale, v[8 * e + 5] * p.scale),
+                                       pack_bf16(v[8 * e + 6] * p.scale, v[8 * e + 7] * p.scale));
                 }
             }
         }
@@ -585,59 +584,61 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
     }
 }
 
-// dK / dV, one CTA per (key block of 128, kv head, batch row): loops over the
-// units (query block of 64, query head of this kv group) that can see the
-// key block, in a fixed order (deterministic, no atomics): query blocks from
-// the last one down, so the CTAs of all key blocks of a batch row read the
-// same Q / dO tiles at about the same time and hit them in L2.  Per unit, with
-// the key row as the MMA M dimension: S^T = K Q^T and dP^T = V dO^T into
-// double-buffered TMEM; per key row (one per thread) P^T with the causal
-// mask and dS^T = P^T (dP^T - D) as bf16 into shared memory; dV += P^T dO and
-// dK += dS^T Q accumulate in TMEM over all units.  dk = dK / sqrt(hd).
-constexpr int DKV_STG = 3;  // Q/dO/lse/D stages of the dK/dV kernel
-
+// dK / dV, one CTA per (key block of 128, K/V head, batch row).  Units are
+// (query block i of 128, query head h of the group), the last query block
+// first, so the CTAs of all key blocks of a batch row read the same Q / dO
+// tiles at about the same time and find them in L2:
+//   warp 0      TMA: K and V once; Q_i, dO_i with their lse2 / D rows into a
+//               2-stage ring;
+//   warp 1      tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM,
+//               dV += P^T dO_i with P^T read from TMEM, dK += dS^T Q_i with
+//               dS^T from shared memory (Q_i, dO_i as MN-major operands),
+//               in the order dV_u, S^T_{u+1}, dP^T_{u+1}, dK_u so the next
+//               unit's scores run while the softmax warps finish dS^T_u;
+//   warps 2-17  per unit: load the warp's S^T and dP^T columns (32 queries),
+//               release dP^T, form P^T = 2^(S^T*scale*log2e - lse2) with the
+//               causal mask and store it as packed bf16 over its own S^T
+//               columns, then dS^T = P^T (dP^T - D) into shared memory.
+// dk = dK / sqrt(hd).
 template <int HD>
 struct DkvLayout {
     static constexpr int KB = HD / 64;
-    static constexpr int TILE = KB * 16384;   // [128 x HD]
-    static constexpr int HTILE = KB * 8192;   // [64 x HD]
+    static constexpr int TILE = KB * 16384;    // [128 x HD] bf16
     static constexpr int K = 0;
     static constexpr int V = K + TILE;
-    static constexpr int Q = V + TILE;
-    static constexpr int DO = Q + DKV_STG * HTILE;
-    static constexpr int PT = DO + DKV_STG * HTILE;  // [2][128 x 64] bf16, by unit parity
-    static constexpr int DST = PT + 2 * 16384;       // [2][128 x 64] bf16, by unit parity
-    static constexpr int LSE = DST + 2 * 16384;      // [DKV_STG][64] floats: lse of the unit's queries
-    static constexpr int DD = LSE + DKV_STG * 256;   // [DKV_STG][64] floats: D of the unit's queries
-    static constexpr int BAR = DD + DKV_STG * 256;
-    static constexpr int BYTES = BAR + 256 + 1024;
+    static constexpr int Q = V + TILE;         // [2] stages
+    static constexpr int DO = Q + 2 * TILE;    // [2] stages
+    static constexpr int DST = DO + 2 * TILE;  // dS^T [128 keys x 128 queries] bf16, two 64-query boxes
+    static constexpr int LSE = DST + 32768;    // [2][128] fp32 lse2 of the stage's queries
+    static constexpr int DD = LSE + 1024;      // [2][128] fp32 D
+    static constexpr int BAR = DD + 1024;
+    static constexpr int BYTES = BAR + 256;  // the dynamic shared memory base is 1024-aligned (checked)
     static_assert(BYTES <= 232448, "dK/dV shared memory exceeds the per-block limit");
 };
 
 template <int HD>
-__global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmKV,
-                                                            const __grid_constant__ CUtensorMap tmQ64,
-                                                            const __grid_constant__ CUtensorMap tmDO64,
+__global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
+                                                            const __grid_constant__ CUtensorMap tmDO,
                                                             const BwdParams p) {
     using Lay = DkvLayout<HD>;
-    constexpr int KB = Lay::KB, TILE = Lay::TILE, HTILE = Lay::HTILE;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    constexpr int KB = Lay::KB, TILE = Lay::TILE;
+    extern __shared__ __align__(1024) uint8_t smem_dyn[];
+    if ((smem_u32(smem_dyn) & 1023u) != 0) {
+        if (threadIdx.x == 0) set_status(p.status, ST_BAD_LAYOUT);
+        return;
+    }
+    uint8_t* smem = smem_dyn;
     const uint32_t base = smem_u32(smem);
     const uint32_t sK = base + Lay::K, sV = base + Lay::V, sQ = base + Lay::Q, sDO = base + Lay::DO;
-    const uint32_t sPT = base + Lay::PT, sDST = base + Lay::DST;
-    float* lse_s = reinterpret_cast<float*>(smem + Lay::LSE);
-    float* d_s = reinterpret_cast<float*>(smem + Lay::DD);
+    const uint32_t sDST = base + Lay::DST;
+    const float* lse_s = reinterpret_cast<const float*>(smem + Lay::LSE);
+    const float* d_s = reinterpret_cast<const float*>(smem + Lay::DD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
-    const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 32;  // qo_*[DKV_STG]
-    const uint32_t st_full = b0 + 56, st_empty = b0 + 72;              // [2]
-    // pd_full[b] / pd_done[b]: P^T and dS^T of the units with parity b written /
-    // consumed (once per two units each).  Per-parity barriers keep every wait
-    // from being lapped: the softmax warps may run two units ahead of the MMA
-    // thread's wait on pd_full.
-    const uint32_t pd_full = b0 + 88, pd_done = b0 + 104;              // [2] each
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24;  // qo_*[2]
+    const uint32_t st_full = b0 + 40, dpt_full = b0 + 48, dpt_free = b0 + 56;
+    const uint32_t p_full = b0 + 64, ds_full = b0 + 72, ds_free = b0 + 80, dkv_done = b0 + 88;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -646,23 +647,23 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
     const int Hg = p.H / p.nkv;
     const int row0 = b * p.T;
     const int Nqkv = (p.H + 2 * p.nkv) * HD;
-    const int nq64 = (p.T + 63) / 64;
-    const int i0 = 2 * kvb;
-    const int nunits = (nq64 - i0) * Hg;
+    const int nunits = (p.nqb - kvb) * Hg;
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
-        for (int s = 0; s < DKV_STG; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(st_full + 8 * s, 1); mbar_init(st_empty + 8 * s, 8); }
-        mbar_init(pd_full, 8);
-        mbar_init(pd_full + 8, 8);
-        mbar_init(pd_done, 1);
-        mbar_init(pd_done + 8, 1);
+        for (int s = 0; s < 2; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
+        mbar_init(st_full, 1);
+        mbar_init(dpt_full, 1);
+        mbar_init(dpt_free, NSM);
+        mbar_init(p_full, NSM);
+        mbar_init(ds_full, NSM);
+        mbar_init(ds_free, 1);
+        mbar_init(dkv_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
-    if (warp == 0 && lane == 0) { tma_prefetch(&tmKV); tma_prefetch(&tmQ64); tma_prefetch(&tmDO64); }
+    if (warp == 0 && lane == 0) { tma_prefetch(&tmQKV); tma_prefetch(&tmDO); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -675,173 +676,194 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             mbar_expect_tx(kv_full, 2 * TILE);
 #pragma unroll
             for (int kb = 0; kb < KB; ++kb) {
-                tma_load_2d(sK + kb * 16384, &tmKV, xk + kb * 64, row0 + kvb * 128, kv_full);
-                tma_load_2d(sV + kb * 16384, &tmKV, xv + kb * 64, row0 + kvb * 128, kv_full);
+                tma_load_2d(sK + kb * 16384, &tmQKV, xk + kb * 64, row0 + kvb * 128, kv_full);
+                tma_load_2d(sV + kb * 16384, &tmQKV, xv + kb * 64, row0 + kvb * 128, kv_full);
             }
             int issued = 0;
             for (int u = 0; u < nunits; ++u) {
-                const int st = u % DKV_STG;
-                const int i = nq64 - 1 - u / Hg, h = g * Hg + u % Hg;  // last query block first
-                if (!mbar_wait(qo_empty + 8 * st, ((u / DKV_STG) & 1) ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(qo_full + 8 * st, 2 * HTILE + 512);
-                const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + (size_t)i * 64;
-                bulk_load(base + Lay::LSE + st * 256, p.lse + si, 256, qo_full + 8 * st);
-                bulk_load(base + Lay::DD + st * 256, p.D + si, 256, qo_full + 8 * st);
+                const int st = u & 1;
+                const int i = p.nqb - 1 - u / Hg, h = g * Hg + u % Hg;  // last query block first
+                if (!mbar_wait(qo_empty + 8 * st, ((u >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(qo_full + 8 * st, 2 * TILE + 1024);
+                const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + (size_t)i * 128;
+                bulk_load(base + Lay::LSE + st * 512, p.lse2 + si, 512, qo_full + 8 * st);
+                bulk_load(base + Lay::DD + st * 512, p.D + si, 512, qo_full + 8 * st);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_2d(sQ + st * HTILE + kb * 8192, &tmQ64, h * HD + kb * 64, row0 + i * 64, qo_full + 8 * st);
-                    tma_load_2d(sDO + st * HTILE + kb * 8192, &tmDO64, h * HD + kb * 64, row0 + i * 64,
+                    tma_load_2d(sQ + st * TILE + kb * 16384, &tmQKV, h * HD + kb * 64, row0 + i * 128,
+                                qo_full + 8 * st);
+                    tma_load_2d(sDO + st * TILE + kb * 16384, &tmDO, h * HD + kb * 64, row0 + i * 128,
                                 qo_full + 8 * st);
                 }
                 issued = u + 1;
             }
             if (*abort_flag) {
                 drain(kv_full, 0);
-                for (int u = (issued > DKV_STG ? issued - DKV_STG : 0); u < issued; ++u)
-                    drain(qo_full + 8 * (u % DKV_STG), (u / DKV_STG) & 1);
+                for (int u = (issued > 2 ? issued - 2 : 0); u < issued; ++u) drain(qo_full + 8 * (u & 1), (u >> 1) & 1);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id_st = idesc_bf16(128, 64, false, false);
+            const uint32_t id_s = idesc_bf16(128, 128, false, false);
             const uint32_t id_kv = idesc_bf16(128, HD, false, true);
-            if (mbar_wait(kv_full, 0, abort_flag, p.status)) {
-                for (int u = 0; u <= nunits; ++u) {
-                    if (u < nunits) {
-                        const int st = u % DKV_STG, sb = u & 1;
-                        if (!mbar_wait(qo_full + 8 * st, (u / DKV_STG) & 1, abort_flag, p.status)) break;
-                        if (!mbar_wait(st_empty + 8 * sb, ((u >> 1) & 1) ^ 1, abort_flag, p.status)) break;
-                        tc_fence_after();
+            // S^T_u = K Q_u^T and dP^T_u = V dO_u^T
+            auto scores = [&](int u) -> bool {
+                const int st = u & 1;
+                if (!mbar_wait(qo_full + 8 * st, (u >> 1) & 1, abort_flag, p.status)) return false;
+                tc_fence_after();
 #pragma unroll
-                        for (int ks = 0; ks < HD / 16; ++ks) {
-                            const uint32_t ok_ = (ks >> 2) * 16384 + (ks & 3) * 32;
-                            const uint32_t oq = (ks >> 2) * 8192 + (ks & 3) * 32;
-                            mma_bf16(tSt + sb * 64, smem_desc(sK + ok_, 16, 1024),
-                                     smem_desc(sQ + st * HTILE + oq, 16, 1024), id_st, ks > 0 ? 1u : 0u);
-                            mma_bf16(tdPt + sb * 64, smem_desc(sV + ok_, 16, 1024),
-                                     smem_desc(sDO + st * HTILE + oq, 16, 1024), id_st, ks > 0 ? 1u : 0u);
-                        }
-                        mma_commit(st_full + 8 * sb);
-                    }
-                    if (u > 0) {
-                        const int uu = u - 1, st = uu % DKV_STG;
-                        if (!mbar_wait(pd_full + 8 * (uu & 1), (uu >> 1) & 1, abort_flag, p.status)) break;
-                        tc_fence_after();
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) {
-                            const uint32_t pb = (uu & 1) * 16384 + ks * 32;
-                            mma_bf16(tdV, smem_desc(sPT + pb, 16, 1024),
-                                     smem_desc(sDO + st * HTILE + ks * 2048, 8192, 1024), id_kv,
-                                     (uu > 0 || ks > 0) ? 1u : 0u);
-                            mma_bf16(tdK, smem_desc(sDST + pb, 16, 1024),
-                                     smem_desc(sQ + st * HTILE + ks * 2048, 8192, 1024), id_kv,
-                                     (uu > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        mma_commit(pd_done + 8 * (uu & 1));
-                        mma_commit(qo_empty + 8 * st);
-                    }
+                for (int ks = 0; ks < HD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    mma_bf16(tSt, smem_desc(sK + off, 16, 1024), smem_desc(sQ + st * TILE + off, 16, 1024), id_s,
+                             ks > 0 ? 1u : 0u);
                 }
+                mma_commit(st_full);
+                // the softmax warps have read dP^T_{u-1} out of TMEM
+                if (u > 0 && !mbar_wait(dpt_free, (u - 1) & 1, abort_flag, p.status)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < HD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    mma_bf16(tdPt, smem_desc(sV + off, 16, 1024), smem_desc(sDO + st * TILE + off, 16, 1024), id_s,
+                             ks > 0 ? 1u : 0u);
+                }
+                mma_commit(dpt_full);
+                return true;
+            };
+            bool ok = mbar_wait(kv_full, 0, abort_flag, p.status) && scores(0);
+            for (int u = 0; ok && u < nunits; ++u) {
+                const int st = u & 1;
+                // dV += P^T_u dO_u: queries 16kk..16kk+15 sit in the packed columns
+                // 32*(kk/2) + 8*(kk%2) of S^T (written by column group kk/2)
+                if (!mbar_wait(p_full, u & 1, abort_flag, p.status)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tdV, tSt + 32 * (kk >> 1) + 8 * (kk & 1),
+                                smem_desc(sDO + st * TILE + kk * 2048, 16384, 1024), id_kv,
+                                (u > 0 || kk > 0) ? 1u : 0u);
+                // the next unit's scores overwrite S^T only after the dV MMAs (issue order)
+                if (u + 1 < nunits && !scores(u + 1)) break;
+                if (!mbar_wait(ds_full, u & 1, abort_flag, p.status)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tdK, smem_desc(sDST + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                             smem_desc(sQ + st * TILE + kk * 2048, 16384, 1024), id_kv, (u > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(ds_free);
+                mma_commit(qo_empty + 8 * st);
             }
+            mma_commit(dkv_done);
         }
     } else {
-        // warps 2..9: TMEM lane quarter q = warp % 4 (key rows), query half ch of each unit
-        const int q = warp & 3, ch = (warp - 2) >> 2;
+        // warps 2..17: TMEM lane quarter q (key rows), query column group cg (32 queries)
+        const int q = warp & 3, cg = (warp - 2) >> 2;
         const int r = q * 32 + lane;
         const int kpos = kvb * 128 + r;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         bool ok = true;
         for (int u = 0; u < nunits; ++u) {
-            const int sb = u & 1, st = u % DKV_STG;
-            const int i = nq64 - 1 - u / Hg;
-            if (!warp_wait(st_full + 8 * sb, (u >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            // this unit's Q/dO/lse/D stage has landed (the phase cannot move on
-            // before this warp finishes the unit, which frees the stage)
-            if (!warp_wait(qo_full + 8 * st, (u / DKV_STG) & 1, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
-            // this warp's 32 query columns of the unit: lse (to log2 units) and D
-            float l2[32], dd[32];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float4 a = reinterpret_cast<const float4*>(lse_s + st * 64 + ch * 32)[k];
-                const float4 b = reinterpret_cast<const float4*>(d_s + st * 64 + ch * 32)[k];
-                l2[4 * k] = a.x * kLog2e; l2[4 * k + 1] = a.y * kLog2e; l2[4 * k + 2] = a.z * kLog2e;
-                l2[4 * k + 3] = a.w * kLog2e;
-                dd[4 * k] = b.x; dd[4 * k + 1] = b.y; dd[4 * k + 2] = b.z; dd[4 * k + 3] = b.w;
-            }
-            // units whose queries all see every key of the block need no mask
-            const bool full = i * 64 + ch * 32 >= kvb * 128 + 127 && i * 64 + ch * 32 + 31 < p.T;
-            float sv[32], dp[32];
-            {
-                uint32_t rs[32], rd[32];
-                tmem_ld32_issue(tSt + lane_off + sb * 64 + ch * 32, rs);
-                tmem_ld32_issue(tdPt + lane_off + sb * 64 + ch * 32, rd);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) { sv[i] = __uint_as_float(rs[i]); dp[i] = __uint_as_float(rd[i]); }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(st_empty + 8 * sb);
-            if (full) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float P = ex2(sv[e] * p.scale_log2 - l2[e]);
-                    dp[e] = P * (dp[e] - dd[e]);
-                    sv[e] = P;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int qpos = i * 64 + ch * 32 + e;
-                    const bool valid = qpos >= kpos && qpos < p.T;
-                    const float P = valid ? ex2(sv[e] * p.scale_log2 - l2[e]) : 0.f;
-                    dp[e] = valid ? P * (dp[e] - dd[e]) : 0.f;
-                    sv[e] = P;
-                }
-            }
-            // P^T / dS^T buffer (u & 1) was last read by the dV/dK MMAs of unit u-2
-            if (u > 1 && !warp_wait(pd_done + 8 * (u & 1), ((u >> 1) - 1) & 1, abort_flag, p.status)) {
+            const int st = u & 1;
+            const int i = p.nqb - 1 - u / Hg;
+            if (!warp_wait(st_full, u & 1, abort_flag, p.status) ||
+                !warp_wait(qo_full + 8 * st, (u >> 1) & 1, abort_flag, p.status)) {
                 ok = false;
                 break;
             }
-            uint8_t* prow = smem + Lay::PT + (u & 1) * 16384 + r * 128;
-            uint8_t* drow = smem + Lay::DST + (u & 1) * 16384 + r * 128;
+            tc_fence_after();
+            uint32_t rs[32];
+            tmem_ld32_issue(tSt + lane_off + cg * 32, rs);
+            tmem_wait_ld();
+            // query q0 + e sees this key when lo <= e (causal) and e <= hi (inside the row)
+            const int q0 = i * 128 + cg * 32;
+            const int lo = kpos - q0, hi = p.T - 1 - q0;
+            const float4* l4 = reinterpret_cast<const float4*>(lse_s + st * 128 + cg * 32);
+            float pv[32];
+            if (__all_sync(0xffffffffu, lo <= 0 && hi >= 31)) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float4 l = l4[k];
+                    pv[4 * k] = ex2(fmaf(__uint_as_float(rs[4 * k]), p.scale_log2, -l.x));
+                    pv[4 * k + 1] = ex2(fmaf(__uint_as_float(rs[4 * k + 1]), p.scale_log2, -l.y));
+                    pv[4 * k + 2] = ex2(fmaf(__uint_as_float(rs[4 * k + 2]), p.scale_log2, -l.z));
+                    pv[4 * k + 3] = ex2(fmaf(__uint_as_float(rs[4 * k + 3]), p.scale_log2, -l.w));
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float4 l = l4[k];
+                    const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int e = 4 * k + t;
+                        pv[e] = (e >= lo && e <= hi) ? ex2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -lv[t])) : 0.f;
+                    }
+                }
+            }
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(pv[16 * hf + 2 * e], pv[16 * hf + 2 * e + 1]);
+                tmem_st8_nowait(tSt + lane_off + cg * 32 + 8 * hf, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+            // dP^T only now (the MMA thread needs P^T before it can use a free dP^T buffer anyway)
+            if (!warp_wait(dpt_full, u & 1, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t rd[32];
+            tmem_ld32_issue(tdPt + lane_off + cg * 32, rd);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dpt_free);
+            // dS^T = P^T (dP^T - D); masked entries have P = 0 and D, dP finite
+            const float4* d4 = reinterpret_cast<const float4*>(d_s + st * 128 + cg * 32);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float4 dd = d4[k];
+                pv[4 * k] *= __uint_as_float(rd[4 * k]) - dd.x;
+                pv[4 * k + 1] *= __uint_as_float(rd[4 * k + 1]) - dd.y;
+                pv[4 * k + 2] *= __uint_as_float(rd[4 * k + 2]) - dd.z;
+                pv[4 * k + 3] *= __uint_as_float(rd[4 * k + 3]) - dd.w;
+            }
+            // the dK MMAs of the previous unit have read the dS^T tile
+            if (u > 0 && !warp_wait(ds_free, (u - 1) & 1, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            uint8_t* drow = smem + Lay::DST + (cg >> 1) * 16384 + r * 128;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int idx = ch * 4 + k;
-                const uint32_t sw = (uint32_t)((idx ^ (r & 7)) << 4);
-                const float* a = sv + 8 * k;
-                const float* d = dp + 8 * k;
-                *reinterpret_cast<uint4*>(prow + sw) = make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]),
-                                                                  pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
-                *reinterpret_cast<uint4*>(drow + sw) = make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]),
-                                                                  pack_bf16(d[4], d[5]), pack_bf16(d[6], d[7]));
+                const int c8 = (cg & 1) * 4 + k;
+                const float* d = pv + 8 * k;
+                *reinterpret_cast<uint4*>(drow + ((c8 ^ (r & 7)) << 4)) =
+                    make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
+                               pack_bf16(d[6], d[7]));
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(pd_full + 8 * (u & 1));
+            if (lane == 0) mbar_arrive(ds_full);
         }
-        if (ok && warp_wait(pd_done + 8 * ((nunits - 1) & 1), ((nunits - 1) >> 1) & 1, abort_flag, p.status)) {
+        if (ok && warp_wait(dkv_done, 0, abort_flag, p.status)) {
             tc_fence_after();
+            // column groups 0 and 1 write the two halves of dv, 2 and 3 those of dk
+            const bool isk = cg >= 2;
+            const int c0 = (cg & 1) * (HD / 2);
+            const uint32_t tsrc = (isk ? tdK : tdV) + lane_off + c0;
+            const float sc = isk ? p.scale : 1.f;
             const bool live = kpos < p.T;
-            if (p.rqk && ch == 1) {
-                // dK through the QK-norm backward (the other four warps write dV below)
-                const size_t rowi = (size_t)row0 + (live ? kpos : 0);
-                const int pos = live ? kpos : 0;
-                bf16* outk = p.dqkv + rowi * Nqkv + (p.H + g) * HD;
-                store_grad_through_qknorm<HD>(tdK + lane_off, p.scale, p.qkv + rowi * Nqkv + (p.H + g) * HD,
-                                              live ? p.rqk[rowi * (p.H + p.nkv) + p.H + g] : 0.f,
-                                              p.cos_t + (size_t)pos * (HD / 2), p.sin_t + (size_t)pos * (HD / 2),
-                                              outk, live);
-            } else {
-            // the first four softmax warps write dV, the other four dK
-            bf16* out = p.dqkv + ((size_t)row0 + kpos) * Nqkv + (ch == 0 ? (p.H + p.nkv + g) : (p.H + g)) * HD;
-            const uint32_t tsrc = ch == 0 ? tdV : tdK;
-            const float sc = ch == 0 ? 1.f : p.scale;
+            bf16* out = p.dqkv + ((size_t)row0 + (live ? kpos : 0)) * Nqkv + (isk ? p.H + g : p.H + p.nkv + g) * HD + c0;
 #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
+            for (int c = 0; c < HD / 64; ++c) {
                 float v[32];
-                tmem_ld32(tsrc + lane_off + c * 32, v);
+                tmem_ld32(tsrc + c * 32, v);
                 if (live) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
@@ -851,7 +873,6 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                                        pack_bf16(v[8 * e + 4] * sc, v[8 * e + 5] * sc),
                                        pack_bf16(v[8 * e + 6] * sc, v[8 * e + 7] * sc));
                 }
-            }
             }
         }
     }
@@ -907,8 +928,7 @@ int fwd_launch(const CUtensorMap& map, const AttnParams& p, cudaStream_t s) {
 }
 
 template <int HD>
-int dq_launch(const CUtensorMap& kv, const CUtensorMap& kv64, const CUtensorMap& do128, const BwdParams& p,
-              cudaStream_t s) {
+int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(attn_dq_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -916,14 +936,13 @@ int dq_launch(const CUtensorMap& kv, const CUtensorMap& kv64, const CUtensorMap&
             return -1;
         attr = true;
     }
-    attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NTB, DqLayout<HD>::BYTES, s>>>(kv, kv64, do128, p);
+    attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NTB, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 template <int HD>
-int dkv_launch(const CUtensorMap& kv, const CUtensorMap& q64, const CUtensorMap& do64, const BwdParams& p,
-               cudaStream_t s) {
+int dkv_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(attn_dkv_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -931,21 +950,30 @@ int dkv_launch(const CUtensorMap& kv, const CUtensorMap& q64, const CUtensorMap&
             return -1;
         attr = true;
     }
-    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NTB, DkvLayout<HD>::BYTES, s>>>(kv, q64, do64, p);
+    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NTB, DkvLayout<HD>::BYTES, s>>>(kv, do128, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
-BwdParams bwd_params(const float* lse, const float* Dbuf, void* dqkv, int B, int T, int H, int nkv, int hd,
-                     int* status) {
-    BwdParams p{};
-    p.B = B; p.T = T; p.H = H; p.nkv = nkv; p.nqb = (T + 127) / 128;
-    p.scale = 1.f / sqrtf((float)hd);
-    p.scale_log2 = kLog2e * p.scale;
-    p.lse = lse; p.D = Dbuf;
-    p.dqkv = reinterpret_cast<bf16*>(dqkv);
-    p.status = status;
-    return p;
+// Parameters and the two tensor maps (qkv and dO, 128-row boxes) of both kernels.
+bool bwd_setup(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv, int B,
+               int T, int H, int nkv, int hd, int* status, BwdParams* p, CUtensorMap* kv, CUtensorMap* do128) {
+    if (!attention_tc_bwd_supported(hd)) return false;
+    if (!aligned16(qkv) || !aligned16(dO) || !aligned16(dqkv) || !aligned16(Dbuf) || (o && !aligned16(o)))
+        return false;
+    if (B > 65535 || H > 65535 || nkv < 1 || H % nkv != 0) return false;
+    const int Nqkv = (H + 2 * nkv) * hd;
+    if (!map_rows(kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128))
+        return false;
+    *p = BwdParams{};
+    p->B = B; p->T = T; p->H = H; p->nkv = nkv; p->nqb = (T + 127) / 128;
+    p->scale = 1.f / sqrtf((float)hd);
+    p->scale_log2 = kLog2e * p->scale;
+    p->D = Dbuf;
+    p->lse2 = Dbuf + attn_stat_elems(B, T, H);
+    p->dqkv = reinterpret_cast<bf16*>(dqkv);
+    p->status = status;
+    return true;
 }
 
 }  // namespace
@@ -969,45 +997,38 @@ int attention_tc_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, 
 bool attention_tc_bwd_supported(int hd) { return hd == 64 || hd == 128; }
 
 int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
-                        int B, int T, int H, int nkv, int hd, int* status, cudaStream_t s, const QkNormFuse* fuse) {
-    if (!attention_tc_bwd_supported(hd)) return 1;
-    if (!aligned16(qkv) || !aligned16(o) || !aligned16(dO) || !aligned16(dqkv) || B > 65535 || H > 65535) return 1;
-    const int Nqkv = (H + 2 * nkv) * hd;
-    CUtensorMap kv, kv64, do128;
-    if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&kv64, qkv, Nqkv, (uint64_t)B * T, 64) ||
-        !map_rows(&do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128))
-        return 1;
-    if (launch_attention_bwd_dot(DT_BF16, o, dO, Dbuf, B, T, H, hd, s) != cudaSuccess) return -1;
-    BwdParams p = bwd_params(lse, Dbuf, dqkv, B, T, H, nkv, hd, status);
-    if (fuse) {
-        p.qkv = reinterpret_cast<const bf16*>(qkv);
-        p.rqk = fuse->rqk; p.cos_t = fuse->cos_t; p.sin_t = fuse->sin_t;
+                        int B, int T, int H, int nkv, int hd, int* status, cudaStream_t s) {
+    BwdParams p;
+    CUtensorMap kv, do128;
+    if (!o || !lse || !bwd_setup(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, &p, &kv, &do128)) return 1;
+    {
+        const long long threads = (long long)attn_stat_elems(B, T, H) * (hd / 8);
+        const unsigned blocks = (unsigned)((threads + 255) / 256);
+        const bf16* ob = reinterpret_cast<const bf16*>(o);
+        const bf16* db = reinterpret_cast<const bf16*>(dO);
+        float* D = Dbuf;
+        float* l2 = Dbuf + attn_stat_elems(B, T, H);
+        if (hd == 128) attn_bwd_stats_kernel<128><<<blocks, 256, 0, s>>>(ob, db, lse, D, l2, B, T, H);
+        else attn_bwd_stats_kernel<64><<<blocks, 256, 0, s>>>(ob, db, lse, D, l2, B, T, H);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return -1;
     }
-    return hd == 128 ? dq_launch<128>(kv, kv64, do128, p, s) : dq_launch<64>(kv, kv64, do128, p, s);
+    return hd == 128 ? dq_launch<128>(kv, do128, p, s) : dq_launch<64>(kv, do128, p, s);
 }
 
-int attention_tc_bwd_dkv(const void* qkv, const void* dO, const float* lse, const float* Dbuf, void* dqkv, int B,
-                         int T, int H, int nkv, int hd, int* status, cudaStream_t s, const QkNormFuse* fuse) {
-    if (!attention_tc_bwd_supported(hd)) return 1;
-    if (!aligned16(qkv) || !aligned16(dO) || !aligned16(dqkv) || B > 65535 || nkv > 65535) return 1;
-    const int Nqkv = (H + 2 * nkv) * hd;
-    CUtensorMap kv, q64, do64;
-    if (!map_rows(&kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(&q64, qkv, Nqkv, (uint64_t)B * T, 64) ||
-        !map_rows(&do64, dO, (uint64_t)H * hd, (uint64_t)B * T, 64))
-        return 1;
-    BwdParams p = bwd_params(lse, Dbuf, dqkv, B, T, H, nkv, hd, status);
-    if (fuse) {
-        p.qkv = reinterpret_cast<const bf16*>(qkv);
-        p.rqk = fuse->rqk; p.cos_t = fuse->cos_t; p.sin_t = fuse->sin_t;
-    }
-    return hd == 128 ? dkv_launch<128>(kv, q64, do64, p, s) : dkv_launch<64>(kv, q64, do64, p, s);
+int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqkv, int B, int T, int H, int nkv,
+                         int hd, int* status, cudaStream_t s) {
+    BwdParams p;
+    CUtensorMap kv, do128;
+    if (!bwd_setup(qkv, nullptr, dO, nullptr, Dbuf, dqkv, B, T, H, nkv, hd, status, &p, &kv, &do128)) return 1;
+    return hd == 128 ? dkv_launch<128>(kv, do128, p, s) : dkv_launch<64>(kv, do128, p, s);
 }
 
 int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
                      int B, int T, int H, int nkv, int hd, void*, size_t, int* status, cudaStream_t s) {
-    int r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s, nullptr);
+    int r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s);
     if (r != 0) return r;
-    return attention_tc_bwd_dkv(qkv, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s, nullptr);
+    return attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, B, T, H, nkv, hd, status, s);
 }
 
 size_t attention_tc_workspace_bytes(int, int, int, int, int) { return 0; }

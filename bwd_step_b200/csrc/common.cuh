@@ -12,7 +12,7 @@ typedef __nv_bfloat16 bf16;
 constexpr float kRmsEps = 1e-6f;
 
 // Device status word flags (OR-ed together, read and cleared by nc_check).
-enum : int { ST_BAD_TOKEN = 1, ST_TIMEOUT = 2 };
+enum : int { ST_BAD_TOKEN = 1, ST_TIMEOUT = 2, ST_BAD_LAYOUT = 4 };
 
 __device__ __forceinline__ void set_status(int* st, int flag) {
     if (st) atomicOr(st, flag);

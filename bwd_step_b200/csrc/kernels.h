@@ -109,9 +109,11 @@ cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t s);
 // qkv rows [B*T, (H+2nkv)*hd] hold q (post norm+rope), k (same), v.
 // o [B*T, H*hd].  Per-(row, head) softmax statistics (lse, natural log, and
 // the backward's D) are stored head-major with the sequence padded to a
-// multiple of 64: index (b*H + h)*attn_tpad(T) + t.
-__host__ __device__ inline int attn_tpad(int T) { return (T + 63) / 64 * 64; }
+// multiple of 128 (one query block): index (b*H + h)*attn_tpad(T) + t.
+__host__ __device__ inline int attn_tpad(int T) { return (T + 127) / 128 * 128; }
 inline size_t attn_stat_elems(int B, int T, int H) { return (size_t)B * H * attn_tpad(T); }
+// The backward's buffer: D, then (tensor-core path) lse * log2(e), each attn_stat_elems.
+inline size_t attn_dbuf_elems(int B, int T, int H) { return 2 * attn_stat_elems(B, T, H); }
 cudaError_t launch_attention_fwd_simt(DType at, const void* qkv, void* o, float* lse, int B, int T, int H,
                                       int nkv, int hd, cudaStream_t s);
 // Writes dq (into the q columns), dk, dv of dqkv.  Dbuf [B*T, H] scratch.

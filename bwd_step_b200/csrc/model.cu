@@ -107,7 +107,7 @@ Plan make_plan(const nc_model* m, int B, int T) {
     p.du = take(A * M * m->F);
     p.dO = take(A * M * m->H * m->hd);
     p.dqkv = take(A * M * m->Nqkv);
-    p.Dbuf = take(4 * attn_stat_elems(B, T, m->H));
+    p.Dbuf = take(4 * attn_dbuf_elems(B, T, m->H));
     p.R = lm_chunk_rows(m, p.M);
     p.zc = take(4ull * p.R * m->V);
     p.dlc = take(A * (size_t)p.R * m->V);
@@ -209,30 +209,21 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
     return NC_OK;
 }
 
-// Attention backward.  With rqk set and the tensor-core path, dq and dk come
-// out already through the QK-norm + RoPE backward (*qk_fused = true);
-// otherwise the caller runs that backward as its own kernel (faster on B200:
-// the fused form lengthens the tail of every attention CTA).
-int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv,
-                  const float* rqk, bool* qk_fused) {
+// Attention backward: dq, then dk / dv (tensor cores), or the plain-FMA kernels.
+int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv) {
     const nc_model* m = c.m;
     float* Dbuf = c.at<float>(c.p.Dbuf);
-    *qk_fused = false;
     if (m->tc && attention_tc_bwd_supported(m->hd)) {
-        QkNormFuse fz{rqk, c.at<float>(c.p.cosb), c.at<float>(c.p.sinb)};
-        const QkNormFuse* fzp = rqk ? &fz : nullptr;
         int r;
         {
             Prof pr(c, P_ATTN_BWD_DQ, attn_flops(c), 0.0);
-            r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s,
-                                    fzp);
+            r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s);
         }
         if (r == 0) {
             Prof pr(c, P_ATTN_BWD_DKV, attn_flops(c), 0.0);
-            r = attention_tc_bwd_dkv(qkv, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s,
-                                     fzp);
+            r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s);
         }
-        if (r == 0) { *qk_fused = fzp != nullptr; return NC_OK; }
+        if (r == 0) return NC_OK;
         if (r < 0) return NC_ERR_CUDA;
     }
     Prof pr(c, P_ATTN_BWD, 2.0 * attn_flops(c), 0.0);
@@ -366,10 +357,8 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at), P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
                           DT_F32), P_GEMM_WGRAD));
-        bool qk_fused = false;
-        RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), dqkv, nullptr,
-                         &qk_fused));
-        if (!qk_fused) {
+        RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), dqkv));
+        {
             Prof pr(c, P_QKROPE_BWD, 0.0, (double)M * (m->H + m->nkv) * (3.0 * A * m->hd + 4.0));
             CK(launch_qknorm_rope_bwd(m->at, dqkv, lb + c.p.l_qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, T, m->H,
                                       m->nkv, m->hd, s));
@@ -537,6 +526,7 @@ int nc_check(nc_model* m, void* stream) {
     if (cudaMemcpy(&st, m->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return NC_ERR_CUDA;
     if (cudaMemset(m->status, 0, sizeof(int)) != cudaSuccess) return NC_ERR_CUDA;
     if (st & ST_TIMEOUT) return NC_ERR_DEVICE_TIMEOUT;
+    if (st & ST_BAD_LAYOUT) return NC_ERR_CUDA;
     if (st & ST_BAD_TOKEN) return NC_ERR_BAD_TOKEN;
     return NC_OK;
 }

@@ -88,9 +88,9 @@ def bench_attention(iters, B=16, T=2048, H=10, nkv=1, hd=128):
     qkv = torch.randn(B * T * nq, device="cuda", generator=g).to(torch.bfloat16)
     dO = torch.randn(B * T * H * hd, device="cuda", generator=g).to(torch.bfloat16)
     o = torch.empty(B * T * H * hd, device="cuda", dtype=torch.bfloat16)
-    lse = torch.empty(B * H * ((T + 63) // 64 * 64), device="cuda", dtype=torch.float32)
+    lse = torch.empty(B * H * ((T + 127) // 128 * 128), device="cuda", dtype=torch.float32)
     dqkv = torch.empty_like(qkv)
-    Dbuf = torch.empty_like(lse)
+    Dbuf = torch.empty(2 * lse.numel(), device="cuda", dtype=torch.float32)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     stream = P(torch.cuda.current_stream().cuda_stream)
 

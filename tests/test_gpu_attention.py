@@ -27,10 +27,10 @@ def _run(B, T, H, nkv, hd, use_tc, seed=0, scale=1.0):
     dO = _bf16(rng.standard_normal((B * T, H * hd)))
     qkv_d, dO_d = qkv.cuda(), dO.cuda()
     o = torch.full((B * T, H * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
-    Tp = (T + 63) // 64 * 64  # softmax statistics are [B, H, T padded to 64]
+    Tp = (T + 127) // 128 * 128  # softmax statistics are [B, H, T padded to 128]
     lse = torch.full((B * H * Tp,), float("nan"), dtype=torch.float32, device="cuda")
     dqkv = torch.full((B * T, Nqkv), float("nan"), dtype=torch.bfloat16, device="cuda")
-    Dbuf = torch.full((B * H * Tp,), float("nan"), dtype=torch.float32, device="cuda")
+    Dbuf = torch.full((2 * B * H * Tp,), float("nan"), dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     r = lib().nc_test_attention(B, T, H, nkv, hd, P(qkv_d.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
                                 P(dO_d.data_ptr()), P(dqkv.data_ptr()), P(Dbuf.data_ptr()), use_tc,
