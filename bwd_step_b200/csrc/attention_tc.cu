@@ -291,9 +291,11 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 // dQ, one CTA per (query block of 128, head, batch row), key blocks j = 0..qb:
 //   warp 0      TMA: Q and dO once; K_j into a 3-stage ring (freed by the dQ
 //               MMA), V_j into a 2-stage ring (freed by the dP MMA);
-//   warp 1      tcgen05.mma: S_j = Q K_j^T into one of two TMEM buffers,
-//               dP_j = dO V_j^T into one buffer, then dQ += dS_{j-1} K_{j-1}
-//               with dS read from TMEM and K as an MN-major operand;
+//   warp 1      tcgen05.mma: S_j = Q K_j^T into one of two TMEM buffers and
+//               dP_j = dO V_j^T into one buffer as one group of 16 MMAs
+//               (every wait or commit between 128-wide MMAs idles the tensor
+//               core), then dQ += dS_{j-1} K_{j-1} with dS read from TMEM and
+//               K as an MN-major operand;
 //   warps 2-17  per key block: load the warp's S and dP columns, release dP,
 //               form
 //               P = 2^(S*scale*log2e - lse*log2e) with the causal mask on the
@@ -393,7 +395,6 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
     const uint32_t qd_full = b0;
     const uint32_t k_full = b0 + 8, k_empty = b0 + 32;   // [KSTG]
     const uint32_t v_full = b0 + 56, v_empty = b0 + 72;  // [VSTG]
-    const uint32_t s_full = b0 + 88;                     // [2]: S_j landed in TMEM buffer j & 1
     const uint32_t dp_full = b0 + 104, dp_free = b0 + 112;
     const uint32_t ds_full = b0 + 120;                   // [2]: dS_j written over buffer j & 1
     const uint32_t dq_done = b0 + 136;
@@ -411,7 +412,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
         mbar_init(qd_full, 1);
         for (int s = 0; s < KSTG; ++s) { mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1); }
         for (int s = 0; s < VSTG; ++s) { mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(ds_full + 8 * s, NSM); }
+        for (int s = 0; s < 2; ++s) mbar_init(ds_full + 8 * s, NSM);
         mbar_init(dp_full, 1);
         mbar_init(dp_free, NSM);
         mbar_init(dq_done, 1);
@@ -464,8 +465,11 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
             bool ok = mbar_wait(qd_full, 0, abort_flag, p.status);
             for (int j = 0; ok && j <= nblk; ++j) {
                 if (j < nblk) {
+                    // S_j and dP_j as one group: K_j, V_j landed, dP_{j-1} read out of TMEM
                     const int kst = j % KSTG, vst = j % VSTG, sb = j & 1;
                     if (!mbar_wait(k_full + 8 * kst, (j / KSTG) & 1, abort_flag, p.status)) break;
+                    if (!mbar_wait(v_full + 8 * vst, (j / VSTG) & 1, abort_flag, p.status)) break;
+                    if (j > 0 && !mbar_wait(dp_free, (j - 1) & 1, abort_flag, p.status)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < HD / 16; ++ks) {
@@ -473,11 +477,6 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
                         mma_bf16(tS + sb * 128, smem_desc(sQ + off, 16, 1024),
                                  smem_desc(sK + kst * TILE + off, 16, 1024), id_s, ks > 0 ? 1u : 0u);
                     }
-                    mma_commit(s_full + 8 * sb);
-                    if (!mbar_wait(v_full + 8 * vst, (j / VSTG) & 1, abort_flag, p.status)) break;
-                    // the softmax warps have read dP_{j-1} out of TMEM
-                    if (j > 0 && !mbar_wait(dp_free, (j - 1) & 1, abort_flag, p.status)) break;
-                    tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < HD / 16; ++ks) {
                         const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -515,8 +514,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
         bool ok = true;
         for (int j = 0; j < nblk; ++j) {
             const int sb = j & 1;
-            if (!warp_wait(s_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status) ||
-                !warp_wait(dp_full, j & 1, abort_flag, p.status)) {
+            if (!warp_wait(dp_full, j & 1, abort_flag, p.status)) {
                 ok = false;
                 break;
             }
@@ -593,12 +591,14 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
 //   warp 1      tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM,
 //               dV += P^T dO_i with P^T read from TMEM, dK += dS^T Q_i with
 //               dS^T from shared memory (Q_i, dO_i as MN-major operands),
-//               in the order dV_u, S^T_{u+1}, dP^T_{u+1}, dK_u so the next
-//               unit's scores run while the softmax warps finish dS^T_u;
-//   warps 2-17  per unit: load the warp's S^T and dP^T columns (32 queries),
-//               release dP^T, form P^T = 2^(S^T*scale*log2e - lse2) with the
-//               causal mask and store it as packed bf16 over its own S^T
-//               columns, then dS^T = P^T (dP^T - D) into shared memory.
+//               in the order dV_u, S^T_{u+1}, dP^T_{u+1}, dK_u (the Q / dO
+//               tiles of unit u+1 land while P^T_u is formed; those of the
+//               unit after are prefetched into L2);
+//   warps 2-17  per unit: load the warp's S^T columns (32 queries), release
+//               S^T, form P^T = 2^(S^T*scale*log2e - lse2) with the causal
+//               mask, load the dP^T columns and store P^T as packed bf16 over
+//               the warp's own dP^T columns, then dS^T = P^T (dP^T - D) into
+//               shared memory.
 // dk = dK / sqrt(hd).
 template <int HD>
 struct DkvLayout {
@@ -636,7 +636,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24;  // qo_*[2]
-    const uint32_t st_full = b0 + 40, dpt_full = b0 + 48, dpt_free = b0 + 56;
+    const uint32_t st_full = b0 + 40, dpt_full = b0 + 48, st_free = b0 + 56;
     const uint32_t p_full = b0 + 64, ds_full = b0 + 72, ds_free = b0 + 80, dkv_done = b0 + 88;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -654,7 +654,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         for (int s = 0; s < 2; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
         mbar_init(st_full, 1);
         mbar_init(dpt_full, 1);
-        mbar_init(dpt_free, NSM);
+        mbar_init(st_free, NSM);
         mbar_init(p_full, NSM);
         mbar_init(ds_full, NSM);
         mbar_init(ds_free, 1);
@@ -696,6 +696,15 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                                 qo_full + 8 * st);
                 }
                 issued = u + 1;
+                // the unit after next into L2, so its load finds it there once a stage frees
+                if (u + 2 < nunits) {
+                    const int i2 = p.nqb - 1 - (u + 2) / Hg, h2 = g * Hg + (u + 2) % Hg;
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb) {
+                        tma_prefetch_l2_2d(&tmQKV, h2 * HD + kb * 64, row0 + i2 * 128);
+                        tma_prefetch_l2_2d(&tmDO, h2 * HD + kb * 64, row0 + i2 * 128);
+                    }
+                }
             }
             if (*abort_flag) {
                 drain(kv_full, 0);
@@ -706,7 +715,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);
             const uint32_t id_kv = idesc_bf16(128, HD, false, true);
-            // S^T_u = K Q_u^T and dP^T_u = V dO_u^T
+            // S^T_u = K Q_u^T
             auto scores = [&](int u) -> bool {
                 const int st = u & 1;
                 if (!mbar_wait(qo_full + 8 * st, (u >> 1) & 1, abort_flag, p.status)) return false;
@@ -718,9 +727,11 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                              ks > 0 ? 1u : 0u);
                 }
                 mma_commit(st_full);
-                // the softmax warps have read dP^T_{u-1} out of TMEM
-                if (u > 0 && !mbar_wait(dpt_free, (u - 1) & 1, abort_flag, p.status)) return false;
-                tc_fence_after();
+                return true;
+            };
+            // dP^T_u = V dO_u^T (Q_u / dO_u already landed)
+            auto dpt = [&](int u) {
+                const int st = u & 1;
 #pragma unroll
                 for (int ks = 0; ks < HD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -728,22 +739,26 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                              ks > 0 ? 1u : 0u);
                 }
                 mma_commit(dpt_full);
-                return true;
             };
             bool ok = mbar_wait(kv_full, 0, abort_flag, p.status) && scores(0);
+            if (ok) dpt(0);
             for (int u = 0; ok && u < nunits; ++u) {
                 const int st = u & 1;
                 // dV += P^T_u dO_u: queries 16kk..16kk+15 sit in the packed columns
-                // 32*(kk/2) + 8*(kk%2) of S^T (written by column group kk/2)
+                // 32*(kk/2) + 8*(kk%2) of dP^T (written by column group kk/2)
                 if (!mbar_wait(p_full, u & 1, abort_flag, p.status)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tdV, tSt + 32 * (kk >> 1) + 8 * (kk & 1),
+                    mma_bf16_ts(tdV, tdPt + 32 * (kk >> 1) + 8 * (kk & 1),
                                 smem_desc(sDO + st * TILE + kk * 2048, 16384, 1024), id_kv,
                                 (u > 0 || kk > 0) ? 1u : 0u);
-                // the next unit's scores overwrite S^T only after the dV MMAs (issue order)
-                if (u + 1 < nunits && !scores(u + 1)) break;
+                // the next unit's scores (its Q / dO tiles are loaded by now), then its
+                // dP^T, which overwrites P^T only after the dV MMAs (issue order)
+                if (u + 1 < nunits) {
+                    if (!mbar_wait(st_free, u & 1, abort_flag, p.status) || !scores(u + 1)) break;
+                    dpt(u + 1);
+                }
                 if (!mbar_wait(ds_full, u & 1, abort_flag, p.status)) break;
                 tc_fence_after();
 #pragma unroll
@@ -774,6 +789,9 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             uint32_t rs[32];
             tmem_ld32_issue(tSt + lane_off + cg * 32, rs);
             tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(st_free);
             // query q0 + e sees this key when lo <= e (causal) and e <= hi (inside the row)
             const int q0 = i * 128 + cg * 32;
             const int lo = kpos - q0, hi = p.T - 1 - q0;
@@ -800,18 +818,6 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                     }
                 }
             }
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t pk[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(pv[16 * hf + 2 * e], pv[16 * hf + 2 * e + 1]);
-                tmem_st8_nowait(tSt + lane_off + cg * 32 + 8 * hf, pk);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
-            // dP^T only now (the MMA thread needs P^T before it can use a free dP^T buffer anyway)
             if (!warp_wait(dpt_full, u & 1, abort_flag, p.status)) {
                 ok = false;
                 break;
@@ -820,9 +826,18 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             uint32_t rd[32];
             tmem_ld32_issue(tdPt + lane_off + cg * 32, rd);
             tmem_wait_ld();
+            // P^T over the first half of this warp's own dP^T columns (just read)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(pv[16 * hf + 2 * e], pv[16 * hf + 2 * e + 1]);
+                tmem_st8_nowait(tdPt + lane_off + cg * 32 + 8 * hf, pk);
+            }
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(dpt_free);
+            if (lane == 0) mbar_arrive(p_full);
             // dS^T = P^T (dP^T - D); masked entries have P = 0 and D, dP finite
             const float4* d4 = reinterpret_cast<const float4*>(d_s + st * 128 + cg * 32);
 #pragma unroll
