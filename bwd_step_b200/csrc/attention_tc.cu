@@ -5,17 +5,19 @@
 // scaled by 1/sqrt(hd).
 //
 // Forward, one CTA per (query block of 128 positions, head, batch row):
-//   warp 0     TMA: the Q tile once, then K_j / V_j tiles (2-stage rings)
-//              for key blocks j = 0..qb (causal: blocks past the diagonal
-//              are never loaded);
-//   warp 1     tcgen05.mma: S_j = Q K_j^T into one of two TMEM score
-//              buffers, then O += P_{j-1} V_{j-1} (issued one block behind,
-//              so the next score tile is computed while softmax runs);
-//   warps 2-5  softmax, one query row per thread: scores from TMEM, causal
-//              mask on the diagonal block, running max in the log2 domain
-//              with lazy rescaling of O (only when the max grows by more
-//              than 2^8), P as bf16 into shared memory in the 128-byte
-//              swizzled K-major layout the next MMA reads.
+//   warp 0     TMA: the Q tile once, then K_j (lane 0) and V_j (lane 1) in
+//              3-stage rings for key blocks j = 0..qb (causal: blocks past
+//              the diagonal are never loaded);
+//   warp 1     tcgen05.mma: S_j = Q K_j^T into one of two 128-column TMEM
+//              buffers, two blocks ahead; O += P_j V_j with P_j read from
+//              TMEM (A operand) and V_j as an MN-major operand;
+//   warps 2-9  softmax, two warps per TMEM lane quarter (one query row per
+//              thread, 64 keys each): scores from TMEM, causal mask on the
+//              diagonal block, running row max in the log2 domain shared by
+//              the two warps of a row through shared memory, lazy rescaling
+//              of O (only when the max grows by more than 2^8), and P stored
+//              as packed bf16 over the first half of the warp's own score
+//              columns.
 // The K/V head is shared by all query heads; its tiles are re-read by the
 // H CTAs of a query block from L2.
 #include "attention_tc.h"
@@ -26,8 +28,8 @@ namespace nc {
 namespace {
 using namespace tc;
 
-constexpr int NT = 192;   // forward: producer, MMA, 4 softmax warps
-constexpr int STG = 2;
+constexpr int NT = 320;  // forward: producer, MMA, 8 softmax warps (two per TMEM lane quarter)
+constexpr int FSTG = 3;  // K and V ring stages
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -41,14 +43,15 @@ struct AttnParams {
 
 template <int HD>
 struct FwdLayout {
-    static constexpr int KB = HD / 64;          // 64-column blocks of the head dim
-    static constexpr int TILE = KB * 16384;     // [128 x HD] bf16, 128B-swizzled
+    static constexpr int KB = HD / 64;       // 64-column blocks of the head dim
+    static constexpr int TILE = KB * 16384;  // [128 x HD] bf16, 128B-swizzled
     static constexpr int Q = 0;
     static constexpr int K = Q + TILE;
-    static constexpr int V = K + STG * TILE;
-    static constexpr int P = V + STG * TILE;    // [128 x 128] bf16
-    static constexpr int BAR = P + 32768;
-    static constexpr int BYTES = BAR + 256 + 1024;  // + barriers, + alignment slack
+    static constexpr int V = K + FSTG * TILE;
+    static constexpr int MX = V + FSTG * TILE;  // [2][2][128] fp32 partial row maxima (then row sums)
+    static constexpr int BAR = MX + 2048;
+    static constexpr int BYTES = BAR + 256;  // the dynamic shared memory base is 1024-aligned (checked)
+    static_assert(BYTES <= 232448, "attention forward shared memory exceeds the per-block limit");
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -56,20 +59,46 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// the two softmax warps of TMEM lane quarter q (64 threads)
+__device__ __forceinline__ void pair_sync(int q) {
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+}
+
+// Store 32 consecutive 32-bit columns of this thread's TMEM lane, then wait.
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 template <int HD>
 __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnParams p) {
     using Lay = FwdLayout<HD>;
     constexpr int KB = Lay::KB;
     constexpr int TILE = Lay::TILE;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem_dyn[];
+    if ((smem_u32(smem_dyn) & 1023u) != 0) {
+        if (threadIdx.x == 0) set_status(p.status, ST_BAD_LAYOUT);
+        return;
+    }
+    uint8_t* smem = smem_dyn;
     const uint32_t base = smem_u32(smem);
-    const uint32_t sQ = base + Lay::Q, sK = base + Lay::K, sV = base + Lay::V, sP = base + Lay::P;
+    const uint32_t sQ = base + Lay::Q, sK = base + Lay::K, sV = base + Lay::V;
+    float* mxs = reinterpret_cast<float*>(smem + Lay::MX);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
-    const uint32_t q_full = b0, k_full = b0 + 8, k_empty = b0 + 24, v_full = b0 + 40, v_empty = b0 + 56;
-    const uint32_t s_full = b0 + 72, s_empty = b0 + 88, p_full = b0 + 104, o_done = b0 + 112;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    const uint32_t q_full = b0;
+    const uint32_t k_full = b0 + 8, k_empty = b0 + 32, v_full = b0 + 56, v_empty = b0 + 80;  // [FSTG]
+    const uint32_t s_full = b0 + 104, p_full = b0 + 120;  // [2]: per TMEM score buffer
+    const uint32_t o_last = b0 + 136;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -80,13 +109,12 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < STG; ++s) {
+        for (int s = 0; s < FSTG; ++s) {
             mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1);
             mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1);
         }
-        for (int s = 0; s < 2; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(s_empty + 8 * s, 4); }
-        mbar_init(p_full, 4);
-        mbar_init(o_done, 1);
+        for (int s = 0; s < 2; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(p_full + 8 * s, 8); }
+        mbar_init(o_last, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -96,11 +124,11 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 256;
+    const uint32_t tS = tmem, tO = tmem + 256;  // S[2] of 128 columns, O (HD columns)
 
     if (warp == 0) {
-        // lane 0 loads Q and the K ring, lane 1 the V ring: each waits only on
-        // its own ring, so K tiles run ahead of the V slots that P*V frees late
+        // lane 0 loads Q and the K ring (a slot frees once S_j is computed), lane 1
+        // the V ring (a slot frees after O += P_j V_j)
         if (lane < 2) {
             const bool kl = lane == 0;
             const int xq = h * HD, xkv = kl ? (p.H + g) * HD : (p.H + p.nkv + g) * HD;
@@ -114,9 +142,8 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
             }
             int issued = 0;
             for (int j = 0; j < nblk; ++j) {
-                const int st = j % STG;
-                const uint32_t ph = (j / STG) & 1;
-                if (!mbar_wait(empty + 8 * st, ph ^ 1, abort_flag, p.status)) break;
+                const int st = j % FSTG;
+                if (!mbar_wait(empty + 8 * st, ((j / FSTG) & 1) ^ 1, abort_flag, p.status)) break;
                 mbar_expect_tx(full + 8 * st, TILE);
 #pragma unroll
                 for (int kb = 0; kb < KB; ++kb)
@@ -127,9 +154,9 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 // let copies in flight land before the block exits
                 uint64_t t0 = globaltimer();
                 if (kl) while (!mbar_try(q_full, 0) && globaltimer() - t0 < 1000000ull) {}
-                for (int j = (issued > STG ? issued - STG : 0); j < issued; ++j) {
+                for (int j = (issued > FSTG ? issued - FSTG : 0); j < issued; ++j) {
                     t0 = globaltimer();
-                    while (!mbar_try(full + 8 * (j % STG), (j / STG) & 1) && globaltimer() - t0 < 1000000ull) {}
+                    while (!mbar_try(full + 8 * (j % FSTG), (j / FSTG) & 1) && globaltimer() - t0 < 1000000ull) {}
                 }
             }
         }
@@ -137,126 +164,136 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);
             const uint32_t id_o = idesc_bf16(128, HD, false, true);
-            bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-            for (int j = 0; ok && j <= nblk; ++j) {
-                if (j < nblk) {
-                    const int st = j % STG, sb = j & 1;
-                    if (!mbar_wait(k_full + 8 * st, (j / STG) & 1, abort_flag, p.status)) break;
-                    if (!mbar_wait(s_empty + 8 * sb, ((j >> 1) & 1) ^ 1, abort_flag, p.status)) break;
-                    tc_fence_after();
+            // S_j = Q K_j^T into buffer j & 1
+            auto scores = [&](int j) -> bool {
+                const int st = j % FSTG, sb = j & 1;
+                if (!mbar_wait(k_full + 8 * st, (j / FSTG) & 1, abort_flag, p.status)) return false;
+                tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < HD / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16(tS + sb * 128, smem_desc(sQ + off, 16, 1024), smem_desc(sK + st * TILE + off, 16, 1024),
-                                 id_s, ks > 0 ? 1u : 0u);
-                    }
-                    mma_commit(s_full + 8 * sb);
-                    mma_commit(k_empty + 8 * st);
+                for (int ks = 0; ks < HD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    mma_bf16(tS + sb * 128, smem_desc(sQ + off, 16, 1024), smem_desc(sK + st * TILE + off, 16, 1024),
+                             id_s, ks > 0 ? 1u : 0u);
                 }
-                if (j > 0) {
-                    const int jj = j - 1, st = jj % STG;
-                    if (!mbar_wait(p_full, jj & 1, abort_flag, p.status)) break;
-                    if (!mbar_wait(v_full + 8 * st, (jj / STG) & 1, abort_flag, p.status)) break;
-                    tc_fence_after();
+                mma_commit(s_full + 8 * sb);
+                mma_commit(k_empty + 8 * st);
+                return true;
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && scores(0) && (nblk < 2 || scores(1));
+            for (int j = 0; ok && j < nblk; ++j) {
+                const int st = j % FSTG, sb = j & 1;
+                // O += P_j V_j: keys 16kk..16kk+15 sit in the packed columns
+                // 64*(kk/4) + 8*(kk%4) of score buffer j & 1 (written by column group kk/4)
+                if (!mbar_wait(p_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status)) break;
+                if (!mbar_wait(v_full + 8 * st, (j / FSTG) & 1, abort_flag, p.status)) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t offp = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16(tO, smem_desc(sP + offp, 16, 1024), smem_desc(sV + st * TILE + ks * 2048, 16384, 1024),
-                                 id_o, (jj > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    mma_commit(o_done);
-                    mma_commit(v_empty + 8 * st);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tO, tS + sb * 128 + 64 * (kk >> 2) + 8 * (kk & 3),
+                                smem_desc(sV + st * TILE + kk * 2048, 16384, 1024), id_o, (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(v_empty + 8 * st);
+                // S_{j+2} overwrites P_j only after these MMAs (issue order)
+                if (j + 2 < nblk && !scores(j + 2)) break;
             }
+            mma_commit(o_last);
         }
     } else {
-        // ---------------- softmax warps: warp w reads TMEM lanes 32*(w%4)..
-        const int q = warp & 3;
+        // ---------------- softmax warps: warp w reads TMEM lanes 32*(w%4).., keys 64*cg..
+        const int q = warp & 3, cg = (warp - 2) >> 2;
         const int r = q * 32 + lane;  // row of the tile
         const int qpos = qb * 128 + r;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         float m = -INFINITY, l = 0.f;
+        // After a failed (timed-out or aborted) wait a warp skips its TMEM and
+        // barrier work but still meets its partner at every pair_sync, so the
+        // pair never waits on a warp that has left the loop.
         bool ok = true;
         for (int j = 0; j < nblk; ++j) {
             const int sb = j & 1;
-            if (!warp_wait(s_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
-            float s[128];
-            {
-                uint32_t rr[128];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32_issue(tS + lane_off + sb * 128 + c * 32, rr + 32 * c);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(rr[i]);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty + 8 * sb);
+            ok = ok && warp_wait(s_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status);
+            float s[64];
             float mx = -INFINITY;
-            if (j == qb) {
+            if (ok) {
+                tc_fence_after();
+                {
+                    uint32_t rr[64];
+                    tmem_ld32_issue(tS + lane_off + sb * 128 + cg * 64, rr);
+                    tmem_ld32_issue(tS + lane_off + sb * 128 + cg * 64 + 32, rr + 32);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    s[c] = (c <= r) ? s[c] * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, s[c]);
+                    for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(rr[i]);
                 }
-            } else {
+                if (j == qb) {
+                    const int lim = r - cg * 64;  // keys cg*64 + c with c <= lim are visible
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    s[c] *= p.scale_log2;
-                    mx = fmaxf(mx, s[c]);
+                    for (int c = 0; c < 64; ++c) {
+                        s[c] = (c <= lim) ? s[c] * p.scale_log2 : -INFINITY;
+                        mx = fmaxf(mx, s[c]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        s[c] *= p.scale_log2;
+                        mx = fmaxf(mx, s[c]);
+                    }
                 }
             }
+            // the row max over both halves of the block
+            mxs[(sb * 2 + cg) * 128 + r] = mx;
+            pair_sync(q);
+            if (!ok) continue;
+            mx = fmaxf(mx, mxs[(sb * 2 + (cg ^ 1)) * 128 + r]);
             const bool rescale = mx > m + 8.f;
             const float mu = rescale ? mx : m;
             const float alpha = rescale ? ex2(m - mx) : 1.f;
             float sum = 0.f;
+            uint32_t pk[32];
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                s[c] = ex2(s[c] - mu);
-                sum += s[c];
+            for (int c = 0; c < 64; c += 2) {
+                const float e0 = ex2(s[c] - mu), e1 = ex2(s[c + 1] - mu);
+                sum += e0 + e1;
+                pk[c >> 1] = pack_bf16(e0, e1);
             }
-            if (j > 0) {
-                if (!warp_wait(o_done, (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                // O += P_{j-1} V_{j-1} has finished (its V slot was released); O(j) cannot
+                // have started, so this phase of the barrier is the latest one
+                const int jj = j - 1;
+                ok = warp_wait(v_empty + 8 * (jj % FSTG), (jj / FSTG) & 1, abort_flag, p.status);
+                if (!ok) continue;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
+                // this warp rescales its half of the O columns
+#pragma unroll 1
+                for (int c = 0; c < HD / 32; ++c) {
+                    float o[16];
+                    tmem_ld16(tO + lane_off + cg * (HD / 2) + c * 16, o);
+                    uint32_t u[16];
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
-                        float o[32];
-                        tmem_ld32(tO + lane_off + c * 32, o);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        tmem_st32(tO + lane_off + c * 32, o);
-                    }
+                    for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(o[i] * alpha);
+                    tmem_st16(tO + lane_off + cg * (HD / 2) + c * 16, u);
                 }
             }
             l = l * alpha + sum;
             m = mu;
-            uint8_t* prow = smem + Lay::P + r * 128;
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb) {
-#pragma unroll
-                for (int c8 = 0; c8 < 8; ++c8) {
-                    const float* v = s + kb * 64 + c8 * 8;
-                    uint4 u = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                                         pack_bf16(v[6], v[7]));
-                    *reinterpret_cast<uint4*>(prow + kb * 16384 + ((c8 ^ (r & 7)) << 4)) = u;
-                }
-            }
-            fence_proxy_async_smem();
+            tmem_st32u(tS + lane_off + sb * 128 + cg * 64, pk);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(p_full + 8 * sb);
         }
-        if (ok && warp_wait(o_done, (nblk - 1) & 1, abort_flag, p.status)) {
+        ok = ok && warp_wait(o_last, 0, abort_flag, p.status);
+        // row sums of both halves (buffer 0 of the maxima is free: the partner read
+        // this warp's last maximum before its P was handed over, which O needed)
+        mxs[cg * 128 + r] = l;
+        pair_sync(q);
+        if (ok) {
             tc_fence_after();
-            const float inv = 1.f / l;
+            const float lt = l + mxs[(cg ^ 1) * 128 + r];
+            const float inv = 1.f / lt;
             const bool live = qpos < p.T;
-            bf16* orow = p.o + ((size_t)row0 + qpos) * (size_t)(p.H * HD) + h * HD;
+            bf16* orow = p.o + ((size_t)row0 + qpos) * (size_t)(p.H * HD) + h * HD + cg * (HD / 2);
 #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
+            for (int c = 0; c < HD / 64; ++c) {
                 float o[32];
-                tmem_ld32(tO + lane_off + c * 32, o);
+                tmem_ld32(tO + lane_off + cg * (HD / 2) + c * 32, o);
                 if (live) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
@@ -268,7 +305,7 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                     }
                 }
             }
-            if (live) p.lse[((size_t)b * p.H + h) * attn_tpad(p.T) + qpos] = (m + __log2f(l)) * kLn2;
+            if (live && cg == 0) p.lse[((size_t)b * p.H + h) * attn_tpad(p.T) + qpos] = (m + __log2f(lt)) * kLn2;
         }
     }
     tc_fence_before();
