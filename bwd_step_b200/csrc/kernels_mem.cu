@@ -102,34 +102,66 @@ __global__ void embed_norm_bwd_kernel(const float* __restrict__ dx, const int32_
 }
 
 // ---------------------------------------------------------------- RMSNorm
-template <typename A>
+// One warp per row, lane l owns the 8-element chunks l*8 + 256*i.  With NCH > 0
+// (d <= 256*NCH) the row stays in registers between the reduction and the
+// output pass, so every input is read from memory once; NCH = 0 is the plain
+// two-pass loop for wider rows.
+template <typename A, int NCH>
 __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, A* __restrict__ y, float* __restrict__ r,
                                    int M, int d) {
     int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
     int lane = threadIdx.x & 31;
     if (row >= M) return;
     const float* src = x + (size_t)row * d;
-    float ss = 0.f;
-    for (int c = lane * 8; c < d; c += 256) {
-        float v[8];
-        load8(src + c, v);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) ss += v[k] * v[k];
-    }
-    ss = warp_sum(ss);
-    float rr = rsqrtf(ss / (float)d + kRmsEps);
     A* dst = y + (size_t)row * d;
-    for (int c = lane * 8; c < d; c += 256) {
-        float v[8];
-        load8(src + c, v);
+    float ss = 0.f;
+    if constexpr (NCH > 0) {
+        float v[NCH][8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] *= rr;
-        store8(dst + c, v);
+        for (int i = 0; i < NCH; ++i) {
+            const int c = lane * 8 + 256 * i;
+            if (c < d) load8(src + c, v[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            if (lane * 8 + 256 * i < d) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) ss += v[i][k] * v[i][k];
+            }
+        }
+        ss = warp_sum(ss);
+        const float rr = rsqrtf(ss / (float)d + kRmsEps);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int c = lane * 8 + 256 * i;
+            if (c < d) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[i][k] *= rr;
+                store8(dst + c, v[i]);
+            }
+        }
+        if (lane == 0) r[row] = rr;
+    } else {
+        for (int c = lane * 8; c < d; c += 256) {
+            float v[8];
+            load8(src + c, v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) ss += v[k] * v[k];
+        }
+        ss = warp_sum(ss);
+        const float rr = rsqrtf(ss / (float)d + kRmsEps);
+        for (int c = lane * 8; c < d; c += 256) {
+            float v[8];
+            load8(src + c, v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] *= rr;
+            store8(dst + c, v);
+        }
+        if (lane == 0) r[row] = rr;
     }
-    if (lane == 0) r[row] = rr;
 }
 
-template <typename A>
+template <typename A, int NCH>
 __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const A* __restrict__ y,
                                    const float* __restrict__ r, float* dx, bool accumulate, A* dxb,
                                    int M, int d) {
@@ -138,29 +170,64 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const A* __rest
     if (row >= M) return;
     const float* g = dy + (size_t)row * d;
     const A* yy = y + (size_t)row * d;
-    float dot = 0.f;
-    for (int c = lane * 8; c < d; c += 256) {
-        float a[8], b[8];
-        load8(g + c, a);
-        load8(yy + c, b);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) dot += a[k] * b[k];
-    }
-    dot = warp_sum(dot) / (float)d;
-    float rr = r[row];
     float* out = dx + (size_t)row * d;
-    for (int c = lane * 8; c < d; c += 256) {
-        float a[8], b[8], o[8];
-        load8(g + c, a);
-        load8(yy + c, b);
-        if (accumulate) load8(out + c, o);
+    const float rr = r[row];
+    float dot = 0.f;
+    if constexpr (NCH > 0) {
+        float a[NCH][8], b[NCH][8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            float v = rr * (a[k] - b[k] * dot);
-            o[k] = accumulate ? o[k] + v : v;
+        for (int i = 0; i < NCH; ++i) {
+            const int c = lane * 8 + 256 * i;
+            if (c < d) {
+                load8(g + c, a[i]);
+                load8(yy + c, b[i]);
+            }
         }
-        store8(out + c, o);
-        if (dxb) store8(dxb + (size_t)row * d + c, o);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            if (lane * 8 + 256 * i < d) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) dot += a[i][k] * b[i][k];
+            }
+        }
+        dot = warp_sum(dot) / (float)d;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int c = lane * 8 + 256 * i;
+            if (c < d) {
+                float o[8];
+                if (accumulate) load8(out + c, o);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float v = rr * (a[i][k] - b[i][k] * dot);
+                    o[k] = accumulate ? o[k] + v : v;
+                }
+                store8(out + c, o);
+                if (dxb) store8(dxb + (size_t)row * d + c, o);
+            }
+        }
+    } else {
+        for (int c = lane * 8; c < d; c += 256) {
+            float a[8], b[8];
+            load8(g + c, a);
+            load8(yy + c, b);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) dot += a[k] * b[k];
+        }
+        dot = warp_sum(dot) / (float)d;
+        for (int c = lane * 8; c < d; c += 256) {
+            float a[8], b[8], o[8];
+            load8(g + c, a);
+            load8(yy + c, b);
+            if (accumulate) load8(out + c, o);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float v = rr * (a[k] - b[k] * dot);
+                o[k] = accumulate ? o[k] + v : v;
+            }
+            store8(out + c, o);
+            if (dxb) store8(dxb + (size_t)row * d + c, o);
+        }
     }
 }
 
@@ -253,6 +320,9 @@ __global__ void __launch_bounds__(256) qknorm_rope_fwd_kernel(A* qkv, float* __r
     if (lane == 0) rqk[(size_t)m * nh + head] = r;
 }
 
+// One warp per position: the RoPE factors are loaded once, and the head
+// vectors of the position are processed G at a time with all their loads
+// issued before any of them is used.
 template <typename A, int HD>
 __global__ void __launch_bounds__(256) qknorm_rope_bwd_kernel(A* dqkv, const A* __restrict__ qkv,
                                                               const float* __restrict__ rqk,
@@ -260,37 +330,50 @@ __global__ void __launch_bounds__(256) qknorm_rope_bwd_kernel(A* dqkv, const A* 
                                                               const float* __restrict__ sin_t, int M, int T, int H,
                                                               int nkv) {
     using S = QkShape<HD>;
+    constexpr int G = 4;
     const int nh = H + nkv;
-    const int vi = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (vi >= M * nh) return;
-    const int m = vi / nh, head = vi % nh, pos = m % T;
+    const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (m >= M) return;
+    const int pos = m % T;
     const bool act = lane < S::LANES;
     const int l = act ? lane : 0;
-    const size_t off = (size_t)m * (size_t)(H + 2 * nkv) * HD + (size_t)head * HD + l * S::EPL;
-    float g[S::EPL], y[S::EPL];
-    ldN<A, S::EPL>(dqkv + off, g);
-    ldN<A, S::EPL>(qkv + off, y);
     const bool first = l * S::EPL < HD / 2;
-    const int j0 = first ? l * S::EPL : l * S::EPL - HD / 2;
-    float gu[S::EPL], yu[S::EPL], dot = 0.f;
+    const int j0 = first ? l * S::EPL : l * S::EPL - HD / 2;  // pair index of element 0
+    float cs[S::EPL], sn[S::EPL];
+    ldN<float, S::EPL>(cos_t + (size_t)pos * (HD / 2) + j0, cs);
+    ldN<float, S::EPL>(sin_t + (size_t)pos * (HD / 2) + j0, sn);
+    const size_t rowoff = (size_t)m * (size_t)(H + 2 * nkv) * HD + l * S::EPL;
+    for (int h0 = 0; h0 < nh; h0 += G) {
+        float g[G][S::EPL], y[G][S::EPL], r[G];
 #pragma unroll
-    for (int i = 0; i < S::EPL; ++i) {
-        const float go = __shfl_xor_sync(0xffffffffu, g[i], S::XOR);
-        const float yo = __shfl_xor_sync(0xffffffffu, y[i], S::XOR);
-        const float c = cos_t[pos * (HD / 2) + j0 + i], s = sin_t[pos * (HD / 2) + j0 + i];
-        // inverse rotation of (x1, x2): (x1 c + x2 s, -x1 s + x2 c)
-        const float g1 = first ? g[i] : go, g2 = first ? go : g[i];
-        const float y1 = first ? y[i] : yo, y2 = first ? yo : y[i];
-        gu[i] = first ? g1 * c + g2 * s : -g1 * s + g2 * c;
-        yu[i] = first ? y1 * c + y2 * s : -y1 * s + y2 * c;
-        dot += act ? gu[i] * yu[i] : 0.f;
+        for (int k = 0; k < G; ++k) {
+            if (h0 + k < nh) {
+                ldN<A, S::EPL>(dqkv + rowoff + (size_t)(h0 + k) * HD, g[k]);
+                ldN<A, S::EPL>(qkv + rowoff + (size_t)(h0 + k) * HD, y[k]);
+                r[k] = rqk[(size_t)m * nh + h0 + k];
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < G; ++k) {
+            if (h0 + k >= nh) break;
+            float gu[S::EPL], yu[S::EPL], dot = 0.f;
+#pragma unroll
+            for (int i = 0; i < S::EPL; ++i) {
+                const float go = __shfl_xor_sync(0xffffffffu, g[k][i], S::XOR);
+                const float yo = __shfl_xor_sync(0xffffffffu, y[k][i], S::XOR);
+                // inverse rotation of (x1, x2): (x1 c + x2 s, -x1 s + x2 c)
+                const float g1 = first ? g[k][i] : go, g2 = first ? go : g[k][i];
+                const float y1 = first ? y[k][i] : yo, y2 = first ? yo : y[k][i];
+                gu[i] = first ? g1 * cs[i] + g2 * sn[i] : -g1 * sn[i] + g2 * cs[i];
+                yu[i] = first ? y1 * cs[i] + y2 * sn[i] : -y1 * sn[i] + y2 * cs[i];
+                dot += act ? gu[i] * yu[i] : 0.f;
+            }
+            dot = warp_sum(dot) / (float)HD;
+#pragma unroll
+            for (int i = 0; i < S::EPL; ++i) gu[i] = r[k] * (gu[i] - yu[i] * dot);
+            if (act) stN<A, S::EPL>(dqkv + rowoff + (size_t)(h0 + k) * HD, gu);
+        }
     }
-    dot = warp_sum(dot) / (float)HD;
-    if (!act) return;
-    const float r = rqk[(size_t)m * nh + head];
-#pragma unroll
-    for (int i = 0; i < S::EPL; ++i) gu[i] = r * (gu[i] - yu[i] * dot);
-    stN<A, S::EPL>(dqkv + off, gu);
 }
 
 // ---------------------------------------------------------------- cross-entropy
@@ -606,22 +689,69 @@ cudaError_t launch_embed_norm_fwd(DType wt, const int32_t* idx, const void* wte,
 }
 
 cudaError_t launch_rmsnorm_fwd(DType at, const float* x, void* y, float* r, int M, int d, cudaStream_t s) {
-    if (at == DT_BF16)
-        rmsnorm_fwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(x, (bf16*)y, r, M, d);
-    else
-        rmsnorm_fwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(x, (float*)y, r, M, d);
+    const int nch = (d + 255) / 256;
+#define NC_RMS_FWD(A, N) rmsnorm_fwd_kernel<A, N><<<row_blocks(M), 256, 0, s>>>(x, (A*)y, r, M, d)
+    if (at == DT_BF16) {
+        switch (nch) {
+            case 1: NC_RMS_FWD(bf16, 1); break;
+            case 2: NC_RMS_FWD(bf16, 2); break;
+            case 3: NC_RMS_FWD(bf16, 3); break;
+            case 4: NC_RMS_FWD(bf16, 4); break;
+            case 5: NC_RMS_FWD(bf16, 5); break;
+            case 6: NC_RMS_FWD(bf16, 6); break;
+            case 7: NC_RMS_FWD(bf16, 7); break;
+            case 8: NC_RMS_FWD(bf16, 8); break;
+            default: NC_RMS_FWD(bf16, 0); break;
+        }
+    } else {
+        switch (nch) {
+            case 1: NC_RMS_FWD(float, 1); break;
+            case 2: NC_RMS_FWD(float, 2); break;
+            case 3: NC_RMS_FWD(float, 3); break;
+            case 4: NC_RMS_FWD(float, 4); break;
+            case 5: NC_RMS_FWD(float, 5); break;
+            case 6: NC_RMS_FWD(float, 6); break;
+            case 7: NC_RMS_FWD(float, 7); break;
+            case 8: NC_RMS_FWD(float, 8); break;
+            default: NC_RMS_FWD(float, 0); break;
+        }
+    }
+#undef NC_RMS_FWD
     count_launch();
     return cudaGetLastError();
 }
 
 cudaError_t launch_rmsnorm_bwd(DType at, const float* dy, const void* y, const float* r, float* dx,
                                bool accumulate, void* dxb, int M, int d, cudaStream_t s) {
-    if (at == DT_BF16)
-        rmsnorm_bwd_kernel<bf16><<<row_blocks(M), 256, 0, s>>>(dy, (const bf16*)y, r, dx, accumulate,
-                                                               (bf16*)dxb, M, d);
-    else
-        rmsnorm_bwd_kernel<float><<<row_blocks(M), 256, 0, s>>>(dy, (const float*)y, r, dx, accumulate,
-                                                                (float*)dxb, M, d);
+    const int nch = (d + 255) / 256;
+#define NC_RMS_BWD(A, N) \
+    rmsnorm_bwd_kernel<A, N><<<row_blocks(M), 256, 0, s>>>(dy, (const A*)y, r, dx, accumulate, (A*)dxb, M, d)
+    if (at == DT_BF16) {
+        switch (nch) {
+            case 1: NC_RMS_BWD(bf16, 1); break;
+            case 2: NC_RMS_BWD(bf16, 2); break;
+            case 3: NC_RMS_BWD(bf16, 3); break;
+            case 4: NC_RMS_BWD(bf16, 4); break;
+            case 5: NC_RMS_BWD(bf16, 5); break;
+            case 6: NC_RMS_BWD(bf16, 6); break;
+            case 7: NC_RMS_BWD(bf16, 7); break;
+            case 8: NC_RMS_BWD(bf16, 8); break;
+            default: NC_RMS_BWD(bf16, 0); break;
+        }
+    } else {
+        switch (nch) {
+            case 1: NC_RMS_BWD(float, 1); break;
+            case 2: NC_RMS_BWD(float, 2); break;
+            case 3: NC_RMS_BWD(float, 3); break;
+            case 4: NC_RMS_BWD(float, 4); break;
+            case 5: NC_RMS_BWD(float, 5); break;
+            case 6: NC_RMS_BWD(float, 6); break;
+            case 7: NC_RMS_BWD(float, 7); break;
+            case 8: NC_RMS_BWD(float, 8); break;
+            default: NC_RMS_BWD(float, 0); break;
+        }
+    }
+#undef NC_RMS_BWD
     count_launch();
     return cudaGetLastError();
 }
@@ -645,7 +775,7 @@ static void qk_fwd_t(void* qkv, float* rqk, const float* c, const float* sn, int
 template <typename A, int HD>
 static void qk_bwd_t(void* dqkv, const void* qkv, const float* rqk, const float* c, const float* sn, int M, int T,
                      int H, int nkv, cudaStream_t s) {
-    const long long vecs = (long long)M * (H + nkv);
+    const long long vecs = M;  // one warp per position
     qknorm_rope_bwd_kernel<A, HD><<<(unsigned)((vecs + 7) / 8), 256, 0, s>>>((A*)dqkv, (const A*)qkv, rqk, c, sn, M,
                                                                               T, H, nkv);
 }
