@@ -37,9 +37,9 @@ cudaError_t launch_qknorm_rope_fwd(DType at, void* qkv, float* rqk, const float*
 cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const float* rqk,
                                    const float* cos_t, const float* sin_t, int M, int T, int H, int nkv,
                                    int hd, cudaStream_t s);
-// Cross-entropy over R rows of softcapped logits z [R, V] (fp32):
+// Cross-entropy over R rows of softcapped logits z [R, V] (fp32 or bf16, V % 4 == 0):
 // loss_rows[r] = lse - z[tgt]; dl = inv_M*(softmax - onehot)*(1-(z/cap)^2).
-cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R, int V, float cap,
+cudaError_t launch_ce_chunk(DType zt, DType dlt, const void* z, const int32_t* tgt, int R, int V, float cap,
                             float inv_M, float* loss_rows, void* dl, int* status, cudaStream_t s);
 // loss = mean(loss_rows[0..M)), fixed summation order.
 cudaError_t launch_loss_reduce(const float* loss_rows, int M, float* loss, cudaStream_t s);

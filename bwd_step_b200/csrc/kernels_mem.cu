@@ -397,52 +397,67 @@ __device__ __forceinline__ void store4(bf16* p, const float* v) {
     *reinterpret_cast<uint2*>(p) = u;
 }
 
-// dl for one row given its LSE: one pass over z (4 logits per thread step).
-template <typename D>
-__device__ __forceinline__ void ce_write_dl(const float* zr, D* out, int V, int t, bool bad, float lse, float cap,
-                                            float inv_M) {
-    const float inv_cap = 1.f / cap;
-    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
-        const float4 v = *reinterpret_cast<const float4*>(zr + c);
-        const float zz[4] = {v.x, v.y, v.z, v.w};
-        float g[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float pk = __expf(zz[k] - lse) - ((c + k) == t ? 1.f : 0.f);
-            const float q = zz[k] * inv_cap;
-            g[k] = bad ? 0.f : pk * inv_M * (1.f - q * q);
-        }
-        store4(out + c, g);
-    }
+// four logits (fp32 or bf16) as floats
+__device__ __forceinline__ void load4z(const float* p, float* v) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+__device__ __forceinline__ void load4z(const bf16* p, float* v) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
 }
 
-template <typename D>
-__global__ void ce_chunk_kernel(const float* __restrict__ z, const int32_t* __restrict__ tgt, int R, int V,
-                                float cap, float inv_M, float* __restrict__ loss_rows, D* __restrict__ dl,
-                                int* status) {
+// Loss and dl of one chunk of rows, one 1024-thread block per row (V % 4 == 0).
+// Pass 1: running (max, sum of exp) over the row's softcapped logits z, two
+// vectors of 4 logits in flight per thread (two blocks per SM); the block combines the partials
+// into the LSE.  Pass 2 reads the row again (from L2: about 300 rows are in
+// flight) and writes dl = (softmax - onehot) / M * (1 - (z/cap)^2).
+template <typename Z, typename D>
+__global__ void __launch_bounds__(1024, 2) ce_chunk_kernel(const Z* __restrict__ z, const int32_t* __restrict__ tgt,
+                                                        int R, int V, float cap, float inv_M,
+                                                        float* __restrict__ loss_rows, D* __restrict__ dl,
+                                                        int* status) {
+    constexpr float kL2e = 1.44269504088896340736f;
+    constexpr int U = 2;
     __shared__ MaxSum red[32];
     __shared__ float s_lse;
-    int row = blockIdx.x;
-    const float* zr = z + (size_t)row * V;
+    const int row = blockIdx.x;
+    const Z* zr = z + (size_t)row * V;
+    const int stride = blockDim.x * 4;
     MaxSum acc = {-INFINITY, 0.f};
-    for (int c = threadIdx.x * 4; c < V; c += blockDim.x * 4) {
-        float4 v = *reinterpret_cast<const float4*>(zr + c);
-        float m4 = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
-        float m = fmaxf(acc.m, m4);
-        float s = (acc.s == 0.f ? 0.f : acc.s * expf(acc.m - m));
-        s += expf(v.x - m) + expf(v.y - m) + expf(v.z - m) + expf(v.w - m);
-        acc = {m, s};
+    for (int c0 = threadIdx.x * 4; c0 < V; c0 += U * stride) {
+        float v[U][4];
+        float m = acc.m;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + u * stride;
+            if (c < V) {
+                load4z(zr + c, v[u]);
+            } else {
+                v[u][0] = v[u][1] = v[u][2] = v[u][3] = -INFINITY;
+            }
+            m = fmaxf(m, fmaxf(fmaxf(v[u][0], v[u][1]), fmaxf(v[u][2], v[u][3])));
+        }
+        const float m2 = m * kL2e;
+        float sacc = acc.s == 0.f ? 0.f : acc.s * exp2f(fmaf(acc.m, kL2e, -m2));
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sacc += exp2f(fmaf(v[u][k], kL2e, -m2));
+        acc = {m, sacc};
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         MaxSum other = {__shfl_xor_sync(0xffffffffu, acc.m, o), __shfl_xor_sync(0xffffffffu, acc.s, o)};
         acc = ms_combine(acc, other);
     }
-    int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (lane == 0) red[w] = acc;
     __syncthreads();
     if (w == 0) {
-        int nw = blockDim.x >> 5;
+        const int nw = blockDim.x >> 5;
         acc = lane < nw ? red[lane] : MaxSum{-INFINITY, 0.f};
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -452,14 +467,36 @@ __global__ void ce_chunk_kernel(const float* __restrict__ z, const int32_t* __re
         if (lane == 0) s_lse = acc.m + logf(acc.s);
     }
     __syncthreads();
-    float lse = s_lse;
-    int t = tgt[row];
-    bool bad = t < 0 || t >= V;
+    const float lse = s_lse;
+    const int t = tgt[row];
+    const bool bad = t < 0 || t >= V;
     if (threadIdx.x == 0) {
         if (bad) set_status(status, ST_BAD_TOKEN);
-        loss_rows[row] = bad ? 0.f : lse - zr[t];
+        loss_rows[row] = bad ? 0.f : lse - tof(zr[t]);
     }
-    ce_write_dl(zr, dl + (size_t)row * V, V, t, bad, lse, cap, inv_M);
+    const float inv_cap = 1.f / cap, lse2 = lse * kL2e;
+    D* out = dl + (size_t)row * V;
+    for (int c0 = threadIdx.x * 4; c0 < V; c0 += U * stride) {
+        float v[U][4];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + u * stride;
+            if (c < V) load4z(zr + c, v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + u * stride;
+            if (c >= V) break;
+            float g[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float pk = exp2f(fmaf(v[u][k], kL2e, -lse2)) - ((c + k) == t ? 1.f : 0.f);
+                const float q = v[u][k] * inv_cap;
+                g[k] = bad ? 0.f : pk * inv_M * (1.f - q * q);
+            }
+            store4(out + c, g);
+        }
+    }
 }
 
 __global__ void loss_reduce_kernel(const float* __restrict__ rows, int M, float* loss) {
@@ -819,15 +856,18 @@ cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const 
                          : qk_bwd_d<float>(dqkv, qkv, rqk, c, sn, M, T, H, nkv, hd, s);
 }
 
-cudaError_t launch_ce_chunk(DType dlt, const float* z, const int32_t* tgt, int R, int V, float cap, float inv_M,
-                            float* loss_rows, void* dl, int* status, cudaStream_t s) {
+cudaError_t launch_ce_chunk(DType zt, DType dlt, const void* z, const int32_t* tgt, int R, int V, float cap,
+                            float inv_M, float* loss_rows, void* dl, int* status, cudaStream_t s) {
     if (R <= 0) return cudaSuccess;
-    // 1024 threads per row: about 300 rows in flight (76 MB of fp32 logits at V =
-    // 65536), so each row's second pass reads it back from L2, not HBM
-    if (dlt == DT_BF16)
-        ce_chunk_kernel<bf16><<<R, 1024, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (bf16*)dl, status);
-    else
-        ce_chunk_kernel<float><<<R, 1024, 0, s>>>(z, tgt, R, V, cap, inv_M, loss_rows, (float*)dl, status);
+    if (V % 4 != 0) return cudaErrorInvalidValue;
+#define NC_CE(ZT, DT) \
+    ce_chunk_kernel<ZT, DT><<<R, 1024, 0, s>>>((const ZT*)z, tgt, R, V, cap, inv_M, loss_rows, (DT*)dl, status)
+    if (zt == DT_BF16) {
+        if (dlt == DT_BF16) NC_CE(bf16, bf16); else NC_CE(bf16, float);
+    } else {
+        if (dlt == DT_BF16) NC_CE(float, bf16); else NC_CE(float, float);
+    }
+#undef NC_CE
     count_launch();
     return cudaGetLastError();
 }

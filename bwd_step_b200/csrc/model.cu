@@ -310,7 +310,9 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     // ---- LM head + softcap + cross-entropy, then its backward, R rows at a time
     void* xf = c.at(c.p.xf);
     float* gbuf = c.at<float>(c.p.g);
-    float* zc = c.at<float>(c.p.zc);
+    // softcapped logits in the activation type (bf16 on the mixed-precision path, as
+    // the autocast LM head of the reference produces them; fp32 on the debug path)
+    void* zc = c.at(c.p.zc);
     void* dlc = c.at(c.p.dlc);
     float* loss_rows = c.at<float>(c.p.loss_rows);
     const size_t A = dt_size(m->at);
@@ -318,11 +320,11 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     for (int r0 = 0; r0 < M; r0 += c.p.R) {
         int rc = std::min(c.p.R, M - r0);
         const char* xfc = (const char*)xf + (size_t)r0 * d * A;
-        RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, DT_F32), P_GEMM_LM_Z));
+        RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, m->at), P_GEMM_LM_Z));
         {
-            Prof pr(c, P_CE, 0.0, (double)rc * V * (4.0 + A));
-            CK(launch_ce_chunk(m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M, loss_rows + r0, dlc,
-                               m->status, s));
+            Prof pr(c, P_CE, 0.0, (double)rc * V * (2.0 * A));
+            CK(launch_ce_chunk(m->at, m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M, loss_rows + r0,
+                               dlc, m->status, s));
         }
         RG(run_gemm(c, mk(m, rc, d, V, dlc, V, true, w.wlm(), d, false, EPI_STORE, gbuf + (size_t)r0 * d, d,
                           DT_F32), P_GEMM_LM_DX));
