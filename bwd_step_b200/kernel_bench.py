@@ -37,7 +37,7 @@ GEMMS = {
     "wgrad_fc": (F, D, M, 0, 0, 0, 0),
     "wgrad_oproj": (D, HHD, M, 0, 0, 0, 0),
     "wgrad_qkv": (NQKV, D, M, 0, 0, 0, 0),
-    "lmhead_z": (R, V, D, 1, 1, 4, 0),
+    "lmhead_z": (R, V, D, 1, 1, 4, 1),
     "lmhead_dx": (R, D, V, 1, 0, 0, 0),
     "lmhead_dw": (V, D, R, 0, 0, 1, 0),
 }
