@@ -499,6 +499,122 @@ __global__ void __launch_bounds__(1024, 2) ce_chunk_kernel(const Z* __restrict__
     }
 }
 
+// Loss and dl of one chunk of rows with bf16 logits, the whole row resident in
+// registers as packed bf16 (one 512-thread block per row, CER_K 16-byte vectors
+// per thread issued at once): the logits are read from HBM once and dl written
+// once, with two block reductions (max, then sum of 2^((z - max)*log2 e)) in
+// between.  For V a multiple of CER_NT * 8 up to CER_NT * CER_K * 8.
+constexpr int CER_NT = 512, CER_K = 16;
+
+// 2^x on the special-function unit (PTX ex2.approx, flush-to-zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void store8f(float* p, const float* g) {
+    *reinterpret_cast<float4*>(p) = make_float4(g[0], g[1], g[2], g[3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(g[4], g[5], g[6], g[7]);
+}
+
+// block-wide reduction of one float (max or sum) over CER_NT threads
+template <bool MAX>
+__device__ __forceinline__ float ce_block_reduce(float v, float* red) {
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    v = MAX ? warp_max(v) : warp_sum(v);
+    if (lane == 0) red[w] = v;
+    __syncthreads();
+    float r = red[0];
+#pragma unroll
+    for (int i = 1; i < CER_NT / 32; ++i) r = MAX ? fmaxf(r, red[i]) : r + red[i];
+    __syncthreads();  // red is reused by the next reduction
+    return r;
+}
+
+template <typename D>
+__global__ void __launch_bounds__(CER_NT, 1) ce_chunk_resident_kernel(const bf16* __restrict__ z,
+                                                                       const int32_t* __restrict__ tgt, int V,
+                                                                       float cap, float inv_M,
+                                                                       float* __restrict__ loss_rows,
+                                                                       D* __restrict__ dl, int* status) {
+    constexpr float kL2e = 1.44269504088896340736f;
+    constexpr int STEP = CER_NT * 8;  // logits per vector slot of the block
+    __shared__ float red[CER_NT / 32];
+    const int row = blockIdx.x;
+    const int nk = V / STEP;  // V % STEP == 0: every slot is full or unused for all threads
+    const bf16* zr = z + (size_t)row * V;
+    const bf16* zt = zr + threadIdx.x * 8;
+    uint4 v[CER_K];
+#pragma unroll
+    for (int k = 0; k < CER_K; ++k)
+        if (k < nk) v[k] = *reinterpret_cast<const uint4*>(zt + k * STEP);
+    float mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < CER_K; ++k) {
+        if (k < nk) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h[i]);
+                mx = fmaxf(mx, fmaxf(f.x, f.y));
+            }
+        }
+    }
+    mx = ce_block_reduce<true>(mx, red);
+    const float m2 = mx * kL2e;
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < CER_K; ++k) {
+        if (k < nk) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h[i]);
+                sum += ex2_approx(fmaf(f.x, kL2e, -m2)) + ex2_approx(fmaf(f.y, kL2e, -m2));
+            }
+        }
+    }
+    sum = ce_block_reduce<false>(sum, red);
+    const float lse = mx + logf(sum);
+    const int t = tgt[row];
+    const bool bad = t < 0 || t >= V;
+    if (threadIdx.x == 0) {
+        if (bad) set_status(status, ST_BAD_TOKEN);
+        loss_rows[row] = bad ? 0.f : lse - __bfloat162float(zr[t]);
+    }
+    const float inv_cap = 1.f / cap, lse2 = lse * kL2e;
+    const float gs = bad ? 0.f : inv_M;
+    const int tl = t - (int)threadIdx.x * 8;  // target relative to this thread's first logit
+    D* out = dl + (size_t)row * V + threadIdx.x * 8;
+#pragma unroll
+    for (int k = 0; k < CER_K; ++k) {
+        if (k < nk) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[k]);
+            const int tk = tl - k * STEP;  // in 0..7 when the target is in this vector
+            uint32_t w[4];
+            float g[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h[i]);
+                const float q0 = f.x * inv_cap, q1 = f.y * inv_cap;
+                const float p0 = ex2_approx(fmaf(f.x, kL2e, -lse2)) - (tk == 2 * i ? 1.f : 0.f);
+                const float p1 = ex2_approx(fmaf(f.y, kL2e, -lse2)) - (tk == 2 * i + 1 ? 1.f : 0.f);
+                g[2 * i] = p0 * gs * (1.f - q0 * q0);
+                g[2 * i + 1] = p1 * gs * (1.f - q1 * q1);
+                if constexpr (sizeof(D) == 2) {
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(g[2 * i], g[2 * i + 1]);
+                    w[i] = *reinterpret_cast<uint32_t*>(&b2);
+                }
+            }
+            if constexpr (sizeof(D) == 2)
+                *reinterpret_cast<uint4*>(out + k * STEP) = make_uint4(w[0], w[1], w[2], w[3]);
+            else
+                store8f(reinterpret_cast<float*>(out) + k * STEP, g);
+        }
+    }
+}
+
 __global__ void loss_reduce_kernel(const float* __restrict__ rows, int M, float* loss) {
     __shared__ float sh[1024];
     float s = 0.f;
@@ -860,6 +976,16 @@ cudaError_t launch_ce_chunk(DType zt, DType dlt, const void* z, const int32_t* t
                             float inv_M, float* loss_rows, void* dl, int* status, cudaStream_t s) {
     if (R <= 0) return cudaSuccess;
     if (V % 4 != 0) return cudaErrorInvalidValue;
+    if (zt == DT_BF16 && V % (CER_NT * 8) == 0 && V <= CER_NT * CER_K * 8) {
+        if (dlt == DT_BF16)
+            ce_chunk_resident_kernel<bf16><<<R, CER_NT, 0, s>>>((const bf16*)z, tgt, V, cap, inv_M, loss_rows,
+                                                                (bf16*)dl, status);
+        else
+            ce_chunk_resident_kernel<float><<<R, CER_NT, 0, s>>>((const bf16*)z, tgt, V, cap, inv_M, loss_rows,
+                                                                 (float*)dl, status);
+        count_launch();
+        return cudaGetLastError();
+    }
 #define NC_CE(ZT, DT) \
     ce_chunk_kernel<ZT, DT><<<R, 1024, 0, s>>>((const ZT*)z, tgt, R, V, cap, inv_M, loss_rows, (DT*)dl, status)
     if (zt == DT_BF16) {
