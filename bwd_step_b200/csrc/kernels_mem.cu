@@ -784,11 +784,20 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits,
                                      float* __restrict__ out, bool accumulate) {
     size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n4) return;
-    const float4* p = reinterpret_cast<const float4*>(part);
+    const float4* p = reinterpret_cast<const float4*>(part) + i;
     float4 acc = accumulate ? reinterpret_cast<float4*>(out)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < splits; ++s) {
-        float4 g = p[(size_t)s * n4 + i];
-        acc.x += g.x; acc.y += g.y; acc.z += g.z; acc.w += g.w;
+    // partials added in split order, all loads (up to eight) issued first
+    constexpr int KMAX = 8;
+    float4 g[KMAX];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k)
+        if (k < splits) g[k] = p[(size_t)k * n4];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k)
+        if (k < splits) { acc.x += g[k].x; acc.y += g[k].y; acc.z += g[k].z; acc.w += g[k].w; }
+    for (int k = KMAX; k < splits; ++k) {
+        const float4 h = p[(size_t)k * n4];
+        acc.x += h.x; acc.y += h.y; acc.z += h.z; acc.w += h.w;
     }
     reinterpret_cast<float4*>(out)[i] = acc;
 }
