@@ -5,9 +5,9 @@
 // scaled by 1/sqrt(hd).
 //
 // Forward, one CTA per (query block of 128 positions, head, batch row):
-//   warp 0     TMA: the Q tile once, then K_j (lane 0) and V_j (lane 1) in
-//              3-stage rings for key blocks j = 0..qb (causal: blocks past
-//              the diagonal are never loaded);
+//   warp 0     TMA: the Q tile once, then K_j and V_j together in a 3-stage
+//              ring for key blocks j = 0..qb (causal: blocks past the
+//              diagonal are never loaded);
 //   warp 1     tcgen05.mma: S_j = Q K_j^T into one of two 128-column TMEM
 //              buffers, two blocks ahead; O += P_j V_j with P_j read from
 //              TMEM (A operand) and V_j as an MN-major operand;
@@ -29,7 +29,7 @@ namespace {
 using namespace tc;
 
 constexpr int NT = 320;  // forward: producer, MMA, 8 softmax warps (two per TMEM lane quarter)
-constexpr int FSTG = 3;  // K and V ring stages
+constexpr int FSTG = 3;  // K/V ring stages
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -95,10 +95,10 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t q_full = b0;
-    const uint32_t k_full = b0 + 8, k_empty = b0 + 32, v_full = b0 + 56, v_empty = b0 + 80;  // [FSTG]
-    const uint32_t s_full = b0 + 104, p_full = b0 + 120;  // [2]: per TMEM score buffer
-    const uint32_t o_last = b0 + 136;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+    const uint32_t kv_full = b0 + 8, kv_empty = b0 + 32;  // [FSTG]: K_j and V_j share a stage
+    const uint32_t s_full = b0 + 56, p_full = b0 + 72;    // [2]: per TMEM score buffer
+    const uint32_t o_last = b0 + 88;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -109,10 +109,7 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < FSTG; ++s) {
-            mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1);
-            mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1);
-        }
+        for (int s = 0; s < FSTG; ++s) { mbar_init(kv_full + 8 * s, 1); mbar_init(kv_empty + 8 * s, 1); }
         for (int s = 0; s < 2; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(p_full + 8 * s, 8); }
         mbar_init(o_last, 1);
         *abort_flag = 0;
@@ -127,36 +124,32 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
     const uint32_t tS = tmem, tO = tmem + 256;  // S[2] of 128 columns, O (HD columns)
 
     if (warp == 0) {
-        // lane 0 loads Q and the K ring (a slot frees once S_j is computed), lane 1
-        // the V ring (a slot frees after O += P_j V_j)
-        if (lane < 2) {
-            const bool kl = lane == 0;
-            const int xq = h * HD, xkv = kl ? (p.H + g) * HD : (p.H + p.nkv + g) * HD;
-            const uint32_t full = kl ? k_full : v_full, empty = kl ? k_empty : v_empty;
-            const uint32_t dst = kl ? sK : sV;
-            if (kl) {
-                mbar_expect_tx(q_full, TILE);
+        // one thread loads Q, then K_j and V_j together into a 3-stage ring (a stage
+        // frees after O += P_j V_j): one wait per key block for the MMA thread
+        if (lane == 0) {
+            const int xq = h * HD, xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
+            mbar_expect_tx(q_full, TILE);
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb)
-                    tma_load_2d(sQ + kb * 16384, &tm, xq + kb * 64, row0 + qb * 128, q_full);
-            }
+            for (int kb = 0; kb < KB; ++kb) tma_load_2d(sQ + kb * 16384, &tm, xq + kb * 64, row0 + qb * 128, q_full);
             int issued = 0;
             for (int j = 0; j < nblk; ++j) {
                 const int st = j % FSTG;
-                if (!mbar_wait(empty + 8 * st, ((j / FSTG) & 1) ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(full + 8 * st, TILE);
+                if (!mbar_wait(kv_empty + 8 * st, ((j / FSTG) & 1) ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(kv_full + 8 * st, 2 * TILE);
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb)
-                    tma_load_2d(dst + st * TILE + kb * 16384, &tm, xkv + kb * 64, row0 + j * 128, full + 8 * st);
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_2d(sK + st * TILE + kb * 16384, &tm, xk + kb * 64, row0 + j * 128, kv_full + 8 * st);
+                    tma_load_2d(sV + st * TILE + kb * 16384, &tm, xv + kb * 64, row0 + j * 128, kv_full + 8 * st);
+                }
                 issued = j + 1;
             }
             if (*abort_flag) {
                 // let copies in flight land before the block exits
                 uint64_t t0 = globaltimer();
-                if (kl) while (!mbar_try(q_full, 0) && globaltimer() - t0 < 1000000ull) {}
+                while (!mbar_try(q_full, 0) && globaltimer() - t0 < 1000000ull) {}
                 for (int j = (issued > FSTG ? issued - FSTG : 0); j < issued; ++j) {
                     t0 = globaltimer();
-                    while (!mbar_try(full + 8 * (j % FSTG), (j / FSTG) & 1) && globaltimer() - t0 < 1000000ull) {}
+                    while (!mbar_try(kv_full + 8 * (j % FSTG), (j / FSTG) & 1) && globaltimer() - t0 < 1000000ull) {}
                 }
             }
         }
@@ -167,7 +160,7 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
             // S_j = Q K_j^T into buffer j & 1
             auto scores = [&](int j) -> bool {
                 const int st = j % FSTG, sb = j & 1;
-                if (!mbar_wait(k_full + 8 * st, (j / FSTG) & 1, abort_flag, p.status)) return false;
+                if (!mbar_wait(kv_full + 8 * st, (j / FSTG) & 1, abort_flag, p.status)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < HD / 16; ++ks) {
@@ -176,7 +169,6 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                              id_s, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full + 8 * sb);
-                mma_commit(k_empty + 8 * st);
                 return true;
             };
             bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && scores(0) && (nblk < 2 || scores(1));
@@ -184,14 +176,14 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 const int st = j % FSTG, sb = j & 1;
                 // O += P_j V_j: keys 16kk..16kk+15 sit in the packed columns
                 // 64*(kk/4) + 8*(kk%4) of score buffer j & 1 (written by column group kk/4)
+                // (V_j landed with K_j, waited for before S_j)
                 if (!mbar_wait(p_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status)) break;
-                if (!mbar_wait(v_full + 8 * st, (j / FSTG) & 1, abort_flag, p.status)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_bf16_ts(tO, tS + sb * 128 + 64 * (kk >> 2) + 8 * (kk & 3),
                                 smem_desc(sV + st * TILE + kk * 2048, 16384, 1024), id_o, (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(v_empty + 8 * st);
+                mma_commit(kv_empty + 8 * st);
                 // S_{j+2} overwrites P_j only after these MMAs (issue order)
                 if (j + 2 < nblk && !scores(j + 2)) break;
             }
@@ -255,10 +247,10 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 pk[c >> 1] = pack_bf16(e0, e1);
             }
             if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-                // O += P_{j-1} V_{j-1} has finished (its V slot was released); O(j) cannot
+                // O += P_{j-1} V_{j-1} has finished (its K/V stage was released); O(j) cannot
                 // have started, so this phase of the barrier is the latest one
                 const int jj = j - 1;
-                ok = warp_wait(v_empty + 8 * (jj % FSTG), (jj / FSTG) & 1, abort_flag, p.status);
+                ok = warp_wait(kv_empty + 8 * (jj % FSTG), (jj / FSTG) & 1, abort_flag, p.status);
                 if (!ok) continue;
                 tc_fence_after();
                 // this warp rescales its half of the O columns
@@ -327,7 +319,8 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 //
 // dQ, one CTA per (query block of 128, head, batch row), key blocks j = 0..qb:
 //   warp 0      TMA: Q and dO once; K_j into a 3-stage ring (freed by the dQ
-//               MMA), V_j into a 2-stage ring (freed by the dP MMA);
+//               MMA), V_j into a 2-stage ring (freed by the dP MMA), both on
+//               one barrier per key block;
 //   warp 1      tcgen05.mma: S_j = Q K_j^T into one of two TMEM buffers and
 //               dP_j = dO V_j^T into one buffer as one group of 16 MMAs
 //               (every wait or commit between 128-wide MMAs idles the tensor
@@ -430,8 +423,8 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t qd_full = b0;
-    const uint32_t k_full = b0 + 8, k_empty = b0 + 32;   // [KSTG]
-    const uint32_t v_full = b0 + 56, v_empty = b0 + 72;  // [VSTG]
+    const uint32_t k_empty = b0 + 32;                    // [KSTG]
+    const uint32_t v_full = b0 + 56, v_empty = b0 + 72;  // [VSTG]: v_full covers K_j and V_j
     const uint32_t dp_full = b0 + 104, dp_free = b0 + 112;
     const uint32_t ds_full = b0 + 120;                   // [2]: dS_j written over buffer j & 1
     const uint32_t dq_done = b0 + 136;
@@ -447,7 +440,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
 
     if (threadIdx.x == 0) {
         mbar_init(qd_full, 1);
-        for (int s = 0; s < KSTG; ++s) { mbar_init(k_full + 8 * s, 1); mbar_init(k_empty + 8 * s, 1); }
+        for (int s = 0; s < KSTG; ++s) mbar_init(k_empty + 8 * s, 1);
         for (int s = 0; s < VSTG; ++s) { mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1); }
         for (int s = 0; s < 2; ++s) mbar_init(ds_full + 8 * s, NSM);
         mbar_init(dp_full, 1);
@@ -465,34 +458,35 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
     const uint32_t tS = tmem, tdP = tmem + 256, tdQ = tmem + 384;  // S[2] of 128 columns, dP, dQ
 
     if (warp == 0) {
-        // lane 0 loads Q, dO and the K ring, lane 1 the V ring
-        if (lane < 2) {
-            const bool kl = lane == 0;
-            const int xkv = (kl ? p.H + g : p.H + p.nkv + g) * HD;
-            const int nst = kl ? KSTG : VSTG;
-            const uint32_t full = kl ? k_full : v_full, empty = kl ? k_empty : v_empty;
-            const uint32_t dst = kl ? sK : sV;
-            if (kl) {
-                mbar_expect_tx(qd_full, 2 * TILE);
+        // one thread loads Q and dO, then per key block K_j into the 3-stage K ring
+        // (a slot frees after the dQ MMA) and V_j into the 2-stage V ring (after
+        // the dP MMA); both land on the V stage's barrier, so the MMA thread waits
+        // once per key block
+        if (lane == 0) {
+            const int xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
+            mbar_expect_tx(qd_full, 2 * TILE);
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_2d(sQ + kb * 16384, &tmQKV, h * HD + kb * 64, row0 + qb * 128, qd_full);
-                    tma_load_2d(sDO + kb * 16384, &tmDO, h * HD + kb * 64, row0 + qb * 128, qd_full);
-                }
+            for (int kb = 0; kb < KB; ++kb) {
+                tma_load_2d(sQ + kb * 16384, &tmQKV, h * HD + kb * 64, row0 + qb * 128, qd_full);
+                tma_load_2d(sDO + kb * 16384, &tmDO, h * HD + kb * 64, row0 + qb * 128, qd_full);
             }
             int issued = 0;
             for (int j = 0; j < nblk; ++j) {
-                const int st = j % nst;
-                if (!mbar_wait(empty + 8 * st, ((j / nst) & 1) ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(full + 8 * st, TILE);
+                const int kst = j % KSTG, vst = j % VSTG;
+                if (!mbar_wait(k_empty + 8 * kst, ((j / KSTG) & 1) ^ 1, abort_flag, p.status)) break;
+                if (!mbar_wait(v_empty + 8 * vst, ((j / VSTG) & 1) ^ 1, abort_flag, p.status)) break;
+                mbar_expect_tx(v_full + 8 * vst, 2 * TILE);
 #pragma unroll
-                for (int kb = 0; kb < KB; ++kb)
-                    tma_load_2d(dst + st * TILE + kb * 16384, &tmQKV, xkv + kb * 64, row0 + j * 128, full + 8 * st);
+                for (int kb = 0; kb < KB; ++kb) {
+                    tma_load_2d(sK + kst * TILE + kb * 16384, &tmQKV, xk + kb * 64, row0 + j * 128, v_full + 8 * vst);
+                    tma_load_2d(sV + vst * TILE + kb * 16384, &tmQKV, xv + kb * 64, row0 + j * 128, v_full + 8 * vst);
+                }
                 issued = j + 1;
             }
             if (*abort_flag) {
-                if (kl) drain(qd_full, 0);
-                for (int j = (issued > nst ? issued - nst : 0); j < issued; ++j) drain(full + 8 * (j % nst), (j / nst) & 1);
+                drain(qd_full, 0);
+                for (int j = (issued > VSTG ? issued - VSTG : 0); j < issued; ++j)
+                    drain(v_full + 8 * (j % VSTG), (j / VSTG) & 1);
             }
         }
     } else if (warp == 1) {
@@ -504,7 +498,6 @@ __global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constan
                 if (j < nblk) {
                     // S_j and dP_j as one group: K_j, V_j landed, dP_{j-1} read out of TMEM
                     const int kst = j % KSTG, vst = j % VSTG, sb = j & 1;
-                    if (!mbar_wait(k_full + 8 * kst, (j / KSTG) & 1, abort_flag, p.status)) break;
                     if (!mbar_wait(v_full + 8 * vst, (j / VSTG) & 1, abort_flag, p.status)) break;
                     if (j > 0 && !mbar_wait(dp_free, (j - 1) & 1, abort_flag, p.status)) break;
                     tc_fence_after();
