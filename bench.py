@@ -88,6 +88,47 @@ def profile_traffic(kernel):
     return float(vals["bytes_per_launch"])
 
 
+def max_over_ranks(x, world, dist=None, device="cuda"):
+    """The maximum of x over all ranks: the slowest rank sets the timed region."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_rank_step, steps, ms):
+    """Whole-job tokens/s over `ms` milliseconds: every rank runs its own batch
+    (independent replicas, weak scaling)."""
+    return world * tokens_per_rank_step * steps / (ms / 1e3)
+
+
+def roofline_of(rows, pk, src, traffic_of=None):
+    """Roofline of the dominant kernel class from the profiler rows (one row per
+    class: launches, ms, flops, bytes).  The gemm_* classes are the roles
+    (forward, input grad, weight grad, LM head) of one tcgen05 GEMM kernel and
+    are aggregated; a class with FLOPs is tensor-bound against the sustained
+    bf16 peak, otherwise HBM-bound against the copy bandwidth."""
+    traffic_of = traffic_of or profile_traffic
+    by_kernel = {}
+    for r in rows:
+        k = "gemm_tcgen05" if r["kernel"].startswith("gemm_") and r["kernel"] != "gemm_fma" else r["kernel"]
+        a = by_kernel.setdefault(k, {"kernel": k, "launches": 0, "ms": 0.0, "flops": 0.0, "bytes": 0.0})
+        for f in ("launches", "ms", "flops", "bytes"):
+            a[f] += r[f]
+    dom = max(by_kernel.values(), key=lambda r: r["ms"])
+    if dom["flops"] > 0:
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        peak, unit, bound = pk["bf16_tflops_sustained"], "TFLOP/s", "tensor"
+    else:
+        achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+        peak, unit, bound = pk["hbm_gbs"], "GB/s", "hbm"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": traffic_of(dom["kernel"]), "kernel": dom["kernel"], "launches": dom["launches"],
+            "peak_source": f"{src} ({'sustained' if bound == 'tensor' else 'copy'})"}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
 
@@ -240,13 +281,6 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # ---------------- device-resident timing
     for _ in range(args.warmup):
         model.forward_backward(tok_d, tgt_d, W, grads, loss, ws, stream)
@@ -271,9 +305,9 @@ def main():
     code = model.check(stream)
     if code != 0:
         raise RuntimeError(f"device status {code}")
-    ms = max_over_ranks(ms)
+    ms = max_over_ranks(ms, world, dist)
     ms_step = ms / args.steps
-    value = world * M * args.steps / (ms / 1e3)
+    value = job_throughput(world, M, args.steps, ms)
     final_loss = float(loss.item())
 
     # ---------------- end to end through the host-buffer entry point
@@ -288,8 +322,8 @@ def main():
         model.forward_backward_host(h_tok, h_tgt, W, grads, ws, stream)
     f1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
-    e2e_value = world * M * args.steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dist)
+    e2e_value = job_throughput(world, M, args.steps, e2e_ms)
 
     if rank != 0:
         if world > 1:
@@ -297,26 +331,8 @@ def main():
         return
 
     # ---------------- roofline of the dominant kernel
-    # the gemm_* classes are the roles (forward, input grad, weight grad,
-    # LM head) of one tcgen05 GEMM kernel; aggregate them for the roofline
     pk, src = peaks()
-    by_kernel = {}
-    for r in rows:
-        k = "gemm_tcgen05" if r["kernel"].startswith("gemm_") and r["kernel"] != "gemm_fma" else r["kernel"]
-        a = by_kernel.setdefault(k, {"kernel": k, "launches": 0, "ms": 0.0, "flops": 0.0, "bytes": 0.0})
-        for f in ("launches", "ms", "flops", "bytes"):
-            a[f] += r[f]
-    dom = max(by_kernel.values(), key=lambda r: r["ms"])
-    if dom["flops"] > 0:
-        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
-        peak, unit, bound = pk["bf16_tflops_sustained"], "TFLOP/s", "tensor"
-    else:
-        achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
-        peak, unit, bound = pk["hbm_gbs"], "GB/s", "hbm"
-    traffic = profile_traffic(dom["kernel"])
-    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": traffic, "kernel": dom["kernel"], "launches": dom["launches"],
-                "peak_source": f"{src} ({'sustained' if bound == 'tensor' else 'copy'})"}
+    roofline = roofline_of(rows, pk, src)
 
     fpt = step_flops_per_token(cfg, T)
     tflops = value * fpt / 1e12
