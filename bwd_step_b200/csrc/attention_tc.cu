@@ -313,8 +313,8 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 // Both backward kernels keep every MMA at N = 128 (a 128 x 64 tile runs the
 // tensor core at well under half rate on sm_100a) and feed one operand of the
 // second product from TMEM: the softmax warps write their bf16 result back
-// over the fp32 score columns they have just read, and the MMA reads it there
-// as the A operand.  Sixteen softmax warps (four per TMEM lane quarter, 32
+// over fp32 columns they have just read (S in dQ, dP^T in dK/dV), and the MMA
+// reads it there as the A operand.  Sixteen softmax warps (four per TMEM lane quarter, 32
 // columns each) keep the special-function unit busy.
 //
 // dQ, one CTA per (query block of 128, head, batch row), key blocks j = 0..qb:
@@ -327,9 +327,8 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 //               core), then dQ += dS_{j-1} K_{j-1} with dS read from TMEM and
 //               K as an MN-major operand;
 //   warps 2-17  per key block: load the warp's S and dP columns, release dP,
-//               form
-//               P = 2^(S*scale*log2e - lse*log2e) with the causal mask on the
-//               diagonal block and dS = P (dP - D), and store dS as packed
+//               form P = 2^(S*scale*log2e - lse*log2e) with the causal mask on
+//               the diagonal block and dS = P (dP - D), and store dS as packed
 //               bf16 over the first half of the warp's own S columns.
 // dq = dQ / sqrt(hd).
 constexpr int NTB = 576;  // backward: producer, MMA, 16 softmax warps
