@@ -56,6 +56,9 @@ SIGNATURES = {
     "nc_profile_enable": (_I, [_P, _I]),
     "nc_profile_read": (_I, [_P, _P, ctypes.POINTER(NcProfileRow), _I]),
     "nc_launch_count": (ctypes.c_int64, []),
+    "nc_grad_bucket_count": (_I, [_P]),
+    "nc_grad_bucket": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]),
+    "nc_set_grad_events": (_I, [_P, ctypes.POINTER(ctypes.c_void_p), _I]),
     "nc_debug_expired_wait": (_I, [_P, _I, _P]),
     "nc_gemm_wgrad_noalloc": (_I, [_I, _I, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _I, _P, _P]),
     # include/nanochat_b200_testing.h

@@ -142,6 +142,26 @@ class Model:
         return [dict(kernel=r.kernel.decode(), launches=r.launches, ms=r.ms, flops=r.flops, bytes=r.bytes)
                 for r in rows[:n]]
 
+    def grad_buckets(self):
+        """[(offset, count)] of the flat gradient buffer in the order the backward
+        finishes them: LM head, layers last to first, token embedding."""
+        n = lib().nc_grad_bucket_count(self._h)
+        if n < 0:
+            raise NcError(n, "nc_grad_bucket_count")
+        out = []
+        for i in range(n):
+            off, cnt = ctypes.c_int64(), ctypes.c_int64()
+            _ok(lib().nc_grad_bucket(self._h, i, ctypes.byref(off), ctypes.byref(cnt)), "nc_grad_bucket")
+            out.append((off.value, cnt.value))
+        return out
+
+    def set_grad_events(self, events):
+        """Have every step record events[i] (torch.cuda.Event, already created by a
+        record) when gradient bucket i is final; an empty list clears them."""
+        handles = (ctypes.c_void_p * max(len(events), 1))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        _ok(lib().nc_set_grad_events(self._h, handles, len(events)), "nc_set_grad_events")
+        self._grad_events = list(events)  # the handles must outlive their use
+
     def debug_expired_wait(self, max_iters: int, stream=None):
         _ok(lib().nc_debug_expired_wait(self._h, max_iters, ctypes.c_void_p(_stream_handle(stream))),
             "nc_debug_expired_wait")

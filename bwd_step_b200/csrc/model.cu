@@ -30,6 +30,8 @@ struct nc_model {
     int V, d, L, H, nkv, hd, F, Nqkv;
     DType at;  // weight / activation type
     bool tc = false;  // tcgen05 path available (bf16 on sm_100)
+    // caller-owned events recorded when each gradient bucket is final (may be empty)
+    std::vector<cudaEvent_t> grad_events;
     // profiler: CUDA events around every launch while enabled
     struct Rec { int cls; cudaEvent_t a, b; double flops, bytes; long long launches; };
     bool prof_on = false;
@@ -332,6 +334,12 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
                           DT_F32), P_GEMM_LM_DW));
     }
     { Prof pr(c, P_OTHER, 0.0, 4.0 * M); CK(launch_loss_reduce(loss_rows, M, loss, s)); }
+    // bucket i of the gradients is final: record the caller's event, if any
+    auto bucket_done = [&](int i) -> int {
+        if (!m->grad_events.empty() && cudaEventRecord(m->grad_events[i], s) != cudaSuccess) return NC_ERR_CUDA;
+        return NC_OK;
+    };
+    RG(bucket_done(0));  // dWlm
 
     // ---- backward through the blocks
     float* dx = c.at<float>(c.p.dx);
@@ -374,6 +382,7 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
             CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_a, (float*)(lb + c.p.l_r1), dx, true,
                                   l > 0 ? dxb : nullptr, M, d, s));
         }
+        RG(bucket_done(m->L - l));  // this layer's six weight gradients
     }
     // ---- token embedding: norm backward, then the deterministic scatter-add
     {
@@ -382,6 +391,7 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         CK(launch_embed_norm_bwd(m->at, dx, tok, w.wte(), c.at<float>(c.p.r0), gbuf, M, V, d, s));
         CK(launch_embed_scatter(tok, gbuf, M, V, d, G(0), embed_scratch_carve(c.ws + c.p.emb, M, V, d), s));
     }
+    RG(bucket_done(m->L + 1));  // dWte
     return NC_OK;
 }
 
@@ -581,6 +591,42 @@ int64_t nc_launch_count(void) { return g_launches.load(); }
 int nc_debug_expired_wait(nc_model* m, int max_iters, void* stream) {
     if (!m || max_iters <= 0) return NC_ERR_INVALID_ARG;
     CK(launch_expired_wait(m->status, max_iters, (cudaStream_t)stream));
+    return NC_OK;
+}
+
+int nc_grad_bucket_count(const nc_model* m) { return m ? m->L + 2 : NC_ERR_INVALID_ARG; }
+
+int nc_grad_bucket(const nc_model* m, int i, int64_t* offset, int64_t* count) {
+    if (!m || !offset || !count || i < 0 || i > m->L + 1) return NC_ERR_INVALID_ARG;
+    auto size = [&](int idx) { return (int64_t)m->layout[idx].rows * m->layout[idx].cols; };
+    int first, last;  // layout entries of the bucket (adjacent in the flat layout)
+    if (i == 0) {
+        first = last = 1 + 6 * m->L;  // wlm
+    } else if (i == m->L + 1) {
+        first = last = 0;  // wte
+    } else {
+        const int l = m->L - i;  // layers in backward order
+        first = 1 + 6 * l;
+        last = first + 5;
+    }
+    *offset = m->layout[first].offset;
+    *count = m->layout[last].offset + size(last) - m->layout[first].offset;
+    return NC_OK;
+}
+
+int nc_set_grad_events(nc_model* m, void* const* events, int n) {
+    if (!m) return NC_ERR_INVALID_ARG;
+    if (n == 0) {
+        m->grad_events.clear();
+        return NC_OK;
+    }
+    if (!events || n != m->L + 2) return NC_ERR_INVALID_ARG;
+    std::vector<cudaEvent_t> ev((size_t)n);
+    for (int i = 0; i < n; ++i) {
+        if (!events[i]) return NC_ERR_INVALID_ARG;
+        ev[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    m->grad_events.swap(ev);
     return NC_OK;
 }
 

@@ -155,6 +155,28 @@ int nc_profile_read(nc_model* m, void* stream, nc_profile_row* rows, int max_row
 /* Kernels launched by the library in this process so far. */
 int64_t nc_launch_count(void);
 
+/* Gradient buckets for data-parallel averaging, in the order in which the
+ * backward of nc_forward_backward finishes them: bucket 0 is the LM head
+ * (wlm), bucket 1 + k the six matrices of layer n_layer - 1 - k (adjacent in
+ * the flat layout), bucket n_layer + 1 the token embedding (wte).
+ *   nc_grad_bucket_count: n_layer + 2, or NC_ERR_INVALID_ARG for a null handle.
+ *   nc_grad_bucket: element offset and element count of bucket i in the flat
+ *   gradient buffer; NC_ERR_INVALID_ARG for a null argument or i out of range.
+ * Host-only: neither call touches the device. */
+int nc_grad_bucket_count(const nc_model* m);
+int nc_grad_bucket(const nc_model* m, int i, int64_t* offset, int64_t* count);
+
+/* Optional per-bucket completion events, for overlapping a gradient exchange
+ * with the backward.  events: n cudaEvent_t handles passed as void*, created
+ * and owned by the caller, with n == nc_grad_bucket_count(m); n == 0 (events
+ * may be NULL) clears them.  While they are set, nc_forward_backward and
+ * nc_forward_backward_host record event i on the step's stream as soon as
+ * bucket i of the gradients is final, so another stream can wait on it and
+ * reduce that bucket while the backward continues.  The events must stay
+ * valid while set.  NC_ERR_INVALID_ARG for a null handle, a wrong n or a null
+ * event; nothing is recorded by this call itself. */
+int nc_set_grad_events(nc_model* m, void* const* events, int n);
+
 /* Weight-gradient GEMM that allocates no memory at all.
  *
  * No counterpart in the paper: this is an extra entry point of this library.
