@@ -232,7 +232,8 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const A* __rest
 }
 
 // ---------------------------------------------------------------- QK-norm + RoPE
-// One warp per (token, head) vector of HD elements.  Lane l holds EPL = HD/32
+// A warp handles a head vector of HD elements at a time (the forward one per
+// warp, the backward all heads of a position).  Lane l holds EPL = HD/32
 // consecutive elements (HD = 16: lanes 0..15 one each); the pair partner of
 // element j < HD/2 is element j + HD/2, held by lane l ^ (HD/2/EPL).  Every
 // access is a contiguous EPL-element vector, so a warp reads and writes each
