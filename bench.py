@@ -41,12 +41,13 @@ NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def step_flops_per_token(cfg, T):
-    """6 * matmul params (layer linears + LM head) + 6*L*H*hd*T causal attention."""
+def step_flops_per_token(cfg, T, causal=True):
+    """6 * matmul params (layer linears + LM head) + 6*L*H*hd*T causal attention;
+    with causal=False the PaLM convention 12*L*H*hd*T (no causal halving)."""
     d, hd, F = cfg.d_model, cfg.head_dim, cfg.mlp_mult * cfg.d_model
     per_layer = d * (cfg.n_head * hd + 2 * cfg.n_kv_head * hd) + cfg.n_head * hd * d + 2 * F * d
     n_mm = cfg.n_layer * per_layer + cfg.vocab * d
-    return 6.0 * n_mm + 6.0 * cfg.n_layer * cfg.n_head * hd * T
+    return 6.0 * n_mm + (6.0 if causal else 12.0) * cfg.n_layer * cfg.n_head * hd * T
 
 
 def workload_desc(wl):
@@ -363,6 +364,7 @@ def main():
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "no flush: per-step working set (weights, activations, grads) far exceeds the 126 MB L2"},
         "tflops": tflops, "mfu": tflops / NOMINAL_BF16_TFLOPS,
+        "tflops_palm_convention": value * step_flops_per_token(cfg, T, causal=False) / 1e12,
         "mfu_vs_measured": tflops / pk["bf16_tflops"], "gflop_per_token": fpt / 1e9,
         "loss": final_loss,
         "roofline": roofline,

@@ -1,7 +1,7 @@
 """Host-side logic of bench.py without a GPU: the max-over-ranks reduction of the
 timed region and the whole-job throughput on two gloo ranks (the N > 1 path),
-the roofline aggregation of the profiler rows, and the source-hash check of the
-committed DRAM-traffic summary."""
+the roofline aggregation of the profiler rows, the source-hash check of the
+committed DRAM-traffic summary, and the two FLOP-per-token conventions."""
 import hashlib
 import importlib.util
 import json
@@ -94,3 +94,14 @@ def test_traffic_is_reported_only_for_the_profiled_source(tmp_path):
     src.write_text("// kernel v2\n")
     assert bench.profile_traffic("demo") is None
     assert bench.profile_traffic("absent") is None
+
+
+def test_flops_per_token_conventions():
+    import synth
+    bench = _bench()
+    cfg = synth.WORKLOADS["d20"].model
+    causal = bench.step_flops_per_token(cfg, 2048)
+    palm = bench.step_flops_per_token(cfg, 2048, causal=False)
+    assert causal / 1e9 == pytest.approx(2.823, abs=1e-3)
+    # the PaLM convention counts the full T x T attention: 6 L H hd T more per token
+    assert palm - causal == pytest.approx(6.0 * 20 * 10 * 128 * 2048)
