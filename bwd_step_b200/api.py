@@ -32,11 +32,15 @@ def _stream_handle(stream):
     return getattr(stream, "cuda_stream", stream)
 
 
-def _ptr(t, dtype=None, name="tensor"):
+def _ptr(t, dtype=None, name="tensor", on_device=True):
+    """Pointer to a contiguous tensor of the given dtype, on the GPU (on_device)
+    or in host memory: a host pointer handed to a kernel would fault the GPU."""
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if bool(t.is_cuda) != on_device:
+        raise ValueError(f"{name} must be in {'device' if on_device else 'host'} memory")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -107,8 +111,8 @@ class Model:
         import torch
         B, T = h_tokens.shape
         out = ctypes.c_float()
-        _ok(lib().nc_forward_backward_host(self._h, _ptr(h_tokens, torch.int32, "tokens"),
-                                           _ptr(h_targets, torch.int32, "targets"), B, T,
+        _ok(lib().nc_forward_backward_host(self._h, _ptr(h_tokens, torch.int32, "tokens", on_device=False),
+                                           _ptr(h_targets, torch.int32, "targets", on_device=False), B, T,
                                            _ptr(weights, self.weight_dtype, "weights"),
                                            _ptr(grads, torch.float32, "grads"), ctypes.byref(out),
                                            _ptr(workspace, None, "workspace"),

@@ -75,3 +75,18 @@ def test_product_path_does_not_reference_the_oracle():
         if path.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
             src = open(path).read()
             assert not re.search(r"\boracle\b", src), path
+
+
+def test_marshalling_rejects_memory_on_the_wrong_side():
+    """A host pointer handed to a kernel would fault the GPU: the binding checks
+    where every tensor lives before passing its address."""
+    import torch
+    from bwd_step_b200.api import _ptr
+    t = torch.zeros(8, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        _ptr(t, torch.int32, "tokens")  # device memory expected
+    assert _ptr(t, torch.int32, "tokens", on_device=False).value == t.data_ptr()
+    with pytest.raises(TypeError):
+        _ptr(t, torch.float32, "grads", on_device=False)
+    with pytest.raises(ValueError):
+        _ptr(torch.zeros(4, 4, dtype=torch.int32).t(), torch.int32, "tokens", on_device=False)
