@@ -44,6 +44,19 @@ def _ptr(t, dtype=None, name="tensor", on_device=True):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _check_extents(n_params, vocab, tokens, targets=None, weights=None, grads=None, loss=None, logits=None):
+    """The C ABI takes bare pointers, so sizes are checked here: a buffer shorter
+    than the flat layout (or than [B, T, V] logits) would be written past its end."""
+    if tokens.dim() != 2:
+        raise ValueError("tokens must be [B, T]")
+    if targets is not None and tuple(targets.shape) != tuple(tokens.shape):
+        raise ValueError("targets must have the shape of tokens")
+    for name, t, need in (("weights", weights, n_params), ("grads", grads, n_params), ("loss", loss, 1),
+                          ("logits", logits, tokens.numel() * vocab)):
+        if t is not None and t.numel() < need:
+            raise ValueError(f"{name} holds {t.numel()} elements, needs {need}")
+
+
 def launch_count() -> int:
     """Kernels launched by the CUDA library in this process so far."""
     return int(lib().nc_launch_count())
@@ -98,6 +111,7 @@ class Model:
     def forward_backward(self, tokens, targets, weights, grads, loss, workspace, stream=None):
         """One step on device tensors; grads (fp32) and loss (fp32 [1]) are overwritten."""
         import torch
+        _check_extents(self.num_params(), self.cfg.vocab, tokens, targets, weights, grads, loss)
         B, T = tokens.shape
         _ok(lib().nc_forward_backward(self._h, _ptr(tokens, torch.int32, "tokens"),
                                       _ptr(targets, torch.int32, "targets"), B, T,
@@ -109,6 +123,7 @@ class Model:
     def forward_backward_host(self, h_tokens, h_targets, weights, grads, workspace, stream=None) -> float:
         """One step with host (ideally pinned) int32 token/target tensors; returns the loss."""
         import torch
+        _check_extents(self.num_params(), self.cfg.vocab, h_tokens, h_targets, weights, grads)
         B, T = h_tokens.shape
         out = ctypes.c_float()
         _ok(lib().nc_forward_backward_host(self._h, _ptr(h_tokens, torch.int32, "tokens", on_device=False),
@@ -121,7 +136,9 @@ class Model:
         return out.value
 
     def forward_logits(self, tokens, weights, logits, workspace, stream=None):
+        """Softcapped logits [B, T, V] of the forward pass (weight dtype)."""
         import torch
+        _check_extents(self.num_params(), self.cfg.vocab, tokens, weights=weights, logits=logits)
         B, T = tokens.shape
         _ok(lib().nc_forward_logits(self._h, _ptr(tokens, torch.int32, "tokens"), B, T,
                                     _ptr(weights, self.weight_dtype, "weights"),

@@ -90,3 +90,24 @@ def test_marshalling_rejects_memory_on_the_wrong_side():
         _ptr(t, torch.float32, "grads", on_device=False)
     with pytest.raises(ValueError):
         _ptr(torch.zeros(4, 4, dtype=torch.int32).t(), torch.int32, "tokens", on_device=False)
+
+
+def test_marshalling_checks_buffer_extents():
+    """Buffers shorter than the flat layout or the logits are refused before any
+    pointer reaches the library."""
+    import torch
+    from bwd_step_b200.api import _check_extents
+    tok = torch.zeros(2, 8, dtype=torch.int32)
+    w, g, l = torch.zeros(100), torch.zeros(100), torch.zeros(1)
+    _check_extents(100, 16, tok, tok.clone(), w, g, l)
+    for bad in (dict(targets=torch.zeros(2, 7, dtype=torch.int32)), dict(weights=torch.zeros(99)),
+                dict(grads=torch.zeros(99)), dict(loss=torch.zeros(0))):
+        args = dict(targets=tok.clone(), weights=w, grads=g, loss=l)
+        args.update(bad)
+        with pytest.raises(ValueError):
+            _check_extents(100, 16, tok, **args)
+    _check_extents(100, 16, tok, weights=w, logits=torch.zeros(2 * 8 * 16))
+    with pytest.raises(ValueError):
+        _check_extents(100, 16, tok, weights=w, logits=torch.zeros(2 * 8 * 16 - 1))
+    with pytest.raises(ValueError):
+        _check_extents(100, 16, torch.zeros(16, dtype=torch.int32), weights=w)
