@@ -184,6 +184,46 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
 
 
+def time_workload(wl, steps, warmup):
+    """Device-timed throughput of one workload at its full batch (inputs
+    resident, no profiler): tokens/s, TFLOP/s and MFU.  Frees its buffers."""
+    import torch
+    from bwd_step_b200 import Model
+    cfg = wl.model
+    B, T = wl.batch, wl.seq_len
+    bits, _ = synth.make_weights(cfg, seed=0, dtype="bf16")
+    tok, tgt = synth.make_tokens(wl, seed=1)
+    model = Model(cfg.as_dict(), "bf16")
+    W = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    del bits
+    grads = torch.empty(model.num_params(), dtype=torch.float32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(model.workspace_bytes(B, T), dtype=torch.uint8, device="cuda")
+    tok_d, tgt_d = torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        model.forward_backward(tok_d, tgt_d, W, grads, loss, ws, stream)
+    if model.check(stream) != 0:
+        raise RuntimeError(f"{wl.name}: device status")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        model.forward_backward(tok_d, tgt_d, W, grads, loss, ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    out = {"workload": wl.name, "tokens_per_step": B * T, "ms_per_step": ms,
+           "tokens_per_s": B * T / (ms / 1e3)}
+    out["tflops"] = out["tokens_per_s"] * step_flops_per_token(cfg, T) / 1e12
+    out["mfu"] = out["tflops"] / NOMINAL_BF16_TFLOPS
+    out["loss"] = float(loss.item())
+    model.close()
+    del W, grads, loss, ws, tok_d, tgt_d
+    torch.cuda.empty_cache()
+    return out
+
+
 def cpu_oracle_sample(wl, tokens_in_sample):
     """Times the float64 oracle on the first `tokens_in_sample` positions of
     row 0 (causal: identical to those positions of the full row)."""
@@ -244,6 +284,10 @@ def main():
     ap.add_argument("--reference-tokens", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--table", action="store_true", help="print the per-kernel table to stderr")
+    ap.add_argument("--profile-steps", type=int, default=5,
+                    help="steps of the separate per-kernel profiling pass")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the short per-workload throughput lines (all five workloads)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     wl = synth.WORKLOADS[args.workload]
@@ -282,7 +326,7 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    # ---------------- device-resident timing
+    # ---------------- device-resident timing (no per-launch events inside the timed region)
     for _ in range(args.warmup):
         model.forward_backward(tok_d, tgt_d, W, grads, loss, ws, stream)
     code = model.check(stream)
@@ -293,16 +337,13 @@ def main():
     with ClockSampler(torch.cuda.current_device()) as clk:
         barrier()
         l0 = launch_count()
-        model.profile(True)
         e0.record(stream)
         for _ in range(args.steps):
             model.forward_backward(tok_d, tgt_d, W, grads, loss, ws, stream)
         e1.record(stream)
         barrier()
         launches = launch_count() - l0
-        model.profile(False)
     ms = e0.elapsed_time(e1)
-    rows = model.profile_read(stream)
     code = model.check(stream)
     if code != 0:
         raise RuntimeError(f"device status {code}")
@@ -310,6 +351,16 @@ def main():
     ms_step = ms / args.steps
     value = job_throughput(world, M, args.steps, ms)
     final_loss = float(loss.item())
+
+    # ---------------- per-kernel table: a separate pass with an event pair
+    # around every launch (the library's profiler), same inputs and stream
+    prof_steps = max(1, min(args.steps, args.profile_steps))
+    model.profile(True)
+    for _ in range(prof_steps):
+        model.forward_backward(tok_d, tgt_d, W, grads, loss, ws, stream)
+    model.profile(False)
+    rows = model.profile_read(stream)
+    barrier()
 
     # ---------------- end to end through the host-buffer entry point
     h_tok = torch.from_numpy(tok).pin_memory()
@@ -331,6 +382,22 @@ def main():
             dist.destroy_process_group()
         return
 
+    # ---------------- every workload, briefly (one GPU only: keeps the run short)
+    configs = None
+    if world == 1 and not args.no_configs:
+        model.close()
+        del W, grads, loss, ws, tok_d, tgt_d
+        torch.cuda.empty_cache()
+        configs = []
+        for name in ("tiny", "gpt2_124m", "d20", "d30", "long"):
+            if name == args.workload:
+                configs.append({"workload": name, "tokens_per_step": M, "ms_per_step": ms_step,
+                                "tokens_per_s": value, "tflops": value * step_flops_per_token(cfg, T) / 1e12,
+                                "mfu": value * step_flops_per_token(cfg, T) / 1e12 / NOMINAL_BF16_TFLOPS,
+                                "loss": final_loss, "note": "the headline measurement above"})
+            else:
+                configs.append(time_workload(synth.WORKLOADS[name], steps=5, warmup=3))
+
     # ---------------- roofline of the dominant kernel
     pk, src = peaks()
     roofline = roofline_of(rows, pk, src)
@@ -348,7 +415,7 @@ def main():
 
     kernels = []
     for r in sorted(rows, key=lambda r: -r["ms"]):
-        k = {"kernel": r["kernel"], "launches": r["launches"], "ms_per_step": r["ms"] / args.steps,
+        k = {"kernel": r["kernel"], "launches": r["launches"], "ms_per_step": r["ms"] / prof_steps,
              "share": r["ms"] / sum(x["ms"] for x in rows)}
         if r["flops"] > 0:
             k["tflops"] = r["flops"] / (r["ms"] / 1e3) / 1e12
@@ -373,10 +440,12 @@ def main():
         "gpu_launches": int(launches),
         "clocks": clocks,
         "kernels": kernels,
+        "kernel_table_source": f"separate pass of {prof_steps} steps with an event pair around every launch",
+        "configs": configs,
     }
     if args.table:
         for k in kernels:
-            print(f"{k['kernel']:18s} {k['launches'] / args.steps:6.0f}/step {k['ms_per_step']:8.3f} ms "
+            print(f"{k['kernel']:18s} {k['launches'] / prof_steps:6.0f}/step {k['ms_per_step']:8.3f} ms "
                   f"{100 * k['share']:5.1f}%  " + (f"{k['tflops']:7.1f} TFLOP/s" if "tflops" in k else "") +
                   (f"{k['gbs']:8.0f} GB/s" if "gbs" in k else ""), file=sys.stderr)
     print(json.dumps(line), flush=True)

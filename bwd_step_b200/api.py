@@ -32,15 +32,19 @@ def _stream_handle(stream):
     return getattr(stream, "cuda_stream", stream)
 
 
-def _ptr(t, dtype=None, name="tensor", on_device=True):
+def _ptr(t, dtype=None, name="tensor", on_device=True, device=None):
     """Pointer to a contiguous tensor of the given dtype, on the GPU (on_device)
-    or in host memory: a host pointer handed to a kernel would fault the GPU."""
+    or in host memory: a host pointer handed to a kernel would fault the GPU.
+    With `device` (a CUDA ordinal) a device tensor must live on that GPU: a
+    buffer on another GPU would reach the kernels as peer memory."""
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if bool(t.is_cuda) != on_device:
         raise ValueError(f"{name} must be in {'device' if on_device else 'host'} memory")
+    if on_device and device is not None and t.device.index != device:
+        raise ValueError(f"{name} is on cuda:{t.device.index}, the model on cuda:{device}")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -74,6 +78,10 @@ class Model:
         _ok(lib().nc_model_create(ctypes.byref(self.cfg), PRECISIONS[precision], ctypes.byref(h)),
             "nc_model_create")
         self._h = h
+        import torch
+        # nc_model_create bound the model to the current device; every device
+        # tensor handed to it later must live there
+        self.device = torch.cuda.current_device()
 
     def close(self):
         if getattr(self, "_h", None):
@@ -108,16 +116,22 @@ class Model:
     def workspace_bytes(self, B: int, T: int) -> int:
         return int(lib().nc_workspace_bytes(self._h, B, T))
 
+    def _dev(self, t, dtype, name):
+        """Pointer to a device tensor on the model's GPU."""
+        return _ptr(t, dtype, name, device=self.device)
+
     def forward_backward(self, tokens, targets, weights, grads, loss, workspace, stream=None):
         """One step on device tensors; grads (fp32) and loss (fp32 [1]) are overwritten."""
         import torch
         _check_extents(self.num_params(), self.cfg.vocab, tokens, targets, weights, grads, loss)
         B, T = tokens.shape
-        _ok(lib().nc_forward_backward(self._h, _ptr(tokens, torch.int32, "tokens"),
-                                      _ptr(targets, torch.int32, "targets"), B, T,
-                                      _ptr(weights, self.weight_dtype, "weights"),
-                                      _ptr(grads, torch.float32, "grads"), _ptr(loss, torch.float32, "loss"),
-                                      _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+        _ok(lib().nc_forward_backward(self._h, self._dev(tokens, torch.int32, "tokens"),
+                                      self._dev(targets, torch.int32, "targets"), B, T,
+                                      self._dev(weights, self.weight_dtype, "weights"),
+                                      self._dev(grads, torch.float32, "grads"),
+                                      self._dev(loss, torch.float32, "loss"),
+                                      self._dev(workspace, None, "workspace"),
+                                      workspace.numel() * workspace.element_size(),
                                       ctypes.c_void_p(_stream_handle(stream))), "nc_forward_backward")
 
     def forward_backward_host(self, h_tokens, h_targets, weights, grads, workspace, stream=None) -> float:
@@ -128,9 +142,9 @@ class Model:
         out = ctypes.c_float()
         _ok(lib().nc_forward_backward_host(self._h, _ptr(h_tokens, torch.int32, "tokens", on_device=False),
                                            _ptr(h_targets, torch.int32, "targets", on_device=False), B, T,
-                                           _ptr(weights, self.weight_dtype, "weights"),
-                                           _ptr(grads, torch.float32, "grads"), ctypes.byref(out),
-                                           _ptr(workspace, None, "workspace"),
+                                           self._dev(weights, self.weight_dtype, "weights"),
+                                           self._dev(grads, torch.float32, "grads"), ctypes.byref(out),
+                                           self._dev(workspace, None, "workspace"),
                                            workspace.numel() * workspace.element_size(),
                                            ctypes.c_void_p(_stream_handle(stream))), "nc_forward_backward_host")
         return out.value
@@ -140,9 +154,10 @@ class Model:
         import torch
         _check_extents(self.num_params(), self.cfg.vocab, tokens, weights=weights, logits=logits)
         B, T = tokens.shape
-        _ok(lib().nc_forward_logits(self._h, _ptr(tokens, torch.int32, "tokens"), B, T,
-                                    _ptr(weights, self.weight_dtype, "weights"),
-                                    _ptr(logits, self.weight_dtype, "logits"), _ptr(workspace, None, "workspace"),
+        _ok(lib().nc_forward_logits(self._h, self._dev(tokens, torch.int32, "tokens"), B, T,
+                                    self._dev(weights, self.weight_dtype, "weights"),
+                                    self._dev(logits, self.weight_dtype, "logits"),
+                                    self._dev(workspace, None, "workspace"),
                                     workspace.numel() * workspace.element_size(),
                                     ctypes.c_void_p(_stream_handle(stream))), "nc_forward_logits")
 

@@ -958,13 +958,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 template <int HD>
 int fwd_launch(const CUtensorMap& map, const AttnParams& p, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(attn_fwd_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 FwdLayout<HD>::BYTES) != cudaSuccess)
-            return -1;
-        attr = true;
-    }
+    if (ensure_smem_limit((const void*)attn_fwd_tc_kernel<HD>, FwdLayout<HD>::BYTES) != cudaSuccess) return -1;
     dim3 grid(p.H, p.B, p.nqb);
     attn_fwd_tc_kernel<HD><<<grid, NT, FwdLayout<HD>::BYTES, s>>>(map, p);
     count_launch();
@@ -973,13 +967,7 @@ int fwd_launch(const CUtensorMap& map, const AttnParams& p, cudaStream_t s) {
 
 template <int HD>
 int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(attn_dq_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 DqLayout<HD>::BYTES) != cudaSuccess)
-            return -1;
-        attr = true;
-    }
+    if (ensure_smem_limit((const void*)attn_dq_tc_kernel<HD>, DqLayout<HD>::BYTES) != cudaSuccess) return -1;
     attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NTB, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
@@ -987,13 +975,7 @@ int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& 
 
 template <int HD>
 int dkv_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(attn_dkv_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 DkvLayout<HD>::BYTES) != cudaSuccess)
-            return -1;
-        attr = true;
-    }
+    if (ensure_smem_limit((const void*)attn_dkv_tc_kernel<HD>, DkvLayout<HD>::BYTES) != cudaSuccess) return -1;
     attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NTB, DkvLayout<HD>::BYTES, s>>>(kv, do128, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;

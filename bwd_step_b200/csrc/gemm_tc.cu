@@ -638,16 +638,7 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer
     return r == CUDA_SUCCESS;
 }
 
-int num_sms() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
+int num_sms() { return device_sm_count(); }
 
 }  // namespace
 
@@ -662,20 +653,9 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 1;
     auto al16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
     if (!al16(g.A) || !al16(g.B) || (g.lda * 2) % 16 || (g.ldb * 2) % 16) return 1;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) !=
-            cudaSuccess)
-            return -1;
-        attr_set = true;
-    }
-    static bool attr2_set = false;
-    if (!attr2_set) {
-        if (cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_BYTES) !=
-            cudaSuccess)
-            return -1;
-        attr2_set = true;
-    }
+    if (ensure_smem_limit((const void*)gemm_tc_kernel, (int)SMEM_BYTES) != cudaSuccess ||
+        ensure_smem_limit((const void*)gemm_tc2_kernel, (int)SMEM2_BYTES) != cudaSuccess)
+        return -1;
 
     // CTA pairs (256x256 tiles) when there are at least 256 rows
     const bool pair = g.M >= 256;
@@ -711,8 +691,9 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     const int sms = pair ? num_sms() / 2 : num_sms();
     const int tiles = p.tiles_m * p.tiles_n;
     int splits = 1;
+    // the split-K reduction reads and writes C as float4: C must be 16-byte aligned
     const bool can_split = (g.epi == EPI_STORE || g.epi == EPI_ACCUM) && !p.c_bf16 && g.ldc == g.N && splitk &&
-                           g.N % 4 == 0;
+                           g.N % 4 == 0 && al16(g.C);
     if (can_split && tiles < 2 * sms) {
         double best = (double)((tiles + sms - 1) / sms);
         for (int sp = 2; sp <= MAX_SPLITS; ++sp) {

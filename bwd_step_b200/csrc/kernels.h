@@ -125,6 +125,14 @@ cudaError_t launch_attention_bwd_simt(DType at, const void* qkv, const void* o, 
 cudaError_t launch_attention_bwd_dot(DType at, const void* o, const void* dO, float* D, int B, int T, int H, int hd,
                                      cudaStream_t s);
 
+// ---------------------------------------------------------------- launch helpers
+// Raises the dynamic shared-memory limit of kernel `func` to `bytes` on the
+// current device, once per (kernel, device): the attribute is per device.
+// Thread-safe.
+cudaError_t ensure_smem_limit(const void* func, int bytes);
+// Streaming multiprocessors of the current device.
+int device_sm_count();
+
 // ---------------------------------------------------------------- bounded wait
 cudaError_t launch_expired_wait(int* status, int max_iters, cudaStream_t s);
 

@@ -395,8 +395,16 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     return NC_OK;
 }
 
+// The model's device must be current: its buffers are that device's memory,
+// and kernels launched on another device would reach them as peer memory.
+bool on_model_device(const nc_model* m) {
+    int dev = -1;
+    return cudaGetDevice(&dev) == cudaSuccess && dev == m->device;
+}
+
 int validate_call(nc_model* m, int B, int T, size_t ws_bytes, const void* const* ptrs, int nptr) {
     if (!m || B <= 0 || T <= 0) return NC_ERR_INVALID_ARG;
+    if (!on_model_device(m)) return NC_ERR_INVALID_ARG;
     if ((long long)B * T > (1 << 24)) return NC_ERR_UNSUPPORTED_SHAPE;
     for (int i = 0; i < nptr; ++i)
         if (!ptrs[i]) return NC_ERR_INVALID_ARG;
@@ -589,7 +597,7 @@ int nc_profile_read(nc_model* m, void* stream, nc_profile_row* rows, int max_row
 int64_t nc_launch_count(void) { return g_launches.load(); }
 
 int nc_debug_expired_wait(nc_model* m, int max_iters, void* stream) {
-    if (!m || max_iters <= 0) return NC_ERR_INVALID_ARG;
+    if (!m || max_iters <= 0 || !on_model_device(m)) return NC_ERR_INVALID_ARG;
     CK(launch_expired_wait(m->status, max_iters, (cudaStream_t)stream));
     return NC_OK;
 }

@@ -41,6 +41,10 @@ extern "C" int nc_gemm_wgrad_noalloc(int rows, int n_out, int n_in, const void* 
                                      int64_t ld_x, float* dw, int accumulate, int* status, void* stream) {
     if (rows <= 0 || n_out <= 0 || n_in <= 0 || !dy || !x || !dw) return NC_ERR_INVALID_ARG;
     if (ld_dy < n_out || ld_x < n_in) return NC_ERR_INVALID_ARG;
+    // TMA reads dy and x in 16-byte units and the split-K reduction writes dw as
+    // float4: every base address and row pitch must be 16-byte aligned
+    auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+    if (!al16(dy) || !al16(x) || !al16(dw) || ld_dy % 8 || ld_x % 8) return NC_ERR_INVALID_ARG;
     // the array must hold at least two K-split partials of the [n_out, n_in] result
     if ((size_t)n_out * (size_t)n_in * sizeof(float) * 2 > kWgradScratchBytes) return NC_ERR_UNSUPPORTED_SHAPE;
     void* scratch = nullptr;

@@ -39,7 +39,8 @@ extern "C" {
 
 /* Return codes. */
 #define NC_OK                       0
-#define NC_ERR_INVALID_ARG         -1  /* null pointer, non-positive size, bad index      */
+#define NC_ERR_INVALID_ARG         -1  /* null pointer, non-positive size, bad index,
+                                          misaligned buffer, or not the model's device */
 #define NC_ERR_UNSUPPORTED_SHAPE   -2  /* config outside what the kernels implement      */
 #define NC_ERR_WORKSPACE_TOO_SMALL -3  /* ws_bytes < nc_workspace_bytes(model, B, T)      */
 #define NC_ERR_CUDA                -4  /* a CUDA runtime call or kernel launch failed    */
@@ -74,7 +75,11 @@ typedef struct nc_model nc_model; /* opaque */
 
 /* Validates cfg and creates a model bound to the current CUDA device.  Host
  * state plus one small device status word (allocated here, freed by
- * nc_model_destroy).  *out is set to NULL on error. */
+ * nc_model_destroy).  *out is set to NULL on error.  That device must be the
+ * current one whenever a step, logits or debug call is made on the model:
+ * those calls return NC_ERR_INVALID_ARG, launching nothing, when another
+ * device is current (its kernels would otherwise reach the buffers as peer
+ * memory). */
 int nc_model_create(const nc_config* cfg, nc_precision prec, nc_model** out);
 void nc_model_destroy(nc_model* m);
 
@@ -193,7 +198,9 @@ int nc_set_grad_events(nc_model* m, void* const* events, int n);
  *   dw: device fp32 [n_out, n_in], contiguous; overwritten, or added to when
  *       accumulate != 0
  *   status: device int status word for the bounded waits (may be NULL)
- * Rows must be 16-byte aligned (ld_dy, ld_x multiples of 8).
+ * dy, x and dw must start on a 16-byte boundary and ld_dy, ld_x must be
+ * multiples of 8 (16-byte rows); otherwise the call returns
+ * NC_ERR_INVALID_ARG before anything is launched.
  *
  * Split-K partial sums live in one file-scope static device array of
  * NC_WGRAD_NOALLOC_SCRATCH_BYTES; every GPU that loads the library holds it

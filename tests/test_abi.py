@@ -92,6 +92,30 @@ def test_marshalling_rejects_memory_on_the_wrong_side():
         _ptr(torch.zeros(4, 4, dtype=torch.int32).t(), torch.int32, "tokens", on_device=False)
 
 
+def test_marshalling_rejects_a_tensor_on_another_gpu():
+    """A buffer on another GPU would reach the model's kernels as peer memory:
+    the binding compares every device tensor's ordinal with the model's."""
+    import torch
+    from bwd_step_b200.api import _ptr
+
+    class OnGpu:  # stands in for a CUDA tensor (no GPU is needed for the check)
+        dtype = torch.float32
+        is_cuda = True
+
+        def __init__(self, index):
+            self.device = torch.device("cuda", index)
+
+        def is_contiguous(self):
+            return True
+
+        def data_ptr(self):
+            return 4096
+
+    assert _ptr(OnGpu(0), torch.float32, "grads", device=0).value == 4096
+    with pytest.raises(ValueError, match="cuda:1"):
+        _ptr(OnGpu(1), torch.float32, "grads", device=0)
+
+
 def test_marshalling_checks_buffer_extents():
     """Buffers shorter than the flat layout or the logits are refused before any
     pointer reaches the library."""

@@ -20,14 +20,18 @@ def _operand(R, K, kmajor, gen, scale=1.0):
     return x.double(), stored.cuda(), (K if kmajor else R)
 
 
-def _run(M, N, K, ak, bk, epi, c_bf16, use_tc=1, seed=0, scale=1.0, scratch_mb=0):
+def _run(M, N, K, ak, bk, epi, c_bf16, use_tc=1, seed=0, scale=1.0, scratch_mb=0, c_offset=0):
     gen = torch.Generator().manual_seed(seed)
     A64, A, lda = _operand(M, K, ak, gen, scale)
     B64, B, ldb = _operand(N, K, bk, gen, scale)
     acc = A64 @ B64.t()
     cdt = torch.bfloat16 if c_bf16 else torch.float32
     C0 = torch.randn(M, N, generator=gen)
-    C = C0.to(cdt).cuda()
+    # c_offset > 0 places C that many elements into a larger buffer (a view
+    # whose base is not 16-byte aligned)
+    Cbuf = torch.zeros(M * N + c_offset, dtype=cdt, device="cuda")
+    C = Cbuf[c_offset:].view(M, N)
+    C.copy_(C0.to(cdt))
     C2 = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
     aux = torch.rand(M, N, generator=gen).to(torch.bfloat16)
     auxd = aux.cuda()
@@ -88,6 +92,14 @@ def test_split_k_ragged_rows(M, N):
     # spill into the next split's partial sums
     _run(M, N, 4096, False, False, 0, False, scratch_mb=128, seed=M)
     _run(M, N, 4096, False, False, 1, False, scratch_mb=128, seed=M + 1)
+
+
+@pytest.mark.parametrize("epi", [0, 1])
+def test_split_k_candidate_with_unaligned_output(epi):
+    # a shape that takes split-K, with C one float past a 16-byte boundary: the
+    # vectorised split-K reduction must not be used (it would be a misaligned
+    # access); the GEMM still runs, on the single-pass epilogue
+    _run(256, 256, 8192, False, False, epi, False, scratch_mb=64, seed=11 + epi, c_offset=1)
 
 
 def test_fma_gemm_matches_too():

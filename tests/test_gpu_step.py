@@ -69,46 +69,55 @@ def test_gpt2_124m_shape_one_row(precision):
     _parity(wl.model, 1, wl.seq_len, precision, ids="zipf")
 
 
-def _replicated_full_size(name, min_layer=0):
-    """Full launch configuration (every row of the batch equal to row 0) vs
-    the oracle on that one row: duplicating rows leaves the mean loss and
-    the gradients unchanged."""
+def _full_launch(name, patterns, min_layer=0):
+    """The bench's launch configuration (full B and T) with `patterns` distinct
+    seeded rows repeated in turn over the batch (row b holds pattern
+    b % patterns), against the oracle on the distinct rows: repeating rows
+    leaves the mean loss and the gradients unchanged (a pinned property), so
+    a kernel that mixes batch rows or takes an offset from the wrong row
+    fails here while the host cost stays that of `patterns` rows.  With
+    min_layer > 0 only the LM head and the layers >= min_layer are compared."""
     wl = synth.WORKLOADS[name]
     cfg = wl.model
+    assert wl.batch % patterns == 0
     bits, w = synth.make_weights(cfg, seed=0, dtype="bf16")
-    tok1, tgt1 = synth.make_tokens(wl, seed=1, batch=1)
-    ref_loss, ref_g = oracle.step(cfg, w, tok1, tgt1, min_layer=min_layer)
-    tok = np.repeat(tok1, wl.batch, axis=0)
-    tgt = np.repeat(tgt1, wl.batch, axis=0)
+    tok_p, tgt_p = synth.make_tokens(wl, seed=1, batch=patterns)
+    assert patterns == 1 or not np.array_equal(tok_p[0], tok_p[1])
+    ref_loss, ref_g = oracle.step(cfg, w, tok_p, tgt_p, min_layer=min_layer)
+    tok = np.tile(tok_p, (wl.batch // patterns, 1))
+    tgt = np.tile(tgt_p, (wl.batch // patterns, 1))
     m = Model(cfg.as_dict(), "bf16")
     loss, g = gpu_step(m, to_device_weights(bits, w, "bf16"), tok, tgt)
-    if min_layer > 0:
-        keep = np.zeros(g.shape, dtype=bool)
-        for n, r, c, off in synth.param_layout(cfg):
-            if n == "wlm" or (n.startswith("h.") and int(n.split(".")[1]) >= min_layer):
-                keep[off:off + r * c] = True
-        g = np.where(keep, g, 0.0)
-        lay = [x for x in synth.param_layout(cfg) if x[0] == "wlm" or
-               (x[0].startswith("h.") and int(x[0].split(".")[1]) >= min_layer)]
-        tl, tg = TOL["bf16"]
-        assert abs(loss - ref_loss) <= tl
-        for n, r, c, off in lay:
-            rel = np.linalg.norm(g[off:off + r * c] - ref_g[off:off + r * c]) / np.linalg.norm(ref_g[off:off + r * c])
-            assert rel <= tg, (n, rel)
-        return
-    compare(cfg, loss, g, ref_loss, ref_g, "bf16")
+    if min_layer == 0:
+        return compare(cfg, loss, g, ref_loss, ref_g, "bf16")
+    lay = [x for x in synth.param_layout(cfg) if x[0] == "wlm" or
+           (x[0].startswith("h.") and int(x[0].split(".")[1]) >= min_layer)]
+    tl, tg = TOL["bf16"]
+    assert abs(loss - ref_loss) <= tl
+    for n, r, c, off in lay:
+        rel = np.linalg.norm(g[off:off + r * c] - ref_g[off:off + r * c]) / np.linalg.norm(ref_g[off:off + r * c])
+        assert rel <= tg, (n, rel)
+
+
+def test_gpt2_124m_full_launch_configuration_distinct_rows():
+    _full_launch("gpt2_124m", patterns=8)
 
 
 def test_d20_full_launch_configuration():
-    _replicated_full_size("d20")
+    _full_launch("d20", patterns=2)
 
 
-def test_d30_full_launch_configuration_last_layers():
-    _replicated_full_size("d30", min_layer=28)
+def test_d30_full_launch_configuration_every_layer():
+    _full_launch("d30", patterns=2)
 
 
-def test_long_context_full_launch_configuration_last_layers():
-    _replicated_full_size("long", min_layer=19)
+def test_long_context_full_launch_configuration_every_layer():
+    _full_launch("long", patterns=1)
+
+
+def test_fp32_debug_full_d20_row():
+    wl = synth.WORKLOADS["d20"]
+    _parity(wl.model, 1, wl.seq_len, "fp32", ids="zipf")
 
 
 def test_forward_logits_match_oracle():

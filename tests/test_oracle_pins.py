@@ -381,3 +381,40 @@ def test_truncated_backward_matches_full_on_the_layers_it_keeps():
             np.testing.assert_array_equal(G1[name], G[name])
         else:
             assert np.all(G1[name] == 0)
+
+
+# ---------------------------------------------------------------- forward logits
+def test_forward_logits_match_library_forward():
+    """oracle.forward_logits equals the softcapped LM-head output of the
+    independent torch float64 forward (library rms_norm, complex RoPE, SDPA):
+    a swapped weight, a dropped softcap or a missing final norm fails here."""
+    cfg, w, tok, tgt = _tiny_inputs(seed_w=71)
+    w = w * 10.0
+    oracle.views(cfg, w)["wlm"][:] *= 5.0  # drive the logits into the curved range of the tanh
+    z = oracle.forward_logits(cfg, w, tok)
+    xf = _torch_forward(cfg, torch.from_numpy(w), tok, tgt, return_xf=True).numpy()
+    wlm = oracle.views(cfg, w)["wlm"]
+    expect = cfg.softcap * np.tanh((xf @ wlm.T) / cfg.softcap)
+    assert z.shape == (tok.shape[0], tok.shape[1], cfg.vocab)
+    np.testing.assert_allclose(z, expect, rtol=1e-12, atol=1e-12)
+    assert np.max(np.abs(z)) > 0.5 * cfg.softcap  # the cap is exercised
+
+
+def test_forward_logits_log_softmax_gives_position_losses():
+    """-log softmax(z)[target] of the returned logits is the per-position loss
+    (whose LM head is the separately pinned lm_head_loss)."""
+    cfg, w, tok, tgt = _tiny_inputs(seed_w=72)
+    w = w * 5.0
+    z = oracle.forward_logits(cfg, w, tok)
+    zmax = z.max(axis=-1, keepdims=True)
+    lse = zmax[..., 0] + np.log(np.exp(z - zmax).sum(axis=-1))
+    ce = lse - np.take_along_axis(z, tgt[..., None], axis=-1)[..., 0]
+    np.testing.assert_allclose(ce, oracle.position_losses(cfg, w, tok, tgt), rtol=1e-12, atol=1e-13)
+
+
+def test_forward_logits_zero_lm_head_are_zero():
+    """Wlm = 0 gives z = c tanh(0) = 0 exactly at every position."""
+    cfg, w, tok, _ = _tiny_inputs(seed_w=73)
+    oracle.views(cfg, w)["wlm"][:] = 0.0
+    z = oracle.forward_logits(cfg, w, tok)
+    assert np.all(z == 0.0)

@@ -58,3 +58,21 @@ def test_rejects_results_larger_than_the_static_array():
     r = lib().nc_gemm_wgrad_noalloc(64, n, n, P(dy.data_ptr()), n, P(dy.data_ptr()), n, P(dw.data_ptr()), 0,
                                     P(status.data_ptr()), _stream())
     assert r == _lib.NC_ERR_UNSUPPORTED_SHAPE
+
+
+def test_rejects_misaligned_buffers_before_launching():
+    """dw one float past a 16-byte boundary (a torch view at an odd offset) is
+    refused with NC_ERR_INVALID_ARG; nothing runs, so its contents stay."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rows, n = 4096, 256
+    dy = torch.ones(rows, n, dtype=torch.bfloat16, device="cuda")
+    buf = torch.full((n * n + 1,), 7.0, dtype=torch.float32, device="cuda")
+    dw = buf[1:]
+    r = lib().nc_gemm_wgrad_noalloc(rows, n, n, P(dy.data_ptr()), n, P(dy.data_ptr()), n, P(dw.data_ptr()), 0,
+                                    P(status.data_ptr()), _stream())
+    assert r == _lib.NC_ERR_INVALID_ARG
+    r = lib().nc_gemm_wgrad_noalloc(rows, n, n, P(dy.data_ptr() + 2), n, P(dy.data_ptr()), n,
+                                    P(buf.data_ptr()), 0, P(status.data_ptr()), _stream())
+    assert r == _lib.NC_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.all(buf == 7.0) and status.item() == 0
