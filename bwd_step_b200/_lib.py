@@ -21,6 +21,9 @@ NC_ERR_BAD_TOKEN = -5
 NC_ERR_DEVICE_TIMEOUT = -6
 NC_ERR_NO_DEVICE = -7
 
+NC_LM_HEAD_FUSED = 0
+NC_LM_HEAD_MATERIALISED = 1
+
 NC_PREC_BF16 = 0
 NC_PREC_FP32_DEBUG = 1
 
@@ -60,12 +63,14 @@ SIGNATURES = {
     "nc_grad_bucket": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]),
     "nc_set_grad_events": (_I, [_P, ctypes.POINTER(ctypes.c_void_p), _I]),
     "nc_debug_expired_wait": (_I, [_P, _I, _P]),
+    "nc_set_lm_head": (_I, [_P, _I, _I]),
     "nc_gemm_wgrad_noalloc": (_I, [_I, _I, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _I, _P, _P]),
     # include/nanochat_b200_testing.h
     "nc_test_gemm": (_I, [_I, _I, _I, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _P,
                           ctypes.c_int64, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_float, _I, _P,
                           _SZ, _P, _P]),
-    "nc_test_attention": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P]),
+    "nc_test_attention_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "nc_test_attention": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _I, _P, _P]),
 }
 
 _lib = None

@@ -161,6 +161,13 @@ class Model:
                                     workspace.numel() * workspace.element_size(),
                                     ctypes.c_void_p(_stream_handle(stream))), "nc_forward_logits")
 
+    def set_lm_head(self, mode: str = "fused", chunk_rows: int = 0):
+        """LM head strategy: "fused" (logits never stored; bf16 only) or
+        "materialised" (logit chunks plus a cross-entropy pass); chunk_rows 0 =
+        default.  Query workspace_bytes afterwards: it depends on both."""
+        code = {"fused": _lib.NC_LM_HEAD_FUSED, "materialised": _lib.NC_LM_HEAD_MATERIALISED}[mode]
+        _ok(lib().nc_set_lm_head(self._h, code, int(chunk_rows)), "nc_set_lm_head")
+
     def check(self, stream=None) -> int:
         """Synchronise the stream and return (and clear) the device status code."""
         return int(lib().nc_check(self._h, ctypes.c_void_p(_stream_handle(stream))))

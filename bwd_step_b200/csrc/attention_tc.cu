@@ -4,38 +4,46 @@
 // announcement, vpshk.cn, architecture list), causal within a row, scores
 // scaled by 1/sqrt(hd).
 //
-// Forward, one CTA per (query block of 128 positions, head, batch row):
-//   warp 0     TMA: the Q tile once, then K_j and V_j together in a 3-stage
-//              ring for key blocks j = 0..qb (causal: blocks past the
+// Forward, persistent: one CTA per SM walks the units (query block of 128
+// positions, pair of query heads of one K/V group, batch row), longest first.
+// Both heads of a pair read the same K_j / V_j tiles from shared memory (the
+// K/V head is shared), and their work is interleaved so that one head's
+// softmax runs while the tensor core computes the other head's products:
+//   warp 0     TMA: Q of both heads per unit, then K_j and V_j together into
+//              a ring for key blocks j = 0..qb (causal: blocks past the
 //              diagonal are never loaded);
-//   warp 1     tcgen05.mma: S_j = Q K_j^T into one of two 128-column TMEM
-//              buffers, two blocks ahead; O += P_j V_j with P_j read from
-//              TMEM (A operand) and V_j as an MN-major operand;
-//   warps 2-9  softmax, two warps per TMEM lane quarter (one query row per
-//              thread, 64 keys each): scores from TMEM, causal mask on the
-//              diagonal block, running row max in the log2 domain shared by
-//              the two warps of a row through shared memory, lazy rescaling
-//              of O (only when the max grows by more than 2^8), and P stored
-//              as packed bf16 over the first half of the warp's own score
-//              columns.
-// The K/V head is shared by all query heads; its tiles are re-read by the
-// H CTAs of a query block from L2.
+//   warp 1     tcgen05.mma in the order ... O_a += P_a(j) V_j, S_a(j+1),
+//              O_b += P_b(j) V_j, S_b(j+1) ...: S = Q K^T into the head's
+//              128 TMEM score columns, O += P V with P read from TMEM (A
+//              operand) over the first half of those columns and V as an
+//              MN-major operand;
+//   warps 2-5  softmax of head a, warps 6-9 of head b: one query row per
+//              thread, all 128 keys of the block from TMEM, causal mask on
+//              the diagonal block, running max in the log2 domain, lazy
+//              rescaling of O (only when the max grows by more than 2^8),
+//              P stored as packed bf16; then the normalised output and the
+//              log-sum-exp of the unit.
+// 2^x is taken from the special-function unit (ex2) for three of every four
+// scores and from a cubic on the FMA pipe for the fourth, so that the two
+// units share the work of the exponentials.
 #include "attention_tc.h"
 #include "tc_common.cuh"
 #include <cudaTypedefs.h>
+#include <algorithm>
+#include <type_traits>
 
 namespace nc {
 namespace {
 using namespace tc;
 
-constexpr int NT = 320;  // forward: producer, MMA, 8 softmax warps (two per TMEM lane quarter)
-constexpr int FSTG = 3;  // K/V ring stages
+constexpr int NT = 320;  // forward: producer, MMA, 2 x 4 softmax warps
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
 struct AttnParams {
     int B, T, H, nkv, nqb;
-    float scale_log2;  // log2(e) / sqrt(hd)
+    int pairs_per_group, npair, num_units;  // head pairs within each K/V group; units = B * npair * nqb
+    float scale_log2;                       // log2(e) / sqrt(hd)
     bf16* o;
     float* lse;
     int* status;
@@ -45,11 +53,11 @@ template <int HD>
 struct FwdLayout {
     static constexpr int KB = HD / 64;       // 64-column blocks of the head dim
     static constexpr int TILE = KB * 16384;  // [128 x HD] bf16, 128B-swizzled
-    static constexpr int Q = 0;
-    static constexpr int K = Q + TILE;
-    static constexpr int V = K + FSTG * TILE;
-    static constexpr int MX = V + FSTG * TILE;  // [2][2][128] fp32 partial row maxima (then row sums)
-    static constexpr int BAR = MX + 2048;
+    static constexpr int KVSTG = HD == 128 ? 2 : 3;
+    static constexpr int QA = 0;             // Q of head a, then Q of head b
+    static constexpr int K = 2 * TILE;
+    static constexpr int V = K + KVSTG * TILE;
+    static constexpr int BAR = V + KVSTG * TILE;
     static constexpr int BYTES = BAR + 256;  // the dynamic shared memory base is 1024-aligned (checked)
     static_assert(BYTES <= 232448, "attention forward shared memory exceeds the per-block limit");
 };
@@ -59,13 +67,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// the two softmax warps of TMEM lane quarter q (64 threads)
-__device__ __forceinline__ void pair_sync(int q) {
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
-}
-
-// Store 32 consecutive 32-bit columns of this thread's TMEM lane, then wait.
-__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
+// Store 32 consecutive 32-bit columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_st32u_nowait(uint32_t taddr, const uint32_t* v) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -75,43 +78,77 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t* v) {
         "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
         "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Waits (at most 1 ms) for a barrier phase: used on the abort path to let
+// copies in flight land before the block exits.
+__device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
+    uint64_t t0 = globaltimer();
+    while (!mbar_try(bar, parity) && globaltimer() - t0 < 1000000ull) {}
+}
+
+// 2^x on the FMA pipe, for x >= -126 (smaller x give a value below 2^-125):
+// x = n + f with n = round(x) and |f| <= 1/2; 2^f by a cubic fitted here to
+// 2^f on [-1/2, 1/2] with the Remez exchange on the relative error (maximum
+// relative error 7.5e-5, below the bf16 rounding of P); n is added to the
+// exponent field.  The rounding uses the 1.5 * 2^23 shift, after which the
+// low mantissa bits of t hold n in two's complement.
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fmaxf(x, -126.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    float p = fmaf(0.0551716685f, f, 0.2426111251f);
+    p = fmaf(p, f, 0.6932609677f);
+    p = fmaf(p, f, 0.9999280572f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Unit u -> batch row, query block (longest first), first head of the pair and
+// whether the pair has a second head (a K/V group of odd size ends with a
+// single head).
+__device__ __forceinline__ void fwd_unit(const AttnParams& p, int u, int& b, int& qb, int& h0, bool& two) {
+    const int per = p.B * p.npair;
+    qb = p.nqb - 1 - u / per;
+    const int rem = u % per;
+    b = rem / p.npair;
+    const int pi = rem % p.npair;
+    const int Hg = p.H / p.nkv;
+    const int g = pi / p.pairs_per_group, k = pi % p.pairs_per_group;
+    h0 = g * Hg + 2 * k;
+    two = 2 * k + 1 < Hg;
 }
 
 template <int HD>
 __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnParams p) {
     using Lay = FwdLayout<HD>;
-    constexpr int KB = Lay::KB;
-    constexpr int TILE = Lay::TILE;
+    constexpr int KB = Lay::KB, TILE = Lay::TILE, KVSTG = Lay::KVSTG;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     if ((smem_u32(smem_dyn) & 1023u) != 0) {
         if (threadIdx.x == 0) set_status(p.status, ST_BAD_LAYOUT);
         return;
     }
-    uint8_t* smem = smem_dyn;
-    const uint32_t base = smem_u32(smem);
-    const uint32_t sQ = base + Lay::Q, sK = base + Lay::K, sV = base + Lay::V;
-    float* mxs = reinterpret_cast<float*>(smem + Lay::MX);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
+    const uint32_t base = smem_u32(smem_dyn);
+    const uint32_t sQ = base + Lay::QA, sK = base + Lay::K, sV = base + Lay::V;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_dyn + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
-    const uint32_t q_full = b0;
-    const uint32_t kv_full = b0 + 8, kv_empty = b0 + 32;  // [FSTG]: K_j and V_j share a stage
-    const uint32_t s_full = b0 + 56, p_full = b0 + 72;    // [2]: per TMEM score buffer
-    const uint32_t o_last = b0 + 88;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+    const uint32_t q_full = b0, q_empty = b0 + 8;
+    const uint32_t kv_full = b0 + 16, kv_empty = kv_full + 8 * KVSTG;  // [KVSTG]: K_j and V_j share a stage
+    const uint32_t s_full = kv_empty + 8 * KVSTG;                       // [2] per head of the pair
+    const uint32_t p_full = s_full + 16;                                // [2]
+    const uint32_t o_full = p_full + 16;                                // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * KVSTG);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb = p.nqb - 1 - (int)blockIdx.z;  // grid z slowest: the longest blocks launch first
-    const int h = blockIdx.x, b = blockIdx.y, g = h / (p.H / p.nkv);
-    const int nblk = qb + 1;
-    const int row0 = b * p.T;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < FSTG; ++s) { mbar_init(kv_full + 8 * s, 1); mbar_init(kv_empty + 8 * s, 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(s_full + 8 * s, 1); mbar_init(p_full + 8 * s, 8); }
-        mbar_init(o_last, 1);
+        mbar_init(q_empty, 1);
+        for (int st = 0; st < KVSTG; ++st) { mbar_init(kv_full + 8 * st, 1); mbar_init(kv_empty + 8 * st, 1); }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(s_full + 8 * x, 1);
+            mbar_init(p_full + 8 * x, 4);
+            mbar_init(o_full + 8 * x, 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -121,183 +158,227 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 256;  // S[2] of 128 columns, O (HD columns)
+    // TMEM: scores (then P) of heads a and b in columns [0,128) and [128,256),
+    // their outputs O in [256, 256 + HD) and [256 + HD, 256 + 2 HD)
 
     if (warp == 0) {
-        // one thread loads Q, then K_j and V_j together into a 3-stage ring (a stage
-        // frees after O += P_j V_j): one wait per key block for the MMA thread
         if (lane == 0) {
-            const int xq = h * HD, xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
-            mbar_expect_tx(q_full, TILE);
+            int k = 0, kvi = 0, inflight_q = 0;
+            uint32_t q_par = 0;
+            uint32_t kv_issued = 0, kv_phase_bits = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++k) {
+                int b, qb, h0;
+                bool two;
+                fwd_unit(p, u, b, qb, h0, two);
+                const int g = h0 / (p.H / p.nkv);
+                const int xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
+                const int row0 = b * p.T;
+                if (!mbar_wait(q_empty, (k & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+                mbar_expect_tx(q_full, two ? 2 * TILE : TILE);
 #pragma unroll
-            for (int kb = 0; kb < KB; ++kb) tma_load_2d(sQ + kb * 16384, &tm, xq + kb * 64, row0 + qb * 128, q_full);
-            int issued = 0;
-            for (int j = 0; j < nblk; ++j) {
-                const int st = j % FSTG;
-                if (!mbar_wait(kv_empty + 8 * st, ((j / FSTG) & 1) ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(kv_full + 8 * st, 2 * TILE);
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_2d(sK + st * TILE + kb * 16384, &tm, xk + kb * 64, row0 + j * 128, kv_full + 8 * st);
-                    tma_load_2d(sV + st * TILE + kb * 16384, &tm, xv + kb * 64, row0 + j * 128, kv_full + 8 * st);
+                for (int c = 0; c < KB; ++c) {
+                    tma_load_2d(sQ + c * 16384, &tm, h0 * HD + 64 * c, row0 + qb * 128, q_full);
+                    if (two) tma_load_2d(sQ + TILE + c * 16384, &tm, (h0 + 1) * HD + 64 * c, row0 + qb * 128, q_full);
                 }
-                issued = j + 1;
+                inflight_q = 1;
+                q_par = k & 1;
+                for (int j = 0; j <= qb; ++j, ++kvi) {
+                    const int st = kvi % KVSTG;
+                    const uint32_t ph = (kvi / KVSTG) & 1;
+                    if (!mbar_wait(kv_empty + 8 * st, ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+                    mbar_expect_tx(kv_full + 8 * st, 2 * TILE);
+#pragma unroll
+                    for (int c = 0; c < KB; ++c) {
+                        tma_load_2d(sK + st * TILE + c * 16384, &tm, xk + 64 * c, row0 + j * 128, kv_full + 8 * st);
+                        tma_load_2d(sV + st * TILE + c * 16384, &tm, xv + 64 * c, row0 + j * 128, kv_full + 8 * st);
+                    }
+                    kv_issued |= 1u << st;
+                    kv_phase_bits = (kv_phase_bits & ~(1u << st)) | (ph << st);
+                }
             }
-            if (*abort_flag) {
-                // let copies in flight land before the block exits
-                uint64_t t0 = globaltimer();
-                while (!mbar_try(q_full, 0) && globaltimer() - t0 < 1000000ull) {}
-                for (int j = (issued > FSTG ? issued - FSTG : 0); j < issued; ++j) {
-                    t0 = globaltimer();
-                    while (!mbar_try(kv_full + 8 * (j % FSTG), (j / FSTG) & 1) && globaltimer() - t0 < 1000000ull) {}
-                }
+            if (!ok) {
+                // let the copies in flight land before the block exits
+                if (inflight_q) drain(q_full, q_par);
+                for (int st = 0; st < KVSTG; ++st)
+                    if (kv_issued >> st & 1) drain(kv_full + 8 * st, (kv_phase_bits >> st) & 1);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);
             const uint32_t id_o = idesc_bf16(128, HD, false, true);
-            // S_j = Q K_j^T into buffer j & 1
-            auto scores = [&](int j) -> bool {
-                const int st = j % FSTG, sb = j & 1;
-                if (!mbar_wait(kv_full + 8 * st, (j / FSTG) & 1, abort_flag, p.status)) return false;
-                tc_fence_after();
+            int k = 0, kvi = 0;
+            uint32_t pcnt0 = 0, pcnt1 = 0;  // P hand-overs waited for, per head
+            bool ok = true;
+            // S_x = Q_x K^T for head x of the pair, from the K/V stage st
+            auto scores = [&](int x, int st) {
 #pragma unroll
                 for (int ks = 0; ks < HD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    mma_bf16(tS + sb * 128, smem_desc(sQ + off, 16, 1024), smem_desc(sK + st * TILE + off, 16, 1024),
-                             id_s, ks > 0 ? 1u : 0u);
+                    mma_bf16(tmem + 128 * x, smem_desc(sQ + x * TILE + off, 16, 1024),
+                             smem_desc(sK + st * TILE + off, 16, 1024), id_s, ks > 0 ? 1u : 0u);
                 }
-                mma_commit(s_full + 8 * sb);
-                return true;
+                mma_commit(s_full + 8 * x);
             };
-            bool ok = mbar_wait(q_full, 0, abort_flag, p.status) && scores(0) && (nblk < 2 || scores(1));
-            for (int j = 0; ok && j < nblk; ++j) {
-                const int st = j % FSTG, sb = j & 1;
-                // O += P_j V_j: keys 16kk..16kk+15 sit in the packed columns
-                // 64*(kk/4) + 8*(kk%4) of score buffer j & 1 (written by column group kk/4)
-                // (V_j landed with K_j, waited for before S_j)
-                if (!mbar_wait(p_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status)) break;
+            // O_x += P_x V: keys 16kk..16kk+15 sit in the packed columns 8kk..8kk+7
+            auto pv = [&](int x, int st, bool acc) -> bool {
+                if (!mbar_wait(p_full + 8 * x, (x ? pcnt1 : pcnt0) & 1, abort_flag, p.status)) return false;
+                if (x) ++pcnt1;
+                else ++pcnt0;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tO, tS + sb * 128 + 64 * (kk >> 2) + 8 * (kk & 3),
-                                smem_desc(sV + st * TILE + kk * 2048, 16384, 1024), id_o, (j > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(kv_empty + 8 * st);
-                // S_{j+2} overwrites P_j only after these MMAs (issue order)
-                if (j + 2 < nblk && !scores(j + 2)) break;
+                    mma_bf16_ts(tmem + 256 + x * HD, tmem + 128 * x + 8 * kk,
+                                smem_desc(sV + st * TILE + kk * 2048, 16384, 1024), id_o, (acc || kk > 0) ? 1u : 0u);
+                return true;
+            };
+            auto kv_ready = [&](int i) -> bool {
+                return mbar_wait(kv_full + 8 * (i % KVSTG), (i / KVSTG) & 1, abort_flag, p.status);
+            };
+            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++k) {
+                int b, qb, h0;
+                bool two;
+                fwd_unit(p, u, b, qb, h0, two);
+                const int nblk = qb + 1;
+                if (!mbar_wait(q_full, k & 1, abort_flag, p.status) || !kv_ready(kvi)) { ok = false; break; }
+                tc_fence_after();
+                scores(0, kvi % KVSTG);
+                if (two) scores(1, kvi % KVSTG);
+                if (nblk == 1) mma_commit(q_empty);  // the unit's last products that read Q
+                for (int j = 0; j < nblk; ++j) {
+                    const int st = (kvi + j) % KVSTG, st1 = (kvi + j + 1) % KVSTG;
+                    const bool more = j + 1 < nblk;
+                    if (!pv(0, st, j > 0)) { ok = false; break; }
+                    if (more) {
+                        if (!kv_ready(kvi + j + 1)) { ok = false; break; }
+                        tc_fence_after();
+                        scores(0, st1);
+                    } else {
+                        mma_commit(o_full);
+                    }
+                    if (two && !pv(1, st, j > 0)) { ok = false; break; }
+                    mma_commit(kv_empty + 8 * st);  // K_j, V_j read by every product of this block
+                    if (two) {
+                        if (more) scores(1, st1);
+                        else mma_commit(o_full + 8);
+                    }
+                    if (j + 2 == nblk) mma_commit(q_empty);
+                }
+                kvi += nblk;
             }
-            mma_commit(o_last);
         }
     } else {
-        // ---------------- softmax warps: warp w reads TMEM lanes 32*(w%4).., keys 64*cg..
-        const int q = warp & 3, cg = (warp - 2) >> 2;
-        const int r = q * 32 + lane;  // row of the tile
-        const int qpos = qb * 128 + r;
+        // ---------------- softmax: head x of the pair, TMEM lane quarter q, one query row per thread
+        const int x = (warp - 2) >> 2, q = warp & 3;
+        const int r = q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        float m = -INFINITY, l = 0.f;
-        // After a failed (timed-out or aborted) wait a warp skips its TMEM and
-        // barrier work but still meets its partner at every pair_sync, so the
-        // pair never waits on a warp that has left the loop.
-        bool ok = true;
-        for (int j = 0; j < nblk; ++j) {
-            const int sb = j & 1;
-            ok = ok && warp_wait(s_full + 8 * sb, (j >> 1) & 1, abort_flag, p.status);
-            float s[64];
-            float mx = -INFINITY;
-            if (ok) {
+        const uint32_t tS = tmem + lane_off + 128 * x, tO = tmem + lane_off + 256 + x * HD;
+        uint32_t scnt = 0, ocnt = 0;
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+            int b, qb, h0;
+            bool two;
+            fwd_unit(p, u, b, qb, h0, two);
+            if (x == 1 && !two) continue;
+            const int h = h0 + x;
+            float m = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j <= qb; ++j) {
+                if (!warp_wait(s_full + 8 * x, scnt & 1, abort_flag, p.status)) { ok = false; break; }
+                ++scnt;
                 tc_fence_after();
-                {
-                    uint32_t rr[64];
-                    tmem_ld32_issue(tS + lane_off + sb * 128 + cg * 64, rr);
-                    tmem_ld32_issue(tS + lane_off + sb * 128 + cg * 64 + 32, rr + 32);
+                const bool diag = j == qb;  // key c of the diagonal block is visible from row r iff c <= r
+                // pass 1: the row maximum (scores read from TMEM 64 columns at a time)
+                float mx = -INFINITY;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t s[64];
+                    tmem_ld32_issue(tS + 64 * hf, s);
+                    tmem_ld32_issue(tS + 64 * hf + 32, s + 32);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(rr[i]);
+                    for (int c = 0; c < 64; ++c)
+                        mx = fmaxf(mx, (diag && 64 * hf + c > r) ? -INFINITY : __uint_as_float(s[c]));
                 }
-                if (j == qb) {
-                    const int lim = r - cg * 64;  // keys cg*64 + c with c <= lim are visible
+                mx *= p.scale_log2;
+                const bool rescale = mx > m + 8.f;
+                const float mu = rescale ? mx : m;
+                const float alpha = rescale ? ex2(m - mx) : 1.f;
+                float sum = 0.f;
+                // pass 2: P = 2^(s*scale - mu) as packed bf16 over the first 64 score
+                // columns (the scores of each half are read before they are overwritten);
+                // with kPoly one score in four comes from the FMA pipe (full blocks only:
+                // exp2_fma does not take the masked -inf scores of the diagonal block)
+                auto exp_pack = [&](auto poly) {
+                    constexpr bool kPoly = decltype(poly)::value;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        s[c] = (c <= lim) ? s[c] * p.scale_log2 : -INFINITY;
-                        mx = fmaxf(mx, s[c]);
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint32_t s[64];
+                        tmem_ld32_issue(tS + 64 * hf, s);
+                        tmem_ld32_issue(tS + 64 * hf + 32, s + 32);
+                        tmem_wait_ld();
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int c = 0; c < 64; c += 2) {
+                            float x0 = fmaf(__uint_as_float(s[c]), p.scale_log2, -mu);
+                            float x1 = fmaf(__uint_as_float(s[c + 1]), p.scale_log2, -mu);
+                            if (!kPoly && diag) {
+                                if (64 * hf + c > r) x0 = -INFINITY;
+                                if (64 * hf + c + 1 > r) x1 = -INFINITY;
+                            }
+                            const float e0 = ex2(x0);
+                            const float e1 = (kPoly && (c & 2)) ? exp2_fma(x1) : ex2(x1);
+                            sum += e0 + e1;
+                            pk[c >> 1] = pack_bf16(e0, e1);
+                        }
+                        tmem_st32u_nowait(tS + 32 * hf, pk);
                     }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        s[c] *= p.scale_log2;
-                        mx = fmaxf(mx, s[c]);
-                    }
-                }
-            }
-            // the row max over both halves of the block
-            mxs[(sb * 2 + cg) * 128 + r] = mx;
-            pair_sync(q);
-            if (!ok) continue;
-            mx = fmaxf(mx, mxs[(sb * 2 + (cg ^ 1)) * 128 + r]);
-            const bool rescale = mx > m + 8.f;
-            const float mu = rescale ? mx : m;
-            const float alpha = rescale ? ex2(m - mx) : 1.f;
-            float sum = 0.f;
-            uint32_t pk[32];
-#pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-                const float e0 = ex2(s[c] - mu), e1 = ex2(s[c + 1] - mu);
-                sum += e0 + e1;
-                pk[c >> 1] = pack_bf16(e0, e1);
-            }
-            if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-                // O += P_{j-1} V_{j-1} has finished (its K/V stage was released); O(j) cannot
-                // have started, so this phase of the barrier is the latest one
-                const int jj = j - 1;
-                ok = warp_wait(kv_empty + 8 * (jj % FSTG), (jj / FSTG) & 1, abort_flag, p.status);
-                if (!ok) continue;
-                tc_fence_after();
-                // this warp rescales its half of the O columns
+                };
+                if (!diag) exp_pack(std::true_type{});
+                else exp_pack(std::false_type{});
+                tmem_wait_st();
+                if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                    // O_x += P(j-1) V has completed (S(j) was issued after it and has landed);
+                    // O_x += P(j) V waits for this warp's hand-over below
 #pragma unroll 1
-                for (int c = 0; c < HD / 32; ++c) {
-                    float o[16];
-                    tmem_ld16(tO + lane_off + cg * (HD / 2) + c * 16, o);
-                    uint32_t u[16];
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32_issue(tO + c * 32, o);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(o[i] * alpha);
-                    tmem_st16(tO + lane_off + cg * (HD / 2) + c * 16, u);
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32u_nowait(tO + c * 32, o);
+                        tmem_wait_st();
+                    }
                 }
+                l = l * alpha + sum;
+                m = mu;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full + 8 * x);
             }
-            l = l * alpha + sum;
-            m = mu;
-            tmem_st32u(tS + lane_off + sb * 128 + cg * 64, pk);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(p_full + 8 * sb);
-        }
-        ok = ok && warp_wait(o_last, 0, abort_flag, p.status);
-        // row sums of both halves (buffer 0 of the maxima is free: the partner read
-        // this warp's last maximum before its P was handed over, which O needed)
-        mxs[cg * 128 + r] = l;
-        pair_sync(q);
-        if (ok) {
+            if (!ok || !warp_wait(o_full + 8 * x, ocnt & 1, abort_flag, p.status)) break;
+            ++ocnt;
             tc_fence_after();
-            const float lt = l + mxs[(cg ^ 1) * 128 + r];
-            const float inv = 1.f / lt;
+            const int qpos = qb * 128 + r;
             const bool live = qpos < p.T;
-            bf16* orow = p.o + ((size_t)row0 + qpos) * (size_t)(p.H * HD) + h * HD + cg * (HD / 2);
-#pragma unroll
-            for (int c = 0; c < HD / 64; ++c) {
+            const float inv = 1.f / l;
+            bf16* orow = p.o + ((size_t)b * p.T + (live ? qpos : 0)) * (size_t)(p.H * HD) + (size_t)h * HD;
+#pragma unroll 1
+            for (int c = 0; c < HD / 32; ++c) {
                 float o[32];
-                tmem_ld32(tO + lane_off + cg * (HD / 2) + c * 32, o);
+                tmem_ld32(tO + c * 32, o);
                 if (live) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint4 u = make_uint4(pack_bf16(o[8 * i] * inv, o[8 * i + 1] * inv),
-                                             pack_bf16(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
-                                             pack_bf16(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
-                                             pack_bf16(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
-                        *reinterpret_cast<uint4*>(orow + c * 32 + 8 * i) = u;
-                    }
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4*>(orow + c * 32 + 8 * i) =
+                            make_uint4(pack_bf16(o[8 * i] * inv, o[8 * i + 1] * inv),
+                                       pack_bf16(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                       pack_bf16(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                       pack_bf16(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
                 }
             }
-            if (live && cg == 0) p.lse[((size_t)b * p.H + h) * attn_tpad(p.T) + qpos] = (m + __log2f(lt)) * kLn2;
+            if (live) p.lse[((size_t)b * p.H + h) * attn_tpad(p.T) + qpos] = (m + __log2f(l)) * kLn2;
         }
     }
     tc_fence_before();
@@ -308,59 +389,43 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
     }
 }
 
-
 // ============================================================================ backward
-// Both backward kernels keep every MMA at N = 128 (a 128 x 64 tile runs the
-// tensor core at well under half rate on sm_100a) and feed one operand of the
-// second product from TMEM: the softmax warps write their bf16 result back
-// over fp32 columns they have just read (S in dQ, dP^T in dK/dV), and the MMA
-// reads it there as the A operand.  Sixteen softmax warps (four per TMEM lane quarter, 32
-// columns each) keep the special-function unit busy.
+// Three launches: (1) D = rowsum(dO * o) and lse * log2(e) per (row, head);
+// (2) the dK/dV kernel, which recomputes S^T and dP^T per (key block, query
+// block, query head), forms P^T and dS^T, accumulates dV and dK, and stores
+// every dS^T tile; (3) dq = dS K / sqrt(hd) as a plain tensor-core product
+// over the stored tiles.  S and dP are formed once (in (2)), so the backward
+// issues the minimal five 128-wide products per tile pair (S^T, dP^T, dV,
+// dK, dQ), deterministically: every sum runs in a fixed order, no atomics.
 //
-// dQ, one CTA per (query block of 128, head, batch row), key blocks j = 0..qb:
-//   warp 0      TMA: Q and dO once; K_j into a 3-stage ring (freed by the dQ
-//               MMA), V_j into a 2-stage ring (freed by the dP MMA), both on
-//               one barrier per key block;
-//   warp 1      tcgen05.mma: S_j = Q K_j^T into one of two TMEM buffers and
-//               dP_j = dO V_j^T into one buffer as one group of 16 MMAs
-//               (every wait or commit between 128-wide MMAs idles the tensor
-//               core), then dQ += dS_{j-1} K_{j-1} with dS read from TMEM and
-//               K as an MN-major operand;
-//   warps 2-17  per key block: load the warp's S and dP columns, release dP,
-//               form P = 2^(S*scale*log2e - lse*log2e) with the causal mask on
-//               the diagonal block and dS = P (dP - D), and store dS as packed
-//               bf16 over the first half of the warp's own S columns.
-// dq = dQ / sqrt(hd).
-constexpr int NTB = 576;  // backward: producer, MMA, 16 softmax warps
+// The dK/dV kernel keeps every MMA at N = 128 (a 128 x 64 tile runs the
+// tensor core at well under half rate on sm_100a) and feeds one operand of the
+// second product from TMEM: the softmax warps write P^T as bf16 back over
+// dP^T columns they have just read, and the dV MMA reads it there as the A
+// operand.  Sixteen softmax warps (four per TMEM lane quarter, 32 columns
+// each) keep the special-function unit busy.
+constexpr int NTB = 576;  // dK/dV: producer, MMA, 16 softmax warps
 constexpr int NSM = 16;   // softmax warps
 
-template <int HD>
-struct DqLayout {
-    static constexpr int KB = HD / 64;
-    static constexpr int TILE = KB * 16384;  // [128 x HD] bf16, 128B-swizzled: Q, dO, a K or V block
-    static constexpr int KSTG = 3, VSTG = 2;
-    static constexpr int Q = 0;
-    static constexpr int DO = Q + TILE;
-    static constexpr int K = DO + TILE;
-    static constexpr int V = K + KSTG * TILE;
-    static constexpr int BAR = V + VSTG * TILE;
-    static constexpr int BYTES = BAR + 256;  // the dynamic shared memory base is 1024-aligned (checked)
-    static_assert(BYTES <= 232448, "dQ shared memory exceeds the per-block limit");
-};
-
 struct BwdParams {
-    int B, T, H, nkv, nqb;
+    int B, T, H, nkv, nqb, ntri;
     float scale_log2, scale;
     const float* D;     // [B, H, Tp] rowsum(dO * o)
     const float* lse2;  // [B, H, Tp] lse * log2(e) (both zero past the sequence end)
     bf16* dqkv;
+    bf16* ds;           // dS^T tiles (see ds_tile), written by the dK/dV kernel
     int* status;
 };
 
-__device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
-    uint64_t t0 = globaltimer();
-    while (!mbar_try(bar, parity) && globaltimer() - t0 < 1000000ull) {}
+// The dK/dV kernel stores every causal 128 x 128 tile of dS = P (dP - D) it
+// forms, transposed ([128 keys][128 queries] bf16, row-major), for the dQ
+// product.  Tiles of one (batch row, query head) are packed by query block,
+// then key block: tile (qb, kb), kb <= qb, is number qb (qb + 1) / 2 + kb of
+// its head, so the key blocks of one query block are adjacent.
+__host__ __device__ inline size_t ds_tile(int b, int h, int H, int ntri, int qb, int kb) {
+    return ((size_t)b * H + h) * (size_t)ntri + (size_t)qb * (qb + 1) / 2 + kb;
 }
+
 
 // sum of the products of two vectors of eight bf16
 __device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
@@ -405,209 +470,174 @@ __global__ void __launch_bounds__(256) attn_bwd_stats_kernel(const bf16* __restr
     }
 }
 
+// dq = dS K / sqrt(hd) from the stored dS^T tiles.  Persistent: one CTA per
+// SM walks the units (query block, head, batch row), longest first.
+//   warp 0      TMA: per key block kb <= qb, the dS^T tile (two boxes of
+//               [128 keys][64 queries]) and the K_kb tile into a ring;
+//   warp 1      tcgen05.mma: D[q, c] += sum_k dS^T[k, q] K[k, c] with both
+//               operands MN-major in shared memory, into one of two TMEM
+//               accumulators, so the epilogue of one unit overlaps the next;
+//   warps 2-5   epilogue: one query row per thread, scaled, bf16, into the
+//               q columns of dqkv.
 template <int HD>
-__global__ void __launch_bounds__(NTB, 1) attn_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
-                                                           const __grid_constant__ CUtensorMap tmDO,
-                                                           const BwdParams p) {
-    using Lay = DqLayout<HD>;
-    constexpr int KB = Lay::KB, TILE = Lay::TILE, KSTG = Lay::KSTG, VSTG = Lay::VSTG;
+struct DqdsLayout {
+    static constexpr int KB = HD / 64;
+    static constexpr int A_BYTES = 32768;       // dS^T tile, bf16, two 64-query boxes
+    static constexpr int B_BYTES = KB * 16384;  // K tile [128 keys x HD] bf16
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES = HD == 128 ? 3 : 4;
+    static constexpr int BAR = STAGES * STAGE;
+    static constexpr int BYTES = BAR + 256;  // the dynamic shared memory base is 1024-aligned (checked)
+    static_assert(BYTES <= 232448, "dQ shared memory exceeds the per-block limit");
+};
+constexpr int NTQ = 192;  // dQ product: producer, MMA, four epilogue warps
+
+struct DqdsParams {
+    int B, T, H, nkv, nqb, ntri, num_units;
+    float scale;
+    bf16* dqkv;
+    int* status;
+};
+
+__device__ __forceinline__ void dq_unit(const DqdsParams& p, int u, int& b, int& h, int& qb) {
+    const int bh = u % (p.B * p.H);
+    qb = p.nqb - 1 - u / (p.B * p.H);  // the longest units first
+    b = bh / p.H;
+    h = bh % p.H;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(NTQ, 1) attn_dq_ds_kernel(const __grid_constant__ CUtensorMap tmDS,
+                                                           const __grid_constant__ CUtensorMap tmQKV,
+                                                           const DqdsParams p) {
+    using Lay = DqdsLayout<HD>;
+    constexpr int KB = Lay::KB, STAGES = Lay::STAGES;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
     if ((smem_u32(smem_dyn) & 1023u) != 0) {
         if (threadIdx.x == 0) set_status(p.status, ST_BAD_LAYOUT);
         return;
     }
-    uint8_t* smem = smem_dyn;
-    const uint32_t base = smem_u32(smem);
-    const uint32_t sQ = base + Lay::Q, sDO = base + Lay::DO, sK = base + Lay::K, sV = base + Lay::V;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
+    const uint32_t base = smem_u32(smem_dyn);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_dyn + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
-    const uint32_t qd_full = b0;
-    const uint32_t k_empty = b0 + 32;                    // [KSTG]
-    const uint32_t v_full = b0 + 56, v_empty = b0 + 72;  // [VSTG]: v_full covers K_j and V_j
-    const uint32_t dp_full = b0 + 104, dp_free = b0 + 112;
-    const uint32_t ds_full = b0 + 120;                   // [2]: dS_j written over buffer j & 1
-    const uint32_t dq_done = b0 + 136;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+    const uint32_t full = b0, empty = b0 + 8 * STAGES;              // [STAGES]
+    const uint32_t acc_full = b0 + 16 * STAGES, acc_empty = acc_full + 16;  // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qb = p.nqb - 1 - (int)blockIdx.z;  // longest blocks launch first
-    const int h = blockIdx.x, b = blockIdx.y, g = h / (p.H / p.nkv);
-    const int nblk = qb + 1;
-    const int row0 = b * p.T;
-    const int Nqkv = (p.H + 2 * p.nkv) * HD;
+    constexpr uint32_t kCols = 2 * HD;  // two accumulators (128 or 256 columns)
 
     if (threadIdx.x == 0) {
-        mbar_init(qd_full, 1);
-        for (int s = 0; s < KSTG; ++s) mbar_init(k_empty + 8 * s, 1);
-        for (int s = 0; s < VSTG; ++s) { mbar_init(v_full + 8 * s, 1); mbar_init(v_empty + 8 * s, 1); }
-        for (int s = 0; s < 2; ++s) mbar_init(ds_full + 8 * s, NSM);
-        mbar_init(dp_full, 1);
-        mbar_init(dp_free, NSM);
-        mbar_init(dq_done, 1);
+        for (int st = 0; st < STAGES; ++st) { mbar_init(full + 8 * st, 1); mbar_init(empty + 8 * st, 1); }
+        for (int a = 0; a < 2; ++a) { mbar_init(acc_full + 8 * a, 1); mbar_init(acc_empty + 8 * a, 4); }
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), 512);
-    if (warp == 0 && lane == 0) { tma_prefetch(&tmQKV); tma_prefetch(&tmDO); }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), kCols);
+    if (warp == 0 && lane == 0) { tma_prefetch(&tmDS); tma_prefetch(&tmQKV); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tdP = tmem + 256, tdQ = tmem + 384;  // S[2] of 128 columns, dP, dQ
 
     if (warp == 0) {
-        // one thread loads Q and dO, then per key block K_j into the 3-stage K ring
-        // (a slot frees after the dQ MMA) and V_j into the 2-stage V ring (after
-        // the dP MMA); both land on the V stage's barrier, so the MMA thread waits
-        // once per key block
         if (lane == 0) {
-            const int xk = (p.H + g) * HD, xv = (p.H + p.nkv + g) * HD;
-            mbar_expect_tx(qd_full, 2 * TILE);
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, issued_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+                int b, h, qb;
+                dq_unit(p, u, b, h, qb);
+                const int g = h / (p.H / p.nkv);
+                const int xk = (p.H + g) * HD;
+                const int trow = (int)(ds_tile(b, h, p.H, p.ntri, qb, 0) * 128);
+                for (int kb = 0; kb <= qb; ++kb) {
+                    if (!mbar_wait(empty + 8 * stage, phase ^ 1, abort_flag, p.status)) { ok = false; break; }
+                    const uint32_t fb = full + 8 * stage;
+                    const uint32_t sa = base + stage * Lay::STAGE, sb = sa + Lay::A_BYTES;
+                    mbar_expect_tx(fb, Lay::STAGE);
+                    tma_load_2d(sa, &tmDS, 0, trow + kb * 128, fb);
+                    tma_load_2d(sa + 16384, &tmDS, 64, trow + kb * 128, fb);
 #pragma unroll
-            for (int kb = 0; kb < KB; ++kb) {
-                tma_load_2d(sQ + kb * 16384, &tmQKV, h * HD + kb * 64, row0 + qb * 128, qd_full);
-                tma_load_2d(sDO + kb * 16384, &tmDO, h * HD + kb * 64, row0 + qb * 128, qd_full);
-            }
-            int issued = 0;
-            for (int j = 0; j < nblk; ++j) {
-                const int kst = j % KSTG, vst = j % VSTG;
-                if (!mbar_wait(k_empty + 8 * kst, ((j / KSTG) & 1) ^ 1, abort_flag, p.status)) break;
-                if (!mbar_wait(v_empty + 8 * vst, ((j / VSTG) & 1) ^ 1, abort_flag, p.status)) break;
-                mbar_expect_tx(v_full + 8 * vst, 2 * TILE);
-#pragma unroll
-                for (int kb = 0; kb < KB; ++kb) {
-                    tma_load_2d(sK + kst * TILE + kb * 16384, &tmQKV, xk + kb * 64, row0 + j * 128, v_full + 8 * vst);
-                    tma_load_2d(sV + vst * TILE + kb * 16384, &tmQKV, xv + kb * 64, row0 + j * 128, v_full + 8 * vst);
+                    for (int c = 0; c < KB; ++c) tma_load_2d(sb + c * 16384, &tmQKV, xk + 64 * c, b * p.T + kb * 128, fb);
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                issued = j + 1;
             }
-            if (*abort_flag) {
-                drain(qd_full, 0);
-                for (int j = (issued > VSTG ? issued - VSTG : 0); j < issued; ++j)
-                    drain(v_full + 8 * (j % VSTG), (j / VSTG) & 1);
+            if (!ok) {
+                for (int st = 0; st < STAGES; ++st)
+                    if (issued >> st & 1) drain(full + 8 * st, (issued_phase >> st) & 1);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id_s = idesc_bf16(128, 128, false, false);
-            const uint32_t id_q = idesc_bf16(128, HD, false, true);
-            bool ok = mbar_wait(qd_full, 0, abort_flag, p.status);
-            for (int j = 0; ok && j <= nblk; ++j) {
-                if (j < nblk) {
-                    // S_j and dP_j as one group: K_j, V_j landed, dP_{j-1} read out of TMEM
-                    const int kst = j % KSTG, vst = j % VSTG, sb = j & 1;
-                    if (!mbar_wait(v_full + 8 * vst, (j / VSTG) & 1, abort_flag, p.status)) break;
-                    if (j > 0 && !mbar_wait(dp_free, (j - 1) & 1, abort_flag, p.status)) break;
+            const uint32_t idesc = idesc_bf16(128, HD, true, true);
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+                int b, h, qb;
+                dq_unit(p, u, b, h, qb);
+                if (!mbar_wait(acc_empty + 8 * acc, acc_phase ^ 1, abort_flag, p.status)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + acc * HD;
+                for (int kb = 0; kb <= qb; ++kb) {
+                    if (!mbar_wait(full + 8 * stage, phase, abort_flag, p.status)) { ok = false; break; }
                     tc_fence_after();
+                    const uint32_t sa = base + stage * Lay::STAGE, sb = sa + Lay::A_BYTES;
 #pragma unroll
-                    for (int ks = 0; ks < HD / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16(tS + sb * 128, smem_desc(sQ + off, 16, 1024),
-                                 smem_desc(sK + kst * TILE + off, 16, 1024), id_s, ks > 0 ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int ks = 0; ks < HD / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        mma_bf16(tdP, smem_desc(sDO + off, 16, 1024), smem_desc(sV + vst * TILE + off, 16, 1024),
-                                 id_s, ks > 0 ? 1u : 0u);
-                    }
-                    mma_commit(dp_full);
-                    mma_commit(v_empty + 8 * vst);
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16(d, smem_desc(sa + ks * 2048, 16384, 1024), smem_desc(sb + ks * 2048, 16384, 1024),
+                                 idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+                    mma_commit(empty + 8 * stage);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                if (j > 0) {
-                    // dQ += dS_{j-1} K_{j-1}: keys 16kk..16kk+15 sit in the packed columns
-                    // 32*(kk/2) + 8*(kk%2) of the S buffer (written by column group kk/2)
-                    const int jj = j - 1, sb = jj & 1;
-                    if (!mbar_wait(ds_full + 8 * sb, (jj >> 1) & 1, abort_flag, p.status)) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ts(tdQ, tS + sb * 128 + 32 * (kk >> 1) + 8 * (kk & 1),
-                                    smem_desc(sK + (jj % KSTG) * TILE + kk * 2048, 16384, 1024), id_q,
-                                    (jj > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(k_empty + 8 * (jj % KSTG));
-                }
+                if (!ok) break;
+                mma_commit(acc_full + 8 * acc);
+                if (++acc == 2) { acc = 0; acc_phase ^= 1; }
             }
-            mma_commit(dq_done);
         }
     } else {
-        // warps 2..17: TMEM lane quarter q (query rows), key column group cg (32 keys)
-        const int q = warp & 3, cg = (warp - 2) >> 2;
-        const int r = q * 32 + lane;
-        const int qpos = qb * 128 + r;
-        const bool live = qpos < p.T;
-        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const size_t si = ((size_t)b * p.H + h) * attn_tpad(p.T) + qpos;
-        const float Dr = p.D[si], lse2 = p.lse2[si];
-        bool ok = true;
-        for (int j = 0; j < nblk; ++j) {
-            const int sb = j & 1;
-            if (!warp_wait(dp_full, j & 1, abort_flag, p.status)) {
-                ok = false;
-                break;
-            }
+        // epilogue warps 2..5: warp w reads TMEM lanes 32*(w%4).. (query rows)
+        const int q = warp & 3;
+        const int Nqkv = (p.H + 2 * p.nkv) * HD;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+            int b, h, qb;
+            dq_unit(p, u, b, h, qb);
+            if (!warp_wait(acc_full + 8 * acc, acc_phase, abort_flag, p.status)) break;
             tc_fence_after();
-            uint32_t rs[32], rd[32];
-            tmem_ld32_issue(tS + lane_off + sb * 128 + cg * 32, rs);
-            tmem_ld32_issue(tdP + lane_off + cg * 32, rd);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dp_free);
-            // keys j*128 + cg*32 + e, e <= lim, are visible from this row
-            const int lim = !live ? -1 : (j == qb ? r - cg * 32 : 31);
-            uint32_t pk[16];
-            if (__all_sync(0xffffffffu, lim >= 31)) {
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float d0 = ex2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -lse2)) *
-                                     (__uint_as_float(rd[e]) - Dr);
-                    const float d1 = ex2(fmaf(__uint_as_float(rs[e + 1]), p.scale_log2, -lse2)) *
-                                     (__uint_as_float(rd[e + 1]) - Dr);
-                    pk[e >> 1] = pack_bf16(d0, d1);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const float d0 = e <= lim ? ex2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -lse2)) *
-                                                    (__uint_as_float(rd[e]) - Dr)
-                                              : 0.f;
-                    const float d1 = e + 1 <= lim ? ex2(fmaf(__uint_as_float(rs[e + 1]), p.scale_log2, -lse2)) *
-                                                        (__uint_as_float(rd[e + 1]) - Dr)
-                                                  : 0.f;
-                    pk[e >> 1] = pack_bf16(d0, d1);
-                }
-            }
-            tmem_st16(tS + lane_off + sb * 128 + cg * 32, pk);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ds_full + 8 * sb);
-        }
-        if (ok && warp_wait(dq_done, 0, abort_flag, p.status)) {
-            tc_fence_after();
-            // column group cg writes dq columns 32*cg .. 32*cg+31 (hd 64: groups 0 and 1)
-            if (cg * 32 < HD) {
+            const int qpos = qb * 128 + q * 32 + lane;
+            const bool live = qpos < p.T;
+            bf16* out = p.dqkv + ((size_t)b * p.T + (live ? qpos : 0)) * Nqkv + (size_t)h * HD;
+            const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * HD;
+#pragma unroll 1
+            for (int c = 0; c < HD / 32; ++c) {
                 float v[32];
-                tmem_ld32(tdQ + lane_off + cg * 32, v);
+                tmem_ld32(tb + c * 32, v);
                 if (live) {
-                    bf16* out = p.dqkv + ((size_t)row0 + qpos) * Nqkv + h * HD + cg * 32;
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        *reinterpret_cast<uint4*>(out + 8 * e) =
+                        *reinterpret_cast<uint4*>(out + c * 32 + 8 * e) =
                             make_uint4(pack_bf16(v[8 * e] * p.scale, v[8 * e + 1] * p.scale),
                                        pack_bf16(v[8 * e + 2] * p.scale, v[8 * e + 3] * p.scale),
                                        pack_bf16(v[8 * e + 4] * p.scale, v[8 * e + 5] * p.scale),
                                        pack_bf16(v[8 * e + 6] * p.scale, v[8 * e + 7] * p.scale));
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + 8 * acc);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, kCols);
     }
 }
 
@@ -808,7 +838,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         bool ok = true;
         for (int u = 0; u < nunits; ++u) {
             const int st = u & 1;
-            const int i = p.nqb - 1 - u / Hg;
+            const int i = p.nqb - 1 - u / Hg, h = g * Hg + u % Hg;
             if (!warp_wait(st_full, u & 1, abort_flag, p.status) ||
                 !warp_wait(qo_full + 8 * st, (u >> 1) & 1, abort_flag, p.status)) {
                 ok = false;
@@ -877,6 +907,18 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                 pv[4 * k + 2] *= __uint_as_float(rd[4 * k + 2]) - dd.z;
                 pv[4 * k + 3] *= __uint_as_float(rd[4 * k + 3]) - dd.w;
             }
+            uint4 dsv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float* d = pv + 8 * k;
+                dsv[k] = make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
+                                    pack_bf16(d[6], d[7]));
+            }
+            // this row's 32 queries of the dS^T tile, for the dQ product
+            uint4* gds = reinterpret_cast<uint4*>(p.ds + (ds_tile(b, h, p.H, p.ntri, i, kvb) * 128 + r) * 128 +
+                                                  cg * 32);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) gds[k] = dsv[k];
             // the dK MMAs of the previous unit have read the dS^T tile
             if (u > 0 && !warp_wait(ds_free, (u - 1) & 1, abort_flag, p.status)) {
                 ok = false;
@@ -886,10 +928,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int c8 = (cg & 1) * 4 + k;
-                const float* d = pv + 8 * k;
-                *reinterpret_cast<uint4*>(drow + ((c8 ^ (r & 7)) << 4)) =
-                    make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
-                               pack_bf16(d[6], d[7]));
+                *reinterpret_cast<uint4*>(drow + ((c8 ^ (r & 7)) << 4)) = dsv[k];
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -959,16 +998,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 template <int HD>
 int fwd_launch(const CUtensorMap& map, const AttnParams& p, cudaStream_t s) {
     if (ensure_smem_limit((const void*)attn_fwd_tc_kernel<HD>, FwdLayout<HD>::BYTES) != cudaSuccess) return -1;
-    dim3 grid(p.H, p.B, p.nqb);
+    const int grid = std::min(p.num_units, device_sm_count());
     attn_fwd_tc_kernel<HD><<<grid, NT, FwdLayout<HD>::BYTES, s>>>(map, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
 template <int HD>
-int dq_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
-    if (ensure_smem_limit((const void*)attn_dq_tc_kernel<HD>, DqLayout<HD>::BYTES) != cudaSuccess) return -1;
-    attn_dq_tc_kernel<HD><<<dim3(p.H, p.B, p.nqb), NTB, DqLayout<HD>::BYTES, s>>>(kv, do128, p);
+int dq_ds_launch(const CUtensorMap& ds, const CUtensorMap& kv, const DqdsParams& p, cudaStream_t s) {
+    if (ensure_smem_limit((const void*)attn_dq_ds_kernel<HD>, DqdsLayout<HD>::BYTES) != cudaSuccess) return -1;
+    const int grid = std::min(p.num_units, device_sm_count());
+    attn_dq_ds_kernel<HD><<<grid, NTQ, DqdsLayout<HD>::BYTES, s>>>(ds, kv, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -982,22 +1022,28 @@ int dkv_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams&
 }
 
 // Parameters and the two tensor maps (qkv and dO, 128-row boxes) of both kernels.
-bool bwd_setup(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv, int B,
-               int T, int H, int nkv, int hd, int* status, BwdParams* p, CUtensorMap* kv, CUtensorMap* do128) {
+int ntri_of(int T) {
+    const int nqb = (T + 127) / 128;
+    return nqb * (nqb + 1) / 2;
+}
+
+// Parameters and the two tensor maps (qkv and dO, 128-row boxes) of the dK/dV kernel.
+bool bwd_setup(const void* qkv, const void* dO, float* Dbuf, void* dqkv, void* ds, int B, int T, int H, int nkv,
+               int hd, int* status, BwdParams* p, CUtensorMap* kv, CUtensorMap* do128) {
     if (!attention_tc_bwd_supported(hd)) return false;
-    if (!aligned16(qkv) || !aligned16(dO) || !aligned16(dqkv) || !aligned16(Dbuf) || (o && !aligned16(o)))
-        return false;
+    if (!aligned16(qkv) || !aligned16(dO) || !aligned16(dqkv) || !aligned16(Dbuf) || !aligned16(ds)) return false;
     if (B > 65535 || H > 65535 || nkv < 1 || H % nkv != 0) return false;
     const int Nqkv = (H + 2 * nkv) * hd;
     if (!map_rows(kv, qkv, Nqkv, (uint64_t)B * T, 128) || !map_rows(do128, dO, (uint64_t)H * hd, (uint64_t)B * T, 128))
         return false;
     *p = BwdParams{};
-    p->B = B; p->T = T; p->H = H; p->nkv = nkv; p->nqb = (T + 127) / 128;
+    p->B = B; p->T = T; p->H = H; p->nkv = nkv; p->nqb = (T + 127) / 128; p->ntri = ntri_of(T);
     p->scale = 1.f / sqrtf((float)hd);
     p->scale_log2 = kLog2e * p->scale;
     p->D = Dbuf;
     p->lse2 = Dbuf + attn_stat_elems(B, T, H);
     p->dqkv = reinterpret_cast<bf16*>(dqkv);
+    p->ds = reinterpret_cast<bf16*>(ds);
     p->status = status;
     return true;
 }
@@ -1007,12 +1053,17 @@ bool bwd_setup(const void* qkv, const void* o, const void* dO, const float* lse,
 int attention_tc_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, int nkv, int hd, void*, size_t,
                      int* status, cudaStream_t s) {
     if (hd != 64 && hd != 128) return 1;
-    if (!aligned16(qkv) || !aligned16(o) || B > 65535 || H > 65535) return 1;
+    if (!aligned16(qkv) || !aligned16(o) || nkv < 1 || H % nkv) return 1;
     const int Nqkv = (H + 2 * nkv) * hd;
     CUtensorMap map;
     if (!map_rows(&map, qkv, Nqkv, (uint64_t)B * T, 128)) return 1;
-    AttnParams p;
+    AttnParams p{};
     p.B = B; p.T = T; p.H = H; p.nkv = nkv; p.nqb = (T + 127) / 128;
+    p.pairs_per_group = (H / nkv + 1) / 2;
+    p.npair = nkv * p.pairs_per_group;
+    const long long units = (long long)B * p.npair * p.nqb;
+    if (units > (1ll << 30)) return 1;
+    p.num_units = (int)units;
     p.scale_log2 = kLog2e / sqrtf((float)hd);
     p.o = reinterpret_cast<bf16*>(o);
     p.lse = lse;
@@ -1022,41 +1073,57 @@ int attention_tc_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, 
 
 bool attention_tc_bwd_supported(int hd) { return hd == 64 || hd == 128; }
 
-int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
-                        int B, int T, int H, int nkv, int hd, int* status, cudaStream_t s) {
-    BwdParams p;
-    CUtensorMap kv, do128;
-    if (!o || !lse || !bwd_setup(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, &p, &kv, &do128)) return 1;
-    {
-        const long long threads = (long long)attn_stat_elems(B, T, H) * (hd / 8);
-        const unsigned blocks = (unsigned)((threads + 255) / 256);
-        const bf16* ob = reinterpret_cast<const bf16*>(o);
-        const bf16* db = reinterpret_cast<const bf16*>(dO);
-        float* D = Dbuf;
-        float* l2 = Dbuf + attn_stat_elems(B, T, H);
-        if (hd == 128) attn_bwd_stats_kernel<128><<<blocks, 256, 0, s>>>(ob, db, lse, D, l2, B, T, H);
-        else attn_bwd_stats_kernel<64><<<blocks, 256, 0, s>>>(ob, db, lse, D, l2, B, T, H);
-        count_launch();
-        if (cudaGetLastError() != cudaSuccess) return -1;
-    }
-    return hd == 128 ? dq_launch<128>(kv, do128, p, s) : dq_launch<64>(kv, do128, p, s);
+size_t attention_tc_workspace_bytes(int B, int T, int H, int, int hd) {
+    if (!attention_tc_bwd_supported(hd)) return 0;
+    return (size_t)B * H * ntri_of(T) * 128 * 128 * sizeof(bf16);
 }
 
-int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqkv, int B, int T, int H, int nkv,
-                         int hd, int* status, cudaStream_t s) {
+int attention_tc_bwd_stats(const void* o, const void* dO, const float* lse, float* Dbuf, int B, int T, int H, int hd,
+                           cudaStream_t s) {
+    if (!attention_tc_bwd_supported(hd) || !aligned16(o) || !aligned16(dO) || !lse || !Dbuf) return 1;
+    const long long threads = (long long)attn_stat_elems(B, T, H) * (hd / 8);
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    const bf16* ob = reinterpret_cast<const bf16*>(o);
+    const bf16* db = reinterpret_cast<const bf16*>(dO);
+    float* l2 = Dbuf + attn_stat_elems(B, T, H);
+    if (hd == 128) attn_bwd_stats_kernel<128><<<blocks, 256, 0, s>>>(ob, db, lse, Dbuf, l2, B, T, H);
+    else attn_bwd_stats_kernel<64><<<blocks, 256, 0, s>>>(ob, db, lse, Dbuf, l2, B, T, H);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqkv, void* ws, size_t ws_bytes, int B,
+                         int T, int H, int nkv, int hd, int* status, cudaStream_t s) {
     BwdParams p;
     CUtensorMap kv, do128;
-    if (!bwd_setup(qkv, nullptr, dO, nullptr, Dbuf, dqkv, B, T, H, nkv, hd, status, &p, &kv, &do128)) return 1;
+    if (!ws || ws_bytes < attention_tc_workspace_bytes(B, T, H, nkv, hd)) return 1;
+    if (!bwd_setup(qkv, dO, Dbuf, dqkv, ws, B, T, H, nkv, hd, status, &p, &kv, &do128)) return 1;
     return hd == 128 ? dkv_launch<128>(kv, do128, p, s) : dkv_launch<64>(kv, do128, p, s);
 }
 
-int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
-                     int B, int T, int H, int nkv, int hd, void*, size_t, int* status, cudaStream_t s) {
-    int r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, status, s);
-    if (r != 0) return r;
-    return attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, B, T, H, nkv, hd, status, s);
+int attention_tc_bwd_dq(const void* qkv, const void* ws, size_t ws_bytes, void* dqkv, int B, int T, int H, int nkv,
+                        int hd, int* status, cudaStream_t s) {
+    if (!attention_tc_bwd_supported(hd) || !ws || ws_bytes < attention_tc_workspace_bytes(B, T, H, nkv, hd)) return 1;
+    if (!aligned16(qkv) || !aligned16(ws) || !aligned16(dqkv) || B > 65535 || nkv < 1 || H % nkv) return 1;
+    const int Nqkv = (H + 2 * nkv) * hd;
+    CUtensorMap mds, mkv;
+    const uint64_t ds_rows = (uint64_t)B * H * ntri_of(T) * 128;
+    if (!map_rows(&mds, ws, 128, ds_rows, 128) || !map_rows(&mkv, qkv, Nqkv, (uint64_t)B * T, 128)) return 1;
+    DqdsParams p{};
+    p.B = B; p.T = T; p.H = H; p.nkv = nkv; p.nqb = (T + 127) / 128; p.ntri = ntri_of(T);
+    p.num_units = B * H * p.nqb;
+    p.scale = 1.f / sqrtf((float)hd);
+    p.dqkv = reinterpret_cast<bf16*>(dqkv);
+    p.status = status;
+    return hd == 128 ? dq_ds_launch<128>(mds, mkv, p, s) : dq_ds_launch<64>(mds, mkv, p, s);
 }
 
-size_t attention_tc_workspace_bytes(int, int, int, int, int) { return 0; }
+int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
+                     int B, int T, int H, int nkv, int hd, void* ws, size_t ws_bytes, int* status, cudaStream_t s) {
+    int r = attention_tc_bwd_stats(o, dO, lse, Dbuf, B, T, H, hd, s);
+    if (r == 0) r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, ws, ws_bytes, B, T, H, nkv, hd, status, s);
+    if (r == 0) r = attention_tc_bwd_dq(qkv, ws, ws_bytes, dqkv, B, T, H, nkv, hd, status, s);
+    return r;
+}
 
 }  // namespace nc

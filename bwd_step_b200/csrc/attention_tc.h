@@ -7,15 +7,20 @@ namespace nc {
 // < 0 on a CUDA error.
 int attention_tc_fwd(const void* qkv, void* o, float* lse, int B, int T, int H, int nkv, int hd, void* ws,
                      size_t ws_bytes, int* status, cudaStream_t s);
-// Dbuf holds attn_dbuf_elems(B, T, H) floats: D = rowsum(dO * o) and lse * log2(e),
-// both [B, H, attn_tpad(T)], written by the dq kernel and read by the dk/dv kernel.
+bool attention_tc_bwd_supported(int hd);
+// Scratch of the backward: the stored dS^T tiles (bf16), one 128 x 128 tile
+// per causal (query block, key block) pair of every (batch row, query head).
+size_t attention_tc_workspace_bytes(int B, int T, int H, int nkv, int hd);
+// The whole backward: stats, then dk/dv (storing dS), then dq.  Dbuf holds
+// attn_dbuf_elems(B, T, H) floats: D = rowsum(dO * o) and lse * log2(e), both
+// [B, H, attn_tpad(T)].
 int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
                      int B, int T, int H, int nkv, int hd, void* ws, size_t ws_bytes, int* status, cudaStream_t s);
-// The two halves of attention_tc_bwd: dq (with D and the log2-domain lse), then dk/dv.
-bool attention_tc_bwd_supported(int hd);
-int attention_tc_bwd_dq(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
-                        int B, int T, int H, int nkv, int hd, int* status, cudaStream_t s);
-int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqkv, int B, int T, int H, int nkv,
-                         int hd, int* status, cudaStream_t s);
-size_t attention_tc_workspace_bytes(int B, int T, int H, int nkv, int hd);
+// Its three launches, in order.
+int attention_tc_bwd_stats(const void* o, const void* dO, const float* lse, float* Dbuf, int B, int T, int H, int hd,
+                           cudaStream_t s);
+int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqkv, void* ws, size_t ws_bytes, int B,
+                         int T, int H, int nkv, int hd, int* status, cudaStream_t s);
+int attention_tc_bwd_dq(const void* qkv, const void* ws, size_t ws_bytes, void* dqkv, int B, int T, int H, int nkv,
+                        int hd, int* status, cudaStream_t s);
 }  // namespace nc

@@ -28,6 +28,7 @@ namespace {
 using namespace tc;
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+static_assert(BN == kGemmTileN, "the LM-head epilogue writes one sum per BN-column tile");
 constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int NTHREADS = 192;
@@ -50,7 +51,60 @@ struct TcParams {
     const float* cos_t;
     const float* sin_t;
     int tma_out;  // epilogue stages 32x32 sub-tiles in shared memory and writes them by TMA
+    const int32_t* tgt;  // EPI_LMHEAD
+    float* stats;
+    int stats_ld;
+    float* zt;
+    float* ut;
+    const float* rs;  // EPI_ROWSCALE
 };
+
+// Per-row state of the epilogue across the 32-column chunks of one tile.
+struct RowCtx {
+    int tgt;    // EPI_LMHEAD: the row's target column (-1 for rows past M)
+    float rs;   // EPI_ROWSCALE: the row's factor
+    float sum;  // EPI_LMHEAD: sum of e over the tile's columns so far
+};
+
+__device__ __forceinline__ RowCtx row_ctx(const TcParams& p, int row) {
+    RowCtx c;
+    const bool live = row < p.M;
+    c.tgt = (p.epi == EPI_LMHEAD && live) ? p.tgt[row] : -1;
+    c.rs = (p.epi == EPI_ROWSCALE && live) ? p.rs[row] : 0.f;
+    c.sum = 0.f;
+    return c;
+}
+
+// LM-head epilogue of one 32-column chunk n0.. of a row (untied LM head and
+// tanh logit softcap of the nanochat announcement, vpshk.cn, architecture
+// list, followed by the cross-entropy's softmax): the softcapped logit
+// z = cap tanh(l/cap) is bounded by cap, so e = exp(z - cap) lies in
+// [exp(-2 cap), 1] and needs no running maximum; v becomes
+// u = e (1 - (z/cap)^2), the product of the unnormalised softmax and the
+// softcap's derivative.  The logits themselves are never stored.
+__device__ __forceinline__ void lmhead_chunk(const TcParams& p, int row, int n0, float* v, RowCtx& rc) {
+    constexpr float kL2e = 1.44269504088896340736f;
+    const float ic = 1.f / p.cap, cl2 = p.cap * kL2e;
+    if ((unsigned)(rc.tgt - n0) < 32u) {  // the target column is in this chunk: its z and u in fp32
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (n0 + i == rc.tgt) {
+                const float t = tanhf(v[i] * ic);
+                p.zt[row] = p.cap * t;
+                p.ut[row] = ex2((t - 1.f) * cl2) * (1.f - t * t);
+            }
+    }
+    const int nv = min(32, p.N - n0);
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float t = tanhf(v[i] * ic);
+        const float e = ex2((t - 1.f) * cl2);
+        if (i < nv) sum += e;
+        v[i] = e * (1.f - t * t);
+    }
+    rc.sum += sum;
+}
 
 __device__ __forceinline__ void decode(const TcParams& p, int u, int& tm, int& tn, int& ks) {
     int tile = u % (p.tiles_m * p.tiles_n);
@@ -86,7 +140,7 @@ __device__ __forceinline__ void store_row(void* C, bool bf, int64_t off, const f
 }
 
 // Epilogue of 32 consecutive columns n0.. of one output row.
-__device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int n0, float* v) {
+__device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int n0, float* v, RowCtx& rc) {
     const int nv = min(32, p.N - n0);
     const bool vec = p.vec_ok != 0;
     if (p.part) {
@@ -141,6 +195,15 @@ __device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int
             for (int i = 0; i < 32; ++i) v[i] = p.cap * tanhf(v[i] * ic);
             store_row(p.C, p.c_bf16, off, v, nv, vec);
         } break;
+        case EPI_LMHEAD:
+            lmhead_chunk(p, row, n0, v, rc);
+            store_row_bf16(reinterpret_cast<bf16*>(p.C) + off, v, nv, vec);
+            break;
+        case EPI_ROWSCALE:
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= rc.rs;
+            store_row_f32(reinterpret_cast<float*>(p.C) + off, v, nv, vec);
+            break;
     }
 }
 
@@ -168,7 +231,7 @@ __device__ __forceinline__ void stage_bf16(uint8_t* buf, int lane, const float* 
 // One 32-column chunk through the staging buffers; called by all lanes of the warp.
 __device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUtensorMap* tmC, const CUtensorMap* tmC2,
                                                    uint8_t* stg, int lane, int ks, int row, int row0w, int n0, float* v,
-                                                   int cnt) {
+                                                   int cnt, RowCtx& rc) {
     uint8_t* buf = stg + (cnt & 1) * 4096;
     if (cnt >= 2) {
         if (lane == 0) bulk_wait_read_1();
@@ -203,6 +266,11 @@ __device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUte
             const float ic = 1.f / p.cap;
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = p.cap * tanhf(v[i] * ic);
+        } else if (mode == EPI_LMHEAD) {
+            if (row < p.M) lmhead_chunk(p, row, n0, v, rc);
+        } else if (mode == EPI_ROWSCALE) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= rc.rs;
         }
         if (bf) stage_bf16(buf, lane, v);
         else stage_f32(buf, lane, v);
@@ -399,14 +467,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
                 else epilogue_qkrope<64>(p, row, tn * BN, tb);
             } else {
+                RowCtx rc = row_ctx(p, row);
                 for (int c = 0; c < BN / 32; ++c) {
                     const int n0 = tn * BN + c * 32;
                     if (n0 >= p.N) break;
                     float v[32];
                     tmem_ld32(tb + c * 32, v);
-                    if (p.tma_out) epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++);
-                    else if (row < p.M) epilogue(p, ks, row, n0, v);
+                    if (p.tma_out) epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++, rc);
+                    else if (row < p.M) epilogue(p, ks, row, n0, v, rc);
                 }
+                if (p.epi == EPI_LMHEAD && row < p.M) p.stats[(size_t)row * p.stats_ld + tn] = rc.sum;
             }
             tc_fence_before();
             __syncwarp();
@@ -557,14 +627,16 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
                 else epilogue_qkrope<64>(p, row, tn * BN, tb);
             } else {
+                RowCtx rc = row_ctx(p, row);
                 for (int c = 0; c < BN / 32; ++c) {
                     const int n0 = tn * BN + c * 32;
                     if (n0 >= p.N) break;
                     float v[32];
                     tmem_ld32(tb + c * 32, v);
-                    if (p.tma_out) epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++);
-                    else if (row < p.M) epilogue(p, ks, row, n0, v);
+                    if (p.tma_out) epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++, rc);
+                    else if (row < p.M) epilogue(p, ks, row, n0, v, rc);
                 }
+                if (p.epi == EPI_LMHEAD && row < p.M) p.stats[(size_t)row * p.stats_ld + tn] = rc.sum;
             }
             tc_fence_before();
             __syncwarp();
@@ -650,6 +722,10 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
         ((g.hd != 64 && g.hd != 128) || g.c_t != DT_BF16 || g.T <= 0 || !g.rqk || !g.cos_t || !g.sin_t ||
          (reinterpret_cast<uintptr_t>(g.C) & 15) || (g.ldc % 8) || (g.N % g.hd)))
         return 1;
+    if (g.epi == EPI_LMHEAD &&
+        (g.c_t != DT_BF16 || !g.tgt || !g.stats || !g.zt || !g.ut || g.stats_ld < gemm_tiles_n(g.N) || !(g.cap > 0.f)))
+        return 1;
+    if (g.epi == EPI_ROWSCALE && (g.c_t != DT_F32 || !g.rs)) return 1;
     if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 1;
     auto al16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
     if (!al16(g.A) || !al16(g.B) || (g.lda * 2) % 16 || (g.ldb * 2) % 16) return 1;
@@ -675,6 +751,8 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     p.status = g.status;
     p.hd = g.hd; p.T = g.T; p.qk_heads = g.qk_heads;
     p.rqk = g.rqk; p.cos_t = g.cos_t; p.sin_t = g.sin_t;
+    p.tgt = g.tgt; p.stats = g.stats; p.stats_ld = g.stats_ld; p.zt = g.zt; p.ut = g.ut;
+    p.rs = g.rs;
     const int esz = p.c_bf16 ? 2 : 4;
     bool vec = al16(g.C) && (g.ldc * esz) % 16 == 0;
     if (g.epi == EPI_RELU2) vec = vec && al16(g.C2) && (g.ldc2 * 2) % 16 == 0;

@@ -41,6 +41,14 @@ cudaError_t launch_qknorm_rope_bwd(DType at, void* dqkv, const void* qkv, const 
 // loss_rows[r] = lse - z[tgt]; dl = inv_M*(softmax - onehot)*(1-(z/cap)^2).
 cudaError_t launch_ce_chunk(DType zt, DType dlt, const void* z, const int32_t* tgt, int R, int V, float cap,
                             float inv_M, float* loss_rows, void* dl, int* status, cudaStream_t s);
+// After the EPI_LMHEAD GEMM of R rows (u [R, V] bf16, stats [R, ntiles]): per row
+// S = sum of the tile sums (fixed order), loss_rows[r] = cap + log S - zt[r];
+// rs[r] = inv_M / S; u[r, tgt] = ut[r] - (1 - (zt/cap)^2) S (folds the one-hot
+// term into u, in fp32, before the single rounding); xfs[r] = xf[r] * rs[r].
+// A target outside [0, V) sets ST_BAD_TOKEN and zeroes the row's loss, rs and xfs.
+cudaError_t launch_lm_rowstats(const float* stats, int ntiles, const float* zt, const float* ut,
+                               const int32_t* tgt, int R, int V, int d, float cap, float inv_M, void* u,
+                               const void* xf, void* xfs, float* rs, float* loss_rows, int* status, cudaStream_t s);
 // loss = mean(loss_rows[0..M)), fixed summation order.
 cudaError_t launch_loss_reduce(const float* loss_rows, int M, float* loss, cudaStream_t s);
 
@@ -81,6 +89,11 @@ enum Epi : int {
     EPI_QKROPE = 5,     // fused qkv rows: per head of the first qk_heads heads,
                         // C = rope(rmsnorm_hd(acc)) and rqk = its inverse RMS; other
                         // columns (v) C = acc.  bf16 C, head_dim 64 or 128 (tcgen05 only)
+    EPI_LMHEAD = 6,     // LM head, logits never stored: z = cap*tanh(acc/cap), e = exp(z - cap),
+                        // C = e * (1 - (z/cap)^2) (bf16); per (row, 256-column tile) the sum of e
+                        // into stats[row * stats_ld + tile]; at the column tgt[row], z and C in
+                        // fp32 into zt[row], ut[row] (tcgen05 only)
+    EPI_ROWSCALE = 7,   // C = acc * rs[row]                 (C fp32; tcgen05 only)
 };
 
 struct GemmDesc {
@@ -100,7 +113,19 @@ struct GemmDesc {
     float* rqk = nullptr;
     const float* cos_t = nullptr;
     const float* sin_t = nullptr;
+    // EPI_LMHEAD: targets of the M rows, per-(row, tile) sums, target z / C values
+    const int32_t* tgt = nullptr;
+    float* stats = nullptr;
+    int stats_ld = 0;
+    float* zt = nullptr;
+    float* ut = nullptr;
+    // EPI_ROWSCALE: one factor per row
+    const float* rs = nullptr;
 };
+
+// Column tiles of the tensor-core GEMM's output (EPI_LMHEAD writes one sum per tile).
+constexpr int kGemmTileN = 256;
+inline int gemm_tiles_n(int N) { return (N + kGemmTileN - 1) / kGemmTileN; }
 
 // Plain fp32-FMA tiled GEMM (any strides, any sizes).
 cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t s);

@@ -616,6 +616,52 @@ __global__ void __launch_bounds__(CER_NT, 1) ce_chunk_resident_kernel(const bf16
     }
 }
 
+// One warp per row of the fused LM head's chunk (see launch_lm_rowstats).
+template <typename A>
+__global__ void __launch_bounds__(256) lm_rowstats_kernel(const float* __restrict__ stats, int ntiles,
+                                                         const float* __restrict__ zt, const float* __restrict__ ut,
+                                                         const int32_t* __restrict__ tgt, int R, int V, int d,
+                                                         float cap, float inv_M, A* __restrict__ u,
+                                                         const A* __restrict__ xf, A* __restrict__ xfs,
+                                                         float* __restrict__ rs, float* __restrict__ loss_rows,
+                                                         int* status) {
+    const int row = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= R) return;
+    // S = sum over the row's tiles of sum exp(z - cap): lane-strided partial sums,
+    // then a fixed butterfly (the same order on every run)
+    const float* st = stats + (size_t)row * ntiles;
+    float S = 0.f;
+    for (int t = lane; t < ntiles; t += 32) S += st[t];
+    S = warp_sum(S);
+    const int t = tgt[row];
+    const bool bad = t < 0 || t >= V;
+    const float scale = bad ? 0.f : inv_M / S;
+    if (lane == 0) {
+        if (bad) set_status(status, ST_BAD_TOKEN);
+        const float z = bad ? 0.f : zt[row];
+        loss_rows[row] = bad ? 0.f : cap + logf(S) - z;
+        rs[row] = scale;
+        if (!bad) {
+            // dl at the target is (e/S - 1)(1 - (z/cap)^2) / M = (ut - g S) * scale: fold the
+            // one-hot term into u in fp32, so the target entry is rounded once
+            const float q = z / cap;
+            u[(size_t)row * V + t] = fromf<A>(ut[row] - (1.f - q * q) * S);
+        }
+    }
+    // xfs = xf * scale (the dW product's operand: dW = u^T xfs)
+    const A* x = xf + (size_t)row * d;
+    A* y = xfs + (size_t)row * d;
+    constexpr int VEC = Vec<A>::N;
+    for (int c = lane * VEC; c < d; c += 32 * VEC) {
+        float v[VEC];
+        load_vec(x + c, v);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) v[i] *= scale;
+        store_vec(y + c, v);
+    }
+}
+
 __global__ void loss_reduce_kernel(const float* __restrict__ rows, int M, float* loss) {
     __shared__ float sh[1024];
     float s = 0.f;
@@ -1004,6 +1050,17 @@ cudaError_t launch_ce_chunk(DType zt, DType dlt, const void* z, const int32_t* t
         if (dlt == DT_BF16) NC_CE(float, bf16); else NC_CE(float, float);
     }
 #undef NC_CE
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lm_rowstats(const float* stats, int ntiles, const float* zt, const float* ut,
+                               const int32_t* tgt, int R, int V, int d, float cap, float inv_M, void* u,
+                               const void* xf, void* xfs, float* rs, float* loss_rows, int* status, cudaStream_t s) {
+    const unsigned blocks = (unsigned)(((size_t)R * 32 + 255) / 256);
+    lm_rowstats_kernel<bf16><<<blocks, 256, 0, s>>>(stats, ntiles, zt, ut, tgt, R, V, d, cap, inv_M,
+                                                    reinterpret_cast<bf16*>(u), reinterpret_cast<const bf16*>(xf),
+                                                    reinterpret_cast<bf16*>(xfs), rs, loss_rows, status);
     count_launch();
     return cudaGetLastError();
 }

@@ -30,6 +30,10 @@ struct nc_model {
     int V, d, L, H, nkv, hd, F, Nqkv;
     DType at;  // weight / activation type
     bool tc = false;  // tcgen05 path available (bf16 on sm_100)
+    // LM head: fused (logits never stored; tensor-core path only) or materialised
+    // logit chunks with a separate cross-entropy pass; rows per chunk (0 = default)
+    int lm_mode = NC_LM_HEAD_FUSED;
+    int lm_rows = 0;
     // caller-owned events recorded when each gradient bucket is final (may be empty)
     std::vector<cudaEvent_t> grad_events;
     // profiler: CUDA events around every launch while enabled
@@ -61,16 +65,25 @@ struct Plan {
     size_t layers, lay_stride;
     size_t l_a, l_r1, l_qkv, l_rqk, l_o, l_lse, l_m, l_r2, l_ru, l_h;
     size_t du, dO, dqkv, Dbuf, zc, dlc, loss_rows, emb, splitk, splitk_bytes, attn_ws, attn_ws_bytes;
+    size_t lm_stats, lm_zt, lm_ut, lm_rs, lm_xfs;
+    int lm_tiles = 0;
 };
 
-// Rows of the LM head processed at once: the [R, V] fp32 logit chunk plus its
-// gradient stay near 1.5 GiB, so the full [B*T, V] logit tensor is never
-// materialised.
+bool lm_fused(const nc_model* m) { return m->tc && m->lm_mode == NC_LM_HEAD_FUSED; }
+
+// Rows of the LM head processed at once, so that the full [B*T, V] tensor is
+// never materialised.  Fused: the [R, V] bf16 chunk of u = e (1 - (z/cap)^2)
+// (no logits) is kept near 512 MiB; materialised: the [R, V] logit chunk and
+// its gradient near 1 GiB together.  A caller-chosen row count overrides.
 int lm_chunk_rows(const nc_model* m, int M) {
-    size_t per_row = (size_t)m->V * (4 + dt_size(m->at));
-    size_t budget = (size_t)1536 << 20;
-    size_t R = budget / per_row;
-    R = std::max<size_t>(128, R / 128 * 128);
+    size_t R;
+    if (m->lm_rows > 0) {
+        R = (size_t)m->lm_rows;
+    } else {
+        const size_t per_row = (size_t)m->V * dt_size(m->at) * (lm_fused(m) ? 1 : 2);
+        const size_t budget = lm_fused(m) ? ((size_t)512 << 20) : ((size_t)1024 << 20);
+        R = std::max<size_t>(128, budget / per_row / 128 * 128);
+    }
     return (int)std::min<size_t>(R, (size_t)M);
 }
 
@@ -111,8 +124,14 @@ Plan make_plan(const nc_model* m, int B, int T) {
     p.dqkv = take(A * M * m->Nqkv);
     p.Dbuf = take(4 * attn_dbuf_elems(B, T, m->H));
     p.R = lm_chunk_rows(m, p.M);
-    p.zc = take(4ull * p.R * m->V);
-    p.dlc = take(A * (size_t)p.R * m->V);
+    p.zc = take(A * (size_t)p.R * m->V);                      // logits, or u on the fused path
+    p.dlc = take(lm_fused(m) ? 0 : A * (size_t)p.R * m->V);  // their gradient (materialised path)
+    p.lm_tiles = gemm_tiles_n(m->V);
+    p.lm_stats = take(lm_fused(m) ? 4ull * p.R * p.lm_tiles : 0);
+    p.lm_zt = take(lm_fused(m) ? 4ull * p.R : 0);
+    p.lm_ut = take(lm_fused(m) ? 4ull * p.R : 0);
+    p.lm_rs = take(lm_fused(m) ? 4ull * p.R : 0);
+    p.lm_xfs = take(lm_fused(m) ? A * (size_t)p.R * d : 0);
     p.loss_rows = take(4 * M);
     p.emb = take(embed_scratch_bytes(p.M, m->V, m->d));
     size_t max_out = std::max({(size_t)p.R * d, (size_t)m->F * d, (size_t)m->H * m->hd * d, (size_t)m->Nqkv * d});
@@ -178,6 +197,15 @@ int run_gemm(const Ctx& c, const GemmDesc& g, int role) {
     return NC_OK;
 }
 
+// A GEMM whose epilogue only the tensor-core kernel implements.
+int run_gemm_tc(const Ctx& c, const GemmDesc& g, int role) {
+    Prof pr(c, role, 2.0 * g.M * g.N * (double)g.K,
+            2.0 * ((double)g.M * g.K + (double)g.N * g.K) + (g.c_t == DT_BF16 ? 2.0 : 4.0) * g.M * (double)g.N);
+    const int r = gemm_tc(g, c.ws + c.p.splitk, c.p.splitk_bytes, c.s);
+    if (r > 0) return NC_ERR_UNSUPPORTED_SHAPE;
+    return r == 0 ? NC_OK : NC_ERR_CUDA;
+}
+
 GemmDesc mk(const nc_model* m, int M, int N, int K, const void* A, int64_t lda, bool ak, const void* B,
             int64_t ldb, bool bk, Epi epi, void* C, int64_t ldc, DType ct) {
     GemmDesc g;
@@ -211,19 +239,25 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
     return NC_OK;
 }
 
-// Attention backward: dq, then dk / dv (tensor cores), or the plain-FMA kernels.
+// Attention backward: statistics and dk / dv (which also stores the dS tiles),
+// then dq from those tiles (tensor cores), or the plain-FMA kernels.
 int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv) {
     const nc_model* m = c.m;
     float* Dbuf = c.at<float>(c.p.Dbuf);
     if (m->tc && attention_tc_bwd_supported(m->hd)) {
+        void* ws = c.ws + c.p.attn_ws;
         int r;
         {
-            Prof pr(c, P_ATTN_BWD_DQ, attn_flops(c), 0.0);
-            r = attention_tc_bwd_dq(qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s);
+            Prof pr(c, P_ATTN_BWD_DKV, 2.0 * attn_flops(c), 0.0);
+            r = attention_tc_bwd_stats(o, dO, lse, Dbuf, c.p.B, c.p.T, m->H, m->hd, c.s);
+            if (r == 0)
+                r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, ws, c.p.attn_ws_bytes, c.p.B, c.p.T, m->H, m->nkv,
+                                         m->hd, m->status, c.s);
         }
         if (r == 0) {
-            Prof pr(c, P_ATTN_BWD_DKV, attn_flops(c), 0.0);
-            r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status, c.s);
+            Prof pr(c, P_ATTN_BWD_DQ, 0.5 * attn_flops(c), 0.0);
+            r = attention_tc_bwd_dq(qkv, ws, c.p.attn_ws_bytes, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status,
+                                    c.s);
         }
         if (r == 0) return NC_OK;
         if (r < 0) return NC_ERR_CUDA;
@@ -312,26 +346,57 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     // ---- LM head + softcap + cross-entropy, then its backward, R rows at a time
     void* xf = c.at(c.p.xf);
     float* gbuf = c.at<float>(c.p.g);
-    // softcapped logits in the activation type (bf16 on the mixed-precision path, as
-    // the autocast LM head of the reference produces them; fp32 on the debug path)
-    void* zc = c.at(c.p.zc);
-    void* dlc = c.at(c.p.dlc);
     float* loss_rows = c.at<float>(c.p.loss_rows);
     const size_t A = dt_size(m->at);
     float* dwlm = G(1 + 6 * m->L);
-    for (int r0 = 0; r0 < M; r0 += c.p.R) {
-        int rc = std::min(c.p.R, M - r0);
-        const char* xfc = (const char*)xf + (size_t)r0 * d * A;
-        RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, m->at), P_GEMM_LM_Z));
-        {
-            Prof pr(c, P_CE, 0.0, (double)rc * V * (2.0 * A));
-            CK(launch_ce_chunk(m->at, m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M, loss_rows + r0,
-                               dlc, m->status, s));
+    if (lm_fused(m)) {
+        // fused: the GEMM epilogue turns each logit tile into u = e (1 - (z/cap)^2),
+        // e = exp(z - cap), with per-tile sums of e; a row pass gives the loss and the
+        // row factors 1 / (S M); then dX = diag(1/(S M)) u Wlm and dWlm += u^T (xf / (S M))
+        void* uc = c.at(c.p.zc);
+        float* stats = c.at<float>(c.p.lm_stats);
+        float* zt = c.at<float>(c.p.lm_zt);
+        float* ut = c.at<float>(c.p.lm_ut);
+        float* rs = c.at<float>(c.p.lm_rs);
+        void* xfs = c.at(c.p.lm_xfs);
+        for (int r0 = 0; r0 < M; r0 += c.p.R) {
+            const int rc = std::min(c.p.R, M - r0);
+            const char* xfc = (const char*)xf + (size_t)r0 * d * A;
+            GemmDesc gz = mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_LMHEAD, uc, V, DT_BF16);
+            gz.tgt = tgt + r0; gz.stats = stats; gz.stats_ld = c.p.lm_tiles; gz.zt = zt; gz.ut = ut;
+            RG(run_gemm_tc(c, gz, P_GEMM_LM_Z));
+            {
+                Prof pr(c, P_CE, 0.0, (double)rc * (4.0 * c.p.lm_tiles + 2.0 * A * d + 16.0));
+                CK(launch_lm_rowstats(stats, c.p.lm_tiles, zt, ut, tgt + r0, rc, V, d, m->cfg.softcap,
+                                      1.0f / (float)M, uc, xfc, xfs, rs, loss_rows + r0, m->status, s));
+            }
+            GemmDesc gx = mk(m, rc, d, V, uc, V, true, w.wlm(), d, false, EPI_ROWSCALE, gbuf + (size_t)r0 * d, d,
+                             DT_F32);
+            gx.rs = rs;
+            RG(run_gemm_tc(c, gx, P_GEMM_LM_DX));
+            RG(run_gemm(c, mk(m, V, d, rc, uc, V, false, xfs, d, false, r0 == 0 ? EPI_STORE : EPI_ACCUM, dwlm, d,
+                              DT_F32), P_GEMM_LM_DW));
         }
-        RG(run_gemm(c, mk(m, rc, d, V, dlc, V, true, w.wlm(), d, false, EPI_STORE, gbuf + (size_t)r0 * d, d,
-                          DT_F32), P_GEMM_LM_DX));
-        RG(run_gemm(c, mk(m, V, d, rc, dlc, V, false, xfc, d, false, r0 == 0 ? EPI_STORE : EPI_ACCUM, dwlm, d,
-                          DT_F32), P_GEMM_LM_DW));
+    } else {
+        // materialised: softcapped logits in the activation type (bf16 on the
+        // mixed-precision path, fp32 on the debug path), then a cross-entropy pass
+        // writing dl, then dX = dl Wlm and dWlm += dl^T xf
+        void* zc = c.at(c.p.zc);
+        void* dlc = c.at(c.p.dlc);
+        for (int r0 = 0; r0 < M; r0 += c.p.R) {
+            int rc = std::min(c.p.R, M - r0);
+            const char* xfc = (const char*)xf + (size_t)r0 * d * A;
+            RG(run_gemm(c, mk(m, rc, V, d, xfc, d, true, w.wlm(), d, true, EPI_SOFTCAP, zc, V, m->at), P_GEMM_LM_Z));
+            {
+                Prof pr(c, P_CE, 0.0, (double)rc * V * (2.0 * A));
+                CK(launch_ce_chunk(m->at, m->at, zc, tgt + r0, rc, V, m->cfg.softcap, 1.0f / (float)M,
+                                   loss_rows + r0, dlc, m->status, s));
+            }
+            RG(run_gemm(c, mk(m, rc, d, V, dlc, V, true, w.wlm(), d, false, EPI_STORE, gbuf + (size_t)r0 * d, d,
+                              DT_F32), P_GEMM_LM_DX));
+            RG(run_gemm(c, mk(m, V, d, rc, dlc, V, false, xfc, d, false, r0 == 0 ? EPI_STORE : EPI_ACCUM, dwlm, d,
+                              DT_F32), P_GEMM_LM_DW));
+        }
     }
     { Prof pr(c, P_OTHER, 0.0, 4.0 * M); CK(launch_loss_reduce(loss_rows, M, loss, s)); }
     // bucket i of the gradients is final: record the caller's event, if any
@@ -444,6 +509,7 @@ int nc_model_create(const nc_config* cfg, nc_precision prec, nc_model** out) {
     m->hd = c.head_dim; m->F = c.mlp_mult * c.d_model; m->Nqkv = (c.n_head + 2 * c.n_kv_head) * c.head_dim;
     m->at = prec == NC_PREC_BF16 ? DT_BF16 : DT_F32;
     m->tc = prec == NC_PREC_BF16;
+    m->lm_mode = m->tc ? NC_LM_HEAD_FUSED : NC_LM_HEAD_MATERIALISED;
     int64_t off = 0;
     auto add = [&](const std::string& n, int r, int cc) { m->layout.push_back({n, off, r, cc}); off += (int64_t)r * cc; };
     add("wte", m->V, m->d);
@@ -602,6 +668,15 @@ int nc_debug_expired_wait(nc_model* m, int max_iters, void* stream) {
     return NC_OK;
 }
 
+int nc_set_lm_head(nc_model* m, int mode, int chunk_rows) {
+    if (!m || chunk_rows < 0) return NC_ERR_INVALID_ARG;
+    if (mode != NC_LM_HEAD_FUSED && mode != NC_LM_HEAD_MATERIALISED) return NC_ERR_INVALID_ARG;
+    if (mode == NC_LM_HEAD_FUSED && !m->tc) return NC_ERR_INVALID_ARG;
+    m->lm_mode = mode;
+    m->lm_rows = chunk_rows;
+    return NC_OK;
+}
+
 int nc_grad_bucket_count(const nc_model* m) { return m ? m->L + 2 : NC_ERR_INVALID_ARG; }
 
 int nc_grad_bucket(const nc_model* m, int i, int64_t* offset, int64_t* count) {
@@ -664,8 +739,14 @@ extern "C" int nc_test_gemm(int M, int N, int K, int in_bf16, const void* A, int
     return gemm_simt(g, s) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
+extern "C" size_t nc_test_attention_workspace_bytes(int B, int T, int H, int nkv, int hd) {
+    if (B <= 0 || T <= 0 || H <= 0 || nkv <= 0) return 0;
+    return attention_tc_workspace_bytes(B, T, H, nkv, hd);
+}
+
 extern "C" int nc_test_attention(int B, int T, int H, int nkv, int hd, const void* qkv, void* o, float* lse,
-                                 const void* dO, void* dqkv, float* Dbuf, int use_tc, int* status, void* stream) {
+                                 const void* dO, void* dqkv, float* Dbuf, void* ws, size_t ws_bytes, int use_tc,
+                                 int* status, void* stream) {
     if (B <= 0 || T <= 0 || H <= 0 || nkv <= 0 || H % nkv || !qkv || !o || !lse) return NC_ERR_INVALID_ARG;
     if (hd != 16 && hd != 32 && hd != 64 && hd != 128) return NC_ERR_UNSUPPORTED_SHAPE;
     cudaStream_t s = (cudaStream_t)stream;
@@ -674,7 +755,7 @@ extern "C" int nc_test_attention(int B, int T, int H, int nkv, int hd, const voi
         if (r != 0) return r > 0 ? NC_ERR_UNSUPPORTED_SHAPE : NC_ERR_CUDA;
         if (dO) {
             if (!dqkv || !Dbuf) return NC_ERR_INVALID_ARG;
-            r = attention_tc_bwd(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, nullptr, 0, status, s);
+            r = attention_tc_bwd(qkv, o, dO, lse, Dbuf, dqkv, B, T, H, nkv, hd, ws, ws_bytes, status, s);
             if (r != 0) return r > 0 ? NC_ERR_UNSUPPORTED_SHAPE : NC_ERR_CUDA;
         }
         return NC_OK;

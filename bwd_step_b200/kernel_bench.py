@@ -92,16 +92,18 @@ def bench_attention(iters, B=16, T=2048, H=10, nkv=1, hd=128):
     dqkv = torch.empty_like(qkv)
     Dbuf = torch.empty(2 * lse.numel(), device="cuda", dtype=torch.float32)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nws = lib().nc_test_attention_workspace_bytes(B, T, H, nkv, hd)
+    ws = torch.empty(nws, device="cuda", dtype=torch.uint8)
     stream = P(torch.cuda.current_stream().cuda_stream)
 
     def fwd():
         assert lib().nc_test_attention(B, T, H, nkv, hd, P(qkv.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
-                                       P(0), P(0), P(0), 1, P(status.data_ptr()), stream) == 0
+                                       P(0), P(0), P(0), P(0), 0, 1, P(status.data_ptr()), stream) == 0
 
     def both():
         assert lib().nc_test_attention(B, T, H, nkv, hd, P(qkv.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
-                                       P(dO.data_ptr()), P(dqkv.data_ptr()), P(Dbuf.data_ptr()), 1,
-                                       P(status.data_ptr()), stream) == 0
+                                       P(dO.data_ptr()), P(dqkv.data_ptr()), P(Dbuf.data_ptr()), P(ws.data_ptr()),
+                                       nws, 1, P(status.data_ptr()), stream) == 0
 
     flops = 4.0 * B * H * hd * T * (T + 1) / 2
     t_f = _timed(fwd, iters)

@@ -182,6 +182,24 @@ int nc_grad_bucket(const nc_model* m, int i, int64_t* offset, int64_t* count);
  * event; nothing is recorded by this call itself. */
 int nc_set_grad_events(nc_model* m, void* const* events, int n);
 
+/* LM head strategy of nc_forward_backward (both never hold the full [B*T, V]
+ * logit tensor; B*T rows are processed R at a time):
+ *   NC_LM_HEAD_FUSED (default on the bf16 path; bf16 only): the logit GEMM's
+ *     epilogue applies the softcap z = cap tanh(l/cap) and, because |z| <= cap,
+ *     writes u = exp(z - cap) (1 - (z/cap)^2) and per-tile sums of exp(z - cap)
+ *     instead of the logits; a row pass forms the loss (cap + log S - z[target])
+ *     and folds the one-hot term into u, and the two backward products read u
+ *     with a per-row factor 1 / (S B T).  The logits are never written.
+ *   NC_LM_HEAD_MATERIALISED (the fp32 debug path's only mode): the softcapped
+ *     logits of R rows are written, a cross-entropy pass reads them and writes
+ *     their gradient, and the backward products read that.
+ * chunk_rows: R (0 = the default: R V elements near 512 MiB fused, 1 GiB
+ * materialised).  Changes nc_workspace_bytes.  NC_ERR_INVALID_ARG for an
+ * unknown mode, a negative chunk_rows, or FUSED on the fp32 debug path. */
+#define NC_LM_HEAD_FUSED 0
+#define NC_LM_HEAD_MATERIALISED 1
+int nc_set_lm_head(nc_model* m, int mode, int chunk_rows);
+
 /* Weight-gradient GEMM that allocates no memory at all.
  *
  * No counterpart in the paper: this is an extra entry point of this library.

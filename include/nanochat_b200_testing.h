@@ -37,10 +37,15 @@ int nc_test_gemm(int M, int N, int K, int in_bf16, const void* A, int64_t lda, i
  * o [B*T, H*hd] and lse (natural log).  When dO != NULL also runs
  * the backward: dq, dk, dv into the matching columns of dqkv (same layout as
  * qkv), with Dbuf fp32 scratch.  lse is laid out [B, H, Tp] with Tp = T
- * rounded up to a multiple of 128; Dbuf holds 2 * B * H * Tp floats.  use_tc: 1 = tcgen05 kernels
- * (head_dim 64 or 128), 0 = plain FMA kernels. */
+ * rounded up to a multiple of 128; Dbuf holds 2 * B * H * Tp floats.  ws /
+ * ws_bytes: device scratch of the tensor-core backward (the dS tiles),
+ * nc_test_attention_workspace_bytes(B, T, H, nkv, hd) bytes (0 when the
+ * kernels need none).  use_tc: 1 = tcgen05 kernels (head_dim 64 or 128), 0 =
+ * plain FMA kernels. */
+size_t nc_test_attention_workspace_bytes(int B, int T, int H, int nkv, int hd);
 int nc_test_attention(int B, int T, int H, int nkv, int hd, const void* qkv, void* o, float* lse,
-                      const void* dO, void* dqkv, float* Dbuf, int use_tc, int* status, void* stream);
+                      const void* dO, void* dqkv, float* Dbuf, void* ws, size_t ws_bytes, int use_tc, int* status,
+                      void* stream);
 
 #ifdef __cplusplus
 }

@@ -32,9 +32,12 @@ def _run(B, T, H, nkv, hd, use_tc, seed=0, scale=1.0):
     dqkv = torch.full((B * T, Nqkv), float("nan"), dtype=torch.bfloat16, device="cuda")
     Dbuf = torch.full((2 * B * H * Tp,), float("nan"), dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nws = lib().nc_test_attention_workspace_bytes(B, T, H, nkv, hd) if use_tc else 0
+    # scratch starts as NaN bit patterns: every tile the kernels read must have been written
+    ws = torch.full((max(nws // 2, 1),), float("nan"), dtype=torch.bfloat16, device="cuda")
     r = lib().nc_test_attention(B, T, H, nkv, hd, P(qkv_d.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
-                                P(dO_d.data_ptr()), P(dqkv.data_ptr()), P(Dbuf.data_ptr()), use_tc,
-                                P(status.data_ptr()), P(torch.cuda.current_stream().cuda_stream))
+                                P(dO_d.data_ptr()), P(dqkv.data_ptr()), P(Dbuf.data_ptr()), P(ws.data_ptr()), nws,
+                                use_tc, P(status.data_ptr()), P(torch.cuda.current_stream().cuda_stream))
     assert r == 0, r
     torch.cuda.synchronize()
     assert status.item() == 0

@@ -30,12 +30,31 @@ def _case(cfg, B, T, precision, ids="uniform", seed_w=0, seed_t=1, std=0.02):
     return bits, w, tok, tgt
 
 
-def _parity(cfg, B, T, precision, **kw):
+def _parity(cfg, B, T, precision, lm_head=None, chunk_rows=0, **kw):
     bits, w, tok, tgt = _case(cfg, B, T, precision, **kw)
     ref_loss, ref_g = oracle.step(cfg, w, tok, tgt)
     m = Model(cfg.as_dict(), precision)
+    if lm_head is not None:
+        m.set_lm_head(lm_head, chunk_rows)
     loss, g = gpu_step(m, to_device_weights(bits, w, precision), tok, tgt)
     return compare(cfg, loss, g, ref_loss, ref_g, precision)
+
+
+@pytest.mark.parametrize("lm_head", ["fused", "materialised"])
+@pytest.mark.parametrize("B,T,chunk_rows,std", [(2, 32, 0, 0.02), (3, 37, 128, 0.02), (2, 200, 128, 0.3),
+                                                (1, 129, 0, 0.3)])
+def test_lm_head_modes(lm_head, B, T, chunk_rows, std):
+    # several row chunks (chunk_rows < B*T), a ragged last chunk, and weights that
+    # drive the logits into the softcap's curved range
+    _parity(_cfg(), B, T, "bf16", lm_head=lm_head, chunk_rows=chunk_rows, std=std, seed_w=B + T,
+            seed_t=7 * T)
+
+
+def test_lm_head_fused_needs_the_bf16_path():
+    m = Model(_cfg().as_dict(), "fp32")
+    with pytest.raises(NcError):
+        m.set_lm_head("fused")
+    m.set_lm_head("materialised", 256)
 
 
 @pytest.mark.parametrize("precision", ["bf16", "fp32"])

@@ -89,14 +89,17 @@ def test_attention_writes_only_its_outputs(T, hd):
     lbuf, lse = _guarded(B * H * Tp, torch.float32)
     dbuf, dq = _guarded(B * T * nq, torch.bfloat16)
     Dbb, Dbuf = _guarded(2 * B * H * Tp, torch.float32)
+    nws = lib().nc_test_attention_workspace_bytes(B, T, H, nkv, hd)
+    wbuf, ws = _guarded(nws // 2, torch.bfloat16)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     r = lib().nc_test_attention(B, T, H, nkv, hd, P(qkv.data_ptr()), P(o.data_ptr()), P(lse.data_ptr()),
-                                P(dO.data_ptr()), P(dq.data_ptr()), P(Dbuf.data_ptr()), 1,
+                                P(dO.data_ptr()), P(dq.data_ptr()), P(Dbuf.data_ptr()), P(ws.data_ptr()), nws, 1,
                                 P(status.data_ptr()), P(torch.cuda.current_stream().cuda_stream))
     assert r == 0, r
     torch.cuda.synchronize()
     assert status.item() == 0
     assert _guard_intact(obuf, B * T * H * hd) and _guard_intact(lbuf, B * H * Tp)
     assert _guard_intact(dbuf, B * T * nq) and _guard_intact(Dbb, 2 * B * H * Tp)
+    assert _guard_intact(wbuf, nws // 2)
     assert torch.isfinite(o.float()).all() and torch.isfinite(dq.float()).all()
     assert np.isfinite(lse.view(B, H, Tp)[:, :, :T].cpu().numpy()).all()
