@@ -33,6 +33,15 @@ class NcProfileRow(ctypes.Structure):
                 ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
+class NcAdamwGroup(ctypes.Structure):
+    _fields_ = [("offset", ctypes.c_int64), ("count", ctypes.c_int64), ("lr", ctypes.c_float),
+                ("beta1", ctypes.c_float), ("beta2", ctypes.c_float), ("eps", ctypes.c_float),
+                ("weight_decay", ctypes.c_float)]
+
+
+NC_ADAMW_MAX_GROUPS = 16
+
+
 class NcConfig(ctypes.Structure):
     _fields_ = [("vocab", ctypes.c_int), ("d_model", ctypes.c_int), ("n_layer", ctypes.c_int),
                 ("n_head", ctypes.c_int), ("n_kv_head", ctypes.c_int), ("head_dim", ctypes.c_int),
@@ -64,6 +73,7 @@ SIGNATURES = {
     "nc_set_grad_events": (_I, [_P, ctypes.POINTER(ctypes.c_void_p), _I]),
     "nc_debug_expired_wait": (_I, [_P, _I, _P]),
     "nc_set_lm_head": (_I, [_P, _I, _I]),
+    "nc_adamw_step": (_I, [ctypes.POINTER(NcAdamwGroup), _I, ctypes.c_int64, _I, _P, _P, _I, _P, _P, _P, _P]),
     "nc_gemm_wgrad_noalloc": (_I, [_I, _I, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _I, _P, _P]),
     # include/nanochat_b200_testing.h
     "nc_test_gemm": (_I, [_I, _I, _I, _I, _P, ctypes.c_int64, _I, _P, ctypes.c_int64, _I, _I, _P,

@@ -61,6 +61,28 @@ def _check_extents(n_params, vocab, tokens, targets=None, weights=None, grads=No
             raise ValueError(f"{name} holds {t.numel()} elements, needs {need}")
 
 
+def adamw_step(groups, step, master, weights, grads, m, v, stream=None):
+    """AdamW update of parameter groups [(offset, count, lr, beta1, beta2, eps,
+    weight_decay)] of the flat fp32 master weights (in place), the moments m and
+    v (in place) and the compute copy `weights` (bf16 or fp32); step >= 1."""
+    import torch
+    n = master.numel()
+    for name, t in (("weights", weights), ("grads", grads), ("m", m), ("v", v)):
+        if t.numel() != n:
+            raise ValueError(f"{name} holds {t.numel()} elements, master {n}")
+    dev = master.device.index
+    arr = (_lib.NcAdamwGroup * max(len(groups), 1))(
+        *[_lib.NcAdamwGroup(int(o), int(c), float(lr), float(b1), float(b2), float(e), float(wd))
+          for o, c, lr, b1, b2, e, wd in groups])
+    if weights.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("weights must be bf16 or fp32")
+    _ok(lib().nc_adamw_step(arr, len(groups), n, int(step), _ptr(master, torch.float32, "master", device=dev),
+                            _ptr(weights, None, "weights", device=dev), 1 if weights.dtype == torch.bfloat16 else 0,
+                            _ptr(grads, torch.float32, "grads", device=dev), _ptr(m, torch.float32, "m", device=dev),
+                            _ptr(v, torch.float32, "v", device=dev), ctypes.c_void_p(_stream_handle(stream))),
+        "nc_adamw_step")
+
+
 def launch_count() -> int:
     """Kernels launched by the CUDA library in this process so far."""
     return int(lib().nc_launch_count())

@@ -200,6 +200,32 @@ int nc_set_grad_events(nc_model* m, void* const* events, int n);
 #define NC_LM_HEAD_MATERIALISED 1
 int nc_set_lm_head(nc_model* m, int mode, int chunk_rows);
 
+/* AdamW update of (ranges of) the flat parameter vector, the optimizer the
+ * announcement names beside Muon (vpshk.cn, optimizer paragraph: Muon +
+ * AdamW, with a plan to use Adam alone with a learning rate per module).  Muon
+ * is not defined on the pages and is not provided.  Textbook AdamW (Adam,
+ * Kingma & Ba 2015, with decoupled weight decay, Loshchilov & Hutter 2019);
+ * for every element of each group, with t = step (1 for the first update):
+ *   m <- b1 m + (1 - b1) g;   v <- b2 v + (1 - b2) g^2
+ *   theta <- theta - lr (wd theta + (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps))
+ *   weights <- theta in the step's type (bf16 rounded to nearest even, or fp32)
+ * groups: n_groups (1..NC_ADAMW_MAX_GROUPS) host descriptors of disjoint
+ *   element ranges [offset, offset + count) of the flat layout, each with its
+ *   own hyper-parameters (0 <= beta < 1, eps > 0, lr >= 0, weight_decay >= 0).
+ * master, grads, m, v: device fp32 [n_params]; weights: device [n_params],
+ *   bf16 when weights_bf16 != 0, else fp32.  All five 16-byte aligned; m and v
+ *   start at zero before step 1 (the caller clears them).  Elements outside
+ *   every group are not touched.
+ * One kernel on `stream`.  NC_ERR_INVALID_ARG for a null or misaligned
+ * pointer, step < 1, a range outside [0, n_params) or a bad hyper-parameter. */
+#define NC_ADAMW_MAX_GROUPS 16
+typedef struct {
+    int64_t offset, count;
+    float lr, beta1, beta2, eps, weight_decay;
+} nc_adamw_group;
+int nc_adamw_step(const nc_adamw_group* groups, int n_groups, int64_t n_params, int step, float* master,
+                  void* weights, int weights_bf16, const float* grads, float* m, float* v, void* stream);
+
 /* Weight-gradient GEMM that allocates no memory at all.
  *
  * No counterpart in the paper: this is an extra entry point of this library.

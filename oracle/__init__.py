@@ -6,7 +6,8 @@ baseline may import it.  The product path never touches it.
 from .model import (RMS_EPS, layout, views, rmsnorm, rmsnorm_backward, rope_tables, rope,
                     rope_backward, attention, attention_backward, softcap, lm_head_loss,
                     step, position_losses, forward_logits)
+from .optim import adamw_step
 
 __all__ = ["RMS_EPS", "layout", "views", "rmsnorm", "rmsnorm_backward", "rope_tables", "rope",
            "rope_backward", "attention", "attention_backward", "softcap", "lm_head_loss",
-           "step", "position_losses", "forward_logits"]
+           "step", "position_losses", "forward_logits", "adamw_step"]
