@@ -73,6 +73,10 @@ SIGNATURES = {
     "nc_set_grad_events": (_I, [_P, ctypes.POINTER(ctypes.c_void_p), _I]),
     "nc_debug_expired_wait": (_I, [_P, _I, _P]),
     "nc_set_lm_head": (_I, [_P, _I, _I]),
+    "nc_kv_cache_bytes": (_SZ, [_P, _I, _I]),
+    "nc_inference_workspace_bytes": (_SZ, [_P, _I, _I]),
+    "nc_prefill": (_I, [_P, _P, _I, _I, _P, _P, _I, _P, _P, _SZ, _P]),
+    "nc_decode_step": (_I, [_P, _P, _I, _I, _P, _P, _I, _P, _P, _SZ, _P]),
     "nc_adamw_step": (_I, [ctypes.POINTER(NcAdamwGroup), _I, ctypes.c_int64, _I, _P, _P, _I, _P, _P, _P, _P]),
     "nc_gemm_wgrad_noalloc": (_I, [_I, _I, _I, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _I, _P, _P]),
     # include/nanochat_b200_testing.h

@@ -183,6 +183,47 @@ class Model:
                                     workspace.numel() * workspace.element_size(),
                                     ctypes.c_void_p(_stream_handle(stream))), "nc_forward_logits")
 
+    def kv_cache_bytes(self, B: int, T_max: int) -> int:
+        return int(lib().nc_kv_cache_bytes(self._h, B, T_max))
+
+    def inference_workspace_bytes(self, B: int, T_max: int) -> int:
+        return int(lib().nc_inference_workspace_bytes(self._h, B, T_max))
+
+    def prefill(self, tokens, weights, kv_cache, T_max, logits, workspace, stream=None):
+        """Forward over the prompt tokens [B, T] (device int32); fills cache
+        positions 0..T-1 and writes the last position's softcapped logits [B, V]."""
+        import torch
+        B, T = tokens.shape
+        self._check_inference(B, T_max, weights, kv_cache, logits)
+        _ok(lib().nc_prefill(self._h, self._dev(tokens, torch.int32, "tokens"), B, T,
+                             self._dev(weights, self.weight_dtype, "weights"), self._dev(kv_cache, None, "kv_cache"),
+                             int(T_max), self._dev(logits, self.weight_dtype, "logits"),
+                             self._dev(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+                             ctypes.c_void_p(_stream_handle(stream))), "nc_prefill")
+
+    def decode_step(self, tokens, pos, weights, kv_cache, T_max, logits, workspace, stream=None):
+        """One new token per row (device int32 [B]) at position pos: appends to
+        the cache and writes that position's softcapped logits [B, V]."""
+        import torch
+        B = tokens.shape[0]
+        if tokens.dim() != 1:
+            raise ValueError("tokens must be [B]")
+        self._check_inference(B, T_max, weights, kv_cache, logits)
+        _ok(lib().nc_decode_step(self._h, self._dev(tokens, torch.int32, "tokens"), B, int(pos),
+                                 self._dev(weights, self.weight_dtype, "weights"),
+                                 self._dev(kv_cache, None, "kv_cache"), int(T_max),
+                                 self._dev(logits, self.weight_dtype, "logits"),
+                                 self._dev(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+                                 ctypes.c_void_p(_stream_handle(stream))), "nc_decode_step")
+
+    def _check_inference(self, B, T_max, weights, kv_cache, logits):
+        if weights.numel() < self.num_params():
+            raise ValueError("weights shorter than the flat layout")
+        if kv_cache.numel() * kv_cache.element_size() < self.kv_cache_bytes(B, T_max):
+            raise ValueError("kv_cache smaller than kv_cache_bytes(B, T_max)")
+        if logits.numel() < B * self.cfg.vocab:
+            raise ValueError("logits must hold [B, V]")
+
     def set_lm_head(self, mode: str = "fused", chunk_rows: int = 0):
         """LM head strategy: "fused" (logits never stored; bf16 only) or
         "materialised" (logit chunks plus a cross-entropy pass); chunk_rows 0 =

@@ -16,8 +16,8 @@ enum DType : int { DT_F32 = 0, DT_BF16 = 1 };
 inline size_t dt_size(DType t) { return t == DT_BF16 ? 2 : 4; }
 
 // ---------------------------------------------------------------- memory-bound
-// cos/sin [T, hd/2] of pos * base^(-2j/hd), evaluated in double.
-cudaError_t launch_rope_table(float* cos_t, float* sin_t, int T, int hd, float base, cudaStream_t s);
+// cos/sin [T, hd/2] of pos * base^(-2j/hd) for pos = pos0 .. pos0 + T - 1, evaluated in double.
+cudaError_t launch_rope_table(float* cos_t, float* sin_t, int T, int hd, float base, cudaStream_t s, int pos0 = 0);
 
 // x[m] = rmsnorm(wte[idx[m]]) (fp32 residual stream), r0[m] = its inverse RMS.
 cudaError_t launch_embed_norm_fwd(DType wt, const int32_t* idx, const void* wte, int M, int V, int d,
@@ -49,6 +49,15 @@ cudaError_t launch_ce_chunk(DType zt, DType dlt, const void* z, const int32_t* t
 cudaError_t launch_lm_rowstats(const float* stats, int ntiles, const float* zt, const float* ut,
                                const int32_t* tgt, int R, int V, int d, float cap, float inv_M, void* u,
                                const void* xf, void* xfs, float* rs, float* loss_rows, int* status, cudaStream_t s);
+// Inference KV cache, K and V each [B, T_max, nkv, hd] in the activation type:
+// copies the k, v heads of `rows` qkv rows (batch row r / rows_per_b, position
+// pos0 + r % rows_per_b) into it.
+cudaError_t launch_kv_append(DType at, const void* qkv, int H, int nkv, int hd, int rows, int rows_per_b,
+                             int pos0, void* kc, void* vc, int T_max, cudaStream_t s);
+// o[b, h] = softmax(q_bh . K[b, 0..len)^T / sqrt(hd)) V[b, 0..len) for the one
+// query per row in qkv rows [B, (H+2nkv) hd] (kv head h / (H / nkv)).
+cudaError_t launch_decode_attention(DType at, const void* qkv, const void* kc, const void* vc, int T_max, int len,
+                                    int B, int H, int nkv, int hd, void* o, cudaStream_t s);
 // loss = mean(loss_rows[0..M)), fixed summation order.
 cudaError_t launch_loss_reduce(const float* loss_rows, int M, float* loss, cudaStream_t s);
 

@@ -26,11 +26,11 @@ constexpr int kRowWarps = 8;  // rows per 256-thread block
 inline int row_blocks(int M) { return (M + kRowWarps - 1) / kRowWarps; }
 
 // ---------------------------------------------------------------- RoPE table
-__global__ void rope_table_kernel(float* c, float* s, int T, int hd, double base) {
+__global__ void rope_table_kernel(float* c, float* s, int T, int hd, double base, int pos0) {
     int half = hd / 2;
     int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= T * half) return;
-    int pos = i / half, j = i % half;
+    int pos = pos0 + i / half, j = i % half;
     double theta = pow(base, -2.0 * (double)j / (double)hd);
     double ang = (double)pos * theta;
     c[i] = (float)cos(ang);
@@ -675,6 +675,91 @@ __global__ void loss_reduce_kernel(const float* __restrict__ rows, int M, float*
     if (threadIdx.x == 0) *loss = sh[0] / (float)M;
 }
 
+// ---------------------------------------------------------------- KV cache (inference)
+// Copies the k and v heads of `rows` fused qkv rows (row r = batch row
+// r / rows_per_b, position pos0 + r % rows_per_b) into the cache, one 16-byte
+// vector per thread.  Cache: K and V each [B, T_max, nkv, hd].
+template <typename A>
+__global__ void kv_append_kernel(const A* __restrict__ qkv, int H, int nkv, int hd, int rows, int rows_per_b,
+                                 int pos0, A* __restrict__ kc, A* __restrict__ vc, int T_max) {
+    constexpr int VEC = Vec<A>::N;
+    const int per_row = 2 * nkv * hd / VEC;  // vectors of k then v
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)rows * per_row) return;
+    const int r = (int)(i / per_row), e = (int)(i % per_row) * VEC;
+    const int b = r / rows_per_b, t = pos0 + r % rows_per_b;
+    const size_t Nqkv = (size_t)(H + 2 * nkv) * hd;
+    const A* src = qkv + (size_t)r * Nqkv + (size_t)H * hd + e;
+    const int kvn = nkv * hd;
+    A* dst = (e < kvn ? kc : vc) + ((size_t)b * T_max + t) * kvn + (e < kvn ? e : e - kvn);
+    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+}
+
+// One query per (batch row, head) against the cached positions 0..len-1 (all
+// visible: the query is the newest position).  Four warps split the
+// positions; each keeps an online softmax in the log2 domain (running max,
+// sum, and its share of the output, HD/32 dims per lane), and the four are
+// combined at the end.  Scores scaled by 1/sqrt(hd).
+template <typename A, int HD>
+__global__ void __launch_bounds__(128) decode_attention_kernel(const A* __restrict__ qkv, const A* __restrict__ kc,
+                                                               const A* __restrict__ vc, int T_max, int len, int H,
+                                                               int nkv, float scale_log2, A* __restrict__ o) {
+    constexpr int EPL = HD >= 32 ? HD / 32 : 1;  // dims per lane
+    constexpr int LANES = HD / EPL;              // lanes holding dims
+    __shared__ float sm[4], sl[4], so[4][HD];
+    const int b = blockIdx.x, h = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = h / (H / nkv);
+    const bool act = lane < LANES;
+    const int c0 = (act ? lane : 0) * EPL;
+    const size_t Nqkv = (size_t)(H + 2 * nkv) * HD;
+    float q[EPL], acc[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        q[i] = act ? tof(qkv[(size_t)b * Nqkv + (size_t)h * HD + c0 + i]) * scale_log2 : 0.f;
+        acc[i] = 0.f;
+    }
+    float m = -INFINITY, l = 0.f;
+    const A* kb = kc + ((size_t)b * T_max * nkv + g) * HD;
+    const A* vb = vc + ((size_t)b * T_max * nkv + g) * HD;
+    for (int j = warp; j < len; j += 4) {
+        const A* kr = kb + (size_t)j * nkv * HD + c0;
+        const A* vr = vb + (size_t)j * nkv * HD + c0;
+        float sdot = 0.f, vv[EPL];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            sdot += act ? q[i] * tof(kr[i]) : 0.f;
+            vv[i] = act ? tof(vr[i]) : 0.f;
+        }
+        const float sc = warp_sum(sdot);
+        const float mn = fmaxf(m, sc);
+        const float alpha = exp2f(m - mn), pj = exp2f(sc - mn);
+        l = l * alpha + pj;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) acc[i] = acc[i] * alpha + pj * vv[i];
+        m = mn;
+    }
+    if (lane == 0) { sm[warp] = m; sl[warp] = l; }
+    if (act) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) so[warp][c0 + i] = acc[i];
+    }
+    __syncthreads();
+    const float M = fmaxf(fmaxf(sm[0], sm[1]), fmaxf(sm[2], sm[3]));
+    float wsc[4], L = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        wsc[w] = sm[w] == -INFINITY ? 0.f : exp2f(sm[w] - M);  // a warp without positions adds nothing
+        L += sl[w] * wsc[w];
+    }
+    for (int c = threadIdx.x; c < HD; c += blockDim.x) {
+        float r = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) r += so[w][c] * wsc[w];
+        o[(size_t)b * H * HD + (size_t)h * HD + c] = fromf<A>(r / L);
+    }
+}
+
 // ---------------------------------------------------------------- embedding scatter
 // dWte[v] = sum of de[m] over the positions m with idx[m] == v, in increasing m.
 // Positions are bucketed by id (counting sort, then a canonical in-bucket
@@ -880,9 +965,9 @@ __global__ void expired_wait_kernel(int* status, int max_iters) {
 std::atomic<long long> g_launches{0};
 
 // ============================================================================ launchers
-cudaError_t launch_rope_table(float* c, float* s, int T, int hd, float base, cudaStream_t st) {
+cudaError_t launch_rope_table(float* c, float* s, int T, int hd, float base, cudaStream_t st, int pos0) {
     int n = T * (hd / 2);
-    rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(c, s, T, hd, (double)base);
+    rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(c, s, T, hd, (double)base, pos0);
     count_launch();
     return cudaGetLastError();
 }
@@ -1052,6 +1137,49 @@ cudaError_t launch_ce_chunk(DType zt, DType dlt, const void* z, const int32_t* t
 #undef NC_CE
     count_launch();
     return cudaGetLastError();
+}
+
+cudaError_t launch_kv_append(DType at, const void* qkv, int H, int nkv, int hd, int rows, int rows_per_b,
+                             int pos0, void* kc, void* vc, int T_max, cudaStream_t s) {
+    const int vec = at == DT_BF16 ? 8 : 4;
+    const long long n = (long long)rows * (2 * nkv * hd / vec);
+    const unsigned blocks = (unsigned)((n + 255) / 256);
+    if (at == DT_BF16)
+        kv_append_kernel<bf16><<<blocks, 256, 0, s>>>(reinterpret_cast<const bf16*>(qkv), H, nkv, hd, rows, rows_per_b,
+                                                      pos0, reinterpret_cast<bf16*>(kc), reinterpret_cast<bf16*>(vc),
+                                                      T_max);
+    else
+        kv_append_kernel<float><<<blocks, 256, 0, s>>>(reinterpret_cast<const float*>(qkv), H, nkv, hd, rows,
+                                                       rows_per_b, pos0, reinterpret_cast<float*>(kc),
+                                                       reinterpret_cast<float*>(vc), T_max);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <typename A>
+static cudaError_t decode_attention_t(const void* qkv, const void* kc, const void* vc, int T_max, int len, int B,
+                                      int H, int nkv, int hd, void* o, cudaStream_t s) {
+    const float sl = 1.44269504088896340736f / sqrtf((float)hd);
+    const dim3 grid(B, H);
+    const A* q = reinterpret_cast<const A*>(qkv);
+    const A* k = reinterpret_cast<const A*>(kc);
+    const A* v = reinterpret_cast<const A*>(vc);
+    A* out = reinterpret_cast<A*>(o);
+    switch (hd) {
+        case 16: decode_attention_kernel<A, 16><<<grid, 128, 0, s>>>(q, k, v, T_max, len, H, nkv, sl, out); break;
+        case 32: decode_attention_kernel<A, 32><<<grid, 128, 0, s>>>(q, k, v, T_max, len, H, nkv, sl, out); break;
+        case 64: decode_attention_kernel<A, 64><<<grid, 128, 0, s>>>(q, k, v, T_max, len, H, nkv, sl, out); break;
+        case 128: decode_attention_kernel<A, 128><<<grid, 128, 0, s>>>(q, k, v, T_max, len, H, nkv, sl, out); break;
+        default: return cudaErrorInvalidValue;
+    }
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_attention(DType at, const void* qkv, const void* kc, const void* vc, int T_max, int len,
+                                    int B, int H, int nkv, int hd, void* o, cudaStream_t s) {
+    return at == DT_BF16 ? decode_attention_t<bf16>(qkv, kc, vc, T_max, len, B, H, nkv, hd, o, s)
+                         : decode_attention_t<float>(qkv, kc, vc, T_max, len, B, H, nkv, hd, o, s);
 }
 
 cudaError_t launch_lm_rowstats(const float* stats, int ntiles, const float* zt, const float* ut,

@@ -87,20 +87,23 @@ int lm_chunk_rows(const nc_model* m, int M) {
     return (int)std::min<size_t>(R, (size_t)M);
 }
 
-Plan make_plan(const nc_model* m, int B, int T) {
+// Workspace layout for (B, T).  fwd_only: the forward alone (logits, inference
+// prefill): one reused layer slot and none of the backward's buffers.
+Plan make_plan(const nc_model* m, int B, int T, bool fwd_only = false) {
     Plan p;
     p.B = B; p.T = T; p.M = B * T;
     const size_t M = p.M, d = m->d, A = dt_size(m->at);
+    const bool bwd = !fwd_only;
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off += al256(bytes); return o; };
     p.tok = take(4 * M);
-    p.tgt = take(4 * M);
+    p.tgt = take(bwd ? 4 * M : 0);
     p.cosb = take(4ull * T * (m->hd / 2));
     p.sinb = take(4ull * T * (m->hd / 2));
     p.x = take(4 * M * d);
-    p.dx = take(4 * M * d);
-    p.g = take(4 * M * d);
-    p.dxb = take(A * M * d);
+    p.dx = take(bwd ? 4 * M * d : 0);
+    p.g = take(bwd ? 4 * M * d : 0);
+    p.dxb = take(bwd ? A * M * d : 0);
     p.xf = take(A * M * d);
     p.r0 = take(4 * M);
     p.rf = take(4 * M);
@@ -118,26 +121,28 @@ Plan make_plan(const nc_model* m, int B, int T) {
     p.l_ru = ltake(A * M * m->F);
     p.l_h = ltake(A * M * m->F);
     p.lay_stride = lo;
-    p.layers = take(lo * m->L);
-    p.du = take(A * M * m->F);
-    p.dO = take(A * M * m->H * m->hd);
-    p.dqkv = take(A * M * m->Nqkv);
-    p.Dbuf = take(4 * attn_dbuf_elems(B, T, m->H));
+    p.layers = take(lo * (bwd ? m->L : 1));
+    p.du = take(bwd ? A * M * m->F : 0);
+    p.dO = take(bwd ? A * M * m->H * m->hd : 0);
+    p.dqkv = take(bwd ? A * M * m->Nqkv : 0);
+    p.Dbuf = take(bwd ? 4 * attn_dbuf_elems(B, T, m->H) : 0);
     p.R = lm_chunk_rows(m, p.M);
-    p.zc = take(A * (size_t)p.R * m->V);                      // logits, or u on the fused path
-    p.dlc = take(lm_fused(m) ? 0 : A * (size_t)p.R * m->V);  // their gradient (materialised path)
+    const bool fz = bwd && lm_fused(m);
+    p.zc = take(bwd ? A * (size_t)p.R * m->V : 0);                     // logits, or u on the fused path
+    p.dlc = take(bwd && !lm_fused(m) ? A * (size_t)p.R * m->V : 0);   // their gradient (materialised path)
     p.lm_tiles = gemm_tiles_n(m->V);
-    p.lm_stats = take(lm_fused(m) ? 4ull * p.R * p.lm_tiles : 0);
-    p.lm_zt = take(lm_fused(m) ? 4ull * p.R : 0);
-    p.lm_ut = take(lm_fused(m) ? 4ull * p.R : 0);
-    p.lm_rs = take(lm_fused(m) ? 4ull * p.R : 0);
-    p.lm_xfs = take(lm_fused(m) ? A * (size_t)p.R * d : 0);
-    p.loss_rows = take(4 * M);
-    p.emb = take(embed_scratch_bytes(p.M, m->V, m->d));
-    size_t max_out = std::max({(size_t)p.R * d, (size_t)m->F * d, (size_t)m->H * m->hd * d, (size_t)m->Nqkv * d});
+    p.lm_stats = take(fz ? 4ull * p.R * p.lm_tiles : 0);
+    p.lm_zt = take(fz ? 4ull * p.R : 0);
+    p.lm_ut = take(fz ? 4ull * p.R : 0);
+    p.lm_rs = take(fz ? 4ull * p.R : 0);
+    p.lm_xfs = take(fz ? A * (size_t)p.R * d : 0);
+    p.loss_rows = take(bwd ? 4 * M : 0);
+    p.emb = take(bwd ? embed_scratch_bytes(p.M, m->V, m->d) : 0);
+    size_t max_out = std::max({(size_t)m->F * d, (size_t)m->H * m->hd * d, (size_t)m->Nqkv * d});
+    max_out = std::max(max_out, bwd ? (size_t)p.R * d : std::min(M * d, (size_t)1 << 22));
     p.splitk_bytes = m->tc ? gemm_tc_splitk_bytes(max_out) : 0;
     p.splitk = take(p.splitk_bytes);
-    p.attn_ws_bytes = m->tc ? attention_tc_workspace_bytes(B, T, m->H, m->nkv, m->hd) : 0;
+    p.attn_ws_bytes = m->tc && bwd ? attention_tc_workspace_bytes(B, T, m->H, m->nkv, m->hd) : 0;
     p.attn_ws = take(p.attn_ws_bytes);
     p.total = off;
     return p;
@@ -278,17 +283,33 @@ struct W {  // weight pointers of one call
     const void* wlm() const { return p(1 + 6 * m->L); }
 };
 
+// Inference KV cache of one call: K and V [n_layer][B, T_max, nkv, hd] each
+// (activation type).  Prefill writes positions 0..T-1; a decode step (one
+// token per row, T = 1 in the plan) writes position pos and attends to 0..pos.
+struct KvCache {
+    char* base;
+    int T_max, pos;
+    bool decode;
+    size_t layer_bytes;  // K + V of one layer
+    void* k(int l) const { return base + (size_t)l * layer_bytes; }
+    void* v(int l) const { return base + (size_t)l * layer_bytes + layer_bytes / 2; }
+};
+
 // Forward through the blocks; with `save` every layer keeps its own
-// activations for the backward, otherwise layer slot 0 is reused.
-int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save) {
+// activations for the backward, otherwise layer slot 0 is reused.  With `kv`
+// the k, v heads of every layer go to the inference cache, and in a decode
+// step the attention reads the cache instead of the call's own positions.
+int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save, const KvCache* kv = nullptr) {
     nc_model* m = c.m;
     const int M = c.p.M, d = m->d;
     float* x = c.at<float>(c.p.x);
     const float* cs = c.at<float>(c.p.cosb);
     const float* sn = c.at<float>(c.p.sinb);
+    const bool decode = kv && kv->decode;
     {
         Prof pr(c, P_OTHER, 0.0, 8.0 * c.p.T * (m->hd / 2));
-        CK(launch_rope_table(c.at<float>(c.p.cosb), c.at<float>(c.p.sinb), c.p.T, m->hd, m->cfg.rope_base, c.s));
+        CK(launch_rope_table(c.at<float>(c.p.cosb), c.at<float>(c.p.sinb), c.p.T, m->hd, m->cfg.rope_base, c.s,
+                             decode ? kv->pos : 0));
     }
     const double A = (double)dt_size(m->at);
     { Prof pr(c, P_EMBED_FWD, 0.0, (double)M * (A * d + 4.0 * d + 8.0)); CK(launch_embed_norm_fwd(m->at, tok, w.wte(), M, m->V, d, x, c.at<float>(c.p.r0), m->status, c.s)); }
@@ -322,7 +343,18 @@ int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save) {
             Prof pr(c, P_QKROPE_FWD, 0.0, (double)M * (m->H + m->nkv) * (2.0 * A * m->hd + 4.0));
             CK(launch_qknorm_rope_fwd(m->at, qkv, rqk, cs, sn, M, c.p.T, m->H, m->nkv, m->hd, c.s));
         }
-        RG(attention_fwd(c, qkv, o, (float*)(lb + c.p.l_lse)));
+        if (kv) {
+            Prof pr(c, P_OTHER, 0.0, 4.0 * A * M * m->nkv * m->hd);
+            CK(launch_kv_append(m->at, qkv, m->H, m->nkv, m->hd, M, c.p.T, decode ? kv->pos : 0, kv->k(l), kv->v(l),
+                                kv->T_max, c.s));
+        }
+        if (decode) {
+            Prof pr(c, P_ATTN_FWD, 4.0 * M * m->H * (double)m->hd * (kv->pos + 1), 0.0);
+            CK(launch_decode_attention(m->at, qkv, kv->k(l), kv->v(l), kv->T_max, kv->pos + 1, c.p.B, m->H, m->nkv,
+                                       m->hd, o, c.s));
+        } else {
+            RG(attention_fwd(c, qkv, o, (float*)(lb + c.p.l_lse)));
+        }
         RG(run_gemm(c, mk(m, M, d, (int)Hhd, o, Hhd, true, w.wo(l), Hhd, true, EPI_ACCUM, x, d, DT_F32), P_GEMM_FWD));
         { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, mm, (float*)(lb + c.p.l_r2), M, d, c.s)); }
         GemmDesc fc = mk(m, M, m->F, d, mm, d, true, w.wfc(l), d, true, EPI_RELU2, h, m->F, m->at);
@@ -467,13 +499,14 @@ bool on_model_device(const nc_model* m) {
     return cudaGetDevice(&dev) == cudaSuccess && dev == m->device;
 }
 
-int validate_call(nc_model* m, int B, int T, size_t ws_bytes, const void* const* ptrs, int nptr) {
+int validate_call(nc_model* m, int B, int T, size_t ws_bytes, const void* const* ptrs, int nptr,
+                  bool fwd_only = false) {
     if (!m || B <= 0 || T <= 0) return NC_ERR_INVALID_ARG;
     if (!on_model_device(m)) return NC_ERR_INVALID_ARG;
     if ((long long)B * T > (1 << 24)) return NC_ERR_UNSUPPORTED_SHAPE;
     for (int i = 0; i < nptr; ++i)
         if (!ptrs[i]) return NC_ERR_INVALID_ARG;
-    if (ws_bytes < make_plan(m, B, T).total) return NC_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_bytes < make_plan(m, B, T, fwd_only).total) return NC_ERR_WORKSPACE_TOO_SMALL;
     return NC_OK;
 }
 
@@ -594,13 +627,55 @@ int nc_forward_backward_host(nc_model* m, const int32_t* h_tokens, const int32_t
 int nc_forward_logits(nc_model* m, const int32_t* tokens, int B, int T, const void* weights, void* logits,
                       void* workspace, size_t ws_bytes, void* stream) {
     const void* ptrs[] = {tokens, weights, logits, workspace};
-    int v = validate_call(m, B, T, ws_bytes, ptrs, 4);
+    int v = validate_call(m, B, T, ws_bytes, ptrs, 4, true);
     if (v != NC_OK) return v;
-    Ctx c{m, make_plan(m, B, T), (char*)workspace, (cudaStream_t)stream};
+    Ctx c{m, make_plan(m, B, T, true), (char*)workspace, (cudaStream_t)stream};
     W w{(const char*)weights, dt_size(m->at), m};
     RG(forward_blocks(c, w, tokens, false));
     RG(run_gemm(c, mk(m, c.p.M, m->V, m->d, c.at(c.p.xf), m->d, true, w.wlm(), m->d, true, EPI_SOFTCAP, logits,
                       m->V, m->at), P_GEMM_LM_Z));
+    return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+size_t nc_kv_cache_bytes(const nc_model* m, int B, int T_max) {
+    if (!m || B <= 0 || T_max <= 0) return 0;
+    return (size_t)m->L * 2 * B * (size_t)T_max * m->nkv * m->hd * dt_size(m->at);
+}
+
+size_t nc_inference_workspace_bytes(const nc_model* m, int B, int T_max) {
+    if (!m || B <= 0 || T_max <= 0 || (long long)B * T_max > (1 << 24)) return 0;
+    return std::max(make_plan(m, B, T_max, true).total, make_plan(m, B, 1, true).total);
+}
+
+int nc_prefill(nc_model* m, const int32_t* tokens, int B, int T, const void* weights, void* kv_cache, int T_max,
+               void* logits, void* workspace, size_t ws_bytes, void* stream) {
+    const void* ptrs[] = {tokens, weights, kv_cache, logits, workspace};
+    if (T_max < T) return NC_ERR_INVALID_ARG;
+    int v = validate_call(m, B, T, ws_bytes, ptrs, 5, true);
+    if (v != NC_OK) return v;
+    Ctx c{m, make_plan(m, B, T, true), (char*)workspace, (cudaStream_t)stream};
+    W w{(const char*)weights, dt_size(m->at), m};
+    const KvCache kv{(char*)kv_cache, T_max, 0, false, nc_kv_cache_bytes(m, B, T_max) / m->L};
+    RG(forward_blocks(c, w, tokens, false, &kv));
+    // logits of the last position of every row: rows b*T + T-1 of xf (row stride T*d)
+    const char* last = (const char*)c.at(c.p.xf) + (size_t)(T - 1) * m->d * dt_size(m->at);
+    RG(run_gemm(c, mk(m, B, m->V, m->d, last, (int64_t)T * m->d, true, w.wlm(), m->d, true, EPI_SOFTCAP, logits,
+                      m->V, m->at), P_GEMM_LM_Z));
+    return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+int nc_decode_step(nc_model* m, const int32_t* tokens, int B, int pos, const void* weights, void* kv_cache,
+                   int T_max, void* logits, void* workspace, size_t ws_bytes, void* stream) {
+    const void* ptrs[] = {tokens, weights, kv_cache, logits, workspace};
+    if (pos < 0 || pos >= T_max) return NC_ERR_INVALID_ARG;
+    int v = validate_call(m, B, 1, ws_bytes, ptrs, 5, true);
+    if (v != NC_OK) return v;
+    Ctx c{m, make_plan(m, B, 1, true), (char*)workspace, (cudaStream_t)stream};
+    W w{(const char*)weights, dt_size(m->at), m};
+    const KvCache kv{(char*)kv_cache, T_max, pos, true, nc_kv_cache_bytes(m, B, T_max) / m->L};
+    RG(forward_blocks(c, w, tokens, false, &kv));
+    RG(run_gemm(c, mk(m, B, m->V, m->d, c.at(c.p.xf), m->d, true, w.wlm(), m->d, true, EPI_SOFTCAP, logits, m->V,
+                      m->at), P_GEMM_LM_Z));
     return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

@@ -128,7 +128,9 @@ int nc_forward_backward_host(nc_model* m, const int32_t* h_tokens, const int32_t
 
 /* Forward pass only; writes the softcapped logits z [B, T, V] (bf16 for
  * NC_PREC_BF16, fp32 for NC_PREC_FP32_DEBUG) to the device buffer `logits`.
- * This is the only call that materialises logits. */
+ * This is the only call that materialises the logits of every position.  It
+ * needs only nc_inference_workspace_bytes(m, B, T) bytes of workspace (the
+ * forward alone); nc_workspace_bytes(m, B, T) is more than enough. */
 int nc_forward_logits(nc_model* m, const int32_t* tokens, int B, int T, const void* weights,
                       void* logits, void* workspace, size_t ws_bytes, void* stream);
 
@@ -181,6 +183,31 @@ int nc_grad_bucket(const nc_model* m, int i, int64_t* offset, int64_t* count);
  * valid while set.  NC_ERR_INVALID_ARG for a null handle, a wrong n or a null
  * event; nothing is recorded by this call itself. */
 int nc_set_grad_events(nc_model* m, void* const* events, int n);
+
+/* Inference with a KV cache (the nanochat pipeline's inference engine with
+ * prefill and decode, tianqi.csdn.net pipeline paragraph).  Multi-query
+ * attention keeps one K and one V head per K/V group: the cache is
+ * [n_layer] x {K, V} x [B, T_max, n_kv_head, head_dim] in the weights' type
+ * (K after QK-norm and RoPE), nc_kv_cache_bytes(m, B, T_max) bytes of device
+ * memory owned by the caller, passed unchanged from the prefill to every
+ * decode step of the same B rows.
+ *   nc_inference_workspace_bytes: workspace for nc_prefill with any T <= T_max
+ *     and for nc_decode_step (0 for bad sizes).
+ *   nc_prefill: the forward over tokens [B, T] (device int32, every row T
+ *     long), cache positions 0..T-1 written, softcapped logits of position T-1
+ *     of every row into logits [B, V] (weights' type).
+ *   nc_decode_step: one new token per row, tokens [B] (device int32), at
+ *     position pos (the number of positions already cached, same for every
+ *     row; pos < T_max): writes that position's k, v into the cache and the
+ *     softcapped logits [B, V] of the new position, attending to 0..pos.
+ * Errors as nc_forward_logits, plus NC_ERR_INVALID_ARG for T > T_max or pos
+ * outside [0, T_max).  Both only enqueue on `stream`. */
+size_t nc_kv_cache_bytes(const nc_model* m, int B, int T_max);
+size_t nc_inference_workspace_bytes(const nc_model* m, int B, int T_max);
+int nc_prefill(nc_model* m, const int32_t* tokens, int B, int T, const void* weights, void* kv_cache, int T_max,
+               void* logits, void* workspace, size_t ws_bytes, void* stream);
+int nc_decode_step(nc_model* m, const int32_t* tokens, int B, int pos, const void* weights, void* kv_cache,
+                   int T_max, void* logits, void* workspace, size_t ws_bytes, void* stream);
 
 /* LM head strategy of nc_forward_backward (both never hold the full [B*T, V]
  * logit tensor; B*T rows are processed R at a time):

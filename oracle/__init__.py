@@ -7,7 +7,9 @@ from .model import (RMS_EPS, layout, views, rmsnorm, rmsnorm_backward, rope_tabl
                     rope_backward, attention, attention_backward, softcap, lm_head_loss,
                     step, position_losses, forward_logits)
 from .optim import adamw_step
+from .decode import prefill, decode_step
 
 __all__ = ["RMS_EPS", "layout", "views", "rmsnorm", "rmsnorm_backward", "rope_tables", "rope",
            "rope_backward", "attention", "attention_backward", "softcap", "lm_head_loss",
-           "step", "position_losses", "forward_logits", "adamw_step"]
+           "step", "position_losses", "forward_logits", "adamw_step",
+           "prefill", "decode_step"]
