@@ -21,6 +21,9 @@ NC_ERR_BAD_TOKEN = -5
 NC_ERR_DEVICE_TIMEOUT = -6
 NC_ERR_NO_DEVICE = -7
 
+NC_RECOMPUTE_NONE = 0
+NC_RECOMPUTE_MLP = 1
+
 NC_LM_HEAD_FUSED = 0
 NC_LM_HEAD_MATERIALISED = 1
 
@@ -73,6 +76,7 @@ SIGNATURES = {
     "nc_set_grad_events": (_I, [_P, ctypes.POINTER(ctypes.c_void_p), _I]),
     "nc_debug_expired_wait": (_I, [_P, _I, _P]),
     "nc_set_lm_head": (_I, [_P, _I, _I]),
+    "nc_set_recompute": (_I, [_P, _I]),
     "nc_kv_cache_bytes": (_SZ, [_P, _I, _I]),
     "nc_inference_workspace_bytes": (_SZ, [_P, _I, _I]),
     "nc_prefill": (_I, [_P, _P, _I, _I, _P, _P, _I, _P, _P, _SZ, _P]),

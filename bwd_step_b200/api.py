@@ -224,6 +224,12 @@ class Model:
         if logits.numel() < B * self.cfg.vocab:
             raise ValueError("logits must hold [B, V]")
 
+    def set_recompute(self, mlp: bool):
+        """Recompute the MLP's relu(u), relu(u)^2 in the backward instead of
+        saving them per layer (less workspace; query workspace_bytes afterwards)."""
+        _ok(lib().nc_set_recompute(self._h, _lib.NC_RECOMPUTE_MLP if mlp else _lib.NC_RECOMPUTE_NONE),
+            "nc_set_recompute")
+
     def set_lm_head(self, mode: str = "fused", chunk_rows: int = 0):
         """LM head strategy: "fused" (logits never stored; bf16 only) or
         "materialised" (logit chunks plus a cross-entropy pass); chunk_rows 0 =

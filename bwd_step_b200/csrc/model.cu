@@ -34,6 +34,8 @@ struct nc_model {
     // logit chunks with a separate cross-entropy pass; rows per chunk (0 = default)
     int lm_mode = NC_LM_HEAD_FUSED;
     int lm_rows = 0;
+    // activations recomputed in the backward instead of saved (NC_RECOMPUTE_*)
+    int recompute = NC_RECOMPUTE_NONE;
     // caller-owned events recorded when each gradient bucket is final (may be empty)
     std::vector<cudaEvent_t> grad_events;
     // profiler: CUDA events around every launch while enabled
@@ -64,6 +66,8 @@ struct Plan {
     size_t tok, tgt, cosb, sinb, x, dx, g, dxb, xf, r0, rf;
     size_t layers, lay_stride;
     size_t l_a, l_r1, l_qkv, l_rqk, l_o, l_lse, l_m, l_r2, l_ru, l_h;
+    bool mlp_shared = false;  // relu(u), relu(u)^2 in one slot for all layers (recomputed in the backward)
+    size_t mlp_ru, mlp_h;
     size_t du, dO, dqkv, Dbuf, zc, dlc, loss_rows, emb, splitk, splitk_bytes, attn_ws, attn_ws_bytes;
     size_t lm_stats, lm_zt, lm_ut, lm_rs, lm_xfs;
     int lm_tiles = 0;
@@ -118,10 +122,13 @@ Plan make_plan(const nc_model* m, int B, int T, bool fwd_only = false) {
     p.l_lse = ltake(4 * attn_stat_elems(B, T, m->H));
     p.l_m = ltake(A * M * d);
     p.l_r2 = ltake(4 * M);
-    p.l_ru = ltake(A * M * m->F);
-    p.l_h = ltake(A * M * m->F);
+    p.mlp_shared = bwd && (m->recompute & NC_RECOMPUTE_MLP);
+    p.l_ru = ltake(p.mlp_shared ? 0 : A * M * m->F);
+    p.l_h = ltake(p.mlp_shared ? 0 : A * M * m->F);
     p.lay_stride = lo;
     p.layers = take(lo * (bwd ? m->L : 1));
+    p.mlp_ru = take(p.mlp_shared ? A * M * m->F : 0);
+    p.mlp_h = take(p.mlp_shared ? A * M * m->F : 0);
     p.du = take(bwd ? A * M * m->F : 0);
     p.dO = take(bwd ? A * M * m->H * m->hd : 0);
     p.dqkv = take(bwd ? A * M * m->Nqkv : 0);
@@ -155,19 +162,23 @@ struct Ctx {
     cudaStream_t s;
     template <typename T = void> T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
     char* layer(int l) const { return ws + p.layers + (size_t)l * p.lay_stride; }
+    // relu(u) and relu(u)^2 of layer l's MLP (one shared slot when they are recomputed)
+    void* mlp_ru(char* lb) const { return p.mlp_shared ? ws + p.mlp_ru : lb + p.l_ru; }
+    void* mlp_h(char* lb) const { return p.mlp_shared ? ws + p.mlp_h : lb + p.l_h; }
 };
 
 enum ProfCls {
     P_GEMM_FWD = 0, P_GEMM_DGRAD, P_GEMM_WGRAD, P_GEMM_LM_Z, P_GEMM_LM_DX, P_GEMM_LM_DW, P_GEMM_FMA,
     P_ATTN_FWD, P_ATTN_BWD, P_ATTN_BWD_DQ, P_ATTN_BWD_DKV, P_NORM_FWD, P_NORM_BWD, P_QKROPE_FWD, P_QKROPE_BWD,
-    P_EMBED_FWD, P_EMBED_BWD, P_CE, P_OTHER, P_COUNT
+    P_EMBED_FWD, P_EMBED_BWD, P_CE, P_OTHER, P_GEMM_RECOMPUTE, P_COUNT
 };
 // tcgen05 GEMM launches are tagged by role: forward y = x W^T, input
 // gradient dX = dY W, weight gradient dW = dY^T X, and the three LM-head products.
 const char* const kProfNames[P_COUNT] = {
     "gemm_fwd", "gemm_dgrad", "gemm_wgrad", "gemm_lmhead_z", "gemm_lmhead_dx", "gemm_lmhead_dw", "gemm_fma",
     "attention_fwd", "attention_bwd", "attention_bwd_dq", "attention_bwd_dkv", "rmsnorm_fwd", "rmsnorm_bwd",
-    "qknorm_rope_fwd", "qknorm_rope_bwd", "embed_fwd", "embed_bwd", "cross_entropy", "other"};
+    "qknorm_rope_fwd", "qknorm_rope_bwd", "embed_fwd", "embed_bwd", "cross_entropy", "other",
+    "gemm_recompute"};
 
 // Records a CUDA event pair around the launches made in its lifetime (only
 // while profiling is enabled), with the algorithmic FLOPs / HBM bytes of the work.
@@ -320,8 +331,8 @@ int forward_blocks(const Ctx& c, const W& w, const int32_t* tok, bool save, cons
         void* qkv = lb + c.p.l_qkv;
         void* o = lb + c.p.l_o;
         void* mm = lb + c.p.l_m;
-        void* ru = lb + c.p.l_ru;
-        void* h = lb + c.p.l_h;
+        void* ru = c.mlp_ru(lb);
+        void* h = c.mlp_h(lb);
         { Prof pr(c, P_NORM_FWD, 0.0, (double)M * (4.0 * d + A * d + 4.0)); CK(launch_rmsnorm_fwd(m->at, x, a, (float*)(lb + c.p.l_r1), M, d, c.s)); }
         // q, k, v = a Wq^T, a Wk^T, a Wv^T; then q, k <- rope(rmsnorm(q, k)) per head, fused into
         // the GEMM epilogue on the tensor-core path
@@ -451,10 +462,16 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         char* lb = c.layer(l);
         int base = 1 + 6 * l;
         // MLP: x_out = x_mid + h Wproj^T, h = relu(u)^2, u = m Wfc^T
+        if (c.p.mlp_shared && l != m->L - 1) {
+            // recompute relu(u) and relu(u)^2 from the saved m (the last layer's are still in the slot)
+            GemmDesc fc = mk(m, M, F, d, lb + c.p.l_m, d, true, w.wfc(l), d, true, EPI_RELU2, c.mlp_h(lb), F, m->at);
+            fc.C2 = c.mlp_ru(lb); fc.ldc2 = F;
+            RG(run_gemm(c, fc, P_GEMM_RECOMPUTE));
+        }
         GemmDesc g1 = mk(m, M, F, d, dxb, d, true, w.wproj(l), F, false, EPI_RELU2_BWD, du, F, m->at);
-        g1.aux = lb + c.p.l_ru; g1.ldaux = F;
+        g1.aux = c.mlp_ru(lb); g1.ldaux = F;
         RG(run_gemm(c, g1, P_GEMM_DGRAD));
-        RG(run_gemm(c, mk(m, d, F, M, dxb, d, false, lb + c.p.l_h, F, false, EPI_STORE, G(base + 5), F, DT_F32),
+        RG(run_gemm(c, mk(m, d, F, M, dxb, d, false, c.mlp_h(lb), F, false, EPI_STORE, G(base + 5), F, DT_F32),
                     P_GEMM_WGRAD));
         RG(run_gemm(c, mk(m, M, d, F, du, F, true, w.wfc(l), d, false, EPI_STORE, gbuf, d, DT_F32), P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32),
@@ -749,6 +766,12 @@ int nc_set_lm_head(nc_model* m, int mode, int chunk_rows) {
     if (mode == NC_LM_HEAD_FUSED && !m->tc) return NC_ERR_INVALID_ARG;
     m->lm_mode = mode;
     m->lm_rows = chunk_rows;
+    return NC_OK;
+}
+
+int nc_set_recompute(nc_model* m, int flags) {
+    if (!m || (flags & ~NC_RECOMPUTE_MLP)) return NC_ERR_INVALID_ARG;
+    m->recompute = flags;
     return NC_OK;
 }
 

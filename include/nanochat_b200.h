@@ -253,6 +253,19 @@ typedef struct {
 int nc_adamw_step(const nc_adamw_group* groups, int n_groups, int64_t n_params, int step, float* master,
                   void* weights, int weights_bf16, const float* grads, float* m, float* v, void* stream);
 
+/* Activation recomputation (the llm.c training command's option to
+ * recompute activations in the backward, qian.cx llm.c article): with
+ * NC_RECOMPUTE_MLP, nc_forward_backward keeps relu(u) and relu(u)^2 of the MLP
+ * in one slot shared by all layers and recomputes them from the saved input
+ * of the MLP (one extra up-projection GEMM per layer but the last) in the
+ * backward, instead of saving them per layer: 2 * 2 * B*T * mlp_mult*d_model
+ * bytes per layer less workspace (bf16).  The results are bitwise those of
+ * NC_RECOMPUTE_NONE (the same GEMM runs again on the same operands).  Changes
+ * nc_workspace_bytes.  NC_ERR_INVALID_ARG for unknown flags. */
+#define NC_RECOMPUTE_NONE 0
+#define NC_RECOMPUTE_MLP 1
+int nc_set_recompute(nc_model* m, int flags);
+
 /* Weight-gradient GEMM that allocates no memory at all.
  *
  * No counterpart in the paper: this is an extra entry point of this library.

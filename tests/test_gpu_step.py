@@ -222,3 +222,26 @@ def test_argument_errors():
         m.forward_backward(torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda(), W, grads, loss, small)
     assert e.value.code == _lib.NC_ERR_WORKSPACE_TOO_SMALL
     assert m.workspace_bytes(0, 16) == 0 and m.workspace_bytes(2, -1) == 0
+
+
+@pytest.mark.parametrize("precision", ["bf16", "fp32"])
+@pytest.mark.parametrize("base,B,T", [("tiny", 3, 37), ("gpt2_124m", 1, 256)])
+def test_recompute_mlp_is_bitwise_equal_and_smaller(precision, base, B, T):
+    """Recomputing relu(u), relu(u)^2 in the backward runs the same GEMM on the
+    same operands: loss and gradients are bitwise those of the saved path, and
+    the workspace shrinks by 2 * 2 (or 4) * B*T*F bytes per layer but one."""
+    cfg = _cfg(base) if base == "tiny" else synth.WORKLOADS[base].model
+    bits, w, tok, tgt = _case(cfg, B, T, precision, ids="zipf" if base != "tiny" else "uniform")
+    m = Model(cfg.as_dict(), precision)
+    W = to_device_weights(bits, w, precision)
+    n0 = m.workspace_bytes(B, T)
+    l0, g0 = gpu_step(m, W, tok, tgt)
+    m.set_recompute(True)
+    n1 = m.workspace_bytes(B, T)
+    l1, g1 = gpu_step(m, W, tok, tgt)
+    assert l1 == l0 and np.array_equal(g0.view(np.uint32), g1.view(np.uint32))
+    es = 2 if precision == "bf16" else 4
+    assert n0 - n1 >= 2 * es * B * T * cfg.mlp_mult * cfg.d_model * (cfg.n_layer - 1)
+    if base == "tiny":
+        ref_loss, ref_g = oracle.step(cfg, w, tok, tgt)
+        compare(cfg, l1, g1, ref_loss, ref_g, precision)
