@@ -286,6 +286,8 @@ def main():
     ap.add_argument("--table", action="store_true", help="print the per-kernel table to stderr")
     ap.add_argument("--profile-steps", type=int, default=5,
                     help="steps of the separate per-kernel profiling pass")
+    ap.add_argument("--no-lm-modes", action="store_true",
+                    help="skip timing the materialised LM-head strategy next to the fused default")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the short per-workload throughput lines (all five workloads)")
     args = ap.parse_args()
@@ -351,6 +353,28 @@ def main():
     ms_step = ms / args.steps
     value = job_throughput(world, M, args.steps, ms)
     final_loss = float(loss.item())
+
+    # ---------------- the LM head's two strategies, same inputs (fused is the default)
+    lm_modes = None
+    if not args.no_lm_modes:
+        lm_modes = {"fused": ms_step}
+        model.set_lm_head("materialised")
+        ws2 = torch.empty(model.workspace_bytes(B, T), dtype=torch.uint8, device="cuda")
+        for _ in range(2):
+            model.forward_backward(tok_d, tgt_d, W, grads, loss, ws2, stream)
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(max(3, min(args.steps, 10))):
+            model.forward_backward(tok_d, tgt_d, W, grads, loss, ws2, stream)
+        g1.record(stream)
+        barrier()
+        lm_modes["materialised"] = max_over_ranks(g0.elapsed_time(g1), world, dist) / max(3, min(args.steps, 10))
+        lm_modes["materialised_loss"] = float(loss.item())
+        lm_modes["unit"] = "ms per step"
+        model.set_lm_head("fused")
+        del ws2
+        torch.cuda.empty_cache()
 
     # ---------------- per-kernel table: a separate pass with an event pair
     # around every launch (the library's profiler), same inputs and stream
@@ -442,6 +466,7 @@ def main():
         "kernels": kernels,
         "kernel_table_source": f"separate pass of {prof_steps} steps with an event pair around every launch",
         "configs": configs,
+        "lm_head_modes": lm_modes,
     }
     if args.table:
         for k in kernels:

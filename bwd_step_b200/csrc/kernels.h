@@ -81,10 +81,6 @@ EmbedScratch embed_scratch_carve(void* base, int M, int V, int d);
 // rows of unused ids are zero.  Deterministic.
 cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int V, int d, float* dwte,
                                  EmbedScratch sc, cudaStream_t s);
-// out[i] = sum_{s < splits} part[s*n + i] in increasing s.
-cudaError_t launch_splitk_reduce(const float* part, int splits, size_t n, float* out, bool accumulate,
-                                 cudaStream_t s);
-
 // ---------------------------------------------------------------- GEMM
 // C[m,n] = sum_k A(m,k) * B(n,k).
 //   A(m,k) = a_kmajor ? A[m*lda + k] : A[k*lda + m]

@@ -2,12 +2,16 @@
 
     python -m bwd_step_b200.kernel_bench gemm [--only NAME] [--iters N]
     python -m bwd_step_b200.kernel_bench attention [--iters N]
+    python -m bwd_step_b200.kernel_bench step [--workload d20] [--batch B] [--warmup W] [--iters K]
 
 `gemm` runs every GEMM shape of one depth-20 step (32768 tokens, d 1280,
 MLP 5120, 10x128 MQA, vocab 65536 with a 4096-row LM-head chunk) through the
 testing ABI with its real operand layouts and fused epilogue, and prints
 TFLOP/s from CUDA events.  `attention` times the tcgen05 attention forward and
-backward at seq 2048, batch 16.  Each case holds at most a few GB on the device.
+backward at seq 2048, batch 16.  `step` runs W warm-up steps and then K
+steps of a workload (optionally at a smaller batch, for profiler captures
+that must stay small) and prints the library's kernel launches per step.
+Each case holds at most a few GB on the device, except `step` at full batch.
 """
 from __future__ import annotations
 
@@ -113,9 +117,39 @@ def bench_attention(iters, B=16, T=2048, H=10, nkv=1, hd=128):
             {"kernel": "attention_bwd", "ms": t_b, "tflops": 2 * flops / t_b / 1e9}]
 
 
+def run_steps(workload, batch, warmup, iters):
+    import numpy as np
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import synth
+    from . import Model, launch_count
+    wl = synth.WORKLOADS[workload]
+    B = batch or wl.batch
+    bits, _ = synth.make_weights(wl.model, seed=0, dtype="bf16")
+    tok, tgt = synth.make_tokens(wl, seed=1, batch=B)
+    m = Model(wl.model.as_dict(), "bf16")
+    W = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    grads = torch.empty(m.num_params(), dtype=torch.float32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(m.workspace_bytes(B, wl.seq_len), dtype=torch.uint8, device="cuda")
+    tok_d, tgt_d = torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()
+    for _ in range(warmup):
+        m.forward_backward(tok_d, tgt_d, W, grads, loss, ws)
+    torch.cuda.synchronize()
+    l0 = launch_count()
+    t = _timed(lambda: m.forward_backward(tok_d, tgt_d, W, grads, loss, ws), iters) if iters else 0.0
+    per = (launch_count() - l0) // max(iters + 2, 1) if iters else 0
+    assert m.check() == 0
+    return {"workload": workload, "batch": B, "ms_per_step": t, "launches_per_step": per, "loss": float(loss.item())}
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["gemm", "attention"])
+    ap.add_argument("what", choices=["gemm", "attention", "step"])
+    ap.add_argument("--workload", default="d20")
+    ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--only", default=None)
     ap.add_argument("--iters", type=int, default=10)
     args = ap.parse_args()
@@ -125,9 +159,11 @@ def main():
                 continue
             print(json.dumps(bench_gemm(name, args.iters)), flush=True)
             torch.cuda.empty_cache()
-    else:
+    elif args.what == "attention":
         for r in bench_attention(args.iters):
             print(json.dumps(r), flush=True)
+    else:
+        print(json.dumps(run_steps(args.workload, args.batch, args.warmup, args.iters)), flush=True)
 
 
 if __name__ == "__main__":
