@@ -2,7 +2,7 @@
 
     python -m bwd_step_b200.kernel_bench gemm [--only NAME] [--iters N]
     python -m bwd_step_b200.kernel_bench attention [--iters N]
-    python -m bwd_step_b200.kernel_bench step [--workload d20] [--batch B] [--warmup W] [--iters K]
+    python -m bwd_step_b200.kernel_bench step [--workload d20] [--batch B] [--layers L] [--warmup W] [--iters K]
 
 `gemm` runs every GEMM shape of one depth-20 step (32768 tokens, d 1280,
 MLP 5120, 10x128 MQA, vocab 65536 with a 4096-row LM-head chunk) through the
@@ -117,7 +117,7 @@ def bench_attention(iters, B=16, T=2048, H=10, nkv=1, hd=128):
             {"kernel": "attention_bwd", "ms": t_b, "tflops": 2 * flops / t_b / 1e9}]
 
 
-def run_steps(workload, batch, warmup, iters):
+def run_steps(workload, batch, warmup, iters, layers=0):
     import numpy as np
     import os
     import sys
@@ -125,6 +125,10 @@ def run_steps(workload, batch, warmup, iters):
     import synth
     from . import Model, launch_count
     wl = synth.WORKLOADS[workload]
+    if layers:
+        # same shapes with fewer layers: full-size activations in a smaller workspace
+        cfg = synth.ModelConfig(**{**wl.model.as_dict(), "n_layer": layers})
+        wl = synth.Workload(wl.name, cfg, wl.seq_len, wl.batch, wl.ids)
     B = batch or wl.batch
     bits, _ = synth.make_weights(wl.model, seed=0, dtype="bf16")
     tok, tgt = synth.make_tokens(wl, seed=1, batch=B)
@@ -149,6 +153,7 @@ def main():
     ap.add_argument("what", choices=["gemm", "attention", "step"])
     ap.add_argument("--workload", default="d20")
     ap.add_argument("--batch", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--only", default=None)
     ap.add_argument("--iters", type=int, default=10)
@@ -163,7 +168,7 @@ def main():
         for r in bench_attention(args.iters):
             print(json.dumps(r), flush=True)
     else:
-        print(json.dumps(run_steps(args.workload, args.batch, args.warmup, args.iters)), flush=True)
+        print(json.dumps(run_steps(args.workload, args.batch, args.warmup, args.iters, args.layers)), flush=True)
 
 
 if __name__ == "__main__":
