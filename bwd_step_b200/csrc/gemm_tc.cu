@@ -15,8 +15,9 @@
 // Two 256-column accumulators let the epilogue of one tile overlap the main
 // loop of the next.  Operands may be K-major or M/N-major (the backward
 // products read activations and weights transposed without a copy).
-// Split-K (fixed order, deterministic reduction) is used when there are too
-// few output tiles to fill the SMs.  Every mbarrier wait is bounded.
+// Split-K is used when there are too few output tiles to fill the SMs: the
+// last split to finish a 32-row slice of a tile adds the partials in split
+// order (deterministic, no reduction kernel).  Every mbarrier wait is bounded.
 #include "gemm_tc.h"
 #include "tc_common.cuh"
 #include <cudaTypedefs.h>
@@ -125,6 +126,7 @@ __device__ __forceinline__ void splitk_finish(const TcParams& p, int tile, int s
     __threadfence();  // every split's partial rows of this slice are visible
     if (row < p.M) {
         float* crow = reinterpret_cast<float*>(p.C) + (size_t)row * p.N;
+        const float rsr = p.epi == EPI_ROWSCALE ? p.rs[row] : 1.f;
         for (int c = 0; c < BN / 32; ++c) {
             const int n0 = tn * BN + c * 32;
             if (n0 >= p.N) break;
@@ -139,13 +141,14 @@ __device__ __forceinline__ void splitk_finish(const TcParams& p, int tile, int s
                                                     p.part + ((size_t)ks * p.M + row) * p.N + n0) + q);
                         a.x += g.x; a.y += g.y; a.z += g.z; a.w += g.w;
                     }
+                    if (p.epi == EPI_ROWSCALE) { a.x *= rsr; a.y *= rsr; a.z *= rsr; a.w *= rsr; }
                     reinterpret_cast<float4*>(crow + n0)[q] = a;
                 }
             } else {
                 for (int i = 0; i < nv; ++i) {
                     float a = p.epi == EPI_ACCUM ? __ldcg(crow + n0 + i) : 0.f;
                     for (int ks = 0; ks < p.splits; ++ks) a += __ldcg(p.part + ((size_t)ks * p.M + row) * p.N + n0 + i);
-                    crow[n0 + i] = a;
+                    crow[n0 + i] = p.epi == EPI_ROWSCALE ? a * rsr : a;
                 }
             }
         }
@@ -811,9 +814,9 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     const int sms = pair ? num_sms() / 2 : num_sms();
     const int tiles = p.tiles_m * p.tiles_n;
     int splits = 1;
-    // the split-K reduction reads and writes C as float4: C must be 16-byte aligned
-    const bool can_split = (g.epi == EPI_STORE || g.epi == EPI_ACCUM) && !p.c_bf16 && g.ldc == g.N && splitk &&
-                           g.N % 4 == 0 && al16(g.C);
+    // the split-K completion reads and writes C as float4: C must be 16-byte aligned
+    const bool can_split = (g.epi == EPI_STORE || g.epi == EPI_ACCUM || g.epi == EPI_ROWSCALE) && !p.c_bf16 &&
+                           g.ldc == g.N && splitk && g.N % 4 == 0 && al16(g.C);
     if (can_split && tiles < 2 * sms && tiles * kSlicesPerTile <= kMaxCounters && splitk_bytes > kCounterBytes) {
         double best = (double)((tiles + sms - 1) / sms);
         for (int sp = 2; sp <= MAX_SPLITS; ++sp) {
