@@ -20,7 +20,7 @@ def _operand(R, K, kmajor, gen, scale=1.0):
     return x.double(), stored.cuda(), (K if kmajor else R)
 
 
-def _run(M, N, K, ak, bk, epi, c_bf16, use_tc=1, seed=0, scale=1.0, scratch_mb=0, c_offset=0):
+def _run(M, N, K, ak, bk, epi, c_bf16, use_tc=1, seed=0, scale=1.0, scratch_mb=0, c_offset=0, tol=None):
     gen = torch.Generator().manual_seed(seed)
     A64, A, lda = _operand(M, K, ak, gen, scale)
     B64, B, ldb = _operand(N, K, bk, gen, scale)
@@ -52,17 +52,17 @@ def _run(M, N, K, ak, bk, epi, c_bf16, use_tc=1, seed=0, scale=1.0, scratch_mb=0
     elif epi == 2:
         exp = torch.relu(acc) ** 2
         got2 = C2.double().cpu()
-        _close(got2, torch.relu(acc), True)
+        _close(got2, torch.relu(acc), True, tol)
     elif epi == 3:
         exp = acc * 2 * aux.double()
     else:
         exp = 15.0 * torch.tanh(acc / 15.0)
-    _close(C.double().cpu(), exp, c_bf16)
+    _close(C.double().cpu(), exp, c_bf16, tol)
 
 
-def _close(got, exp, bf):
+def _close(got, exp, bf, tol=None):
     err = (got - exp).norm() / max(exp.norm(), 1e-30)
-    assert err <= (4e-3 if bf else 2e-6), float(err)
+    assert err <= (tol or (4e-3 if bf else 2e-6)), float(err)
 
 
 @pytest.mark.parametrize("ak,bk", [(True, True), (True, False), (False, False), (False, True)])
@@ -98,8 +98,9 @@ def test_split_k_ragged_rows(M, N):
 def test_split_k_candidate_with_unaligned_output(epi):
     # a shape that takes split-K, with C one float past a 16-byte boundary: the
     # vectorised split-K reduction must not be used (it would be a misaligned
-    # access); the GEMM still runs, on the single-pass epilogue
-    _run(256, 256, 8192, False, False, epi, False, scratch_mb=64, seed=11 + epi, c_offset=1)
+    # access); the GEMM still runs, on the single-pass epilogue, whose one
+    # 8192-long fp32 accumulation is looser than a sum of split partials
+    _run(256, 256, 8192, False, False, epi, False, scratch_mb=64, seed=11 + epi, c_offset=1, tol=2e-5)
 
 
 def test_fma_gemm_matches_too():
