@@ -9,9 +9,9 @@
 // Both heads of a pair read the same K_j / V_j tiles from shared memory (the
 // K/V head is shared), and their work is interleaved so that one head's
 // softmax runs while the tensor core computes the other head's products:
-//   warp 0     TMA: Q of both heads per unit, then K_j and V_j together into
-//              a ring for key blocks j = 0..qb (causal: blocks past the
-//              diagonal are never loaded);
+//   warp 0     TMA: Q of both heads per unit, then K_j and V_j into two rings
+//              for key blocks j = 0..qb (causal: blocks past the diagonal are
+//              never loaded), K running one block ahead of V;
 //   warp 1     tcgen05.mma in the order ... O_a += P_a(j) V_j, S_a(j+1),
 //              O_b += P_b(j) V_j, S_b(j+1) ...: S = Q K^T into the head's
 //              128 TMEM score columns, O += P V with P read from TMEM (A
@@ -132,18 +132,22 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem_dyn + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t q_full = b0, q_empty = b0 + 8;
-    const uint32_t kv_full = b0 + 16, kv_empty = kv_full + 8 * KVSTG;  // [KVSTG]: K_j and V_j share a stage
-    const uint32_t s_full = kv_empty + 8 * KVSTG;                       // [2] per head of the pair
+    const uint32_t k_full = b0 + 16, k_empty = k_full + 8 * KVSTG;    // [KVSTG] K ring
+    const uint32_t v_full = k_empty + 8 * KVSTG, v_empty = v_full + 8 * KVSTG;  // [KVSTG] V ring
+    const uint32_t s_full = v_empty + 8 * KVSTG;                        // [2] per head of the pair
     const uint32_t p_full = s_full + 16;                                // [2]
     const uint32_t o_full = p_full + 16;                                // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * KVSTG);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 4 * KVSTG);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int st = 0; st < KVSTG; ++st) { mbar_init(kv_full + 8 * st, 1); mbar_init(kv_empty + 8 * st, 1); }
+        for (int st = 0; st < KVSTG; ++st) {
+            mbar_init(k_full + 8 * st, 1); mbar_init(k_empty + 8 * st, 1);
+            mbar_init(v_full + 8 * st, 1); mbar_init(v_empty + 8 * st, 1);
+        }
         for (int x = 0; x < 2; ++x) {
             mbar_init(s_full + 8 * x, 1);
             mbar_init(p_full + 8 * x, 4);
@@ -163,10 +167,26 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 
     if (warp == 0) {
         if (lane == 0) {
-            int k = 0, kvi = 0, inflight_q = 0;
-            uint32_t q_par = 0;
-            uint32_t kv_issued = 0, kv_phase_bits = 0;
+            // Q of the pair, then K and V in two rings: K_{j+1} is loaded before V_j,
+            // because K_j is free as soon as both heads' scores S(j) have been formed,
+            // long before O += P(j) V_j releases V_j
+            int k = 0, ki = 0, vi = 0, inflight_q = 0;
+            uint32_t q_par = 0, issued = 0, phase_bits = 0;  // bit st: K stage st, bit 8 + st: V stage st
             bool ok = true;
+            auto load = [&](bool isv, int i, int xsrc, int row) -> bool {
+                const int st = i % KVSTG;
+                const uint32_t ph = (i / KVSTG) & 1;
+                const uint32_t full = (isv ? v_full : k_full) + 8 * st, empty = (isv ? v_empty : k_empty) + 8 * st;
+                if (!mbar_wait(empty, ph ^ 1, abort_flag, p.status)) return false;
+                mbar_expect_tx(full, TILE);
+                const uint32_t dst = (isv ? sV : sK) + st * TILE;
+#pragma unroll
+                for (int c = 0; c < KB; ++c) tma_load_2d(dst + c * 16384, &tm, xsrc + 64 * c, row, full);
+                const int bit = (isv ? 8 : 0) + st;
+                issued |= 1u << bit;
+                phase_bits = (phase_bits & ~(1u << bit)) | (ph << bit);
+                return true;
+            };
             for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++k) {
                 int b, qb, h0;
                 bool two;
@@ -183,35 +203,32 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 }
                 inflight_q = 1;
                 q_par = k & 1;
-                for (int j = 0; j <= qb; ++j, ++kvi) {
-                    const int st = kvi % KVSTG;
-                    const uint32_t ph = (kvi / KVSTG) & 1;
-                    if (!mbar_wait(kv_empty + 8 * st, ph ^ 1, abort_flag, p.status)) { ok = false; break; }
-                    mbar_expect_tx(kv_full + 8 * st, 2 * TILE);
-#pragma unroll
-                    for (int c = 0; c < KB; ++c) {
-                        tma_load_2d(sK + st * TILE + c * 16384, &tm, xk + 64 * c, row0 + j * 128, kv_full + 8 * st);
-                        tma_load_2d(sV + st * TILE + c * 16384, &tm, xv + 64 * c, row0 + j * 128, kv_full + 8 * st);
-                    }
-                    kv_issued |= 1u << st;
-                    kv_phase_bits = (kv_phase_bits & ~(1u << st)) | (ph << st);
+                if (!load(false, ki++, xk, row0)) { ok = false; break; }
+                for (int j = 0; j <= qb; ++j) {
+                    if (j < qb && !load(false, ki++, xk, row0 + (j + 1) * 128)) { ok = false; break; }
+                    if (!load(true, vi++, xv, row0 + j * 128)) { ok = false; break; }
                 }
             }
             if (!ok) {
                 // let the copies in flight land before the block exits
                 if (inflight_q) drain(q_full, q_par);
-                for (int st = 0; st < KVSTG; ++st)
-                    if (kv_issued >> st & 1) drain(kv_full + 8 * st, (kv_phase_bits >> st) & 1);
+                for (int st = 0; st < KVSTG; ++st) {
+                    if (issued >> st & 1) drain(k_full + 8 * st, (phase_bits >> st) & 1);
+                    if (issued >> (8 + st) & 1) drain(v_full + 8 * st, (phase_bits >> (8 + st)) & 1);
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);
             const uint32_t id_o = idesc_bf16(128, HD, false, true);
-            int k = 0, kvi = 0;
+            int k = 0, ki = 0, vi = 0;
             uint32_t pcnt0 = 0, pcnt1 = 0;  // P hand-overs waited for, per head
             bool ok = true;
-            // S_x = Q_x K^T for head x of the pair, from the K/V stage st
+            auto ready = [&](bool isv, int i) -> bool {
+                return mbar_wait((isv ? v_full : k_full) + 8 * (i % KVSTG), (i / KVSTG) & 1, abort_flag, p.status);
+            };
+            // S_x = Q_x K^T for head x of the pair, from K stage st
             auto scores = [&](int x, int st) {
 #pragma unroll
                 for (int ks = 0; ks < HD / 16; ++ks) {
@@ -220,6 +237,17 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                              smem_desc(sK + st * TILE + off, 16, 1024), id_s, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full + 8 * x);
+            };
+            // both heads' scores of the next K tile, then K's stage is released
+            auto scores_both = [&](bool two) -> bool {
+                if (!ready(false, ki)) return false;
+                tc_fence_after();
+                const int st = ki % KVSTG;
+                scores(0, st);
+                if (two) scores(1, st);
+                mma_commit(k_empty + 8 * st);
+                ++ki;
+                return true;
             };
             // O_x += P_x V: keys 16kk..16kk+15 sit in the packed columns 8kk..8kk+7
             auto pv = [&](int x, int st, bool acc) -> bool {
@@ -233,39 +261,39 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                                 smem_desc(sV + st * TILE + kk * 2048, 16384, 1024), id_o, (acc || kk > 0) ? 1u : 0u);
                 return true;
             };
-            auto kv_ready = [&](int i) -> bool {
-                return mbar_wait(kv_full + 8 * (i % KVSTG), (i / KVSTG) & 1, abort_flag, p.status);
-            };
             for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++k) {
                 int b, qb, h0;
                 bool two;
                 fwd_unit(p, u, b, qb, h0, two);
                 const int nblk = qb + 1;
-                if (!mbar_wait(q_full, k & 1, abort_flag, p.status) || !kv_ready(kvi)) { ok = false; break; }
-                tc_fence_after();
-                scores(0, kvi % KVSTG);
-                if (two) scores(1, kvi % KVSTG);
+                if (!mbar_wait(q_full, k & 1, abort_flag, p.status) || !scores_both(two)) { ok = false; break; }
                 if (nblk == 1) mma_commit(q_empty);  // the unit's last products that read Q
                 for (int j = 0; j < nblk; ++j) {
-                    const int st = (kvi + j) % KVSTG, st1 = (kvi + j + 1) % KVSTG;
                     const bool more = j + 1 < nblk;
-                    if (!pv(0, st, j > 0)) { ok = false; break; }
+                    const int vst = vi % KVSTG;
+                    if (!ready(true, vi)) { ok = false; break; }
+                    // head a: O += P(j) V_j, then S(j+1) (which overwrites P(j) after it, in issue order)
+                    if (!pv(0, vst, j > 0)) { ok = false; break; }
                     if (more) {
-                        if (!kv_ready(kvi + j + 1)) { ok = false; break; }
+                        if (!ready(false, ki)) { ok = false; break; }
                         tc_fence_after();
-                        scores(0, st1);
+                        scores(0, ki % KVSTG);
                     } else {
                         mma_commit(o_full);
                     }
-                    if (two && !pv(1, st, j > 0)) { ok = false; break; }
-                    mma_commit(kv_empty + 8 * st);  // K_j, V_j read by every product of this block
-                    if (two) {
-                        if (more) scores(1, st1);
-                        else mma_commit(o_full + 8);
+                    // head b likewise; V_j and (after both heads' scores) K_{j+1} are then released
+                    if (two && !pv(1, vst, j > 0)) { ok = false; break; }
+                    mma_commit(v_empty + 8 * vst);
+                    ++vi;
+                    if (more) {
+                        if (two) scores(1, ki % KVSTG);
+                        mma_commit(k_empty + 8 * (ki % KVSTG));
+                        ++ki;
+                    } else if (two) {
+                        mma_commit(o_full + 8);
                     }
                     if (j + 2 == nblk) mma_commit(q_empty);
                 }
-                kvi += nblk;
             }
         }
     } else {
