@@ -255,31 +255,42 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
     return NC_OK;
 }
 
-// Attention backward: statistics and dk / dv (which also stores the dS tiles),
-// then dq from those tiles (tensor cores), or the plain-FMA kernels.
-int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, void* dqkv) {
+// Attention backward, then the QK-norm + RoPE backward into the pre-norm q, k
+// gradients.  Tensor cores: statistics and dk / dv (which also stores the dS
+// tiles), then dq from those tiles, with the QK-norm + RoPE backward fused into
+// the dk and dq epilogues; otherwise the plain-FMA kernels and a separate pass.
+int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, const float* rqk,
+                  void* dqkv) {
     const nc_model* m = c.m;
     float* Dbuf = c.at<float>(c.p.Dbuf);
+    const float* cs = c.at<float>(c.p.cosb);
+    const float* sn = c.at<float>(c.p.sinb);
     if (m->tc && attention_tc_bwd_supported(m->hd)) {
         void* ws = c.ws + c.p.attn_ws;
+        const QkNormRope qk{rqk, cs, sn};
         int r;
         {
             Prof pr(c, P_ATTN_BWD_DKV, 2.0 * attn_flops(c), 0.0);
             r = attention_tc_bwd_stats(o, dO, lse, Dbuf, c.p.B, c.p.T, m->H, m->hd, c.s);
             if (r == 0)
                 r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, ws, c.p.attn_ws_bytes, c.p.B, c.p.T, m->H, m->nkv,
-                                         m->hd, m->status, c.s);
+                                         m->hd, &qk, m->status, c.s);
         }
         if (r == 0) {
             Prof pr(c, P_ATTN_BWD_DQ, 0.5 * attn_flops(c), 0.0);
-            r = attention_tc_bwd_dq(qkv, ws, c.p.attn_ws_bytes, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status,
-                                    c.s);
+            r = attention_tc_bwd_dq(qkv, ws, c.p.attn_ws_bytes, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, &qk,
+                                    m->status, c.s);
         }
         if (r == 0) return NC_OK;
         if (r < 0) return NC_ERR_CUDA;
     }
-    Prof pr(c, P_ATTN_BWD, 2.0 * attn_flops(c), 0.0);
-    CK(launch_attention_bwd_simt(m->at, qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.s));
+    {
+        Prof pr(c, P_ATTN_BWD, 2.0 * attn_flops(c), 0.0);
+        CK(launch_attention_bwd_simt(m->at, qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.s));
+    }
+    const double A = (double)dt_size(m->at);
+    Prof pr(c, P_QKROPE_BWD, 0.0, (double)c.p.M * (m->H + m->nkv) * (3.0 * A * m->hd + 4.0));
+    CK(launch_qknorm_rope_bwd(m->at, dqkv, qkv, rqk, cs, sn, c.p.M, c.p.T, m->H, m->nkv, m->hd, c.s));
     return NC_OK;
 }
 
@@ -481,12 +492,8 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at), P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
                           DT_F32), P_GEMM_WGRAD));
-        RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), dqkv));
-        {
-            Prof pr(c, P_QKROPE_BWD, 0.0, (double)M * (m->H + m->nkv) * (3.0 * A * m->hd + 4.0));
-            CK(launch_qknorm_rope_bwd(m->at, dqkv, lb + c.p.l_qkv, (float*)(lb + c.p.l_rqk), cs, sn, M, T, m->H,
-                                      m->nkv, m->hd, s));
-        }
+        RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), (float*)(lb + c.p.l_rqk),
+                         dqkv));
         RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, DT_F32),
                     P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, Nqkv, d, M, dqkv, Nqkv, false, lb + c.p.l_a, d, false, EPI_STORE, G(base), d,
