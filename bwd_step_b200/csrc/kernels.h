@@ -73,6 +73,8 @@ struct EmbedScratch {
     int* part_base;    // [V] first partial-sum slot of each multi-piece id
     int* piece_bucket; // [pieces] id of each piece
     int* totals;       // [2] pieces, partial slots
+    int* fpre;         // [V] used ids before each id within its block of 1024
+    void* blk;         // [ceil(V/1024)] per-block scan totals, then prefixes
     float* partial;    // [partial slots, d] piece sums of multi-piece ids
 };
 size_t embed_scratch_bytes(int M, int V, int d);

@@ -776,45 +776,93 @@ __global__ void emb_hist_kernel(const int32_t* __restrict__ idx, int M, int V, i
     if (id >= 0 && id < V) atomicAdd(&count[id], 1);
 }
 
-// Single block of 1024 threads: exclusive scans over the V buckets of
-// (count, used?, pieces, partial pieces) and the list of used ids.
-__global__ void emb_scan_kernel(const int* __restrict__ count, int V, int* offset, int* active, int* n_active,
-                                int* piece_base, int* part_base, int* totals) {
-    __shared__ int sc[1024], sf[1024], sp[1024], sq[1024];
-    int t = threadIdx.x;
-    int per = (V + 1023) / 1024;
-    int lo = min(V, t * per), hi = min(V, lo + per);
-    int c = 0, f = 0, pc = 0, pq = 0;
-    for (int i = lo; i < hi; ++i) {
-        int k = count[i];
-        int np = (k + kPiece - 1) / kPiece;
-        c += k; f += k > 0; pc += np; pq += np > 1 ? np : 0;
+// Exclusive scans over the V buckets of (count, used?, pieces, partial pieces),
+// and the list of used ids in increasing order, in three parallel passes:
+// (1) every 1024-id block scans its own ids and records its totals, (2) one
+// block scans the block totals, (3) every id adds its block's prefix.
+struct Scan4 { int c, f, p, q; };
+
+__device__ __forceinline__ Scan4 emb_vals(int k) {
+    const int np = (k + kPiece - 1) / kPiece;
+    return {k, k > 0 ? 1 : 0, np, np > 1 ? np : 0};
+}
+
+// Exclusive block-wide scan of four ints over 1024 threads; *total gets the block sums.
+__device__ __forceinline__ Scan4 block_scan4(Scan4 v, Scan4* total) {
+    __shared__ Scan4 warp_sums[32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    Scan4 inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int c = __shfl_up_sync(0xffffffffu, inc.c, o), f = __shfl_up_sync(0xffffffffu, inc.f, o);
+        const int p = __shfl_up_sync(0xffffffffu, inc.p, o), q = __shfl_up_sync(0xffffffffu, inc.q, o);
+        if (lane >= o) { inc.c += c; inc.f += f; inc.p += p; inc.q += q; }
     }
-    sc[t] = c; sf[t] = f; sp[t] = pc; sq[t] = pq;
+    if (lane == 31) warp_sums[w] = inc;
     __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-        int a = t >= o ? sc[t - o] : 0, b = t >= o ? sf[t - o] : 0;
-        int e = t >= o ? sp[t - o] : 0, g = t >= o ? sq[t - o] : 0;
-        __syncthreads();
-        sc[t] += a; sf[t] += b; sp[t] += e; sq[t] += g;
-        __syncthreads();
+    if (w == 0) {
+        Scan4 t = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int c = __shfl_up_sync(0xffffffffu, t.c, o), f = __shfl_up_sync(0xffffffffu, t.f, o);
+            const int p = __shfl_up_sync(0xffffffffu, t.p, o), q = __shfl_up_sync(0xffffffffu, t.q, o);
+            if (lane >= o) { t.c += c; t.f += f; t.p += p; t.q += q; }
+        }
+        warp_sums[lane] = t;  // inclusive over warps
     }
-    int bc = sc[t] - c, bf = sf[t] - f, bp = sp[t] - pc, bq = sq[t] - pq;
-    for (int i = lo; i < hi; ++i) {
-        int k = count[i];
-        int np = (k + kPiece - 1) / kPiece;
-        offset[i] = bc;
-        piece_base[i] = bp;
-        part_base[i] = bq;
-        if (k > 0) active[bf++] = i;
-        bc += k; bp += np; bq += np > 1 ? np : 0;
+    __syncthreads();
+    const Scan4 before = w > 0 ? warp_sums[w - 1] : Scan4{0, 0, 0, 0};
+    *total = warp_sums[31];
+    return {before.c + inc.c - v.c, before.f + inc.f - v.f, before.p + inc.p - v.p, before.q + inc.q - v.q};
+}
+
+__global__ void __launch_bounds__(1024) emb_scan_local_kernel(const int* __restrict__ count, int V, int* offset,
+                                                              int* fpre, int* piece_base, int* part_base, Scan4* blk) {
+    const int i = blockIdx.x * 1024 + threadIdx.x;
+    const Scan4 v = i < V ? emb_vals(count[i]) : Scan4{0, 0, 0, 0};
+    Scan4 tot;
+    const Scan4 ex = block_scan4(v, &tot);
+    if (i < V) {
+        offset[i] = ex.c;
+        fpre[i] = ex.f;
+        piece_base[i] = ex.p;
+        part_base[i] = ex.q;
     }
-    if (t == 1023) {
-        offset[V] = sc[1023];
-        *n_active = sf[1023];
-        totals[0] = sp[1023];  // pieces
-        totals[1] = sq[1023];  // partial slots
+    if (threadIdx.x == 0) blk[blockIdx.x] = tot;
+}
+
+// One block: exclusive scan of the nb block totals in place, and the grand totals.
+__global__ void __launch_bounds__(1024) emb_scan_blocks_kernel(Scan4* blk, int nb, int V, int* offset, int* n_active,
+                                                               int* totals) {
+    const int per = (nb + 1023) / 1024;
+    const int lo = min(nb, (int)threadIdx.x * per), hi = min(nb, lo + per);
+    Scan4 sum{0, 0, 0, 0};
+    for (int j = lo; j < hi; ++j) { const Scan4 b = blk[j]; sum.c += b.c; sum.f += b.f; sum.p += b.p; sum.q += b.q; }
+    Scan4 tot;
+    Scan4 run = block_scan4(sum, &tot);
+    for (int j = lo; j < hi; ++j) {
+        const Scan4 b = blk[j];
+        blk[j] = run;
+        run.c += b.c; run.f += b.f; run.p += b.p; run.q += b.q;
     }
+    if (threadIdx.x == 0) {
+        offset[V] = tot.c;
+        *n_active = tot.f;
+        totals[0] = tot.p;  // pieces
+        totals[1] = tot.q;  // partial slots
+    }
+}
+
+__global__ void __launch_bounds__(1024) emb_scan_add_kernel(const int* __restrict__ count, int V, const Scan4* blk,
+                                                            int* offset, const int* __restrict__ fpre, int* piece_base,
+                                                            int* part_base, int* active) {
+    const int i = blockIdx.x * 1024 + threadIdx.x;
+    if (i >= V) return;
+    const Scan4 b = blk[blockIdx.x];
+    offset[i] += b.c;
+    piece_base[i] += b.p;
+    part_base[i] += b.q;
+    if (count[i] > 0) active[fpre[i] + b.f] = i;
 }
 
 __global__ void emb_fill_kernel(const int32_t* __restrict__ idx, int M, int V, const int* __restrict__ offset,
@@ -1177,11 +1225,12 @@ static inline size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 static inline int emb_max_pieces(int M, int V) { return M / kPiece + (M < V ? M : V) + 1; }
 static inline int emb_max_partials(int M) { return 2 * (M / kPiece) + 2; }
+static inline int emb_scan_blocks(int V) { return (V + 1023) / 1024; }
 
 size_t embed_scratch_bytes(int M, int V, int d) {
     return al256(4ull * V) * 2 + al256(4ull * (V + 1)) + al256(4ull * M) * 2 + al256(4ull * V) + 256 +
-           al256(4ull * V) * 2 + al256(4ull * emb_max_pieces(M, V)) + 256 +
-           al256(4ull * emb_max_partials(M) * d);
+           al256(4ull * V) * 2 + al256(4ull * emb_max_pieces(M, V)) + 256 + al256(4ull * V) +
+           al256(16ull * emb_scan_blocks(V)) + al256(4ull * emb_max_partials(M) * d);
 }
 
 EmbedScratch embed_scratch_carve(void* base, int M, int V, int d) {
@@ -1198,6 +1247,8 @@ EmbedScratch embed_scratch_carve(void* base, int M, int V, int d) {
     s.part_base = (int*)p;    p += al256(4ull * V);
     s.piece_bucket = (int*)p; p += al256(4ull * emb_max_pieces(M, V));
     s.totals = (int*)p;       p += 256;
+    s.fpre = (int*)p;         p += al256(4ull * V);
+    s.blk = p;                p += al256(16ull * emb_scan_blocks(V));
     s.partial = (float*)p;
     (void)d;
     return s;
@@ -1209,8 +1260,12 @@ cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int
     if (e != cudaSuccess) return e;
     int mb = (M + 255) / 256;
     emb_hist_kernel<<<mb, 256, 0, s>>>(idx, M, V, sc.count);
-    emb_scan_kernel<<<1, 1024, 0, s>>>(sc.count, V, sc.offset, sc.active, sc.n_active, sc.piece_base, sc.part_base,
-                                       sc.totals);
+    const int nb = emb_scan_blocks(V);
+    Scan4* blk = reinterpret_cast<Scan4*>(sc.blk);
+    emb_scan_local_kernel<<<nb, 1024, 0, s>>>(sc.count, V, sc.offset, sc.fpre, sc.piece_base, sc.part_base, blk);
+    emb_scan_blocks_kernel<<<1, 1024, 0, s>>>(blk, nb, V, sc.offset, sc.n_active, sc.totals);
+    emb_scan_add_kernel<<<nb, 1024, 0, s>>>(sc.count, V, blk, sc.offset, sc.fpre, sc.piece_base, sc.part_base,
+                                            sc.active);
     emb_fill_kernel<<<mb, 256, 0, s>>>(idx, M, V, sc.offset, sc.cursor, sc.perm);
     emb_canon_kernel<<<mb, 256, 0, s>>>(idx, V, sc.offset, sc.perm, sc.perm2);
     int na = M < V ? M : V;
@@ -1222,7 +1277,7 @@ cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int
     emb_combine_kernel<<<na, 128, 0, s>>>(d, sc.count, sc.active, sc.n_active, sc.part_base, sc.partial, dwte);
     size_t n4 = (size_t)V * (d / 4);
     emb_zero_unused_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(sc.count, V, d / 4, dwte);
-    count_launch(9);
+    count_launch(11);
     return cudaGetLastError();
 }
 
