@@ -59,14 +59,47 @@ struct TcParams {
     float* zt;
     float* ut;
     const float* rs;  // EPI_ROWSCALE
+    float* attn_d;    // EPI_ATTN_DO
+    float* attn_lse2;
+    const float* attn_lse;
+    int attn_H;
 };
 
 // Per-row state of the epilogue across the 32-column chunks of one tile.
 struct RowCtx {
     int tgt;    // EPI_LMHEAD: the row's target column (-1 for rows past M)
     float rs;   // EPI_ROWSCALE: the row's factor
-    float sum;  // EPI_LMHEAD: sum of e over the tile's columns so far
+    float sum;  // EPI_LMHEAD: sum of e over the tile's columns so far; EPI_ATTN_DO: dO . o of the head so far
 };
+
+// Attention-backward statistics in the epilogue of the GEMM that forms dO
+// (softmax backward: dS = P (dP - D) with D = rowsum(dO * o)): the 32-column
+// chunk n0.. of this row is rounded to the stored bf16 dO (so D uses the same
+// values as the dP product), multiplied with o and summed; at the last chunk
+// of a head, D and lse * log2(e) are written for (batch row, head, position).
+__device__ __forceinline__ void attn_do_chunk(const TcParams& p, int row, int n0, float* v, RowCtx& rc) {
+    constexpr float kL2e = 1.44269504088896340736f;
+    const bf16* o = p.aux + (int64_t)row * p.ldaux + n0;
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        float ov[8];
+        load_vec(o + 8 * e, ov);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            v[8 * e + i] = __bfloat162float(__float2bfloat16_rn(v[8 * e + i]));
+            s = fmaf(v[8 * e + i], ov[i], s);
+        }
+    }
+    rc.sum += s;
+    if ((n0 + 32) % p.hd == 0) {  // last chunk of head h
+        const int h = n0 / p.hd, b = row / p.T, t = row % p.T;
+        const size_t i = ((size_t)b * p.attn_H + h) * (size_t)attn_tpad(p.T) + t;
+        p.attn_d[i] = rc.sum;
+        p.attn_lse2[i] = p.attn_lse[i] * kL2e;
+        rc.sum = 0.f;
+    }
+}
 
 __device__ __forceinline__ RowCtx row_ctx(const TcParams& p, int row) {
     RowCtx c;
@@ -255,6 +288,10 @@ __device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int
             for (int i = 0; i < 32; ++i) v[i] *= rc.rs;
             store_row_f32(reinterpret_cast<float*>(p.C) + off, v, nv, vec);
             break;
+        case EPI_ATTN_DO:
+            attn_do_chunk(p, row, n0, v, rc);
+            store_row_bf16(reinterpret_cast<bf16*>(p.C) + off, v, nv, vec);
+            break;
     }
 }
 
@@ -322,6 +359,8 @@ __device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUte
         } else if (mode == EPI_ROWSCALE) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] *= rc.rs;
+        } else if (mode == EPI_ATTN_DO) {
+            if (row < p.M) attn_do_chunk(p, row, n0, v, rc);
         }
         if (bf) stage_bf16(buf, lane, v);
         else stage_f32(buf, lane, v);
@@ -771,6 +810,11 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
         (g.c_t != DT_BF16 || !g.tgt || !g.stats || !g.zt || !g.ut || g.stats_ld < gemm_tiles_n(g.N) || !(g.cap > 0.f)))
         return 1;
     if (g.epi == EPI_ROWSCALE && (g.c_t != DT_F32 || !g.rs)) return 1;
+    if (g.epi == EPI_ATTN_DO &&
+        (g.c_t != DT_BF16 || !g.aux || !g.attn_d || !g.attn_lse2 || !g.attn_lse || g.T <= 0 || g.attn_H <= 0 ||
+         (g.hd != 32 && g.hd != 64 && g.hd != 128) || g.N != g.attn_H * g.hd || g.ldaux % 8 ||
+         (reinterpret_cast<uintptr_t>(g.aux) & 15)))
+        return 1;
     if (g.M <= 0 || g.N <= 0 || g.K <= 0) return 1;
     auto al16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; };
     if (!al16(g.A) || !al16(g.B) || (g.lda * 2) % 16 || (g.ldb * 2) % 16) return 1;
@@ -798,6 +842,7 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     p.rqk = g.rqk; p.cos_t = g.cos_t; p.sin_t = g.sin_t;
     p.tgt = g.tgt; p.stats = g.stats; p.stats_ld = g.stats_ld; p.zt = g.zt; p.ut = g.ut;
     p.rs = g.rs;
+    p.attn_d = g.attn_d; p.attn_lse2 = g.attn_lse2; p.attn_lse = g.attn_lse; p.attn_H = g.attn_H;
     const int esz = p.c_bf16 ? 2 : 4;
     bool vec = al16(g.C) && (g.ldc * esz) % 16 == 0;
     if (g.epi == EPI_RELU2) vec = vec && al16(g.C2) && (g.ldc2 * 2) % 16 == 0;

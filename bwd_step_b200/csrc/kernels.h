@@ -101,6 +101,10 @@ enum Epi : int {
                         // into stats[row * stats_ld + tile]; at the column tgt[row], z and C in
                         // fp32 into zt[row], ut[row] (tcgen05 only)
     EPI_ROWSCALE = 7,   // C = acc * rs[row]                 (C fp32; tcgen05 only)
+    EPI_ATTN_DO = 8,    // attention output gradient dO: C = acc (bf16), and per (row, head of hd
+                        // columns) D = sum of C * aux (aux = o, the attention output) and
+                        // lse * log2(e), into the [B, H, Tp] statistics of the backward
+                        // (row = b T + t; tcgen05 only)
 };
 
 struct GemmDesc {
@@ -128,6 +132,12 @@ struct GemmDesc {
     float* ut = nullptr;
     // EPI_ROWSCALE: one factor per row
     const float* rs = nullptr;
+    // EPI_ATTN_DO: statistics D and lse*log2(e) [B, H, attn_tpad(T)], the lse they come from,
+    // the number of heads (hd and T as above)
+    float* attn_d = nullptr;
+    float* attn_lse2 = nullptr;
+    const float* attn_lse = nullptr;
+    int attn_H = 0;
 };
 
 // Column tiles of the tensor-core GEMM's output (EPI_LMHEAD writes one sum per tile).

@@ -260,7 +260,7 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
 // tiles), then dq from those tiles, with the QK-norm + RoPE backward fused into
 // the dk and dq epilogues; otherwise the plain-FMA kernels and a separate pass.
 int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, const float* rqk,
-                  void* dqkv) {
+                  void* dqkv, bool stats_ready) {
     const nc_model* m = c.m;
     float* Dbuf = c.at<float>(c.p.Dbuf);
     const float* cs = c.at<float>(c.p.cosb);
@@ -271,7 +271,7 @@ int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, 
         int r;
         {
             Prof pr(c, P_ATTN_BWD_DKV, 2.0 * attn_flops(c), 0.0);
-            r = attention_tc_bwd_stats(o, dO, lse, Dbuf, c.p.B, c.p.T, m->H, m->hd, c.s);
+            r = stats_ready ? 0 : attention_tc_bwd_stats(o, dO, lse, Dbuf, c.p.B, c.p.T, m->H, m->hd, c.s);
             if (r == 0)
                 r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, ws, c.p.attn_ws_bytes, c.p.B, c.p.T, m->H, m->nkv,
                                          m->hd, &qk, m->status, c.s);
@@ -467,6 +467,11 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     void* du = c.at(c.p.du);
     void* dO = c.at(c.p.dO);
     void* dqkv = c.at(c.p.dqkv);
+    float* Dbuf = c.at<float>(c.p.Dbuf);
+    // the attention statistics come from the dO GEMM's epilogue (rows t < T only): the
+    // padding of the last query block past T stays zero for the whole backward
+    const bool fuse_stats = m->tc && attention_tc_bwd_supported(m->hd);
+    if (fuse_stats && T % 128 != 0) CK(cudaMemsetAsync(Dbuf, 0, 4 * attn_dbuf_elems(B, T, m->H), s));
     const float* cs = c.at<float>(c.p.cosb);
     const float* sn = c.at<float>(c.p.sinb);
     for (int l = m->L - 1; l >= 0; --l) {
@@ -488,12 +493,25 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         RG(run_gemm(c, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32),
                     P_GEMM_WGRAD));
         { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (12.0 * d + 2.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_m, (float*)(lb + c.p.l_r2), dx, true, dxb, M, d, s)); }
-        // attention: x_mid = x_in + o Wo^T
-        RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at), P_GEMM_DGRAD));
+        // attention: x_mid = x_in + o Wo^T; dO = dx Wo, with the softmax-backward statistics
+        // D = rowsum(dO * o) and lse*log2(e) formed in the same GEMM's epilogue (tensor-core path)
+        bool stats_ready = false;
+        if (fuse_stats) {
+            GemmDesc gd = mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_ATTN_DO, dO, Hhd, m->at);
+            gd.aux = lb + c.p.l_o; gd.ldaux = Hhd;
+            gd.hd = m->hd; gd.T = T; gd.attn_H = m->H;
+            gd.attn_d = Dbuf; gd.attn_lse2 = Dbuf + attn_stat_elems(B, T, m->H);
+            gd.attn_lse = (const float*)(lb + c.p.l_lse);
+            RG(run_gemm_tc(c, gd, P_GEMM_DGRAD));
+            stats_ready = true;
+        } else {
+            RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at),
+                        P_GEMM_DGRAD));
+        }
         RG(run_gemm(c, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
                           DT_F32), P_GEMM_WGRAD));
         RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), (float*)(lb + c.p.l_rqk),
-                         dqkv));
+                         dqkv, stats_ready));
         RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, DT_F32),
                     P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, Nqkv, d, M, dqkv, Nqkv, false, lb + c.p.l_a, d, false, EPI_STORE, G(base), d,
