@@ -472,8 +472,6 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     // padding of the last query block past T stays zero for the whole backward
     const bool fuse_stats = m->tc && attention_tc_bwd_supported(m->hd);
     if (fuse_stats && T % 128 != 0) CK(cudaMemsetAsync(Dbuf, 0, 4 * attn_dbuf_elems(B, T, m->H), s));
-    const float* cs = c.at<float>(c.p.cosb);
-    const float* sn = c.at<float>(c.p.sinb);
     for (int l = m->L - 1; l >= 0; --l) {
         char* lb = c.layer(l);
         int base = 1 + 6 * l;
