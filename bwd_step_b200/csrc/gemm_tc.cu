@@ -15,9 +15,8 @@
 // Two 256-column accumulators let the epilogue of one tile overlap the main
 // loop of the next.  Operands may be K-major or M/N-major (the backward
 // products read activations and weights transposed without a copy).
-// Split-K is used when there are too few output tiles to fill the SMs: the
-// last split to finish a 32-row slice of a tile adds the partials in split
-// order (deterministic, no reduction kernel).  Every mbarrier wait is bounded.
+// Split-K (fixed order, deterministic reduction) is used when there are too
+// few output tiles to fill the SMs.  Every mbarrier wait is bounded.
 #include "gemm_tc.h"
 #include "tc_common.cuh"
 #include <cudaTypedefs.h>
@@ -45,8 +44,7 @@ struct TcParams {
     void* C2; int64_t ldc2;
     const bf16* aux; int64_t ldaux;
     float cap;
-    float* part;    // split-K partial sums [splits][M][N], or null
-    int* counters;  // split-K arrivals per (tile, 32-row slice), zero before the launch
+    float* part;  // split-K partial sums [splits][M][N], or null
     int* status;
     int hd, T, qk_heads;
     float* rqk;
@@ -139,55 +137,6 @@ __device__ __forceinline__ void lmhead_chunk(const TcParams& p, int row, int n0,
         v[i] = e * (1.f - t * t);
     }
     rc.sum += sum;
-}
-
-// Split-K completion of one 32-row slice of an output tile: every split
-// writes its partial rows, then counts itself in; the split that arrives last
-// (whichever it is) adds the partials in split order 0, 1, ... -- onto C for
-// the residual-add epilogue -- and writes C, so the result does not depend on
-// the arrival order.  The partials are read back right after they are written
-// (from L2), and no separate reduction kernel runs.
-constexpr int kSlicesPerTile = 8;  // 256 rows of a CTA-pair tile / 32 (a 128-row tile uses 4)
-
-__device__ __forceinline__ void splitk_finish(const TcParams& p, int tile, int slice, int row, int tn, int lane) {
-    __threadfence();  // this lane's partial row is visible device-wide ...
-    __syncwarp();     // ... before lane 0 counts the warp in
-    int old = 0;
-    if (lane == 0) old = atomicAdd(p.counters + tile * kSlicesPerTile + slice, 1);
-    old = __shfl_sync(0xffffffffu, old, 0);
-    if (old != p.splits - 1) return;
-    __threadfence();  // every split's partial rows of this slice are visible
-    if (row < p.M) {
-        float* crow = reinterpret_cast<float*>(p.C) + (size_t)row * p.N;
-        const float rsr = p.epi == EPI_ROWSCALE ? p.rs[row] : 1.f;
-        for (int c = 0; c < BN / 32; ++c) {
-            const int n0 = tn * BN + c * 32;
-            if (n0 >= p.N) break;
-            const int nv = min(32, p.N - n0);
-            if (nv == 32) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    float4 a = p.epi == EPI_ACCUM ? __ldcg(reinterpret_cast<const float4*>(crow + n0) + q)
-                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int ks = 0; ks < p.splits; ++ks) {
-                        const float4 g = __ldcg(reinterpret_cast<const float4*>(
-                                                    p.part + ((size_t)ks * p.M + row) * p.N + n0) + q);
-                        a.x += g.x; a.y += g.y; a.z += g.z; a.w += g.w;
-                    }
-                    if (p.epi == EPI_ROWSCALE) { a.x *= rsr; a.y *= rsr; a.z *= rsr; a.w *= rsr; }
-                    reinterpret_cast<float4*>(crow + n0)[q] = a;
-                }
-            } else {
-                for (int i = 0; i < nv; ++i) {
-                    float a = p.epi == EPI_ACCUM ? __ldcg(crow + n0 + i) : 0.f;
-                    for (int ks = 0; ks < p.splits; ++ks) a += __ldcg(p.part + ((size_t)ks * p.M + row) * p.N + n0 + i);
-                    crow[n0 + i] = p.epi == EPI_ROWSCALE ? a * rsr : a;
-                }
-            }
-        }
-    }
-    __syncwarp();
-    if (lane == 0) p.counters[tile * kSlicesPerTile + slice] = 0;  // ready for the next launch
 }
 
 __device__ __forceinline__ void decode(const TcParams& p, int u, int& tm, int& tn, int& ks) {
@@ -325,8 +274,8 @@ __device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUte
         if (lane == 0) bulk_wait_read_1();
         __syncwarp();
     }
-    const int mode = p.epi;
-    const bool bf = p.c_bf16 != 0;
+    const int mode = p.part ? EPI_STORE : p.epi;
+    const bool bf = p.part ? false : p.c_bf16 != 0;
     if (mode == EPI_RELU2) {
         float r[32];
 #pragma unroll
@@ -368,7 +317,8 @@ __device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUte
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-        if (mode == EPI_ACCUM) tma_reduce_add_2d(tmC, n0, row0w, smem_u32(buf));
+        if (p.part) tma_store_3d(tmC, n0, row0w, ks, smem_u32(buf));  // [splits, M, N]: clipped at M per split
+        else if (mode == EPI_ACCUM) tma_reduce_add_2d(tmC, n0, row0w, smem_u32(buf));
         else tma_store_2d(tmC, n0, row0w, smem_u32(buf));
         if (mode == EPI_RELU2) tma_store_2d(tmC2, n0, row0w, smem_u32(buf + 2048));
         bulk_commit();
@@ -570,7 +520,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_tempty + 8 * acc);
-            if (p.part) splitk_finish(p, tm * p.tiles_n + tn, q, row, tn, lane);
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
         if (lane == 0) bulk_wait_all();  // staged stores finished before the block exits
@@ -731,7 +680,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_addr(bar_tempty + 8 * acc));
-            if (p.part) splitk_finish(p, tm * p.tiles_n + tn, (int)rank * 4 + q, row, tn, lane);
             if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
         if (lane == 0) bulk_wait_all();  // staged stores finished before the block exits
@@ -772,6 +720,19 @@ bool make_out_map(CUtensorMap* map, void* base, bool bf16, uint64_t cols, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Same for the split-K partial sums, fp32 [splits, rows, cols] contiguous.
+bool make_partial_map(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows, uint64_t splits) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cols, rows, splits};
+    cuuint64_t strides[2] = {cols * 4, cols * rows * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D bf16 tensor map over a row-major [outer, inner] array with row stride ld
 // elements; box [box_outer, box_inner], 128-byte swizzle, zero fill out of range.
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld, uint32_t box_inner,
@@ -792,13 +753,7 @@ int num_sms() { return device_sm_count(); }
 
 }  // namespace
 
-// Split-K scratch: the arrival counters, then the partial sums.
-constexpr size_t kCounterBytes = 64 << 10;
-constexpr int kMaxCounters = (int)(kCounterBytes / sizeof(int));
-
-size_t gemm_tc_splitk_bytes(size_t max_out_elems) {
-    return kCounterBytes + (size_t)MAX_SPLITS * max_out_elems * sizeof(float);
-}
+size_t gemm_tc_splitk_bytes(size_t max_out_elems) { return (size_t)MAX_SPLITS * max_out_elems * sizeof(float); }
 
 int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s) {
     if (g.in_t != DT_BF16) return 1;
@@ -862,19 +817,18 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     // the split-K completion reads and writes C as float4: C must be 16-byte aligned
     const bool can_split = (g.epi == EPI_STORE || g.epi == EPI_ACCUM || g.epi == EPI_ROWSCALE) && !p.c_bf16 &&
                            g.ldc == g.N && splitk && g.N % 4 == 0 && al16(g.C);
-    if (can_split && tiles < 2 * sms && tiles * kSlicesPerTile <= kMaxCounters && splitk_bytes > kCounterBytes) {
+    if (can_split && tiles < 2 * sms) {
         double best = (double)((tiles + sms - 1) / sms);
         for (int sp = 2; sp <= MAX_SPLITS; ++sp) {
             if (p.num_kb / sp < 8) break;
-            if ((size_t)sp * g.M * g.N * sizeof(float) > splitk_bytes - kCounterBytes) break;
+            if ((size_t)sp * g.M * g.N * sizeof(float) > splitk_bytes) break;
             double cost = (double)((tiles * sp + sms - 1) / sms) / sp;
             if (cost < best - 1e-9) { best = cost; splits = sp; }
         }
     }
     p.kb_per_split = (p.num_kb + splits - 1) / splits;
     p.splits = (p.num_kb + p.kb_per_split - 1) / p.kb_per_split;
-    p.part = p.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(splitk) + kCounterBytes) : nullptr;
-    p.counters = p.splits > 1 ? static_cast<int*>(splitk) : nullptr;
+    p.part = p.splits > 1 ? reinterpret_cast<float*>(splitk) : nullptr;
     p.vec_ok = (p.part ? (g.N % 4 == 0) : vec) ? 1 : 0;
     p.num_units = tiles * p.splits;
     // staged (TMA) epilogue for the plain, residual-add, relu^2 (both outputs),
@@ -884,8 +838,7 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     memset(&tc_out2, 0, sizeof(tc_out2));
     p.tma_out = 0;
     if (p.part) {
-        // partial rows are written with plain stores and summed by the last split (splitk_finish)
-        if (cudaMemsetAsync(p.counters, 0, (size_t)tiles * kSlicesPerTile * sizeof(int), s) != cudaSuccess) return -1;
+        if (make_partial_map(&tc_out, p.part, g.N, g.M, p.splits)) p.tma_out = 1;
     } else if (vec && g.epi != EPI_QKROPE) {
         const bool bf = p.c_bf16 != 0;
         if (g.epi == EPI_ACCUM && bf) {
@@ -900,6 +853,12 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     else gemm_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, s>>>(ta, tb, tc_out, tc_out2, p);
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return -1;
+    if (p.part) {
+        // the partials in split order (deterministic), then the row scale of EPI_ROWSCALE
+        if (launch_splitk_reduce(p.part, p.splits, (size_t)g.M * g.N, reinterpret_cast<float*>(g.C),
+                                 g.epi == EPI_ACCUM, g.epi == EPI_ROWSCALE ? g.rs : nullptr, g.N, s) != cudaSuccess)
+            return -1;
+    }
     return 0;
 }
 

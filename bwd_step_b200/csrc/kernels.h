@@ -83,6 +83,11 @@ EmbedScratch embed_scratch_carve(void* base, int M, int V, int d);
 // rows of unused ids are zero.  Deterministic.
 cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int V, int d, float* dwte,
                                  EmbedScratch sc, cudaStream_t s);
+// out[i] = ((accumulate ? out[i] : 0) + sum_{s < splits} part[s*n + i]) * (rs ? rs[i / N] : 1),
+// in increasing s (N = row length, a multiple of 4).
+cudaError_t launch_splitk_reduce(const float* part, int splits, size_t n, float* out, bool accumulate,
+                                 const float* rs, int N, cudaStream_t s);
+
 // ---------------------------------------------------------------- GEMM
 // C[m,n] = sum_k A(m,k) * B(n,k).
 //   A(m,k) = a_kmajor ? A[m*lda + k] : A[k*lda + m]

@@ -960,6 +960,38 @@ __global__ void emb_zero_unused_kernel(const int* __restrict__ count, int V, int
     if (count[i / d4] == 0) reinterpret_cast<float4*>(dwte)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// out[i] = ((accumulate ? out[i] : 0) + sum_s part[s][i]) * (rs ? rs[i / N] : 1),
+// partials added in split order; up to eight of them loaded at once.
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, size_t n4,
+                                     float* __restrict__ out, bool accumulate, const float* __restrict__ rs,
+                                     int N4) {
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const float4* p = reinterpret_cast<const float4*>(part) + i;
+    float4 acc = accumulate ? reinterpret_cast<float4*>(out)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    constexpr int KMAX = 8;
+    float4 g[KMAX];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k)
+        if (k < splits) g[k] = p[(size_t)k * n4];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k)
+        if (k < splits) { acc.x += g[k].x; acc.y += g[k].y; acc.z += g[k].z; acc.w += g[k].w; }
+    for (int k = KMAX; k < splits; ++k) {
+        const float4 h = p[(size_t)k * n4];
+        acc.x += h.x; acc.y += h.y; acc.z += h.z; acc.w += h.w;
+    }
+    if (rs) {
+        const float f = rs[i / N4];
+        acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
+    }
+    reinterpret_cast<float4*>(out)[i] = acc;
+}
+
+// ---------------------------------------------------------------- bounded wait
+// Waits on an mbarrier that nobody arrives at; each try_wait is bounded by
+// the hardware's time limit and the loop by max_iters.  On expiry it records
+// ST_TIMEOUT and returns.
 __global__ void expired_wait_kernel(int* status, int max_iters) {
     __shared__ __align__(8) uint64_t bar;
     uint32_t addr = (uint32_t)__cvta_generic_to_shared(&bar);
@@ -1278,6 +1310,14 @@ cudaError_t launch_embed_scatter(const int32_t* idx, const float* de, int M, int
     size_t n4 = (size_t)V * (d / 4);
     emb_zero_unused_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(sc.count, V, d / 4, dwte);
     count_launch(11);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_splitk_reduce(const float* part, int splits, size_t n, float* out, bool accumulate,
+                                 const float* rs, int N, cudaStream_t s) {
+    size_t n4 = n / 4;
+    splitk_reduce_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(part, splits, n4, out, accumulate, rs, N / 4);
+    count_launch();
     return cudaGetLastError();
 }
 

@@ -286,14 +286,13 @@ int nc_set_recompute(nc_model* m, int flags);
  * multiples of 8 (16-byte rows); otherwise the call returns
  * NC_ERR_INVALID_ARG before anything is launched.
  *
- * Split-K counters and partial sums live in one file-scope static device array of
+ * Split-K partial sums live in one file-scope static device array of
  * NC_WGRAD_NOALLOC_SCRATCH_BYTES; every GPU that loads the library holds it
  * until the process exits.  Results of shape n_out * n_in * 4 * 2 bytes
  * larger than that array (room for two partials) are rejected with
  * NC_ERR_UNSUPPORTED_SHAPE.  Every call shares the array and it keeps the
- * last call's contents; each call clears the split-K arrival counters at the
- * start of the array (cudaMemsetAsync on the array, no allocation) and
- * overwrites every partial it reads, so nothing has to start at zero.  Calls that overlap on the GPU (other
+ * last call's contents; each call overwrites every partial it reads, so
+ * nothing has to start at zero.  Calls that overlap on the GPU (other
  * streams, other host threads) race on the array: serialise them.  The first
  * call on a device looks up the array's device address with
  * cudaGetSymbolAddress (with that device current); make that first call
