@@ -23,9 +23,9 @@
 //              rescaling of O (only when the max grows by more than 2^8),
 //              P stored as packed bf16; then the normalised output and the
 //              log-sum-exp of the unit.
-// 2^x is taken from the special-function unit (ex2) for three of every four
-// scores and from a cubic on the FMA pipe for the fourth, so that the two
-// units share the work of the exponentials.
+// 2^x is taken from the special-function unit (ex2), except for one score in
+// kPolyEvery of the full blocks, which takes a cubic on the FMA pipe, so that
+// the two units share the work of the exponentials.
 #include "attention_tc.h"
 #include "tc_common.cuh"
 #include <cudaTypedefs.h>
@@ -37,6 +37,9 @@ namespace {
 using namespace tc;
 
 constexpr int NT = 320;  // forward: producer, MMA, 2 x 4 softmax warps
+// One score in kPolyEvery (even, or 0 for none) of the forward's full blocks takes
+// 2^x from the FMA pipe (exp2_fma) instead of the special-function unit.
+constexpr int kPolyEvery = 8;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
@@ -85,6 +88,16 @@ __device__ __forceinline__ void tmem_st32u_nowait(uint32_t taddr, const uint32_t
 __device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
     uint64_t t0 = globaltimer();
     while (!mbar_try(bar, parity) && globaltimer() - t0 < 1000000ull) {}
+}
+
+// Store 16 consecutive 32-bit columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_st16_nowait(uint32_t taddr, const uint32_t* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
 }
 
 // 2^x on the FMA pipe, for x >= -126 (smaller x give a value below 2^-125):
@@ -316,55 +329,70 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 ++scnt;
                 tc_fence_after();
                 const bool diag = j == qb;  // key c of the diagonal block is visible from row r iff c <= r
-                // pass 1: the row maximum (scores read from TMEM 64 columns at a time)
-                float mx = -INFINITY;
+                // pass 1: the row maximum (scores read from TMEM 64 columns at a time),
+                // as eight independent partial maxima (no 128-long dependency chain)
+                float mx8[8];
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t s[64];
-                    tmem_ld32_issue(tS + 64 * hf, s);
-                    tmem_ld32_issue(tS + 64 * hf + 32, s + 32);
-                    tmem_wait_ld();
+                for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+                auto row_max = [&](auto dg) {
+                    constexpr bool kDiag = decltype(dg)::value;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        mx = fmaxf(mx, (diag && 64 * hf + c > r) ? -INFINITY : __uint_as_float(s[c]));
-                }
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t s[32];
+                        tmem_ld32_issue(tS + 32 * q4, s);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            mx8[c & 7] = fmaxf(mx8[c & 7], (kDiag && 32 * q4 + c > r) ? -INFINITY : __uint_as_float(s[c]));
+                    }
+                };
+                if (diag) row_max(std::true_type{});
+                else row_max(std::false_type{});
+                float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
                 mx *= p.scale_log2;
                 const bool rescale = mx > m + 8.f;
                 const float mu = rescale ? mx : m;
                 const float alpha = rescale ? ex2(m - mx) : 1.f;
-                float sum = 0.f;
                 // pass 2: P = 2^(s*scale - mu) as packed bf16 over the first 64 score
-                // columns (the scores of each half are read before they are overwritten);
-                // with kPoly one score in four comes from the FMA pipe (full blocks only:
-                // exp2_fma does not take the masked -inf scores of the diagonal block)
+                // columns (the scores of each half are read before they are overwritten),
+                // the row sum as eight independent partial sums; with kPoly one score in
+                // kPolyEvery comes from the FMA pipe (full blocks only: exp2_fma does not
+                // take the masked -inf scores of the diagonal block)
+                float sum8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
                 auto exp_pack = [&](auto poly) {
                     constexpr bool kPoly = decltype(poly)::value;
+                    constexpr int kPE = kPolyEvery > 0 ? kPolyEvery : 2;
+                    // 32 scores at a time; their packed P (16 columns) lands on columns
+                    // already read (16 q4 + 15 < 32 q4 for q4 >= 1, and the chunk itself for q4 = 0)
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        uint32_t s[64];
-                        tmem_ld32_issue(tS + 64 * hf, s);
-                        tmem_ld32_issue(tS + 64 * hf + 32, s + 32);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t s[32];
+                        tmem_ld32_issue(tS + 32 * q4, s);
                         tmem_wait_ld();
-                        uint32_t pk[32];
+                        uint32_t pk[16];
 #pragma unroll
-                        for (int c = 0; c < 64; c += 2) {
+                        for (int c = 0; c < 32; c += 2) {
                             float x0 = fmaf(__uint_as_float(s[c]), p.scale_log2, -mu);
                             float x1 = fmaf(__uint_as_float(s[c + 1]), p.scale_log2, -mu);
                             if (!kPoly && diag) {
-                                if (64 * hf + c > r) x0 = -INFINITY;
-                                if (64 * hf + c + 1 > r) x1 = -INFINITY;
+                                if (32 * q4 + c > r) x0 = -INFINITY;
+                                if (32 * q4 + c + 1 > r) x1 = -INFINITY;
                             }
                             const float e0 = ex2(x0);
-                            const float e1 = (kPoly && (c & 2)) ? exp2_fma(x1) : ex2(x1);
-                            sum += e0 + e1;
+                            const float e1 = (kPoly && (c / 2) % (kPE / 2) == kPE / 2 - 1) ? exp2_fma(x1) : ex2(x1);
+                            sum8[(c >> 1) & 7] += e0 + e1;
                             pk[c >> 1] = pack_bf16(e0, e1);
                         }
-                        tmem_st32u_nowait(tS + 32 * hf, pk);
+                        tmem_st16_nowait(tS + 16 * q4, pk);
                     }
                 };
-                if (!diag) exp_pack(std::true_type{});
+                if (!diag && kPolyEvery > 0) exp_pack(std::true_type{});
                 else exp_pack(std::false_type{});
                 tmem_wait_st();
+                const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
                 if (j > 0 && __any_sync(0xffffffffu, rescale)) {
                     // O_x += P(j-1) V has completed (S(j) was issued after it and has landed);
                     // O_x += P(j) V waits for this warp's hand-over below
@@ -432,7 +460,7 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 // dP^T columns they have just read, and the dV MMA reads it there as the A
 // operand.  Sixteen softmax warps (four per TMEM lane quarter, 32 columns
 // each) keep the special-function unit busy.
-constexpr int NTB = 576;  // dK/dV: producer, MMA, 16 softmax warps
+constexpr int NTB = 608;  // dK/dV: producer, MMA, 16 softmax warps, dS store
 constexpr int NSM = 16;   // softmax warps
 
 struct BwdParams {
@@ -792,6 +820,7 @@ struct DkvLayout {
 template <int HD>
 __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
                                                             const __grid_constant__ CUtensorMap tmDO,
+                                                            const __grid_constant__ CUtensorMap tmDS,
                                                             const BwdParams p) {
     using Lay = DkvLayout<HD>;
     constexpr int KB = Lay::KB, TILE = Lay::TILE;
@@ -811,7 +840,8 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
     const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24;  // qo_*[2]
     const uint32_t st_full = b0 + 40, dpt_full = b0 + 48, st_free = b0 + 56;
     const uint32_t p_full = b0 + 64, ds_full = b0 + 72, ds_free = b0 + 80, dkv_done = b0 + 88;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+    const uint32_t dst_read = b0 + 96;  // the dS^T tile has been read out of shared memory by its store
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -832,6 +862,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         mbar_init(ds_full, NSM);
         mbar_init(ds_free, 1);
         mbar_init(dkv_done, 1);
+        mbar_init(dst_read, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -943,6 +974,22 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             }
             mma_commit(dkv_done);
         }
+    } else if (warp == 2 + NSM) {
+        // one thread writes every finished dS^T tile to global memory (two TMA stores
+        // of [128 keys][64 queries]) and reports when shared memory may be reused
+        if (lane == 0) {
+            for (int u = 0; u < nunits; ++u) {
+                const int i = p.nqb - 1 - u / Hg, h = g * Hg + u % Hg;
+                if (!mbar_wait(ds_full, u & 1, abort_flag, p.status)) break;
+                const int trow = (int)(ds_tile(b, h, p.H, p.ntri, i, kvb) * 128);
+                tma_store_2d(&tmDS, 0, trow, sDST);
+                tma_store_2d(&tmDS, 64, trow, sDST + 16384);
+                bulk_commit();
+                bulk_wait_read_0();
+                mbar_arrive(dst_read);
+            }
+            bulk_wait_all();  // the tiles are in global memory before the block exits
+        }
     } else {
         // warps 2..17: TMEM lane quarter q (key rows), query column group cg (32 queries)
         const int q = warp & 3, cg = (warp - 2) >> 2;
@@ -1028,13 +1075,10 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                 dsv[k] = make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
                                     pack_bf16(d[6], d[7]));
             }
-            // this row's 32 queries of the dS^T tile, for the dQ product
-            uint4* gds = reinterpret_cast<uint4*>(p.ds + (ds_tile(b, h, p.H, p.ntri, i, kvb) * 128 + r) * 128 +
-                                                  cg * 32);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) gds[k] = dsv[k];
-            // the dK MMAs of the previous unit have read the dS^T tile
-            if (u > 0 && !warp_wait(ds_free, (u - 1) & 1, abort_flag, p.status)) {
+            // the dK MMAs of the previous unit and the store of its tile to global
+            // memory (for the dQ product) have read the dS^T tile
+            if (u > 0 && (!warp_wait(ds_free, (u - 1) & 1, abort_flag, p.status) ||
+                          !warp_wait(dst_read, (u - 1) & 1, abort_flag, p.status))) {
                 ok = false;
                 break;
             }
@@ -1152,9 +1196,10 @@ int dq_ds_launch(const CUtensorMap& ds, const CUtensorMap& kv, const DqdsParams&
 }
 
 template <int HD>
-int dkv_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
+int dkv_launch(const CUtensorMap& kv, const CUtensorMap& do128, const CUtensorMap& ds, const BwdParams& p,
+               cudaStream_t s) {
     if (ensure_smem_limit((const void*)attn_dkv_tc_kernel<HD>, DkvLayout<HD>::BYTES) != cudaSuccess) return -1;
-    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NTB, DkvLayout<HD>::BYTES, s>>>(kv, do128, p);
+    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NTB, DkvLayout<HD>::BYTES, s>>>(kv, do128, ds, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -1241,7 +1286,9 @@ int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqk
         p.qkv = reinterpret_cast<const bf16*>(qkv);
         p.rqk = qk->rqk; p.cos_t = qk->cos_t; p.sin_t = qk->sin_t;
     }
-    return hd == 128 ? dkv_launch<128>(kv, do128, p, s) : dkv_launch<64>(kv, do128, p, s);
+    CUtensorMap mds;
+    if (!map_rows(&mds, ws, 128, (uint64_t)B * H * ntri_of(T) * 128, 128)) return 1;
+    return hd == 128 ? dkv_launch<128>(kv, do128, mds, p, s) : dkv_launch<64>(kv, do128, mds, p, s);
 }
 
 int attention_tc_bwd_dq(const void* qkv, const void* ws, size_t ws_bytes, void* dqkv, int B, int T, int H, int nkv,
