@@ -115,6 +115,15 @@ __device__ __forceinline__ RowCtx row_ctx(const TcParams& p, int row) {
 // [exp(-2 cap), 1] and needs no running maximum; v becomes
 // u = e (1 - (z/cap)^2), the product of the unnormalised softmax and the
 // softcap's derivative.  The logits themselves are never stored.
+// tanh on the special-function unit (PTX tanh.approx.f32: one instruction,
+// relative error about 2^-11, i.e. |dz| <= 0.01 at cap 15 -- below the bf16
+// rounding of a stored logit).  Used by the fused LM head only.
+__device__ __forceinline__ float tanh_sfu(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void lmhead_chunk(const TcParams& p, int row, int n0, float* v, RowCtx& rc) {
     constexpr float kL2e = 1.44269504088896340736f;
     const float ic = 1.f / p.cap, cl2 = p.cap * kL2e;
@@ -122,7 +131,7 @@ __device__ __forceinline__ void lmhead_chunk(const TcParams& p, int row, int n0,
 #pragma unroll
         for (int i = 0; i < 32; ++i)
             if (n0 + i == rc.tgt) {
-                const float t = tanhf(v[i] * ic);
+                const float t = tanh_sfu(v[i] * ic);
                 p.zt[row] = p.cap * t;
                 p.ut[row] = ex2((t - 1.f) * cl2) * (1.f - t * t);
             }
@@ -131,7 +140,7 @@ __device__ __forceinline__ void lmhead_chunk(const TcParams& p, int row, int n0,
     float sum = 0.f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-        const float t = tanhf(v[i] * ic);
+        const float t = tanh_sfu(v[i] * ic);
         const float e = ex2((t - 1.f) * cl2);
         if (i < nv) sum += e;
         v[i] = e * (1.f - t * t);
