@@ -790,16 +790,17 @@ __global__ void __launch_bounds__(NTQ, 1) attn_dq_ds_kernel(const __grid_constan
 //   warp 0      TMA: K and V once; Q_i, dO_i with their lse2 / D rows into a
 //               2-stage ring;
 //   warp 1      tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM,
-//               dV += P^T dO_i with P^T read from TMEM, dK += dS^T Q_i with
-//               dS^T from shared memory (Q_i, dO_i as MN-major operands),
-//               in the order dV_u, S^T_{u+1}, dP^T_{u+1}, dK_u (the Q / dO
-//               tiles of unit u+1 land while P^T_u is formed; those of the
-//               unit after are prefetched into L2);
-//   warps 2-17  per unit: load the warp's S^T columns (32 queries), release
-//               S^T, form P^T = 2^(S^T*scale*log2e - lse2) with the causal
-//               mask, load the dP^T columns and store P^T as packed bf16 over
-//               the warp's own dP^T columns, then dS^T = P^T (dP^T - D) into
-//               shared memory.
+//               dV += P^T dO_i and dK += dS^T Q_i with P^T, then dS^T, in one
+//               shared-memory tile X (Q_i, dO_i as MN-major operands).  The
+//               next unit's S^T and dP^T are issued as soon as the softmax warps
+//               have read this unit's into registers, so they overlap this
+//               unit's softmax: S^T_{u+1}, dV_u, dP^T_{u+1}, dK_u;
+//   warps 2-17  per unit: load the warp's S^T columns (32 queries), form
+//               P^T = 2^(S^T*scale*log2e - lse2) with the causal mask, write it
+//               to X, load the dP^T columns, form dS^T = P^T (dP^T - D) and
+//               write it to X once dV_u has read P^T;
+//   warp 18     TMA-stores each finished dS^T tile to global memory (for the dQ
+//               product) and reports when X may be reused.
 // dk = dK / sqrt(hd).
 template <int HD>
 struct DkvLayout {
@@ -809,8 +810,8 @@ struct DkvLayout {
     static constexpr int V = K + TILE;
     static constexpr int Q = V + TILE;         // [2] stages
     static constexpr int DO = Q + 2 * TILE;    // [2] stages
-    static constexpr int DST = DO + 2 * TILE;  // dS^T [128 keys x 128 queries] bf16, two 64-query boxes
-    static constexpr int LSE = DST + 32768;    // [2][128] fp32 lse2 of the stage's queries
+    static constexpr int X = DO + 2 * TILE;    // P^T, then dS^T [128 keys x 128 queries] bf16, two 64-query boxes
+    static constexpr int LSE = X + 32768;      // [2][128] fp32 lse2 of the stage's queries
     static constexpr int DD = LSE + 1024;      // [2][128] fp32 D
     static constexpr int BAR = DD + 1024;
     static constexpr int BYTES = BAR + 256;  // the dynamic shared memory base is 1024-aligned (checked)
@@ -832,16 +833,19 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
     uint8_t* smem = smem_dyn;
     const uint32_t base = smem_u32(smem);
     const uint32_t sK = base + Lay::K, sV = base + Lay::V, sQ = base + Lay::Q, sDO = base + Lay::DO;
-    const uint32_t sDST = base + Lay::DST;
+    const uint32_t sX = base + Lay::X;
     const float* lse_s = reinterpret_cast<const float*>(smem + Lay::LSE);
     const float* d_s = reinterpret_cast<const float*>(smem + Lay::DD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24;  // qo_*[2]
-    const uint32_t st_full = b0 + 40, dpt_full = b0 + 48, st_free = b0 + 56;
-    const uint32_t p_full = b0 + 64, ds_full = b0 + 72, ds_free = b0 + 80, dkv_done = b0 + 88;
-    const uint32_t dst_read = b0 + 96;  // the dS^T tile has been read out of shared memory by its store
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+    const uint32_t s_full = b0 + 40, dp_full = b0 + 48;    // S^T / dP^T of the unit in TMEM
+    const uint32_t s_free = b0 + 56, dp_free = b0 + 64;    // ... read by the softmax warps
+    const uint32_t p_full = b0 + 72, pv_done = b0 + 80;    // P^T in X / read by the dV MMAs
+    const uint32_t ds_full = b0 + 88, dk_done = b0 + 96;   // dS^T in X / read by the dK MMAs
+    const uint32_t dst_read = b0 + 104;                    // dS^T read out of X by its store
+    const uint32_t dkv_done = b0 + 112;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -855,14 +859,16 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
         for (int s = 0; s < 2; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
-        mbar_init(st_full, 1);
-        mbar_init(dpt_full, 1);
-        mbar_init(st_free, NSM);
+        mbar_init(s_full, 1);
+        mbar_init(dp_full, 1);
+        mbar_init(s_free, NSM);
+        mbar_init(dp_free, NSM);
         mbar_init(p_full, NSM);
+        mbar_init(pv_done, 1);
         mbar_init(ds_full, NSM);
-        mbar_init(ds_free, 1);
-        mbar_init(dkv_done, 1);
+        mbar_init(dk_done, 1);
         mbar_init(dst_read, 1);
+        mbar_init(dkv_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -919,7 +925,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);
             const uint32_t id_kv = idesc_bf16(128, HD, false, true);
-            // S^T_u = K Q_u^T
+            // S^T_u = K Q_u^T (waits for the unit's Q / dO stage)
             auto scores = [&](int u) -> bool {
                 const int st = u & 1;
                 if (!mbar_wait(qo_full + 8 * st, (u >> 1) & 1, abort_flag, p.status)) return false;
@@ -930,7 +936,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                     mma_bf16(tSt, smem_desc(sK + off, 16, 1024), smem_desc(sQ + st * TILE + off, 16, 1024), id_s,
                              ks > 0 ? 1u : 0u);
                 }
-                mma_commit(st_full);
+                mma_commit(s_full);
                 return true;
             };
             // dP^T_u = V dO_u^T (Q_u / dO_u already landed)
@@ -942,34 +948,39 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                     mma_bf16(tdPt, smem_desc(sV + off, 16, 1024), smem_desc(sDO + st * TILE + off, 16, 1024), id_s,
                              ks > 0 ? 1u : 0u);
                 }
-                mma_commit(dpt_full);
+                mma_commit(dp_full);
+            };
+            // acc (+)= X Bop^T over the 128 queries of the unit: X = P^T or dS^T [keys x queries]
+            // (K-major, two 64-query boxes), Bop = dO_u or Q_u as an MN-major operand
+            auto x_product = [&](uint32_t acc, uint32_t bop, int u) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(acc, smem_desc(sX + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                             smem_desc(bop + kk * 2048, 16384, 1024), id_kv, (u > 0 || kk > 0) ? 1u : 0u);
             };
             bool ok = mbar_wait(kv_full, 0, abort_flag, p.status) && scores(0);
             if (ok) dpt(0);
             for (int u = 0; ok && u < nunits; ++u) {
                 const int st = u & 1;
-                // dV += P^T_u dO_u: queries 16kk..16kk+15 sit in the packed columns
-                // 32*(kk/2) + 8*(kk%2) of dP^T (written by column group kk/2)
+                const bool more = u + 1 < nunits;
+                // S^T of the next unit once this unit's S^T is in registers
+                if (more && (!mbar_wait(s_free, u & 1, abort_flag, p.status) || !scores(u + 1))) break;
+                // dV += P^T_u dO_u
                 if (!mbar_wait(p_full, u & 1, abort_flag, p.status)) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tdV, tdPt + 32 * (kk >> 1) + 8 * (kk & 1),
-                                smem_desc(sDO + st * TILE + kk * 2048, 16384, 1024), id_kv,
-                                (u > 0 || kk > 0) ? 1u : 0u);
-                // the next unit's scores (its Q / dO tiles are loaded by now), then its
-                // dP^T, which overwrites P^T only after the dV MMAs (issue order)
-                if (u + 1 < nunits) {
-                    if (!mbar_wait(st_free, u & 1, abort_flag, p.status) || !scores(u + 1)) break;
+                x_product(tdV, sDO + st * TILE, u);
+                mma_commit(pv_done);
+                // dP^T of the next unit once this unit's dP^T is in registers
+                if (more) {
+                    if (!mbar_wait(dp_free, u & 1, abort_flag, p.status)) break;
+                    tc_fence_after();
                     dpt(u + 1);
                 }
+                // dK += dS^T_u Q_u
                 if (!mbar_wait(ds_full, u & 1, abort_flag, p.status)) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tdK, smem_desc(sDST + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                             smem_desc(sQ + st * TILE + kk * 2048, 16384, 1024), id_kv, (u > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(ds_free);
+                x_product(tdK, sQ + st * TILE, u);
+                mma_commit(dk_done);
                 mma_commit(qo_empty + 8 * st);
             }
             mma_commit(dkv_done);
@@ -982,8 +993,8 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                 const int i = p.nqb - 1 - u / Hg, h = g * Hg + u % Hg;
                 if (!mbar_wait(ds_full, u & 1, abort_flag, p.status)) break;
                 const int trow = (int)(ds_tile(b, h, p.H, p.ntri, i, kvb) * 128);
-                tma_store_2d(&tmDS, 0, trow, sDST);
-                tma_store_2d(&tmDS, 64, trow, sDST + 16384);
+                tma_store_2d(&tmDS, 0, trow, sX);
+                tma_store_2d(&tmDS, 64, trow, sX + 16384);
                 bulk_commit();
                 bulk_wait_read_0();
                 mbar_arrive(dst_read);
@@ -1000,7 +1011,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         for (int u = 0; u < nunits; ++u) {
             const int st = u & 1;
             const int i = p.nqb - 1 - u / Hg, h = g * Hg + u % Hg;
-            if (!warp_wait(st_full, u & 1, abort_flag, p.status) ||
+            if (!warp_wait(s_full, u & 1, abort_flag, p.status) ||
                 !warp_wait(qo_full + 8 * st, (u >> 1) & 1, abort_flag, p.status)) {
                 ok = false;
                 break;
@@ -1011,7 +1022,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(st_free);
+            if (lane == 0) mbar_arrive(s_free);
             // query q0 + e sees this key when lo <= e (causal) and e <= hi (inside the row)
             const int q0 = i * 128 + cg * 32;
             const int lo = kpos - q0, hi = p.T - 1 - q0;
@@ -1038,7 +1049,30 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                     }
                 }
             }
-            if (!warp_wait(dpt_full, u & 1, abort_flag, p.status)) {
+            // this warp's 32 queries of row r in the swizzled [128 keys x 64 queries] boxes of X
+            uint8_t* xrow = smem + Lay::X + (cg >> 1) * 16384 + r * 128;
+            auto put_x = [&](const float* v) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float* d = v + 8 * k;
+                    const int c8 = (cg & 1) * 4 + k;
+                    *reinterpret_cast<uint4*>(xrow + ((c8 ^ (r & 7)) << 4)) =
+                        make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
+                                   pack_bf16(d[6], d[7]));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            };
+            // X is free once the dK MMAs of the previous unit and the store of its
+            // dS^T tile to global memory (for the dQ product) have read it
+            if (u > 0 && (!warp_wait(dk_done, (u - 1) & 1, abort_flag, p.status) ||
+                          !warp_wait(dst_read, (u - 1) & 1, abort_flag, p.status))) {
+                ok = false;
+                break;
+            }
+            put_x(pv);
+            if (lane == 0) mbar_arrive(p_full);
+            if (!warp_wait(dp_full, u & 1, abort_flag, p.status)) {
                 ok = false;
                 break;
             }
@@ -1046,18 +1080,9 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             uint32_t rd[32];
             tmem_ld32_issue(tdPt + lane_off + cg * 32, rd);
             tmem_wait_ld();
-            // P^T over the first half of this warp's own dP^T columns (just read)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t pk[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(pv[16 * hf + 2 * e], pv[16 * hf + 2 * e + 1]);
-                tmem_st8_nowait(tdPt + lane_off + cg * 32 + 8 * hf, pk);
-            }
-            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(dp_free);
             // dS^T = P^T (dP^T - D); masked entries have P = 0 and D, dP finite
             const float4* d4 = reinterpret_cast<const float4*>(d_s + st * 128 + cg * 32);
 #pragma unroll
@@ -1068,28 +1093,12 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                 pv[4 * k + 2] *= __uint_as_float(rd[4 * k + 2]) - dd.z;
                 pv[4 * k + 3] *= __uint_as_float(rd[4 * k + 3]) - dd.w;
             }
-            uint4 dsv[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float* d = pv + 8 * k;
-                dsv[k] = make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
-                                    pack_bf16(d[6], d[7]));
-            }
-            // the dK MMAs of the previous unit and the store of its tile to global
-            // memory (for the dQ product) have read the dS^T tile
-            if (u > 0 && (!warp_wait(ds_free, (u - 1) & 1, abort_flag, p.status) ||
-                          !warp_wait(dst_read, (u - 1) & 1, abort_flag, p.status))) {
+            // the dV MMAs have read P^T out of X
+            if (!warp_wait(pv_done, u & 1, abort_flag, p.status)) {
                 ok = false;
                 break;
             }
-            uint8_t* drow = smem + Lay::DST + (cg >> 1) * 16384 + r * 128;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int c8 = (cg & 1) * 4 + k;
-                *reinterpret_cast<uint4*>(drow + ((c8 ^ (r & 7)) << 4)) = dsv[k];
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
+            put_x(pv);
             if (lane == 0) mbar_arrive(ds_full);
         }
         if (ok && warp_wait(dkv_done, 0, abort_flag, p.status)) {
