@@ -132,7 +132,7 @@ __device__ __forceinline__ void fwd_unit(const AttnParams& p, int u, int& b, int
 }
 
 template <int HD>
-__global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnParams p) {
+__global__ void __maxnreg__(200) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnParams p) {
     using Lay = FwdLayout<HD>;
     constexpr int KB = Lay::KB, TILE = Lay::TILE, KVSTG = Lay::KVSTG;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -329,33 +329,30 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 ++scnt;
                 tc_fence_after();
                 const bool diag = j == qb;  // key c of the diagonal block is visible from row r iff c <= r
-                // pass 1: the row maximum (scores read from TMEM 64 columns at a time),
-                // as eight independent partial maxima (no 128-long dependency chain)
+                // the whole score row in registers: four loads in flight, one wait
+                uint32_t sr[128];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) tmem_ld32_issue(tS + 32 * q4, sr + 32 * q4);
+                tmem_wait_ld();
+                // the row maximum as eight independent partial maxima (no 128-long
+                // dependency chain)
                 float mx8[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
-                auto row_max = [&](auto dg) {
-                    constexpr bool kDiag = decltype(dg)::value;
+                if (diag) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t s[32];
-                        tmem_ld32_issue(tS + 32 * q4, s);
-                        tmem_wait_ld();
+                    for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], c > r ? -INFINITY : __uint_as_float(sr[c]));
+                } else {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            mx8[c & 7] = fmaxf(mx8[c & 7], (kDiag && 32 * q4 + c > r) ? -INFINITY : __uint_as_float(s[c]));
-                    }
-                };
-                if (diag) row_max(std::true_type{});
-                else row_max(std::false_type{});
+                    for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+                }
                 float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                  fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
                 mx *= p.scale_log2;
                 const bool rescale = mx > m + 8.f;
                 const float mu = rescale ? mx : m;
                 const float alpha = rescale ? ex2(m - mx) : 1.f;
-                // pass 2: P = 2^(s*scale - mu) as packed bf16 over the first 64 score
-                // columns (the scores of each half are read before they are overwritten),
+                // P = 2^(s*scale - mu) as packed bf16 over the first 64 score columns,
                 // the row sum as eight independent partial sums; with kPoly one score in
                 // kPolyEvery comes from the FMA pipe (full blocks only: exp2_fma does not
                 // take the masked -inf scores of the diagonal block)
@@ -365,21 +362,17 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 auto exp_pack = [&](auto poly) {
                     constexpr bool kPoly = decltype(poly)::value;
                     constexpr int kPE = kPolyEvery > 0 ? kPolyEvery : 2;
-                    // 32 scores at a time; their packed P (16 columns) lands on columns
-                    // already read (16 q4 + 15 < 32 q4 for q4 >= 1, and the chunk itself for q4 = 0)
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t s[32];
-                        tmem_ld32_issue(tS + 32 * q4, s);
-                        tmem_wait_ld();
                         uint32_t pk[16];
 #pragma unroll
                         for (int c = 0; c < 32; c += 2) {
-                            float x0 = fmaf(__uint_as_float(s[c]), p.scale_log2, -mu);
-                            float x1 = fmaf(__uint_as_float(s[c + 1]), p.scale_log2, -mu);
+                            const int cc = 32 * q4 + c;
+                            float x0 = fmaf(__uint_as_float(sr[cc]), p.scale_log2, -mu);
+                            float x1 = fmaf(__uint_as_float(sr[cc + 1]), p.scale_log2, -mu);
                             if (!kPoly && diag) {
-                                if (32 * q4 + c > r) x0 = -INFINITY;
-                                if (32 * q4 + c + 1 > r) x1 = -INFINITY;
+                                if (cc > r) x0 = -INFINITY;
+                                if (cc + 1 > r) x1 = -INFINITY;
                             }
                             const float e0 = ex2(x0);
                             const float e1 = (kPoly && (c / 2) % (kPE / 2) == kPE / 2 - 1) ? exp2_fma(x1) : ex2(x1);
@@ -471,12 +464,6 @@ struct BwdParams {
     bf16* dqkv;
     bf16* ds;           // dS^T tiles (see ds_tile), written by the dK/dV kernel
     int* status;
-    // with rqk: the k gradient is taken through the QK-norm + RoPE backward
-    // (qkv: the saved rotated, normalised rows; rqk [B*T, H + nkv]; cos/sin [T, HD/2])
-    const bf16* qkv;
-    const float* rqk;
-    const float* cos_t;
-    const float* sin_t;
 };
 
 // The dK/dV kernel stores every causal 128 x 128 tile of dS = P (dP - D) it
@@ -487,75 +474,6 @@ struct BwdParams {
 __host__ __device__ inline size_t ds_tile(int b, int h, int H, int ntri, int qb, int kb) {
     return ((size_t)b * H + h) * (size_t)ntri + (size_t)qb * (qb + 1) / 2 + kb;
 }
-
-// Backward of the QK-norm + RoPE of one head vector of this thread's row,
-// fused into the epilogue that produces the gradient of the rotated,
-// normalised vector (nanochat announcement, vpshk.cn, architecture list:
-// rotary embeddings, QK norm).  With out = rope(y), y = r x (r the inverse RMS
-// of x): g = rope^-1(d out), y = rope^-1(out), dx = r (g - y (g.y) / HD).
-// d out comes from TMEM columns tsrc.. (times sc), out from the saved bf16
-// vector; the pairs (j, j + HD/2) are both in this thread.  W-column chunks
-// (16 or 32) bound the registers.  Every lane must call it (TMEM loads are
-// warp-collective); only live rows touch memory.
-template <int HD, int W>
-__device__ __forceinline__ void qknorm_rope_bwd_row(uint32_t tsrc, float sc, const bf16* yo, float r,
-                                                    const float* cs, const float* sn, bf16* out, bool live) {
-    constexpr int HALF = HD / 2;
-    auto load = [&](int c, float* d1, float* d2, float* y1, float* y2) {
-        if constexpr (W == 32) {
-            tmem_ld32(tsrc + c, d1);
-            tmem_ld32(tsrc + c + HALF, d2);
-        } else {
-            tmem_ld16(tsrc + c, d1);
-            tmem_ld16(tsrc + c + HALF, d2);
-        }
-        if (live) {
-#pragma unroll
-            for (int e = 0; e < W / 8; ++e) {
-                load_vec(yo + c + 8 * e, y1 + 8 * e);
-                load_vec(yo + c + HALF + 8 * e, y2 + 8 * e);
-            }
-        }
-    };
-    float dot = 0.f;
-#pragma unroll 1
-    for (int c = 0; c < HALF; c += W) {
-        float d1[W], d2[W], y1[W], y2[W];
-        load(c, d1, d2, y1, y2);
-        if (live) {
-#pragma unroll
-            for (int i = 0; i < W; ++i) {
-                const float co = cs[c + i], si = sn[c + i];
-                const float g1 = (d1[i] * co + d2[i] * si) * sc, g2 = (d2[i] * co - d1[i] * si) * sc;
-                const float u1 = y1[i] * co + y2[i] * si, u2 = y2[i] * co - y1[i] * si;
-                dot += g1 * u1 + g2 * u2;
-            }
-        }
-    }
-    dot *= 1.f / (float)HD;
-#pragma unroll 1
-    for (int c = 0; c < HALF; c += W) {
-        float d1[W], d2[W], y1[W], y2[W];
-        load(c, d1, d2, y1, y2);
-        if (live) {
-            float o1[W], o2[W];
-#pragma unroll
-            for (int i = 0; i < W; ++i) {
-                const float co = cs[c + i], si = sn[c + i];
-                const float g1 = (d1[i] * co + d2[i] * si) * sc, g2 = (d2[i] * co - d1[i] * si) * sc;
-                const float u1 = y1[i] * co + y2[i] * si, u2 = y2[i] * co - y1[i] * si;
-                o1[i] = r * (g1 - u1 * dot);
-                o2[i] = r * (g2 - u2 * dot);
-            }
-#pragma unroll
-            for (int e = 0; e < W / 8; ++e) {
-                store_vec(out + c + 8 * e, o1 + 8 * e);
-                store_vec(out + c + HALF + 8 * e, o2 + 8 * e);
-            }
-        }
-    }
-}
-
 
 // sum of the products of two vectors of eight bf16
 __device__ __forceinline__ float dot8(const uint4& a, const uint4& b) {
@@ -627,10 +545,6 @@ struct DqdsParams {
     float scale;
     bf16* dqkv;
     int* status;
-    const bf16* qkv;  // with rqk: q gradient through the QK-norm + RoPE backward (as BwdParams)
-    const float* rqk;
-    const float* cos_t;
-    const float* sin_t;
 };
 
 __device__ __forceinline__ void dq_unit(const DqdsParams& p, int u, int& b, int& h, int& qb) {
@@ -748,13 +662,6 @@ __global__ void __launch_bounds__(NTQ, 1) attn_dq_ds_kernel(const __grid_constan
             const size_t rowi = (size_t)b * p.T + (live ? qpos : 0);
             bf16* out = p.dqkv + rowi * Nqkv + (size_t)h * HD;
             const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + acc * HD;
-            if (p.rqk) {
-                const int pos = live ? qpos : 0;
-                qknorm_rope_bwd_row<HD, 32>(tb, p.scale, p.qkv + rowi * Nqkv + (size_t)h * HD,
-                                            live ? p.rqk[rowi * (p.H + p.nkv) + h] : 0.f,
-                                            p.cos_t + (size_t)pos * (HD / 2), p.sin_t + (size_t)pos * (HD / 2), out,
-                                            live);
-            } else
 #pragma unroll 1
             for (int c = 0; c < HD / 32; ++c) {
                 float v[32];
@@ -1105,47 +1012,24 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             tc_fence_after();
             const bool live = kpos < p.T;
             const size_t rowi = (size_t)row0 + (live ? kpos : 0);
-            if (p.rqk) {
-                // column group 0 writes dv; group 1 takes dk through the QK-norm + RoPE
-                // backward (whole rows per thread: the norm needs the row's dot product)
-                if (cg == 0) {
-                    bf16* out = p.dqkv + rowi * Nqkv + (size_t)(p.H + p.nkv + g) * HD;
-#pragma unroll 1
-                    for (int c = 0; c < HD / 32; ++c) {
-                        float v[32];
-                        tmem_ld32(tdV + lane_off + c * 32, v);
-                        if (live) {
+            // column groups 0 and 1 write the two halves of dv, 2 and 3 those of dk
+            const bool isk = cg >= 2;
+            const int c0 = (cg & 1) * (HD / 2);
+            const uint32_t tsrc = (isk ? tdK : tdV) + lane_off + c0;
+            const float sc = isk ? p.scale : 1.f;
+            bf16* out = p.dqkv + rowi * Nqkv + (size_t)(isk ? p.H + g : p.H + p.nkv + g) * HD + c0;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) store_vec(out + c * 32 + 8 * e, v + 8 * e);
-                        }
-                    }
-                } else if (cg == 1) {
-                    const int pos = live ? kpos : 0;
-                    qknorm_rope_bwd_row<HD, 16>(tdK + lane_off, p.scale, p.qkv + rowi * Nqkv + (size_t)(p.H + g) * HD,
-                                                live ? p.rqk[rowi * (p.H + p.nkv) + p.H + g] : 0.f,
-                                                p.cos_t + (size_t)pos * (HD / 2), p.sin_t + (size_t)pos * (HD / 2),
-                                                p.dqkv + rowi * Nqkv + (size_t)(p.H + g) * HD, live);
-                }
-            } else {
-                // column groups 0 and 1 write the two halves of dv, 2 and 3 those of dk
-                const bool isk = cg >= 2;
-                const int c0 = (cg & 1) * (HD / 2);
-                const uint32_t tsrc = (isk ? tdK : tdV) + lane_off + c0;
-                const float sc = isk ? p.scale : 1.f;
-                bf16* out = p.dqkv + rowi * Nqkv + (size_t)(isk ? p.H + g : p.H + p.nkv + g) * HD + c0;
+            for (int c = 0; c < HD / 64; ++c) {
+                float v[32];
+                tmem_ld32(tsrc + c * 32, v);
+                if (live) {
 #pragma unroll
-                for (int c = 0; c < HD / 64; ++c) {
-                    float v[32];
-                    tmem_ld32(tsrc + c * 32, v);
-                    if (live) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            *reinterpret_cast<uint4*>(out + c * 32 + 8 * e) =
-                                make_uint4(pack_bf16(v[8 * e] * sc, v[8 * e + 1] * sc),
-                                           pack_bf16(v[8 * e + 2] * sc, v[8 * e + 3] * sc),
-                                           pack_bf16(v[8 * e + 4] * sc, v[8 * e + 5] * sc),
-                                           pack_bf16(v[8 * e + 6] * sc, v[8 * e + 7] * sc));
-                    }
+                    for (int e = 0; e < 4; ++e)
+                        *reinterpret_cast<uint4*>(out + c * 32 + 8 * e) =
+                            make_uint4(pack_bf16(v[8 * e] * sc, v[8 * e + 1] * sc),
+                                       pack_bf16(v[8 * e + 2] * sc, v[8 * e + 3] * sc),
+                                       pack_bf16(v[8 * e + 4] * sc, v[8 * e + 5] * sc),
+                                       pack_bf16(v[8 * e + 6] * sc, v[8 * e + 7] * sc));
                 }
             }
         }
@@ -1285,23 +1169,18 @@ int attention_tc_bwd_stats(const void* o, const void* dO, const float* lse, floa
 }
 
 int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqkv, void* ws, size_t ws_bytes, int B,
-                         int T, int H, int nkv, int hd, const QkNormRope* qk, int* status, cudaStream_t s) {
+                         int T, int H, int nkv, int hd, int* status, cudaStream_t s) {
     BwdParams p;
     CUtensorMap kv, do128;
     if (!ws || ws_bytes < attention_tc_workspace_bytes(B, T, H, nkv, hd)) return 1;
     if (!bwd_setup(qkv, dO, Dbuf, dqkv, ws, B, T, H, nkv, hd, status, &p, &kv, &do128)) return 1;
-    if (qk) {
-        if (!qk->rqk || !qk->cos_t || !qk->sin_t) return 1;
-        p.qkv = reinterpret_cast<const bf16*>(qkv);
-        p.rqk = qk->rqk; p.cos_t = qk->cos_t; p.sin_t = qk->sin_t;
-    }
     CUtensorMap mds;
     if (!map_rows(&mds, ws, 128, (uint64_t)B * H * ntri_of(T) * 128, 128)) return 1;
     return hd == 128 ? dkv_launch<128>(kv, do128, mds, p, s) : dkv_launch<64>(kv, do128, mds, p, s);
 }
 
 int attention_tc_bwd_dq(const void* qkv, const void* ws, size_t ws_bytes, void* dqkv, int B, int T, int H, int nkv,
-                        int hd, const QkNormRope* qk, int* status, cudaStream_t s) {
+                        int hd, int* status, cudaStream_t s) {
     if (!attention_tc_bwd_supported(hd) || !ws || ws_bytes < attention_tc_workspace_bytes(B, T, H, nkv, hd)) return 1;
     if (!aligned16(qkv) || !aligned16(ws) || !aligned16(dqkv) || B > 65535 || nkv < 1 || H % nkv) return 1;
     const int Nqkv = (H + 2 * nkv) * hd;
@@ -1314,19 +1193,14 @@ int attention_tc_bwd_dq(const void* qkv, const void* ws, size_t ws_bytes, void* 
     p.scale = 1.f / sqrtf((float)hd);
     p.dqkv = reinterpret_cast<bf16*>(dqkv);
     p.status = status;
-    if (qk) {
-        if (!qk->rqk || !qk->cos_t || !qk->sin_t) return 1;
-        p.qkv = reinterpret_cast<const bf16*>(qkv);
-        p.rqk = qk->rqk; p.cos_t = qk->cos_t; p.sin_t = qk->sin_t;
-    }
     return hd == 128 ? dq_ds_launch<128>(mds, mkv, p, s) : dq_ds_launch<64>(mds, mkv, p, s);
 }
 
 int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
                      int B, int T, int H, int nkv, int hd, void* ws, size_t ws_bytes, int* status, cudaStream_t s) {
     int r = attention_tc_bwd_stats(o, dO, lse, Dbuf, B, T, H, hd, s);
-    if (r == 0) r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, ws, ws_bytes, B, T, H, nkv, hd, nullptr, status, s);
-    if (r == 0) r = attention_tc_bwd_dq(qkv, ws, ws_bytes, dqkv, B, T, H, nkv, hd, nullptr, status, s);
+    if (r == 0) r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, ws, ws_bytes, B, T, H, nkv, hd, status, s);
+    if (r == 0) r = attention_tc_bwd_dq(qkv, ws, ws_bytes, dqkv, B, T, H, nkv, hd, status, s);
     return r;
 }
 

@@ -16,20 +16,11 @@ size_t attention_tc_workspace_bytes(int B, int T, int H, int nkv, int hd);
 // [B, H, attn_tpad(T)].
 int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
                      int B, int T, int H, int nkv, int hd, void* ws, size_t ws_bytes, int* status, cudaStream_t s);
-// Optional fusion of the QK-norm + RoPE backward into the dk and dq epilogues:
-// qkv holds the saved rotated, normalised q/k heads; rqk [B*T, H + nkv] their
-// inverse RMS; cos/sin [T, hd/2] the RoPE table.  With it the dq and dk columns
-// of dqkv receive the gradient with respect to the pre-norm q and k.
-struct QkNormRope {
-    const float* rqk;
-    const float* cos_t;
-    const float* sin_t;
-};
-// Its three launches, in order (qk may be null).
+// Its three launches, in order.
 int attention_tc_bwd_stats(const void* o, const void* dO, const float* lse, float* Dbuf, int B, int T, int H, int hd,
                            cudaStream_t s);
 int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqkv, void* ws, size_t ws_bytes, int B,
-                         int T, int H, int nkv, int hd, const QkNormRope* qk, int* status, cudaStream_t s);
+                         int T, int H, int nkv, int hd, int* status, cudaStream_t s);
 int attention_tc_bwd_dq(const void* qkv, const void* ws, size_t ws_bytes, void* dqkv, int B, int T, int H, int nkv,
-                        int hd, const QkNormRope* qk, int* status, cudaStream_t s);
+                        int hd, int* status, cudaStream_t s);
 }  // namespace nc

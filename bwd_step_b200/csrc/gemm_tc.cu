@@ -334,6 +334,39 @@ __device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUte
     }
 }
 
+// The epilogue of one accumulator row over the tile's 32-column chunks; the
+// TMEM load of chunk c + 1 is in flight while chunk c is processed.
+__device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorMap* tmC, const CUtensorMap* tmC2,
+                                              uint8_t* stg, int lane, int ks, int row, int row0w, int tn, uint32_t tb,
+                                              int& cnt) {
+    RowCtx rc = row_ctx(p, row);
+    const int nch = min(BN / 32, (p.N - tn * BN + 31) / 32);
+    uint32_t b0[32], b1[32];
+    auto chunk = [&](int c, uint32_t* cur) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(cur[i]);
+        const int n0 = tn * BN + c * 32;
+        if (p.tma_out) epilogue_chunk_tma(p, tmC, tmC2, stg, lane, ks, row, row0w, n0, v, cnt++, rc);
+        else if (row < p.M) epilogue(p, ks, row, n0, v, rc);
+    };
+    tmem_ld32_issue(tb, b0);
+    tmem_wait_ld();
+    reg_fence32(b0);
+    for (int c = 0; c < nch; c += 2) {
+        if (c + 1 < nch) tmem_ld32_issue(tb + (c + 1) * 32, b1);
+        chunk(c, b0);
+        if (c + 1 >= nch) break;
+        tmem_wait_ld();
+        reg_fence32(b1);
+        if (c + 2 < nch) tmem_ld32_issue(tb + (c + 2) * 32, b0);
+        chunk(c + 1, b1);
+        tmem_wait_ld();
+        reg_fence32(b0);
+    }
+    if (p.epi == EPI_LMHEAD && row < p.M) p.stats[(size_t)row * p.stats_ld + tn] = rc.sum;
+}
+
 // Fused QK-norm + RoPE epilogue over one 256-column tile of the qkv
 // projection (nanochat announcement, vpshk.cn, architecture list: rotary
 // embeddings, QK norm): every head of HD columns is loaded whole from TMEM,
@@ -515,16 +548,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
                 else epilogue_qkrope<64>(p, row, tn * BN, tb);
             } else {
-                RowCtx rc = row_ctx(p, row);
-                for (int c = 0; c < BN / 32; ++c) {
-                    const int n0 = tn * BN + c * 32;
-                    if (n0 >= p.N) break;
-                    float v[32];
-                    tmem_ld32(tb + c * 32, v);
-                    if (p.tma_out) epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++, rc);
-                    else if (row < p.M) epilogue(p, ks, row, n0, v, rc);
-                }
-                if (p.epi == EPI_LMHEAD && row < p.M) p.stats[(size_t)row * p.stats_ld + tn] = rc.sum;
+                epilogue_tile(p, &tmC, &tmC2, stg, lane, ks, row, row0w, tn, tb, cnt);
             }
             tc_fence_before();
             __syncwarp();
@@ -675,16 +699,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
                 else epilogue_qkrope<64>(p, row, tn * BN, tb);
             } else {
-                RowCtx rc = row_ctx(p, row);
-                for (int c = 0; c < BN / 32; ++c) {
-                    const int n0 = tn * BN + c * 32;
-                    if (n0 >= p.N) break;
-                    float v[32];
-                    tmem_ld32(tb + c * 32, v);
-                    if (p.tma_out) epilogue_chunk_tma(p, &tmC, &tmC2, stg, lane, ks, row, row0w, n0, v, cnt++, rc);
-                    else if (row < p.M) epilogue(p, ks, row, n0, v, rc);
-                }
-                if (p.epi == EPI_LMHEAD && row < p.M) p.stats[(size_t)row * p.stats_ld + tn] = rc.sum;
+                epilogue_tile(p, &tmC, &tmC2, stg, lane, ks, row, row0w, tn, tb, cnt);
             }
             tc_fence_before();
             __syncwarp();

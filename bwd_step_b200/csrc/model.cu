@@ -256,35 +256,35 @@ int attention_fwd(const Ctx& c, const void* qkv, void* o, float* lse) {
 }
 
 // Attention backward, then the QK-norm + RoPE backward into the pre-norm q, k
-// gradients.  Tensor cores: statistics and dk / dv (which also stores the dS
-// tiles), then dq from those tiles, with the QK-norm + RoPE backward fused into
-// the dk and dq epilogues; otherwise the plain-FMA kernels and a separate pass.
+// gradients (one pass over all heads of each position).  Tensor cores:
+// statistics (unless the dO GEMM's epilogue wrote them) and dk / dv (which also
+// stores the dS tiles), then dq from those tiles; otherwise the plain-FMA kernels.
 int attention_bwd(const Ctx& c, const void* qkv, const void* o, const void* dO, const float* lse, const float* rqk,
                   void* dqkv, bool stats_ready) {
     const nc_model* m = c.m;
     float* Dbuf = c.at<float>(c.p.Dbuf);
     const float* cs = c.at<float>(c.p.cosb);
     const float* sn = c.at<float>(c.p.sinb);
+    bool done = false;
     if (m->tc && attention_tc_bwd_supported(m->hd)) {
         void* ws = c.ws + c.p.attn_ws;
-        const QkNormRope qk{rqk, cs, sn};
         int r;
         {
             Prof pr(c, P_ATTN_BWD_DKV, 2.0 * attn_flops(c), 0.0);
             r = stats_ready ? 0 : attention_tc_bwd_stats(o, dO, lse, Dbuf, c.p.B, c.p.T, m->H, m->hd, c.s);
             if (r == 0)
                 r = attention_tc_bwd_dkv(qkv, dO, Dbuf, dqkv, ws, c.p.attn_ws_bytes, c.p.B, c.p.T, m->H, m->nkv,
-                                         m->hd, &qk, m->status, c.s);
+                                         m->hd, m->status, c.s);
         }
         if (r == 0) {
             Prof pr(c, P_ATTN_BWD_DQ, 0.5 * attn_flops(c), 0.0);
-            r = attention_tc_bwd_dq(qkv, ws, c.p.attn_ws_bytes, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, &qk,
-                                    m->status, c.s);
+            r = attention_tc_bwd_dq(qkv, ws, c.p.attn_ws_bytes, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, m->status,
+                                    c.s);
         }
-        if (r == 0) return NC_OK;
         if (r < 0) return NC_ERR_CUDA;
+        done = r == 0;
     }
-    {
+    if (!done) {
         Prof pr(c, P_ATTN_BWD, 2.0 * attn_flops(c), 0.0);
         CK(launch_attention_bwd_simt(m->at, qkv, o, dO, lse, Dbuf, dqkv, c.p.B, c.p.T, m->H, m->nkv, m->hd, c.s));
     }

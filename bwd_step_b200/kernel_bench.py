@@ -2,7 +2,7 @@
 
     python -m bwd_step_b200.kernel_bench gemm [--only NAME] [--iters N]
     python -m bwd_step_b200.kernel_bench attention [--iters N]
-    python -m bwd_step_b200.kernel_bench step [--workload d20] [--batch B] [--layers L] [--warmup W] [--iters K]
+    python -m bwd_step_b200.kernel_bench step [--workload d20] [--batch B] [--layers L] [--lm-rows R] [--warmup W] [--iters K]
 
 `gemm` runs every GEMM shape of one depth-20 step (32768 tokens, d 1280,
 MLP 5120, 10x128 MQA, vocab 65536 with a 4096-row LM-head chunk) through the
@@ -117,7 +117,7 @@ def bench_attention(iters, B=16, T=2048, H=10, nkv=1, hd=128):
             {"kernel": "attention_bwd", "ms": t_b, "tflops": 2 * flops / t_b / 1e9}]
 
 
-def run_steps(workload, batch, warmup, iters, layers=0):
+def run_steps(workload, batch, warmup, iters, layers=0, lm_rows=0):
     import numpy as np
     import os
     import sys
@@ -133,6 +133,8 @@ def run_steps(workload, batch, warmup, iters, layers=0):
     bits, _ = synth.make_weights(wl.model, seed=0, dtype="bf16")
     tok, tgt = synth.make_tokens(wl, seed=1, batch=B)
     m = Model(wl.model.as_dict(), "bf16")
+    if lm_rows:
+        m.set_lm_head("fused", lm_rows)
     W = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
     grads = torch.empty(m.num_params(), dtype=torch.float32, device="cuda")
     loss = torch.empty(1, dtype=torch.float32, device="cuda")
@@ -145,7 +147,7 @@ def run_steps(workload, batch, warmup, iters, layers=0):
     t = _timed(lambda: m.forward_backward(tok_d, tgt_d, W, grads, loss, ws), iters) if iters else 0.0
     per = (launch_count() - l0) // max(iters + 2, 1) if iters else 0
     assert m.check() == 0
-    return {"workload": workload, "batch": B, "ms_per_step": t, "launches_per_step": per, "loss": float(loss.item())}
+    return {"workload": workload, "batch": B, "lm_rows": lm_rows, "ms_per_step": t, "launches_per_step": per, "loss": float(loss.item())}
 
 
 def main():
@@ -155,6 +157,7 @@ def main():
     ap.add_argument("--batch", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--lm-rows", type=int, default=0, help="LM-head chunk rows (0 = default)")
     ap.add_argument("--only", default=None)
     ap.add_argument("--iters", type=int, default=10)
     args = ap.parse_args()
@@ -168,7 +171,7 @@ def main():
         for r in bench_attention(args.iters):
             print(json.dumps(r), flush=True)
     else:
-        print(json.dumps(run_steps(args.workload, args.batch, args.warmup, args.iters, args.layers)), flush=True)
+        print(json.dumps(run_steps(args.workload, args.batch, args.warmup, args.iters, args.layers, args.lm_rows)), flush=True)
 
 
 if __name__ == "__main__":
