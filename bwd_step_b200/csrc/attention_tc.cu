@@ -132,7 +132,7 @@ __device__ __forceinline__ void fwd_unit(const AttnParams& p, int u, int& b, int
 }
 
 template <int HD>
-__global__ void __maxnreg__(200) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnParams p) {
+__global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm, const AttnParams p) {
     using Lay = FwdLayout<HD>;
     constexpr int KB = Lay::KB, TILE = Lay::TILE, KVSTG = Lay::KVSTG;
     extern __shared__ __align__(1024) uint8_t smem_dyn[];
@@ -334,40 +334,39 @@ __global__ void __maxnreg__(200) attn_fwd_tc_kernel(const __grid_constant__ CUte
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) tmem_ld32_issue(tS + 32 * q4, sr + 32 * q4);
                 tmem_wait_ld();
-                // the row maximum as eight independent partial maxima (no 128-long
+                // the row maximum as four independent partial maxima (no 128-long
                 // dependency chain)
-                float mx8[8];
+                float mx4[4];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+                for (int k = 0; k < 4; ++k) mx4[k] = -INFINITY;
                 if (diag) {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], c > r ? -INFINITY : __uint_as_float(sr[c]));
+                    for (int c = 0; c < 128; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], c > r ? -INFINITY : __uint_as_float(sr[c]));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+                    for (int c = 0; c < 128; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(sr[c]));
                 }
-                float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                 mx *= p.scale_log2;
                 const bool rescale = mx > m + 8.f;
                 const float mu = rescale ? mx : m;
                 const float alpha = rescale ? ex2(m - mx) : 1.f;
                 // P = 2^(s*scale - mu) as packed bf16 over the first 64 score columns,
-                // the row sum as eight independent partial sums; with kPoly one score in
+                // the row sum as four independent partial sums; with kPoly one score in
                 // kPolyEvery comes from the FMA pipe (full blocks only: exp2_fma does not
                 // take the masked -inf scores of the diagonal block)
-                float sum8[8];
+                float sum4[4];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
+                for (int k = 0; k < 4; ++k) sum4[k] = 0.f;
                 auto exp_pack = [&](auto poly) {
                     constexpr bool kPoly = decltype(poly)::value;
                     constexpr int kPE = kPolyEvery > 0 ? kPolyEvery : 2;
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint32_t pk[16];
+                    for (int q8 = 0; q8 < 8; ++q8) {
+                        uint32_t pk[8];
 #pragma unroll
-                        for (int c = 0; c < 32; c += 2) {
-                            const int cc = 32 * q4 + c;
+                        for (int c = 0; c < 16; c += 2) {
+                            const int cc = 16 * q8 + c;
                             float x0 = fmaf(__uint_as_float(sr[cc]), p.scale_log2, -mu);
                             float x1 = fmaf(__uint_as_float(sr[cc + 1]), p.scale_log2, -mu);
                             if (!kPoly && diag) {
@@ -376,16 +375,16 @@ __global__ void __maxnreg__(200) attn_fwd_tc_kernel(const __grid_constant__ CUte
                             }
                             const float e0 = ex2(x0);
                             const float e1 = (kPoly && (c / 2) % (kPE / 2) == kPE / 2 - 1) ? exp2_fma(x1) : ex2(x1);
-                            sum8[(c >> 1) & 7] += e0 + e1;
+                            sum4[(c >> 1) & 3] += e0 + e1;
                             pk[c >> 1] = pack_bf16(e0, e1);
                         }
-                        tmem_st16_nowait(tS + 16 * q4, pk);
+                        tmem_st8_nowait(tS + 8 * q8, pk);
                     }
                 };
                 if (!diag && kPolyEvery > 0) exp_pack(std::true_type{});
                 else exp_pack(std::false_type{});
                 tmem_wait_st();
-                const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+                const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
                 if (j > 0 && __any_sync(0xffffffffu, rescale)) {
                     // O_x += P(j-1) V has completed (S(j) was issued after it and has landed);
                     // O_x += P(j) V waits for this warp's hand-over below
