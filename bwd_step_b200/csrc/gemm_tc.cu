@@ -10,8 +10,10 @@
 //   warp 1     allocates 512 TMEM columns and issues tcgen05.mma
 //              (M=128, N=256, K=16) from one thread; commits release ring
 //              slots and hand finished accumulators to the epilogue;
-//   warps 2-5  epilogue: tcgen05.ld of their 32 TMEM lanes (one output row per
-//              thread), fused elementwise work, 16-byte global stores.
+//   warps 2-9  epilogue: two warps per 32-lane TMEM quarter, one per 128-column
+//              half of the tile; tcgen05.ld of their lanes (one output row per
+//              thread), fused elementwise work, staged TMA stores.  Two warps per
+//              SM sub-partition hide each other's latencies.
 // Two 256-column accumulators let the epilogue of one tile overlap the main
 // loop of the next.  Operands may be K-major or M/N-major (the backward
 // products read activations and weights transposed without a copy).
@@ -28,10 +30,10 @@ namespace {
 using namespace tc;
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-static_assert(BN == kGemmTileN, "the LM-head epilogue writes one sum per BN-column tile");
+static_assert(BN == 2 * kGemmStatCols, "each epilogue warp covers one 128-column half of a tile");
 constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int TMEM_COLS = 2 * BN;
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 320;
 constexpr int MAX_SPLITS = 8;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 32768 + 256;  // + epilogue staging
 
@@ -254,14 +256,15 @@ __device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int
 }
 
 // ------------------------------------------------------------------ staged epilogue
-// Each epilogue warp owns two 4 KB staging buffers.  A 32-row x 32-column
-// sub-tile is written into one of them in the layout of the output tensor
-// map's swizzle (fp32: 128-byte rows, 128B swizzle; bf16: 64-byte rows, 64B
+// Each epilogue warp owns a 4 KB staging buffer.  A 32-row x 32-column
+// sub-tile is written into it in the layout of the output tensor map's
+// swizzle (fp32: 128-byte rows, 128B swizzle; bf16: 64-byte rows, 64B
 // swizzle; conflict-free for the row-per-thread writes), then one lane issues
 // a TMA store -- or, for the residual-add epilogue, a TMA reduce-add, so C is
-// never read into the SM.  A buffer is reused only after the store issued two
-// chunks earlier has finished reading it.
-constexpr int STAGING_BYTES = 4 * 2 * 4096;
+// never read into the SM.  The buffer is rewritten only after the previous
+// chunk's store has finished reading it (the next chunk is already computed
+// in registers by then).
+constexpr int STAGING_BYTES = 8 * 4096;
 
 __device__ __forceinline__ void stage_f32(uint8_t* buf, int lane, const float* v) {
 #pragma unroll
@@ -278,9 +281,9 @@ __device__ __forceinline__ void stage_bf16(uint8_t* buf, int lane, const float* 
 __device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUtensorMap* tmC, const CUtensorMap* tmC2,
                                                    uint8_t* stg, int lane, int ks, int row, int row0w, int n0, float* v,
                                                    int cnt, RowCtx& rc) {
-    uint8_t* buf = stg + (cnt & 1) * 4096;
-    if (cnt >= 2) {
-        if (lane == 0) bulk_wait_read_1();
+    uint8_t* buf = stg;
+    if (cnt >= 1) {
+        if (lane == 0) bulk_wait_read_0();
         __syncwarp();
     }
     const int mode = p.part ? EPI_STORE : p.epi;
@@ -334,37 +337,23 @@ __device__ __forceinline__ void epilogue_chunk_tma(const TcParams& p, const CUte
     }
 }
 
-// The epilogue of one accumulator row over the tile's 32-column chunks; the
-// TMEM load of chunk c + 1 is in flight while chunk c is processed.
+// The epilogue of one accumulator row over the 32-column chunks of one
+// 128-column half of the tile.  tb addresses the tile's first column.
 __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorMap* tmC, const CUtensorMap* tmC2,
-                                              uint8_t* stg, int lane, int ks, int row, int row0w, int tn, uint32_t tb,
-                                              int& cnt) {
+                                              uint8_t* stg, int lane, int ks, int row, int row0w, int tn, int half,
+                                              uint32_t tb, int& cnt) {
+    const int col0 = tn * BN + half * kGemmStatCols;
+    if (col0 >= p.N) return;
     RowCtx rc = row_ctx(p, row);
-    const int nch = min(BN / 32, (p.N - tn * BN + 31) / 32);
-    uint32_t b0[32], b1[32];
-    auto chunk = [&](int c, uint32_t* cur) {
+    const int nch = min(kGemmStatCols / 32, (p.N - col0 + 31) / 32);
+    for (int c = 0; c < nch; ++c) {
         float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(cur[i]);
-        const int n0 = tn * BN + c * 32;
+        tmem_ld32(tb + half * kGemmStatCols + c * 32, v);
+        const int n0 = col0 + c * 32;
         if (p.tma_out) epilogue_chunk_tma(p, tmC, tmC2, stg, lane, ks, row, row0w, n0, v, cnt++, rc);
         else if (row < p.M) epilogue(p, ks, row, n0, v, rc);
-    };
-    tmem_ld32_issue(tb, b0);
-    tmem_wait_ld();
-    reg_fence32(b0);
-    for (int c = 0; c < nch; c += 2) {
-        if (c + 1 < nch) tmem_ld32_issue(tb + (c + 1) * 32, b1);
-        chunk(c, b0);
-        if (c + 1 >= nch) break;
-        tmem_wait_ld();
-        reg_fence32(b1);
-        if (c + 2 < nch) tmem_ld32_issue(tb + (c + 2) * 32, b0);
-        chunk(c + 1, b1);
-        tmem_wait_ld();
-        reg_fence32(b0);
     }
-    if (p.epi == EPI_LMHEAD && row < p.M) p.stats[(size_t)row * p.stats_ld + tn] = rc.sum;
+    if (p.epi == EPI_LMHEAD && row < p.M) p.stats[(size_t)row * p.stats_ld + tn * 2 + half] = rc.sum;
 }
 
 // Fused QK-norm + RoPE epilogue over one 256-column tile of the qkv
@@ -373,14 +362,14 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& p, const CUtensorM
 // normalised by its RMS (no parameters), rotated pair-wise (j, j + HD/2) by the
 // row's position, and stored as bf16; value heads are stored unchanged.
 template <int HD>
-__device__ __forceinline__ void epilogue_qkrope(const TcParams& p, int row, int n_tile, uint32_t tb) {
+__device__ __forceinline__ void epilogue_qkrope(const TcParams& p, int row, int n_tile, uint32_t tb, int half) {
     constexpr int NC = HD / 32, HALF = HD / 2;
     const bool live = row < p.M;
     const int pos = live ? row % p.T : 0;
     const float* cs = p.cos_t + (size_t)pos * HALF;
     const float* sn = p.sin_t + (size_t)pos * HALF;
     bf16* crow = reinterpret_cast<bf16*>(p.C) + (int64_t)row * p.ldc;
-    for (int h0 = 0; h0 < BN; h0 += HD) {
+    for (int h0 = half * kGemmStatCols; h0 < (half + 1) * kGemmStatCols; h0 += HD) {
         const int col = n_tile + h0;
         if (col >= p.N) break;
         const int head = col / HD;
@@ -445,7 +434,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(bar_full + 8 * s, 1); mbar_init(bar_empty + 8 * s, 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(bar_tfull + 8 * b, 1); mbar_init(bar_tempty + 8 * b, 4); }
+        for (int b = 0; b < 2; ++b) { mbar_init(bar_tfull + 8 * b, 1); mbar_init(bar_tempty + 8 * b, 8); }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -530,9 +519,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
         }
     } else {
-        // ---------------- epilogue warps 2..5; warp w reads TMEM lanes 32*(w%4)..
-        const int q = warp & 3;
-        uint8_t* stg = staging + (warp - 2) * 8192;
+        // ---------------- epilogue warps 2..9; warp w reads TMEM lanes 32*(w%4)..,
+        // the columns of half (w - 2) / 4 of each tile
+        const int q = warp & 3, half = (warp - 2) >> 2;
+        uint8_t* stg = staging + (warp - 2) * 4096;
         int cnt = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -545,10 +535,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const int row = row0w + lane;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             if (p.epi == EPI_QKROPE) {
-                if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
-                else epilogue_qkrope<64>(p, row, tn * BN, tb);
+                if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb, half);
+                else epilogue_qkrope<64>(p, row, tn * BN, tb, half);
             } else {
-                epilogue_tile(p, &tmC, &tmC2, stg, lane, ks, row, row0w, tn, tb, cnt);
+                epilogue_tile(p, &tmC, &tmC2, stg, lane, ks, row, row0w, tn, half, tb, cnt);
             }
             tc_fence_before();
             __syncwarp();
@@ -596,7 +586,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES2; ++s) { mbar_init(bar_full + 8 * s, 1); mbar_init(bar_empty + 8 * s, 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(bar_tfull + 8 * b, 1); mbar_init(bar_tempty + 8 * b, 8); }
+        for (int b = 0; b < 2; ++b) { mbar_init(bar_tfull + 8 * b, 1); mbar_init(bar_tempty + 8 * b, 16); }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -681,9 +671,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             }
         }
     } else {
-        // ---------------- epilogue warps 2..5 of both CTAs
-        const int q = warp & 3;
-        uint8_t* stg = staging + (warp - 2) * 8192;
+        // ---------------- epilogue warps 2..9 of both CTAs (lane quarter w%4, column half (w-2)/4)
+        const int q = warp & 3, half = (warp - 2) >> 2;
+        uint8_t* stg = staging + (warp - 2) * 4096;
         int cnt = 0;
         int acc = 0;
         uint32_t acc_phase = 0;
@@ -696,10 +686,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const int row = row0w + lane;
             const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
             if (p.epi == EPI_QKROPE) {
-                if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb);
-                else epilogue_qkrope<64>(p, row, tn * BN, tb);
+                if (p.hd == 128) epilogue_qkrope<128>(p, row, tn * BN, tb, half);
+                else epilogue_qkrope<64>(p, row, tn * BN, tb, half);
             } else {
-                epilogue_tile(p, &tmC, &tmC2, stg, lane, ks, row, row0w, tn, tb, cnt);
+                epilogue_tile(p, &tmC, &tmC2, stg, lane, ks, row, row0w, tn, half, tb, cnt);
             }
             tc_fence_before();
             __syncwarp();
@@ -786,7 +776,7 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
          (reinterpret_cast<uintptr_t>(g.C) & 15) || (g.ldc % 8) || (g.N % g.hd)))
         return 1;
     if (g.epi == EPI_LMHEAD &&
-        (g.c_t != DT_BF16 || !g.tgt || !g.stats || !g.zt || !g.ut || g.stats_ld < gemm_tiles_n(g.N) || !(g.cap > 0.f)))
+        (g.c_t != DT_BF16 || !g.tgt || !g.stats || !g.zt || !g.ut || g.stats_ld < gemm_stat_groups(g.N) || !(g.cap > 0.f)))
         return 1;
     if (g.epi == EPI_ROWSCALE && (g.c_t != DT_F32 || !g.rs)) return 1;
     if (g.epi == EPI_ATTN_DO &&

@@ -102,8 +102,8 @@ enum Epi : int {
                         // C = rope(rmsnorm_hd(acc)) and rqk = its inverse RMS; other
                         // columns (v) C = acc.  bf16 C, head_dim 64 or 128 (tcgen05 only)
     EPI_LMHEAD = 6,     // LM head, logits never stored: z = cap*tanh(acc/cap), e = exp(z - cap),
-                        // C = e * (1 - (z/cap)^2) (bf16); per (row, 256-column tile) the sum of e
-                        // into stats[row * stats_ld + tile]; at the column tgt[row], z and C in
+                        // C = e * (1 - (z/cap)^2) (bf16); per (row, 128-column group) the sum of e
+                        // into stats[row * stats_ld + group]; at the column tgt[row], z and C in
                         // fp32 into zt[row], ut[row] (tcgen05 only)
     EPI_ROWSCALE = 7,   // C = acc * rs[row]                 (C fp32; tcgen05 only)
     EPI_ATTN_DO = 8,    // attention output gradient dO: C = acc (bf16), and per (row, head of hd
@@ -145,9 +145,9 @@ struct GemmDesc {
     int attn_H = 0;
 };
 
-// Column tiles of the tensor-core GEMM's output (EPI_LMHEAD writes one sum per tile).
-constexpr int kGemmTileN = 256;
-inline int gemm_tiles_n(int N) { return (N + kGemmTileN - 1) / kGemmTileN; }
+// Column groups of the tensor-core GEMM's output (EPI_LMHEAD writes one sum per group).
+constexpr int kGemmStatCols = 128;
+inline int gemm_stat_groups(int N) { return (N + kGemmStatCols - 1) / kGemmStatCols; }
 
 // Plain fp32-FMA tiled GEMM (any strides, any sizes).
 cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t s);

@@ -137,7 +137,7 @@ Plan make_plan(const nc_model* m, int B, int T, bool fwd_only = false) {
     const bool fz = bwd && lm_fused(m);
     p.zc = take(bwd ? A * (size_t)p.R * m->V : 0);                     // logits, or u on the fused path
     p.dlc = take(bwd && !lm_fused(m) ? A * (size_t)p.R * m->V : 0);   // their gradient (materialised path)
-    p.lm_tiles = gemm_tiles_n(m->V);
+    p.lm_tiles = gemm_stat_groups(m->V);
     p.lm_stats = take(fz ? 4ull * p.R * p.lm_tiles : 0);
     p.lm_zt = take(fz ? 4ull * p.R : 0);
     p.lm_ut = take(fz ? 4ull * p.R : 0);
