@@ -697,10 +697,11 @@ __global__ void __launch_bounds__(NTQ, 1) attn_dq_ds_kernel(const __grid_constan
 //               2-stage ring;
 //   warp 1      tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM,
 //               dV += P^T dO_i and dK += dS^T Q_i with P^T, then dS^T, in one
-//               shared-memory tile X (Q_i, dO_i as MN-major operands).  The
-//               next unit's S^T and dP^T are issued as soon as the softmax warps
-//               have read this unit's into registers, so they overlap this
-//               unit's softmax: S^T_{u+1}, dV_u, dP^T_{u+1}, dK_u;
+//               shared-memory tile X (Q_i, dO_i as MN-major operands).  Each
+//               product is issued as soon as its inputs are ready (the thread
+//               polls the four barriers), so the next unit's S^T and dP^T
+//               overlap this unit's softmax and a Q / dO load in flight does
+//               not hold back this unit's dV and dK;
 //   warps 2-17  per unit: load the warp's S^T columns (32 queries), form
 //               P^T = 2^(S^T*scale*log2e - lse2) with the causal mask, write it
 //               to X, load the dP^T columns, form dS^T = P^T (dP^T - D) and
@@ -831,11 +832,9 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, 128, false, false);
             const uint32_t id_kv = idesc_bf16(128, HD, false, true);
-            // S^T_u = K Q_u^T (waits for the unit's Q / dO stage)
-            auto scores = [&](int u) -> bool {
+            // S^T_u = K Q_u^T
+            auto scores = [&](int u) {
                 const int st = u & 1;
-                if (!mbar_wait(qo_full + 8 * st, (u >> 1) & 1, abort_flag, p.status)) return false;
-                tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < HD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -843,9 +842,8 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                              ks > 0 ? 1u : 0u);
                 }
                 mma_commit(s_full);
-                return true;
             };
-            // dP^T_u = V dO_u^T (Q_u / dO_u already landed)
+            // dP^T_u = V dO_u^T
             auto dpt = [&](int u) {
                 const int st = u & 1;
 #pragma unroll
@@ -864,30 +862,62 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                     mma_bf16(acc, smem_desc(sX + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                              smem_desc(bop + kk * 2048, 16384, 1024), id_kv, (u > 0 || kk > 0) ? 1u : 0u);
             };
-            bool ok = mbar_wait(kv_full, 0, abort_flag, p.status) && scores(0);
-            if (ok) dpt(0);
-            for (int u = 0; ok && u < nunits; ++u) {
-                const int st = u & 1;
-                const bool more = u + 1 < nunits;
-                // S^T of the next unit once this unit's S^T is in registers
-                if (more && (!mbar_wait(s_free, u & 1, abort_flag, p.status) || !scores(u + 1))) break;
-                // dV += P^T_u dO_u
-                if (!mbar_wait(p_full, u & 1, abort_flag, p.status)) break;
+            // The four products are issued as their inputs become ready (polled, so a
+            // Q / dO load still in flight for the next unit does not hold back this
+            // unit's dV and dK): dV_u once P^T_u is in X, dK_u once dS^T_u is, S^T_{u+1}
+            // once the softmax warps have read S^T_u and Q_{u+1} has landed, dP^T_{u+1}
+            // once they have read dP^T_u.  Each barrier is polled for its next phase
+            // only, which it cannot pass before the product waiting on it is issued.
+            bool ok = mbar_wait(kv_full, 0, abort_flag, p.status) && mbar_wait(qo_full, 0, abort_flag, p.status);
+            if (ok) {
                 tc_fence_after();
-                x_product(tdV, sDO + st * TILE, u);
-                mma_commit(pv_done);
-                // dP^T of the next unit once this unit's dP^T is in registers
-                if (more) {
-                    if (!mbar_wait(dp_free, u & 1, abort_flag, p.status)) break;
+                scores(0);
+                dpt(0);
+            }
+            int nv = 0, nk = 0, ns = 1, np = 1;  // next dV, dK, S^T, dP^T unit
+            uint64_t t0 = globaltimer();
+            uint32_t idle = 0;
+            while (ok && nk < nunits) {
+                bool prog = false;
+                if (nv == nk && nv < nunits && mbar_try(p_full, nv & 1)) {
                     tc_fence_after();
-                    dpt(u + 1);
+                    x_product(tdV, sDO + (nv & 1) * TILE, nv);
+                    mma_commit(pv_done);
+                    ++nv;
+                    prog = true;
                 }
-                // dK += dS^T_u Q_u
-                if (!mbar_wait(ds_full, u & 1, abort_flag, p.status)) break;
-                tc_fence_after();
-                x_product(tdK, sQ + st * TILE, u);
-                mma_commit(dk_done);
-                mma_commit(qo_empty + 8 * st);
+                if (nk < nv && mbar_try(ds_full, nk & 1)) {
+                    tc_fence_after();
+                    x_product(tdK, sQ + (nk & 1) * TILE, nk);
+                    mma_commit(dk_done);
+                    mma_commit(qo_empty + 8 * (nk & 1));
+                    ++nk;
+                    prog = true;
+                }
+                if (ns < nunits && mbar_try(s_free, (ns - 1) & 1) && mbar_try(qo_full + 8 * (ns & 1), (ns >> 1) & 1)) {
+                    tc_fence_after();
+                    scores(ns);
+                    ++ns;
+                    prog = true;
+                }
+                if (np < ns && mbar_try(dp_free, (np - 1) & 1)) {
+                    tc_fence_after();
+                    dpt(np);
+                    ++np;
+                    prog = true;
+                }
+                if (prog) {
+                    t0 = globaltimer();
+                    idle = 0;
+                } else if ((++idle & 63) == 0) {
+                    if (*abort_flag) {
+                        ok = false;
+                    } else if (globaltimer() - t0 > kWaitLimitNs) {
+                        set_status(p.status, ST_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                    }
+                }
             }
             mma_commit(dkv_done);
         }
@@ -935,13 +965,15 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             const float4* l4 = reinterpret_cast<const float4*>(lse_s + st * 128 + cg * 32);
             float pv[32];
             if (__all_sync(0xffffffffu, lo <= 0 && hi >= 31)) {
+                // one exponential in four on the FMA pipe (exp2_fma), the others on the
+                // special-function unit
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const float4 l = l4[k];
                     pv[4 * k] = ex2(fmaf(__uint_as_float(rs[4 * k]), p.scale_log2, -l.x));
                     pv[4 * k + 1] = ex2(fmaf(__uint_as_float(rs[4 * k + 1]), p.scale_log2, -l.y));
                     pv[4 * k + 2] = ex2(fmaf(__uint_as_float(rs[4 * k + 2]), p.scale_log2, -l.z));
-                    pv[4 * k + 3] = ex2(fmaf(__uint_as_float(rs[4 * k + 3]), p.scale_log2, -l.w));
+                    pv[4 * k + 3] = exp2_fma(fmaf(__uint_as_float(rs[4 * k + 3]), p.scale_log2, -l.w));
                 }
             } else {
 #pragma unroll
