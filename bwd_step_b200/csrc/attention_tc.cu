@@ -868,19 +868,19 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             uint32_t idle = 0;
             while (ok && nk < nunits) {
                 bool prog = false;
-                if (nv < ns && mbar_try(p_full, nv & 1)) {  // P^T_nv written
+                if (nv < ns && mbar_test(p_full, nv & 1)) {  // P^T_nv written
                     tc_fence_after();
                     x_product(tdV, tSt, sDO + (nv & 1) * TILE, nv);
                     ++nv;
                     prog = true;
                 }
-                if (ns < nunits && ns == nv && mbar_try(qo_full + 8 * (ns & 1), (ns >> 1) & 1)) {
+                if (ns < nunits && ns == nv && mbar_test(qo_full + 8 * (ns & 1), (ns >> 1) & 1)) {
                     tc_fence_after();
                     scores(ns);  // after dV_{ns-1}, which reads P^T from these columns
                     ++ns;
                     prog = true;
                 }
-                if (nk < np && nk < nv && mbar_try(ds_full, nk & 1)) {  // dS^T_nk written (dV_nk first)
+                if (nk < np && nk < nv && mbar_test(ds_full, nk & 1)) {  // dS^T_nk written (dV_nk first)
                     tc_fence_after();
                     x_product(tdK, tdPt, sQ + (nk & 1) * TILE, nk);
                     mma_commit(qo_empty + 8 * (nk & 1));  // the unit's last product that reads Q / dO
