@@ -438,8 +438,7 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 }
 
 // ============================================================================ backward
-// Three launches: (1) D = rowsum(dO * o) and lse * log2(e) per (row, head)
-// (or the same statistics from the epilogue of the GEMM that forms dO);
+// Three launches: (1) D = rowsum(dO * o) and lse * log2(e) per (row, head);
 // (2) the dK/dV kernel, which recomputes S^T and dP^T per (key block, query
 // block, query head), forms P^T and dS^T, accumulates dV and dK, and stores
 // every dS^T tile; (3) dq = dS K / sqrt(hd) as a plain tensor-core product
@@ -448,13 +447,12 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 // dK, dQ), deterministically: every sum runs in a fixed order, no atomics.
 //
 // The dK/dV kernel keeps every MMA at N = 128 (a 128 x 64 tile runs the
-// tensor core at well under half rate on sm_100a) and feeds the A operand of
-// the dV and dK products from TMEM: the softmax warps write P^T and dS^T as
-// bf16 back over the S^T and dP^T columns they have just read, so those two
-// products read only one operand from shared memory.  Sixteen softmax warps
-// (four per TMEM lane quarter, 32 columns each) keep the special-function
-// unit busy.
-constexpr int NTB = 576;  // dK/dV: producer, MMA, 16 softmax warps
+// tensor core at well under half rate on sm_100a) and feeds one operand of the
+// second product from TMEM: the softmax warps write P^T as bf16 back over
+// dP^T columns they have just read, and the dV MMA reads it there as the A
+// operand.  Sixteen softmax warps (four per TMEM lane quarter, 32 columns
+// each) keep the special-function unit busy.
+constexpr int NTB = 608;  // dK/dV: producer, MMA, 16 softmax warps, dS store
 constexpr int NSM = 16;   // softmax warps
 
 struct BwdParams {
@@ -697,19 +695,19 @@ __global__ void __launch_bounds__(NTQ, 1) attn_dq_ds_kernel(const __grid_constan
 // tiles at about the same time and find them in L2:
 //   warp 0      TMA: K and V once; Q_i, dO_i with their lse2 / D rows into a
 //               2-stage ring;
-//   warp 1      tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM;
-//               dV += P^T dO_i and dK += dS^T Q_i with P^T and dS^T read from
-//               TMEM as the A operand (Q_i, dO_i as MN-major operands from
-//               shared memory).  Issue order per unit: dV_u, S^T_{u+1}, dK_u,
-//               dP^T_{u+1} -- S^T_{u+1} overwrites P^T_u and dP^T_{u+1}
-//               overwrites dS^T_u only after the products that read them, in
-//               issue order.  The thread polls its barriers and issues each
-//               product once its inputs are ready;
+//   warp 1      tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM,
+//               dV += P^T dO_i and dK += dS^T Q_i with P^T, then dS^T, in one
+//               shared-memory tile X (Q_i, dO_i as MN-major operands).  Each
+//               product is issued as soon as its inputs are ready (the thread
+//               polls the four barriers), so the next unit's S^T and dP^T
+//               overlap this unit's softmax and a Q / dO load in flight does
+//               not hold back this unit's dV and dK;
 //   warps 2-17  per unit: load the warp's S^T columns (32 queries), form
-//               P^T = 2^(S^T*scale*log2e - lse2) with the causal mask and write
-//               it as packed bf16 over the columns just read; load the dP^T
-//               columns, form dS^T = P^T (dP^T - D) and write it likewise over
-//               them, and store it to global memory for the dQ product.
+//               P^T = 2^(S^T*scale*log2e - lse2) with the causal mask, write it
+//               to X, load the dP^T columns, form dS^T = P^T (dP^T - D) and
+//               write it to X once dV_u has read P^T;
+//   warp 18     TMA-stores each finished dS^T tile to global memory (for the dQ
+//               product) and reports when X may be reused.
 // dk = dK / sqrt(hd).
 template <int HD>
 struct DkvLayout {
@@ -719,7 +717,8 @@ struct DkvLayout {
     static constexpr int V = K + TILE;
     static constexpr int Q = V + TILE;         // [2] stages
     static constexpr int DO = Q + 2 * TILE;    // [2] stages
-    static constexpr int LSE = DO + 2 * TILE;  // [2][128] fp32 lse2 of the stage's queries
+    static constexpr int X = DO + 2 * TILE;    // P^T, then dS^T [128 keys x 128 queries] bf16, two 64-query boxes
+    static constexpr int LSE = X + 32768;      // [2][128] fp32 lse2 of the stage's queries
     static constexpr int DD = LSE + 1024;      // [2][128] fp32 D
     static constexpr int BAR = DD + 1024;
     static constexpr int BYTES = BAR + 256;  // the dynamic shared memory base is 1024-aligned (checked)
@@ -729,6 +728,7 @@ struct DkvLayout {
 template <int HD>
 __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQKV,
                                                             const __grid_constant__ CUtensorMap tmDO,
+                                                            const __grid_constant__ CUtensorMap tmDS,
                                                             const BwdParams p) {
     using Lay = DkvLayout<HD>;
     constexpr int KB = Lay::KB, TILE = Lay::TILE;
@@ -740,15 +740,19 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
     uint8_t* smem = smem_dyn;
     const uint32_t base = smem_u32(smem);
     const uint32_t sK = base + Lay::K, sV = base + Lay::V, sQ = base + Lay::Q, sDO = base + Lay::DO;
+    const uint32_t sX = base + Lay::X;
     const float* lse_s = reinterpret_cast<const float*>(smem + Lay::LSE);
     const float* d_s = reinterpret_cast<const float*>(smem + Lay::DD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR);
     const uint32_t b0 = smem_u32(bars);
     const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24;  // qo_*[2]
-    const uint32_t s_full = b0 + 40, dp_full = b0 + 48;  // S^T / dP^T of the unit in TMEM
-    const uint32_t p_full = b0 + 56, ds_full = b0 + 64;  // P^T / dS^T written over them
-    const uint32_t dkv_done = b0 + 72;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+    const uint32_t s_full = b0 + 40, dp_full = b0 + 48;    // S^T / dP^T of the unit in TMEM
+    const uint32_t s_free = b0 + 56, dp_free = b0 + 64;    // ... read by the softmax warps
+    const uint32_t p_full = b0 + 72, pv_done = b0 + 80;    // P^T in X / read by the dV MMAs
+    const uint32_t ds_full = b0 + 88, dk_done = b0 + 96;   // dS^T in X / read by the dK MMAs
+    const uint32_t dst_read = b0 + 104;                    // dS^T read out of X by its store
+    const uint32_t dkv_done = b0 + 112;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -764,8 +768,13 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         for (int s = 0; s < 2; ++s) { mbar_init(qo_full + 8 * s, 1); mbar_init(qo_empty + 8 * s, 1); }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
+        mbar_init(s_free, NSM);
+        mbar_init(dp_free, NSM);
         mbar_init(p_full, NSM);
+        mbar_init(pv_done, 1);
         mbar_init(ds_full, NSM);
+        mbar_init(dk_done, 1);
+        mbar_init(dst_read, 1);
         mbar_init(dkv_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -845,50 +854,55 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                 }
                 mma_commit(dp_full);
             };
-            // acc (+)= X Bop over the 128 queries of unit u: X = P^T (in the S^T columns)
-            // or dS^T (in the dP^T columns) as the TMEM A operand -- queries 16kk..16kk+15
-            // sit in the packed columns 32*(kk/2) + 8*(kk%2), written by column group
-            // kk/2 -- and Bop = dO_u or Q_u as an MN-major operand
-            auto x_product = [&](uint32_t acc, uint32_t tx, uint32_t bop, int u) {
+            // acc (+)= X Bop^T over the 128 queries of the unit: X = P^T or dS^T [keys x queries]
+            // (K-major, two 64-query boxes), Bop = dO_u or Q_u as an MN-major operand
+            auto x_product = [&](uint32_t acc, uint32_t bop, int u) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(acc, tx + 32 * (kk >> 1) + 8 * (kk & 1), smem_desc(bop + kk * 2048, 16384, 1024),
-                                id_kv, (u > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16(acc, smem_desc(sX + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                             smem_desc(bop + kk * 2048, 16384, 1024), id_kv, (u > 0 || kk > 0) ? 1u : 0u);
             };
+            // The four products are issued as their inputs become ready (polled, so a
+            // Q / dO load still in flight for the next unit does not hold back this
+            // unit's dV and dK): dV_u once P^T_u is in X, dK_u once dS^T_u is, S^T_{u+1}
+            // once the softmax warps have read S^T_u and Q_{u+1} has landed, dP^T_{u+1}
+            // once they have read dP^T_u.  Each barrier is polled for its next phase
+            // only, which it cannot pass before the product waiting on it is issued.
             bool ok = mbar_wait(kv_full, 0, abort_flag, p.status) && mbar_wait(qo_full, 0, abort_flag, p.status);
             if (ok) {
                 tc_fence_after();
                 scores(0);
                 dpt(0);
             }
-            // next dV, S^T, dK, dP^T unit; each barrier is polled for its next phase only,
-            // which it cannot pass before the product waiting on it has been issued
-            int nv = 0, ns = 1, nk = 0, np = 1;
+            int nv = 0, nk = 0, ns = 1, np = 1;  // next dV, dK, S^T, dP^T unit
             uint64_t t0 = globaltimer();
             uint32_t idle = 0;
             while (ok && nk < nunits) {
                 bool prog = false;
-                if (nv < ns && mbar_test(p_full, nv & 1)) {  // P^T_nv written
+                if (nv == nk && nv < nunits && mbar_test(p_full, nv & 1)) {
                     tc_fence_after();
-                    x_product(tdV, tSt, sDO + (nv & 1) * TILE, nv);
+                    x_product(tdV, sDO + (nv & 1) * TILE, nv);
+                    mma_commit(pv_done);
                     ++nv;
                     prog = true;
                 }
-                if (ns < nunits && ns == nv && mbar_test(qo_full + 8 * (ns & 1), (ns >> 1) & 1)) {
+                if (nk < nv && mbar_test(ds_full, nk & 1)) {
                     tc_fence_after();
-                    scores(ns);  // after dV_{ns-1}, which reads P^T from these columns
-                    ++ns;
-                    prog = true;
-                }
-                if (nk < np && nk < nv && mbar_test(ds_full, nk & 1)) {  // dS^T_nk written (dV_nk first)
-                    tc_fence_after();
-                    x_product(tdK, tdPt, sQ + (nk & 1) * TILE, nk);
-                    mma_commit(qo_empty + 8 * (nk & 1));  // the unit's last product that reads Q / dO
+                    x_product(tdK, sQ + (nk & 1) * TILE, nk);
+                    mma_commit(dk_done);
+                    mma_commit(qo_empty + 8 * (nk & 1));
                     ++nk;
                     prog = true;
                 }
-                if (np < ns && np == nk) {
-                    dpt(np);  // after dK_{np-1}, which reads dS^T from these columns
+                if (ns < nunits && mbar_test(s_free, (ns - 1) & 1) && mbar_test(qo_full + 8 * (ns & 1), (ns >> 1) & 1)) {
+                    tc_fence_after();
+                    scores(ns);
+                    ++ns;
+                    prog = true;
+                }
+                if (np < ns && mbar_test(dp_free, (np - 1) & 1)) {
+                    tc_fence_after();
+                    dpt(np);
                     ++np;
                     prog = true;
                 }
@@ -906,6 +920,22 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                 }
             }
             mma_commit(dkv_done);
+        }
+    } else if (warp == 2 + NSM) {
+        // one thread writes every finished dS^T tile to global memory (two TMA stores
+        // of [128 keys][64 queries]) and reports when shared memory may be reused
+        if (lane == 0) {
+            for (int u = 0; u < nunits; ++u) {
+                const int i = p.nqb - 1 - u / Hg, h = g * Hg + u % Hg;
+                if (!mbar_wait(ds_full, u & 1, abort_flag, p.status)) break;
+                const int trow = (int)(ds_tile(b, h, p.H, p.ntri, i, kvb) * 128);
+                tma_store_2d(&tmDS, 0, trow, sX);
+                tma_store_2d(&tmDS, 64, trow, sX + 16384);
+                bulk_commit();
+                bulk_wait_read_0();
+                mbar_arrive(dst_read);
+            }
+            bulk_wait_all();  // the tiles are in global memory before the block exits
         }
     } else {
         // warps 2..17: TMEM lane quarter q (key rows), query column group cg (32 queries)
@@ -926,6 +956,9 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             uint32_t rs[32];
             tmem_ld32_issue(tSt + lane_off + cg * 32, rs);
             tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(s_free);
             // query q0 + e sees this key when lo <= e (causal) and e <= hi (inside the row)
             const int q0 = i * 128 + cg * 32;
             const int lo = kpos - q0, hi = p.T - 1 - q0;
@@ -954,14 +987,28 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                     }
                 }
             }
-            // P^T as packed bf16 over the first 16 of the warp's own (already read) S^T columns
-            uint32_t pk[16];
+            // this warp's 32 queries of row r in the swizzled [128 keys x 64 queries] boxes of X
+            uint8_t* xrow = smem + Lay::X + (cg >> 1) * 16384 + r * 128;
+            auto put_x = [&](const float* v) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pv[2 * e], pv[2 * e + 1]);
-            tmem_st16_nowait(tSt + lane_off + cg * 32, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
+                for (int k = 0; k < 4; ++k) {
+                    const float* d = v + 8 * k;
+                    const int c8 = (cg & 1) * 4 + k;
+                    *reinterpret_cast<uint4*>(xrow + ((c8 ^ (r & 7)) << 4)) =
+                        make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
+                                   pack_bf16(d[6], d[7]));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            };
+            // X is free once the dK MMAs of the previous unit and the store of its
+            // dS^T tile to global memory (for the dQ product) have read it
+            if (u > 0 && (!warp_wait(dk_done, (u - 1) & 1, abort_flag, p.status) ||
+                          !warp_wait(dst_read, (u - 1) & 1, abort_flag, p.status))) {
+                ok = false;
+                break;
+            }
+            put_x(pv);
             if (lane == 0) mbar_arrive(p_full);
             if (!warp_wait(dp_full, u & 1, abort_flag, p.status)) {
                 ok = false;
@@ -971,6 +1018,9 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             uint32_t rd[32];
             tmem_ld32_issue(tdPt + lane_off + cg * 32, rd);
             tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dp_free);
             // dS^T = P^T (dP^T - D); masked entries have P = 0 and D, dP finite
             const float4* d4 = reinterpret_cast<const float4*>(d_s + st * 128 + cg * 32);
 #pragma unroll
@@ -981,18 +1031,13 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                 pv[4 * k + 2] *= __uint_as_float(rd[4 * k + 2]) - dd.z;
                 pv[4 * k + 3] *= __uint_as_float(rd[4 * k + 3]) - dd.w;
             }
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pv[2 * e], pv[2 * e + 1]);
-            tmem_st16_nowait(tdPt + lane_off + cg * 32, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
+            // the dV MMAs have read P^T out of X
+            if (!warp_wait(pv_done, u & 1, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            put_x(pv);
             if (lane == 0) mbar_arrive(ds_full);
-            // the tile row (key r, queries q0 .. q0 + 31) of the stored dS^T for the dQ product
-            uint4* dst = reinterpret_cast<uint4*>(p.ds + ds_tile(b, h, p.H, p.ntri, i, kvb) * (128 * 128) +
-                                                  (size_t)r * 128 + cg * 32);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
         if (ok && warp_wait(dkv_done, 0, abort_flag, p.status)) {
             tc_fence_after();
@@ -1075,9 +1120,10 @@ int dq_ds_launch(const CUtensorMap& ds, const CUtensorMap& kv, const DqdsParams&
 }
 
 template <int HD>
-int dkv_launch(const CUtensorMap& kv, const CUtensorMap& do128, const BwdParams& p, cudaStream_t s) {
+int dkv_launch(const CUtensorMap& kv, const CUtensorMap& do128, const CUtensorMap& ds, const BwdParams& p,
+               cudaStream_t s) {
     if (ensure_smem_limit((const void*)attn_dkv_tc_kernel<HD>, DkvLayout<HD>::BYTES) != cudaSuccess) return -1;
-    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NTB, DkvLayout<HD>::BYTES, s>>>(kv, do128, p);
+    attn_dkv_tc_kernel<HD><<<dim3(p.B, p.nkv, p.nqb), NTB, DkvLayout<HD>::BYTES, s>>>(kv, do128, ds, p);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
@@ -1159,7 +1205,9 @@ int attention_tc_bwd_dkv(const void* qkv, const void* dO, float* Dbuf, void* dqk
     CUtensorMap kv, do128;
     if (!ws || ws_bytes < attention_tc_workspace_bytes(B, T, H, nkv, hd)) return 1;
     if (!bwd_setup(qkv, dO, Dbuf, dqkv, ws, B, T, H, nkv, hd, status, &p, &kv, &do128)) return 1;
-    return hd == 128 ? dkv_launch<128>(kv, do128, p, s) : dkv_launch<64>(kv, do128, p, s);
+    CUtensorMap mds;
+    if (!map_rows(&mds, ws, 128, (uint64_t)B * H * ntri_of(T) * 128, 128)) return 1;
+    return hd == 128 ? dkv_launch<128>(kv, do128, mds, p, s) : dkv_launch<64>(kv, do128, mds, p, s);
 }
 
 int attention_tc_bwd_dq(const void* qkv, const void* ws, size_t ws_bytes, void* dqkv, int B, int T, int H, int nkv,
