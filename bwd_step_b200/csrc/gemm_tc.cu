@@ -35,7 +35,9 @@ constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE_BYTES = A_BYTE
 constexpr int TMEM_COLS = 2 * BN;
 constexpr int NTHREADS = 320;
 constexpr int MAX_SPLITS = 8;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 32768 + 256;  // + epilogue staging
+constexpr int STAGING_BYTES = 8 * 4096;  // epilogue staging: 4 KB per epilogue warp
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + STAGING_BYTES + 256;
+static_assert(SMEM_BYTES <= 232448, "GEMM shared memory exceeds the per-block limit");
 
 struct TcParams {
     int M, N, K;
@@ -264,7 +266,6 @@ __device__ __forceinline__ void epilogue(const TcParams& p, int ks, int row, int
 // never read into the SM.  The buffer is rewritten only after the previous
 // chunk's store has finished reading it (the next chunk is already computed
 // in registers by then).
-constexpr int STAGING_BYTES = 8 * 4096;
 
 __device__ __forceinline__ void stage_f32(uint8_t* buf, int lane, const float* v) {
 #pragma unroll
@@ -567,6 +568,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 constexpr int STAGES2 = 6;
 constexpr int STAGE2_BYTES = 2 * 128 * BK * 2;  // A 128x64 + B 128x64, bf16
 constexpr size_t SMEM2_BYTES = 1024 + (size_t)STAGES2 * STAGE2_BYTES + STAGING_BYTES + 256;
+static_assert(SMEM2_BYTES <= 232448, "paired GEMM shared memory exceeds the per-block limit");
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
