@@ -62,6 +62,12 @@ def test_tcgen05_attention(B, T, H, nkv, hd):
     _run(B, T, H, nkv, hd, 1, seed=T + H)
 
 
+def test_tcgen05_attention_long_context():
+    # the attention-heavy workload's sequence length (T = 8192, 64 query blocks), one
+    # MQA pair of query heads; the oracle holds 8192 x 8192 float64 matrices per head
+    _run(1, 8192, 2, 1, 128, 1, seed=8192)
+
+
 def test_tcgen05_attention_sharp_softmax():
     # large scores: exercises the running-max rescale of the output
     _run(1, 640, 2, 1, 128, 1, seed=3, scale=4.0)
