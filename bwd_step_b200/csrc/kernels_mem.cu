@@ -10,7 +10,6 @@
 // reduced with warp shuffles.
 #include "common.cuh"
 #include "kernels.h"
-#include <type_traits>
 #include <math.h>
 
 namespace nc {
@@ -374,73 +373,6 @@ __global__ void __launch_bounds__(256) qknorm_rope_bwd_kernel(A* dqkv, const A* 
 #pragma unroll
             for (int i = 0; i < S::EPL; ++i) gu[i] = r[k] * (gu[i] - yu[i] * dot);
             if (act) stN<A, S::EPL>(dqkv + rowoff + (size_t)(h0 + k) * HD, gu);
-        }
-    }
-}
-
-// bf16 variant for head dims 64 and 128 with 16-byte accesses: a head vector is
-// spread over HD/8 lanes (8 elements each), so one warp instruction covers
-// 32/(HD/8) heads; KU such groups are loaded before any is used.
-template <int HD>
-__global__ void __launch_bounds__(256, 3) qknorm_rope_bwd_v8_kernel(bf16* dqkv, const bf16* __restrict__ qkv,
-                                                                 const float* __restrict__ rqk,
-                                                                 const float* __restrict__ cos_t,
-                                                                 const float* __restrict__ sin_t, int M, int T, int H,
-                                                                 int nkv) {
-    constexpr int LPH = HD / 8, HPW = 32 / LPH, KU = 3;
-    const int nh = H + nkv;
-    const int m = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (m >= M) return;
-    const int sub = lane / LPH, l = lane % LPH;
-    const bool first = l < LPH / 2;
-    const int j0 = (first ? l : l - LPH / 2) * 8;  // pair index of element 0
-    const int pos = m % T;
-    float cs[8], sn[8];
-#pragma unroll
-    for (int i = 0; i < 8; i += 4) {
-        const float4 c4 = *reinterpret_cast<const float4*>(cos_t + (size_t)pos * (HD / 2) + j0 + i);
-        const float4 s4 = *reinterpret_cast<const float4*>(sin_t + (size_t)pos * (HD / 2) + j0 + i);
-        cs[i] = c4.x; cs[i + 1] = c4.y; cs[i + 2] = c4.z; cs[i + 3] = c4.w;
-        sn[i] = s4.x; sn[i + 1] = s4.y; sn[i + 2] = s4.z; sn[i + 3] = s4.w;
-    }
-    const size_t rowoff = (size_t)m * (size_t)(H + 2 * nkv) * HD + l * 8;
-    for (int h0 = 0; h0 < nh; h0 += HPW * KU) {
-        float g[KU][8], y[KU][8], r[KU];
-#pragma unroll
-        for (int k = 0; k < KU; ++k) {
-            const int h = h0 + k * HPW + sub;
-            if (h < nh) {
-                load_vec(dqkv + rowoff + (size_t)h * HD, g[k]);
-                load_vec(qkv + rowoff + (size_t)h * HD, y[k]);
-                r[k] = rqk[(size_t)m * nh + h];
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) g[k][i] = y[k][i] = 0.f;
-                r[k] = 0.f;
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < KU; ++k) {
-            if (h0 + k * HPW >= nh) break;  // warp-uniform: no head of this group is live
-            float gu[8], yu[8], dot = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float go = __shfl_xor_sync(0xffffffffu, g[k][i], LPH / 2);
-                const float yo = __shfl_xor_sync(0xffffffffu, y[k][i], LPH / 2);
-                // inverse rotation of (x1, x2): (x1 c + x2 s, -x1 s + x2 c)
-                const float g1 = first ? g[k][i] : go, g2 = first ? go : g[k][i];
-                const float y1 = first ? y[k][i] : yo, y2 = first ? yo : y[k][i];
-                gu[i] = first ? g1 * cs[i] + g2 * sn[i] : -g1 * sn[i] + g2 * cs[i];
-                yu[i] = first ? y1 * cs[i] + y2 * sn[i] : -y1 * sn[i] + y2 * cs[i];
-                dot += gu[i] * yu[i];
-            }
-#pragma unroll
-            for (int o = LPH / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-            dot *= 1.f / (float)HD;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) gu[i] = r[k] * (gu[i] - yu[i] * dot);
-            const int h = h0 + k * HPW + sub;
-            if (h < nh) store_vec(dqkv + rowoff + (size_t)h * HD, gu);
         }
     }
 }
@@ -1192,12 +1124,8 @@ template <typename A, int HD>
 static void qk_bwd_t(void* dqkv, const void* qkv, const float* rqk, const float* c, const float* sn, int M, int T,
                      int H, int nkv, cudaStream_t s) {
     const long long vecs = M;  // one warp per position
-    if constexpr (std::is_same<A, bf16>::value && (HD == 64 || HD == 128))
-        qknorm_rope_bwd_v8_kernel<HD><<<(unsigned)((vecs + 7) / 8), 256, 0, s>>>((bf16*)dqkv, (const bf16*)qkv, rqk,
-                                                                                c, sn, M, T, H, nkv);
-    else
-        qknorm_rope_bwd_kernel<A, HD><<<(unsigned)((vecs + 7) / 8), 256, 0, s>>>((A*)dqkv, (const A*)qkv, rqk, c, sn,
-                                                                                  M, T, H, nkv);
+    qknorm_rope_bwd_kernel<A, HD><<<(unsigned)((vecs + 7) / 8), 256, 0, s>>>((A*)dqkv, (const A*)qkv, rqk, c, sn, M,
+                                                                              T, H, nkv);
 }
 
 template <typename A>
