@@ -25,7 +25,8 @@ cudaError_t launch_embed_norm_fwd(DType wt, const int32_t* idx, const void* wte,
 // y = x * r, r = (mean(x^2)+eps)^-1/2 per row; y in activation type.
 cudaError_t launch_rmsnorm_fwd(DType at, const float* x, void* y, float* r, int M, int d, cudaStream_t s);
 // dx = (accumulate ? dx : 0) + r*(dy - y*mean(dy*y)); optional dxb = dx in activation type.
-cudaError_t launch_rmsnorm_bwd(DType at, const float* dy, const void* y, const float* r, float* dx,
+// dy is fp32, or in the activation type when dy_act.
+cudaError_t launch_rmsnorm_bwd(DType at, const void* dy, bool dy_act, const void* y, const float* r, float* dx,
                                bool accumulate, void* dxb, int M, int d, cudaStream_t s);
 // de = gradient through the token-embedding norm, recomputing y = wte[idx]*r0.
 cudaError_t launch_embed_norm_bwd(DType wt, const float* dx, const int32_t* idx, const void* wte,

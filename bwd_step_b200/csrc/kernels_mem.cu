@@ -161,14 +161,14 @@ __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, A* __restrict__ 
     }
 }
 
-template <typename A, int NCH>
-__global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const A* __restrict__ y,
+template <typename A, typename DY, int NCH>
+__global__ void rmsnorm_bwd_kernel(const DY* __restrict__ dy, const A* __restrict__ y,
                                    const float* __restrict__ r, float* dx, bool accumulate, A* dxb,
                                    int M, int d) {
     int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
     int lane = threadIdx.x & 31;
     if (row >= M) return;
-    const float* g = dy + (size_t)row * d;
+    const DY* g = dy + (size_t)row * d;
     const A* yy = y + (size_t)row * d;
     float* out = dx + (size_t)row * d;
     const float rr = r[row];
@@ -1069,36 +1069,34 @@ cudaError_t launch_rmsnorm_fwd(DType at, const float* x, void* y, float* r, int 
     return cudaGetLastError();
 }
 
-cudaError_t launch_rmsnorm_bwd(DType at, const float* dy, const void* y, const float* r, float* dx,
+cudaError_t launch_rmsnorm_bwd(DType at, const void* dy, bool dy_act, const void* y, const float* r, float* dx,
                                bool accumulate, void* dxb, int M, int d, cudaStream_t s) {
     const int nch = (d + 255) / 256;
-#define NC_RMS_BWD(A, N) \
-    rmsnorm_bwd_kernel<A, N><<<row_blocks(M), 256, 0, s>>>(dy, (const A*)y, r, dx, accumulate, (A*)dxb, M, d)
+#define NC_RMS_BWD(A, DY, N)                                                                                  \
+    rmsnorm_bwd_kernel<A, DY, N><<<row_blocks(M), 256, 0, s>>>((const DY*)dy, (const A*)y, r, dx, accumulate, \
+                                                             (A*)dxb, M, d)
+#define NC_RMS_BWD_N(A, DY)                     \
+    switch (nch) {                              \
+        case 1: NC_RMS_BWD(A, DY, 1); break;    \
+        case 2: NC_RMS_BWD(A, DY, 2); break;    \
+        case 3: NC_RMS_BWD(A, DY, 3); break;    \
+        case 4: NC_RMS_BWD(A, DY, 4); break;    \
+        case 5: NC_RMS_BWD(A, DY, 5); break;    \
+        case 6: NC_RMS_BWD(A, DY, 6); break;    \
+        case 7: NC_RMS_BWD(A, DY, 7); break;    \
+        case 8: NC_RMS_BWD(A, DY, 8); break;    \
+        default: NC_RMS_BWD(A, DY, 0); break;   \
+    }
     if (at == DT_BF16) {
-        switch (nch) {
-            case 1: NC_RMS_BWD(bf16, 1); break;
-            case 2: NC_RMS_BWD(bf16, 2); break;
-            case 3: NC_RMS_BWD(bf16, 3); break;
-            case 4: NC_RMS_BWD(bf16, 4); break;
-            case 5: NC_RMS_BWD(bf16, 5); break;
-            case 6: NC_RMS_BWD(bf16, 6); break;
-            case 7: NC_RMS_BWD(bf16, 7); break;
-            case 8: NC_RMS_BWD(bf16, 8); break;
-            default: NC_RMS_BWD(bf16, 0); break;
+        if (dy_act) {
+            NC_RMS_BWD_N(bf16, bf16)
+        } else {
+            NC_RMS_BWD_N(bf16, float)
         }
     } else {
-        switch (nch) {
-            case 1: NC_RMS_BWD(float, 1); break;
-            case 2: NC_RMS_BWD(float, 2); break;
-            case 3: NC_RMS_BWD(float, 3); break;
-            case 4: NC_RMS_BWD(float, 4); break;
-            case 5: NC_RMS_BWD(float, 5); break;
-            case 6: NC_RMS_BWD(float, 6); break;
-            case 7: NC_RMS_BWD(float, 7); break;
-            case 8: NC_RMS_BWD(float, 8); break;
-            default: NC_RMS_BWD(float, 0); break;
-        }
+        NC_RMS_BWD_N(float, float)
     }
+#undef NC_RMS_BWD_N
 #undef NC_RMS_BWD
     count_launch();
     return cudaGetLastError();

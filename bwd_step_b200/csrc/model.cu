@@ -463,7 +463,7 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     // ---- backward through the blocks
     float* dx = c.at<float>(c.p.dx);
     void* dxb = c.at(c.p.dxb);
-    { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (8.0 * d + 2.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, xf, c.at<float>(c.p.rf), dx, false, dxb, M, d, s)); }
+    { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (8.0 * d + 2.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, false, xf, c.at<float>(c.p.rf), dx, false, dxb, M, d, s)); }
     void* du = c.at(c.p.du);
     void* dO = c.at(c.p.dO);
     void* dqkv = c.at(c.p.dqkv);
@@ -487,10 +487,10 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
         RG(run_gemm(c, g1, P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, d, F, M, dxb, d, false, c.mlp_h(lb), F, false, EPI_STORE, G(base + 5), F, DT_F32),
                     P_GEMM_WGRAD));
-        RG(run_gemm(c, mk(m, M, d, F, du, F, true, w.wfc(l), d, false, EPI_STORE, gbuf, d, DT_F32), P_GEMM_DGRAD));
+        RG(run_gemm(c, mk(m, M, d, F, du, F, true, w.wfc(l), d, false, EPI_STORE, gbuf, d, m->at), P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32),
                     P_GEMM_WGRAD));
-        { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (12.0 * d + 2.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_m, (float*)(lb + c.p.l_r2), dx, true, dxb, M, d, s)); }
+        { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (8.0 * d + 3.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, true, lb + c.p.l_m, (float*)(lb + c.p.l_r2), dx, true, dxb, M, d, s)); }
         // attention: x_mid = x_in + o Wo^T; dO = dx Wo, with the softmax-backward statistics
         // D = rowsum(dO * o) and lse*log2(e) formed in the same GEMM's epilogue (tensor-core path)
         bool stats_ready = false;
@@ -510,13 +510,13 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
                           DT_F32), P_GEMM_WGRAD));
         RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), (float*)(lb + c.p.l_rqk),
                          dqkv, stats_ready));
-        RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, DT_F32),
+        RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, m->at),
                     P_GEMM_DGRAD));
         RG(run_gemm(c, mk(m, Nqkv, d, M, dqkv, Nqkv, false, lb + c.p.l_a, d, false, EPI_STORE, G(base), d,
                           DT_F32), P_GEMM_WGRAD));
         {
-            Prof pr(c, P_NORM_BWD, 0.0, (double)M * (12.0 * d + (l > 0 ? 2.0 : 1.0) * A * d + 4.0));
-            CK(launch_rmsnorm_bwd(m->at, gbuf, lb + c.p.l_a, (float*)(lb + c.p.l_r1), dx, true,
+            Prof pr(c, P_NORM_BWD, 0.0, (double)M * (8.0 * d + (l > 0 ? 3.0 : 2.0) * A * d + 4.0));
+            CK(launch_rmsnorm_bwd(m->at, gbuf, true, lb + c.p.l_a, (float*)(lb + c.p.l_r1), dx, true,
                                   l > 0 ? dxb : nullptr, M, d, s));
         }
         RG(bucket_done(m->L - l));  // this layer's six weight gradients
