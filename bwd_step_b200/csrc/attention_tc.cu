@@ -70,6 +70,32 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Pairs of fp32 in one 64-bit register for the sm_100 packed f32x2 arithmetic
+// (one instruction does the work of two), and the three-input maximum.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Store 32 consecutive 32-bit columns of this thread's TMEM lane (no wait).
 __device__ __forceinline__ void tmem_st32u_nowait(uint32_t taddr, const uint32_t* v) {
     asm volatile(
@@ -341,23 +367,25 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 for (int k = 0; k < 4; ++k) mx4[k] = -INFINITY;
                 if (diag) {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], c > r ? -INFINITY : __uint_as_float(sr[c]));
+                    for (int c = 0; c < 128; c += 2)
+                        mx4[(c >> 1) & 3] = max3f(mx4[(c >> 1) & 3], c > r ? -INFINITY : __uint_as_float(sr[c]),
+                                                  c + 1 > r ? -INFINITY : __uint_as_float(sr[c + 1]));
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(sr[c]));
+                    for (int c = 0; c < 128; c += 2)
+                        mx4[(c >> 1) & 3] = max3f(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
                 }
                 float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
                 mx *= p.scale_log2;
                 const bool rescale = mx > m + 8.f;
                 const float mu = rescale ? mx : m;
                 const float alpha = rescale ? ex2(m - mx) : 1.f;
-                // P = 2^(s*scale - mu) as packed bf16 over the first 64 score columns,
-                // the row sum as four independent partial sums; with kPoly one score in
-                // kPolyEvery comes from the FMA pipe (full blocks only: exp2_fma does not
-                // take the masked -inf scores of the diagonal block)
-                float sum4[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) sum4[k] = 0.f;
+                // P = 2^(s*scale - mu) as packed bf16 over the first 64 score columns (the
+                // scaling as packed f32x2 FMAs), the row sum as two partial sums of pairs;
+                // with kPoly one score in kPolyEvery comes from the FMA pipe (full blocks
+                // only: exp2_fma does not take the masked -inf scores of the diagonal block)
+                const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nmu2 = f2_pack(-mu, -mu);
+                uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
                 auto exp_pack = [&](auto poly) {
                     constexpr bool kPoly = decltype(poly)::value;
                     constexpr int kPE = kPolyEvery > 0 ? kPolyEvery : 2;
@@ -367,15 +395,16 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 #pragma unroll
                         for (int c = 0; c < 16; c += 2) {
                             const int cc = 16 * q8 + c;
-                            float x0 = fmaf(__uint_as_float(sr[cc]), p.scale_log2, -mu);
-                            float x1 = fmaf(__uint_as_float(sr[cc + 1]), p.scale_log2, -mu);
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])), sc2, nmu2),
+                                      x0, x1);
                             if (!kPoly && diag) {
                                 if (cc > r) x0 = -INFINITY;
                                 if (cc + 1 > r) x1 = -INFINITY;
                             }
                             const float e0 = ex2(x0);
                             const float e1 = (kPoly && (c / 2) % (kPE / 2) == kPE / 2 - 1) ? exp2_fma(x1) : ex2(x1);
-                            sum4[(c >> 1) & 3] += e0 + e1;
+                            sum2[(c >> 1) & 1] = f2_add(sum2[(c >> 1) & 1], f2_pack(e0, e1));
                             pk[c >> 1] = pack_bf16(e0, e1);
                         }
                         tmem_st8_nowait(tS + 8 * q8, pk);
@@ -384,7 +413,10 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
                 if (!diag && kPolyEvery > 0) exp_pack(std::true_type{});
                 else exp_pack(std::false_type{});
                 tmem_wait_st();
-                const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+                float s00, s01, s10, s11;
+                f2_unpack(sum2[0], s00, s01);
+                f2_unpack(sum2[1], s10, s11);
+                const float sum = (s00 + s01) + (s10 + s11);
                 if (j > 0 && __any_sync(0xffffffffu, rescale)) {
                     // O_x += P(j-1) V has completed (S(j) was issued after it and has landed);
                     // O_x += P(j) V waits for this warp's hand-over below
