@@ -90,6 +90,11 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -490,8 +495,9 @@ constexpr int NSM = 16;   // softmax warps
 struct BwdParams {
     int B, T, H, nkv, nqb, ntri;
     float scale_log2, scale;
-    const float* D;     // [B, H, Tp] rowsum(dO * o)
-    const float* lse2;  // [B, H, Tp] lse * log2(e) (both zero past the sequence end)
+    const float* D;     // [B, H, Tp] -rowsum(dO * o)
+    const float* lse2;  // [B, H, Tp] -lse * log2(e) (both zero past the sequence end; negated so the
+                        // softmax warps add them with packed f32x2 FMAs)
     bf16* dqkv;
     bf16* ds;           // dS^T tiles (see ds_tile), written by the dK/dV kernel
     int* status;
@@ -544,8 +550,8 @@ __global__ void __launch_bounds__(256) attn_bwd_stats_kernel(const bf16* __restr
 #pragma unroll
     for (int m = G / 2; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
     if (w < n && k == 0) {
-        D[w] = s;
-        lse2[w] = live ? lse[w] * kLog2e : 0.f;
+        D[w] = -s;
+        lse2[w] = live ? -lse[w] * kLog2e : 0.f;
     }
 }
 
@@ -1000,12 +1006,18 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                 // one exponential in four on the FMA pipe (exp2_fma), the others on the
                 // special-function unit
 #pragma unroll
+                const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
                 for (int k = 0; k < 8; ++k) {
-                    const float4 l = l4[k];
-                    pv[4 * k] = ex2(fmaf(__uint_as_float(rs[4 * k]), p.scale_log2, -l.x));
-                    pv[4 * k + 1] = ex2(fmaf(__uint_as_float(rs[4 * k + 1]), p.scale_log2, -l.y));
-                    pv[4 * k + 2] = ex2(fmaf(__uint_as_float(rs[4 * k + 2]), p.scale_log2, -l.z));
-                    pv[4 * k + 3] = exp2_fma(fmaf(__uint_as_float(rs[4 * k + 3]), p.scale_log2, -l.w));
+                    const float4 l = l4[k];  // -lse2
+                    float x0, x1, x2, x3;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[4 * k]), __uint_as_float(rs[4 * k + 1])), sc2,
+                                     f2_pack(l.x, l.y)), x0, x1);
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(rs[4 * k + 2]), __uint_as_float(rs[4 * k + 3])), sc2,
+                                     f2_pack(l.z, l.w)), x2, x3);
+                    pv[4 * k] = ex2(x0);
+                    pv[4 * k + 1] = ex2(x1);
+                    pv[4 * k + 2] = ex2(x2);
+                    pv[4 * k + 3] = exp2_fma(x3);
                 }
             } else {
 #pragma unroll
@@ -1015,7 +1027,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
                         const int e = 4 * k + t;
-                        pv[e] = (e >= lo && e <= hi) ? ex2(fmaf(__uint_as_float(rs[e]), p.scale_log2, -lv[t])) : 0.f;
+                        pv[e] = (e >= lo && e <= hi) ? ex2(fmaf(__uint_as_float(rs[e]), p.scale_log2, lv[t])) : 0.f;
                     }
                 }
             }
@@ -1053,15 +1065,19 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dp_free);
-            // dS^T = P^T (dP^T - D); masked entries have P = 0 and D, dP finite
+            // dS^T = P^T (dP^T - D) (d_s holds -D); masked entries have P = 0 and D, dP finite
             const float4* d4 = reinterpret_cast<const float4*>(d_s + st * 128 + cg * 32);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const float4 dd = d4[k];
-                pv[4 * k] *= __uint_as_float(rd[4 * k]) - dd.x;
-                pv[4 * k + 1] *= __uint_as_float(rd[4 * k + 1]) - dd.y;
-                pv[4 * k + 2] *= __uint_as_float(rd[4 * k + 2]) - dd.z;
-                pv[4 * k + 3] *= __uint_as_float(rd[4 * k + 3]) - dd.w;
+                f2_unpack(f2_mul(f2_pack(pv[4 * k], pv[4 * k + 1]),
+                                 f2_add(f2_pack(__uint_as_float(rd[4 * k]), __uint_as_float(rd[4 * k + 1])),
+                                        f2_pack(dd.x, dd.y))),
+                          pv[4 * k], pv[4 * k + 1]);
+                f2_unpack(f2_mul(f2_pack(pv[4 * k + 2], pv[4 * k + 3]),
+                                 f2_add(f2_pack(__uint_as_float(rd[4 * k + 2]), __uint_as_float(rd[4 * k + 3])),
+                                        f2_pack(dd.z, dd.w))),
+                          pv[4 * k + 2], pv[4 * k + 3]);
             }
             // the dV MMAs have read P^T out of X
             if (!warp_wait(pv_done, u & 1, abort_flag, p.status)) {

@@ -12,8 +12,8 @@ bool attention_tc_bwd_supported(int hd);
 // per causal (query block, key block) pair of every (batch row, query head).
 size_t attention_tc_workspace_bytes(int B, int T, int H, int nkv, int hd);
 // The whole backward: stats, then dk/dv (storing dS), then dq.  Dbuf holds
-// attn_dbuf_elems(B, T, H) floats: D = rowsum(dO * o) and lse * log2(e), both
-// [B, H, attn_tpad(T)].
+// attn_dbuf_elems(B, T, H) floats: -D = -rowsum(dO * o) and -lse * log2(e), both
+// [B, H, attn_tpad(T)] (negated: the dK/dV softmax adds them).
 int attention_tc_bwd(const void* qkv, const void* o, const void* dO, const float* lse, float* Dbuf, void* dqkv,
                      int B, int T, int H, int nkv, int hd, void* ws, size_t ws_bytes, int* status, cudaStream_t s);
 // Its three launches, in order.

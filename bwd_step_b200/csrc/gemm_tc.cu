@@ -78,7 +78,7 @@ struct RowCtx {
 // (softmax backward: dS = P (dP - D) with D = rowsum(dO * o)): the 32-column
 // chunk n0.. of this row is rounded to the stored bf16 dO (so D uses the same
 // values as the dP product), multiplied with o and summed; at the last chunk
-// of a head, D and lse * log2(e) are written for (batch row, head, position).
+// of a head, -D and -lse * log2(e) are written for (batch row, head, position).
 __device__ __forceinline__ void attn_do_chunk(const TcParams& p, int row, int n0, float* v, RowCtx& rc) {
     constexpr float kL2e = 1.44269504088896340736f;
     const bf16* o = p.aux + (int64_t)row * p.ldaux + n0;
@@ -97,8 +97,8 @@ __device__ __forceinline__ void attn_do_chunk(const TcParams& p, int row, int n0
     if ((n0 + 32) % p.hd == 0) {  // last chunk of head h
         const int h = n0 / p.hd, b = row / p.T, t = row % p.T;
         const size_t i = ((size_t)b * p.attn_H + h) * (size_t)attn_tpad(p.T) + t;
-        p.attn_d[i] = rc.sum;
-        p.attn_lse2[i] = p.attn_lse[i] * kL2e;
+        p.attn_d[i] = -rc.sum;  // both negated: the attention backward adds them
+        p.attn_lse2[i] = -p.attn_lse[i] * kL2e;
         rc.sum = 0.f;
     }
 }

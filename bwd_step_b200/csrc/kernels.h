@@ -108,9 +108,9 @@ enum Epi : int {
                         // fp32 into zt[row], ut[row] (tcgen05 only)
     EPI_ROWSCALE = 7,   // C = acc * rs[row]                 (C fp32; tcgen05 only)
     EPI_ATTN_DO = 8,    // attention output gradient dO: C = acc (bf16), and per (row, head of hd
-                        // columns) D = sum of C * aux (aux = o, the attention output) and
-                        // lse * log2(e), into the [B, H, Tp] statistics of the backward
-                        // (row = b T + t; tcgen05 only)
+                        // columns) -D = -(sum of C * aux) (aux = o, the attention output) and
+                        // -lse * log2(e), into the [B, H, Tp] statistics of the tensor-core
+                        // backward (row = b T + t; tcgen05 only)
 };
 
 struct GemmDesc {
@@ -160,7 +160,8 @@ cudaError_t gemm_simt(const GemmDesc& g, cudaStream_t s);
 // multiple of 128 (one query block): index (b*H + h)*attn_tpad(T) + t.
 __host__ __device__ inline int attn_tpad(int T) { return (T + 127) / 128 * 128; }
 inline size_t attn_stat_elems(int B, int T, int H) { return (size_t)B * H * attn_tpad(T); }
-// The backward's buffer: D, then (tensor-core path) lse * log2(e), each attn_stat_elems.
+// The backward's buffer: D (tensor-core path: -D), then (tensor-core path) -lse * log2(e),
+// each attn_stat_elems.
 inline size_t attn_dbuf_elems(int B, int T, int H) { return 2 * attn_stat_elems(B, T, H); }
 cudaError_t launch_attention_fwd_simt(DType at, const void* qkv, void* o, float* lse, int B, int T, int H,
                                       int nkv, int hd, cudaStream_t s);
