@@ -141,15 +141,24 @@ __device__ __forceinline__ void lmhead_chunk(const TcParams& p, int row, int n0,
             }
     }
     const int nv = min(32, p.N - n0);
-    float sum = 0.f;
+    // the scaling, the exponent and the sum as packed f32x2 operations on column pairs
+    const uint64_t ic2 = f2_pack(ic, ic), cl2x = f2_pack(cl2, cl2), ncl2 = f2_pack(-cl2, -cl2);
+    uint64_t s2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float t = tanh_sfu(v[i] * ic);
-        const float e = ex2((t - 1.f) * cl2);
-        if (i < nv) sum += e;
-        v[i] = e * (1.f - t * t);
+    for (int i = 0; i < 32; i += 2) {
+        float a0, a1, x0, x1;
+        f2_unpack(f2_mul(f2_pack(v[i], v[i + 1]), ic2), a0, a1);
+        const float t0 = tanh_sfu(a0), t1 = tanh_sfu(a1);
+        f2_unpack(f2_fma(f2_pack(t0, t1), cl2x, ncl2), x0, x1);  // (t - 1) cap log2(e)
+        const float e0 = ex2(x0), e1 = ex2(x1);
+        s2[(i >> 1) & 1] = f2_add(s2[(i >> 1) & 1], f2_pack(i < nv ? e0 : 0.f, i + 1 < nv ? e1 : 0.f));
+        v[i] = e0 * (1.f - t0 * t0);
+        v[i + 1] = e1 * (1.f - t1 * t1);
     }
-    rc.sum += sum;
+    float a, b, c, d;
+    f2_unpack(s2[0], a, b);
+    f2_unpack(s2[1], c, d);
+    rc.sum += (a + b) + (c + d);
 }
 
 __device__ __forceinline__ void decode(const TcParams& p, int u, int& tm, int& tn, int& ks) {
