@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(256) qknorm_rope_fwd_kernel(A* qkv, float* __r
 // vectors of the position are processed G at a time with all their loads
 // issued before any of them is used.
 template <typename A, int HD>
-__global__ void __launch_bounds__(256) qknorm_rope_bwd_kernel(A* dqkv, const A* __restrict__ qkv,
+__global__ void __launch_bounds__(256, 4) qknorm_rope_bwd_kernel(A* dqkv, const A* __restrict__ qkv,
                                                               const float* __restrict__ rqk,
                                                               const float* __restrict__ cos_t,
                                                               const float* __restrict__ sin_t, int M, int T, int H,
