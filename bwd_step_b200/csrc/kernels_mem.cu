@@ -191,19 +191,30 @@ __global__ void rmsnorm_bwd_kernel(const DY* __restrict__ dy, const A* __restric
             }
         }
         dot = warp_sum(dot) / (float)d;
+        // the row's contribution into a (b is dead afterwards), then every chunk of the
+        // accumulated gradient loaded at once into b's registers (the loads in flight
+        // together), added and stored
+#pragma unroll
+        for (int i = 0; i < NCH; ++i)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) a[i][k] = rr * (a[i][k] - b[i][k] * dot);
+        if (accumulate) {
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) {
+                const int c = lane * 8 + 256 * i;
+                if (c < d) load8(out + c, b[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < NCH; ++i)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) a[i][k] += b[i][k];
+        }
 #pragma unroll
         for (int i = 0; i < NCH; ++i) {
             const int c = lane * 8 + 256 * i;
             if (c < d) {
-                float o[8];
-                if (accumulate) load8(out + c, o);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float v = rr * (a[i][k] - b[i][k] * dot);
-                    o[k] = accumulate ? o[k] + v : v;
-                }
-                store8(out + c, o);
-                if (dxb) store8(dxb + (size_t)row * d + c, o);
+                store8(out + c, a[i]);
+                if (dxb) store8(dxb + (size_t)row * d + c, a[i]);
             }
         }
     } else {
