@@ -710,16 +710,18 @@ __global__ void __launch_bounds__(NTQ, 1) attn_dq_ds_kernel(const __grid_constan
 //   warp 0      TMA: K and V once; Q_i, dO_i with their lse2 / D rows into a
 //               2-stage ring;
 //   warp 1      tcgen05.mma: S^T = K Q_i^T and dP^T = V dO_i^T into TMEM,
-//               dV += P^T dO_i and dK += dS^T Q_i with P^T, then dS^T, in one
+//               dV += P^T dO_i with P^T read from TMEM (the A operand, written
+//               over the dP^T columns) and dK += dS^T Q_i with dS^T from one
 //               shared-memory tile X (Q_i, dO_i as MN-major operands).  Each
 //               product is issued as soon as its inputs are ready (the thread
-//               polls the four barriers), so the next unit's S^T and dP^T
-//               overlap this unit's softmax and a Q / dO load in flight does
-//               not hold back this unit's dV and dK;
+//               polls its barriers): the next unit's S^T once the softmax warps
+//               have read this unit's, its dP^T after this unit's dV (which
+//               reads P^T from those columns), dK once dS^T is in X;
 //   warps 2-17  per unit: load the warp's S^T columns (32 queries), form
-//               P^T = 2^(S^T*scale*log2e - lse2) with the causal mask, write it
-//               to X, load the dP^T columns, form dS^T = P^T (dP^T - D) and
-//               write it to X once dV_u has read P^T;
+//               P^T = 2^(S^T*scale*log2e - lse2) with the causal mask, load the
+//               dP^T columns and write P^T (bf16) over them, form
+//               dS^T = P^T (dP^T - D) and write it to X once the previous unit's
+//               dK and dS^T store have read X;
 //   warp 18     TMA-stores each finished dS^T tile to global memory (for the dQ
 //               product) and reports when X may be reused.
 // dk = dK / sqrt(hd).
@@ -731,7 +733,7 @@ struct DkvLayout {
     static constexpr int V = K + TILE;
     static constexpr int Q = V + TILE;         // [2] stages
     static constexpr int DO = Q + 2 * TILE;    // [2] stages
-    static constexpr int X = DO + 2 * TILE;    // P^T, then dS^T [128 keys x 128 queries] bf16, two 64-query boxes
+    static constexpr int X = DO + 2 * TILE;    // dS^T [128 keys x 128 queries] bf16, two 64-query boxes
     static constexpr int LSE = X + 32768;      // [2][128] fp32 lse2 of the stage's queries
     static constexpr int DD = LSE + 1024;      // [2][128] fp32 D
     static constexpr int BAR = DD + 1024;
@@ -761,8 +763,8 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
     const uint32_t b0 = smem_u32(bars);
     const uint32_t kv_full = b0, qo_full = b0 + 8, qo_empty = b0 + 24;  // qo_*[2]
     const uint32_t s_full = b0 + 40, dp_full = b0 + 48;    // S^T / dP^T of the unit in TMEM
-    const uint32_t s_free = b0 + 56, dp_free = b0 + 64;    // ... read by the softmax warps
-    const uint32_t p_full = b0 + 72, pv_done = b0 + 80;    // P^T in X / read by the dV MMAs
+    const uint32_t s_free = b0 + 56;                       // S^T read by the softmax warps
+    const uint32_t p_full = b0 + 72;                       // P^T written over the dP^T columns
     const uint32_t ds_full = b0 + 88, dk_done = b0 + 96;   // dS^T in X / read by the dK MMAs
     const uint32_t dst_read = b0 + 104;                    // dS^T read out of X by its store
     const uint32_t dkv_done = b0 + 112;
@@ -783,9 +785,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
         mbar_init(s_free, NSM);
-        mbar_init(dp_free, NSM);
         mbar_init(p_full, NSM);
-        mbar_init(pv_done, 1);
         mbar_init(ds_full, NSM);
         mbar_init(dk_done, 1);
         mbar_init(dst_read, 1);
@@ -870,6 +870,15 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             };
             // acc (+)= X Bop^T over the 128 queries of the unit: X = P^T or dS^T [keys x queries]
             // (K-major, two 64-query boxes), Bop = dO_u or Q_u as an MN-major operand
+            // dV += P^T dO_u with P^T as the TMEM A operand: queries 16kk..16kk+15 sit in the
+            // packed columns 32*(kk/2) + 8*(kk%2) of dP^T (written by column group kk/2)
+            auto pv_product = [&](int u) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tdV, tdPt + 32 * (kk >> 1) + 8 * (kk & 1),
+                                smem_desc(sDO + (u & 1) * TILE + kk * 2048, 16384, 1024), id_kv,
+                                (u > 0 || kk > 0) ? 1u : 0u);
+            };
             auto x_product = [&](uint32_t acc, uint32_t bop, int u) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -893,10 +902,9 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             uint32_t idle = 0;
             while (ok && nk < nunits) {
                 bool prog = false;
-                if (nv == nk && nv < nunits && mbar_test(p_full, nv & 1)) {
+                if (nv < np && mbar_test(p_full, nv & 1)) {  // P^T_nv written over dP^T
                     tc_fence_after();
-                    x_product(tdV, sDO + (nv & 1) * TILE, nv);
-                    mma_commit(pv_done);
+                    pv_product(nv);
                     ++nv;
                     prog = true;
                 }
@@ -914,8 +922,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
                     ++ns;
                     prog = true;
                 }
-                if (np < ns && mbar_test(dp_free, (np - 1) & 1)) {
-                    tc_fence_after();
+                if (np < ns && np == nv) {  // after dV_{np-1}, which reads P^T from these columns
                     dpt(np);
                     ++np;
                     prog = true;
@@ -960,7 +967,7 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
         bool ok = true;
         for (int u = 0; u < nunits; ++u) {
             const int st = u & 1;
-            const int i = p.nqb - 1 - u / Hg, h = g * Hg + u % Hg;
+            const int i = p.nqb - 1 - u / Hg;
             if (!warp_wait(s_full, u & 1, abort_flag, p.status) ||
                 !warp_wait(qo_full + 8 * st, (u >> 1) & 1, abort_flag, p.status)) {
                 ok = false;
@@ -981,8 +988,8 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             if (__all_sync(0xffffffffu, lo <= 0 && hi >= 31)) {
                 // one exponential in four on the FMA pipe (exp2_fma), the others on the
                 // special-function unit
-#pragma unroll
                 const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+#pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const float4 l = l4[k];  // -lse2
                     float x0, x1, x2, x3;
@@ -1009,27 +1016,10 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             }
             // this warp's 32 queries of row r in the swizzled [128 keys x 64 queries] boxes of X
             uint8_t* xrow = smem + Lay::X + (cg >> 1) * 16384 + r * 128;
-            auto put_x = [&](const float* v) {
+            // P^T rounded to bf16 (the values dV uses; dS^T is formed from them as well)
+            uint32_t pk[16];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float* d = v + 8 * k;
-                    const int c8 = (cg & 1) * 4 + k;
-                    *reinterpret_cast<uint4*>(xrow + ((c8 ^ (r & 7)) << 4)) =
-                        make_uint4(pack_bf16(d[0], d[1]), pack_bf16(d[2], d[3]), pack_bf16(d[4], d[5]),
-                                   pack_bf16(d[6], d[7]));
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            };
-            // X is free once the dK MMAs of the previous unit and the store of its
-            // dS^T tile to global memory (for the dQ product) have read it
-            if (u > 0 && (!warp_wait(dk_done, (u - 1) & 1, abort_flag, p.status) ||
-                          !warp_wait(dst_read, (u - 1) & 1, abort_flag, p.status))) {
-                ok = false;
-                break;
-            }
-            put_x(pv);
-            if (lane == 0) mbar_arrive(p_full);
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pv[2 * e], pv[2 * e + 1]);
             if (!warp_wait(dp_full, u & 1, abort_flag, p.status)) {
                 ok = false;
                 break;
@@ -1038,29 +1028,47 @@ __global__ void __launch_bounds__(NTB, 1) attn_dkv_tc_kernel(const __grid_consta
             uint32_t rd[32];
             tmem_ld32_issue(tdPt + lane_off + cg * 32, rd);
             tmem_wait_ld();
+            // P^T over the first 16 of the warp's own (just read) dP^T columns
+            tmem_st16_nowait(tdPt + lane_off + cg * 32, pk);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(dp_free);
+            if (lane == 0) mbar_arrive(p_full);
             // dS^T = P^T (dP^T - D) (d_s holds -D); masked entries have P = 0 and D, dP finite
             const float4* d4 = reinterpret_cast<const float4*>(d_s + st * 128 + cg * 32);
+            uint32_t dk[16];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const float4 dd = d4[k];
-                f2_unpack(f2_mul(f2_pack(pv[4 * k], pv[4 * k + 1]),
+                const float2 p01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[2 * k]));
+                const float2 p23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[2 * k + 1]));
+                float d0, d1, d2, d3;
+                f2_unpack(f2_mul(f2_pack(p01.x, p01.y),
                                  f2_add(f2_pack(__uint_as_float(rd[4 * k]), __uint_as_float(rd[4 * k + 1])),
                                         f2_pack(dd.x, dd.y))),
-                          pv[4 * k], pv[4 * k + 1]);
-                f2_unpack(f2_mul(f2_pack(pv[4 * k + 2], pv[4 * k + 3]),
+                          d0, d1);
+                f2_unpack(f2_mul(f2_pack(p23.x, p23.y),
                                  f2_add(f2_pack(__uint_as_float(rd[4 * k + 2]), __uint_as_float(rd[4 * k + 3])),
                                         f2_pack(dd.z, dd.w))),
-                          pv[4 * k + 2], pv[4 * k + 3]);
+                          d2, d3);
+                dk[2 * k] = pack_bf16(d0, d1);
+                dk[2 * k + 1] = pack_bf16(d2, d3);
             }
-            // the dV MMAs have read P^T out of X
-            if (!warp_wait(pv_done, u & 1, abort_flag, p.status)) {
+            // X is free once the dK MMAs of the previous unit and the store of its dS^T tile
+            // to global memory (for the dQ product) have read it
+            if (u > 0 && (!warp_wait(dk_done, (u - 1) & 1, abort_flag, p.status) ||
+                          !warp_wait(dst_read, (u - 1) & 1, abort_flag, p.status))) {
                 ok = false;
                 break;
             }
-            put_x(pv);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int c8 = (cg & 1) * 4 + k;
+                *reinterpret_cast<uint4*>(xrow + ((c8 ^ (r & 7)) << 4)) =
+                    make_uint4(dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
             if (lane == 0) mbar_arrive(ds_full);
         }
         if (ok && warp_wait(dkv_done, 0, abort_flag, p.status)) {
