@@ -451,7 +451,8 @@ __global__ void __launch_bounds__(NT, 1) attn_fwd_tc_kernel(const __grid_constan
 }
 
 // ============================================================================ backward
-// Three launches: (1) D = rowsum(dO * o) and lse * log2(e) per (row, head);
+// Three launches: (1) -D = -rowsum(dO * o) and -lse * log2(e) per (row, head)
+// (or the same statistics from the epilogue of the GEMM that forms dO);
 // (2) the dK/dV kernel, which recomputes S^T and dP^T per (key block, query
 // block, query head), forms P^T and dS^T, accumulates dV and dK, and stores
 // every dS^T tile; (3) dq = dS K / sqrt(hd) as a plain tensor-core product
