@@ -38,6 +38,11 @@ struct nc_model {
     int recompute = NC_RECOMPUTE_NONE;
     // caller-owned events recorded when each gradient bucket is final (may be empty)
     std::vector<cudaEvent_t> grad_events;
+    // the backward's weight-gradient GEMMs run on this second stream, overlapping the
+    // input-gradient chain on the caller's stream; kSideEvents order the two (null: off)
+    static constexpr int kSideEvents = 6;
+    cudaStream_t side = nullptr;
+    cudaEvent_t sev[kSideEvents] = {};
     // profiler: CUDA events around every launch while enabled
     struct Rec { int cls; cudaEvent_t a, b; double flops, bytes; long long launches; };
     bool prof_on = false;
@@ -472,6 +477,24 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     // padding of the last query block past T stays zero for the whole backward
     const bool fuse_stats = m->tc && attention_tc_bwd_supported(m->hd);
     if (fuse_stats && T % 128 != 0) CK(cudaMemsetAsync(Dbuf, 0, 4 * attn_dbuf_elems(B, T, m->H), s));
+    // Weight-gradient GEMMs on the second stream (when there is one): each starts once the
+    // caller's stream has produced its inputs, and the caller's stream waits for it only
+    // before overwriting an input it reads (dxb by the next norm backward, du by the next
+    // layer's first GEMM, dqkv by the next layer's attention backward).  They are the only
+    // users of the split-K scratch during the loop and run in order on their stream.
+    Ctx c2 = c;
+    if (m->side) c2.s = m->side;
+    enum { EV_FORK = 0, EV_PROJ, EV_FC, EV_OPROJ, EV_QKV, EV_END };
+    auto fork = [&]() -> bool {  // the side stream continues after the caller's stream's work so far
+        return !m->side || (cudaEventRecord(m->sev[EV_FORK], s) == cudaSuccess &&
+                            cudaStreamWaitEvent(m->side, m->sev[EV_FORK], 0) == cudaSuccess);
+    };
+    auto mark = [&](int e) -> bool { return !m->side || cudaEventRecord(m->sev[e], m->side) == cudaSuccess; };
+    auto after = [&](int e) -> bool { return !m->side || cudaStreamWaitEvent(s, m->sev[e], 0) == cudaSuccess; };
+    auto layer_done = [&](int i) -> int {  // this layer's weight gradients are the side stream's work so far
+        if (m->grad_events.empty()) return NC_OK;
+        return cudaEventRecord(m->grad_events[i], m->side ? m->side : s) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+    };
     for (int l = m->L - 1; l >= 0; --l) {
         char* lb = c.layer(l);
         int base = 1 + 6 * l;
@@ -482,14 +505,19 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
             fc.C2 = c.mlp_ru(lb); fc.ldc2 = F;
             RG(run_gemm(c, fc, P_GEMM_RECOMPUTE));
         }
+        if (!after(EV_FC)) return NC_ERR_CUDA;  // the previous layer's dWfc has read du
         GemmDesc g1 = mk(m, M, F, d, dxb, d, true, w.wproj(l), F, false, EPI_RELU2_BWD, du, F, m->at);
         g1.aux = c.mlp_ru(lb); g1.ldaux = F;
         RG(run_gemm(c, g1, P_GEMM_DGRAD));
-        RG(run_gemm(c, mk(m, d, F, M, dxb, d, false, c.mlp_h(lb), F, false, EPI_STORE, G(base + 5), F, DT_F32),
+        if (!fork()) return NC_ERR_CUDA;
+        RG(run_gemm(c2, mk(m, d, F, M, dxb, d, false, c.mlp_h(lb), F, false, EPI_STORE, G(base + 5), F, DT_F32),
                     P_GEMM_WGRAD));
+        if (!mark(EV_PROJ)) return NC_ERR_CUDA;
+        RG(run_gemm(c2, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32),
+                    P_GEMM_WGRAD));
+        if (!mark(EV_FC)) return NC_ERR_CUDA;
         RG(run_gemm(c, mk(m, M, d, F, du, F, true, w.wfc(l), d, false, EPI_STORE, gbuf, d, m->at), P_GEMM_DGRAD));
-        RG(run_gemm(c, mk(m, F, d, M, du, F, false, lb + c.p.l_m, d, false, EPI_STORE, G(base + 4), d, DT_F32),
-                    P_GEMM_WGRAD));
+        if (!after(EV_PROJ)) return NC_ERR_CUDA;  // dWproj has read dxb
         { Prof pr(c, P_NORM_BWD, 0.0, (double)M * (8.0 * d + 3.0 * A * d + 4.0)); CK(launch_rmsnorm_bwd(m->at, gbuf, true, lb + c.p.l_m, (float*)(lb + c.p.l_r2), dx, true, dxb, M, d, s)); }
         // attention: x_mid = x_in + o Wo^T; dO = dx Wo, with the softmax-backward statistics
         // D = rowsum(dO * o) and lse*log2(e) formed in the same GEMM's epilogue (tensor-core path)
@@ -506,21 +534,29 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
             RG(run_gemm(c, mk(m, M, Hhd, d, dxb, d, true, w.wo(l), Hhd, false, EPI_STORE, dO, Hhd, m->at),
                         P_GEMM_DGRAD));
         }
-        RG(run_gemm(c, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
-                          DT_F32), P_GEMM_WGRAD));
+        if (!fork()) return NC_ERR_CUDA;
+        RG(run_gemm(c2, mk(m, d, Hhd, M, dxb, d, false, lb + c.p.l_o, Hhd, false, EPI_STORE, G(base + 3), Hhd,
+                           DT_F32), P_GEMM_WGRAD));
+        if (!mark(EV_OPROJ)) return NC_ERR_CUDA;
+        if (!after(EV_QKV)) return NC_ERR_CUDA;  // the previous layer's dWqkv has read dqkv
         RG(attention_bwd(c, lb + c.p.l_qkv, lb + c.p.l_o, dO, (float*)(lb + c.p.l_lse), (float*)(lb + c.p.l_rqk),
                          dqkv, stats_ready));
         RG(run_gemm(c, mk(m, M, d, Nqkv, dqkv, Nqkv, true, w.wqkv(l), d, false, EPI_STORE, gbuf, d, m->at),
                     P_GEMM_DGRAD));
-        RG(run_gemm(c, mk(m, Nqkv, d, M, dqkv, Nqkv, false, lb + c.p.l_a, d, false, EPI_STORE, G(base), d,
-                          DT_F32), P_GEMM_WGRAD));
+        if (!fork()) return NC_ERR_CUDA;
+        RG(run_gemm(c2, mk(m, Nqkv, d, M, dqkv, Nqkv, false, lb + c.p.l_a, d, false, EPI_STORE, G(base), d,
+                           DT_F32), P_GEMM_WGRAD));
+        if (!mark(EV_QKV)) return NC_ERR_CUDA;
+        RG(layer_done(m->L - l));  // this layer's six weight gradients
+        if (!after(EV_OPROJ)) return NC_ERR_CUDA;  // dWo has read dxb
         {
             Prof pr(c, P_NORM_BWD, 0.0, (double)M * (8.0 * d + (l > 0 ? 3.0 : 2.0) * A * d + 4.0));
             CK(launch_rmsnorm_bwd(m->at, gbuf, true, lb + c.p.l_a, (float*)(lb + c.p.l_r1), dx, true,
                                   l > 0 ? dxb : nullptr, M, d, s));
         }
-        RG(bucket_done(m->L - l));  // this layer's six weight gradients
     }
+    // the caller's stream ends after every weight gradient
+    if (!mark(EV_END) || !after(EV_END)) return NC_ERR_CUDA;
     // ---- token embedding: norm backward, then the deterministic scatter-add
     {
         // norm backward (dx, Wte row, r0 -> de), then de read once and dWte written once
@@ -603,6 +639,17 @@ int nc_model_create(const nc_config* cfg, nc_precision prec, nc_model** out) {
         delete m;
         return NC_ERR_CUDA;
     }
+    // second stream for the weight-gradient GEMMs (the step runs without it if it cannot be made)
+    bool side_ok = cudaStreamCreateWithFlags(&m->side, cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; side_ok && i < nc_model::kSideEvents; ++i)
+        side_ok = cudaEventCreateWithFlags(&m->sev[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!side_ok) {
+        for (int i = 0; i < nc_model::kSideEvents; ++i)
+            if (m->sev[i]) cudaEventDestroy(m->sev[i]), m->sev[i] = nullptr;
+        if (m->side) cudaStreamDestroy(m->side);
+        m->side = nullptr;
+        cudaGetLastError();
+    }
     *out = m;
     return NC_OK;
 }
@@ -610,6 +657,9 @@ int nc_model_create(const nc_config* cfg, nc_precision prec, nc_model** out) {
 void nc_model_destroy(nc_model* m) {
     if (!m) return;
     for (cudaEvent_t e : m->ev_pool) cudaEventDestroy(e);
+    for (cudaEvent_t e : m->sev)
+        if (e) cudaEventDestroy(e);
+    if (m->side) cudaStreamDestroy(m->side);
     cudaFree(m->status);
     delete m;
 }
