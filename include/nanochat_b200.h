@@ -111,7 +111,14 @@ size_t nc_workspace_bytes(const nc_model* m, int B, int T);
  *   workspace: device, at least nc_workspace_bytes(m, B, T) bytes, 256-byte
  *     aligned; its contents on entry are ignored.
  * The full [B*T, V] logit tensor is never written to memory.  Results are
- * bitwise reproducible for a given model, inputs and workspace size. */
+ * bitwise reproducible for a given model, inputs and workspace size.
+ * Streams: the step is enqueued on `stream` (NULL = the legacy default
+ * stream); the weight-gradient GEMMs of the backward pass may run on a second
+ * stream owned by the model, forked from and joined back into `stream` with
+ * events, so every write of the call is ordered before work the caller
+ * enqueues on `stream` afterwards.  A model runs one call at a time: calls on
+ * the same model from several host threads, or interleaved on several
+ * streams, must be serialised by the caller. */
 int nc_forward_backward(nc_model* m, const int32_t* tokens, const int32_t* targets,
                         int B, int T, const void* weights, float* grads, float* loss,
                         void* workspace, size_t ws_bytes, void* stream);
