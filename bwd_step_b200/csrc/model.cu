@@ -482,18 +482,21 @@ int step(nc_model* m, const int32_t* tok, const int32_t* tgt, int B, int T, cons
     // before overwriting an input it reads (dxb by the next norm backward, du by the next
     // layer's first GEMM, dqkv by the next layer's attention backward).  They are the only
     // users of the split-K scratch during the loop and run in order on their stream.
+    // While the per-launch profiler is on everything stays on the caller's stream, so
+    // that each event pair times one kernel running alone.
+    const cudaStream_t side = m->prof_on ? nullptr : m->side;
     Ctx c2 = c;
-    if (m->side) c2.s = m->side;
+    if (side) c2.s = side;
     enum { EV_FORK = 0, EV_PROJ, EV_FC, EV_OPROJ, EV_QKV, EV_END };
     auto fork = [&]() -> bool {  // the side stream continues after the caller's stream's work so far
-        return !m->side || (cudaEventRecord(m->sev[EV_FORK], s) == cudaSuccess &&
-                            cudaStreamWaitEvent(m->side, m->sev[EV_FORK], 0) == cudaSuccess);
+        return !side || (cudaEventRecord(m->sev[EV_FORK], s) == cudaSuccess &&
+                       cudaStreamWaitEvent(side, m->sev[EV_FORK], 0) == cudaSuccess);
     };
-    auto mark = [&](int e) -> bool { return !m->side || cudaEventRecord(m->sev[e], m->side) == cudaSuccess; };
-    auto after = [&](int e) -> bool { return !m->side || cudaStreamWaitEvent(s, m->sev[e], 0) == cudaSuccess; };
+    auto mark = [&](int e) -> bool { return !side || cudaEventRecord(m->sev[e], side) == cudaSuccess; };
+    auto after = [&](int e) -> bool { return !side || cudaStreamWaitEvent(s, m->sev[e], 0) == cudaSuccess; };
     auto layer_done = [&](int i) -> int {  // this layer's weight gradients are the side stream's work so far
         if (m->grad_events.empty()) return NC_OK;
-        return cudaEventRecord(m->grad_events[i], m->side ? m->side : s) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+        return cudaEventRecord(m->grad_events[i], side ? side : s) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
     };
     for (int l = m->L - 1; l >= 0; --l) {
         char* lb = c.layer(l);
