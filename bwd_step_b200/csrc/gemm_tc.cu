@@ -843,12 +843,25 @@ int gemm_tc(const GemmDesc& g, void* splitk, size_t splitk_bytes, cudaStream_t s
     const bool can_split = (g.epi == EPI_STORE || g.epi == EPI_ACCUM || g.epi == EPI_ROWSCALE) && !p.c_bf16 &&
                            g.ldc == g.N && splitk && g.N % 4 == 0 && al16(g.C);
     if (can_split && tiles < 2 * sms) {
-        double best = (double)((tiles + sms - 1) / sms);
+        // Modelled time of each split count: per CTA pair, its waves of units (each 1/sp of
+        // a tile's K loop plus about 5 us of pipeline fill and drain), then the fp32
+        // partials written and read back and the output written.  Rates measured on the
+        // weight-gradient and LM-head shapes of the d20, d30, 124M and long-context steps:
+        // a CTA pair runs a 256x256 tile at about 23 TFLOP/s; partials that fit in half of
+        // the L2 move at about 20 TB/s, larger ones at the HBM rate of about 6 TB/s.
+        // Without the traffic term a 5120x1280 output (26 MB per partial) took 8 splits
+        // and ran 5-12% slower than with 2.
+        const double unit_flops = pair ? 23e12 : 11.5e12, fill = 5e-6;
+        const double t_tile = 2.0 * (pair ? 256 : BM) * BN * (double)g.K / unit_flops;
+        const double out_bytes = 4.0 * (double)g.M * g.N;
+        double best = (double)((tiles + sms - 1) / sms) * (t_tile + fill) + out_bytes / 6e12;
         for (int sp = 2; sp <= MAX_SPLITS; ++sp) {
             if (p.num_kb / sp < 8) break;
             if ((size_t)sp * g.M * g.N * sizeof(float) > splitk_bytes) break;
-            double cost = (double)((tiles * sp + sms - 1) / sms) / sp;
-            if (cost < best - 1e-9) { best = cost; splits = sp; }
+            const double bw = sp * out_bytes <= 64e6 ? 20e12 : 6e12;
+            const double cost =
+                (double)((tiles * sp + sms - 1) / sms) * (t_tile / sp + fill) + (2.0 * sp + 1.0) * out_bytes / bw;
+            if (cost < best * (1.0 - 1e-9)) { best = cost; splits = sp; }
         }
     }
     p.kb_per_split = (p.num_kb + splits - 1) / splits;
