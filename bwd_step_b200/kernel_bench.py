@@ -3,6 +3,7 @@
     python -m bwd_step_b200.kernel_bench gemm [--only NAME] [--iters N]
     python -m bwd_step_b200.kernel_bench attention [--iters N]
     python -m bwd_step_b200.kernel_bench step [--workload d20] [--batch B] [--layers L] [--lm-rows R] [--warmup W] [--iters K]
+    python -m bwd_step_b200.kernel_bench adamw|decode|recompute [--workload d20] [--iters K]
 
 `gemm` runs every GEMM shape of one depth-20 step (32768 tokens, d 1280,
 MLP 5120, 10x128 MQA, vocab 65536 with a 4096-row LM-head chunk) through the
@@ -11,6 +12,10 @@ TFLOP/s from CUDA events.  `attention` times the tcgen05 attention forward and
 backward at seq 2048, batch 16.  `step` runs W warm-up steps and then K
 steps of a workload (optionally at a smaller batch, for profiler captures
 that must stay small) and prints the library's kernel launches per step.
+`adamw` times one AdamW update of every parameter of a workload (fp32 master
+and moments, bf16 copy; 30 bytes per parameter); `decode` prefills 1024 tokens
+in 16 rows and times one-token decode steps over the KV cache; `recompute`
+times the step with the MLP hidden saved and recomputed, with both workspaces.
 Each case holds at most a few GB on the device, except `step` at full batch.
 """
 from __future__ import annotations
@@ -150,9 +155,103 @@ def run_steps(workload, batch, warmup, iters, layers=0, lm_rows=0):
     return {"workload": workload, "batch": B, "lm_rows": lm_rows, "ms_per_step": t, "launches_per_step": per, "loss": float(loss.item())}
 
 
+def _setup(workload):
+    import numpy as np
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import synth
+    from . import Model
+    wl = synth.WORKLOADS[workload]
+    bits, _ = synth.make_weights(wl.model, seed=0, dtype="bf16")
+    m = Model(wl.model.as_dict(), "bf16")
+    W = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+    return synth, wl, m, W
+
+
+def bench_adamw(workload, iters):
+    """One AdamW update of every parameter (two groups), fp32 master and moments,
+    bf16 compute copy: 30 bytes of HBM traffic per parameter."""
+    from . import adamw_step
+    _, _, m, W = _setup(workload)
+    n = m.num_params()
+    g = torch.Generator(device="cuda").manual_seed(0)
+    master = W.float()
+    grads = torch.randn(n, device="cuda", generator=g) * 1e-3
+    mom, vel = torch.zeros(n, device="cuda"), torch.zeros(n, device="cuda")
+    half = n // 2
+    groups = [(0, half, 3e-4, 0.9, 0.95, 1e-8, 0.0), (half, n - half, 1e-3, 0.8, 0.95, 1e-10, 0.01)]
+    step = [0]
+
+    def run():
+        step[0] += 1
+        adamw_step(groups, step[0], master, W, grads, mom, vel)
+
+    ms = _timed(run, iters)
+    m.close()
+    return {"kernel": "adamw", "workload": workload, "params": n, "ms": ms, "gbs": 30.0 * n / ms / 1e6}
+
+
+def bench_decode(workload, iters, B=16, T0=1024):
+    """Prefill T0 tokens per row, then time one-token decode steps (every row
+    one new token at the next position) through the KV cache."""
+    synth, wl, m, W = _setup(workload)
+    T_max = T0 + iters + 8
+    tok, _ = synth.make_tokens(synth.Workload("dec", wl.model, T_max, B, "uniform"), seed=1)
+    tok_d = torch.from_numpy(tok).cuda()
+    cache = torch.empty(m.kv_cache_bytes(B, T_max), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(m.inference_workspace_bytes(B, T_max), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((B, wl.model.vocab), dtype=torch.bfloat16, device="cuda")
+    cols = [tok_d[:, t].contiguous() for t in range(T_max)]
+    m.prefill(tok_d[:, :T0].contiguous(), W, cache, T_max, logits, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_p = _timed(lambda: m.prefill(tok_d[:, :T0].contiguous(), W, cache, T_max, logits, ws), 3)
+    pos = [T0]
+    for _ in range(3):  # warm-up steps
+        m.decode_step(cols[pos[0]], pos[0], W, cache, T_max, logits, ws)
+        pos[0] += 1
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(iters):
+        m.decode_step(cols[pos[0]], pos[0], W, cache, T_max, logits, ws)
+        pos[0] += 1
+    e1.record()
+    torch.cuda.synchronize()
+    assert m.check() == 0
+    ms = e0.elapsed_time(e1) / iters
+    weight_bytes = 2.0 * m.num_params()
+    m.close()
+    return {"kernel": "decode_step", "workload": workload, "batch": B, "prompt": T0, "prefill_ms": t_p,
+            "ms": ms, "tokens_per_s": B / ms * 1e3, "weight_gbs": weight_bytes / ms / 1e6}
+
+
+def bench_recompute(workload, warmup, iters):
+    """The step with and without recomputing the MLP hidden in the backward."""
+    synth, wl, m, W = _setup(workload)
+    tok, tgt = synth.make_tokens(wl, seed=1)
+    tok_d, tgt_d = torch.from_numpy(tok).cuda(), torch.from_numpy(tgt).cuda()
+    grads = torch.empty(m.num_params(), dtype=torch.float32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    out = {"workload": workload}
+    for name, flag in (("saved", False), ("recompute", True), ("saved_again", False)):
+        m.set_recompute(flag)
+        nb = m.workspace_bytes(wl.batch, wl.seq_len)
+        ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        for _ in range(warmup):
+            m.forward_backward(tok_d, tgt_d, W, grads, loss, ws)
+        out[name] = {"ms_per_step": _timed(lambda: m.forward_backward(tok_d, tgt_d, W, grads, loss, ws), iters),
+                     "workspace_gib": nb / 2**30}
+        del ws
+        torch.cuda.empty_cache()
+    assert m.check() == 0
+    m.close()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["gemm", "attention", "step"])
+    ap.add_argument("what", choices=["gemm", "attention", "step", "adamw", "decode", "recompute"])
     ap.add_argument("--workload", default="d20")
     ap.add_argument("--batch", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0)
@@ -170,6 +269,12 @@ def main():
     elif args.what == "attention":
         for r in bench_attention(args.iters):
             print(json.dumps(r), flush=True)
+    elif args.what == "adamw":
+        print(json.dumps(bench_adamw(args.workload, args.iters)), flush=True)
+    elif args.what == "decode":
+        print(json.dumps(bench_decode(args.workload, args.iters)), flush=True)
+    elif args.what == "recompute":
+        print(json.dumps(bench_recompute(args.workload, args.warmup, args.iters)), flush=True)
     else:
         print(json.dumps(run_steps(args.workload, args.batch, args.warmup, args.iters, args.layers, args.lm_rows)), flush=True)
 
